@@ -1,0 +1,383 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU restatement of single-token paged decode
+ * attention, the KV append, the PagedEviction norm-ratio score with its
+ * block-mean argmin, and the symmetric INT8 KV quantiser.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call this file:
+ * only the tests, the smoke check and the benchmark's CPU-baseline leg load
+ * it.  It shares no code, header, table or helper with the CUDA library.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [KVL]  blog.hotdry.top, "KV缓存内存布局优化：分页策略、量化压缩与动态驱逐的工程实践"
+ *          (KV cache memory layout optimisation), sections "PagedAttention 分页策略"
+ *          and "PagedEviction 块级驱逐机制".
+ *   [VKV]  ybb.press, "LLM 推理 KV Cache 内存管理深度工程实践：从 PageAttention 到推测解码"
+ *          (vLLM KV memory engineering notes), §1, §2.1 BlockTable, §2.2
+ *          paged_attention_forward, §6.1 INT8 KV cache, §6.2 GQA.
+ *   [NANO] blog.hotdry.top, nano-vLLM KV cache memory optimisation, section
+ *          "物理内存布局：连续张量与分块策略" (the [2, L, blocks, bs, n_kv, d] tensor).
+ *   [KVP]  t6page.pages.dev knowledge page "KV cache": eq. kv-per-token,
+ *          eq. kv-llama3-8b, table tbl-kv-llama3-context, section
+ *          "PagedAttention 的算子" (the operator).
+ *
+ * Layout conventions (shared with every caller, not with the CUDA code):
+ *   pool  [N physical blocks][bs slots][Hkv heads][d]; block b starts at
+ *         element b * block_stride (block_stride >= bs*Hkv*d).
+ *   bt    [B][MB] int32 block table, logical block j of sequence b -> physical id.
+ *   bf16 values are passed as their uint16 bit patterns.
+ *
+ * Readings where the pages are silent or inconsistent are stated at each
+ * function.  Floating point: fp64 everywhere except the INT8 quantiser, which
+ * the configuration fixes to one fp32 scale per (token, kv head) and which is
+ * therefore restated in fp32 so that its integer codes are decided in the same
+ * precision as any fp32 implementation.
+ *
+ * Build: gcc -O2 -fopenmp -ffp-contract=off -fPIC -shared (see build.py).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* bf16 is the upper half of an IEEE binary32: widen by a 16-bit shift. */
+static float bf16_to_f32(uint16_t x) {
+    uint32_t u = ((uint32_t)x) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static double bf16_to_f64(uint16_t x) { return (double)bf16_to_f32(x); }
+
+/* ------------------------------------------------------------------------ */
+/* Sizes                                                                     */
+/* ------------------------------------------------------------------------ */
+
+/* KV bytes per token: one K and one V vector per layer and kv head.
+ * [KVP] eq. kv-per-token: 2 * L * n_kv * d_head * bytes; [VKV] §1 states the
+ * same product (2 x num_layers x num_kv_heads x head_dim x dtype_size). */
+int64_t or_kv_bytes_per_token(int64_t L, int64_t n_kv, int64_t d, int64_t elt_bytes) {
+    return 2 * L * n_kv * d * elt_bytes;
+}
+
+/* Blocks a sequence of len tokens occupies: ceil(len / bs).
+ * [VKV] §2.1 BlockTable.allocate; [VKV] §2.2 loop bound; [KVP] KVCachePool. */
+int64_t or_num_blocks(int64_t len, int64_t bs) {
+    if (len <= 0) return 0;
+    return (len + bs - 1) / bs;
+}
+
+/* Global slot of token position pos: the physical block holding logical block
+ * pos/bs, times bs, plus the offset pos%bs inside it.
+ * [VKV] §2.1 BlockTable.append_slot returns last_block*block_size+used_slots,
+ * i.e. the same formula for the token that lands in the last block. */
+int64_t or_slot(const int32_t *bt_row, int64_t pos, int64_t bs) {
+    return (int64_t)bt_row[pos / bs] * bs + pos % bs;
+}
+
+/* ------------------------------------------------------------------------ */
+/* KV append                                                                 */
+/* ------------------------------------------------------------------------ */
+
+/* Write n_new tokens per sequence into the pool: token i of sequence b goes to
+ * position positions[b] + i, i.e. to slot or_slot(bt[b], pos, bs), head h.
+ * k_new, v_new: [B][n_new][Hkv][d] bf16 bits.  slot_out (nullable): [B][n_new].
+ * [VKV] §2.1 append_slot; [KVL] "PagedAttention 分页策略" (blocks are filled as
+ * tokens are generated). */
+void or_append_kv(const uint16_t *k_new, const uint16_t *v_new,
+                  uint16_t *k_cache, uint16_t *v_cache, int64_t block_stride,
+                  const int32_t *bt, int MB, const int32_t *positions,
+                  int B, int n_new, int Hkv, int d, int bs, int64_t *slot_out) {
+    for (int b = 0; b < B; ++b) {
+        for (int i = 0; i < n_new; ++i) {
+            int64_t pos = (int64_t)positions[b] + i;
+            int64_t slot = or_slot(bt + (int64_t)b * MB, pos, bs);
+            if (slot_out) slot_out[(int64_t)b * n_new + i] = slot;
+            int64_t phys = slot / bs, off = slot % bs;
+            for (int h = 0; h < Hkv; ++h) {
+                int64_t dst = phys * block_stride + (off * Hkv + h) * (int64_t)d;
+                int64_t src = (((int64_t)b * n_new + i) * Hkv + h) * (int64_t)d;
+                memcpy(k_cache + dst, k_new + src, (size_t)d * sizeof(uint16_t));
+                memcpy(v_cache + dst, v_new + src, (size_t)d * sizeof(uint16_t));
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Attention                                                                 */
+/* ------------------------------------------------------------------------ */
+
+/* Gather sequence b's first len tokens, in logical order, into contiguous fp64
+ * K[len][Hkv][d] and V[len][Hkv][d].  Slots of the last block at or beyond len
+ * are not read ([VKV] §2.2 valid_slots).  The source values are produced by
+ * `load(pool, index, aux)`, so that bf16 and dequantised INT8 pools share it. */
+typedef double (*load_fn)(const void *pool, const void *aux, int64_t idx, int64_t row, int Hd);
+
+static double load_bf16(const void *pool, const void *aux, int64_t idx, int64_t row, int Hd) {
+    (void)aux; (void)row; (void)Hd;
+    return bf16_to_f64(((const uint16_t *)pool)[idx]);
+}
+
+/* INT8: value = scale[token row, head] * code, the dequantisation of [VKV] §6.1. */
+static double load_int8(const void *pool, const void *aux, int64_t idx, int64_t row, int Hd) {
+    (void)Hd;
+    const float *scale = (const float *)aux;
+    return (double)scale[row] * (double)((const int8_t *)pool)[idx];
+}
+
+static void gather_seq(double *Kc, double *Vc, const void *k_cache, const void *v_cache,
+                       const void *k_aux, const void *v_aux, load_fn load,
+                       int64_t block_stride, int64_t scale_block_stride,
+                       const int32_t *bt_row, int len, int Hkv, int d, int bs) {
+    for (int t = 0; t < len; ++t) {
+        int64_t phys = bt_row[t / bs];
+        int64_t off = t % bs;
+        for (int h = 0; h < Hkv; ++h) {
+            int64_t base = phys * block_stride + (off * Hkv + h) * (int64_t)d;
+            int64_t srow = phys * scale_block_stride + off * Hkv + h; /* scale index */
+            for (int e = 0; e < d; ++e) {
+                Kc[((int64_t)t * Hkv + h) * d + e] = load(k_cache, k_aux, base + e, srow, Hkv * d);
+                Vc[((int64_t)t * Hkv + h) * d + e] = load(v_cache, v_aux, base + e, srow, Hkv * d);
+            }
+        }
+    }
+}
+
+/* Softmax attention of one query vector q[d] over len contiguous keys/values of
+ * kv head h (row stride Hkv*d): s_t = scale * q.k_t; p = softmax(s) taken over
+ * ALL len tokens at once ([KVP] "PagedAttention 的算子": the scaled dot product
+ * and softmax are done after merging every block); o = sum_t p_t v_t.
+ * Two passes, max-subtracted.  len == 0 gives o = 0 (nothing to attend to). */
+static void attend_one(double *o, const double *q, const double *Kc, const double *Vc,
+                       int len, int Hkv, int h, int d, double scale, double *s) {
+    for (int e = 0; e < d; ++e) o[e] = 0.0;
+    if (len <= 0) return;
+    double m = -INFINITY;
+    for (int t = 0; t < len; ++t) {
+        const double *k = Kc + ((int64_t)t * Hkv + h) * d;
+        double acc = 0.0;
+        for (int e = 0; e < d; ++e) acc += q[e] * k[e];
+        s[t] = scale * acc;
+        if (s[t] > m) m = s[t];
+    }
+    double z = 0.0;
+    for (int t = 0; t < len; ++t) {
+        s[t] = exp(s[t] - m);
+        z += s[t];
+    }
+    for (int t = 0; t < len; ++t) {
+        const double *v = Vc + ((int64_t)t * Hkv + h) * d;
+        double p = s[t] / z;
+        for (int e = 0; e < d; ++e) o[e] += p * v[e];
+    }
+}
+
+/* Shared body of the bf16 and INT8 decode oracles.
+ * For every sequence b: gather its len_b = ctx_lens[b] tokens, then for every
+ * query head i use kv head h = i / G with G = Hq / Hkv (contiguous GQA groups,
+ * [VKV] §6.2: every G query heads share one KV group), and attend.
+ * Lengths outside [0, MB*bs] are treated as 0 (output zero), as is len 0. */
+static void decode_common(double *out, const uint16_t *q, const void *k_cache,
+                          const void *v_cache, const void *k_aux, const void *v_aux,
+                          load_fn load, int64_t block_stride, int64_t scale_block_stride,
+                          const int32_t *bt, int MB, const int32_t *ctx_lens, int B,
+                          int Hq, int Hkv, int d, int bs, double scale) {
+    int G = Hq / Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b) {
+        int len = ctx_lens[b];
+        if (len < 0 || (int64_t)len > (int64_t)MB * bs) len = 0;
+        double *Kc = (double *)malloc(sizeof(double) * ((size_t)len * Hkv * d + 1));
+        double *Vc = (double *)malloc(sizeof(double) * ((size_t)len * Hkv * d + 1));
+        double *s = (double *)malloc(sizeof(double) * ((size_t)len + 1));
+        double *qv = (double *)malloc(sizeof(double) * (size_t)d);
+        gather_seq(Kc, Vc, k_cache, v_cache, k_aux, v_aux, load, block_stride,
+                   scale_block_stride, bt + (int64_t)b * MB, len, Hkv, d, bs);
+        for (int i = 0; i < Hq; ++i) {
+            for (int e = 0; e < d; ++e) qv[e] = bf16_to_f64(q[((int64_t)b * Hq + i) * d + e]);
+            attend_one(out + ((int64_t)b * Hq + i) * d, qv, Kc, Vc, len, Hkv, i / G, d, scale, s);
+        }
+        free(Kc); free(Vc); free(s); free(qv);
+    }
+}
+
+/* Paged decode attention, bf16 pool.  out [B][Hq][d] fp64; q [B][Hq][d] bf16.
+ * [VKV] §2.2 paged_attention_forward (query, paged cache, block table, context
+ * length, scale), batched over sequences; separate K and V pools ([NANO]
+ * index 0 = key, 1 = value), softmax over the whole context ([KVP] operator). */
+void or_paged_decode(double *out, const uint16_t *q, const uint16_t *k_cache,
+                     const uint16_t *v_cache, int64_t block_stride, const int32_t *bt,
+                     int MB, const int32_t *ctx_lens, int B, int Hq, int Hkv, int d,
+                     int bs, double scale) {
+    decode_common(out, q, k_cache, v_cache, NULL, NULL, load_bf16, block_stride, 0, bt, MB,
+                  ctx_lens, B, Hq, Hkv, d, bs, scale);
+}
+
+/* Paged decode attention over an INT8 pool: every element is dequantised as
+ * scale[token, head] * code ([VKV] §6.1) before the same fp64 attention.
+ * Scale pools are [N][bs][Hkv] fp32 (block stride bs*Hkv). */
+void or_paged_decode_int8(double *out, const uint16_t *q, const int8_t *kq, const int8_t *vq,
+                          const float *k_scale, const float *v_scale, int64_t block_stride,
+                          const int32_t *bt, int MB, const int32_t *ctx_lens, int B, int Hq,
+                          int Hkv, int d, int bs, double scale) {
+    decode_common(out, q, kq, vq, k_scale, v_scale, load_int8, block_stride,
+                  (int64_t)bs * Hkv, bt, MB, ctx_lens, B, Hq, Hkv, d, bs, scale);
+}
+
+/* ------------------------------------------------------------------------ */
+/* PagedEviction                                                             */
+/* ------------------------------------------------------------------------ */
+
+/* Token importance S = ||V||_2 / ||K||_2 over the d elements of one (token,
+ * kv head) vector ([KVL] "PagedEviction 块级驱逐机制": the ratio of the value and
+ * key L2 norms, no attention weights needed).  Reading: the pages give one
+ * S_i per token with no head index; here it is per (token, kv head).
+ * ||K|| = 0: S = +inf when ||V|| > 0, else 0. */
+static double norm_ratio(double kk, double vv) {
+    if (kk == 0.0) return vv > 0.0 ? INFINITY : 0.0;
+    return sqrt(vv) / sqrt(kk);
+}
+
+static void score_common(double *scores, const void *k_cache, const void *v_cache,
+                         const void *k_aux, const void *v_aux, load_fn load,
+                         int64_t block_stride, int64_t scale_block_stride, const int32_t *bt,
+                         int MB, const int32_t *ctx_lens, int B, int Hkv, int d, int bs) {
+    int64_t T = (int64_t)MB * bs;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b) {
+        int len = ctx_lens[b];
+        if (len < 0 || (int64_t)len > T) len = 0;
+        for (int t = 0; t < len; ++t) {
+            int64_t phys = bt[(int64_t)b * MB + t / bs];
+            int64_t off = t % bs;
+            for (int h = 0; h < Hkv; ++h) {
+                int64_t base = phys * block_stride + (off * Hkv + h) * (int64_t)d;
+                int64_t srow = phys * scale_block_stride + off * Hkv + h;
+                double kk = 0.0, vv = 0.0;
+                for (int e = 0; e < d; ++e) {
+                    double k = load(k_cache, k_aux, base + e, srow, Hkv * d);
+                    double v = load(v_cache, v_aux, base + e, srow, Hkv * d);
+                    kk += k * k;
+                    vv += v * v;
+                }
+                scores[((int64_t)b * T + t) * Hkv + h] = norm_ratio(kk, vv);
+            }
+        }
+    }
+}
+
+/* scores [B][MB*bs][Hkv] fp64; entries with t >= len_b are left untouched. */
+void or_score_tokens(double *scores, const uint16_t *k_cache, const uint16_t *v_cache,
+                     int64_t block_stride, const int32_t *bt, int MB, const int32_t *ctx_lens,
+                     int B, int Hkv, int d, int bs) {
+    score_common(scores, k_cache, v_cache, NULL, NULL, load_bf16, block_stride, 0, bt, MB,
+                 ctx_lens, B, Hkv, d, bs);
+}
+
+/* Same score over the dequantised INT8 values. */
+void or_score_tokens_int8(double *scores, const int8_t *kq, const int8_t *vq,
+                          const float *k_scale, const float *v_scale, int64_t block_stride,
+                          const int32_t *bt, int MB, const int32_t *ctx_lens, int B, int Hkv,
+                          int d, int bs) {
+    score_common(scores, kq, vq, k_scale, v_scale, load_int8, block_stride, (int64_t)bs * Hkv,
+                 bt, MB, ctx_lens, B, Hkv, d, bs);
+}
+
+/* Decode-phase block eviction ([KVL] "PagedEviction 块级驱逐机制": when the
+ * newest block is full, average the importance of every existing block and
+ * evict the complete block with the lowest mean; eviction is always whole
+ * blocks).  Reading: candidates are the full logical blocks j < floor(len/bs);
+ * mean_j = sum of S over the bs*Hkv (token, head) entries of block j, divided
+ * by bs*Hkv; ties go to the lowest j; no full block gives -1.
+ * scores [B][MB*bs][Hkv] fp64 (an fp32 score array widened to fp64 is exact);
+ * evict [B]; means (nullable) [B][MB], entries of non-candidate blocks set to
+ * NAN; gap (nullable) [B] = second-lowest minus lowest mean (+inf when fewer
+ * than two candidates), the margin by which the decision is made. */
+void or_select_evict_block(int32_t *evict, double *means, double *gap, const double *scores,
+                           const int32_t *ctx_lens, int B, int MB, int Hkv, int bs) {
+    int64_t T = (int64_t)MB * bs;
+    for (int b = 0; b < B; ++b) {
+        int len = ctx_lens[b];
+        if (len < 0 || (int64_t)len > T) len = 0;
+        int nfull = len / bs;
+        int best = -1;
+        double best_mean = INFINITY, second = INFINITY;
+        for (int j = 0; j < MB; ++j) {
+            if (j >= nfull) {
+                if (means) means[(int64_t)b * MB + j] = NAN;
+                continue;
+            }
+            double sum = 0.0;
+            for (int t = j * bs; t < (j + 1) * bs; ++t)
+                for (int h = 0; h < Hkv; ++h) sum += scores[((int64_t)b * T + t) * Hkv + h];
+            double mean = sum / (double)(bs * Hkv);
+            if (means) means[(int64_t)b * MB + j] = mean;
+            if (best < 0 || mean < best_mean) {
+                second = best_mean;
+                best_mean = mean;
+                best = j;
+            } else if (mean < second) {
+                second = mean;
+            }
+        }
+        evict[b] = best;
+        if (gap) gap[b] = (best < 0 || second == INFINITY) ? INFINITY : second - best_mean;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* INT8 quantiser                                                            */
+/* ------------------------------------------------------------------------ */
+
+/* Symmetric INT8 quantisation of rows of d bf16 values, fp32 arithmetic
+ * ([VKV] §6.1 quantize_kv_cache: scale = amax(|x|, last dim) / 127,
+ * code = round(x / scale) as int8).  Readings: the scale is fp32, one per
+ * (token, kv head) row; round() is PyTorch's, i.e. half to even (rintf in the
+ * default rounding mode); amax = 0 gives scale 0 and all codes 0.  Every step
+ * is one correctly rounded IEEE binary32 operation.
+ * x [rows][d] bf16 bits; codes [rows][d]; scales [rows]. */
+void or_quantize_int8(const uint16_t *x, int64_t rows, int d, int8_t *codes, float *scales) {
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *xr = x + r * d;
+        float amax = 0.0f;
+        for (int e = 0; e < d; ++e) {
+            float a = fabsf(bf16_to_f32(xr[e]));
+            if (a > amax) amax = a;
+        }
+        volatile float s = amax / 127.0f; /* volatile: keep it a single fp32 division */
+        scales[r] = s;
+        for (int e = 0; e < d; ++e) {
+            if (s == 0.0f) {
+                codes[r * d + e] = 0;
+            } else {
+                volatile float y = bf16_to_f32(xr[e]) / s;
+                codes[r * d + e] = (int8_t)(int)rintf(y);
+            }
+        }
+    }
+}
+
+/* INT8 append: quantise token i of sequence b (each kv head row separately)
+ * and store codes into slot or_slot(bt[b], positions[b]+i) and its scale into
+ * the [N][bs][Hkv] scale pools. */
+void or_append_kv_int8(const uint16_t *k_new, const uint16_t *v_new, int8_t *kq, int8_t *vq,
+                       float *k_scale, float *v_scale, int64_t block_stride, const int32_t *bt,
+                       int MB, const int32_t *positions, int B, int n_new, int Hkv, int d, int bs,
+                       int64_t *slot_out) {
+    for (int b = 0; b < B; ++b) {
+        for (int i = 0; i < n_new; ++i) {
+            int64_t pos = (int64_t)positions[b] + i;
+            int64_t slot = or_slot(bt + (int64_t)b * MB, pos, bs);
+            if (slot_out) slot_out[(int64_t)b * n_new + i] = slot;
+            int64_t phys = slot / bs, off = slot % bs;
+            for (int h = 0; h < Hkv; ++h) {
+                int64_t src = (((int64_t)b * n_new + i) * Hkv + h) * (int64_t)d;
+                int64_t dst = phys * block_stride + (off * Hkv + h) * (int64_t)d;
+                int64_t sdst = (phys * bs + off) * Hkv + h;
+                or_quantize_int8(k_new + src, 1, d, kq + dst, k_scale + sdst);
+                or_quantize_int8(v_new + src, 1, d, vq + dst, v_scale + sdst);
+            }
+        }
+    }
+}

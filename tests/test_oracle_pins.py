@@ -1,0 +1,484 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+CPU only.  None of these re-types the oracle's own code: each checks a printed
+value, a closed form, an invariant, a special case that reduces to a textbook
+or library routine, or a brute-force/stateful restatement on tiny inputs.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_396_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16_bits(x) -> np.ndarray:
+    return torch.as_tensor(np.asarray(x, np.float32)).to(torch.bfloat16).view(torch.int16) \
+        .numpy().view(np.uint16)
+
+
+def bf16_vals(bits) -> np.ndarray:
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def rand_case(seed, B=3, Hq=8, Hkv=2, d=16, bs=4, N=40, lens=(1, 7, 13)):
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(N).astype(np.int32)
+    MB = max(-(-n // bs) for n in lens)
+    bt = np.full((B, MB), -1, np.int32)
+    k = 0
+    for b, n in enumerate(lens):
+        for j in range(-(-n // bs)):
+            bt[b, j] = perm[k]
+            k += 1
+    kc = bf16_bits(rng.standard_normal((N, bs, Hkv, d)))
+    vc = bf16_bits(rng.standard_normal((N, bs, Hkv, d)))
+    q = bf16_bits(rng.standard_normal((B, Hq, d)))
+    return dict(q=q, kc=kc, vc=vc, bt=bt, lens=np.asarray(lens, np.int32), B=B, Hq=Hq, Hkv=Hkv,
+                d=d, bs=bs, N=N)
+
+
+def run_decode(c, scale=None):
+    scale = 1.0 / math.sqrt(c["d"]) if scale is None else scale
+    return oracle.paged_decode(c["q"], c["kc"].ravel(), c["vc"].ravel(),
+                               c["bs"] * c["Hkv"] * c["d"], c["bt"], c["lens"], c["Hkv"],
+                               c["bs"], scale)
+
+
+def gather_logical(c, b):
+    """K, V of sequence b in logical order via plain numpy indexing of the table."""
+    n = int(c["lens"][b])
+    ids = c["bt"][b, : -(-n // c["bs"])]
+    K = bf16_vals(c["kc"][ids]).reshape(-1, c["Hkv"], c["d"])[:n]
+    V = bf16_vals(c["vc"][ids]).reshape(-1, c["Hkv"], c["d"])[:n]
+    return K, V
+
+
+# ------------------------------------------------------------------ sizes
+def _golden_sizes():
+    rows = []
+    with open(os.path.join(GOLDEN, "kv_sizes.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+def test_kv_bytes_per_token_printed_values():
+    rows = _golden_sizes()
+    seen = set()
+    for kind, name, L, nkv, d, elt, *vals in rows:
+        L, nkv, d, elt = int(L), int(nkv), int(d), int(elt)
+        per_tok = oracle.kv_bytes_per_token(L, nkv, d, elt)
+        if kind == "token":
+            assert per_tok == int(vals[0])
+        elif kind == "context":
+            for item in vals:
+                ctx, nbytes = map(int, item.split(":"))
+                assert per_tok * ctx == nbytes
+        elif kind == "half":       # the page's 160 KB is K alone (or V alone)
+            assert per_tok // 2 == int(vals[0]) and per_tok == 2 * int(vals[0])
+        elif kind == "halfctx":
+            ctx, nbytes = map(int, vals[0].split(":"))
+            assert per_tok // 2 * ctx == nbytes
+        elif kind == "requests":
+            ctx, nreq, nbytes = map(int, vals[0].split(":"))
+            assert per_tok // 2 * ctx * nreq == nbytes
+        seen.add(kind)
+    assert seen == {"token", "context", "half", "halfctx", "requests"}
+
+
+def test_num_blocks_is_ceiling():
+    for bs in (1, 2, 7, 16, 256):
+        for n in range(0, 600, 3):
+            # brute force: smallest k with k*bs >= n
+            k = 0
+            while k * bs < n:
+                k += 1
+            assert oracle.num_blocks(n, bs) == k
+    # the tiny workload: 38 -> 3 and 101 -> 7 blocks of 16
+    assert oracle.num_blocks(38, 16) == 3 and oracle.num_blocks(101, 16) == 7
+
+
+def test_workload_tables_hold_exactly_the_needed_blocks():
+    for key in ("c1", "c2", "c4"):
+        cfg = W.CONFIGS[key]
+        rng = np.random.default_rng(cfg.seed)
+        old = W._old_lens(cfg, rng)
+        ctx = old + (1 if cfg.append else 0)
+        bt, N = W._allocate(ctx, cfg.block_size, cfg.spare, cfg.pool_blocks, rng)
+        used = bt[bt >= 0]
+        assert len(np.unique(used)) == len(used) and used.max() < N
+        for b in range(cfg.batch):
+            assert (bt[b] >= 0).sum() == oracle.num_blocks(int(ctx[b]), cfg.block_size)
+    c1 = W.CONFIGS["c1"]
+    rng = np.random.default_rng(c1.seed)
+    old = W._old_lens(c1, rng)
+    bt, N = W._allocate(old + 1, c1.block_size, c1.spare, c1.pool_blocks, rng)
+    assert N == 64 and (bt >= 0).sum() == 10
+
+
+# ------------------------------------------------------------------ slots / append
+class BlockTableSim:
+    """Stateful restatement of the BlockTable of the vLLM notes (ybb.press §2.1):
+    append_slot returns last_block*bs + used slots while the last block has room,
+    else takes a new block from the free list and returns its first slot."""
+
+    def __init__(self, bs, free):
+        self.bs, self.free, self.table, self.n = bs, list(free), [], 0
+
+    def append_slot(self):
+        if self.n % self.bs == 0:            # no block yet, or the last block is full
+            self.table.append(self.free.pop())
+            s = self.table[-1] * self.bs
+        else:
+            s = self.table[-1] * self.bs + (self.n % self.bs)
+        self.n += 1
+        return s
+
+
+def test_slot_formula_matches_stateful_block_table():
+    rng = np.random.default_rng(7)
+    for bs in (1, 4, 16, 256):
+        sim = BlockTableSim(bs, rng.permutation(200).tolist())
+        slots = [sim.append_slot() for _ in range(min(40 * bs, 2000))]
+        row = np.asarray(sim.table, np.int32)
+        for pos, s in enumerate(slots):
+            assert oracle.slot(row, pos, bs) == s
+        assert len(set(slots)) == len(slots)
+
+
+def test_append_then_logical_gather_is_identity():
+    rng = np.random.default_rng(11)
+    B, Hkv, d, bs, N = 3, 2, 8, 4, 30
+    lens = np.array([5, 9, 12], np.int32)
+    perm = rng.permutation(N).astype(np.int32)
+    MB = 3
+    bt = np.full((B, MB), -1, np.int32)
+    k = 0
+    for b in range(B):
+        for j in range(-(-int(lens[b]) // bs)):
+            bt[b, j] = perm[k]
+            k += 1
+    kc = np.zeros(N * bs * Hkv * d, np.uint16)
+    vc = np.zeros_like(kc)
+    maxlen = int(lens.max())
+    kn = bf16_bits(rng.standard_normal((B, maxlen, Hkv, d)))
+    vn = bf16_bits(rng.standard_normal((B, maxlen, Hkv, d)))
+    # write every token one at a time (decode-style appends)
+    for pos in range(maxlen):
+        live = [b for b in range(B) if pos < lens[b]]
+        oracle.append_kv(kn[live, pos:pos + 1], vn[live, pos:pos + 1], kc, vc, bs * Hkv * d,
+                         bt[live], np.full(len(live), pos, np.int32), bs)
+    c = dict(kc=kc.reshape(N, bs, Hkv, d), vc=vc.reshape(N, bs, Hkv, d), bt=bt, lens=lens,
+             Hkv=Hkv, d=d, bs=bs)
+    for b in range(B):
+        K, V = gather_logical(c, b)
+        n = int(lens[b])
+        assert np.array_equal(K, bf16_vals(kn[b, :n]))
+        assert np.array_equal(V, bf16_vals(vn[b, :n]))
+    # a multi-token append (prefill-style) writes the same pools
+    kc2 = np.zeros_like(kc)
+    vc2 = np.zeros_like(vc)
+    for b in range(B):
+        n = int(lens[b])
+        oracle.append_kv(kn[b:b + 1, :n], vn[b:b + 1, :n], kc2, vc2, bs * Hkv * d, bt[b:b + 1],
+                         np.zeros(1, np.int32), bs)
+    assert np.array_equal(kc, kc2) and np.array_equal(vc, vc2)
+
+
+# ------------------------------------------------------------------ attention
+def sdpa_reference(c):
+    """Contiguous attention through torch's scaled_dot_product_attention in fp64,
+    on the K/V gathered in logical order (an independent library routine)."""
+    B, Hq, Hkv, d = c["B"], c["Hq"], c["Hkv"], c["d"]
+    out = np.zeros((B, Hq, d))
+    q = bf16_vals(c["q"]).reshape(B, Hq, d)
+    for b in range(B):
+        K, V = gather_logical(c, b)
+        Kt = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)  # [Hq, n, d]
+        Vt = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)
+        qt = torch.from_numpy(q[b]).unsqueeze(1)  # [Hq, 1, d]
+        o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, scale=1 / math.sqrt(d))
+        out[b] = o[:, 0].numpy()
+    return out
+
+
+@pytest.mark.parametrize("seed,Hq,Hkv,d,bs", [(1, 8, 2, 16, 4), (2, 4, 4, 8, 3), (3, 16, 2, 64, 16),
+                                              (4, 8, 1, 32, 5)])
+def test_decode_equals_contiguous_sdpa(seed, Hq, Hkv, d, bs):
+    c = rand_case(seed, Hq=Hq, Hkv=Hkv, d=d, bs=bs, N=60, lens=(1, 9, 2 * bs + 1))
+    np.testing.assert_allclose(run_decode(c), sdpa_reference(c), rtol=1e-12, atol=1e-12)
+
+
+def test_decode_invariant_under_physical_block_permutation():
+    c = rand_case(5, lens=(3, 11, 17), N=30)
+    base = run_decode(c)
+    rng = np.random.default_rng(0)
+    perm = rng.permutation(c["N"])              # new position of each old block
+    inv = np.argsort(perm)
+    c2 = dict(c)
+    c2["kc"] = c["kc"][inv]                    # block p moves to perm[p]
+    c2["vc"] = c["vc"][inv]
+    c2["bt"] = np.where(c["bt"] >= 0, perm[np.maximum(c["bt"], 0)], -1).astype(np.int32)
+    assert np.array_equal(run_decode(c2), base)
+
+
+def test_decode_len_one_returns_v0_and_len_zero_returns_zero():
+    c = rand_case(6, lens=(1, 1, 0))
+    out = run_decode(c)
+    for b in range(2):
+        _, V = gather_logical(c, b)
+        for i in range(c["Hq"]):
+            assert np.array_equal(out[b, i], V[0, i // (c["Hq"] // c["Hkv"])])
+    assert not out[2].any()
+
+
+def test_decode_equal_keys_gives_mean_of_values():
+    c = rand_case(7, lens=(5, 13, 8))
+    kc = c["kc"].copy()
+    kc[...] = bf16_bits(np.linspace(-1, 1, c["d"]))  # every key the same vector
+    c["kc"] = kc
+    out = run_decode(c)
+    for b in range(c["B"]):
+        _, V = gather_logical(c, b)
+        G = c["Hq"] // c["Hkv"]
+        for i in range(c["Hq"]):
+            np.testing.assert_allclose(out[b, i], V[:, i // G].mean(0), rtol=1e-13, atol=1e-13)
+
+
+def test_decode_gqa_groups_are_contiguous():
+    # V[t, h, :] = h + 1 everywhere: each output is the constant of its kv head,
+    # so query head i must read kv head i // G (not i % Hkv).
+    c = rand_case(8, Hq=8, Hkv=4, lens=(6, 3, 10))
+    vc = np.empty_like(c["vc"])
+    for h in range(4):
+        vc[:, :, h, :] = bf16_bits(np.full(c["d"], h + 1.0))
+    c["vc"] = vc
+    out = run_decode(c)
+    for i in range(8):
+        np.testing.assert_allclose(out[:, i, :], i // 2 + 1.0, rtol=0, atol=1e-14)
+
+
+def test_decode_dominant_key_selects_its_value():
+    c = rand_case(9, Hq=2, Hkv=1, lens=(12, 12, 12))
+    kc = c["kc"].copy()
+    qv = bf16_vals(c["q"])
+    for b in range(c["B"]):
+        t = 5 + b
+        blk, off = c["bt"][b, t // c["bs"]], t % c["bs"]
+        kc[blk, off, 0] = bf16_bits(qv[b, 0] * 64.0)   # key aligned with query head 0, huge
+    c["kc"] = kc
+    out = run_decode(c)
+    for b in range(c["B"]):
+        _, V = gather_logical(c, b)
+        np.testing.assert_allclose(out[b, 0], V[5 + b, 0], atol=1e-8)
+
+
+def test_decode_never_reads_slots_beyond_len():
+    c = rand_case(10, lens=(5, 9, 3))
+    base = run_decode(c)
+    kc, vc = c["kc"].copy(), c["vc"].copy()
+    nan = bf16_bits(np.full(c["d"], np.nan))
+    for b in range(c["B"]):
+        n = int(c["lens"][b])
+        last = c["bt"][b, (n - 1) // c["bs"]]
+        for off in range(n % c["bs"] or c["bs"], c["bs"]):
+            kc[last, off] = nan
+            vc[last, off] = nan
+    c["kc"], c["vc"] = kc, vc
+    assert np.array_equal(run_decode(c), base)
+
+
+def test_decode_brute_force_python_loops_tiny_workload():
+    wl = W.generate(W.CONFIGS["c1"], "cpu")
+    s = W.compact(wl, 0, range(2))
+    kc, vc = s["k_pool"].copy(), s["v_pool"].copy()
+    Hkv, d, bs = 2, 64, 16
+    oracle.append_kv(s["k_new"], s["v_new"], kc, vc, bs * Hkv * d, s["block_tables"],
+                     s["positions"], bs)
+    out = oracle.paged_decode(s["q"], kc, vc, bs * Hkv * d, s["block_tables"], s["ctx_lens"],
+                              Hkv, bs, 1 / 8)
+    qv = bf16_vals(s["q"])
+    Kp, Vp = bf16_vals(kc), bf16_vals(vc)
+    for b in range(2):
+        n = int(s["ctx_lens"][b])
+        for i in range(4):
+            h = i // 2
+            sc = []
+            for t in range(n):
+                blk = int(s["block_tables"][b][t // bs])
+                kv = Kp[blk, t % bs, h]
+                sc.append(sum(qv[b, i, e] * kv[e] for e in range(d)) / 8)
+            mx = max(sc)
+            w = [math.exp(x - mx) for x in sc]
+            z = sum(w)
+            for e in range(0, d, 9):
+                o = sum(w[t] * Vp[int(s["block_tables"][b][t // bs]), t % bs, h, e]
+                        for t in range(n)) / z
+                assert abs(o - out[b, i, e]) < 1e-12
+
+
+def test_global_softmax_differs_from_per_block_normalisation():
+    """Reading check: the vLLM notes' pseudocode normalises inside each block and
+    sums block outputs; the operator of the knowledge page takes softmax over all
+    blocks.  The two disagree on any multi-block context, so the oracle must match
+    only the global one (already pinned against SDPA)."""
+    c = rand_case(12, lens=(9, 9, 9))
+    out = run_decode(c)
+    b, i = 0, 0
+    K, V = gather_logical(c, b)
+    q = bf16_vals(c["q"])[b, i]
+    per_block = np.zeros(c["d"])
+    for j in range(0, 9, c["bs"]):
+        s = K[j:j + c["bs"], 0] @ q / math.sqrt(c["d"])
+        p = np.exp(s - s.max())
+        per_block += (p / p.sum()) @ V[j:j + c["bs"], 0]
+    assert np.abs(per_block - out[b, i]).max() > 1e-3
+
+
+# ------------------------------------------------------------------ scores / eviction
+def test_score_is_norm_ratio_closed_forms():
+    B, Hkv, d, bs, N = 1, 2, 4, 2, 3
+    kc = np.zeros((N, bs, Hkv, d), np.float32)
+    vc = np.zeros_like(kc)
+    bt = np.array([[2, 0]], np.int32)
+    kc[2, 0, 0] = [3, 0, 0, 0]; vc[2, 0, 0] = [0, 4, 0, 0]     # 4/3
+    kc[2, 0, 1] = [1, 1, 1, 1]; vc[2, 0, 1] = [2, 2, 2, 2]     # 2
+    kc[2, 1, 0] = [0, 0, 0, 0]; vc[2, 1, 0] = [1, 0, 0, 0]     # ||K||=0, ||V||>0: +inf
+    kc[2, 1, 1] = [0, 0, 0, 0]; vc[2, 1, 1] = [0, 0, 0, 0]     # both zero: 0
+    kc[0, 0, 0] = [1, 2, 2, 0]; vc[0, 0, 0] = [6, 0, 0, 0]     # 6/3
+    kc[0, 0, 1] = [-2, 0, 0, 0]; vc[0, 0, 1] = [-0.5, 0, 0, 0]  # 0.25
+    s = oracle.score_tokens(bf16_bits(kc).ravel(), bf16_bits(vc).ravel(), bs * Hkv * d, bt,
+                            np.array([3], np.int32), Hkv, d, bs)
+    assert s.shape == (1, 4, 2)
+    np.testing.assert_allclose(s[0, :3].ravel(), [4 / 3, 2, np.inf, 0, 2, 0.25], rtol=1e-15)
+    assert np.isnan(s[0, 3]).all()
+
+
+def test_score_value_proportional_to_key_gives_constant():
+    c = rand_case(13, lens=(7, 11, 4), d=32)
+    kv = bf16_vals(c["kc"])
+    for cval in (0.5, -2.0, 4.0):                       # powers of two: V stays exact in bf16
+        vc = bf16_bits(kv * cval)
+        s = oracle.score_tokens(c["kc"].ravel(), vc.ravel(), c["bs"] * c["Hkv"] * c["d"], c["bt"],
+                                c["lens"], c["Hkv"], c["d"], c["bs"])
+        for b in range(c["B"]):
+            np.testing.assert_allclose(s[b, :c["lens"][b]], abs(cval), rtol=1e-14)
+
+
+def test_score_matches_numpy_norms():
+    c = rand_case(14, lens=(7, 11, 13), d=16)
+    s = oracle.score_tokens(c["kc"].ravel(), c["vc"].ravel(), c["bs"] * c["Hkv"] * c["d"],
+                            c["bt"], c["lens"], c["Hkv"], c["d"], c["bs"])
+    for b in range(c["B"]):
+        K, V = gather_logical(c, b)
+        ref = np.linalg.norm(V, axis=-1) / np.linalg.norm(K, axis=-1)
+        np.testing.assert_allclose(s[b, :c["lens"][b]], ref, rtol=1e-13)
+
+
+def test_evict_planted_low_block_and_rules():
+    B, Hkv, bs, MB = 4, 2, 4, 5
+    rng = np.random.default_rng(3)
+    scores = rng.uniform(1.0, 2.0, (B, MB * bs, Hkv))
+    lens = np.array([20, 13, 3, 17], np.int32)   # full blocks: 5, 3, 0, 4
+    scores[0, 8:12] = 0.5                        # block 2 of seq 0
+    scores[1, 4:8] = 0.75                        # block 1 of seq 1
+    scores[1, 12:16] = 0.01                      # seq 1 block 3 is partial: not a candidate
+    scores[3, :] = 1.5                           # seq 3: all equal -> lowest index wins
+    ev, means, gap = oracle.select_evict_block(scores, lens, bs)
+    assert ev.tolist() == [2, 1, -1, 0]
+    np.testing.assert_allclose(means[0, 2], 0.5)
+    assert np.isnan(means[1, 3]) and np.isnan(means[2]).all()
+    assert gap[3] == 0.0 and gap[2] == np.inf
+    # brute force of the block means for seq 0
+    for j in range(5):
+        assert abs(means[0, j] - scores[0, j * bs:(j + 1) * bs].mean()) < 1e-15
+
+
+def test_evict_scaled_value_block_is_chosen():
+    c = rand_case(15, lens=(16, 16, 16), bs=4, d=16)
+    vc = c["vc"].copy()
+    for b in range(3):
+        blk = c["bt"][b, 1 + b]
+        vc[blk] = bf16_bits(bf16_vals(vc[blk]) * 0.125)
+    s = oracle.score_tokens(c["kc"].ravel(), vc.ravel(), c["bs"] * c["Hkv"] * c["d"], c["bt"],
+                            c["lens"], c["Hkv"], c["d"], c["bs"])
+    ev, _, _ = oracle.select_evict_block(s, c["lens"], c["bs"])
+    assert ev.tolist() == [1, 2, 3]
+
+
+# ------------------------------------------------------------------ int8
+def test_quantiser_golden_rows():
+    with open(os.path.join(GOLDEN, "int8_rows.txt")) as f:
+        rows = [ln for ln in f if ln.strip() and not ln.startswith("#")]
+    for ln in rows:
+        xs, s, qs = ln.split("|")
+        x = np.array(xs.split(), np.float32)
+        codes, scales = oracle.quantize_int8(bf16_bits(x)[None])
+        assert scales[0] == np.float32(s)
+        assert codes[0].tolist() == [int(v) for v in qs.split()]
+
+
+def test_quantiser_range_and_error_bound():
+    rng = np.random.default_rng(16)
+    x = rng.standard_normal((500, 128)) * rng.uniform(0.01, 30, (500, 1))
+    bits = bf16_bits(x)
+    codes, scales = oracle.quantize_int8(bits)
+    xv = bf16_vals(bits)
+    assert np.abs(codes).max() <= 127
+    assert (np.abs(codes).max(axis=1) == 127).all()          # the amax element maps to +-127
+    deq = scales[:, None].astype(np.float64) * codes
+    # |code - x/s| <= 1/2 plus the one fp32 rounding of x/s (|x/s| <= 127)
+    bound = scales[:, None].astype(np.float64) * (0.5 + 127 * 2.0 ** -24)
+    assert (np.abs(deq - xv) <= bound).all()
+
+
+def test_int8_decode_equals_sdpa_on_dequantised_values():
+    c = rand_case(17, Hq=8, Hkv=2, d=32, bs=4, N=20, lens=(4, 9, 14))
+    kq, ks = oracle.quantize_int8(c["kc"])
+    vq, vs = oracle.quantize_int8(c["vc"])
+    out = oracle.paged_decode_int8(c["q"], kq.ravel(), vq.ravel(), ks.ravel(), vs.ravel(),
+                                   c["bs"] * c["Hkv"] * c["d"], c["bt"], c["lens"], c["Hkv"],
+                                   c["bs"], 1 / math.sqrt(c["d"]))
+    kd = ks[..., None].astype(np.float64) * kq
+    vd = vs[..., None].astype(np.float64) * vq
+    B, Hq, Hkv, d = c["B"], c["Hq"], c["Hkv"], c["d"]
+    q = bf16_vals(c["q"])
+    for b in range(B):
+        n = int(c["lens"][b])
+        ids = c["bt"][b, : -(-n // c["bs"])]
+        K = kd[ids].reshape(-1, Hkv, d)[:n]
+        V = vd[ids].reshape(-1, Hkv, d)[:n]
+        Kt = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)
+        Vt = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)
+        o = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[b]).unsqueeze(1), Kt, Vt, scale=1 / math.sqrt(d))[:, 0].numpy()
+        np.testing.assert_allclose(out[b], o, rtol=1e-12, atol=1e-12)
+
+
+def test_int8_append_matches_quantiser_and_slots():
+    rng = np.random.default_rng(18)
+    B, Hkv, d, bs, N, MB = 2, 2, 16, 4, 10, 3
+    bt = np.array([[3, 7, -1], [1, 0, 9]], np.int32)
+    kq = np.zeros(N * bs * Hkv * d, np.int8)
+    vq = np.zeros_like(kq)
+    ks = np.zeros(N * bs * Hkv, np.float32)
+    vs = np.zeros_like(ks)
+    kn = bf16_bits(rng.standard_normal((B, 3, Hkv, d)))
+    vn = bf16_bits(rng.standard_normal((B, 3, Hkv, d)))
+    pos = np.array([2, 7], np.int32)
+    slots = oracle.append_kv_int8(kn, vn, kq, vq, ks, vs, bs * Hkv * d, bt, pos, bs)
+    assert slots.tolist() == [[14, 15, 28], [3, 36, 37]]
+    cq, cs = oracle.quantize_int8(kn)
+    kq4 = kq.reshape(N * bs, Hkv, d)
+    ks2 = ks.reshape(N * bs, Hkv)
+    for b in range(B):
+        for i in range(3):
+            assert np.array_equal(kq4[slots[b, i]], cq[b, i])
+            assert np.array_equal(ks2[slots[b, i]], cs[b, i])
