@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the paged KV decode attention library.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c3] [--impl ours|reference]
+
+One step is one decode step of the chosen workload through the C ABI:
+for every layer, the KV append of the new token and paged decode attention
+(c2 adds the PagedEviction score pass and block selection per layer).  Default
+workload: c3, the Llama-3-8B-shape decode (32 layers, 32/8 heads, d=128,
+batch 64, contexts uniform in [512, 8192], block 16), whose pools (~40 GB)
+exceed L2, so no flush is needed between steps.
+
+Prints ONE JSON line (rank 0).  value = decode tokens/s of the whole job
+(batch x ranks / step time, device-timed, max over ranks); the roofline object
+covers the decode kernel (algorithmic bytes / event-timed duration).
+N > 1 (torchrun): every rank runs its own replica of the batch on its own GPU
+(sequences are independent; no collective on the data path), weak scaling.
+
+--impl reference times the fp64 CPU oracle (the correctness reference) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_396_b200 import workloads as W  # noqa: E402
+
+METRIC = "paged decode-attention HBM GB/s (% of B200 peak) and decode tokens/s at 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+DECODE_SOURCES = ["decode_simple.cu", "decode_tc.cu", "kernels.h", "common.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="c3", choices=["c2", "c3", "c4", "c5"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        p = os.path.join(ROOT, "paged_kv_cache_396_b200", "csrc", f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """dram bytes per decode launch from the committed ncu summary, if it was
+    taken on the current decode sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    want = decode_source_hash()
+    for line in open(p):
+        kv = dict(x.split("=", 1) for x in line.split() if "=" in x)
+        if kv.get("workload") == workload and kv.get("sources") == want:
+            return float(kv["bytes_per_launch"])
+    return None
+
+
+class Clocks:
+    """nvidia-smi sampler (200 ms) running during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- model
+def decode_algorithmic_bytes(cfg, ctx_lens, S, chunk):
+    """Bytes one decode launch (one layer) must move: K/V rows of every cached
+    token (plus INT8 scales), q and out, the table entries read, and the
+    partition partials written and read back when S > 1."""
+    elt = 1 if cfg.int8 else 2
+    tok = int(np.sum(ctx_lens))
+    kv = tok * cfg.hkv * cfg.head_dim * 2 * elt
+    if cfg.int8:
+        kv += tok * cfg.hkv * 2 * 4
+    qo = 2 * cfg.batch * cfg.hq * cfg.head_dim * 2
+    nblk = int(sum(-(-int(n) // cfg.block_size) for n in ctx_lens))
+    table = nblk * 4 + cfg.batch * 4
+    parts = 0
+    if S > 1:
+        n_parts = int(sum(max(1, -(-int(n) // chunk)) for n in ctx_lens))
+        parts = 2 * n_parts * cfg.hq * (cfg.head_dim + 2) * 4
+    return kv + qo + table + parts
+
+
+class Runner:
+    """Device state and one decode step of a workload through the binding."""
+
+    def __init__(self, cfg, device, num_splits=0):
+        from paged_kv_cache_396_b200 import pagedkv as pk
+        self.pk, self.cfg, self.dev = pk, cfg, device
+        wl = W.generate(cfg, device)
+        self.wl = wl
+        self.L = cfg.layers
+        self.bt = torch.as_tensor(wl.block_tables, device=device)
+        self.ctx = torch.as_tensor(wl.ctx_lens, device=device)
+        self.pos = torch.as_tensor(wl.positions, device=device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        B, Hq, Hkv, d, bs = cfg.batch, cfg.hq, cfg.hkv, cfg.head_dim, cfg.block_size
+        MB = wl.max_blocks
+        self.out = torch.empty(self.L, B, Hq, d, dtype=torch.bfloat16, device=device)
+        self.ws = pk.alloc_workspace(B, Hq, Hkv, d, bs, MB, num_splits, device)
+        self.num_splits = num_splits
+        self.S, self.chunk = pk.pa_decode_plan(B, Hq, Hkv, d, bs, MB, num_splits)
+        if cfg.int8:
+            N = wl.num_blocks
+            self.kq = torch.zeros(self.L, N, bs, Hkv, d, dtype=torch.int8, device=device)
+            self.vq = torch.zeros_like(self.kq)
+            self.ks = torch.zeros(self.L, N, bs, Hkv, dtype=torch.float32, device=device)
+            self.vs = torch.zeros_like(self.ks)
+            zeros = torch.zeros(B, dtype=torch.int32, device=device)
+            for l in range(self.L):
+                n = int(wl.old_lens.max())
+                assert (wl.old_lens == n).all()
+                pk.pa_append_kv_int8(wl.k_hist[l, :, :n].contiguous(),
+                                     wl.v_hist[l, :, :n].contiguous(), self.kq[l], self.vq[l],
+                                     self.ks[l], self.vs[l], self.bt, zeros, self.err)
+            wl.k_hist = wl.v_hist = None
+        if cfg.score:
+            self.scores = torch.zeros(B, MB * bs, Hkv, dtype=torch.float32, device=device)
+            self.evict = torch.zeros(B, dtype=torch.int32, device=device)
+        torch.cuda.synchronize(device)
+        self.q = wl.q
+        self.k_new, self.v_new = wl.k_new, wl.v_new
+        self.decode_bytes = decode_algorithmic_bytes(cfg, wl.ctx_lens, self.S, self.chunk)
+
+    def launches_per_step(self):
+        per_layer = (1 if self.cfg.append else 0) + (2 if self.S > 1 else 1)
+        if self.cfg.score:
+            per_layer += 2
+        return per_layer * self.L
+
+    def step(self, ev=None):
+        pk, cfg = self.pk, self.cfg
+        for l in range(self.L):
+            if cfg.int8:
+                pk.pa_append_kv_int8(self.k_new[l], self.v_new[l], self.kq[l], self.vq[l],
+                                     self.ks[l], self.vs[l], self.bt, self.pos, self.err)
+                if ev is not None:
+                    ev[l][0].record()
+                pk.pa_decode_int8(self.out[l], self.q[l], self.kq[l], self.vq[l], self.ks[l],
+                                  self.vs[l], self.bt, self.ctx, self.wl.scale, self.err, self.ws,
+                                  self.num_splits)
+            else:
+                kp = self.wl.k_pool[l]
+                vp = self.wl.v_pool[l]
+                if cfg.append:
+                    pk.pa_append_kv(self.k_new[l], self.v_new[l], kp, vp, self.bt, self.pos,
+                                    self.err)
+                if ev is not None:
+                    ev[l][0].record()
+                pk.pa_decode(self.out[l], self.q[l], kp, vp, self.bt, self.ctx, self.wl.scale,
+                             self.err, self.ws, self.num_splits)
+            if ev is not None:
+                ev[l][1].record()
+            if cfg.score:
+                pk.pe_score_tokens(self.scores, self.wl.k_pool[l], self.wl.v_pool[l], self.bt,
+                                   self.ctx, self.err)
+                pk.pe_select_evict_block(self.evict, self.scores, self.ctx, cfg.block_size)
+
+
+# ----------------------------------------------------------------------------- oracle
+def oracle_throughput(wl, budget_s, max_layers=None):
+    """Time the fp64 oracle (append + decode, plus score + select for c2) on
+    (layer, sequence-batch) samples of the workload for about budget_s seconds;
+    scale to decode tokens/s of the whole step.  Returns (tokens/s, cores, desc)."""
+    import oracle
+    cfg = wl.cfg
+    cores = oracle.threads()
+    per_call = max(8, min(cfg.batch, cores))
+    Hkv, d, bs = cfg.hkv, cfg.head_dim, cfg.block_size
+    stride = bs * Hkv * d
+    t_total, tok_total, n_calls = 0.0, 0, 0
+    layers = wl.q.shape[0] if max_layers is None else min(max_layers, wl.q.shape[0])
+    order = [(l, s) for l in range(layers) for s in range(0, cfg.batch, per_call)]
+    for l, s0 in order:
+        seqs = list(range(s0, min(cfg.batch, s0 + per_call)))
+        c = W.compact(wl, l, seqs)
+        t0 = time.perf_counter()
+        if cfg.int8:
+            n = c["num_blocks"]
+            kq = np.zeros(n * stride, np.int8); vq = np.zeros_like(kq)
+            ks = np.zeros(n * bs * Hkv, np.float32); vs = np.zeros_like(ks)
+            oracle.append_kv_int8(c["k_hist"], c["v_hist"], kq, vq, ks, vs, stride,
+                                  c["block_tables"], np.zeros(len(seqs), np.int32), bs)
+            t0 = time.perf_counter()   # the history fill is set-up, not the step
+            oracle.append_kv_int8(c["k_new"], c["v_new"], kq, vq, ks, vs, stride,
+                                  c["block_tables"], c["positions"], bs)
+            oracle.paged_decode_int8(c["q"], kq, vq, ks, vs, stride, c["block_tables"],
+                                     c["ctx_lens"], Hkv, bs, wl.scale)
+        else:
+            kc, vc = c["k_pool"].ravel(), c["v_pool"].ravel()
+            if "k_new" in c:
+                oracle.append_kv(c["k_new"], c["v_new"], kc, vc, stride, c["block_tables"],
+                                 c["positions"], bs)
+            oracle.paged_decode(c["q"], kc, vc, stride, c["block_tables"], c["ctx_lens"], Hkv, bs,
+                                wl.scale)
+            if cfg.score:
+                sc = oracle.score_tokens(kc, vc, stride, c["block_tables"], c["ctx_lens"], Hkv, d,
+                                         bs)
+                oracle.select_evict_block(sc, c["ctx_lens"], bs)
+        t_total += time.perf_counter() - t0
+        tok_total += int(np.sum(c["ctx_lens"]))
+        n_calls += 1
+        if t_total >= budget_s:
+            break
+    full_tok = int(np.sum(wl.ctx_lens)) * cfg.layers
+    step_s = t_total / tok_total * full_tok
+    desc = (f"{n_calls} oracle calls over {tok_total} context tokens "
+            f"({per_call} sequences per call, layers 0..{layers - 1}), {t_total:.1f} s, "
+            f"scaled by {full_tok} context tokens per step")
+    return cfg.batch / step_s, cores, desc
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = W.CONFIGS[args.workload]
+    wl = W.generate(cfg, "cpu", layers=1)
+    per = max(1.0, args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        oracle_throughput(wl, per / 4, max_layers=1)
+    vals = []
+    desc = ""
+    cores = 0
+    for _ in range(args.steps):
+        v, cores, desc = oracle_throughput(wl, per, max_layers=1)
+        vals.append(v)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * cfg.batch / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(cfg),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": "per step: " + desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(cfg):
+    lens = (f"{cfg.old_lens[0]}" if cfg.old_lens and len(set(cfg.old_lens)) == 1
+            else f"uniform[{cfg.old_len_range[0]},{cfg.old_len_range[1]}]"
+            if cfg.old_len_range else "mixed")
+    return {
+        "workload": f"{cfg.key} {cfg.name}", "layers": cfg.layers, "global_batch": cfg.batch,
+        "q_heads": cfg.hq, "kv_heads": cfg.hkv, "head_dim": cfg.head_dim,
+        "block_size": cfg.block_size, "cached_tokens": lens,
+        "append": cfg.append, "score_pass": cfg.score, "kv_dtype": "int8" if cfg.int8 else "bf16",
+        "l2": "working set larger than L2 every step (no flush needed)",
+    }
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    cfg = W.CONFIGS[args.workload]
+    r = Runner(cfg, device, args.num_splits)
+    stream = torch.cuda.current_stream(device)
+
+    for _ in range(max(3, args.warmup)):
+        r.step()
+    torch.cuda.synchronize(device)
+    if r.err.item() != 0:
+        raise SystemExit(f"device error flag {r.err.item()} during warm-up")
+
+    # --- device-timed region: K steps, events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+          for _ in range(r.L * args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    clocks = Clocks(device)
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        r.step(ev[k * r.L:(k + 1) * r.L])
+    t_end.record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    decode_ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor([total_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * cfg.batch / (ms_per_step / 1000.0)
+    dec_avg_s = statistics.mean(decode_ms) / 1000.0
+    achieved = r.decode_bytes / dec_avg_s / 1e9
+    peak, peak_kind = peaks()
+
+    # --- end to end: host inputs -> C ABI -> host outputs, copies inside the timed region
+    B, Hq, Hkv, d = cfg.batch, cfg.hq, cfg.hkv, cfg.head_dim
+    h_q = torch.empty(r.q.shape, dtype=torch.bfloat16, pin_memory=True)
+    h_q.copy_(r.q)
+    h_out = torch.empty(r.out.shape, dtype=torch.bfloat16, pin_memory=True)
+    h_in = [h_q]
+    d_in = [r.q]
+    if cfg.append:
+        for t in (r.k_new, r.v_new):
+            h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            h.copy_(t)
+            h_in.append(h)
+            d_in.append(t)
+    h_ctx = torch.as_tensor(r.wl.ctx_lens).pin_memory()
+    h_pos = torch.as_tensor(r.wl.positions).pin_memory()
+    h_in += [h_ctx, h_pos]
+    d_in += [r.ctx, r.pos]
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_steps = max(3, min(args.steps, 50))
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for h, dv in zip(h_in, d_in):
+            dv.copy_(h, non_blocking=True)
+        r.step()
+        h_out.copy_(r.out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": world * B / (e2e_ms / 1000.0), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    if r.err.item() != 0:
+        raise SystemExit(f"device error flag {r.err.item()} during timing")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, desc = oracle_throughput(r.wl, args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        traffic = recorded_traffic(args.workload)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8" if cfg.int8 else "bf16", "data": "synthetic",
+            "config": dict(workload_config(cfg), parallelism=f"replicas{world}",
+                           num_splits=r.S, chunk_tokens=r.chunk),
+            "roofline": {"bound": "hbm", "kernel": "pa_decode" + ("_int8" if cfg.int8 else ""),
+                         "achieved": achieved, "peak": peak, "peak_source": peak_kind,
+                         "unit": "GB/s", "frac": achieved / peak,
+                         "frac_of_nominal_8tbs": achieved / 8000.0,
+                         "traffic": traffic, "algorithmic_bytes_per_launch": r.decode_bytes,
+                         "avg_launch_us": dec_avg_s * 1e6},
+            "decode_only_tokens_per_s": world * B / (sum(decode_ms) / args.steps / 1000.0),
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": r.launches_per_step() * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,199 @@
+/*
+ * pagedkv.h -- C ABI of the B200 (sm_100a) paged-KV decode attention library
+ * (libpagedkv.so).
+ *
+ * Operations and the passages that define them (web pages, by title/section):
+ *   [VKV]  ybb.press "LLM 推理 KV Cache 内存管理深度工程实践：从 PageAttention 到推测解码":
+ *          §2.1 BlockTable (block table, ceil block count, append_slot),
+ *          §2.2 paged_attention_forward(query, paged_kv_cache, block_table,
+ *          context_len, scale), §6.1 INT8/FP8 KV cache (quantize_kv_cache),
+ *          §6.2 GQA (every G query heads share one KV head).
+ *   [KVP]  t6page.pages.dev "KV cache": "PagedAttention 的算子" (K/V looked up
+ *          through the block table, softmax taken over all blocks together).
+ *   [KVL]  blog.hotdry.top "KV缓存内存布局优化": "PagedEviction 块级驱逐机制"
+ *          (token importance S = ||V||_2 / ||K||_2, decode-phase eviction of the
+ *          complete block with the lowest mean importance).
+ *   [NANO] blog.hotdry.top nano-vLLM KV cache: the [2, L, blocks, bs, n_kv, d]
+ *          tensor, reached here through per-layer K and V base pointers.
+ *
+ * Conventions shared by every entry point
+ *   - All data pointers are DEVICE pointers owned by the caller; the library
+ *     allocates nothing and keeps no state between calls except what the
+ *     caller passes in (the decode workspace).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and returns after enqueueing.
+ *   - Return value: PA_OK (0) when the work was enqueued; a negative PA_ERR_*
+ *     code when an argument is invalid, in which case nothing is launched.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Physical KV pool of one layer: [N blocks][bs slots][Hkv heads][d],
+ *     element (blk, slot, h, e) at blk*block_stride + (slot*Hkv + h)*d + e,
+ *     with block_stride >= bs*Hkv*d elements ([VKV] §2.2 shape
+ *     [num_gpu_blocks, block_size, num_kv_heads, head_dim]).
+ *   - Block table: int32 [B][MB] (MB = max blocks per sequence); entry j of row
+ *     b is the physical block of logical block j.  Only entries below
+ *     ceil(len_b / bs) are read.
+ *   - Device-detected faults never trap: the kernel ORs a PA_DEV_* bit into
+ *     *err_flag (a caller-zeroed device int32, required) and skips the
+ *     offending block or sequence.
+ *   - Supported sizes: d in {64, 128}; Hq % Hkv == 0 with G = Hq/Hkv <= 16;
+ *     bs >= 1 (bs a multiple of 16 selects the staged tensor-core decode);
+ *     pool/base pointers 16-byte aligned and block_stride*elt a multiple of 16.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- host status codes ---------------------------------------------------- */
+#define PA_OK             0
+#define PA_ERR_NULL      -1  /* a required pointer is NULL                          */
+#define PA_ERR_SHAPE     -2  /* unsupported or inconsistent sizes                   */
+#define PA_ERR_ALIGN     -3  /* pointer or stride not 16-byte aligned               */
+#define PA_ERR_WORKSPACE -4  /* workspace missing or smaller than required          */
+#define PA_ERR_CUDA      -5  /* a CUDA runtime call or kernel launch failed          */
+#define PA_ERR_DEVICE    -6  /* current device is not an sm_100 GPU                  */
+
+/* ---- device error-flag bits (ORed into *err_flag) ------------------------- */
+#define PA_DEV_BAD_BLOCK  1  /* a needed block-table entry was outside [0, N)       */
+#define PA_DEV_BAD_LEN    2  /* a context length / position outside [0, MB*bs]     */
+#define PA_DEV_TIMEOUT    4  /* a bounded pipeline wait gave up (kernel returned)   */
+
+/* Human-readable text of a PA_* status code (static storage). */
+const char *pa_status_string(int code);
+
+/* Library version string (static storage). */
+const char *pa_version(void);
+
+/* ============================================================================
+ * a1. KV append  ([VKV] §2.1 append_slot)
+ *
+ * Writes n_new tokens per sequence into the paged pools.  Token i of sequence b
+ * (i < n_new) has position p = positions[b] + i and lands in
+ *     slot = block_tables[b][p / bs] * bs + p % bs,
+ * i.e. physical block block_tables[b][p / bs], offset p % bs, for every kv head.
+ * n_new = 1 is the decode-step append; n_new > 1 writes a prompt (prefill).
+ * The caller's allocator must already have placed every needed block in the
+ * table (the append allocates nothing).
+ *   k_new, v_new : [B][n_new][Hkv][d] bf16, contiguous.
+ *   k_cache, v_cache : one layer's pools (see conventions), written.
+ *   slot_out     : optional [B][n_new] int64, receives the slots (NULL = skip).
+ * Device errors: p outside [0, MB*bs) -> PA_DEV_BAD_LEN; table entry outside
+ * [0, N) -> PA_DEV_BAD_BLOCK; that token is skipped.
+ * ==========================================================================*/
+int pa_append_kv(const uint16_t *k_new, const uint16_t *v_new,
+                 uint16_t *k_cache, uint16_t *v_cache, int64_t block_stride,
+                 const int32_t *block_tables, int max_blocks_per_seq,
+                 const int32_t *positions, int B, int n_new, int Hkv, int d, int bs,
+                 int64_t num_blocks, int64_t *slot_out, int32_t *err_flag, void *stream);
+
+/* ============================================================================
+ * a2 + a3. Paged decode attention  ([VKV] §2.2; [KVP] operator; [VKV] §6.2)
+ *
+ * For every sequence b and query head i, with G = Hq / Hkv and kv head
+ * h = i / G (contiguous GQA groups):
+ *     out[b][i] = sum_t softmax_t(scale * q[b][i] . K[b, t, h]) V[b, t, h]
+ * over the tokens t < ctx_lens[b] read through the block table, the softmax
+ * being taken over the whole context.  Computed with an online softmax in fp32
+ * over a split-KV partition of the context, then a log-sum-exp merge of the
+ * partitions; the result is rounded to bf16 (nearest-even).  ctx_lens[b] == 0
+ * gives a zero row.
+ *   out : [B][Hq][d] bf16, written.          q : [B][Hq][d] bf16.
+ *   ctx_lens : [B] int32 in [0, MB*bs] (the appended token included).
+ *   num_splits : maximum partitions per sequence; 0 = choose automatically.
+ *   workspace  : device scratch of at least pa_decode_workspace_bytes(...)
+ *                bytes for the same sizes and num_splits (may be NULL when that
+ *                is 0).  Its contents are scratch; calls sharing one workspace
+ *                must be ordered on one stream.
+ * Device errors: ctx_lens[b] outside [0, MB*bs] -> PA_DEV_BAD_LEN (row zeroed);
+ * a needed table entry outside [0, N) -> PA_DEV_BAD_BLOCK (block skipped).
+ * ==========================================================================*/
+size_t pa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int bs,
+                                 int max_blocks_per_seq, int num_splits);
+
+/* The partition pa_decode chooses for these sizes (no counterpart in the pages:
+ * the split-KV partition exists only in this implementation).  *num_splits_out
+ * receives the maximum number of partitions of one sequence (1 = no merge
+ * pass), *chunk_tokens_out the tokens per partition.  Returns PA_OK or a
+ * PA_ERR_* code. */
+int pa_decode_plan(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq,
+                   int num_splits, int *num_splits_out, int *chunk_tokens_out);
+
+int pa_decode(uint16_t *out, const uint16_t *q,
+              const uint16_t *k_cache, const uint16_t *v_cache, int64_t block_stride,
+              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *ctx_lens,
+              int B, int Hq, int Hkv, int d, int bs, int64_t num_blocks, float scale,
+              int num_splits, void *workspace, size_t workspace_bytes,
+              int32_t *err_flag, void *stream);
+
+/* ============================================================================
+ * a4. PagedEviction token importance  ([KVL] "PagedEviction 块级驱逐机制")
+ *
+ *   scores[b][t][h] = ||V[b, t, h, :]||_2 / ||K[b, t, h, :]||_2   (fp32)
+ * for t < ctx_lens[b] and every kv head h, on the stored bf16 values.  When
+ * ||K|| == 0 the score is +inf if ||V|| > 0, else 0.  Entries with
+ * t >= ctx_lens[b] are not written.
+ *   scores : [B][MB*bs][Hkv] fp32.
+ * ==========================================================================*/
+int pe_score_tokens(float *scores, const uint16_t *k_cache, const uint16_t *v_cache,
+                    int64_t block_stride, const int32_t *block_tables, int max_blocks_per_seq,
+                    const int32_t *ctx_lens, int B, int Hkv, int d, int bs,
+                    int64_t num_blocks, int32_t *err_flag, void *stream);
+
+/* ============================================================================
+ * a5. PagedEviction block selection  ([KVL] "PagedEviction 块级驱逐机制")
+ *
+ * For each sequence, over its FULL logical blocks j < floor(ctx_lens[b] / bs):
+ *   mean_j = (1 / (bs*Hkv)) * sum_{t in block j, h} scores[b][t][h]
+ * accumulated in fp64 (exact for the fp32 scores of one block), and
+ *   evict[b] = argmin_j mean_j  (lowest j on ties), or -1 if no block is full.
+ * The caller maps evict[b] to the physical block block_tables[b][evict[b]],
+ * drops it from the table and frees it (host bookkeeping, not done here).
+ *   evict       : [B] int32, written.
+ *   block_means : optional [B][MB] fp32 (fp64 mean rounded to nearest); NaN for
+ *                 non-candidate blocks.  NULL = skip.
+ *   scores      : [B][MB*bs][Hkv] fp32 as written by pe_score_tokens.
+ * ==========================================================================*/
+int pe_select_evict_block(int32_t *evict, float *block_means, const float *scores,
+                          const int32_t *ctx_lens, int B, int max_blocks_per_seq, int Hkv,
+                          int bs, void *stream);
+
+/* ============================================================================
+ * a6. INT8 KV append  ([VKV] §6.1 quantize_kv_cache; [VKV] §2.1 append_slot)
+ *
+ * As pa_append_kv, but every (token, kv head) row x[0..d) is quantised first:
+ *   s = max_e |x_e| / 127            (one IEEE fp32 division)
+ *   code_e = round_half_even(x_e / s) (IEEE fp32 division), int8 in [-127, 127]
+ *   s == 0  ->  all codes 0.
+ *   kq_cache, vq_cache : int8 pools [N][bs][Hkv][d] (block_stride elements).
+ *   k_scale, v_scale   : fp32 scale pools [N][bs][Hkv] (block stride bs*Hkv).
+ * ==========================================================================*/
+int pa_append_kv_int8(const uint16_t *k_new, const uint16_t *v_new,
+                      int8_t *kq_cache, int8_t *vq_cache, float *k_scale, float *v_scale,
+                      int64_t block_stride, const int32_t *block_tables, int max_blocks_per_seq,
+                      const int32_t *positions, int B, int n_new, int Hkv, int d, int bs,
+                      int64_t num_blocks, int64_t *slot_out, int32_t *err_flag, void *stream);
+
+/* ============================================================================
+ * a7. INT8 paged decode  ([VKV] §6.1 dequantisation; otherwise as pa_decode)
+ *
+ * pa_decode with K[t, h, e] = k_scale[t, h] * kq[t, h, e] and likewise V,
+ * dequantised in registers (the K scale multiplies the dot product, the V
+ * scale multiplies the softmax weight).  Same workspace rule as pa_decode.
+ * ==========================================================================*/
+int pa_decode_int8(uint16_t *out, const uint16_t *q,
+                   const int8_t *kq_cache, const int8_t *vq_cache,
+                   const float *k_scale, const float *v_scale, int64_t block_stride,
+                   const int32_t *block_tables, int max_blocks_per_seq, const int32_t *ctx_lens,
+                   int B, int Hq, int Hkv, int d, int bs, int64_t num_blocks, float scale,
+                   int num_splits, void *workspace, size_t workspace_bytes,
+                   int32_t *err_flag, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PAGEDKV_H */

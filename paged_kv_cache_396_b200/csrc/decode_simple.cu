@@ -1,0 +1,226 @@
+// decode_simple.cu -- paged decode attention, general-shape kernel, and the
+// cross-partition log-sum-exp merge shared by every decode kernel.
+//
+// Operator (ybb.press "LLM 推理 KV Cache 内存管理深度工程实践" §2.2; t6page.pages.dev
+// "KV cache", "PagedAttention 的算子"): for each sequence, K/V rows are found
+// through the block table and softmax(scale * q.K) V is taken over the whole
+// context.  GQA (§6.2 of the first page): query head i uses kv head i / G.
+//
+// This kernel handles any block size (one CTA per (partition, kv head,
+// sequence), one warp per token, CUDA-core fp32).  Block sizes that are a
+// multiple of 16 use the staged tensor-core kernel in decode_tc.cu instead.
+// Softmax runs online in the log2 domain: logits are pre-scaled by
+// scale*log2(e) so every exponential is an exp2.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pkv {
+
+template <int D, bool INT8>
+__device__ __forceinline__ void load_kv_row(const void *base, int64_t idx, float (&x)[D / 32]) {
+    constexpr int VEC = D / 32;
+    if constexpr (INT8) {
+        const int8_t *p = reinterpret_cast<const int8_t *>(base) + idx;
+        if constexpr (VEC == 4) {
+            const uint32_t w = __ldg(reinterpret_cast<const unsigned int *>(p));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[e] = (float)(int8_t)((w >> (8 * e)) & 0xffu);
+        } else {
+            const uint16_t w = __ldg(reinterpret_cast<const unsigned short *>(p));
+            x[0] = (float)(int8_t)(w & 0xffu);
+            x[1] = (float)(int8_t)(w >> 8);
+        }
+    } else {
+        const uint16_t *p = reinterpret_cast<const uint16_t *>(base) + idx;
+        if constexpr (VEC == 4) {
+            const uint2 w = __ldg(reinterpret_cast<const uint2 *>(p));
+            x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+        } else {
+            const uint32_t w = __ldg(reinterpret_cast<const unsigned int *>(p));
+            x[0] = bf16_lo(w); x[1] = bf16_hi(w);
+        }
+    }
+}
+
+// Grid (partition c, kv head h, sequence b); 4 warps; warp w takes tokens
+// t0+w, t0+w+4, ... of the partition and keeps its own online-softmax state
+// for the GP (>= G, power of two) query heads of the group; the four states are
+// merged through shared memory at the end.
+template <int D, int GP, bool INT8>
+__global__ void __launch_bounds__(128) decode_simple_kernel(DecodeArgs a) {
+    constexpr int VEC = D / 32;
+    constexpr int NW = 4;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int len = a.ctx_lens[b];
+    if (len < 0 || (int64_t)len > (int64_t)a.MB * a.bs) {
+        if (c == 0 && h == 0 && threadIdx.x == 0) raise_flag(a.err, PA_DEV_BAD_LEN);
+        len = 0;
+    }
+    const int t0 = c * a.chunk;
+    if (c > 0 && t0 >= len) return;  // partition past the context: the merge skips it
+    const int t1 = min(t0 + a.chunk, len);
+
+    float qf[GP][VEC];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+        if (g < a.G) {
+            float x[VEC];
+            const int64_t qi = ((int64_t)b * a.Hq + h * a.G + g) * D + lane * VEC;
+            load_kv_row<D, false>(a.q, qi, x);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) qf[g][e] = x[e] * a.scale_log2;
+        } else {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) qf[g][e] = 0.f;
+        }
+    }
+    float m[GP], l[GP], acc[GP][VEC];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+        m[g] = -INFINITY;
+        l[g] = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[g][e] = 0.f;
+    }
+
+    for (int t = t0 + warp; t < t1; t += NW) {
+        const int32_t phys = a.block_tables[(int64_t)b * a.MB + t / a.bs];
+        if (phys < 0 || (int64_t)phys >= a.N) {
+            if (lane == 0) raise_flag(a.err, PA_DEV_BAD_BLOCK);
+            continue;
+        }
+        const int slot = t % a.bs;
+        const int64_t row = (int64_t)phys * a.block_stride + ((int64_t)slot * a.Hkv + h) * D + lane * VEC;
+        float kf[VEC], vf[VEC];
+        load_kv_row<D, INT8>(a.k_cache, row, kf);
+        load_kv_row<D, INT8>(a.v_cache, row, vf);
+        float ks = 1.f, vs = 1.f;
+        if constexpr (INT8) {
+            const int64_t srow = ((int64_t)phys * a.bs + slot) * a.Hkv + h;
+            ks = __ldg(a.k_scale + srow);
+            vs = __ldg(a.v_scale + srow);
+        }
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) s = fmaf(qf[g][e], kf[e], s);
+            s = warp_sum(s) * ks;
+            const float mn = fmaxf(m[g], s);
+            const float alpha = exp2f(m[g] - mn);
+            const float p = exp2f(s - mn);
+            l[g] = l[g] * alpha + p;
+            const float pv = p * vs;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[g][e] = fmaf(pv, vf[e], acc[g][e] * alpha);
+            m[g] = mn;
+        }
+    }
+
+    __shared__ float sm_m[NW][GP], sm_l[NW][GP];
+    __shared__ float sm_acc[NW][GP][D];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+        if (lane == 0) {
+            sm_m[warp][g] = m[g];
+            sm_l[warp][g] = l[g];
+        }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) sm_acc[warp][g][lane * VEC + e] = acc[g][e];
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < a.G * D; idx += blockDim.x) {
+        const int g = idx / D, e = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w][g]);
+        float L = 0.f, A = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float f = exp2f(sm_m[w][g] - M);
+                L = fmaf(sm_l[w][g], f, L);
+                A = fmaf(sm_acc[w][g][e], f, A);
+            }
+        }
+        const int64_t bh = (int64_t)b * a.Hq + h * a.G + g;
+        if (a.num_splits == 1) {
+            a.out[bh * D + e] = f32_to_bf16_rn(L > 0.f ? A / L : 0.f);
+        } else {
+            a.ws_acc[(bh * a.num_splits + c) * D + e] = A;
+            if (e == 0) {
+                a.ws_ml[(bh * a.num_splits + c) * 2 + 0] = M;
+                a.ws_ml[(bh * a.num_splits + c) * 2 + 1] = L;
+            }
+        }
+    }
+}
+
+// Log-sum-exp merge of the partitions of one (sequence, query head):
+// M = max_s m_s, L = sum_s l_s 2^(m_s - M), out = sum_s acc_s 2^(m_s - M) / L.
+// Partitions are visited in index order (deterministic, no atomics).
+template <int D>
+__global__ void __launch_bounds__(D) merge_kernel(DecodeArgs a) {
+    const int64_t bh = blockIdx.x;
+    const int b = (int)(bh / a.Hq);
+    const int e = threadIdx.x;
+    int len = a.ctx_lens[b];
+    if (len < 0 || (int64_t)len > (int64_t)a.MB * a.bs) len = 0;
+    const int ns = len > 0 ? (len + a.chunk - 1) / a.chunk : 1;
+    const float *ml = a.ws_ml + bh * a.num_splits * 2;
+    const float *acc = a.ws_acc + bh * a.num_splits * D;
+    float M = -INFINITY;
+    for (int s = 0; s < ns; ++s) M = fmaxf(M, ml[2 * s]);
+    float L = 0.f, A = 0.f;
+    if (M != -INFINITY) {
+        for (int s = 0; s < ns; ++s) {
+            const float f = exp2f(ml[2 * s] - M);
+            L = fmaf(ml[2 * s + 1], f, L);
+            A = fmaf(acc[(int64_t)s * D + e], f, A);
+        }
+    }
+    a.out[bh * D + e] = f32_to_bf16_rn(L > 0.f ? A / L : 0.f);
+}
+
+template <int D, bool INT8>
+static void launch_simple_gp(const DecodeArgs &a, dim3 grid, cudaStream_t st) {
+    int gp = 1;
+    while (gp < a.G) gp <<= 1;
+    switch (gp) {
+        case 1: decode_simple_kernel<D, 1, INT8><<<grid, 128, 0, st>>>(a); break;
+        case 2: decode_simple_kernel<D, 2, INT8><<<grid, 128, 0, st>>>(a); break;
+        case 4: decode_simple_kernel<D, 4, INT8><<<grid, 128, 0, st>>>(a); break;
+        case 8: decode_simple_kernel<D, 8, INT8><<<grid, 128, 0, st>>>(a); break;
+        default: decode_simple_kernel<D, 16, INT8><<<grid, 128, 0, st>>>(a); break;
+    }
+}
+
+cudaError_t launch_decode_simple(const DecodeArgs &a, bool int8, cudaStream_t st) {
+    dim3 grid(a.num_splits, a.Hkv, a.B);
+    if (a.d == 128) {
+        if (int8) launch_simple_gp<128, true>(a, grid, st);
+        else launch_simple_gp<128, false>(a, grid, st);
+    } else {
+        if (int8) launch_simple_gp<64, true>(a, grid, st);
+        else launch_simple_gp<64, false>(a, grid, st);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || a.num_splits == 1) return e;
+    return launch_merge(a, st);
+}
+
+cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t st) {
+    const unsigned rows = (unsigned)((int64_t)a.B * a.Hq);
+    if (a.d == 128) merge_kernel<128><<<rows, 128, 0, st>>>(a);
+    else merge_kernel<64><<<rows, 64, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const DecodeArgs &a, bool int8, cudaStream_t st) {
+    return launch_decode_simple(a, int8, st);
+}
+
+}  // namespace pkv

@@ -1,0 +1,71 @@
+// kernels.h -- argument blocks and launchers shared between the C-ABI layer
+// (pagedkv_api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pkv {
+
+struct AppendArgs {
+    const int32_t *block_tables;
+    const int32_t *positions;
+    int64_t *slot_out;
+    int32_t *err;
+    int64_t block_stride;  // elements between physical blocks of the pool
+    int64_t N;             // physical blocks in the pool
+    int B, n_new, Hkv, d, bs, MB;
+};
+
+// Decode problem.  K/V element type is given by the launcher (bf16 or int8).
+struct DecodeArgs {
+    uint16_t *out;                // [B][Hq][d] bf16
+    const uint16_t *q;            // [B][Hq][d] bf16
+    const void *k_cache;          // pool base (bf16 or int8)
+    const void *v_cache;
+    const float *k_scale;         // INT8 only: [N][bs][Hkv]
+    const float *v_scale;
+    const int32_t *block_tables;  // [B][MB]
+    const int32_t *ctx_lens;      // [B]
+    int32_t *err;
+    float *ws_acc;                // [B][Hq][S][d] partial numerators (S > 1)
+    float *ws_ml;                 // [B][Hq][S][2] partial (max, sum), log2 domain
+    int64_t block_stride;
+    int64_t N;
+    float scale_log2;             // scale * log2(e)
+    int B, Hq, Hkv, G, d, bs, MB;
+    int num_splits;               // S: partitions per sequence (1 = write out directly)
+    int chunk;                    // tokens per partition (multiple of 16 when S > 1)
+};
+
+struct ScoreArgs {
+    float *scores;
+    const uint16_t *k_cache;
+    const uint16_t *v_cache;
+    const int32_t *block_tables;
+    const int32_t *ctx_lens;
+    int32_t *err;
+    int64_t block_stride;
+    int64_t N;
+    int B, Hkv, d, bs, MB;
+};
+
+cudaError_t launch_append_bf16(const uint16_t *k_new, const uint16_t *v_new, uint16_t *k_cache,
+                               uint16_t *v_cache, const AppendArgs &a, int num_sms,
+                               cudaStream_t stream);
+cudaError_t launch_append_int8(const uint16_t *k_new, const uint16_t *v_new, int8_t *kq,
+                               int8_t *vq, float *k_scale, float *v_scale, const AppendArgs &a,
+                               int num_sms, cudaStream_t stream);
+
+// Decode dispatch: the staged tensor-core kernel when the shape allows it,
+// else the general-shape kernel; then the partition merge when S > 1.
+cudaError_t launch_decode(const DecodeArgs &a, bool int8, cudaStream_t stream);
+cudaError_t launch_decode_simple(const DecodeArgs &a, bool int8, cudaStream_t stream);
+cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t stream);
+
+cudaError_t launch_score(const ScoreArgs &a, cudaStream_t stream);
+cudaError_t launch_select_evict(int32_t *evict, float *means, const float *scores,
+                                const int32_t *ctx_lens, int B, int MB, int Hkv, int bs,
+                                cudaStream_t stream);
+
+}  // namespace pkv

@@ -1,0 +1,286 @@
+// pagedkv_api.cu -- the extern "C" entry points declared in include/pagedkv.h:
+// argument validation, launch-shape decisions and kernel launches.  Nothing
+// here allocates device memory or keeps state between calls beyond a per-device
+// cache of the SM count.
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "kernels.h"
+#include "pagedkv.h"
+
+namespace {
+
+struct DevCache {
+    std::atomic<int> sms{0};
+    std::atomic<int> major{0};
+};
+DevCache g_dev[64];
+
+// Current device's SM count, or a negative PA_ERR_* when it is not an sm_100 GPU.
+int device_sms() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return PA_ERR_DEVICE;
+    int sms = g_dev[dev].sms.load(std::memory_order_relaxed);
+    if (sms == 0) {
+        int major = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return PA_ERR_CUDA;
+        g_dev[dev].major.store(major);
+        g_dev[dev].sms.store(sms);
+    }
+    if (g_dev[dev].major.load() != 10) return PA_ERR_DEVICE;
+    return sms;
+}
+
+inline bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int Hkv, int d, int bs, int MB, int64_t N, int64_t block_stride) {
+    if (B < 0 || Hkv < 1 || bs < 1 || MB < 1 || N < 1) return PA_ERR_SHAPE;
+    if (B > 65535 || Hkv > 65535) return PA_ERR_SHAPE;  // grid y/z limits
+    if (d != 64 && d != 128) return PA_ERR_SHAPE;
+    if ((int64_t)MB * bs > INT32_MAX) return PA_ERR_SHAPE;
+    if (block_stride < (int64_t)bs * Hkv * d) return PA_ERR_SHAPE;
+    if (N > INT32_MAX) return PA_ERR_SHAPE;
+    return PA_OK;
+}
+
+// Partition of the context for the decode kernels.  Partitions are `chunk`
+// tokens (a multiple of 16) of one sequence; S = ceil(MB*bs / chunk) bounds the
+// partitions of any sequence.  Automatic choice: enough (partition, kv head,
+// sequence) units for ~4 CTAs per SM, never partitions below 256 tokens.
+void choose_split(int B, int Hkv, int bs, int MB, int num_splits, int sms, int *S, int *chunk) {
+    const int64_t max_ctx = (int64_t)MB * bs;
+    int64_t s = num_splits;
+    if (s <= 0) {
+        const int64_t units = (int64_t)(B > 0 ? B : 1) * Hkv;
+        const int64_t target = 4LL * sms;
+        s = units >= target ? 1 : (target + units - 1) / units;
+        const int64_t cap = (max_ctx + 255) / 256;
+        if (s > cap) s = cap;
+    }
+    if (s < 1) s = 1;
+    if (s > max_ctx) s = max_ctx;
+    int64_t ch = (max_ctx + s - 1) / s;
+    ch = (ch + 15) / 16 * 16;
+    const int64_t se = (max_ctx + ch - 1) / ch;
+    *S = (int)se;
+    *chunk = (int)(se == 1 ? max_ctx : ch);
+}
+
+struct WsLayout {
+    size_t acc_off, ml_off, total;
+};
+
+WsLayout ws_layout(int B, int Hq, int d, int S) {
+    WsLayout w{0, 0, 0};
+    if (S <= 1) return w;
+    const size_t rows = (size_t)B * Hq * S;
+    w.acc_off = 0;
+    w.ml_off = (rows * d * sizeof(float) + 255) / 256 * 256;
+    w.total = w.ml_off + (rows * 2 * sizeof(float) + 255) / 256 * 256;
+    return w;
+}
+
+int finish(cudaError_t e) { return e == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
+
+// Shared body of pa_decode / pa_decode_int8.
+int decode_entry(uint16_t *out, const uint16_t *q, const void *kc, const void *vc, const float *ks,
+                 const float *vs, bool int8, int64_t block_stride, const int32_t *bt, int MB,
+                 const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs, int64_t N,
+                 float scale, int num_splits, void *ws, size_t ws_bytes, int32_t *err,
+                 void *stream) {
+    if (B == 0) return PA_OK;  // empty batch: nothing to read or write
+    if (!out || !q || !kc || !vc || !bt || !ctx_lens || !err) return PA_ERR_NULL;
+    if (int8 && (!ks || !vs)) return PA_ERR_NULL;
+    int rc = check_common(B, Hkv, d, bs, MB, N, block_stride);
+    if (rc) return rc;
+    if (Hq < Hkv || Hq % Hkv != 0 || Hq / Hkv > 16) return PA_ERR_SHAPE;
+    if (!(scale == scale)) return PA_ERR_SHAPE;
+    const int elt = int8 ? 1 : 2;
+    if (!al16(out) || !al16(q) || !al16(kc) || !al16(vc) || (block_stride * elt) % 16 != 0)
+        return PA_ERR_ALIGN;
+    if (B == 0) return PA_OK;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    int S = 1, chunk = 0;
+    choose_split(B, Hkv, bs, MB, num_splits, sms, &S, &chunk);
+    const WsLayout wl = ws_layout(B, Hq, d, S);
+    if (wl.total > 0) {
+        if (!ws) return PA_ERR_WORKSPACE;
+        if (ws_bytes < wl.total) return PA_ERR_WORKSPACE;
+        if (!al16(ws)) return PA_ERR_ALIGN;
+    }
+    pkv::DecodeArgs a;
+    memset(&a, 0, sizeof a);
+    a.out = out;
+    a.q = q;
+    a.k_cache = kc;
+    a.v_cache = vc;
+    a.k_scale = ks;
+    a.v_scale = vs;
+    a.block_tables = bt;
+    a.ctx_lens = ctx_lens;
+    a.err = err;
+    a.ws_acc = wl.total ? reinterpret_cast<float *>(static_cast<char *>(ws) + wl.acc_off) : nullptr;
+    a.ws_ml = wl.total ? reinterpret_cast<float *>(static_cast<char *>(ws) + wl.ml_off) : nullptr;
+    a.block_stride = block_stride;
+    a.N = N;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.G = Hq / Hkv;
+    a.d = d;
+    a.bs = bs;
+    a.MB = MB;
+    a.num_splits = S;
+    a.chunk = chunk;
+    return finish(pkv::launch_decode(a, int8, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *pa_status_string(int code) {
+    switch (code) {
+        case PA_OK: return "ok";
+        case PA_ERR_NULL: return "a required pointer is NULL";
+        case PA_ERR_SHAPE: return "unsupported or inconsistent sizes";
+        case PA_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
+        case PA_ERR_WORKSPACE: return "workspace missing or too small";
+        case PA_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
+        case PA_ERR_DEVICE: return "current device is not an sm_100 GPU";
+        default: return "unknown status";
+    }
+}
+
+const char *pa_version(void) { return "pagedkv 0.1 sm_100a"; }
+
+int pa_append_kv(const uint16_t *k_new, const uint16_t *v_new, uint16_t *k_cache,
+                 uint16_t *v_cache, int64_t block_stride, const int32_t *block_tables,
+                 int max_blocks_per_seq, const int32_t *positions, int B, int n_new, int Hkv,
+                 int d, int bs, int64_t num_blocks, int64_t *slot_out, int32_t *err_flag,
+                 void *stream) {
+    if (B == 0 || n_new == 0) return PA_OK;
+    if (!k_new || !v_new || !k_cache || !v_cache || !block_tables || !positions || !err_flag)
+        return PA_ERR_NULL;
+    int rc = check_common(B, Hkv, d, bs, max_blocks_per_seq, num_blocks, block_stride);
+    if (rc) return rc;
+    if (n_new < 0) return PA_ERR_SHAPE;
+    if (!al16(k_new) || !al16(v_new) || !al16(k_cache) || !al16(v_cache) ||
+        (block_stride * 2) % 16 != 0)
+        return PA_ERR_ALIGN;
+    if (B == 0 || n_new == 0) return PA_OK;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    pkv::AppendArgs a{block_tables, positions, slot_out, err_flag, block_stride, num_blocks,
+                      B, n_new, Hkv, d, bs, max_blocks_per_seq};
+    return finish(pkv::launch_append_bf16(k_new, v_new, k_cache, v_cache, a, sms,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int pa_append_kv_int8(const uint16_t *k_new, const uint16_t *v_new, int8_t *kq_cache,
+                      int8_t *vq_cache, float *k_scale, float *v_scale, int64_t block_stride,
+                      const int32_t *block_tables, int max_blocks_per_seq,
+                      const int32_t *positions, int B, int n_new, int Hkv, int d, int bs,
+                      int64_t num_blocks, int64_t *slot_out, int32_t *err_flag, void *stream) {
+    if (B == 0 || n_new == 0) return PA_OK;
+    if (!k_new || !v_new || !kq_cache || !vq_cache || !k_scale || !v_scale || !block_tables ||
+        !positions || !err_flag)
+        return PA_ERR_NULL;
+    int rc = check_common(B, Hkv, d, bs, max_blocks_per_seq, num_blocks, block_stride);
+    if (rc) return rc;
+    if (n_new < 0) return PA_ERR_SHAPE;
+    if (!al16(k_new) || !al16(v_new) || !al16(kq_cache) || !al16(vq_cache) || !al16(k_scale) ||
+        !al16(v_scale) || block_stride % 16 != 0)
+        return PA_ERR_ALIGN;
+    if (B == 0 || n_new == 0) return PA_OK;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    pkv::AppendArgs a{block_tables, positions, slot_out, err_flag, block_stride, num_blocks,
+                      B, n_new, Hkv, d, bs, max_blocks_per_seq};
+    return finish(pkv::launch_append_int8(k_new, v_new, kq_cache, vq_cache, k_scale, v_scale, a,
+                                          sms, static_cast<cudaStream_t>(stream)));
+}
+
+size_t pa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq,
+                                 int num_splits) {
+    if (B <= 0 || Hq < 1 || Hkv < 1 || bs < 1 || max_blocks_per_seq < 1) return 0;
+    const int sms = device_sms();
+    if (sms < 0) return 0;
+    int S = 1, chunk = 0;
+    choose_split(B, Hkv, bs, max_blocks_per_seq, num_splits, sms, &S, &chunk);
+    return ws_layout(B, Hq, d, S).total;
+}
+
+int pa_decode_plan(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq, int num_splits,
+                   int *num_splits_out, int *chunk_tokens_out) {
+    if (!num_splits_out || !chunk_tokens_out) return PA_ERR_NULL;
+    if (B < 0 || Hq < 1 || Hkv < 1 || bs < 1 || max_blocks_per_seq < 1) return PA_ERR_SHAPE;
+    if (d != 64 && d != 128) return PA_ERR_SHAPE;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    choose_split(B, Hkv, bs, max_blocks_per_seq, num_splits, sms, num_splits_out,
+                 chunk_tokens_out);
+    return PA_OK;
+}
+
+int pa_decode(uint16_t *out, const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+              int64_t block_stride, const int32_t *block_tables, int max_blocks_per_seq,
+              const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs, int64_t num_blocks,
+              float scale, int num_splits, void *workspace, size_t workspace_bytes,
+              int32_t *err_flag, void *stream) {
+    return decode_entry(out, q, k_cache, v_cache, nullptr, nullptr, false, block_stride,
+                        block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
+                        scale, num_splits, workspace, workspace_bytes, err_flag, stream);
+}
+
+int pa_decode_int8(uint16_t *out, const uint16_t *q, const int8_t *kq_cache,
+                   const int8_t *vq_cache, const float *k_scale, const float *v_scale,
+                   int64_t block_stride, const int32_t *block_tables, int max_blocks_per_seq,
+                   const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
+                   int64_t num_blocks, float scale, int num_splits, void *workspace,
+                   size_t workspace_bytes, int32_t *err_flag, void *stream) {
+    return decode_entry(out, q, kq_cache, vq_cache, k_scale, v_scale, true, block_stride,
+                        block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
+                        scale, num_splits, workspace, workspace_bytes, err_flag, stream);
+}
+
+int pe_score_tokens(float *scores, const uint16_t *k_cache, const uint16_t *v_cache,
+                    int64_t block_stride, const int32_t *block_tables, int max_blocks_per_seq,
+                    const int32_t *ctx_lens, int B, int Hkv, int d, int bs, int64_t num_blocks,
+                    int32_t *err_flag, void *stream) {
+    if (B == 0) return PA_OK;
+    if (!scores || !k_cache || !v_cache || !block_tables || !ctx_lens || !err_flag)
+        return PA_ERR_NULL;
+    int rc = check_common(B, Hkv, d, bs, max_blocks_per_seq, num_blocks, block_stride);
+    if (rc) return rc;
+    if (!al16(k_cache) || !al16(v_cache) || (block_stride * 2) % 16 != 0) return PA_ERR_ALIGN;
+    if (B == 0) return PA_OK;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    pkv::ScoreArgs a{scores, k_cache, v_cache, block_tables, ctx_lens, err_flag, block_stride,
+                     num_blocks, B, Hkv, d, bs, max_blocks_per_seq};
+    return finish(pkv::launch_score(a, static_cast<cudaStream_t>(stream)));
+}
+
+int pe_select_evict_block(int32_t *evict, float *block_means, const float *scores,
+                          const int32_t *ctx_lens, int B, int max_blocks_per_seq, int Hkv, int bs,
+                          void *stream) {
+    if (B == 0) return PA_OK;
+    if (!evict || !scores || !ctx_lens) return PA_ERR_NULL;
+    if (B < 0 || max_blocks_per_seq < 1 || Hkv < 1 || bs < 1) return PA_ERR_SHAPE;
+    if (B == 0) return PA_OK;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    return finish(pkv::launch_select_evict(evict, block_means, scores, ctx_lens, B,
+                                           max_blocks_per_seq, Hkv, bs,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

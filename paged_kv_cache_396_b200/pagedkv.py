@@ -1,0 +1,299 @@
+"""Thin Python binding of libpagedkv.so (the C ABI in include/pagedkv.h).
+
+Argument marshalling only: every function takes torch CUDA tensors, checks
+dtypes and layouts, reads sizes from shapes and strides, and calls the C entry
+point of the same name on the current (or given) CUDA stream.  All the work runs
+in the library's kernels; there is no CPU fallback, and a missing library is an
+error.
+
+Tensor conventions (the C header has the full statement of each operation):
+  pools      [N, bs, Hkv, d] (bf16 or int8); the block stride is stride(0), so a
+             view into a larger tensor such as the nano-vLLM [2, L, N, bs, Hkv, d]
+             works unchanged.  Inner three dims must be contiguous.
+  scales     [N, bs, Hkv] float32, contiguous (INT8 pools).
+  block_tables [B, MB] int32, ctx_lens/positions [B] int32, err_flag [>=1] int32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
+
+PA_OK = 0
+PA_DEV_BAD_BLOCK = 1
+PA_DEV_BAD_LEN = 2
+PA_DEV_TIMEOUT = 4
+
+EXPORTED = (
+    "pa_status_string", "pa_version", "pa_append_kv", "pa_decode_workspace_bytes", "pa_decode_plan",
+    "pa_decode",
+    "pe_score_tokens", "pe_select_evict_block", "pa_append_kv_int8", "pa_decode_int8",
+)
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, fn: str, code: int, text: str):
+        super().__init__(f"{fn} failed with status {code}: {text}")
+        self.code = code
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the shared library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libpagedkv.so not found at {path}; build it with "
+                          "`python -m paged_kv_cache_396_b200.build_lib`")
+    lib = ctypes.CDLL(path)
+    p, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                            ctypes.c_size_t)
+    lib.pa_status_string.restype = ctypes.c_char_p
+    lib.pa_status_string.argtypes = [i32]
+    lib.pa_version.restype = ctypes.c_char_p
+    lib.pa_version.argtypes = []
+    lib.pa_append_kv.restype = i32
+    lib.pa_append_kv.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, i64, p, p, p]
+    lib.pa_append_kv_int8.restype = i32
+    lib.pa_append_kv_int8.argtypes = [p, p, p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32,
+                                      i64, p, p, p]
+    lib.pa_decode_workspace_bytes.restype = sz
+    lib.pa_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32]
+    lib.pa_decode_plan.restype = i32
+    lib.pa_decode_plan.argtypes = [i32, i32, i32, i32, i32, i32, i32, p, p]
+    lib.pa_decode.restype = i32
+    lib.pa_decode.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, i64, f32, i32,
+                              p, sz, p, p]
+    lib.pa_decode_int8.restype = i32
+    lib.pa_decode_int8.argtypes = [p, p, p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, i64,
+                                   f32, i32, p, sz, p, p]
+    lib.pe_score_tokens.restype = i32
+    lib.pe_score_tokens.argtypes = [p, p, p, i64, p, i32, p, i32, i32, i32, i32, i64, p, p]
+    lib.pe_select_evict_block.restype = i32
+    lib.pe_select_evict_block.argtypes = [p, p, p, p, i32, i32, i32, i32, p]
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, code: int):
+    if code != PA_OK:
+        raise PagedKVError(fn, code, load().pa_status_string(code).decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _want(t: torch.Tensor, dtype, name: str):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise TypeError(f"{name}: expected a CUDA tensor")
+
+
+def _pool_geometry(pool: torch.Tensor, name: str):
+    if pool.dim() != 4:
+        raise ValueError(f"{name}: expected [N, bs, Hkv, d], got shape {tuple(pool.shape)}")
+    N, bs, Hkv, d = pool.shape
+    if pool.stride(3) != 1 or pool.stride(2) != d or pool.stride(1) != Hkv * d:
+        raise ValueError(f"{name}: the [bs, Hkv, d] part must be contiguous")
+    return N, bs, Hkv, d, pool.stride(0)
+
+
+def _same_pool(a: torch.Tensor, b: torch.Tensor):
+    if a.shape != b.shape or a.stride() != b.stride():
+        raise ValueError("K and V pools must have the same shape and strides")
+
+
+# ----------------------------------------------------------------------------- append
+def pa_append_kv(k_new, v_new, k_cache, v_cache, block_tables, positions, err_flag,
+                 slot_out=None, stream=None):
+    """Write new tokens into the paged pools.  k_new/v_new: [B, n_new, Hkv, d] or
+    [B, Hkv, d] bf16 (contiguous); positions [B]: position of each sequence's
+    first new token.  slot_out: optional [B, n_new] int64."""
+    for t, n in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _want(t, torch.bfloat16, n)
+    _want(block_tables, torch.int32, "block_tables")
+    _want(positions, torch.int32, "positions")
+    _want(err_flag, torch.int32, "err_flag")
+    N, bs, Hkv, d, stride = _pool_geometry(k_cache, "k_cache")
+    _same_pool(k_cache, v_cache)
+    if k_new.dim() == 3:
+        k_new, v_new = k_new.unsqueeze(1), v_new.unsqueeze(1)
+    if not (k_new.is_contiguous() and v_new.is_contiguous()) or k_new.shape != v_new.shape:
+        raise ValueError("k_new/v_new must be contiguous and of equal shape")
+    B, n_new = k_new.shape[0], k_new.shape[1]
+    if k_new.shape[2:] != (Hkv, d):
+        raise ValueError("k_new inner dims must match the pool's [Hkv, d]")
+    if slot_out is not None:
+        _want(slot_out, torch.int64, "slot_out")
+    bt = block_tables.contiguous()
+    rc = load().pa_append_kv(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), stride,
+                             _ptr(bt), bt.shape[1], _ptr(positions.contiguous()), B, n_new, Hkv, d,
+                             bs, N, _ptr(slot_out), _ptr(err_flag), _stream(stream))
+    _check("pa_append_kv", rc)
+
+
+def pa_append_kv_int8(k_new, v_new, kq_cache, vq_cache, k_scale, v_scale, block_tables,
+                      positions, err_flag, slot_out=None, stream=None):
+    """Quantise (symmetric INT8, one fp32 scale per (token, kv head)) and write
+    new tokens.  Pools [N, bs, Hkv, d] int8, scales [N, bs, Hkv] float32."""
+    _want(k_new, torch.bfloat16, "k_new")
+    _want(v_new, torch.bfloat16, "v_new")
+    _want(kq_cache, torch.int8, "kq_cache")
+    _want(vq_cache, torch.int8, "vq_cache")
+    _want(k_scale, torch.float32, "k_scale")
+    _want(v_scale, torch.float32, "v_scale")
+    _want(block_tables, torch.int32, "block_tables")
+    _want(positions, torch.int32, "positions")
+    _want(err_flag, torch.int32, "err_flag")
+    N, bs, Hkv, d, stride = _pool_geometry(kq_cache, "kq_cache")
+    _same_pool(kq_cache, vq_cache)
+    for s in (k_scale, v_scale):
+        if tuple(s.shape) != (N, bs, Hkv) or not s.is_contiguous():
+            raise ValueError("scale pools must be contiguous [N, bs, Hkv]")
+    if k_new.dim() == 3:
+        k_new, v_new = k_new.unsqueeze(1), v_new.unsqueeze(1)
+    if not (k_new.is_contiguous() and v_new.is_contiguous()) or k_new.shape != v_new.shape:
+        raise ValueError("k_new/v_new must be contiguous and of equal shape")
+    B, n_new = k_new.shape[0], k_new.shape[1]
+    if slot_out is not None:
+        _want(slot_out, torch.int64, "slot_out")
+    bt = block_tables.contiguous()
+    rc = load().pa_append_kv_int8(_ptr(k_new), _ptr(v_new), _ptr(kq_cache), _ptr(vq_cache),
+                                  _ptr(k_scale), _ptr(v_scale), stride, _ptr(bt), bt.shape[1],
+                                  _ptr(positions.contiguous()), B, n_new, Hkv, d, bs, N,
+                                  _ptr(slot_out), _ptr(err_flag), _stream(stream))
+    _check("pa_append_kv_int8", rc)
+
+
+# ----------------------------------------------------------------------------- decode
+def pa_decode_workspace_bytes(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits=0) -> int:
+    return int(load().pa_decode_workspace_bytes(B, Hq, Hkv, d, bs, max_blocks_per_seq,
+                                                num_splits))
+
+
+def pa_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits=0):
+    """(partitions per sequence at most, tokens per partition) pa_decode will use."""
+    s, c = ctypes.c_int(0), ctypes.c_int(0)
+    _check("pa_decode_plan", load().pa_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq,
+                                                   num_splits, ctypes.byref(s), ctypes.byref(c)))
+    return s.value, c.value
+
+
+def alloc_workspace(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits=0, device=None):
+    """Convenience: a device byte tensor of the size pa_decode needs (or None)."""
+    n = pa_decode_workspace_bytes(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits)
+    return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
+
+
+def _decode_checks(out, q, block_tables, ctx_lens, err_flag):
+    _want(out, torch.bfloat16, "out")
+    _want(q, torch.bfloat16, "q")
+    _want(block_tables, torch.int32, "block_tables")
+    _want(ctx_lens, torch.int32, "ctx_lens")
+    _want(err_flag, torch.int32, "err_flag")
+    if not (out.is_contiguous() and q.is_contiguous()) or out.shape != q.shape or q.dim() != 3:
+        raise ValueError("q and out must be contiguous [B, Hq, d] of equal shape")
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
+              workspace=None, num_splits=0, stream=None):
+    """Paged decode attention (bf16 pools): out[b, i] = softmax(scale q.K) V over
+    the ctx_lens[b] tokens of sequence b, kv head i // (Hq/Hkv)."""
+    _decode_checks(out, q, block_tables, ctx_lens, err_flag)
+    _want(k_cache, torch.bfloat16, "k_cache")
+    _want(v_cache, torch.bfloat16, "v_cache")
+    N, bs, Hkv, d, stride = _pool_geometry(k_cache, "k_cache")
+    _same_pool(k_cache, v_cache)
+    B, Hq, dq = q.shape
+    if dq != d:
+        raise ValueError("q head_dim differs from the pool's")
+    bt = block_tables.contiguous()
+    ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel() *
+                                                        workspace.element_size())
+    rc = load().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), stride, _ptr(bt),
+                          bt.shape[1], _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d, bs, N,
+                          float(scale), int(num_splits), ws_ptr, ws_n, _ptr(err_flag),
+                          _stream(stream))
+    _check("pa_decode", rc)
+
+
+def pa_decode_int8(out, q, kq_cache, vq_cache, k_scale, v_scale, block_tables, ctx_lens, scale,
+                   err_flag, workspace=None, num_splits=0, stream=None):
+    """Paged decode attention over INT8 pools dequantised in registers."""
+    _decode_checks(out, q, block_tables, ctx_lens, err_flag)
+    _want(kq_cache, torch.int8, "kq_cache")
+    _want(vq_cache, torch.int8, "vq_cache")
+    _want(k_scale, torch.float32, "k_scale")
+    _want(v_scale, torch.float32, "v_scale")
+    N, bs, Hkv, d, stride = _pool_geometry(kq_cache, "kq_cache")
+    _same_pool(kq_cache, vq_cache)
+    for s in (k_scale, v_scale):
+        if tuple(s.shape) != (N, bs, Hkv) or not s.is_contiguous():
+            raise ValueError("scale pools must be contiguous [N, bs, Hkv]")
+    B, Hq, dq = q.shape
+    if dq != d:
+        raise ValueError("q head_dim differs from the pool's")
+    bt = block_tables.contiguous()
+    ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel() *
+                                                        workspace.element_size())
+    rc = load().pa_decode_int8(_ptr(out), _ptr(q), _ptr(kq_cache), _ptr(vq_cache), _ptr(k_scale),
+                               _ptr(v_scale), stride, _ptr(bt), bt.shape[1],
+                               _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d, bs, N, float(scale),
+                               int(num_splits), ws_ptr, ws_n, _ptr(err_flag), _stream(stream))
+    _check("pa_decode_int8", rc)
+
+
+# ----------------------------------------------------------------------------- eviction
+def pe_score_tokens(scores, k_cache, v_cache, block_tables, ctx_lens, err_flag, stream=None):
+    """scores [B, MB*bs, Hkv] float32 <- ||V|| / ||K|| for t < ctx_lens[b]."""
+    _want(scores, torch.float32, "scores")
+    _want(k_cache, torch.bfloat16, "k_cache")
+    _want(v_cache, torch.bfloat16, "v_cache")
+    _want(block_tables, torch.int32, "block_tables")
+    _want(ctx_lens, torch.int32, "ctx_lens")
+    _want(err_flag, torch.int32, "err_flag")
+    N, bs, Hkv, d, stride = _pool_geometry(k_cache, "k_cache")
+    _same_pool(k_cache, v_cache)
+    bt = block_tables.contiguous()
+    B, MB = bt.shape
+    if tuple(scores.shape) != (B, MB * bs, Hkv) or not scores.is_contiguous():
+        raise ValueError("scores must be contiguous [B, MB*bs, Hkv]")
+    rc = load().pe_score_tokens(_ptr(scores), _ptr(k_cache), _ptr(v_cache), stride, _ptr(bt), MB,
+                                _ptr(ctx_lens.contiguous()), B, Hkv, d, bs, N, _ptr(err_flag),
+                                _stream(stream))
+    _check("pe_score_tokens", rc)
+
+
+def pe_select_evict_block(evict, scores, ctx_lens, bs, block_means=None, stream=None):
+    """evict [B] int32 <- lowest-mean full block per sequence (-1 if none)."""
+    _want(evict, torch.int32, "evict")
+    _want(scores, torch.float32, "scores")
+    _want(ctx_lens, torch.int32, "ctx_lens")
+    B, T, Hkv = scores.shape
+    if T % bs:
+        raise ValueError("scores' token dim must be MB*bs")
+    MB = T // bs
+    if block_means is not None:
+        _want(block_means, torch.float32, "block_means")
+        if tuple(block_means.shape) != (B, MB) or not block_means.is_contiguous():
+            raise ValueError("block_means must be contiguous [B, MB]")
+    rc = load().pe_select_evict_block(_ptr(evict), _ptr(block_means), _ptr(scores.contiguous()),
+                                      _ptr(ctx_lens.contiguous()), B, MB, Hkv, bs,
+                                      _stream(stream))
+    _check("pe_select_evict_block", rc)

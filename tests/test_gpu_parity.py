@@ -1,0 +1,226 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small and medium cases run the oracle on every output; they span several
+16-token tiles, several partitions and ragged last blocks.  Append slots and
+pool contents, INT8 codes and scales, and the evicted block are compared
+exactly; attention within |err| <= 2e-3 + 1e-2 |ref|; scores within 1e-5
+relative."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import (Device, assert_attention_close, assert_evict_consistent,
+                     assert_scores_close, oracle_step)
+from paged_kv_cache_396_b200 import pagedkv as pk
+from paged_kv_cache_396_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+C = W.CONFIGS
+MEDIUM = {
+    # Llama-3.2-1B shape, 2 layers, 6 sequences around 1K tokens (ragged tails)
+    "c2m": W.scaled(C["c2"], key="c2m", layers=2, batch=6, old_lens=(1024, 1000, 17, 300, 1,
+                                                                      1039)),
+    # Llama-3-8B shape with outlier channels, 7 sequences
+    "c3m": W.scaled(C["c3"], key="c3m", layers=1, batch=7, old_len_range=(1, 900)),
+    # nano-vLLM layout, block 256, no append
+    "c4m": W.scaled(C["c4"], key="c4m", batch=3, old_lens=(4096, 3000, 257)),
+    # INT8, G = 8
+    "c5m": W.scaled(C["c5"], key="c5m", batch=5, old_lens=(300, 1, 16, 255, 512)),
+}
+
+
+def _parity(wl, layers, num_splits=0, score=None):
+    cfg = wl.cfg
+    score = cfg.score if score is None else score
+    seqs = range(cfg.batch)
+    refs = [oracle_step(wl, l, seqs, score=score) for l in layers]
+    dev = Device(wl, num_splits)
+    if cfg.int8:
+        for l in layers:
+            dev.fill_int8_history(l)
+    for l, ref in zip(layers, refs):
+        res = dev.step(l, score=score)
+        torch.cuda.synchronize()
+        assert dev.err.item() == 0, f"device error flag {dev.err.item()}"
+        assert_attention_close(dev.out[l], ref["out"], f"{cfg.key} layer {l}")
+        if "slots" in ref:
+            # slots are global ids in the full pool; map the oracle's compact ids back
+            s = ref["compact"]
+            bt_full, bt_c = wl.block_tables, s["block_tables"]
+            bs = cfg.block_size
+            expect = np.empty_like(ref["slots"])
+            for b in range(cfg.batch):
+                blk, off = divmod(int(ref["slots"][b, 0]), bs)
+                j = int(np.nonzero(bt_c[b] == blk)[0][0])
+                expect[b, 0] = int(bt_full[b, j]) * bs + off
+            assert np.array_equal(dev.slots.cpu().numpy(), expect)
+        if score:
+            lens = ref["ctx_lens"]
+            got = res["scores"].cpu().numpy()
+            for b in range(cfg.batch):
+                assert_scores_close(got[b, :lens[b]], ref["scores"][b, :lens[b]], f"seq {b}")
+            assert_evict_consistent(res["evict"].cpu().numpy(), ref["evict"], ref["means"],
+                                    ref["gap"], cfg.key)
+    return dev, refs
+
+
+def test_tiny_workload_full_step():
+    wl = W.generate(C["c1"], "cpu")
+    dev, refs = _parity(wl, [0], score=True)
+    # pool after the append equals the oracle's, bit for bit (tiny pool: compare all of it)
+    ref = refs[0]
+    s = ref["compact"]
+    ids = wl.block_tables[wl.block_tables >= 0]
+    got_k = dev.k_pool[0][torch.as_tensor(ids, device="cuda")].view(torch.int16).cpu().numpy()
+    assert np.array_equal(got_k.view(np.uint16).ravel(), ref["kc"])
+    # the two full blocks per sequence and the decision (38 -> 2 full, 101 -> 6 full)
+    assert (ref["means"][0, 2:] != ref["means"][0, 2:]).all()
+
+
+@pytest.mark.parametrize("key", list(MEDIUM))
+def test_medium_workloads(key):
+    wl = W.generate(MEDIUM[key], "cpu")
+    _parity(wl, list(range(wl.q.shape[0])), score=(key == "c2m"))
+
+
+@pytest.mark.parametrize("num_splits", [1, 2, 3, 8, 0])
+def test_split_count_invariance(num_splits):
+    cfg = W.scaled(C["c3"], key="split", layers=1, batch=3, old_lens=(2000, 700, 45))
+    wl = W.generate(cfg, "cpu")
+    _parity(wl, [0], num_splits=num_splits)
+
+
+def test_physical_block_permutation_gives_identical_output():
+    cfg = W.scaled(C["c2"], key="perm", layers=1, batch=4, old_lens=(100, 77, 300, 5))
+    wl = W.generate(cfg, "cpu")
+    dev = Device(wl)
+    dev.step(0)
+    base = dev.out[0].clone()
+    N = wl.num_blocks
+    perm = torch.randperm(N, generator=torch.Generator().manual_seed(1))
+    inv = torch.argsort(perm)
+    bt = torch.as_tensor(wl.block_tables)
+    dev.bt = torch.where(bt >= 0, perm[bt.clamp(min=0)], bt).to(torch.int32).cuda()
+    dev.k_pool[0] = dev.k_pool[0][inv.cuda()]
+    dev.v_pool[0] = dev.v_pool[0][inv.cuda()]
+    # the append already ran: decode only
+    pk.pa_decode(dev.out[0], dev.q[0], dev.k_pool[0], dev.v_pool[0], dev.bt, dev.ctx, wl.scale,
+                 dev.err, dev.ws)
+    torch.cuda.synchronize()
+    assert dev.err.item() == 0
+    assert torch.equal(dev.out[0], base)
+
+
+def test_unused_blocks_and_slots_are_never_read():
+    cfg = W.scaled(C["c3"], key="nan", layers=1, batch=3, old_lens=(33, 1, 500), spare=0.5)
+    wl = W.generate(cfg, "cpu")
+    ref = oracle_step(wl, 0, range(3))
+    used = set(wl.block_tables[wl.block_tables >= 0].tolist())
+    unused = [p for p in range(wl.num_blocks) if p not in used]
+    wl.k_pool[0, unused] = float("nan")
+    wl.v_pool[0, unused] = float("nan")
+    for b in range(3):   # slots past the new token in each last block
+        n = int(wl.ctx_lens[b])
+        last = wl.block_tables[b, (n - 1) // 16]
+        if n % 16:
+            wl.k_pool[0, last, n % 16:] = float("nan")
+            wl.v_pool[0, last, n % 16:] = float("nan")
+    dev = Device(wl)
+    dev.step(0)
+    torch.cuda.synchronize()
+    assert dev.err.item() == 0
+    assert_attention_close(dev.out[0], ref["out"], "nan-poisoned unused memory")
+
+
+def test_deterministic_bitwise():
+    cfg = W.scaled(C["c3"], key="det", layers=1, batch=5, old_len_range=(100, 3000))
+    wl = W.generate(cfg, "cpu")
+    dev = Device(wl)
+    dev.step(0)
+    a = dev.out[0].clone()
+    pk.pa_decode(dev.out[0], dev.q[0], dev.k_pool[0], dev.v_pool[0], dev.bt, dev.ctx, wl.scale,
+                 dev.err, dev.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a, dev.out[0])
+
+
+def test_int8_codes_and_scales_bit_exact():
+    wl = W.generate(MEDIUM["c5m"], "cpu")
+    ref = oracle_step(wl, 0, range(wl.cfg.batch))
+    dev = Device(wl)
+    dev.fill_int8_history(0)
+    dev.step(0)
+    torch.cuda.synchronize()
+    ids = torch.as_tensor(wl.block_tables[wl.block_tables >= 0], device="cuda")
+    assert np.array_equal(dev.kq[0][ids].cpu().numpy().ravel(), ref["kq"])
+    assert np.array_equal(dev.vq[0][ids].cpu().numpy().ravel(), ref["vq"])
+    assert np.array_equal(dev.ks[0][ids].cpu().numpy().ravel(), ref["ks"])
+    assert np.array_equal(dev.vs[0][ids].cpu().numpy().ravel(), ref["vs"])
+
+
+def test_empty_batch_and_zero_length_context():
+    cfg = W.scaled(C["c2"], key="zero", layers=1, batch=3, old_lens=(40, 0, 16))
+    wl = W.generate(cfg, "cpu")
+    dev = Device(wl)
+    # sequence 1 attends to nothing: give it length 0 explicitly (no append for it)
+    dev.ctx[1] = 0
+    pk.pa_decode(dev.out[0], dev.q[0], dev.k_pool[0], dev.v_pool[0], dev.bt, dev.ctx, wl.scale,
+                 dev.err, dev.ws)
+    torch.cuda.synchronize()
+    assert dev.err.item() == 0
+    assert (dev.out[0, 1] == 0).all()
+    # B = 0 is a no-op that succeeds
+    pk.pa_decode(dev.out[0, :0], dev.q[0, :0], dev.k_pool[0], dev.v_pool[0], dev.bt[:0],
+                 dev.ctx[:0], wl.scale, dev.err, dev.ws)
+
+
+def test_device_flags_on_bad_table_and_length():
+    cfg = W.scaled(C["c2"], key="bad", layers=1, batch=2, old_lens=(100, 50))
+    wl = W.generate(cfg, "cpu")
+    dev = Device(wl)
+    bt = dev.bt.clone()
+    bt[0, 2] = wl.num_blocks + 5        # a needed entry out of range
+    pk.pa_decode(dev.out[0], dev.q[0], dev.k_pool[0], dev.v_pool[0], bt, dev.ctx, wl.scale,
+                 dev.err, dev.ws)
+    torch.cuda.synchronize()
+    assert dev.err.item() & pk.PA_DEV_BAD_BLOCK
+    dev.err.zero_()
+    ctx = dev.ctx.clone()
+    ctx[1] = wl.max_blocks * 16 + 1     # longer than the table can hold
+    pk.pa_decode(dev.out[0], dev.q[0], dev.k_pool[0], dev.v_pool[0], dev.bt, ctx, wl.scale,
+                 dev.err, dev.ws)
+    torch.cuda.synchronize()
+    assert dev.err.item() & pk.PA_DEV_BAD_LEN
+    assert (dev.out[0, 1] == 0).all()
+    dev.err.zero_()
+    pos = dev.pos.clone()
+    pos[0] = wl.max_blocks * 16         # append position past the table
+    pk.pa_append_kv(dev.k_new[0], dev.v_new[0], dev.k_pool[0], dev.v_pool[0], dev.bt, pos,
+                    dev.err, slot_out=dev.slots)
+    torch.cuda.synchronize()
+    assert dev.err.item() & pk.PA_DEV_BAD_LEN
+    assert dev.slots[0, 0].item() == -1
+
+
+def test_select_evict_bit_exact_on_given_scores():
+    """a5 alone: on the same fp32 scores both sides take the decision in fp64, so
+    the means (rounded to fp32) and the chosen block agree exactly."""
+    rng = np.random.default_rng(5)
+    B, MB, bs, Hkv = 9, 33, 16, 8
+    scores = rng.uniform(0.5, 2.0, (B, MB * bs, Hkv)).astype(np.float32)
+    lens = np.array([0, 15, 16, 17, 100, 528, 500, 333, 48], np.int32)
+    scores[4, 32:48] = 0.4   # planted low block 2 of sequence 4
+    scores[8, :] = 1.25      # all equal: lowest index
+    ev, means, gap = __import__("oracle").select_evict_block(scores, lens, bs)
+    evict = torch.empty(B, dtype=torch.int32, device="cuda")
+    gm = torch.empty(B, MB, dtype=torch.float32, device="cuda")
+    pk.pe_select_evict_block(evict, torch.as_tensor(scores).cuda(), torch.as_tensor(lens).cuda(),
+                             bs, gm)
+    torch.cuda.synchronize()
+    assert evict.cpu().numpy().tolist() == ev.tolist()
+    assert ev[4] == 2 and ev[8] == 0 and ev[0] == -1 and ev[1] == -1
+    gmn = gm.cpu().numpy()
+    assert np.array_equal(np.isnan(gmn), np.isnan(means))
+    ok = ~np.isnan(means)
+    assert np.array_equal(gmn[ok], means[ok].astype(np.float32))
