@@ -12,6 +12,7 @@
 // Softmax runs online in the log2 domain: logits are pre-scaled by
 // scale*log2(e) so every exponential is an exp2.
 #include <math.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -220,7 +221,84 @@ cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, bool int8, cudaStream_t st) {
+    if (a.plan.kernel == 1) return launch_decode_tc(a, st);
     return launch_decode_simple(a, int8, st);
+}
+
+namespace {
+inline size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+inline int up1024(int x) { return (x + 1023) / 1024 * 1024; }
+}  // namespace
+
+// Host launch plan.  The staged tensor-core kernel takes bf16 pools with a block
+// size that is a multiple of 16, Hkv in {1, 2, 4, 8} and G <= 16 when at least
+// two pipeline stages fit in shared memory; everything else runs the
+// general-shape kernel.
+DecodePlan make_decode_plan(int B, int Hq, int Hkv, int d, int bs, int MB, int num_splits,
+                            bool int8, int sms) {
+    DecodePlan p;
+    memset(&p, 0, sizeof p);
+    const int64_t max_ctx = (int64_t)MB * bs;
+    const int G = Hq / Hkv;
+    bool tc = !int8 && bs % 16 == 0 && (Hkv == 1 || Hkv == 2 || Hkv == 4 || Hkv == 8) && G <= 16;
+    if (tc) {
+        const int DC = d / 64;
+        const int box = Hkv * 16 * 128;
+        p.n_sub = 8 / Hkv;
+        const int kv_bytes = p.n_sub * DC * box;
+        const int q_bytes = up1024(Hq * d * 2);
+        p.v_off = kv_bytes;
+        p.q_off = 2 * kv_bytes;
+        p.stage_bytes = 2 * kv_bytes + q_bytes;
+        const int avail = 227 * 1024 - 1024;
+        int ns = avail / (p.stage_bytes + 48);
+        if (ns > 4) ns = 4;
+        if (ns < 2) tc = false;
+        p.nstage = ns;
+        p.smem_bytes = ns * p.stage_bytes + ns * 48 + 1024;
+    }
+    if (tc) {
+        p.kernel = 1;
+        int64_t mc = 128;
+        if (num_splits > 0) mc = ((max_ctx + num_splits - 1) / num_splits + 15) / 16 * 16;
+        if (mc < 16) mc = 16;
+        p.chunk = (int)mc;
+        p.S = (int)((max_ctx + mc - 1) / mc);
+        p.grid = sms;
+        p.units_per_cta = 4;
+        const size_t slots = (size_t)B * p.S * p.n_sub * Hq;
+        p.off_hdr = 0;
+        p.off_ns = 256;
+        p.off_units = p.off_ns + up256((size_t)B * 4);
+        p.off_ml = p.off_units + up256((size_t)B * p.S * 16);
+        p.off_acc = p.off_ml + up256(slots * 2 * 4);
+        p.ws_total = p.off_acc + up256(slots * d * 4);
+        return p;
+    }
+    // general-shape kernel: fixed partitions of `chunk` tokens
+    int64_t s = num_splits;
+    if (s <= 0) {
+        const int64_t units = (int64_t)(B > 0 ? B : 1) * Hkv;
+        const int64_t target = 4LL * sms;
+        s = units >= target ? 1 : (target + units - 1) / units;
+        const int64_t cap = (max_ctx + 255) / 256;
+        if (s > cap) s = cap;
+    }
+    if (s < 1) s = 1;
+    if (s > max_ctx) s = max_ctx;
+    int64_t ch = (max_ctx + s - 1) / s;
+    ch = (ch + 15) / 16 * 16;
+    const int64_t se = (max_ctx + ch - 1) / ch;
+    p.kernel = 0;
+    p.S = (int)se;
+    p.chunk = (int)(se == 1 ? max_ctx : ch);
+    if (p.S > 1) {
+        const size_t rows = (size_t)B * Hq * p.S;
+        p.off_acc = 0;
+        p.off_ml = up256(rows * d * 4);
+        p.ws_total = p.off_ml + up256(rows * 2 * 4);
+    }
+    return p;
 }
 
 }  // namespace pkv

@@ -17,6 +17,25 @@ struct AppendArgs {
     int B, n_new, Hkv, d, bs, MB;
 };
 
+// Header at the start of the staged decode's workspace (written by its plan
+// kernel every call): unit counter, unit count, partition size chosen.
+struct TcHeader {
+    unsigned counter;
+    int n_units;
+    int chunk;
+    int pad[61];
+};
+
+// Launch plan of one decode call, decided on the host from the sizes alone.
+struct DecodePlan {
+    int kernel;         // 0: general-shape kernel, 1: staged tensor-core kernel
+    int S;              // partition slots per sequence
+    int chunk;          // general: tokens per partition; staged: minimum tokens per partition
+    int n_sub;          // staged: 16-token sub-tiles per stage (8 / Hkv)
+    int nstage, stage_bytes, q_off, v_off, smem_bytes, grid, units_per_cta;
+    size_t off_hdr, off_ns, off_units, off_ml, off_acc, ws_total;
+};
+
 // Decode problem.  K/V element type is given by the launcher (bf16 or int8).
 struct DecodeArgs {
     uint16_t *out;                // [B][Hq][d] bf16
@@ -36,6 +55,8 @@ struct DecodeArgs {
     int B, Hq, Hkv, G, d, bs, MB;
     int num_splits;               // S: partitions per sequence (1 = write out directly)
     int chunk;                    // tokens per partition (multiple of 16 when S > 1)
+    void *ws;                     // workspace base
+    DecodePlan plan;
 };
 
 struct ScoreArgs {
@@ -61,6 +82,9 @@ cudaError_t launch_append_int8(const uint16_t *k_new, const uint16_t *v_new, int
 // else the general-shape kernel; then the partition merge when S > 1.
 cudaError_t launch_decode(const DecodeArgs &a, bool int8, cudaStream_t stream);
 cudaError_t launch_decode_simple(const DecodeArgs &a, bool int8, cudaStream_t stream);
+cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream);
+DecodePlan make_decode_plan(int B, int Hq, int Hkv, int d, int bs, int MB, int num_splits,
+                            bool int8, int sms);
 cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t stream);
 
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t stream);

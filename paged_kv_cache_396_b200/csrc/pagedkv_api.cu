@@ -48,43 +48,6 @@ int check_common(int B, int Hkv, int d, int bs, int MB, int64_t N, int64_t block
     return PA_OK;
 }
 
-// Partition of the context for the decode kernels.  Partitions are `chunk`
-// tokens (a multiple of 16) of one sequence; S = ceil(MB*bs / chunk) bounds the
-// partitions of any sequence.  Automatic choice: enough (partition, kv head,
-// sequence) units for ~4 CTAs per SM, never partitions below 256 tokens.
-void choose_split(int B, int Hkv, int bs, int MB, int num_splits, int sms, int *S, int *chunk) {
-    const int64_t max_ctx = (int64_t)MB * bs;
-    int64_t s = num_splits;
-    if (s <= 0) {
-        const int64_t units = (int64_t)(B > 0 ? B : 1) * Hkv;
-        const int64_t target = 4LL * sms;
-        s = units >= target ? 1 : (target + units - 1) / units;
-        const int64_t cap = (max_ctx + 255) / 256;
-        if (s > cap) s = cap;
-    }
-    if (s < 1) s = 1;
-    if (s > max_ctx) s = max_ctx;
-    int64_t ch = (max_ctx + s - 1) / s;
-    ch = (ch + 15) / 16 * 16;
-    const int64_t se = (max_ctx + ch - 1) / ch;
-    *S = (int)se;
-    *chunk = (int)(se == 1 ? max_ctx : ch);
-}
-
-struct WsLayout {
-    size_t acc_off, ml_off, total;
-};
-
-WsLayout ws_layout(int B, int Hq, int d, int S) {
-    WsLayout w{0, 0, 0};
-    if (S <= 1) return w;
-    const size_t rows = (size_t)B * Hq * S;
-    w.acc_off = 0;
-    w.ml_off = (rows * d * sizeof(float) + 255) / 256 * 256;
-    w.total = w.ml_off + (rows * 2 * sizeof(float) + 255) / 256 * 256;
-    return w;
-}
-
 int finish(cudaError_t e) { return e == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
 
 // Shared body of pa_decode / pa_decode_int8.
@@ -106,12 +69,10 @@ int decode_entry(uint16_t *out, const uint16_t *q, const void *kc, const void *v
     if (B == 0) return PA_OK;
     const int sms = device_sms();
     if (sms < 0) return sms;
-    int S = 1, chunk = 0;
-    choose_split(B, Hkv, bs, MB, num_splits, sms, &S, &chunk);
-    const WsLayout wl = ws_layout(B, Hq, d, S);
-    if (wl.total > 0) {
+    const pkv::DecodePlan plan = pkv::make_decode_plan(B, Hq, Hkv, d, bs, MB, num_splits, int8, sms);
+    if (plan.ws_total > 0) {
         if (!ws) return PA_ERR_WORKSPACE;
-        if (ws_bytes < wl.total) return PA_ERR_WORKSPACE;
+        if (ws_bytes < plan.ws_total) return PA_ERR_WORKSPACE;
         if (!al16(ws)) return PA_ERR_ALIGN;
     }
     pkv::DecodeArgs a;
@@ -125,8 +86,12 @@ int decode_entry(uint16_t *out, const uint16_t *q, const void *kc, const void *v
     a.block_tables = bt;
     a.ctx_lens = ctx_lens;
     a.err = err;
-    a.ws_acc = wl.total ? reinterpret_cast<float *>(static_cast<char *>(ws) + wl.acc_off) : nullptr;
-    a.ws_ml = wl.total ? reinterpret_cast<float *>(static_cast<char *>(ws) + wl.ml_off) : nullptr;
+    a.ws = ws;
+    a.plan = plan;
+    a.ws_acc = plan.ws_total ? reinterpret_cast<float *>(static_cast<char *>(ws) + plan.off_acc)
+                             : nullptr;
+    a.ws_ml = plan.ws_total ? reinterpret_cast<float *>(static_cast<char *>(ws) + plan.off_ml)
+                            : nullptr;
     a.block_stride = block_stride;
     a.N = N;
     a.scale_log2 = scale * 1.4426950408889634f;
@@ -137,8 +102,8 @@ int decode_entry(uint16_t *out, const uint16_t *q, const void *kc, const void *v
     a.d = d;
     a.bs = bs;
     a.MB = MB;
-    a.num_splits = S;
-    a.chunk = chunk;
+    a.num_splits = plan.S;
+    a.chunk = plan.chunk;
     return finish(pkv::launch_decode(a, int8, static_cast<cudaStream_t>(stream)));
 }
 
@@ -213,9 +178,9 @@ size_t pa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int bs, int max_
     if (B <= 0 || Hq < 1 || Hkv < 1 || bs < 1 || max_blocks_per_seq < 1) return 0;
     const int sms = device_sms();
     if (sms < 0) return 0;
-    int S = 1, chunk = 0;
-    choose_split(B, Hkv, bs, max_blocks_per_seq, num_splits, sms, &S, &chunk);
-    return ws_layout(B, Hq, d, S).total;
+    if (Hq < Hkv || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
+    return pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits, false, sms)
+        .ws_total;
 }
 
 int pa_decode_plan(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq, int num_splits,
@@ -225,8 +190,11 @@ int pa_decode_plan(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq
     if (d != 64 && d != 128) return PA_ERR_SHAPE;
     const int sms = device_sms();
     if (sms < 0) return sms;
-    choose_split(B, Hkv, bs, max_blocks_per_seq, num_splits, sms, num_splits_out,
-                 chunk_tokens_out);
+    if (Hq < Hkv || Hq % Hkv != 0) return PA_ERR_SHAPE;
+    const pkv::DecodePlan p =
+        pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits, false, sms);
+    *num_splits_out = p.S;
+    *chunk_tokens_out = p.chunk;
     return PA_OK;
 }
 

@@ -27,6 +27,11 @@ MEDIUM = {
     "c4m": W.scaled(C["c4"], key="c4m", batch=3, old_lens=(4096, 3000, 257)),
     # INT8, G = 8
     "c5m": W.scaled(C["c5"], key="c5m", batch=5, old_lens=(300, 1, 16, 255, 512)),
+    # block size 12 (not a multiple of 16): the general-shape kernel, with G = 16
+    "bs12": W.scaled(C["c3"], key="bs12", layers=1, batch=4, hq=64, hkv=4, block_size=12,
+                     old_len_range=(1, 700), outlier_frac=0.0),
+    # G = 16 on the staged kernel, d = 64
+    "g16": W.scaled(C["c2"], key="g16", layers=1, batch=3, hq=64, hkv=4, old_lens=(500, 33, 64)),
 }
 
 
