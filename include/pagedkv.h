@@ -193,6 +193,38 @@ int pa_decode_int8(uint16_t *out, const uint16_t *q,
                    int num_splits, void *workspace, size_t workspace_bytes,
                    int32_t *err_flag, void *stream);
 
+/* ============================================================================
+ * pa_decode without a caller-provided workspace (no counterpart in the pages;
+ * it exists for callers, not for the method).
+ *
+ * Some callers cannot allocate device memory: a host runtime whose memory
+ * manager owns every byte of the GPU and forbids raw allocations, a plain-C
+ * caller that holds only device pointers handed to it, or a process that has
+ * reserved its whole memory budget at start-up.  For them this entry point
+ * computes exactly what pa_decode computes, with the same arguments minus the
+ * workspace, and takes its scratch from a fixed array that lives inside the
+ * library: PA_STATIC_SCRATCH_BYTES (16 MiB) on every GPU that loads the library,
+ * held until the process exits.  It allocates nothing.
+ *   num_splits : as pa_decode, except that 0 picks the largest partition count
+ *                whose scratch fits the array.  When the scratch needed for the
+ *                given sizes (and a non-zero num_splits) exceeds the array, the
+ *                call returns PA_ERR_WORKSPACE and launches nothing.
+ *   The first call on each device looks up the array's device address with the
+ *   device current; make that first call before any stream capture.
+ *   All calls on a device share the one array: two calls whose kernels overlap
+ *   on the GPU (different streams, or different host threads) race and give
+ *   wrong results; order them on one stream.  Nothing in the array needs to
+ *   start at zero: every call writes what it later reads.
+ * ==========================================================================*/
+#define PA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+int pa_decode_static_scratch(uint16_t *out, const uint16_t *q,
+                             const uint16_t *k_cache, const uint16_t *v_cache,
+                             int64_t block_stride, const int32_t *block_tables,
+                             int max_blocks_per_seq, const int32_t *ctx_lens, int B, int Hq,
+                             int Hkv, int d, int bs, int64_t num_blocks, float scale,
+                             int num_splits, int32_t *err_flag, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -107,6 +107,24 @@ int decode_entry(uint16_t *out, const uint16_t *q, const void *kc, const void *v
     return finish(pkv::launch_decode(a, int8, static_cast<cudaStream_t>(stream)));
 }
 
+// Scratch for pa_decode_static_scratch: a fixed array inside the library, one
+// copy per device that loads it.  Host code must not use the symbol itself as a
+// device address; static_scratch_address() looks the address up per device.
+__device__ __align__(256) unsigned char g_static_scratch[PA_STATIC_SCRATCH_BYTES];
+std::atomic<void *> g_scratch_addr[64];
+
+// Device address of g_static_scratch on the current device (looked up once per
+// device, with that device current), or nullptr on failure.
+void *static_scratch_address() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    void *p = g_scratch_addr[dev].load();
+    if (p) return p;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    g_scratch_addr[dev].store(p);
+    return p;
+}
+
 }  // namespace
 
 extern "C" {
@@ -249,6 +267,50 @@ int pe_select_evict_block(int32_t *evict, float *block_means, const float *score
     return finish(pkv::launch_select_evict(evict, block_means, scores, ctx_lens, B,
                                            max_blocks_per_seq, Hkv, bs,
                                            static_cast<cudaStream_t>(stream)));
+}
+
+int pa_decode_static_scratch(uint16_t *out, const uint16_t *q, const uint16_t *k_cache,
+                             const uint16_t *v_cache, int64_t block_stride,
+                             const int32_t *block_tables, int max_blocks_per_seq,
+                             const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
+                             int64_t num_blocks, float scale, int num_splits, int32_t *err_flag,
+                             void *stream) {
+    if (B == 0) return PA_OK;
+    if (num_splits < 0) return PA_ERR_SHAPE;
+    int rc = check_common(B, Hkv, d, bs, max_blocks_per_seq, num_blocks, block_stride);
+    if (rc) return rc;
+    if (Hq < Hkv || Hq % Hkv != 0 || Hq / Hkv > 16) return PA_ERR_SHAPE;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    const size_t cap = PA_STATIC_SCRATCH_BYTES;
+    int splits = num_splits;
+    if (splits == 0) {
+        // largest partition count whose scratch fits, starting from the automatic one
+        int auto_s = pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, 0, false, sms).S;
+        int lo = 1, hi = auto_s < 1 ? 1 : auto_s;
+        if (pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, hi, false, sms)
+                .ws_total <= cap) {
+            lo = hi;
+        } else {
+            while (lo < hi) {  // invariant: ws(lo) fits or lo == 1
+                const int mid = (lo + hi + 1) / 2;
+                if (pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, mid, false, sms)
+                        .ws_total <= cap)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+        }
+        splits = lo;
+    }
+    if (pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, splits, false, sms).ws_total >
+        cap)
+        return PA_ERR_WORKSPACE;
+    void *ws = static_scratch_address();
+    if (!ws) return PA_ERR_CUDA;
+    return decode_entry(out, q, k_cache, v_cache, nullptr, nullptr, false, block_stride,
+                        block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
+                        scale, splits, ws, cap, err_flag, stream);
 }
 
 }  // extern "C"

@@ -33,6 +33,7 @@ EXPORTED = (
     "pa_status_string", "pa_version", "pa_append_kv", "pa_decode_workspace_bytes", "pa_decode_plan",
     "pa_decode",
     "pe_score_tokens", "pe_select_evict_block", "pa_append_kv_int8", "pa_decode_int8",
+    "pa_decode_static_scratch",
 )
 
 
@@ -75,6 +76,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode_int8.restype = i32
     lib.pa_decode_int8.argtypes = [p, p, p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, i64,
                                    f32, i32, p, sz, p, p]
+    lib.pa_decode_static_scratch.restype = i32
+    lib.pa_decode_static_scratch.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32,
+                                             i64, f32, i32, p, p]
     lib.pe_score_tokens.restype = i32
     lib.pe_score_tokens.argtypes = [p, p, p, i64, p, i32, p, i32, i32, i32, i32, i64, p, p]
     lib.pe_select_evict_block.restype = i32
@@ -231,6 +235,28 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
                           float(scale), int(num_splits), ws_ptr, ws_n, _ptr(err_flag),
                           _stream(stream))
     _check("pa_decode", rc)
+
+
+def pa_decode_static_scratch(out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
+                             num_splits=0, stream=None):
+    """pa_decode for callers that cannot allocate device memory: the same result,
+    with scratch taken from a fixed 16 MiB array inside the library (shared by all
+    calls on a device; calls that overlap on the GPU race).  num_splits=0 picks the
+    largest partition count that fits; sizes that cannot fit raise PagedKVError."""
+    _decode_checks(out, q, block_tables, ctx_lens, err_flag)
+    _want(k_cache, torch.bfloat16, "k_cache")
+    _want(v_cache, torch.bfloat16, "v_cache")
+    N, bs, Hkv, d, stride = _pool_geometry(k_cache, "k_cache")
+    _same_pool(k_cache, v_cache)
+    B, Hq, dq = q.shape
+    if dq != d:
+        raise ValueError("q head_dim differs from the pool's")
+    bt = block_tables.contiguous()
+    rc = load().pa_decode_static_scratch(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), stride,
+                                         _ptr(bt), bt.shape[1], _ptr(ctx_lens.contiguous()), B, Hq,
+                                         Hkv, d, bs, N, float(scale), int(num_splits),
+                                         _ptr(err_flag), _stream(stream))
+    _check("pa_decode_static_scratch", rc)
 
 
 def pa_decode_int8(out, q, kq_cache, vq_cache, k_scale, v_scale, block_tables, ctx_lens, scale,
