@@ -52,8 +52,12 @@ def parse():
     ap.add_argument("--workload", default="c3", choices=["c2", "c3", "c4", "c5"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling aid: keep only this many layers of the workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every call from Python instead of replaying a CUDA graph")
     return ap.parse_args()
 
 
@@ -139,10 +143,11 @@ class Clocks:
 
 
 # ----------------------------------------------------------------------------- model
-def decode_algorithmic_bytes(cfg, ctx_lens, S, chunk):
-    """Bytes one decode launch (one layer) must move: K/V rows of every cached
-    token (plus INT8 scales), q and out, the table entries read, and the
-    partition partials written and read back when S > 1."""
+def decode_algorithmic_bytes(cfg, ctx_lens, partial_slots, n_units=0):
+    """Bytes one decode call (one layer) must move: K/V rows of every cached
+    token (plus INT8 scales), q and out, the table entries and lengths read, the
+    partition partials written and read back by the merge (partial_slots slots
+    of Hq rows of d + 2 floats), and the partition list of the staged kernel."""
     elt = 1 if cfg.int8 else 2
     tok = int(np.sum(ctx_lens))
     kv = tok * cfg.hkv * cfg.head_dim * 2 * elt
@@ -150,12 +155,10 @@ def decode_algorithmic_bytes(cfg, ctx_lens, S, chunk):
         kv += tok * cfg.hkv * 2 * 4
     qo = 2 * cfg.batch * cfg.hq * cfg.head_dim * 2
     nblk = int(sum(-(-int(n) // cfg.block_size) for n in ctx_lens))
-    table = nblk * 4 + cfg.batch * 4
-    parts = 0
-    if S > 1:
-        n_parts = int(sum(max(1, -(-int(n) // chunk)) for n in ctx_lens))
-        parts = 2 * n_parts * cfg.hq * (cfg.head_dim + 2) * 4
-    return kv + qo + table + parts
+    table = nblk * 4 + 2 * cfg.batch * 4
+    parts = 2 * partial_slots * cfg.hq * (cfg.head_dim + 2) * 4
+    plan = 2 * n_units * 16 + 2 * cfg.batch * 4
+    return kv + qo + table + parts + plan
 
 
 class Runner:
@@ -176,7 +179,10 @@ class Runner:
         self.out = torch.empty(self.L, B, Hq, d, dtype=torch.bfloat16, device=device)
         self.ws = pk.alloc_workspace(B, Hq, Hkv, d, bs, MB, num_splits, device)
         self.num_splits = num_splits
-        self.S, self.chunk = pk.pa_decode_plan(B, Hq, Hkv, d, bs, MB, num_splits)
+        self.S, self.chunk, self.dec_launches = pk.pa_decode_plan(B, Hq, Hkv, d, bs, MB,
+                                                                  num_splits)
+        # the staged kernel launches plan + decode (+ merge); the general one decode (+ merge)
+        self.staged = self.dec_launches - (1 if self.S > 1 else 0) >= 2
         if cfg.int8:
             N = wl.num_blocks
             self.kq = torch.zeros(self.L, N, bs, Hkv, d, dtype=torch.int8, device=device)
@@ -197,10 +203,28 @@ class Runner:
         torch.cuda.synchronize(device)
         self.q = wl.q
         self.k_new, self.v_new = wl.k_new, wl.v_new
-        self.decode_bytes = decode_algorithmic_bytes(cfg, wl.ctx_lens, self.S, self.chunk)
+        self.decode_bytes = None
+
+    def account_bytes(self):
+        """Algorithmic bytes of one decode call, with the partition counts the
+        last call actually used (read back from the workspace)."""
+        cfg, pk = self.cfg, self.pk
+        n_sub = max(1, 8 // cfg.hkv)
+        if self.staged:
+            n_units, chunk, ns = pk.workspace_plan(self.ws, cfg.batch)
+            slots = sum(n * n_sub for n in ns if n > 1 or n_sub > 1)
+            self.chunk_used = chunk
+        else:
+            n_units = 0
+            slots = 0
+            if self.S > 1:
+                slots = sum(max(1, -(-int(n) // self.chunk)) for n in self.wl.ctx_lens)
+            self.chunk_used = self.chunk
+        self.decode_bytes = decode_algorithmic_bytes(cfg, self.wl.ctx_lens, slots, n_units)
+        self.partitions = slots
 
     def launches_per_step(self):
-        per_layer = (1 if self.cfg.append else 0) + (2 if self.S > 1 else 1)
+        per_layer = (1 if self.cfg.append else 0) + self.dec_launches
         if self.cfg.score:
             per_layer += 2
         return per_layer * self.L
@@ -349,6 +373,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
     cfg = W.CONFIGS[args.workload]
+    if args.layers:
+        cfg = W.scaled(cfg, layers=args.layers)
     r = Runner(cfg, device, args.num_splits)
     stream = torch.cuda.current_stream(device)
 
@@ -358,9 +384,31 @@ def main():
     if r.err.item() != 0:
         raise SystemExit(f"device error flag {r.err.item()} during warm-up")
 
-    # --- device-timed region: K steps, events on the launching stream
-    ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-          for _ in range(r.L * args.steps)]
+    r.account_bytes()
+    use_graph = not args.no_graph
+    R = max(1, -(-16 // r.L))          # steps per captured graph: >= 16 decode samples
+
+    def capture(steps, with_events):
+        ev = ([[torch.cuda.Event(enable_timing=True, external=True),
+                torch.cuda.Event(enable_timing=True, external=True)]
+               for _ in range(r.L * steps)] if with_events else None)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for k in range(steps):
+                r.step(ev[k * r.L:(k + 1) * r.L] if ev else None)
+        return g, ev
+
+    if use_graph:
+        gR, evR = capture(R, True)
+        g1, ev1 = capture(1, True)
+        gR.replay()
+        g1.replay()
+        torch.cuda.synchronize(device)
+    else:
+        ev_eager = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+                    for _ in range(r.L * args.steps)]
+
+    # --- device-timed region: exactly K steps
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
@@ -369,13 +417,23 @@ def main():
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for k in range(args.steps):
-        r.step(ev[k * r.L:(k + 1) * r.L])
+    if use_graph:
+        for _ in range(args.steps // R):
+            gR.replay()
+        for _ in range(args.steps % R):
+            g1.replay()
+    else:
+        for k in range(args.steps):
+            r.step(ev_eager[k * r.L:(k + 1) * r.L])
     t_end.record(stream)
     torch.cuda.synchronize(device)
     clk = clocks.stop()
     total_ms = t_start.elapsed_time(t_end)
-    decode_ms = [a.elapsed_time(b) for a, b in ev]
+    if use_graph:
+        samples = evR if args.steps >= R else ev1
+    else:
+        samples = ev_eager
+    decode_ms = [a.elapsed_time(b) for a, b in samples]
     if world > 1:
         t = torch.tensor([total_ms], device=device)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -406,15 +464,27 @@ def main():
     h2d = sum(t.numel() * t.element_size() for t in h_in)
     d2h = h_out.numel() * h_out.element_size()
     e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step():
+        for h, dv in zip(h_in, d_in):
+            dv.copy_(h, non_blocking=True)
+        r.step()
+        h_out.copy_(r.out, non_blocking=True)
+
+    if use_graph:
+        ge = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ge):
+            e2e_step()
+        ge.replay()
     torch.cuda.synchronize(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        for h, dv in zip(h_in, d_in):
-            dv.copy_(h, non_blocking=True)
-        r.step()
-        h_out.copy_(r.out, non_blocking=True)
+        if use_graph:
+            ge.replay()
+        else:
+            e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
@@ -440,7 +510,9 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int8" if cfg.int8 else "bf16", "data": "synthetic",
             "config": dict(workload_config(cfg), parallelism=f"replicas{world}",
-                           num_splits=r.S, chunk_tokens=r.chunk),
+                           decode_kernel="staged-tc" if r.staged else "general",
+                           partitions=r.partitions, chunk_tokens=r.chunk_used,
+                           cuda_graph=use_graph),
             "roofline": {"bound": "hbm", "kernel": "pa_decode" + ("_int8" if cfg.int8 else ""),
                          "achieved": achieved, "peak": peak, "peak_source": peak_kind,
                          "unit": "GB/s", "frac": achieved / peak,

@@ -117,11 +117,13 @@ size_t pa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int bs,
 
 /* The partition pa_decode chooses for these sizes (no counterpart in the pages:
  * the split-KV partition exists only in this implementation).  *num_splits_out
- * receives the maximum number of partitions of one sequence (1 = no merge
- * pass), *chunk_tokens_out the tokens per partition.  Returns PA_OK or a
- * PA_ERR_* code. */
+ * receives the maximum number of partitions of one sequence, *chunk_tokens_out
+ * the tokens per partition (for the staged kernel: the minimum; it sizes the
+ * partitions from the actual lengths on the device), *launches_out (nullable)
+ * the kernels one pa_decode call launches.  Returns PA_OK or a PA_ERR_* code. */
 int pa_decode_plan(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq,
-                   int num_splits, int *num_splits_out, int *chunk_tokens_out);
+                   int num_splits, int *num_splits_out, int *chunk_tokens_out,
+                   int *launches_out);
 
 int pa_decode(uint16_t *out, const uint16_t *q,
               const uint16_t *k_cache, const uint16_t *v_cache, int64_t block_stride,

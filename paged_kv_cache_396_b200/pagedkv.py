@@ -69,7 +69,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode_workspace_bytes.restype = sz
     lib.pa_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32]
     lib.pa_decode_plan.restype = i32
-    lib.pa_decode_plan.argtypes = [i32, i32, i32, i32, i32, i32, i32, p, p]
+    lib.pa_decode_plan.argtypes = [i32, i32, i32, i32, i32, i32, i32, p, p, p]
     lib.pa_decode.restype = i32
     lib.pa_decode.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, i64, f32, i32,
                               p, sz, p, p]
@@ -192,11 +192,23 @@ def pa_decode_workspace_bytes(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits=
 
 
 def pa_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits=0):
-    """(partitions per sequence at most, tokens per partition) pa_decode will use."""
-    s, c = ctypes.c_int(0), ctypes.c_int(0)
+    """(partitions per sequence at most, tokens per partition, kernel launches per
+    call) that pa_decode will use for these sizes."""
+    s, c, n = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
     _check("pa_decode_plan", load().pa_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq,
-                                                   num_splits, ctypes.byref(s), ctypes.byref(c)))
-    return s.value, c.value
+                                                   num_splits, ctypes.byref(s), ctypes.byref(c),
+                                                   ctypes.byref(n)))
+    return s.value, c.value, n.value
+
+
+def workspace_plan(workspace, B):
+    """Diagnostic: the partition plan the staged decode kernel left in its
+    workspace on the last call (header: unit counter, unit count, partition
+    tokens; then partitions per sequence at byte 256).  Returns
+    (n_units, chunk_tokens, partitions_per_sequence[B]) on the host."""
+    head = workspace[:16].view(torch.int32).cpu().tolist()
+    ns = workspace[256:256 + 4 * B].view(torch.int32).cpu().tolist()
+    return head[1], head[2], ns
 
 
 def alloc_workspace(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits=0, device=None):
