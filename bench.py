@@ -191,11 +191,18 @@ class Runner:
             self.vs = torch.zeros_like(self.ks)
             zeros = torch.zeros(B, dtype=torch.int32, device=device)
             for l in range(self.L):
-                n = int(wl.old_lens.max())
-                assert (wl.old_lens == n).all()
-                pk.pa_append_kv_int8(wl.k_hist[l, :, :n].contiguous(),
-                                     wl.v_hist[l, :, :n].contiguous(), self.kq[l], self.vq[l],
-                                     self.ks[l], self.vs[l], self.bt, zeros, self.err)
+                if (wl.old_lens == wl.old_lens[0]).all():
+                    n = int(wl.old_lens[0])
+                    pk.pa_append_kv_int8(wl.k_hist[l, :, :n].contiguous(),
+                                         wl.v_hist[l, :, :n].contiguous(), self.kq[l], self.vq[l],
+                                         self.ks[l], self.vs[l], self.bt, zeros, self.err)
+                    continue
+                for b in range(B):  # unequal lengths: one prompt-style append per sequence
+                    n = int(wl.old_lens[b])
+                    pk.pa_append_kv_int8(wl.k_hist[l, b:b + 1, :n].contiguous(),
+                                         wl.v_hist[l, b:b + 1, :n].contiguous(), self.kq[l],
+                                         self.vq[l], self.ks[l], self.vs[l], self.bt[b:b + 1],
+                                         zeros[b:b + 1], self.err)
             wl.k_hist = wl.v_hist = None
         if cfg.score:
             self.scores = torch.zeros(B, MB * bs, Hkv, dtype=torch.float32, device=device)

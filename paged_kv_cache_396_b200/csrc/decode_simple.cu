@@ -221,7 +221,7 @@ cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, bool int8, cudaStream_t st) {
-    if (a.plan.kernel == 1) return launch_decode_tc(a, st);
+    if (a.plan.kernel == 1) return launch_decode_tc(a, int8, st);
     return launch_decode_simple(a, int8, st);
 }
 
@@ -230,29 +230,40 @@ inline size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 inline int up1024(int x) { return (x + 1023) / 1024 * 1024; }
 }  // namespace
 
-// Host launch plan.  The staged tensor-core kernel takes bf16 pools with a block
-// size that is a multiple of 16, Hkv in {1, 2, 4, 8} and G <= 16 when at least
-// two pipeline stages fit in shared memory; everything else runs the
-// general-shape kernel.
+// Host launch plan.  The staged tensor-core kernel takes pools with a block
+// size that is a multiple of 16, Hkv in {1, 2, 4, 8} and G <= 16 (INT8: d = 128)
+// when at least two pipeline stages fit in shared memory; everything else runs
+// the general-shape kernel.
 DecodePlan make_decode_plan(int B, int Hq, int Hkv, int d, int bs, int MB, int num_splits,
                             bool int8, int sms) {
     DecodePlan p;
     memset(&p, 0, sizeof p);
     const int64_t max_ctx = (int64_t)MB * bs;
     const int G = Hq / Hkv;
-    bool tc = !int8 && bs % 16 == 0 && (Hkv == 1 || Hkv == 2 || Hkv == 4 || Hkv == 8) && G <= 16;
+    bool tc = bs % 16 == 0 && (Hkv == 1 || Hkv == 2 || Hkv == 4 || Hkv == 8) && G <= 16 &&
+              (!int8 || d == 128);
     if (tc) {
-        const int DC = d / 64;
-        const int box = Hkv * 16 * 128;
-        p.n_sub = 8 / Hkv;
-        const int kv_bytes = p.n_sub * DC * box;
-        const int q_bytes = up1024(Hq * d * 2);
+        const int box = Hkv * 16 * 128;  // one 128-byte slice of d of 16 tokens, all heads
+        const int DC = int8 ? d / 128 : d / 64;
+        const int sub_kv = DC * box;                    // K (or V) bytes of one 16-token sub-tile
+        const int sub_sc = int8 ? 16 * Hkv * 4 : 0;     // its scale rows
+        p.wph = 8 / Hkv;
+        // sub-tiles per warp per stage: stages of about 64 KB of K + V amortise the
+        // per-stage cost of the pipeline
+        int tpw = 1;
+        while (tpw < 4 && p.wph * tpw * 2 <= 32 && 2 * (p.wph * tpw * 2) * sub_kv <= 64 * 1024)
+            tpw *= 2;  // doubling keeps the stage (K + V of n_sub sub-tiles) within 64 KB
+        p.tpw = tpw;
+        p.n_sub = p.wph * tpw;
+        const int kv_bytes = p.n_sub * sub_kv;
+        const int sc_bytes = p.n_sub * sub_sc;
         p.v_off = kv_bytes;
-        p.q_off = 2 * kv_bytes;
-        p.stage_bytes = 2 * kv_bytes + q_bytes;
+        p.ks_off = 2 * kv_bytes;
+        p.vs_off = p.ks_off + sc_bytes;
+        p.stage_bytes = up1024(p.vs_off + sc_bytes);
         const int avail = 227 * 1024 - 1024;
         int ns = avail / (p.stage_bytes + 48);
-        if (ns > 4) ns = 4;
+        if (ns > 8) ns = 8;
         if (ns < 2) tc = false;
         p.nstage = ns;
         p.smem_bytes = ns * p.stage_bytes + ns * 48 + 1024;
@@ -266,7 +277,7 @@ DecodePlan make_decode_plan(int B, int Hq, int Hkv, int d, int bs, int MB, int n
         p.S = (int)((max_ctx + mc - 1) / mc);
         p.grid = sms;
         p.units_per_cta = 4;
-        const size_t slots = (size_t)B * p.S * p.n_sub * Hq;
+        const size_t slots = (size_t)B * p.S * p.wph * Hq;
         p.off_hdr = 0;
         p.off_ns = 256;
         p.off_units = p.off_ns + up256((size_t)B * 4);

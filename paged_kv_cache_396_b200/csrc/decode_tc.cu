@@ -14,15 +14,19 @@
 //   per SM); its producer warp takes units from an atomic counter, so long units
 //   start first and short ones fill the tail.
 // Per CTA
-//   warp 8 (producer): for each stage of 16*n_sub tokens, looks the physical
-//   blocks up in the block table and issues 5-D TMA loads of the K and V rows of
-//   ALL kv heads of 16 consecutive tokens (one box per 64-element slice of d),
-//   plus, on a unit's first stage, a bulk copy of the sequence's query rows.
+//   warp 8 (producer): for each stage of 16*n_sub tokens (n_sub sub-tiles of 16
+//   tokens; a stage carries about 64 KB of K and V), lane j looks the physical
+//   block of sub-tile j up in the block table (through a 32-entry per-unit cache
+//   held one id per lane) and issues 5-D TMA loads of the K and V rows of ALL kv
+//   heads of those 16 tokens (one box per 128 bytes of d),
+//   (INT8: plus bulk copies of the 16 tokens' K and V scale rows).
 //   The tensor map orders the box as [head][token][64 elements] with 128-byte
 //   swizzle, so each head's 16 token rows occupy 16 consecutive 128-byte rows
 //   and ldmatrix reads them without bank conflicts.
-//   warps 0..7 (consumers): warp w owns kv head w % Hkv and 16-token sub-tile
-//   w / Hkv of every stage.  S = Q K^T with the G query heads of the group as
+//   warps 0..7 (consumers): warp w owns kv head w % Hkv and sub-tiles
+//   w / Hkv + k * (8 / Hkv), k < tpw, of every stage; at a unit's start it loads
+//   its query fragments
+//   straight from global memory (L2).  S = Q K^T with the G query heads of the group as
 //   the 16 rows of an m16n8k16 MMA (rows >= G are zero), online softmax on the
 //   fp32 accumulators (exp2 domain), P rounded to bf16, O += P V with V read by
 //   ldmatrix.trans.  The stage is released to the producer through an mbarrier.
@@ -69,8 +73,14 @@ struct Args {
     const int32_t *ns;
     float *ws_acc;
     float *ws_ml;
+    const float *k_scale;  // INT8 pools: [N][bs][Hkv] fp32
+    const float *v_scale;
     int64_t N;
-    int B, Hq, Hkv, G, bs, MB, S, n_sub, nstage, stage_bytes, q_off, v_off, box_bytes;
+    int B, Hq, Hkv, G, bs, MB, S, nstage, stage_bytes, v_off, ks_off, vs_off, box_bytes;
+    int wph;        // consumer warps per kv head (8 / Hkv): partial slots per unit
+    int tpw;        // 16-token sub-tiles per warp per stage
+    int n_sub;      // sub-tiles per stage (wph * tpw)
+    int tpb_shift;  // log2(bs / 16) when bs / 16 is a power of two, else -1
     float scale_log2;
 };
 
@@ -127,15 +137,34 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *ctx_lens, int
         }
     }
     __syncthreads();
-    if (tid == 0) {  // exclusive prefix, largest bucket first
-        int run = 0;
-        for (int k = 1023; k >= 0; --k) {
-            const int c = hist[k];
-            hist[k] = run;
-            run += c;
+    {   // exclusive prefix over the buckets, largest first (thread t owns bucket 1023 - t)
+        const int k = 1023 - tid;
+        const int v = hist[k];
+        int inc = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(kFull, inc, o);
+            if ((tid & 31) >= o) inc += n;
         }
-        hdr->n_units = run;
-        hdr->counter = 0u;
+        __shared__ int s_warp[32];
+        if ((tid & 31) == 31) s_warp[tid >> 5] = inc;
+        __syncthreads();
+        if (tid < 32) {
+            int w = s_warp[tid];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(kFull, w, o);
+                if (tid >= o) w += n;
+            }
+            s_warp[tid] = w;  // inclusive totals of warps 0..tid
+        }
+        __syncthreads();
+        const int before = (tid >> 5) ? s_warp[(tid >> 5) - 1] : 0;
+        hist[k] = before + inc - v;
+        if (tid == 1023) {
+            hdr->n_units = before + inc;
+            hdr->counter = 0u;
+        }
     }
     __syncthreads();
     for (int b = tid; b < B; b += blockDim.x) {
@@ -154,14 +183,17 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *ctx_lens, int
 // ---------------------------------------------------------------------------
 // decode: persistent, warp-specialised
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool I8>
 __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensorMap *vmap,
                                          const Args &a, uint8_t *stages, StageMeta *meta,
                                          uint64_t *full, uint64_t *empty) {
-    constexpr int DC = D / 64;
+    // one box covers 128 bytes of d: 64 bf16 or 128 int8 values
+    constexpr int DC = I8 ? D / 128 : D / 64;
     const int lane = threadIdx.x & 31;
     const int T_s = kTile * a.n_sub;
-    const uint32_t qbytes = (uint32_t)a.Hq * D * 2;
+    const uint32_t sc_bytes = (uint32_t)kTile * a.Hkv * 4;  // one sub-tile's scale rows
+    const uint32_t sub_bytes = 2u * DC * (uint32_t)a.box_bytes + (I8 ? 2u * sc_bytes : 0u);
+    const int tpb = a.bs / kTile;                            // 16-token tiles per block
     const int n_units = a.hdr->n_units;
     const uint64_t policy = ptx::policy_evict_first();
     int stage = 0;
@@ -178,74 +210,66 @@ __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensor
         if ((int)u >= n_units) break;
         const int4 un = a.units[u];
         const int b = un.x, c = un.y, t0 = un.z, t1 = un.w;
-        const bool direct = (a.n_sub == 1) && (a.ns[b] == 1);
+        const bool direct = (a.wph == 1) && (a.ns[b] == 1);
         const int nst = t1 > t0 ? (t1 - t0 + T_s - 1) / T_s : 1;
         const int32_t *bt_row = a.bt + (int64_t)b * a.MB;
-        int cache_base = -1, cache = 0;  // lane k caches the id of block cache_base + k
-        for (int si = 0; si < nst; ++si) {
+        // lane k caches the physical id of block cache_base + k (blocks of this unit only)
+        const int last_blk = t1 > t0 ? (t1 - 1) / a.bs : 0;
+        int cache_base = 0x7fffffff, cache = -1;
+        int ti = t0 / kTile;  // 16-token tile index of this lane's sub-tile, stage 0
+        ti += lane;
+        for (int si = 0; si < nst; ++si, ti += a.n_sub) {
             const int ts = t0 + si * T_s, te = min(ts + T_s, t1);
-            if (te > ts) {
-                const int last_blk = (te - 1) / a.bs;
-                if (cache_base < 0 || last_blk >= cache_base + 32) {
-                    cache_base = ts / a.bs;
-                    const int blk = cache_base + lane;
-                    cache = blk <= (t1 - 1) / a.bs ? __ldg(bt_row + blk) : -1;
-                }
+            // sub-tile of lane j (j < n_sub): tokens ts + 16 j .. ; its block and slot
+            const int blk = a.tpb_shift >= 0 ? (ti >> a.tpb_shift) : ti / tpb;
+            const int slot = (ti - blk * tpb) * kTile;
+            const bool mine = lane < a.n_sub && ts + kTile * lane < te;
+            const int blk_hi = __shfl_sync(kFull, blk, min(a.n_sub, 32) - 1);
+            if (blk_hi - cache_base >= 32 || cache_base == 0x7fffffff) {  // (re)fill the cache
+                cache_base = __shfl_sync(kFull, blk, 0);
+                const int bk = cache_base + lane;
+                cache = bk <= last_blk ? __ldg(bt_row + bk) : -1;
             }
-            int phys[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int tok = ts + kTile * j;
-                const int idx = (j < a.n_sub && tok < te) ? tok / a.bs - cache_base : 0;
-                phys[j] = __shfl_sync(kFull, cache, idx & 31);
-            }
+            const int phys = __shfl_sync(kFull, cache, (blk - cache_base) & 31);
+            const bool valid = mine && phys >= 0 && (int64_t)phys < a.N;
+            const unsigned vmask = __ballot_sync(kFull, valid);
+            const unsigned bad = __ballot_sync(kFull, mine && !valid);
             if (!ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
                 if (lane == 0) raise_flag(a.err, PA_DEV_TIMEOUT);
                 ok = false;
                 break;
             }
+            uint8_t *sb = stages + (size_t)stage * a.stage_bytes;
             if (lane == 0) {
-                uint8_t *sb = stages + (size_t)stage * a.stage_bytes;
-                uint32_t bytes = 0;
-                int bad = 0;
-                for (int j = 0; j < a.n_sub; ++j) {
-                    const int tok = ts + kTile * j;
-                    if (tok >= te) break;
-                    if (phys[j] < 0 || (int64_t)phys[j] >= a.N) {
-                        bad |= 1 << j;
-                        continue;
-                    }
-                    bytes += 2u * DC * (uint32_t)a.box_bytes;
-                }
-                if (si == 0) bytes += qbytes;
                 StageMeta &m = meta[stage];
                 m.b = b;
                 m.c = c;
                 m.ts = ts;
                 m.te = te;
-                m.bad = bad;
+                m.bad = (int)bad;
                 m.flags = (si == 0 ? kFirst : 0) | (si == nst - 1 ? kLast : 0) |
                           (direct ? kDirect : 0);
                 if (bad) raise_flag(a.err, PA_DEV_BAD_BLOCK);
-                ptx::mbar_arrive_expect_tx(&full[stage], bytes);
-                for (int j = 0; j < a.n_sub; ++j) {
-                    const int tok = ts + kTile * j;
-                    if (tok >= te) break;
-                    if ((bad >> j) & 1) continue;
-                    const int slot = tok % a.bs;
-#pragma unroll
-                    for (int dc = 0; dc < DC; ++dc) {
-                        const size_t off = (size_t)(j * DC + dc) * a.box_bytes;
-                        ptx::tma_load_5d_hint(sb + off, kmap, &full[stage], 0, slot, 0, dc, phys[j],
-                                              policy);
-                        ptx::tma_load_5d_hint(sb + a.v_off + off, vmap, &full[stage], 0, slot, 0,
-                                              dc, phys[j], policy);
-                    }
-                }
-                if (si == 0) ptx::bulk_load(sb + a.q_off, a.q + (int64_t)b * a.Hq * D, qbytes,
-                                            &full[stage]);
+                ptx::mbar_arrive_expect_tx(&full[stage], __popc(vmask) * sub_bytes);
             }
             __syncwarp();
+            if (valid) {  // each lane loads its own sub-tile
+#pragma unroll
+                for (int dc = 0; dc < DC; ++dc) {
+                    const size_t off = (size_t)(lane * DC + dc) * a.box_bytes;
+                    ptx::tma_load_5d_hint(sb + off, kmap, &full[stage], 0, slot, 0, dc, phys,
+                                          policy);
+                    ptx::tma_load_5d_hint(sb + a.v_off + off, vmap, &full[stage], 0, slot, 0, dc,
+                                          phys, policy);
+                }
+                if (I8) {
+                    const int64_t srow = ((int64_t)phys * a.bs + slot) * a.Hkv;
+                    ptx::bulk_load(sb + a.ks_off + lane * sc_bytes, a.k_scale + srow, sc_bytes,
+                                   &full[stage]);
+                    ptx::bulk_load(sb + a.vs_off + lane * sc_bytes, a.v_scale + srow, sc_bytes,
+                                   &full[stage]);
+                }
+            }
             if (++stage == a.nstage) {
                 stage = 0;
                 phase ^= 1u;
@@ -264,6 +288,28 @@ __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensor
     }
 }
 
+// Load the query fragments of rows g (and g + 8) of kv head h for sequence b
+// straight from global memory (L2): k-step kk of thread (g, tig) takes dims
+// 16*kk + 2*tig (+1) and 16*kk + 8 + 2*tig (+1), the A-operand layout of the
+// m16n8k16 MMA.  Rows >= G are zero.
+template <int D, bool G16>
+__device__ __forceinline__ void load_q_bf16(const Args &a, int b, int h, int g, int tig,
+                                            uint32_t (&qa)[D / 16][2],
+                                            uint32_t (&qb)[G16 ? D / 16 : 1][2]) {
+    const int row = h * a.G + g;
+    const uint32_t *qr =
+        reinterpret_cast<const uint32_t *>(a.q + ((int64_t)b * a.Hq + row) * D) + tig;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        qa[kk][0] = g < a.G ? __ldg(qr + kk * 8) : 0u;
+        qa[kk][1] = g < a.G ? __ldg(qr + kk * 8 + 4) : 0u;
+        if constexpr (G16) {
+            qb[kk][0] = g + 8 < a.G ? __ldg(qr + 4 * D + kk * 8) : 0u;
+            qb[kk][1] = g + 8 < a.G ? __ldg(qr + 4 * D + kk * 8 + 4) : 0u;
+        }
+    }
+}
+
 template <int D, bool G16>
 __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMeta *meta,
                                          uint64_t *full, uint64_t *empty) {
@@ -271,7 +317,7 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
     constexpr int KS = D / 16;  // k-steps of QK^T (and n-tile pairs of PV)
     constexpr int NT = D / 8;   // n-tiles of the output
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = warp % a.Hkv, j = warp / a.Hkv;
+    const int h = warp % a.Hkv, jw = warp / a.Hkv;
     const int g = lane >> 2, tig = lane & 3;
     const int mi = lane >> 3, ri = lane & 7;
     // per-lane byte offsets inside a (head, sub-tile, 64-element) box
@@ -280,7 +326,10 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
     const int tv = ri + ((mi & 1) << 3);         // V: matrices 0,2 -> tokens 0-7; 1,3 -> 8-15
     const int cv = mi >> 1;
     const uint32_t stage0 = ptx::smem_u32(stages);
-    const uint32_t head_off = (uint32_t)(j * DC * a.box_bytes + h * kTile * kBoxRow);
+    // sub-tile jj of a stage: box (jj * DC + dc); head h at row h * 16 + token
+    const uint32_t head_off = (uint32_t)(h * kTile * kBoxRow);
+    const uint32_t sub_bytes = (uint32_t)(DC * a.box_bytes);
+    const uint32_t dc_bytes = (uint32_t)a.box_bytes;
 
     uint32_t qa[KS][2];
     uint32_t qb[G16 ? KS : 1][2];
@@ -298,19 +347,7 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
         if (mt.flags & kEnd) break;
         const uint32_t sb = stage0 + (uint32_t)stage * a.stage_bytes;
         if (mt.flags & kFirst) {
-            const uint32_t qs = sb + a.q_off;
-            const int row = h * a.G + g;
-#pragma unroll
-            for (int kk = 0; kk < KS; ++kk) {
-                const uint32_t ad = qs + (uint32_t)((row * D + kk * 16 + 2 * tig) * 2);
-                qa[kk][0] = g < a.G ? ptx::lds32(ad) : 0u;
-                qa[kk][1] = g < a.G ? ptx::lds32(ad + 16) : 0u;
-                if constexpr (G16) {
-                    const uint32_t adb = ad + 8 * D * 2;
-                    qb[kk][0] = g + 8 < a.G ? ptx::lds32(adb) : 0u;
-                    qb[kk][1] = g + 8 < a.G ? ptx::lds32(adb + 16) : 0u;
-                }
-            }
+            load_q_bf16<D, G16>(a, mt.b, h, g, tig, qa, qb);
             m = -INFINITY;
             l = 0.f;
             mb = -INFINITY;
@@ -321,25 +358,36 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
                 if constexpr (G16) ob[nt][0] = ob[nt][1] = 0.f;
             }
         }
-        const int tj = mt.ts + kTile * j;
+        for (int k = 0; k < a.tpw; ++k) {
+        const int jj = jw + a.wph * k;  // this warp's k-th sub-tile of the stage
+        const int tj = mt.ts + kTile * jj;
         const int nv = max(0, min(kTile, mt.te - tj));
-        if (nv > 0 && !((mt.bad >> j) & 1)) {
-            const uint32_t kbase = sb + head_off;
-            const uint32_t vbase = sb + a.v_off + head_off;
-            // ---- S = Q K^T : two n-tiles of 8 tokens
+        if (nv > 0 && !((mt.bad >> jj) & 1)) {
+            const uint32_t kbase = sb + jj * sub_bytes + head_off;
+            const uint32_t vbase = sb + a.v_off + jj * sub_bytes + head_off;
+            // ---- S = Q K^T : two n-tiles of 8 tokens; even/odd k-steps in separate
+            // accumulators to halve the dependent MMA chain
             float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+            float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
                 const int dc = kk >> 2, c = ((kk & 3) << 1) + ck;
                 uint32_t r[4];
-                ptx::ldmatrix_x4(r, kbase + dc * a.box_bytes + tk * kBoxRow + ((c ^ ri) << 4));
+                ptx::ldmatrix_x4(r, kbase + dc * dc_bytes + tk * kBoxRow + ((c ^ ri) << 4));
+                float(&x0)[4] = (kk & 1) ? e0 : s0;
+                float(&x1)[4] = (kk & 1) ? e1 : s1;
                 if constexpr (G16) {
-                    ptx::mma_bf16(s0, qa[kk][0], qb[kk][0], qa[kk][1], qb[kk][1], r[0], r[1]);
-                    ptx::mma_bf16(s1, qa[kk][0], qb[kk][0], qa[kk][1], qb[kk][1], r[2], r[3]);
+                    ptx::mma_bf16(x0, qa[kk][0], qb[kk][0], qa[kk][1], qb[kk][1], r[0], r[1]);
+                    ptx::mma_bf16(x1, qa[kk][0], qb[kk][0], qa[kk][1], qb[kk][1], r[2], r[3]);
                 } else {
-                    ptx::mma_bf16(s0, qa[kk][0], 0u, qa[kk][1], 0u, r[0], r[1]);
-                    ptx::mma_bf16(s1, qa[kk][0], 0u, qa[kk][1], 0u, r[2], r[3]);
+                    ptx::mma_bf16(x0, qa[kk][0], 0u, qa[kk][1], 0u, r[0], r[1]);
+                    ptx::mma_bf16(x1, qa[kk][0], 0u, qa[kk][1], 0u, r[2], r[3]);
                 }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                s0[i] += e0[i];
+                s1[i] += e1[i];
             }
             // ---- online softmax (rows g and, for G > 8, g + 8)
             const int t_a = 2 * tig, t_b = 8 + 2 * tig;
@@ -376,13 +424,16 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
                 pa1 = ptx::pack_bf16(q0, q1);
                 pa3 = ptx::pack_bf16(q2, q3);
             }
+            // rescale only when some row maximum moved (alpha == 1 exactly otherwise)
+            if (__any_sync(kFull, alpha != 1.f || alphab != 1.f)) {
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                o[nt][0] *= alpha;
-                o[nt][1] *= alpha;
-                if constexpr (G16) {
-                    ob[nt][0] *= alphab;
-                    ob[nt][1] *= alphab;
+                for (int nt = 0; nt < NT; ++nt) {
+                    o[nt][0] *= alpha;
+                    o[nt][1] *= alpha;
+                    if constexpr (G16) {
+                        ob[nt][0] *= alphab;
+                        ob[nt][1] *= alphab;
+                    }
                 }
             }
             // ---- O += P V
@@ -390,38 +441,38 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
             const uint32_t mhi = (vb0 ? 0x0000ffffu : 0u) | (vb1 ? 0xffff0000u : 0u);
             const bool partial = nv < kTile;
 #pragma unroll
-            for (int jj = 0; jj < KS; ++jj) {
-                const int dc = jj >> 2, c = ((jj & 3) << 1) + cv;
+            for (int pj = 0; pj < KS; ++pj) {
+                const int dc = pj >> 2, c = ((pj & 3) << 1) + cv;
                 uint32_t r[4];
-                ptx::ldmatrix_x4_trans(r, vbase + dc * a.box_bytes + tv * kBoxRow +
-                                              ((c ^ ri) << 4));
+                ptx::ldmatrix_x4_trans(r, vbase + dc * dc_bytes + tv * kBoxRow + ((c ^ ri) << 4));
                 if (partial) {
                     r[0] &= mlo;
                     r[1] &= mhi;
                     r[2] &= mlo;
                     r[3] &= mhi;
                 }
-                float d0[4] = {o[2 * jj][0], o[2 * jj][1], 0.f, 0.f};
-                float d1[4] = {o[2 * jj + 1][0], o[2 * jj + 1][1], 0.f, 0.f};
+                float d0[4] = {o[2 * pj][0], o[2 * pj][1], 0.f, 0.f};
+                float d1[4] = {o[2 * pj + 1][0], o[2 * pj + 1][1], 0.f, 0.f};
                 if constexpr (G16) {
-                    d0[2] = ob[2 * jj][0];
-                    d0[3] = ob[2 * jj][1];
-                    d1[2] = ob[2 * jj + 1][0];
-                    d1[3] = ob[2 * jj + 1][1];
+                    d0[2] = ob[2 * pj][0];
+                    d0[3] = ob[2 * pj][1];
+                    d1[2] = ob[2 * pj + 1][0];
+                    d1[3] = ob[2 * pj + 1][1];
                 }
                 ptx::mma_bf16(d0, pa0, pa1, pa2, pa3, r[0], r[1]);
                 ptx::mma_bf16(d1, pa0, pa1, pa2, pa3, r[2], r[3]);
-                o[2 * jj][0] = d0[0];
-                o[2 * jj][1] = d0[1];
-                o[2 * jj + 1][0] = d1[0];
-                o[2 * jj + 1][1] = d1[1];
+                o[2 * pj][0] = d0[0];
+                o[2 * pj][1] = d0[1];
+                o[2 * pj + 1][0] = d1[0];
+                o[2 * pj + 1][1] = d1[1];
                 if constexpr (G16) {
-                    ob[2 * jj][0] = d0[2];
-                    ob[2 * jj][1] = d0[3];
-                    ob[2 * jj + 1][0] = d1[2];
-                    ob[2 * jj + 1][1] = d1[3];
+                    ob[2 * pj][0] = d0[2];
+                    ob[2 * pj][1] = d0[3];
+                    ob[2 * pj + 1][0] = d1[2];
+                    ob[2 * pj + 1][1] = d1[3];
                 }
             }
+        }
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&empty[stage]);
@@ -454,7 +505,7 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
                     }
                 }
             } else {
-                const int64_t slot = ((int64_t)mt.b * a.S + mt.c) * a.n_sub + j;
+                const int64_t slot = ((int64_t)mt.b * a.S + mt.c) * a.wph + jw;
                 if (g < a.G) {
                     const int64_t r = slot * a.Hq + row;
                     float2 *dst = reinterpret_cast<float2 *>(a.ws_acc + r * D + 2 * tig);
@@ -482,7 +533,332 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
     }
 }
 
-template <int D, bool G16>
+// ---------------------------------------------------------------------------
+// INT8 consumer helpers
+// ---------------------------------------------------------------------------
+constexpr uint32_t kFlip = 0x80808080u;   // flips each byte's sign bit: byte = code + 128
+constexpr uint32_t kBias = 0x64646464u;   // fp16 exponent byte of 1024
+constexpr uint32_t kOnes = 0x3c003c00u;   // fp16x2 (1, 1)
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// Two bytes of xf (= codes with the sign bit flipped), chosen by sel (0x4140:
+// bytes 0,1; 0x4342: bytes 2,3), placed in the low mantissa bits of two fp16
+// with exponent 2^10: the values 1024 + code + 128 exactly (10 mantissa bits).
+__device__ __forceinline__ uint32_t biased_f16x2(uint32_t xf, uint32_t sel) {
+    return prmt(xf, kBias, sel);
+}
+
+// The same pair with the bias removed: the exact codes as fp16x2.
+__device__ __forceinline__ uint32_t codes_f16x2(uint32_t xf, uint32_t sel) {
+    uint32_t r = biased_f16x2(xf, sel);
+    asm("sub.rn.f16x2 %0, %0, %1;" : "+r"(r) : "r"(0x64806480u));  // 1152 = 1024 + 128
+    return r;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+// 8 bf16 (one uint4) -> 4 fp16x2
+__device__ __forceinline__ void bf16x8_to_f16x2(const uint4 &v, uint32_t *o) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = ptx::pack_f16(bf16_lo(w[i]), bf16_hi(w[i]));
+}
+
+// Query fragments of the INT8 consumer (fp16): for k-step kk, thread (g, tig)
+// uses dims 16*(tig + 4*(kk/4)) + 4*(kk%4) + 0..3 (see consumer_i8).
+template <bool G16>
+__device__ __forceinline__ void load_q_i8(const Args &a, int b, int row, int g, int tig,
+                                          uint32_t (&qa)[8][2]) {
+    constexpr int D = 128;
+    const uint4 *qr = reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * a.Hq + row) * D);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t f[8];
+        if (g < a.G) {
+            const int c = tig + 4 * half;  // 16 dims = two uint4 of bf16
+            bf16x8_to_f16x2(__ldg(qr + 2 * c), f);
+            bf16x8_to_f16x2(__ldg(qr + 2 * c + 1), f + 4);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = 0u;
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            qa[4 * half + w][0] = f[2 * w];
+            qa[4 * half + w][1] = f[2 * w + 1];
+        }
+    }
+}
+
+// Final write of one query row of the INT8 consumer: this thread holds dims
+// 32*tig + nt (accumulator column 2*tig) and 32*tig + 16 + nt (2*tig + 1); the
+// accumulators still carry the +1152 bias of V, removed here with lb = the
+// same weights summed by the tensor core (sum_t p_t v-scale_t).
+__device__ __forceinline__ void store_i8_row(const Args &a, const StageMeta &mt,
+                                             const float (&oo)[16][2], float bias_sum,
+                                             float lsum, float mm, int row, int tig, int jw) {
+    constexpr int D = 128;
+    const float corr = 1152.f * bias_sum;
+    if (mt.flags & kDirect) {
+        const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+        uint4 *dst = reinterpret_cast<uint4 *>(a.out + ((int64_t)mt.b * a.Hq + row) * D + 32 * tig);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                pk[i] = ptx::pack_bf16((oo[2 * i][c] - corr) * inv, (oo[2 * i + 1][c] - corr) * inv);
+            dst[2 * c] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[2 * c + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+    } else {
+        const int64_t slot = ((int64_t)mt.b * a.S + mt.c) * a.wph + jw;
+        const int64_t r = slot * a.Hq + row;
+        float4 *dst = reinterpret_cast<float4 *>(a.ws_acc + r * D + 32 * tig);
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                dst[4 * c + i] = make_float4(oo[4 * i][c] - corr, oo[4 * i + 1][c] - corr,
+                                             oo[4 * i + 2][c] - corr, oo[4 * i + 3][c] - corr);
+        if (tig == 0) *reinterpret_cast<float2 *>(a.ws_ml + r * 2) = make_float2(mm, lsum);
+    }
+}
+
+// INT8 consumer (d = 128).  Same pipeline and softmax as the bf16 consumer; the
+// tiles hold int8 codes, [head][token][128 bytes], 128-byte swizzled.
+//  QK^T: the dot product over d is order-free, so thread (g, tig) takes, for
+//   k-step kk, the 4 dims 16*(tig + 4*(kk/4)) + 4*(kk%4) + 0..3 of its token row
+//   (one 32-bit word of int8 codes) as its b0/b1 pair, and its query fragment
+//   uses the same dims.  Rows of odd g load their two 16-byte chunks in the
+//   other order (then swap), which keeps the shared-memory reads conflict-free.
+//  PV: n-tile nt, column g stands for dim 16*g + nt, so a thread reads 16 dims
+//   (one 16-byte chunk) of each of its four token rows and byte-transposes
+//   token pairs with prmt into (token, token+1) fp16 pairs, left biased by
+//   +1152; one more MMA against an all-ones B sums the same fp16 weights, and
+//   1152 times that sum is subtracted at the end.  Output column 2*tig (+1) of
+//   n-tile nt is dim 32*tig + nt (+16).
+//  The K scale multiplies the logit, the V scale the softmax weight.
+template <bool G16>
+__device__ __forceinline__ void consumer_i8(const Args &a, uint8_t *stages, StageMeta *meta,
+                                            uint64_t *full, uint64_t *empty) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = warp % a.Hkv, jw = warp / a.Hkv;
+    const int g = lane >> 2, tig = lane & 3;
+    const int odd = g & 1;
+    const uint32_t stage0 = ptx::smem_u32(stages);
+    const uint32_t head_off = (uint32_t)(h * kTile * kBoxRow);
+    const uint32_t sub_bytes = (uint32_t)a.box_bytes;           // one box per sub-tile (d = 128)
+    const uint32_t sc_sub = (uint32_t)(kTile * a.Hkv * 4);      // scale rows of one sub-tile
+
+    uint32_t qa[8][2];
+    uint32_t qb[G16 ? 8 : 1][2];
+    float o[16][2];
+    float ob[G16 ? 16 : 1][2];
+    float ol[4];  // sums of the fp16 weights (all-ones column), rows g and g + 8
+    float m = -INFINITY, l = 0.f, mb = -INFINITY, lb = 0.f;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (;;) {
+        if (!ptx::mbar_wait(&full[stage], phase)) {
+            if (lane == 0) raise_flag(a.err, PA_DEV_TIMEOUT);
+            break;
+        }
+        const StageMeta mt = meta[stage];
+        if (mt.flags & kEnd) break;
+        const uint32_t sb = stage0 + (uint32_t)stage * a.stage_bytes;
+        if (mt.flags & kFirst) {
+            load_q_i8<G16>(a, mt.b, h * a.G + g, g, tig, qa);
+            if constexpr (G16) load_q_i8<G16>(a, mt.b, h * a.G + g + 8, g + 8, tig, qb);
+            m = -INFINITY;
+            l = 0.f;
+            mb = -INFINITY;
+            lb = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ol[i] = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) {
+                o[nt][0] = o[nt][1] = 0.f;
+                if constexpr (G16) ob[nt][0] = ob[nt][1] = 0.f;
+            }
+        }
+        for (int k = 0; k < a.tpw; ++k) {
+        const int jj = jw + a.wph * k;  // this warp's k-th sub-tile of the stage
+        const int tj = mt.ts + kTile * jj;
+        const int nv = max(0, min(kTile, mt.te - tj));
+        if (nv > 0 && !((mt.bad >> jj) & 1)) {
+            const uint32_t kbase = sb + jj * sub_bytes + head_off;
+            const uint32_t vbase = sb + a.v_off + jj * sub_bytes + head_off;
+            const uint32_t ksb = sb + a.ks_off + jj * sc_sub + h * 4;
+            const uint32_t vsb = sb + a.vs_off + jj * sc_sub + h * 4;
+            // ---- S = Q K^T (exact fp16 codes)
+            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+            float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int t = 8 * nt + g;  // swizzle phase of row t is g
+                const uint32_t rb = kbase + t * kBoxRow;
+                const uint4 x0 = lds128(rb + (((tig + 4 * odd) ^ g) << 4));
+                const uint4 x1 = lds128(rb + (((tig + 4 * (1 - odd)) ^ g) << 4));
+                const uint4 lo = odd ? x1 : x0;  // dims 16*tig ..
+                const uint4 hi = odd ? x0 : x1;  // dims 16*(tig+4) ..
+                const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t xf = wd[kk] ^ kFlip;
+                    const uint32_t b0 = codes_f16x2(xf, 0x4140u);
+                    const uint32_t b1 = codes_f16x2(xf, 0x4342u);
+                    float(&acc)[4] = nt == 0 ? ((kk & 1) ? e0 : s0) : ((kk & 1) ? e1 : s1);
+                    if constexpr (G16)
+                        ptx::mma_f16(acc, qa[kk][0], qb[kk][0], qa[kk][1], qb[kk][1], b0, b1);
+                    else
+                        ptx::mma_f16(acc, qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                s0[i] += e0[i];
+                s1[i] += e1[i];
+            }
+            // ---- online softmax; K scale folded into the logit
+            const int t_a = 2 * tig, t_b = 8 + 2 * tig;
+            const bool va0 = t_a < nv, va1 = t_a + 1 < nv, vb0 = t_b < nv, vb1 = t_b + 1 < nv;
+            const float sl = a.scale_log2;
+            const int hs = a.Hkv * 4;
+            const float k0 = lds_f32(ksb + t_a * hs) * sl, k1 = lds_f32(ksb + (t_a + 1) * hs) * sl;
+            const float k2 = lds_f32(ksb + t_b * hs) * sl, k3 = lds_f32(ksb + (t_b + 1) * hs) * sl;
+            const float v0 = lds_f32(vsb + t_a * hs), v1 = lds_f32(vsb + (t_a + 1) * hs);
+            const float v2 = lds_f32(vsb + t_b * hs), v3 = lds_f32(vsb + (t_b + 1) * hs);
+            float x0 = va0 ? s0[0] * k0 : -INFINITY, x1 = va1 ? s0[1] * k1 : -INFINITY;
+            float x2 = vb0 ? s1[0] * k2 : -INFINITY, x3 = vb1 ? s1[1] * k3 : -INFINITY;
+            float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+            const float mn = fmaxf(m, mx);
+            const float mu = mn == -INFINITY ? 0.f : mn;
+            const float alpha = exp2f(m - mu);
+            const float p0 = exp2f(x0 - mu), p1 = exp2f(x1 - mu);
+            const float p2 = exp2f(x2 - mu), p3 = exp2f(x3 - mu);
+            l = l * alpha + ((p0 + p1) + (p2 + p3));
+            m = mn;
+            const uint32_t pa0 = ptx::pack_f16(va0 ? p0 * v0 : 0.f, va1 ? p1 * v1 : 0.f);
+            const uint32_t pa2 = ptx::pack_f16(vb0 ? p2 * v2 : 0.f, vb1 ? p3 * v3 : 0.f);
+            uint32_t pa1 = 0u, pa3 = 0u;
+            float alphab = 1.f;
+            if constexpr (G16) {
+                float y0 = va0 ? s0[2] * k0 : -INFINITY, y1 = va1 ? s0[3] * k1 : -INFINITY;
+                float y2 = vb0 ? s1[2] * k2 : -INFINITY, y3 = vb1 ? s1[3] * k3 : -INFINITY;
+                float my = fmaxf(fmaxf(y0, y1), fmaxf(y2, y3));
+                my = fmaxf(my, __shfl_xor_sync(kFull, my, 1));
+                my = fmaxf(my, __shfl_xor_sync(kFull, my, 2));
+                const float mnb = fmaxf(mb, my);
+                const float mub = mnb == -INFINITY ? 0.f : mnb;
+                alphab = exp2f(mb - mub);
+                const float q0 = exp2f(y0 - mub), q1 = exp2f(y1 - mub);
+                const float q2 = exp2f(y2 - mub), q3 = exp2f(y3 - mub);
+                lb = lb * alphab + ((q0 + q1) + (q2 + q3));
+                mb = mnb;
+                pa1 = ptx::pack_f16(va0 ? q0 * v0 : 0.f, va1 ? q1 * v1 : 0.f);
+                pa3 = ptx::pack_f16(vb0 ? q2 * v2 : 0.f, vb1 ? q3 * v3 : 0.f);
+            }
+            if (__any_sync(kFull, alpha != 1.f || alphab != 1.f)) {
+                ol[0] *= alpha;
+                ol[1] *= alpha;
+                ol[2] *= alphab;
+                ol[3] *= alphab;
+#pragma unroll
+                for (int nt = 0; nt < 16; ++nt) {
+                    o[nt][0] *= alpha;
+                    o[nt][1] *= alpha;
+                    if constexpr (G16) {
+                        ob[nt][0] *= alphab;
+                        ob[nt][1] *= alphab;
+                    }
+                }
+            }
+            // ---- O += P (V + 1152); column g of n-tile nt is dim 16*g + nt
+            const uint4 ra = lds128(vbase + t_a * kBoxRow + ((g ^ (t_a & 7)) << 4));
+            const uint4 rb = lds128(vbase + (t_a + 1) * kBoxRow + ((g ^ ((t_a + 1) & 7)) << 4));
+            const uint4 rc = lds128(vbase + t_b * kBoxRow + ((g ^ (t_b & 7)) << 4));
+            const uint4 rd = lds128(vbase + (t_b + 1) * kBoxRow + ((g ^ ((t_b + 1) & 7)) << 4));
+            const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w}, wb[4] = {rb.x, rb.y, rb.z, rb.w};
+            const uint32_t wc[4] = {rc.x, rc.y, rc.z, rc.w}, wd[4] = {rd.x, rd.y, rd.z, rd.w};
+            {
+                float dd[4] = {ol[0], ol[1], ol[2], ol[3]};
+                ptx::mma_f16(dd, pa0, pa1, pa2, pa3, kOnes, kOnes);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) ol[i] = dd[i];
+            }
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const uint32_t fa = wa[w] ^ kFlip, fb = wb[w] ^ kFlip;
+                const uint32_t fc = wc[w] ^ kFlip, fd = wd[w] ^ kFlip;
+                const uint32_t X = prmt(fa, fb, 0x5140u), Y = prmt(fa, fb, 0x7362u);
+                const uint32_t Z = prmt(fc, fd, 0x5140u), U = prmt(fc, fd, 0x7362u);
+                const uint32_t b0[4] = {biased_f16x2(X, 0x4140u), biased_f16x2(X, 0x4342u),
+                                        biased_f16x2(Y, 0x4140u), biased_f16x2(Y, 0x4342u)};
+                const uint32_t b1[4] = {biased_f16x2(Z, 0x4140u), biased_f16x2(Z, 0x4342u),
+                                        biased_f16x2(U, 0x4140u), biased_f16x2(U, 0x4342u)};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int nt = 4 * w + i;
+                    float dd[4] = {o[nt][0], o[nt][1], 0.f, 0.f};
+                    if constexpr (G16) {
+                        dd[2] = ob[nt][0];
+                        dd[3] = ob[nt][1];
+                    }
+                    ptx::mma_f16(dd, pa0, pa1, pa2, pa3, b0[i], b1[i]);
+                    o[nt][0] = dd[0];
+                    o[nt][1] = dd[1];
+                    if constexpr (G16) {
+                        ob[nt][0] = dd[2];
+                        ob[nt][1] = dd[3];
+                    }
+                }
+            }
+        }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&empty[stage]);
+        if (mt.flags & kLast) {
+            float lt = l + __shfl_xor_sync(kFull, l, 1);
+            lt += __shfl_xor_sync(kFull, lt, 2);
+            float ltb = 0.f;
+            if constexpr (G16) {
+                ltb = lb + __shfl_xor_sync(kFull, lb, 1);
+                ltb += __shfl_xor_sync(kFull, ltb, 2);
+            }
+            const int row = h * a.G + g;
+            if (g < a.G) store_i8_row(a, mt, o, ol[0], lt, m, row, tig, jw);
+            if constexpr (G16) {
+                if (g + 8 < a.G) store_i8_row(a, mt, ob, ol[2], ltb, mb, row + 8, tig, jw);
+            }
+        }
+        if (++stage == a.nstage) {
+            stage = 0;
+            phase ^= 1u;
+        }
+    }
+}
+
+template <int D, bool G16, bool I8>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const Args a) {
@@ -502,7 +878,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     if ((threadIdx.x >> 5) == kConsumerWarps)
-        producer<D>(&kmap, &vmap, a, stages, meta, full, empty);
+        producer<D, I8>(&kmap, &vmap, a, stages, meta, full, empty);
+    else if constexpr (I8)
+        consumer_i8<G16>(a, stages, meta, full, empty);
     else
         consumer<D, G16>(a, stages, meta, full, empty);
 }
@@ -514,9 +892,9 @@ __global__ void __launch_bounds__(D) merge_tc_kernel(const Args a) {
     const int b = (int)(bh / a.Hq), i = (int)(bh % a.Hq);
     const int e = threadIdx.x;
     const int nsb = a.ns[b];
-    if (nsb == 1 && a.n_sub == 1) return;  // written directly by the decode kernel
-    const int cnt = nsb * a.n_sub;
-    const int64_t base = (int64_t)b * a.S * a.n_sub;
+    if (nsb == 1 && a.wph == 1) return;  // written directly by the decode kernel
+    const int cnt = nsb * a.wph;
+    const int64_t base = (int64_t)b * a.S * a.wph;
     float M = -INFINITY;
     for (int s = 0; s < cnt; ++s) M = fmaxf(M, a.ws_ml[((base + s) * a.Hq + i) * 2]);
     float L = 0.f, A = 0.f;
@@ -547,29 +925,43 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// Pool viewed as 5-D (innermost first): 64 elements of d | slot in block |
-// kv head | 64-element slice of d | physical block.  Box (64, 16, Hkv, 1, 1):
-// in shared memory [head][token][64 elements], 128-byte swizzled.
+// Element width (bytes) the tensor maps use to move pool rows.  A TMA copy
+// does not interpret the data, so bf16 and int8 pools are both moved as this
+// many-byte elements; the box is 128 bytes of d either way.
+constexpr int kTmaElt = 2;
+
+// The pool is viewed as 5-D (innermost first):
+//   128 bytes of one (token, head) vector | slot in block | kv head |
+//   128-byte slice of the vector | physical block,
+// and one TMA box is (128 bytes, 16 tokens, Hkv heads, 1, 1): in shared memory
+// [head][token][128 bytes], 128-byte swizzled, so each head's 16 token rows are
+// 16 consecutive swizzled rows that ldmatrix / 16-byte loads read without bank
+// conflicts.
 bool encode_pool_map(CUtensorMap *map, const void *base, int64_t N, int bs, int Hkv, int d,
-                     int64_t block_stride) {
+                     int64_t block_stride, bool int8) {
     auto fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[5] = {64, (cuuint64_t)bs, (cuuint64_t)Hkv, (cuuint64_t)(d / 64),
-                                (cuuint64_t)N};
-    const cuuint64_t strides[4] = {(cuuint64_t)Hkv * d * 2, (cuuint64_t)d * 2, 128,
-                                   (cuuint64_t)block_stride * 2};
-    const cuuint32_t box[5] = {64, (cuuint32_t)kTile, (cuuint32_t)Hkv, 1, 1};
+    const int64_t row = (int64_t)d * (int8 ? 1 : 2);  // bytes of one (token, head) vector
+    const int inner = 128 / kTmaElt;                    // elements in one 128-byte box row
+    const cuuint64_t dims[5] = {(cuuint64_t)inner, (cuuint64_t)bs, (cuuint64_t)Hkv,
+                                (cuuint64_t)(row / 128), (cuuint64_t)N};
+    const cuuint64_t strides[4] = {(cuuint64_t)(Hkv * row), (cuuint64_t)row, 128,
+                                   (cuuint64_t)(block_stride * (int8 ? 1 : 2))};
+    const cuuint32_t box[5] = {(cuuint32_t)inner, (cuuint32_t)kTile, (cuuint32_t)Hkv, 1, 1};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims,
-                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    const CUtensorMapDataType dt = kTmaElt == 4   ? CU_TENSOR_MAP_DATA_TYPE_UINT32
+                                   : kTmaElt == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16
+                                                  : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    CUresult r = fn(map, dt, 5, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-template <int D, bool G16>
+template <int D, bool G16, bool I8>
 cudaError_t launch_typed(const CUtensorMap &km, const CUtensorMap &vm, const Args &a, int grid,
                          int smem, cudaStream_t st) {
-    auto kfn = decode_tc_kernel<D, G16>;
+    auto kfn = decode_tc_kernel<D, G16, I8>;
     static unsigned long long attr_set = 0;  // one bit per device; benign race (idempotent)
     int dev = 0;
     cudaGetDevice(&dev);
@@ -585,12 +977,12 @@ cudaError_t launch_typed(const CUtensorMap &km, const CUtensorMap &vm, const Arg
 
 }  // namespace tc
 
-cudaError_t launch_decode_tc(const DecodeArgs &d, cudaStream_t st) {
+cudaError_t launch_decode_tc(const DecodeArgs &d, bool int8, cudaStream_t st) {
     using namespace tc;
     const DecodePlan &p = d.plan;
     CUtensorMap km, vm;
-    if (!encode_pool_map(&km, d.k_cache, d.N, d.bs, d.Hkv, d.d, d.block_stride) ||
-        !encode_pool_map(&vm, d.v_cache, d.N, d.bs, d.Hkv, d.d, d.block_stride))
+    if (!encode_pool_map(&km, d.k_cache, d.N, d.bs, d.Hkv, d.d, d.block_stride, int8) ||
+        !encode_pool_map(&vm, d.v_cache, d.N, d.bs, d.Hkv, d.d, d.block_stride, int8))
         return cudaErrorInvalidValue;
     char *ws = static_cast<char *>(d.ws);
     Args a;
@@ -604,6 +996,10 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, cudaStream_t st) {
     a.units = reinterpret_cast<const int4 *>(ws + p.off_units);
     a.ws_ml = reinterpret_cast<float *>(ws + p.off_ml);
     a.ws_acc = reinterpret_cast<float *>(ws + p.off_acc);
+    a.k_scale = d.k_scale;
+    a.v_scale = d.v_scale;
+    a.ks_off = p.ks_off;
+    a.vs_off = p.vs_off;
     a.N = d.N;
     a.B = d.B;
     a.Hq = d.Hq;
@@ -612,12 +1008,17 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, cudaStream_t st) {
     a.bs = d.bs;
     a.MB = d.MB;
     a.S = p.S;
-    a.n_sub = p.n_sub;
     a.nstage = p.nstage;
     a.stage_bytes = p.stage_bytes;
-    a.q_off = p.q_off;
     a.v_off = p.v_off;
     a.box_bytes = d.Hkv * kTile * kBoxRow;
+    a.wph = p.wph;
+    a.tpw = p.tpw;
+    a.n_sub = p.n_sub;
+    {
+        const int tpb = d.bs / kTile;
+        a.tpb_shift = (tpb & (tpb - 1)) == 0 ? __builtin_ctz((unsigned)tpb) : -1;
+    }
     a.scale_log2 = d.scale_log2;
     const int max_ctx = d.MB * d.bs;
     plan_kernel<<<1, 1024, 0, st>>>(d.ctx_lens, d.err, a.hdr, const_cast<int32_t *>(a.ns),
@@ -626,14 +1027,17 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, cudaStream_t st) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const bool g16 = d.G > 8;
-    if (d.d == 128)
-        e = g16 ? launch_typed<128, true>(km, vm, a, p.grid, p.smem_bytes, st)
-                : launch_typed<128, false>(km, vm, a, p.grid, p.smem_bytes, st);
+    if (int8)  // d == 128 only (the plan guarantees it)
+        e = g16 ? launch_typed<128, true, true>(km, vm, a, p.grid, p.smem_bytes, st)
+                : launch_typed<128, false, true>(km, vm, a, p.grid, p.smem_bytes, st);
+    else if (d.d == 128)
+        e = g16 ? launch_typed<128, true, false>(km, vm, a, p.grid, p.smem_bytes, st)
+                : launch_typed<128, false, false>(km, vm, a, p.grid, p.smem_bytes, st);
     else
-        e = g16 ? launch_typed<64, true>(km, vm, a, p.grid, p.smem_bytes, st)
-                : launch_typed<64, false>(km, vm, a, p.grid, p.smem_bytes, st);
+        e = g16 ? launch_typed<64, true, false>(km, vm, a, p.grid, p.smem_bytes, st)
+                : launch_typed<64, false, false>(km, vm, a, p.grid, p.smem_bytes, st);
     if (e != cudaSuccess) return e;
-    if (p.S > 1 || p.n_sub > 1) {
+    if (p.S > 1 || p.wph > 1) {
         const unsigned rows = (unsigned)((int64_t)d.B * d.Hq);
         if (d.d == 128) merge_tc_kernel<128><<<rows, 128, 0, st>>>(a);
         else merge_tc_kernel<64><<<rows, 64, 0, st>>>(a);

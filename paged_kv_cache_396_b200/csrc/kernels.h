@@ -31,8 +31,10 @@ struct DecodePlan {
     int kernel;         // 0: general-shape kernel, 1: staged tensor-core kernel
     int S;              // partition slots per sequence
     int chunk;          // general: tokens per partition; staged: minimum tokens per partition
-    int n_sub;          // staged: 16-token sub-tiles per stage (8 / Hkv)
-    int nstage, stage_bytes, q_off, v_off, smem_bytes, grid, units_per_cta;
+    int wph;            // staged: consumer warps per kv head (8 / Hkv) = partial slots per unit
+    int tpw;            // staged: 16-token sub-tiles per consumer warp per stage
+    int n_sub;          // staged: 16-token sub-tiles per stage (wph * tpw)
+    int nstage, stage_bytes, v_off, ks_off, vs_off, smem_bytes, grid, units_per_cta;
     size_t off_hdr, off_ns, off_units, off_ml, off_acc, ws_total;
 };
 
@@ -82,7 +84,7 @@ cudaError_t launch_append_int8(const uint16_t *k_new, const uint16_t *v_new, int
 // else the general-shape kernel; then the partition merge when S > 1.
 cudaError_t launch_decode(const DecodeArgs &a, bool int8, cudaStream_t stream);
 cudaError_t launch_decode_simple(const DecodeArgs &a, bool int8, cudaStream_t stream);
-cudaError_t launch_decode_tc(const DecodeArgs &a, cudaStream_t stream);
+cudaError_t launch_decode_tc(const DecodeArgs &a, bool int8, cudaStream_t stream);
 DecodePlan make_decode_plan(int B, int Hq, int Hkv, int d, int bs, int MB, int num_splits,
                             bool int8, int sms);
 cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t stream);

@@ -197,8 +197,12 @@ size_t pa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int bs, int max_
     const int sms = device_sms();
     if (sms < 0) return 0;
     if (Hq < Hkv || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
-    return pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits, false, sms)
-        .ws_total;
+    // one size serves pa_decode and pa_decode_int8 alike
+    const size_t a = pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits,
+                                           false, sms).ws_total;
+    const size_t b = pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits,
+                                           true, sms).ws_total;
+    return a > b ? a : b;
 }
 
 int pa_decode_plan(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq, int num_splits,
@@ -214,7 +218,7 @@ int pa_decode_plan(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq
     *num_splits_out = p.S;
     *chunk_tokens_out = p.chunk;
     if (launches_out)
-        *launches_out = p.kernel == 1 ? 2 + ((p.S > 1 || p.n_sub > 1) ? 1 : 0) : 1 + (p.S > 1 ? 1 : 0);
+        *launches_out = p.kernel == 1 ? 2 + ((p.S > 1 || p.wph > 1) ? 1 : 0) : 1 + (p.S > 1 ? 1 : 0);
     return PA_OK;
 }
 

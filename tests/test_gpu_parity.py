@@ -32,6 +32,10 @@ MEDIUM = {
                      old_len_range=(1, 700), outlier_frac=0.0),
     # G = 16 on the staged kernel, d = 64
     "g16": W.scaled(C["c2"], key="g16", layers=1, batch=3, hq=64, hkv=4, old_lens=(500, 33, 64)),
+    # INT8 on the staged kernel with G = 16 and two 16-token sub-tiles per stage (Hkv = 4)
+    "i8g16": W.scaled(C["c5"], key="i8g16", batch=3, hq=64, hkv=4, old_lens=(100, 37, 300)),
+    # INT8 with d = 64: the general-shape kernel
+    "i8d64": W.scaled(C["c5"], key="i8d64", batch=3, head_dim=64, old_lens=(70, 5, 200)),
 }
 
 
@@ -90,8 +94,10 @@ def test_medium_workloads(key):
 
 
 @pytest.mark.parametrize("num_splits", [1, 2, 3, 8, 0])
-def test_split_count_invariance(num_splits):
-    cfg = W.scaled(C["c3"], key="split", layers=1, batch=3, old_lens=(2000, 700, 45))
+@pytest.mark.parametrize("kv", ["bf16", "int8"])
+def test_split_count_invariance(num_splits, kv):
+    base = C["c3"] if kv == "bf16" else C["c5"]
+    cfg = W.scaled(base, key="split", layers=1, batch=3, old_lens=(2000, 700, 45))
     wl = W.generate(cfg, "cpu")
     _parity(wl, [0], num_splits=num_splits)
 
