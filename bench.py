@@ -62,6 +62,23 @@ def parse():
 
 
 # ----------------------------------------------------------------------------- helpers
+def reduce_max(x: float, world: int) -> float:
+    """Max of x over all ranks (device times are reported as the slowest rank's)."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, batch: int, ms_per_step: float) -> float:
+    """Whole-job decode throughput: every rank decodes its own batch of sequences
+    (weak scaling), so the job emits world * batch tokens per (slowest) step."""
+    return world * batch / (ms_per_step / 1000.0)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -164,10 +181,10 @@ def decode_algorithmic_bytes(cfg, ctx_lens, partial_slots, n_units=0):
 class Runner:
     """Device state and one decode step of a workload through the binding."""
 
-    def __init__(self, cfg, device, num_splits=0):
+    def __init__(self, cfg, device, num_splits=0, wl=None):
         from paged_kv_cache_396_b200 import pagedkv as pk
         self.pk, self.cfg, self.dev = pk, cfg, device
-        wl = W.generate(cfg, device)
+        wl = W.generate(cfg, device) if wl is None else wl
         self.wl = wl
         self.L = cfg.layers
         self.bt = torch.as_tensor(wl.block_tables, device=device)
@@ -441,12 +458,9 @@ def main():
     else:
         samples = ev_eager
     decode_ms = [a.elapsed_time(b) for a, b in samples]
-    if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(total_ms, world)
     ms_per_step = total_ms / args.steps
-    value = world * cfg.batch / (ms_per_step / 1000.0)
+    value = job_tokens_per_s(world, cfg.batch, ms_per_step)
     dec_avg_s = statistics.mean(decode_ms) / 1000.0
     achieved = r.decode_bytes / dec_avg_s / 1e9
     peak, peak_kind = peaks()
@@ -495,11 +509,8 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": world * B / (e2e_ms / 1000.0), "unit": "tokens/s",
+    e2e_ms = reduce_max(e2e_ms, world)
+    e2e = {"value": job_tokens_per_s(world, B, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
     if r.err.item() != 0:
         raise SystemExit(f"device error flag {r.err.item()} during timing")

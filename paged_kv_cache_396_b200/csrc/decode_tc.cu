@@ -962,14 +962,16 @@ template <int D, bool G16, bool I8>
 cudaError_t launch_typed(const CUtensorMap &km, const CUtensorMap &vm, const Args &a, int grid,
                          int smem, cudaStream_t st) {
     auto kfn = decode_tc_kernel<D, G16, I8>;
-    static unsigned long long attr_set = 0;  // one bit per device; benign race (idempotent)
+    // raise the dynamic shared-memory limit to what this launch needs (per device,
+    // only upwards; static shared memory counts against the same per-block budget)
+    static int smem_set[64] = {0};  // benign race: idempotent
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 64 || !((attr_set >> dev) & 1ull)) {
-        cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             227 * 1024);
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    if (dev >= 64 || smem_set[dev] < smem) {
+        cudaError_t e =
+            cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        if (dev < 64) attr_set |= 1ull << dev;
+        if (dev < 64) smem_set[dev] = smem;
     }
     kfn<<<grid, kThreads, smem, st>>>(km, vm, a);
     return cudaGetLastError();
