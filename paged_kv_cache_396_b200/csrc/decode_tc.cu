@@ -40,6 +40,8 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <utility>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -94,6 +96,10 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *ctx_lens, int
     __shared__ int hist[1024];
     __shared__ int s_chunk;
     const int tid = threadIdx.x;
+    // launched programmatically after the previous kernel (e.g. the KV append):
+    // let the decode kernel's CTAs get resident, then wait for the predecessor
+    ptx::grid_launch_dependents();
+    ptx::grid_dependency_wait();
     long long tot = 0;
     for (int b = tid; b < B; b += blockDim.x) {
         int len = ctx_lens[b];
@@ -877,6 +883,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::fence_mbar_init();
     }
     __syncthreads();
+    // launched programmatically after the plan kernel: the set-up above overlaps
+    // it; the plan (and, through it, the KV append before it) is complete here
+    ptx::grid_launch_dependents();
+    ptx::grid_dependency_wait();
     if ((threadIdx.x >> 5) == kConsumerWarps)
         producer<D, I8>(&kmap, &vmap, a, stages, meta, full, empty);
     else if constexpr (I8)
@@ -888,6 +898,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Merge of the partials of one (sequence, query head) in slot order.
 template <int D>
 __global__ void __launch_bounds__(D) merge_tc_kernel(const Args a) {
+    ptx::grid_dependency_wait();  // the decode kernel's partials are complete
     const int64_t bh = blockIdx.x;
     const int b = (int)(bh / a.Hq), i = (int)(bh % a.Hq);
     const int e = threadIdx.x;
@@ -912,6 +923,25 @@ __global__ void __launch_bounds__(D) merge_tc_kernel(const Args a) {
 // ---------------------------------------------------------------------------
 // host
 // ---------------------------------------------------------------------------
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous kernel in the stream is still running; it calls griddepcontrol.wait
+// before it touches anything the previous kernel produced.
+template <typename... KArgs, typename... Args2>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args2 &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args2>(args)...);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -973,8 +1003,7 @@ cudaError_t launch_typed(const CUtensorMap &km, const CUtensorMap &vm, const Arg
         if (e != cudaSuccess) return e;
         if (dev < 64) smem_set[dev] = smem;
     }
-    kfn<<<grid, kThreads, smem, st>>>(km, vm, a);
-    return cudaGetLastError();
+    return launch_pdl(kfn, dim3(grid), dim3(kThreads), smem, st, km, vm, a);
 }
 
 }  // namespace tc
@@ -1023,10 +1052,9 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, bool int8, cudaStream_t st) {
     }
     a.scale_log2 = d.scale_log2;
     const int max_ctx = d.MB * d.bs;
-    plan_kernel<<<1, 1024, 0, st>>>(d.ctx_lens, d.err, a.hdr, const_cast<int32_t *>(a.ns),
-                                    const_cast<int4 *>(a.units), d.B, max_ctx, p.chunk,
-                                    p.grid * p.units_per_cta);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, d.ctx_lens, d.err, a.hdr,
+                               const_cast<int32_t *>(a.ns), const_cast<int4 *>(a.units), d.B,
+                               max_ctx, p.chunk, p.grid * p.units_per_cta);
     if (e != cudaSuccess) return e;
     const bool g16 = d.G > 8;
     if (int8)  // d == 128 only (the plan guarantees it)
@@ -1041,9 +1069,8 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, bool int8, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (p.S > 1 || p.wph > 1) {
         const unsigned rows = (unsigned)((int64_t)d.B * d.Hq);
-        if (d.d == 128) merge_tc_kernel<128><<<rows, 128, 0, st>>>(a);
-        else merge_tc_kernel<64><<<rows, 64, 0, st>>>(a);
-        e = cudaGetLastError();
+        e = d.d == 128 ? launch_pdl(merge_tc_kernel<128>, dim3(rows), dim3(128), 0, st, a)
+                       : launch_pdl(merge_tc_kernel<64>, dim3(rows), dim3(64), 0, st, a);
     }
     return e;
 }
