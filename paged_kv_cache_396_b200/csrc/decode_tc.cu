@@ -587,30 +587,64 @@ __device__ __forceinline__ void bf16x8_to_f16x2(const uint4 &v, uint32_t *o) {
     for (int i = 0; i < 4; ++i) o[i] = ptx::pack_f16(bf16_lo(w[i]), bf16_hi(w[i]));
 }
 
-// Query fragments of the INT8 consumer (fp16): for k-step kk, thread (g, tig)
-// uses dims 16*(tig + 4*(kk/4)) + 4*(kk%4) + 0..3 (see consumer_i8).
-template <bool G16>
-__device__ __forceinline__ void load_q_i8(const Args &a, int b, int row, int g, int tig,
-                                          uint32_t (&qa)[8][2]) {
+// Query fragments of the INT8 consumer as exact int8 pairs for the s8 MMA.
+// Row g of the group is scaled by a power of two 2^e so that max|q| * 2^e <=
+// 16256, rounded to an integer q' (|q'| < 2^14) and split exactly into
+// q' = 128 * hi + lo with hi in [-127, 127], lo in [-64, 63]; then
+// q.k = (128 * (hi.k) + lo.k) / 2^e with both dot products exact in int32.
+// k-step kk (32 dims) of thread (g, tig) uses dims 16*tig + 4*kk + 0..3 (a0/a1)
+// and 16*(tig + 4) + 4*kk + 0..3 (a2/a3), matching the K words it loads.
+// Returns 1 / 2^e (0 for an all-zero or absent row).
+__device__ __forceinline__ float load_q_i8(const Args &a, int b, int row, bool live, int tig,
+                                           uint32_t (&qh)[4][2], uint32_t (&ql)[4][2]) {
     constexpr int D = 128;
-    const uint4 *qr = reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * a.Hq + row) * D);
+    float v[2][16];
+    if (live) {
+        const uint4 *qr = reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * a.Hq + row) * D);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int c = tig + 4 * half;  // 16 dims = two uint4 of bf16
+            const uint4 w0 = __ldg(qr + 2 * c), w1 = __ldg(qr + 2 * c + 1);
+            const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                v[half][2 * i] = bf16_lo(w[i]);
+                v[half][2 * i + 1] = bf16_hi(w[i]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[half][i] = 0.f;
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int half = 0; half < 2; ++half)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(v[half][i]));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));  // the quad holds the whole row
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+    // largest power of two sc with mx * sc <= 16256
+    const float sc = mx > 0.f ? exp2f(floorf(log2f(16256.f / mx))) : 1.f;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-        uint32_t f[8];
-        if (g < a.G) {
-            const int c = tig + 4 * half;  // 16 dims = two uint4 of bf16
-            bf16x8_to_f16x2(__ldg(qr + 2 * c), f);
-            bf16x8_to_f16x2(__ldg(qr + 2 * c + 1), f + 4);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = 0u;
-        }
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            qa[4 * half + w][0] = f[2 * w];
-            qa[4 * half + w][1] = f[2 * w + 1];
+            uint32_t hw = 0u, lw = 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int qi = __float2int_rn(v[half][4 * w + e] * sc);
+                const int hi = (qi + 64) >> 7;
+                const int lo = qi - hi * 128;
+                hw |= (uint32_t)(hi & 0xff) << (8 * e);
+                lw |= (uint32_t)(lo & 0xff) << (8 * e);
+            }
+            qh[w][half] = hw;
+            ql[w][half] = lw;
         }
     }
+    return mx > 0.f ? 1.f / sc : 0.f;
 }
 
 // Final write of one query row of the INT8 consumer: this thread holds dims
@@ -650,11 +684,13 @@ __device__ __forceinline__ void store_i8_row(const Args &a, const StageMeta &mt,
 
 // INT8 consumer (d = 128).  Same pipeline and softmax as the bf16 consumer; the
 // tiles hold int8 codes, [head][token][128 bytes], 128-byte swizzled.
-//  QK^T: the dot product over d is order-free, so thread (g, tig) takes, for
-//   k-step kk, the 4 dims 16*(tig + 4*(kk/4)) + 4*(kk%4) + 0..3 of its token row
-//   (one 32-bit word of int8 codes) as its b0/b1 pair, and its query fragment
-//   uses the same dims.  Rows of odd g load their two 16-byte chunks in the
-//   other order (then swap), which keeps the shared-memory reads conflict-free.
+//  QK^T: int8 x int8 MMAs (m16n8k32) with exact int32 sums.  The dot product
+//   over d is order-free, so thread (g, tig) takes, for k-step kk, the 32-bit
+//   words kk of its two 16-byte chunks (dims 16*tig + 4*kk and 16*(tig+4) +
+//   4*kk, 4 codes each) of its token row as its b0/b1 operands, and the query's
+//   hi/lo int8 parts (load_q_i8) use the same dims.  Rows of odd g load their
+//   two chunks in the other order (then swap), which keeps the shared-memory
+//   reads conflict-free.
 //  PV: n-tile nt, column g stands for dim 16*g + nt, so a thread reads 16 dims
 //   (one 16-byte chunk) of each of its four token rows and byte-transposes
 //   token pairs with prmt into (token, token+1) fp16 pairs, left biased by
@@ -674,8 +710,9 @@ __device__ __forceinline__ void consumer_i8(const Args &a, uint8_t *stages, Stag
     const uint32_t sub_bytes = (uint32_t)a.box_bytes;           // one box per sub-tile (d = 128)
     const uint32_t sc_sub = (uint32_t)(kTile * a.Hkv * 4);      // scale rows of one sub-tile
 
-    uint32_t qa[8][2];
-    uint32_t qb[G16 ? 8 : 1][2];
+    uint32_t qh[4][2], ql[4][2];                          // rows g: hi / lo int8 parts
+    uint32_t qhb[G16 ? 4 : 1][2], qlb[G16 ? 4 : 1][2];    // rows g + 8
+    float qs = 0.f, qsb = 0.f;                            // 1 / 2^e of rows g and g + 8
     float o[16][2];
     float ob[G16 ? 16 : 1][2];
     float ol[4];  // sums of the fp16 weights (all-ones column), rows g and g + 8
@@ -691,8 +728,8 @@ __device__ __forceinline__ void consumer_i8(const Args &a, uint8_t *stages, Stag
         if (mt.flags & kEnd) break;
         const uint32_t sb = stage0 + (uint32_t)stage * a.stage_bytes;
         if (mt.flags & kFirst) {
-            load_q_i8<G16>(a, mt.b, h * a.G + g, g, tig, qa);
-            if constexpr (G16) load_q_i8<G16>(a, mt.b, h * a.G + g + 8, g + 8, tig, qb);
+            qs = load_q_i8(a, mt.b, h * a.G + g, g < a.G, tig, qh, ql);
+            if constexpr (G16) qsb = load_q_i8(a, mt.b, h * a.G + g + 8, g + 8 < a.G, tig, qhb, qlb);
             m = -INFINITY;
             l = 0.f;
             mb = -INFINITY;
@@ -714,9 +751,8 @@ __device__ __forceinline__ void consumer_i8(const Args &a, uint8_t *stages, Stag
             const uint32_t vbase = sb + a.v_off + jj * sub_bytes + head_off;
             const uint32_t ksb = sb + a.ks_off + jj * sc_sub + h * 4;
             const uint32_t vsb = sb + a.vs_off + jj * sc_sub + h * 4;
-            // ---- S = Q K^T (exact fp16 codes)
-            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-            float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
+            // ---- S = Q K^T on int8 tensor cores: K codes straight from shared memory
+            int sh[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, sl8[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 const int t = 8 * nt + g;  // swizzle phase of row t is g
@@ -725,23 +761,25 @@ __device__ __forceinline__ void consumer_i8(const Args &a, uint8_t *stages, Stag
                 const uint4 x1 = lds128(rb + (((tig + 4 * (1 - odd)) ^ g) << 4));
                 const uint4 lo = odd ? x1 : x0;  // dims 16*tig ..
                 const uint4 hi = odd ? x0 : x1;  // dims 16*(tig+4) ..
-                const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+                const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t xf = wd[kk] ^ kFlip;
-                    const uint32_t b0 = codes_f16x2(xf, 0x4140u);
-                    const uint32_t b1 = codes_f16x2(xf, 0x4342u);
-                    float(&acc)[4] = nt == 0 ? ((kk & 1) ? e0 : s0) : ((kk & 1) ? e1 : s1);
-                    if constexpr (G16)
-                        ptx::mma_f16(acc, qa[kk][0], qb[kk][0], qa[kk][1], qb[kk][1], b0, b1);
-                    else
-                        ptx::mma_f16(acc, qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+                for (int kk = 0; kk < 4; ++kk) {
+                    if constexpr (G16) {
+                        ptx::mma_s8(sh[nt], qh[kk][0], qhb[kk][0], qh[kk][1], qhb[kk][1], wl[kk],
+                                    wh[kk]);
+                        ptx::mma_s8(sl8[nt], ql[kk][0], qlb[kk][0], ql[kk][1], qlb[kk][1], wl[kk],
+                                    wh[kk]);
+                    } else {
+                        ptx::mma_s8(sh[nt], qh[kk][0], 0u, qh[kk][1], 0u, wl[kk], wh[kk]);
+                        ptx::mma_s8(sl8[nt], ql[kk][0], 0u, ql[kk][1], 0u, wl[kk], wh[kk]);
+                    }
                 }
             }
+            float s0[4], s1[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                s0[i] += e0[i];
-                s1[i] += e1[i];
+                s0[i] = (float)(sh[0][i] * 128 + sl8[0][i]) * (i < 2 ? qs : qsb);
+                s1[i] = (float)(sh[1][i] * 128 + sl8[1][i]) * (i < 2 ? qs : qsb);
             }
             // ---- online softmax; K scale folded into the logit
             const int t_a = 2 * tig, t_b = 8 + 2 * tig;
