@@ -54,6 +54,15 @@ def _lib():
         lib.or_select_evict_block.argtypes = [p, p, p, p, p, i32, i32, i32, i32]
         lib.or_quantize_int8.restype = None
         lib.or_quantize_int8.argtypes = [p, i64, i32, p, p]
+        lib.or_quantize_e4m3.restype = None
+        lib.or_quantize_e4m3.argtypes = [p, i64, p]
+        lib.or_e4m3_to_f64.restype = dbl
+        lib.or_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        lib.or_append_kv_fp8.restype = None
+        lib.or_append_kv_fp8.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, p]
+        lib.or_paged_decode_fp8.restype = None
+        lib.or_paged_decode_fp8.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32,
+                                            dbl]
         _LIB = lib
     return _LIB
 
@@ -215,3 +224,49 @@ def quantize_int8(x):
     scales = np.empty(x.shape[:-1], np.float32)
     _lib().or_quantize_int8(_ptr(x), rows, d, _ptr(codes), _ptr(scales))
     return codes, scales
+
+
+# --------------------------------------------------------------------------- fp8
+def quantize_e4m3(x):
+    """bf16 bits -> e4m3 codes (uint8), round to nearest even, saturating at 448
+    ([VKV] §6.1 FP8 branch: cast to float8_e4m3fn)."""
+    x = _c(x, np.uint16)
+    codes = np.empty(x.shape, np.uint8)
+    _lib().or_quantize_e4m3(_ptr(x), x.size, _ptr(codes))
+    return codes
+
+
+def e4m3_values(codes):
+    """Exact values of e4m3 codes as float64."""
+    codes = np.asarray(codes, np.uint8)
+    f = _lib().or_e4m3_to_f64
+    return np.vectorize(lambda c: f(int(c)), otypes=[np.float64])(codes)
+
+
+def append_kv_fp8(k_new, v_new, k_cache, v_cache, block_stride, bt, positions, bs):
+    """FP8 append in place (pools: flat uint8 e4m3 codes).  Returns slots."""
+    k_new = _c(k_new, np.uint16)
+    v_new = _c(v_new, np.uint16)
+    bt = _c(bt, np.int32)
+    positions = _c(positions, np.int32)
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    B, n_new, Hkv, d = k_new.shape
+    slots = np.empty((B, n_new), np.int64)
+    _lib().or_append_kv_fp8(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), block_stride,
+                            _ptr(bt), bt.shape[1], _ptr(positions), B, n_new, Hkv, d, bs,
+                            _ptr(slots))
+    return slots
+
+
+def paged_decode_fp8(q, k_cache, v_cache, block_stride, bt, ctx_lens, Hkv, bs, scale):
+    """fp64 paged decode over e4m3 pools (codes decoded exactly)."""
+    q = _c(q, np.uint16)
+    k_cache = _c(k_cache, np.uint8)
+    v_cache = _c(v_cache, np.uint8)
+    bt = _c(bt, np.int32)
+    ctx_lens = _c(ctx_lens, np.int32)
+    B, Hq, d = q.shape
+    out = np.empty((B, Hq, d), np.float64)
+    _lib().or_paged_decode_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), block_stride,
+                               _ptr(bt), bt.shape[1], _ptr(ctx_lens), B, Hq, Hkv, d, bs, scale)
+    return out

@@ -381,3 +381,79 @@ void or_append_kv_int8(const uint16_t *k_new, const uint16_t *v_new, int8_t *kq,
         }
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* FP8 (e4m3) KV                                                             */
+/* ------------------------------------------------------------------------ */
+
+/* [VKV] §6.1: the FP8 branch of quantize_kv_cache casts the KV tensor to
+ * float8_e4m3fn.  Format (OCP FP8 e4m3): 1 sign bit, 4 exponent bits with bias
+ * 7, 3 mantissa bits; normal values 2^(E-7) * (1 + m/8), subnormals m * 2^-9;
+ * largest finite value 448 (0x7e); 0x7f / 0xff are NaN; there is no infinity.
+ * Reading: round to nearest, ties to even; finite values beyond 448 saturate to
+ * +-448; NaN stays NaN. */
+uint8_t or_f32_to_e4m3(float x) {
+    if (x != x) return 0x7f;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a > 448.0) a = 448.0;
+    if (a < ldexp(1.0, -6)) {                  /* subnormal range: steps of 2^-9 */
+        const double m = rint(a * 512.0);      /* 8 lands exactly on 2^-6, code 0x08 */
+        return (uint8_t)(sign | (uint8_t)m);
+    }
+    int e;
+    frexp(a, &e);                              /* a = f * 2^e, f in [0.5, 1) */
+    int E = e - 1;                             /* a in [2^E, 2^(E+1)) */
+    double m = rint(a / ldexp(1.0, E - 3));    /* in [8, 16] */
+    if (m == 16.0) {
+        m = 8.0;
+        E += 1;
+    }
+    return (uint8_t)(sign | (uint8_t)(((E + 7) << 3) | ((int)m - 8)));
+}
+
+double or_e4m3_to_f64(uint8_t c) {
+    const int s = c >> 7, E = (c >> 3) & 15, m = c & 7;
+    if ((c & 0x7f) == 0x7f) return NAN;
+    const double v = E == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, E - 7);
+    return s ? -v : v;
+}
+
+void or_quantize_e4m3(const uint16_t *x, int64_t n, uint8_t *codes) {
+    for (int64_t i = 0; i < n; ++i) codes[i] = or_f32_to_e4m3(bf16_to_f32(x[i]));
+}
+
+/* FP8 append: the new rows are cast to e4m3 and stored at their slots. */
+void or_append_kv_fp8(const uint16_t *k_new, const uint16_t *v_new, uint8_t *k_cache,
+                      uint8_t *v_cache, int64_t block_stride, const int32_t *bt, int MB,
+                      const int32_t *positions, int B, int n_new, int Hkv, int d, int bs,
+                      int64_t *slot_out) {
+    for (int b = 0; b < B; ++b) {
+        for (int i = 0; i < n_new; ++i) {
+            int64_t pos = (int64_t)positions[b] + i;
+            int64_t slot = or_slot(bt + (int64_t)b * MB, pos, bs);
+            if (slot_out) slot_out[(int64_t)b * n_new + i] = slot;
+            int64_t phys = slot / bs, off = slot % bs;
+            for (int h = 0; h < Hkv; ++h) {
+                int64_t src = (((int64_t)b * n_new + i) * Hkv + h) * (int64_t)d;
+                int64_t dst = phys * block_stride + (off * Hkv + h) * (int64_t)d;
+                or_quantize_e4m3(k_new + src, d, k_cache + dst);
+                or_quantize_e4m3(v_new + src, d, v_cache + dst);
+            }
+        }
+    }
+}
+
+static double load_fp8(const void *pool, const void *aux, int64_t idx, int64_t row, int Hd) {
+    (void)aux; (void)row; (void)Hd;
+    return or_e4m3_to_f64(((const uint8_t *)pool)[idx]);
+}
+
+/* Paged decode attention over e4m3 pools (each element decoded exactly). */
+void or_paged_decode_fp8(double *out, const uint16_t *q, const uint8_t *k_cache,
+                         const uint8_t *v_cache, int64_t block_stride, const int32_t *bt, int MB,
+                         const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
+                         double scale) {
+    decode_common(out, q, k_cache, v_cache, NULL, NULL, load_fp8, block_stride, 0, bt, MB,
+                  ctx_lens, B, Hq, Hkv, d, bs, scale);
+}

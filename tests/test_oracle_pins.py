@@ -482,3 +482,59 @@ def test_int8_append_matches_quantiser_and_slots():
         for i in range(3):
             assert np.array_equal(kq4[slots[b, i]], cq[b, i])
             assert np.array_equal(ks2[slots[b, i]], cs[b, i])
+
+
+# ------------------------------------------------------------------ fp8 (e4m3)
+def test_e4m3_golden_codes():
+    rows = []
+    with open(os.path.join(GOLDEN, "e4m3_values.txt")) as f:
+        for ln in f:
+            if ln.strip() and not ln.startswith("#"):
+                v, c = ln.split()[:2]
+                rows.append((float(v), int(c, 16)))
+    x = np.array([v for v, _ in rows], np.float32)
+    assert np.array_equal(bf16_vals(bf16_bits(x)), x.astype(np.float64))  # inputs exact in bf16
+    codes = oracle.quantize_e4m3(bf16_bits(x))
+    assert codes.tolist() == [c for _, c in rows]
+
+
+def test_e4m3_every_finite_code_round_trips():
+    codes = np.array([c for c in range(256) if (c & 0x7f) != 0x7f], np.uint8)
+    vals = oracle.e4m3_values(codes)
+    # every finite e4m3 value is exact in bf16 (3-bit mantissa, exponent in range)
+    back = oracle.quantize_e4m3(bf16_bits(vals.astype(np.float32)))
+    assert np.array_equal(back[codes != 0x80], codes[codes != 0x80])  # -0 encodes as 0x80
+    pos = vals[(codes > 0) & (codes < 0x7f)]
+    assert np.all(np.diff(pos) > 0) and pos.max() == 448.0 and pos.min() == 2.0 ** -9
+
+
+def test_e4m3_matches_torch_cast_in_range():
+    rng = np.random.default_rng(31)
+    x = np.concatenate([rng.standard_normal(20000) * s for s in (0.01, 1.0, 30.0, 150.0)])
+    bits = bf16_bits(x)
+    xv = bf16_vals(bits)
+    keep = np.abs(xv) <= 448.0
+    ours = oracle.quantize_e4m3(bits)[keep]
+    ref = torch.as_tensor(xv[keep].astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8)
+    assert np.array_equal(ours, ref.numpy())
+
+
+def test_fp8_decode_equals_sdpa_on_decoded_values():
+    c = rand_case(33, Hq=8, Hkv=2, d=32, bs=4, N=20, lens=(5, 9, 14))
+    kq = oracle.quantize_e4m3(c["kc"])
+    vq = oracle.quantize_e4m3(c["vc"])
+    out = oracle.paged_decode_fp8(c["q"], kq.ravel(), vq.ravel(), c["bs"] * c["Hkv"] * c["d"],
+                                  c["bt"], c["lens"], c["Hkv"], c["bs"], 1 / math.sqrt(c["d"]))
+    kd, vd = oracle.e4m3_values(kq), oracle.e4m3_values(vq)
+    B, Hq, Hkv, d = c["B"], c["Hq"], c["Hkv"], c["d"]
+    q = bf16_vals(c["q"])
+    for b in range(B):
+        n = int(c["lens"][b])
+        ids = c["bt"][b, : -(-n // c["bs"])]
+        K = kd[ids].reshape(-1, Hkv, d)[:n]
+        V = vd[ids].reshape(-1, Hkv, d)[:n]
+        Kt = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)
+        Vt = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)
+        o = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q[b]).unsqueeze(1), Kt, Vt, scale=1 / math.sqrt(d))[:, 0].numpy()
+        np.testing.assert_allclose(out[b], o, rtol=1e-12, atol=1e-12)
