@@ -52,6 +52,10 @@ def parse():
     ap.add_argument("--workload", default="c3", choices=["c2", "c3", "c4", "c5"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--evict", default="full", choices=["full", "incremental"],
+                    help="workloads with a score pass: rescore the whole context per layer "
+                         "(full) or score each token once at append into a paged score pool "
+                         "and select blocks from it (incremental)")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling aid: keep only this many layers of the workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -181,7 +185,7 @@ def decode_algorithmic_bytes(cfg, ctx_lens, partial_slots, n_units=0):
 class Runner:
     """Device state and one decode step of a workload through the binding."""
 
-    def __init__(self, cfg, device, num_splits=0, wl=None):
+    def __init__(self, cfg, device, num_splits=0, wl=None, evict="full"):
         from paged_kv_cache_396_b200 import pagedkv as pk
         self.pk, self.cfg, self.dev = pk, cfg, device
         wl = W.generate(cfg, device) if wl is None else wl
@@ -220,10 +224,24 @@ class Runner:
                                          wl.v_hist[l, b:b + 1, :n].contiguous(), self.kq[l],
                                          self.vq[l], self.ks[l], self.vs[l], self.bt[b:b + 1],
                                          zeros[b:b + 1], self.err)
-            wl.k_hist = wl.v_hist = None
+        self.incremental = bool(cfg.score) and evict == "incremental"
         if cfg.score:
             self.scores = torch.zeros(B, MB * bs, Hkv, dtype=torch.float32, device=device)
             self.evict = torch.zeros(B, dtype=torch.int32, device=device)
+        if self.incremental:
+            # paged score pools, filled for the cached history once (set-up): score
+            # every cached token, then place each score at its token's slot
+            N = wl.num_blocks
+            self.score_pool = torch.zeros(self.L, N, bs, Hkv, dtype=torch.float32, device=device)
+            old = torch.as_tensor(wl.old_lens, device=device)
+            t = torch.arange(MB * bs, device=device)
+            live = t[None, :] < old[:, None]
+            bidx, tidx = live.nonzero(as_tuple=True)
+            slots = self.bt[bidx, tidx // bs].long() * bs + tidx % bs
+            for l in range(self.L):
+                pk.pe_score_tokens(self.scores, wl.k_pool[l], wl.v_pool[l], self.bt, self.ctx,
+                                   self.err)
+                self.score_pool[l].view(N * bs, Hkv)[slots] = self.scores[bidx, tidx]
         torch.cuda.synchronize(device)
         self.q = wl.q
         self.k_new, self.v_new = wl.k_new, wl.v_new
@@ -250,7 +268,7 @@ class Runner:
     def launches_per_step(self):
         per_layer = (1 if self.cfg.append else 0) + self.dec_launches
         if self.cfg.score:
-            per_layer += 2
+            per_layer += 1 if self.incremental else 2
         return per_layer * self.L
 
     def step(self, ev=None):
@@ -267,7 +285,10 @@ class Runner:
             else:
                 kp = self.wl.k_pool[l]
                 vp = self.wl.v_pool[l]
-                if cfg.append:
+                if cfg.append and self.incremental:
+                    pk.pa_append_kv_scored(self.k_new[l], self.v_new[l], kp, vp,
+                                           self.score_pool[l], self.bt, self.pos, self.err)
+                elif cfg.append:
                     pk.pa_append_kv(self.k_new[l], self.v_new[l], kp, vp, self.bt, self.pos,
                                     self.err)
                 if ev is not None:
@@ -276,7 +297,10 @@ class Runner:
                              self.err, self.ws, self.num_splits)
             if ev is not None:
                 ev[l][1].record()
-            if cfg.score:
+            if self.incremental:
+                pk.pe_select_evict_block_pooled(self.evict, self.score_pool[l], self.bt, self.ctx,
+                                                self.err)
+            elif cfg.score:
                 pk.pe_score_tokens(self.scores, self.wl.k_pool[l], self.wl.v_pool[l], self.bt,
                                    self.ctx, self.err)
                 pk.pe_select_evict_block(self.evict, self.scores, self.ctx, cfg.block_size)
@@ -399,7 +423,7 @@ def main():
     cfg = W.CONFIGS[args.workload]
     if args.layers:
         cfg = W.scaled(cfg, layers=args.layers)
-    r = Runner(cfg, device, args.num_splits)
+    r = Runner(cfg, device, args.num_splits, evict=args.evict)
     stream = torch.cuda.current_stream(device)
 
     for _ in range(max(3, args.warmup)):
@@ -529,6 +553,8 @@ def main():
             "dtype": "int8" if cfg.int8 else "bf16", "data": "synthetic",
             "config": dict(workload_config(cfg), parallelism=f"replicas{world}",
                            decode_kernel="staged-tc" if r.staged else "general",
+                           evict_scoring=("incremental score pool" if r.incremental else
+                                          "full pass per layer") if cfg.score else None,
                            partitions=r.partitions, chunk_tokens=r.chunk_used,
                            cuda_graph=use_graph),
             "roofline": {"bound": "hbm", "kernel": "pa_decode" + ("_int8" if cfg.int8 else ""),

@@ -196,6 +196,70 @@ int pa_decode_int8(uint16_t *out, const uint16_t *q,
                    int32_t *err_flag, void *stream);
 
 /* ============================================================================
+ * FP8 (e4m3) KV  ([VKV] §6.1: the FP8 branch of quantize_kv_cache casts the
+ * KV tensor to float8_e4m3fn, without a scale)
+ *
+ * pa_append_kv_fp8: pa_append_kv storing each element as an e4m3 code (1 sign,
+ * 4 exponent bits with bias 7, 3 mantissa bits): round to nearest, ties to
+ * even; finite values beyond +-448 saturate to +-448 (reading: the page's cast
+ * does not say; saturation keeps the cache finite); NaN stays NaN.
+ *   k8_cache, v8_cache : uint8 pools [N][bs][Hkv][d] (block_stride elements).
+ * pa_decode_fp8: pa_decode over e4m3 pools; every code is widened exactly (each
+ * e4m3 value is an fp16 value) in registers.  Same workspace rule as pa_decode.
+ * ==========================================================================*/
+int pa_append_kv_fp8(const uint16_t *k_new, const uint16_t *v_new,
+                     uint8_t *k8_cache, uint8_t *v8_cache, int64_t block_stride,
+                     const int32_t *block_tables, int max_blocks_per_seq,
+                     const int32_t *positions, int B, int n_new, int Hkv, int d, int bs,
+                     int64_t num_blocks, int64_t *slot_out, int32_t *err_flag, void *stream);
+
+int pa_decode_fp8(uint16_t *out, const uint16_t *q,
+                  const uint8_t *k8_cache, const uint8_t *v8_cache, int64_t block_stride,
+                  const int32_t *block_tables, int max_blocks_per_seq, const int32_t *ctx_lens,
+                  int B, int Hq, int Hkv, int d, int bs, int64_t num_blocks, float scale,
+                  int num_splits, void *workspace, size_t workspace_bytes,
+                  int32_t *err_flag, void *stream);
+
+/* ============================================================================
+ * Incremental PagedEviction scoring  ([KVL] "PagedEviction 块级驱逐机制": the
+ * importance S = ||V||_2 / ||K||_2 needs only the token's own K and V, and in
+ * the decode phase a block is chosen only when the newest block fills)
+ *
+ * pa_append_kv_scored: pa_append_kv that also writes each new (token, kv head)
+ * score into score_pool at the token's slot.  score_pool is fp32
+ * [N][bs][Hkv] (block stride bs*Hkv), paged exactly like the KV pool, so a
+ * block's scores move, stay and are freed with its K/V.  The score is computed
+ * from the bf16 values written, as pe_score_tokens would compute it from the
+ * pool (same ||K|| == 0 rule).
+ * pa_append_kv_int8_scored: the same for the INT8 append; the score is taken on
+ * the dequantised row (scale * codes).
+ * pe_select_evict_block_pooled: pe_select_evict_block reading the scores of
+ * every full logical block j < floor(ctx_lens[b] / bs) from score_pool through
+ * the block table (physical block block_tables[b][j]), summed in the same order
+ * and precision, so it returns exactly what pe_select_evict_block returns on
+ * the equal [B][MB*bs][Hkv] score array.  A needed table entry outside [0, N)
+ * raises PA_DEV_BAD_BLOCK and that block is not a candidate.
+ * ==========================================================================*/
+int pa_append_kv_scored(const uint16_t *k_new, const uint16_t *v_new,
+                        uint16_t *k_cache, uint16_t *v_cache, int64_t block_stride,
+                        float *score_pool, const int32_t *block_tables, int max_blocks_per_seq,
+                        const int32_t *positions, int B, int n_new, int Hkv, int d, int bs,
+                        int64_t num_blocks, int64_t *slot_out, int32_t *err_flag, void *stream);
+
+int pa_append_kv_int8_scored(const uint16_t *k_new, const uint16_t *v_new,
+                             int8_t *kq_cache, int8_t *vq_cache, float *k_scale, float *v_scale,
+                             float *score_pool, int64_t block_stride,
+                             const int32_t *block_tables, int max_blocks_per_seq,
+                             const int32_t *positions, int B, int n_new, int Hkv, int d, int bs,
+                             int64_t num_blocks, int64_t *slot_out, int32_t *err_flag,
+                             void *stream);
+
+int pe_select_evict_block_pooled(int32_t *evict, float *block_means, const float *score_pool,
+                                 const int32_t *block_tables, int max_blocks_per_seq,
+                                 const int32_t *ctx_lens, int B, int Hkv, int bs,
+                                 int64_t num_blocks, int32_t *err_flag, void *stream);
+
+/* ============================================================================
  * pa_decode without a caller-provided workspace (no counterpart in the pages;
  * it exists for callers, not for the method).
  *

@@ -4,6 +4,8 @@
 // Slot of position p in sequence b: block_tables[b][p / bs] * bs + p % bs
 // (ybb.press "LLM 推理 KV Cache 内存管理深度工程实践" §2.1, append_slot).
 // INT8 rows follow §6.1 of the same page: s = amax / 127, code = round(x / s).
+#include <math.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -91,11 +93,14 @@ __device__ __forceinline__ void store_codes(int8_t *p, const int8_t (&q)[D / 32]
 
 // One warp per (sequence, token, kv head) row: amax by warp reduction, then
 // the per-element code; lane 0 stores the row's scale.
+// score_pool (nullable): also store ||V||_2 / ||K||_2 of the dequantised row
+// (PagedEviction importance, see score_pool.cu) at the row's slot.
 template <int D>
 __global__ void append_int8_kernel(const uint16_t *__restrict__ k_new,
                                    const uint16_t *__restrict__ v_new, int8_t *__restrict__ kq,
                                    int8_t *__restrict__ vq, float *__restrict__ k_scale,
-                                   float *__restrict__ v_scale, AppendArgs a) {
+                                   float *__restrict__ v_scale, float *__restrict__ score_pool,
+                                   AppendArgs a) {
     constexpr int PER = D / 32;
     const int lane = threadIdx.x & 31;
     const int64_t rows = (int64_t)a.B * a.n_new * a.Hkv;
@@ -129,17 +134,103 @@ __global__ void append_int8_kernel(const uint16_t *__restrict__ k_new,
         const int64_t sdst = ((int64_t)phys * a.bs + off) * a.Hkv + h;
         float x[PER];
         int8_t q[PER];
-        float s;
+        float s, kk = 0.f, vv = 0.f;
         load_row<D>(k_new + src, x);
         quantise_row<PER>(x, q, s);
         store_codes<D>(kq + dst, q);
         if (lane == 0) k_scale[sdst] = s;
+        if (score_pool) {
+#pragma unroll
+            for (int e = 0; e < PER; ++e) {
+                const float y = s * (float)q[e];
+                kk = fmaf(y, y, kk);
+            }
+        }
         load_row<D>(v_new + src, x);
         quantise_row<PER>(x, q, s);
         store_codes<D>(vq + dst, q);
         if (lane == 0) v_scale[sdst] = s;
+        if (score_pool) {
+#pragma unroll
+            for (int e = 0; e < PER; ++e) {
+                const float y = s * (float)q[e];
+                vv = fmaf(y, y, vv);
+            }
+            kk = warp_sum(kk);
+            vv = warp_sum(vv);
+            if (lane == 0)
+                score_pool[sdst] = kk == 0.f ? (vv > 0.f ? INFINITY : 0.f) : sqrtf(vv) / sqrtf(kk);
+        }
         if (leader && a.slot_out) a.slot_out[bi] = (int64_t)phys * a.bs + off;
     }
+}
+
+// FP8 append ([VKV] §6.1 FP8 branch: a cast of the KV to float8_e4m3fn).  One
+// thread per 8 elements of a (sequence, token, kv head) row: 16 bytes of bf16
+// in, 8 bytes of e4m3 out, each pair converted round-to-nearest-even with
+// saturation at +-448 (cvt.rn.satfinite.e4m3x2.f32).
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__global__ void append_fp8_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
+                                  uint8_t *__restrict__ k8, uint8_t *__restrict__ v8, AppendArgs a) {
+    const int vec_per_row = a.d / 8;
+    const int64_t total = (int64_t)a.B * a.n_new * a.Hkv * vec_per_row;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int c = (int)(idx % vec_per_row);
+        const int64_t row = idx / vec_per_row;
+        const int h = (int)(row % a.Hkv);
+        const int64_t bi = row / a.Hkv;
+        const int i = (int)(bi % a.n_new);
+        const int b = (int)(bi / a.n_new);
+        const bool leader = (h == 0 && c == 0);
+        const int64_t pos = (int64_t)a.positions[b] + i;
+        if (pos < 0 || pos >= (int64_t)a.MB * a.bs) {
+            if (leader) {
+                raise_flag(a.err, PA_DEV_BAD_LEN);
+                if (a.slot_out) a.slot_out[bi] = -1;
+            }
+            continue;
+        }
+        const int32_t phys = a.block_tables[(int64_t)b * a.MB + pos / a.bs];
+        if (phys < 0 || (int64_t)phys >= a.N) {
+            if (leader) {
+                raise_flag(a.err, PA_DEV_BAD_BLOCK);
+                if (a.slot_out) a.slot_out[bi] = -1;
+            }
+            continue;
+        }
+        const int64_t off = pos % a.bs;
+        const int64_t dst = (int64_t)phys * a.block_stride + (off * a.Hkv + h) * a.d + c * 8;
+        const uint4 kw = __ldg(k_new + idx), vw = __ldg(v_new + idx);
+        const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, vv[4] = {vw.x, vw.y, vw.z, vw.w};
+        uint32_t ko[2], vo[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            ko[q] = f32x2_to_e4m3x2(bf16_lo(kk[2 * q]), bf16_hi(kk[2 * q])) |
+                    (f32x2_to_e4m3x2(bf16_lo(kk[2 * q + 1]), bf16_hi(kk[2 * q + 1])) << 16);
+            vo[q] = f32x2_to_e4m3x2(bf16_lo(vv[2 * q]), bf16_hi(vv[2 * q])) |
+                    (f32x2_to_e4m3x2(bf16_lo(vv[2 * q + 1]), bf16_hi(vv[2 * q + 1])) << 16);
+        }
+        *reinterpret_cast<uint2 *>(k8 + dst) = make_uint2(ko[0], ko[1]);
+        *reinterpret_cast<uint2 *>(v8 + dst) = make_uint2(vo[0], vo[1]);
+        if (leader && a.slot_out) a.slot_out[bi] = (int64_t)phys * a.bs + off;
+    }
+}
+
+cudaError_t launch_append_fp8(const uint16_t *k_new, const uint16_t *v_new, uint8_t *k8,
+                              uint8_t *v8, const AppendArgs &a, int num_sms, cudaStream_t stream) {
+    const int64_t total = (int64_t)a.B * a.n_new * a.Hkv * (a.d / 8);
+    const int threads = 256;
+    int64_t blocks = (total + threads - 1) / threads;
+    blocks = blocks < (int64_t)num_sms * 16 ? blocks : (int64_t)num_sms * 16;
+    append_fp8_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+        reinterpret_cast<const uint4 *>(k_new), reinterpret_cast<const uint4 *>(v_new), k8, v8, a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_append_bf16(const uint16_t *k_new, const uint16_t *v_new, uint16_t *k_cache,
@@ -156,18 +247,18 @@ cudaError_t launch_append_bf16(const uint16_t *k_new, const uint16_t *v_new, uin
 }
 
 cudaError_t launch_append_int8(const uint16_t *k_new, const uint16_t *v_new, int8_t *kq,
-                               int8_t *vq, float *k_scale, float *v_scale, const AppendArgs &a,
-                               int num_sms, cudaStream_t stream) {
+                               int8_t *vq, float *k_scale, float *v_scale, float *score_pool,
+                               const AppendArgs &a, int num_sms, cudaStream_t stream) {
     const int64_t rows = (int64_t)a.B * a.n_new * a.Hkv;
     const int threads = 256;
     int64_t blocks = (rows * 32 + threads - 1) / threads;
     blocks = blocks < (int64_t)num_sms * 16 ? blocks : (int64_t)num_sms * 16;
     if (a.d == 128)
-        append_int8_kernel<128><<<(unsigned)blocks, threads, 0, stream>>>(k_new, v_new, kq, vq,
-                                                                          k_scale, v_scale, a);
+        append_int8_kernel<128><<<(unsigned)blocks, threads, 0, stream>>>(
+            k_new, v_new, kq, vq, k_scale, v_scale, score_pool, a);
     else
-        append_int8_kernel<64><<<(unsigned)blocks, threads, 0, stream>>>(k_new, v_new, kq, vq,
-                                                                         k_scale, v_scale, a);
+        append_int8_kernel<64><<<(unsigned)blocks, threads, 0, stream>>>(
+            k_new, v_new, kq, vq, k_scale, v_scale, score_pool, a);
     return cudaGetLastError();
 }
 

@@ -19,10 +19,25 @@
 
 namespace pkv {
 
-template <int D, bool INT8>
+// fp16 bits -> fp32 (exact)
+__device__ __forceinline__ float half_bits_to_f32(uint16_t h) {
+    float f;
+    asm("{ .reg .f16 t; mov.b16 t, %1; cvt.f32.f16 %0, t; }" : "=f"(f) : "h"(h));
+    return f;
+}
+
+// Two e4m3 codes (low byte first) -> two fp32, exactly (every e4m3 value is an fp16).
+__device__ __forceinline__ void e4m3x2_to_f32(uint16_t c, float &lo, float &hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(c));
+    lo = half_bits_to_f32((uint16_t)(r & 0xffffu));
+    hi = half_bits_to_f32((uint16_t)(r >> 16));
+}
+
+template <int D, int KV>
 __device__ __forceinline__ void load_kv_row(const void *base, int64_t idx, float (&x)[D / 32]) {
     constexpr int VEC = D / 32;
-    if constexpr (INT8) {
+    if constexpr (KV == kKvInt8) {
         const int8_t *p = reinterpret_cast<const int8_t *>(base) + idx;
         if constexpr (VEC == 4) {
             const uint32_t w = __ldg(reinterpret_cast<const unsigned int *>(p));
@@ -32,6 +47,15 @@ __device__ __forceinline__ void load_kv_row(const void *base, int64_t idx, float
             const uint16_t w = __ldg(reinterpret_cast<const unsigned short *>(p));
             x[0] = (float)(int8_t)(w & 0xffu);
             x[1] = (float)(int8_t)(w >> 8);
+        }
+    } else if constexpr (KV == kKvFp8) {
+        const uint8_t *p = reinterpret_cast<const uint8_t *>(base) + idx;
+        if constexpr (VEC == 4) {
+            const uint32_t w = __ldg(reinterpret_cast<const unsigned int *>(p));
+            e4m3x2_to_f32((uint16_t)(w & 0xffffu), x[0], x[1]);
+            e4m3x2_to_f32((uint16_t)(w >> 16), x[2], x[3]);
+        } else {
+            e4m3x2_to_f32(__ldg(reinterpret_cast<const unsigned short *>(p)), x[0], x[1]);
         }
     } else {
         const uint16_t *p = reinterpret_cast<const uint16_t *>(base) + idx;
@@ -49,7 +73,7 @@ __device__ __forceinline__ void load_kv_row(const void *base, int64_t idx, float
 // t0+w, t0+w+4, ... of the partition and keeps its own online-softmax state
 // for the GP (>= G, power of two) query heads of the group; the four states are
 // merged through shared memory at the end.
-template <int D, int GP, bool INT8>
+template <int D, int GP, int KV>
 __global__ void __launch_bounds__(128) decode_simple_kernel(DecodeArgs a) {
     constexpr int VEC = D / 32;
     constexpr int NW = 4;
@@ -70,7 +94,7 @@ __global__ void __launch_bounds__(128) decode_simple_kernel(DecodeArgs a) {
         if (g < a.G) {
             float x[VEC];
             const int64_t qi = ((int64_t)b * a.Hq + h * a.G + g) * D + lane * VEC;
-            load_kv_row<D, false>(a.q, qi, x);
+            load_kv_row<D, kKvBf16>(a.q, qi, x);
 #pragma unroll
             for (int e = 0; e < VEC; ++e) qf[g][e] = x[e] * a.scale_log2;
         } else {
@@ -96,10 +120,10 @@ __global__ void __launch_bounds__(128) decode_simple_kernel(DecodeArgs a) {
         const int slot = t % a.bs;
         const int64_t row = (int64_t)phys * a.block_stride + ((int64_t)slot * a.Hkv + h) * D + lane * VEC;
         float kf[VEC], vf[VEC];
-        load_kv_row<D, INT8>(a.k_cache, row, kf);
-        load_kv_row<D, INT8>(a.v_cache, row, vf);
+        load_kv_row<D, KV>(a.k_cache, row, kf);
+        load_kv_row<D, KV>(a.v_cache, row, vf);
         float ks = 1.f, vs = 1.f;
-        if constexpr (INT8) {
+        if constexpr (KV == kKvInt8) {
             const int64_t srow = ((int64_t)phys * a.bs + slot) * a.Hkv + h;
             ks = __ldg(a.k_scale + srow);
             vs = __ldg(a.v_scale + srow);
@@ -186,28 +210,30 @@ __global__ void __launch_bounds__(D) merge_kernel(DecodeArgs a) {
     a.out[bh * D + e] = f32_to_bf16_rn(L > 0.f ? A / L : 0.f);
 }
 
-template <int D, bool INT8>
+template <int D, int KV>
 static void launch_simple_gp(const DecodeArgs &a, dim3 grid, cudaStream_t st) {
     int gp = 1;
     while (gp < a.G) gp <<= 1;
     switch (gp) {
-        case 1: decode_simple_kernel<D, 1, INT8><<<grid, 128, 0, st>>>(a); break;
-        case 2: decode_simple_kernel<D, 2, INT8><<<grid, 128, 0, st>>>(a); break;
-        case 4: decode_simple_kernel<D, 4, INT8><<<grid, 128, 0, st>>>(a); break;
-        case 8: decode_simple_kernel<D, 8, INT8><<<grid, 128, 0, st>>>(a); break;
-        default: decode_simple_kernel<D, 16, INT8><<<grid, 128, 0, st>>>(a); break;
+        case 1: decode_simple_kernel<D, 1, KV><<<grid, 128, 0, st>>>(a); break;
+        case 2: decode_simple_kernel<D, 2, KV><<<grid, 128, 0, st>>>(a); break;
+        case 4: decode_simple_kernel<D, 4, KV><<<grid, 128, 0, st>>>(a); break;
+        case 8: decode_simple_kernel<D, 8, KV><<<grid, 128, 0, st>>>(a); break;
+        default: decode_simple_kernel<D, 16, KV><<<grid, 128, 0, st>>>(a); break;
     }
 }
 
-cudaError_t launch_decode_simple(const DecodeArgs &a, bool int8, cudaStream_t st) {
+template <int D>
+static void launch_simple_kv(const DecodeArgs &a, int kv, dim3 grid, cudaStream_t st) {
+    if (kv == kKvInt8) launch_simple_gp<D, kKvInt8>(a, grid, st);
+    else if (kv == kKvFp8) launch_simple_gp<D, kKvFp8>(a, grid, st);
+    else launch_simple_gp<D, kKvBf16>(a, grid, st);
+}
+
+cudaError_t launch_decode_simple(const DecodeArgs &a, int kv, cudaStream_t st) {
     dim3 grid(a.num_splits, a.Hkv, a.B);
-    if (a.d == 128) {
-        if (int8) launch_simple_gp<128, true>(a, grid, st);
-        else launch_simple_gp<128, false>(a, grid, st);
-    } else {
-        if (int8) launch_simple_gp<64, true>(a, grid, st);
-        else launch_simple_gp<64, false>(a, grid, st);
-    }
+    if (a.d == 128) launch_simple_kv<128>(a, kv, grid, st);
+    else launch_simple_kv<64>(a, kv, grid, st);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || a.num_splits == 1) return e;
     return launch_merge(a, st);
@@ -220,9 +246,9 @@ cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const DecodeArgs &a, bool int8, cudaStream_t st) {
-    if (a.plan.kernel == 1) return launch_decode_tc(a, int8, st);
-    return launch_decode_simple(a, int8, st);
+cudaError_t launch_decode(const DecodeArgs &a, int kv, cudaStream_t st) {
+    if (a.plan.kernel == 1) return launch_decode_tc(a, kv, st);
+    return launch_decode_simple(a, kv, st);
 }
 
 namespace {
@@ -231,22 +257,23 @@ inline int up1024(int x) { return (x + 1023) / 1024 * 1024; }
 }  // namespace
 
 // Host launch plan.  The staged tensor-core kernel takes pools with a block
-// size that is a multiple of 16, Hkv in {1, 2, 4, 8} and G <= 16 (INT8: d = 128)
+// size that is a multiple of 16, Hkv in {1, 2, 4, 8} and G <= 16 (INT8, FP8: d = 128)
 // when at least two pipeline stages fit in shared memory; everything else runs
 // the general-shape kernel.
 DecodePlan make_decode_plan(int B, int Hq, int Hkv, int d, int bs, int MB, int num_splits,
-                            bool int8, int sms) {
+                            int kv, int sms) {
+    const bool onebyte = kv != kKvBf16;  // int8 and fp8 pools: one byte per element
     DecodePlan p;
     memset(&p, 0, sizeof p);
     const int64_t max_ctx = (int64_t)MB * bs;
     const int G = Hq / Hkv;
     bool tc = bs % 16 == 0 && (Hkv == 1 || Hkv == 2 || Hkv == 4 || Hkv == 8) && G <= 16 &&
-              (!int8 || d == 128);
+              (!onebyte || d == 128);
     if (tc) {
         const int box = Hkv * 16 * 128;  // one 128-byte slice of d of 16 tokens, all heads
-        const int DC = int8 ? d / 128 : d / 64;
+        const int DC = onebyte ? d / 128 : d / 64;
         const int sub_kv = DC * box;                    // K (or V) bytes of one 16-token sub-tile
-        const int sub_sc = int8 ? 16 * Hkv * 4 : 0;     // its scale rows
+        const int sub_sc = kv == kKvInt8 ? 16 * Hkv * 4 : 0;  // its scale rows
         p.wph = 8 / Hkv;
         // sub-tiles per warp per stage: stages of about 64 KB of K + V amortise the
         // per-stage cost of the pipeline

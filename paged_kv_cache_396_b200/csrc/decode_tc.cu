@@ -189,12 +189,13 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *ctx_lens, int
 // ---------------------------------------------------------------------------
 // decode: persistent, warp-specialised
 // ---------------------------------------------------------------------------
-template <int D, bool I8>
+template <int D, int KV>
 __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensorMap *vmap,
                                          const Args &a, uint8_t *stages, StageMeta *meta,
                                          uint64_t *full, uint64_t *empty) {
-    // one box covers 128 bytes of d: 64 bf16 or 128 int8 values
-    constexpr int DC = I8 ? D / 128 : D / 64;
+    // one box covers 128 bytes of d: 64 bf16 or 128 one-byte (int8, e4m3) values
+    constexpr bool I8 = KV == kKvInt8;
+    constexpr int DC = KV != kKvBf16 ? D / 128 : D / 64;
     const int lane = threadIdx.x & 31;
     const int T_s = kTile * a.n_sub;
     const uint32_t sc_bytes = (uint32_t)kTile * a.Hkv * 4;  // one sub-tile's scale rows
@@ -902,7 +903,240 @@ __device__ __forceinline__ void consumer_i8(const Args &a, uint8_t *stages, Stag
     }
 }
 
-template <int D, bool G16, bool I8>
+// Two e4m3 codes (one 16-bit half of w; low byte first) -> exact fp16x2.
+__device__ __forceinline__ void e4m3_word_to_f16x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+}
+
+// Query fragments (fp16) for the FP8 consumer: k-step kk (16 dims) of thread
+// (g, tig) uses dims 16*(tig + 4*(kk/4)) + 4*(kk%4) + 0..3, the dims of the K
+// word it converts (see consumer_fp8).
+__device__ __forceinline__ void load_q_f16perm(const Args &a, int b, int row, bool live, int tig,
+                                               uint32_t (&qa)[8][2]) {
+    constexpr int D = 128;
+    const uint4 *qr = reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * a.Hq + row) * D);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t f[8];
+        if (live) {
+            const int c = tig + 4 * half;  // 16 dims = two uint4 of bf16
+            bf16x8_to_f16x2(__ldg(qr + 2 * c), f);
+            bf16x8_to_f16x2(__ldg(qr + 2 * c + 1), f + 4);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = 0u;
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            qa[4 * half + w][0] = f[2 * w];
+            qa[4 * half + w][1] = f[2 * w + 1];
+        }
+    }
+}
+
+// FP8 (e4m3) consumer (d = 128).  Same pipeline and softmax as the bf16
+// consumer; tiles hold e4m3 codes, [head][token][128 bytes], 128-byte swizzled,
+// converted exactly to fp16 in registers (every e4m3 value is an fp16).
+//  QK^T: k-step kk of thread (g, tig) converts word kk of its two 16-byte
+//   chunks (dims 16*(tig + 4*(kk/4)) + 4*(kk%4) + 0..3) into its b0/b1 pair;
+//   the query fragments use the same dims (load_q_f16perm).
+//  PV: as in the INT8 consumer -- n-tile nt, column g is dim 16*g + nt; token
+//   pairs are byte-transposed with prmt before the conversion.
+template <bool G16>
+__device__ __forceinline__ void consumer_fp8(const Args &a, uint8_t *stages, StageMeta *meta,
+                                             uint64_t *full, uint64_t *empty) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = warp % a.Hkv, jw = warp / a.Hkv;
+    const int g = lane >> 2, tig = lane & 3;
+    const int odd = g & 1;
+    const uint32_t stage0 = ptx::smem_u32(stages);
+    const uint32_t head_off = (uint32_t)(h * kTile * kBoxRow);
+    const uint32_t sub_bytes = (uint32_t)a.box_bytes;
+
+    uint32_t qa[8][2];
+    uint32_t qb[G16 ? 8 : 1][2];
+    float o[16][2];
+    float ob[G16 ? 16 : 1][2];
+    float m = -INFINITY, l = 0.f, mb = -INFINITY, lb = 0.f;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (;;) {
+        if (!ptx::mbar_wait(&full[stage], phase)) {
+            if (lane == 0) raise_flag(a.err, PA_DEV_TIMEOUT);
+            break;
+        }
+        const StageMeta mt = meta[stage];
+        if (mt.flags & kEnd) break;
+        const uint32_t sb = stage0 + (uint32_t)stage * a.stage_bytes;
+        if (mt.flags & kFirst) {
+            load_q_f16perm(a, mt.b, h * a.G + g, g < a.G, tig, qa);
+            if constexpr (G16) {
+                uint32_t t[8][2];
+                load_q_f16perm(a, mt.b, h * a.G + g + 8, g + 8 < a.G, tig, t);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    qb[kk][0] = t[kk][0];
+                    qb[kk][1] = t[kk][1];
+                }
+            }
+            m = -INFINITY;
+            l = 0.f;
+            mb = -INFINITY;
+            lb = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) {
+                o[nt][0] = o[nt][1] = 0.f;
+                if constexpr (G16) ob[nt][0] = ob[nt][1] = 0.f;
+            }
+        }
+        for (int k = 0; k < a.tpw; ++k) {
+        const int jj = jw + a.wph * k;  // this warp's k-th sub-tile of the stage
+        const int tj = mt.ts + kTile * jj;
+        const int nv = max(0, min(kTile, mt.te - tj));
+        if (nv > 0 && !((mt.bad >> jj) & 1)) {
+            const uint32_t kbase = sb + jj * sub_bytes + head_off;
+            const uint32_t vbase = sb + a.v_off + jj * sub_bytes + head_off;
+            // ---- S = Q K^T (exact fp16 values of the codes)
+            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+            float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int t = 8 * nt + g;  // swizzle phase of row t is g
+                const uint32_t rb = kbase + t * kBoxRow;
+                const uint4 x0 = lds128(rb + (((tig + 4 * odd) ^ g) << 4));
+                const uint4 x1 = lds128(rb + (((tig + 4 * (1 - odd)) ^ g) << 4));
+                const uint4 lo = odd ? x1 : x0;  // dims 16*tig ..
+                const uint4 hi = odd ? x0 : x1;  // dims 16*(tig+4) ..
+                const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    uint32_t b0, b1;
+                    e4m3_word_to_f16x2(wd[kk], b0, b1);
+                    float(&acc)[4] = nt == 0 ? ((kk & 1) ? e0 : s0) : ((kk & 1) ? e1 : s1);
+                    if constexpr (G16)
+                        ptx::mma_f16(acc, qa[kk][0], qb[kk][0], qa[kk][1], qb[kk][1], b0, b1);
+                    else
+                        ptx::mma_f16(acc, qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                s0[i] += e0[i];
+                s1[i] += e1[i];
+            }
+            // ---- online softmax
+            const int t_a = 2 * tig, t_b = 8 + 2 * tig;
+            const bool va0 = t_a < nv, va1 = t_a + 1 < nv, vb0 = t_b < nv, vb1 = t_b + 1 < nv;
+            const float sl = a.scale_log2;
+            float x0 = va0 ? s0[0] * sl : -INFINITY, x1 = va1 ? s0[1] * sl : -INFINITY;
+            float x2 = vb0 ? s1[0] * sl : -INFINITY, x3 = vb1 ? s1[1] * sl : -INFINITY;
+            float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+            const float mn = fmaxf(m, mx);
+            const float mu = mn == -INFINITY ? 0.f : mn;
+            const float alpha = exp2f(m - mu);
+            const float p0 = exp2f(x0 - mu), p1 = exp2f(x1 - mu);
+            const float p2 = exp2f(x2 - mu), p3 = exp2f(x3 - mu);
+            l = l * alpha + ((p0 + p1) + (p2 + p3));
+            m = mn;
+            const uint32_t pa0 = ptx::pack_f16(p0, p1), pa2 = ptx::pack_f16(p2, p3);
+            uint32_t pa1 = 0u, pa3 = 0u;
+            float alphab = 1.f;
+            if constexpr (G16) {
+                float y0 = va0 ? s0[2] * sl : -INFINITY, y1 = va1 ? s0[3] * sl : -INFINITY;
+                float y2 = vb0 ? s1[2] * sl : -INFINITY, y3 = vb1 ? s1[3] * sl : -INFINITY;
+                float my = fmaxf(fmaxf(y0, y1), fmaxf(y2, y3));
+                my = fmaxf(my, __shfl_xor_sync(kFull, my, 1));
+                my = fmaxf(my, __shfl_xor_sync(kFull, my, 2));
+                const float mnb = fmaxf(mb, my);
+                const float mub = mnb == -INFINITY ? 0.f : mnb;
+                alphab = exp2f(mb - mub);
+                const float q0 = exp2f(y0 - mub), q1 = exp2f(y1 - mub);
+                const float q2 = exp2f(y2 - mub), q3 = exp2f(y3 - mub);
+                lb = lb * alphab + ((q0 + q1) + (q2 + q3));
+                mb = mnb;
+                pa1 = ptx::pack_f16(q0, q1);
+                pa3 = ptx::pack_f16(q2, q3);
+            }
+            if (__any_sync(kFull, alpha != 1.f || alphab != 1.f)) {
+#pragma unroll
+                for (int nt = 0; nt < 16; ++nt) {
+                    o[nt][0] *= alpha;
+                    o[nt][1] *= alpha;
+                    if constexpr (G16) {
+                        ob[nt][0] *= alphab;
+                        ob[nt][1] *= alphab;
+                    }
+                }
+            }
+            // ---- O += P V; column g of n-tile nt is dim 16*g + nt.  Masked tokens
+            // have P = 0; their codes may be NaN (0x7f), so zero those rows' bytes.
+            const uint4 ra = lds128(vbase + t_a * kBoxRow + ((g ^ (t_a & 7)) << 4));
+            const uint4 rb = lds128(vbase + (t_a + 1) * kBoxRow + ((g ^ ((t_a + 1) & 7)) << 4));
+            const uint4 rc = lds128(vbase + t_b * kBoxRow + ((g ^ (t_b & 7)) << 4));
+            const uint4 rd = lds128(vbase + (t_b + 1) * kBoxRow + ((g ^ ((t_b + 1) & 7)) << 4));
+            const uint32_t za = va0 ? ~0u : 0u, zb = va1 ? ~0u : 0u;
+            const uint32_t zc = vb0 ? ~0u : 0u, zd = vb1 ? ~0u : 0u;
+            const uint32_t wa[4] = {ra.x & za, ra.y & za, ra.z & za, ra.w & za};
+            const uint32_t wb[4] = {rb.x & zb, rb.y & zb, rb.z & zb, rb.w & zb};
+            const uint32_t wc[4] = {rc.x & zc, rc.y & zc, rc.z & zc, rc.w & zc};
+            const uint32_t wdv[4] = {rd.x & zd, rd.y & zd, rd.z & zd, rd.w & zd};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const uint32_t X = prmt(wa[w], wb[w], 0x5140u), Y = prmt(wa[w], wb[w], 0x7362u);
+                const uint32_t Z = prmt(wc[w], wdv[w], 0x5140u), U = prmt(wc[w], wdv[w], 0x7362u);
+                uint32_t b0[4], b1[4];
+                e4m3_word_to_f16x2(X, b0[0], b0[1]);
+                e4m3_word_to_f16x2(Y, b0[2], b0[3]);
+                e4m3_word_to_f16x2(Z, b1[0], b1[1]);
+                e4m3_word_to_f16x2(U, b1[2], b1[3]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int nt = 4 * w + i;
+                    float dd[4] = {o[nt][0], o[nt][1], 0.f, 0.f};
+                    if constexpr (G16) {
+                        dd[2] = ob[nt][0];
+                        dd[3] = ob[nt][1];
+                    }
+                    ptx::mma_f16(dd, pa0, pa1, pa2, pa3, b0[i], b1[i]);
+                    o[nt][0] = dd[0];
+                    o[nt][1] = dd[1];
+                    if constexpr (G16) {
+                        ob[nt][0] = dd[2];
+                        ob[nt][1] = dd[3];
+                    }
+                }
+            }
+        }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&empty[stage]);
+        if (mt.flags & kLast) {
+            float lt = l + __shfl_xor_sync(kFull, l, 1);
+            lt += __shfl_xor_sync(kFull, lt, 2);
+            float ltb = 0.f;
+            if constexpr (G16) {
+                ltb = lb + __shfl_xor_sync(kFull, lb, 1);
+                ltb += __shfl_xor_sync(kFull, ltb, 2);
+            }
+            const int row = h * a.G + g;
+            if (g < a.G) store_i8_row(a, mt, o, 0.f, lt, m, row, tig, jw);
+            if constexpr (G16) {
+                if (g + 8 < a.G) store_i8_row(a, mt, ob, 0.f, ltb, mb, row + 8, tig, jw);
+            }
+        }
+        if (++stage == a.nstage) {
+            stage = 0;
+            phase ^= 1u;
+        }
+    }
+}
+
+template <int D, bool G16, int KV>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const Args a) {
@@ -926,9 +1160,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::grid_launch_dependents();
     ptx::grid_dependency_wait();
     if ((threadIdx.x >> 5) == kConsumerWarps)
-        producer<D, I8>(&kmap, &vmap, a, stages, meta, full, empty);
-    else if constexpr (I8)
+        producer<D, KV>(&kmap, &vmap, a, stages, meta, full, empty);
+    else if constexpr (KV == kKvInt8)
         consumer_i8<G16>(a, stages, meta, full, empty);
+    else if constexpr (KV == kKvFp8)
+        consumer_fp8<G16>(a, stages, meta, full, empty);
     else
         consumer<D, G16>(a, stages, meta, full, empty);
 }
@@ -1026,10 +1262,10 @@ bool encode_pool_map(CUtensorMap *map, const void *base, int64_t N, int bs, int 
     return r == CUDA_SUCCESS;
 }
 
-template <int D, bool G16, bool I8>
+template <int D, bool G16, int KV>
 cudaError_t launch_typed(const CUtensorMap &km, const CUtensorMap &vm, const Args &a, int grid,
                          int smem, cudaStream_t st) {
-    auto kfn = decode_tc_kernel<D, G16, I8>;
+    auto kfn = decode_tc_kernel<D, G16, KV>;
     // raise the dynamic shared-memory limit to what this launch needs (per device,
     // only upwards; static shared memory counts against the same per-block budget)
     static int smem_set[64] = {0};  // benign race: idempotent
@@ -1046,8 +1282,9 @@ cudaError_t launch_typed(const CUtensorMap &km, const CUtensorMap &vm, const Arg
 
 }  // namespace tc
 
-cudaError_t launch_decode_tc(const DecodeArgs &d, bool int8, cudaStream_t st) {
+cudaError_t launch_decode_tc(const DecodeArgs &d, int kv, cudaStream_t st) {
     using namespace tc;
+    const bool int8 = kv != kKvBf16;  // one-byte pools (int8 codes or e4m3)
     const DecodePlan &p = d.plan;
     CUtensorMap km, vm;
     if (!encode_pool_map(&km, d.k_cache, d.N, d.bs, d.Hkv, d.d, d.block_stride, int8) ||
@@ -1095,15 +1332,18 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, bool int8, cudaStream_t st) {
                                max_ctx, p.chunk, p.grid * p.units_per_cta);
     if (e != cudaSuccess) return e;
     const bool g16 = d.G > 8;
-    if (int8)  // d == 128 only (the plan guarantees it)
-        e = g16 ? launch_typed<128, true, true>(km, vm, a, p.grid, p.smem_bytes, st)
-                : launch_typed<128, false, true>(km, vm, a, p.grid, p.smem_bytes, st);
+    if (kv == kKvInt8)  // one-byte pools: d == 128 only (the plan guarantees it)
+        e = g16 ? launch_typed<128, true, kKvInt8>(km, vm, a, p.grid, p.smem_bytes, st)
+                : launch_typed<128, false, kKvInt8>(km, vm, a, p.grid, p.smem_bytes, st);
+    else if (kv == kKvFp8)
+        e = g16 ? launch_typed<128, true, kKvFp8>(km, vm, a, p.grid, p.smem_bytes, st)
+                : launch_typed<128, false, kKvFp8>(km, vm, a, p.grid, p.smem_bytes, st);
     else if (d.d == 128)
-        e = g16 ? launch_typed<128, true, false>(km, vm, a, p.grid, p.smem_bytes, st)
-                : launch_typed<128, false, false>(km, vm, a, p.grid, p.smem_bytes, st);
+        e = g16 ? launch_typed<128, true, kKvBf16>(km, vm, a, p.grid, p.smem_bytes, st)
+                : launch_typed<128, false, kKvBf16>(km, vm, a, p.grid, p.smem_bytes, st);
     else
-        e = g16 ? launch_typed<64, true, false>(km, vm, a, p.grid, p.smem_bytes, st)
-                : launch_typed<64, false, false>(km, vm, a, p.grid, p.smem_bytes, st);
+        e = g16 ? launch_typed<64, true, kKvBf16>(km, vm, a, p.grid, p.smem_bytes, st)
+                : launch_typed<64, false, kKvBf16>(km, vm, a, p.grid, p.smem_bytes, st);
     if (e != cudaSuccess) return e;
     if (p.S > 1 || p.wph > 1) {
         const unsigned rows = (unsigned)((int64_t)d.B * d.Hq);

@@ -7,6 +7,9 @@
 
 namespace pkv {
 
+// Element type of the KV pools.
+enum KvType : int { kKvBf16 = 0, kKvInt8 = 1, kKvFp8 = 2 };
+
 struct AppendArgs {
     const int32_t *block_tables;
     const int32_t *positions;
@@ -77,16 +80,25 @@ cudaError_t launch_append_bf16(const uint16_t *k_new, const uint16_t *v_new, uin
                                uint16_t *v_cache, const AppendArgs &a, int num_sms,
                                cudaStream_t stream);
 cudaError_t launch_append_int8(const uint16_t *k_new, const uint16_t *v_new, int8_t *kq,
-                               int8_t *vq, float *k_scale, float *v_scale, const AppendArgs &a,
-                               int num_sms, cudaStream_t stream);
+                               int8_t *vq, float *k_scale, float *v_scale, float *score_pool,
+                               const AppendArgs &a, int num_sms, cudaStream_t stream);
+cudaError_t launch_append_fp8(const uint16_t *k_new, const uint16_t *v_new, uint8_t *k8,
+                              uint8_t *v8, const AppendArgs &a, int num_sms, cudaStream_t stream);
+cudaError_t launch_append_scored(const uint16_t *k_new, const uint16_t *v_new, uint16_t *k_cache,
+                                 uint16_t *v_cache, float *score_pool, const AppendArgs &a,
+                                 int num_sms, cudaStream_t stream);
+cudaError_t launch_select_pooled(int32_t *evict, float *means, const float *score_pool,
+                                 const int32_t *block_tables, const int32_t *ctx_lens,
+                                 int32_t *err, int B, int MB, int Hkv, int bs, int64_t N,
+                                 cudaStream_t stream);
 
 // Decode dispatch: the staged tensor-core kernel when the shape allows it,
 // else the general-shape kernel; then the partition merge when S > 1.
-cudaError_t launch_decode(const DecodeArgs &a, bool int8, cudaStream_t stream);
-cudaError_t launch_decode_simple(const DecodeArgs &a, bool int8, cudaStream_t stream);
-cudaError_t launch_decode_tc(const DecodeArgs &a, bool int8, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs &a, int kv, cudaStream_t stream);
+cudaError_t launch_decode_simple(const DecodeArgs &a, int kv, cudaStream_t stream);
+cudaError_t launch_decode_tc(const DecodeArgs &a, int kv, cudaStream_t stream);
 DecodePlan make_decode_plan(int B, int Hq, int Hkv, int d, int bs, int MB, int num_splits,
-                            bool int8, int sms);
+                            int kv, int sms);
 cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t stream);
 
 cudaError_t launch_score(const ScoreArgs &a, cudaStream_t stream);

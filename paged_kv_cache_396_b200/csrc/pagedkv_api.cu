@@ -52,24 +52,24 @@ int finish(cudaError_t e) { return e == cudaSuccess ? PA_OK : PA_ERR_CUDA; }
 
 // Shared body of pa_decode / pa_decode_int8.
 int decode_entry(uint16_t *out, const uint16_t *q, const void *kc, const void *vc, const float *ks,
-                 const float *vs, bool int8, int64_t block_stride, const int32_t *bt, int MB,
+                 const float *vs, int kv, int64_t block_stride, const int32_t *bt, int MB,
                  const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs, int64_t N,
                  float scale, int num_splits, void *ws, size_t ws_bytes, int32_t *err,
                  void *stream) {
     if (B == 0) return PA_OK;  // empty batch: nothing to read or write
     if (!out || !q || !kc || !vc || !bt || !ctx_lens || !err) return PA_ERR_NULL;
-    if (int8 && (!ks || !vs)) return PA_ERR_NULL;
+    if (kv == pkv::kKvInt8 && (!ks || !vs)) return PA_ERR_NULL;
     int rc = check_common(B, Hkv, d, bs, MB, N, block_stride);
     if (rc) return rc;
     if (Hq < Hkv || Hq % Hkv != 0 || Hq / Hkv > 16) return PA_ERR_SHAPE;
     if (!(scale == scale)) return PA_ERR_SHAPE;
-    const int elt = int8 ? 1 : 2;
+    const int elt = kv == pkv::kKvBf16 ? 2 : 1;
     if (!al16(out) || !al16(q) || !al16(kc) || !al16(vc) || (block_stride * elt) % 16 != 0)
         return PA_ERR_ALIGN;
     if (B == 0) return PA_OK;
     const int sms = device_sms();
     if (sms < 0) return sms;
-    const pkv::DecodePlan plan = pkv::make_decode_plan(B, Hq, Hkv, d, bs, MB, num_splits, int8, sms);
+    const pkv::DecodePlan plan = pkv::make_decode_plan(B, Hq, Hkv, d, bs, MB, num_splits, kv, sms);
     if (plan.ws_total > 0) {
         if (!ws) return PA_ERR_WORKSPACE;
         if (ws_bytes < plan.ws_total) return PA_ERR_WORKSPACE;
@@ -104,7 +104,7 @@ int decode_entry(uint16_t *out, const uint16_t *q, const void *kc, const void *v
     a.MB = MB;
     a.num_splits = plan.S;
     a.chunk = plan.chunk;
-    return finish(pkv::launch_decode(a, int8, static_cast<cudaStream_t>(stream)));
+    return finish(pkv::launch_decode(a, kv, static_cast<cudaStream_t>(stream)));
 }
 
 // Scratch for pa_decode_static_scratch: a fixed array inside the library, one
@@ -187,8 +187,70 @@ int pa_append_kv_int8(const uint16_t *k_new, const uint16_t *v_new, int8_t *kq_c
     if (sms < 0) return sms;
     pkv::AppendArgs a{block_tables, positions, slot_out, err_flag, block_stride, num_blocks,
                       B, n_new, Hkv, d, bs, max_blocks_per_seq};
-    return finish(pkv::launch_append_int8(k_new, v_new, kq_cache, vq_cache, k_scale, v_scale, a,
-                                          sms, static_cast<cudaStream_t>(stream)));
+    return finish(pkv::launch_append_int8(k_new, v_new, kq_cache, vq_cache, k_scale, v_scale,
+                                          nullptr, a, sms, static_cast<cudaStream_t>(stream)));
+}
+
+int pa_append_kv_scored(const uint16_t *k_new, const uint16_t *v_new, uint16_t *k_cache,
+                        uint16_t *v_cache, int64_t block_stride, float *score_pool,
+                        const int32_t *block_tables, int max_blocks_per_seq,
+                        const int32_t *positions, int B, int n_new, int Hkv, int d, int bs,
+                        int64_t num_blocks, int64_t *slot_out, int32_t *err_flag, void *stream) {
+    if (B == 0 || n_new == 0) return PA_OK;
+    if (!k_new || !v_new || !k_cache || !v_cache || !score_pool || !block_tables || !positions ||
+        !err_flag)
+        return PA_ERR_NULL;
+    int rc = check_common(B, Hkv, d, bs, max_blocks_per_seq, num_blocks, block_stride);
+    if (rc) return rc;
+    if (n_new < 0) return PA_ERR_SHAPE;
+    if (!al16(k_new) || !al16(v_new) || !al16(k_cache) || !al16(v_cache) ||
+        (block_stride * 2) % 16 != 0)
+        return PA_ERR_ALIGN;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    pkv::AppendArgs a{block_tables, positions, slot_out, err_flag, block_stride, num_blocks,
+                      B, n_new, Hkv, d, bs, max_blocks_per_seq};
+    return finish(pkv::launch_append_scored(k_new, v_new, k_cache, v_cache, score_pool, a, sms,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+int pa_append_kv_int8_scored(const uint16_t *k_new, const uint16_t *v_new, int8_t *kq_cache,
+                             int8_t *vq_cache, float *k_scale, float *v_scale, float *score_pool,
+                             int64_t block_stride, const int32_t *block_tables,
+                             int max_blocks_per_seq, const int32_t *positions, int B, int n_new,
+                             int Hkv, int d, int bs, int64_t num_blocks, int64_t *slot_out,
+                             int32_t *err_flag, void *stream) {
+    if (B == 0 || n_new == 0) return PA_OK;
+    if (!k_new || !v_new || !kq_cache || !vq_cache || !k_scale || !v_scale || !score_pool ||
+        !block_tables || !positions || !err_flag)
+        return PA_ERR_NULL;
+    int rc = check_common(B, Hkv, d, bs, max_blocks_per_seq, num_blocks, block_stride);
+    if (rc) return rc;
+    if (n_new < 0) return PA_ERR_SHAPE;
+    if (!al16(k_new) || !al16(v_new) || !al16(kq_cache) || !al16(vq_cache) || !al16(k_scale) ||
+        !al16(v_scale) || block_stride % 16 != 0)
+        return PA_ERR_ALIGN;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    pkv::AppendArgs a{block_tables, positions, slot_out, err_flag, block_stride, num_blocks,
+                      B, n_new, Hkv, d, bs, max_blocks_per_seq};
+    return finish(pkv::launch_append_int8(k_new, v_new, kq_cache, vq_cache, k_scale, v_scale,
+                                          score_pool, a, sms, static_cast<cudaStream_t>(stream)));
+}
+
+int pe_select_evict_block_pooled(int32_t *evict, float *block_means, const float *score_pool,
+                                 const int32_t *block_tables, int max_blocks_per_seq,
+                                 const int32_t *ctx_lens, int B, int Hkv, int bs,
+                                 int64_t num_blocks, int32_t *err_flag, void *stream) {
+    if (B == 0) return PA_OK;
+    if (!evict || !score_pool || !block_tables || !ctx_lens || !err_flag) return PA_ERR_NULL;
+    if (B < 0 || B > 65535 || max_blocks_per_seq < 1 || Hkv < 1 || bs < 1 || num_blocks < 1)
+        return PA_ERR_SHAPE;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    return finish(pkv::launch_select_pooled(evict, block_means, score_pool, block_tables,
+                                            ctx_lens, err_flag, B, max_blocks_per_seq, Hkv, bs,
+                                            num_blocks, static_cast<cudaStream_t>(stream)));
 }
 
 size_t pa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq,
@@ -197,12 +259,14 @@ size_t pa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int bs, int max_
     const int sms = device_sms();
     if (sms < 0) return 0;
     if (Hq < Hkv || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
-    // one size serves pa_decode and pa_decode_int8 alike
-    const size_t a = pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits,
-                                           false, sms).ws_total;
-    const size_t b = pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits,
-                                           true, sms).ws_total;
-    return a > b ? a : b;
+    // one size serves pa_decode, pa_decode_int8 and pa_decode_fp8 alike
+    size_t mx = 0;
+    for (int kv = pkv::kKvBf16; kv <= pkv::kKvFp8; ++kv) {
+        const size_t w = pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits,
+                                               kv, sms).ws_total;
+        mx = w > mx ? w : mx;
+    }
+    return mx;
 }
 
 int pa_decode_plan(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq, int num_splits,
@@ -214,7 +278,7 @@ int pa_decode_plan(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq
     if (sms < 0) return sms;
     if (Hq < Hkv || Hq % Hkv != 0) return PA_ERR_SHAPE;
     const pkv::DecodePlan p =
-        pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits, false, sms);
+        pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits, pkv::kKvBf16, sms);
     *num_splits_out = p.S;
     *chunk_tokens_out = p.chunk;
     if (launches_out)
@@ -227,7 +291,7 @@ int pa_decode(uint16_t *out, const uint16_t *q, const uint16_t *k_cache, const u
               const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs, int64_t num_blocks,
               float scale, int num_splits, void *workspace, size_t workspace_bytes,
               int32_t *err_flag, void *stream) {
-    return decode_entry(out, q, k_cache, v_cache, nullptr, nullptr, false, block_stride,
+    return decode_entry(out, q, k_cache, v_cache, nullptr, nullptr, pkv::kKvBf16, block_stride,
                         block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
                         scale, num_splits, workspace, workspace_bytes, err_flag, stream);
 }
@@ -238,7 +302,39 @@ int pa_decode_int8(uint16_t *out, const uint16_t *q, const int8_t *kq_cache,
                    const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
                    int64_t num_blocks, float scale, int num_splits, void *workspace,
                    size_t workspace_bytes, int32_t *err_flag, void *stream) {
-    return decode_entry(out, q, kq_cache, vq_cache, k_scale, v_scale, true, block_stride,
+    return decode_entry(out, q, kq_cache, vq_cache, k_scale, v_scale, pkv::kKvInt8, block_stride,
+                        block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
+                        scale, num_splits, workspace, workspace_bytes, err_flag, stream);
+}
+
+int pa_append_kv_fp8(const uint16_t *k_new, const uint16_t *v_new, uint8_t *k8_cache,
+                     uint8_t *v8_cache, int64_t block_stride, const int32_t *block_tables,
+                     int max_blocks_per_seq, const int32_t *positions, int B, int n_new, int Hkv,
+                     int d, int bs, int64_t num_blocks, int64_t *slot_out, int32_t *err_flag,
+                     void *stream) {
+    if (B == 0 || n_new == 0) return PA_OK;
+    if (!k_new || !v_new || !k8_cache || !v8_cache || !block_tables || !positions || !err_flag)
+        return PA_ERR_NULL;
+    int rc = check_common(B, Hkv, d, bs, max_blocks_per_seq, num_blocks, block_stride);
+    if (rc) return rc;
+    if (n_new < 0) return PA_ERR_SHAPE;
+    if (!al16(k_new) || !al16(v_new) || !al16(k8_cache) || !al16(v8_cache) ||
+        block_stride % 16 != 0)
+        return PA_ERR_ALIGN;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    pkv::AppendArgs a{block_tables, positions, slot_out, err_flag, block_stride, num_blocks,
+                      B, n_new, Hkv, d, bs, max_blocks_per_seq};
+    return finish(pkv::launch_append_fp8(k_new, v_new, k8_cache, v8_cache, a, sms,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int pa_decode_fp8(uint16_t *out, const uint16_t *q, const uint8_t *k8_cache,
+                  const uint8_t *v8_cache, int64_t block_stride, const int32_t *block_tables,
+                  int max_blocks_per_seq, const int32_t *ctx_lens, int B, int Hq, int Hkv, int d,
+                  int bs, int64_t num_blocks, float scale, int num_splits, void *workspace,
+                  size_t workspace_bytes, int32_t *err_flag, void *stream) {
+    return decode_entry(out, q, k8_cache, v8_cache, nullptr, nullptr, pkv::kKvFp8, block_stride,
                         block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
                         scale, num_splits, workspace, workspace_bytes, err_flag, stream);
 }
@@ -292,15 +388,15 @@ int pa_decode_static_scratch(uint16_t *out, const uint16_t *q, const uint16_t *k
     int splits = num_splits;
     if (splits == 0) {
         // largest partition count whose scratch fits, starting from the automatic one
-        int auto_s = pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, 0, false, sms).S;
+        int auto_s = pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, 0, pkv::kKvBf16, sms).S;
         int lo = 1, hi = auto_s < 1 ? 1 : auto_s;
-        if (pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, hi, false, sms)
+        if (pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, hi, pkv::kKvBf16, sms)
                 .ws_total <= cap) {
             lo = hi;
         } else {
             while (lo < hi) {  // invariant: ws(lo) fits or lo == 1
                 const int mid = (lo + hi + 1) / 2;
-                if (pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, mid, false, sms)
+                if (pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, mid, pkv::kKvBf16, sms)
                         .ws_total <= cap)
                     lo = mid;
                 else
@@ -309,12 +405,12 @@ int pa_decode_static_scratch(uint16_t *out, const uint16_t *q, const uint16_t *k
         }
         splits = lo;
     }
-    if (pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, splits, false, sms).ws_total >
+    if (pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, splits, pkv::kKvBf16, sms).ws_total >
         cap)
         return PA_ERR_WORKSPACE;
     void *ws = static_scratch_address();
     if (!ws) return PA_ERR_CUDA;
-    return decode_entry(out, q, k_cache, v_cache, nullptr, nullptr, false, block_stride,
+    return decode_entry(out, q, k_cache, v_cache, nullptr, nullptr, pkv::kKvBf16, block_stride,
                         block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
                         scale, splits, ws, cap, err_flag, stream);
 }

@@ -33,7 +33,8 @@ EXPORTED = (
     "pa_status_string", "pa_version", "pa_append_kv", "pa_decode_workspace_bytes", "pa_decode_plan",
     "pa_decode",
     "pe_score_tokens", "pe_select_evict_block", "pa_append_kv_int8", "pa_decode_int8",
-    "pa_decode_static_scratch",
+    "pa_decode_static_scratch", "pa_append_kv_scored", "pa_append_kv_int8_scored",
+    "pe_select_evict_block_pooled", "pa_append_kv_fp8", "pa_decode_fp8",
 )
 
 
@@ -79,6 +80,20 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode_static_scratch.restype = i32
     lib.pa_decode_static_scratch.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32,
                                              i64, f32, i32, p, p]
+    lib.pa_append_kv_scored.restype = i32
+    lib.pa_append_kv_scored.argtypes = [p, p, p, p, i64, p, p, i32, p, i32, i32, i32, i32, i32,
+                                        i64, p, p, p]
+    lib.pa_append_kv_int8_scored.restype = i32
+    lib.pa_append_kv_int8_scored.argtypes = [p, p, p, p, p, p, p, i64, p, i32, p, i32, i32, i32,
+                                             i32, i32, i64, p, p, p]
+    lib.pe_select_evict_block_pooled.restype = i32
+    lib.pe_select_evict_block_pooled.argtypes = [p, p, p, p, i32, p, i32, i32, i32, i64, p, p]
+    lib.pa_append_kv_fp8.restype = i32
+    lib.pa_append_kv_fp8.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, i64, p,
+                                     p, p]
+    lib.pa_decode_fp8.restype = i32
+    lib.pa_decode_fp8.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, i64, f32,
+                                  i32, p, sz, p, p]
     lib.pe_score_tokens.restype = i32
     lib.pe_score_tokens.argtypes = [p, p, p, i64, p, i32, p, i32, i32, i32, i32, i64, p, p]
     lib.pe_select_evict_block.restype = i32
@@ -335,3 +350,145 @@ def pe_select_evict_block(evict, scores, ctx_lens, bs, block_means=None, stream=
                                       _ptr(ctx_lens.contiguous()), B, MB, Hkv, bs,
                                       _stream(stream))
     _check("pe_select_evict_block", rc)
+
+
+# ----------------------------------------------------------------------------- incremental scores
+def _score_pool_check(score_pool, N, bs, Hkv):
+    _want(score_pool, torch.float32, "score_pool")
+    if tuple(score_pool.shape) != (N, bs, Hkv) or not score_pool.is_contiguous():
+        raise ValueError("score_pool must be contiguous [N, bs, Hkv] float32")
+
+
+def pa_append_kv_scored(k_new, v_new, k_cache, v_cache, score_pool, block_tables, positions,
+                        err_flag, slot_out=None, stream=None):
+    """pa_append_kv that also writes each new (token, kv head) importance
+    ||V|| / ||K|| into score_pool [N, bs, Hkv] (paged like the KV pool)."""
+    for t, n in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _want(t, torch.bfloat16, n)
+    _want(block_tables, torch.int32, "block_tables")
+    _want(positions, torch.int32, "positions")
+    _want(err_flag, torch.int32, "err_flag")
+    N, bs, Hkv, d, stride = _pool_geometry(k_cache, "k_cache")
+    _same_pool(k_cache, v_cache)
+    _score_pool_check(score_pool, N, bs, Hkv)
+    if k_new.dim() == 3:
+        k_new, v_new = k_new.unsqueeze(1), v_new.unsqueeze(1)
+    if not (k_new.is_contiguous() and v_new.is_contiguous()) or k_new.shape != v_new.shape:
+        raise ValueError("k_new/v_new must be contiguous and of equal shape")
+    B, n_new = k_new.shape[0], k_new.shape[1]
+    if slot_out is not None:
+        _want(slot_out, torch.int64, "slot_out")
+    bt = block_tables.contiguous()
+    rc = load().pa_append_kv_scored(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                    stride, _ptr(score_pool), _ptr(bt), bt.shape[1],
+                                    _ptr(positions.contiguous()), B, n_new, Hkv, d, bs, N,
+                                    _ptr(slot_out), _ptr(err_flag), _stream(stream))
+    _check("pa_append_kv_scored", rc)
+
+
+def pa_append_kv_int8_scored(k_new, v_new, kq_cache, vq_cache, k_scale, v_scale, score_pool,
+                             block_tables, positions, err_flag, slot_out=None, stream=None):
+    """pa_append_kv_int8 that also stores the importance of each dequantised
+    new row into score_pool [N, bs, Hkv]."""
+    _want(k_new, torch.bfloat16, "k_new")
+    _want(v_new, torch.bfloat16, "v_new")
+    _want(kq_cache, torch.int8, "kq_cache")
+    _want(vq_cache, torch.int8, "vq_cache")
+    _want(k_scale, torch.float32, "k_scale")
+    _want(v_scale, torch.float32, "v_scale")
+    _want(block_tables, torch.int32, "block_tables")
+    _want(positions, torch.int32, "positions")
+    _want(err_flag, torch.int32, "err_flag")
+    N, bs, Hkv, d, stride = _pool_geometry(kq_cache, "kq_cache")
+    _same_pool(kq_cache, vq_cache)
+    for sp in (k_scale, v_scale):
+        if tuple(sp.shape) != (N, bs, Hkv) or not sp.is_contiguous():
+            raise ValueError("scale pools must be contiguous [N, bs, Hkv]")
+    _score_pool_check(score_pool, N, bs, Hkv)
+    if k_new.dim() == 3:
+        k_new, v_new = k_new.unsqueeze(1), v_new.unsqueeze(1)
+    if not (k_new.is_contiguous() and v_new.is_contiguous()) or k_new.shape != v_new.shape:
+        raise ValueError("k_new/v_new must be contiguous and of equal shape")
+    B, n_new = k_new.shape[0], k_new.shape[1]
+    if slot_out is not None:
+        _want(slot_out, torch.int64, "slot_out")
+    bt = block_tables.contiguous()
+    rc = load().pa_append_kv_int8_scored(_ptr(k_new), _ptr(v_new), _ptr(kq_cache),
+                                         _ptr(vq_cache), _ptr(k_scale), _ptr(v_scale),
+                                         _ptr(score_pool), stride, _ptr(bt), bt.shape[1],
+                                         _ptr(positions.contiguous()), B, n_new, Hkv, d, bs, N,
+                                         _ptr(slot_out), _ptr(err_flag), _stream(stream))
+    _check("pa_append_kv_int8_scored", rc)
+
+
+def pe_select_evict_block_pooled(evict, score_pool, block_tables, ctx_lens, err_flag,
+                                 block_means=None, stream=None):
+    """Lowest-mean full block per sequence, scores read from score_pool
+    [N, bs, Hkv] through the block table (no K/V pass)."""
+    _want(evict, torch.int32, "evict")
+    _want(score_pool, torch.float32, "score_pool")
+    _want(block_tables, torch.int32, "block_tables")
+    _want(ctx_lens, torch.int32, "ctx_lens")
+    _want(err_flag, torch.int32, "err_flag")
+    N, bs, Hkv = score_pool.shape
+    if not score_pool.is_contiguous():
+        raise ValueError("score_pool must be contiguous")
+    bt = block_tables.contiguous()
+    B, MB = bt.shape
+    if block_means is not None:
+        _want(block_means, torch.float32, "block_means")
+        if tuple(block_means.shape) != (B, MB) or not block_means.is_contiguous():
+            raise ValueError("block_means must be contiguous [B, MB]")
+    rc = load().pe_select_evict_block_pooled(_ptr(evict), _ptr(block_means), _ptr(score_pool),
+                                             _ptr(bt), MB, _ptr(ctx_lens.contiguous()), B, Hkv,
+                                             bs, N, _ptr(err_flag), _stream(stream))
+    _check("pe_select_evict_block_pooled", rc)
+
+
+# ----------------------------------------------------------------------------- fp8
+def pa_append_kv_fp8(k_new, v_new, k8_cache, v8_cache, block_tables, positions, err_flag,
+                     slot_out=None, stream=None):
+    """Cast new tokens to e4m3 (round to nearest even, saturating at 448) and
+    write them.  Pools [N, bs, Hkv, d] uint8 holding e4m3 codes."""
+    _want(k_new, torch.bfloat16, "k_new")
+    _want(v_new, torch.bfloat16, "v_new")
+    _want(k8_cache, torch.uint8, "k8_cache")
+    _want(v8_cache, torch.uint8, "v8_cache")
+    _want(block_tables, torch.int32, "block_tables")
+    _want(positions, torch.int32, "positions")
+    _want(err_flag, torch.int32, "err_flag")
+    N, bs, Hkv, d, stride = _pool_geometry(k8_cache, "k8_cache")
+    _same_pool(k8_cache, v8_cache)
+    if k_new.dim() == 3:
+        k_new, v_new = k_new.unsqueeze(1), v_new.unsqueeze(1)
+    if not (k_new.is_contiguous() and v_new.is_contiguous()) or k_new.shape != v_new.shape:
+        raise ValueError("k_new/v_new must be contiguous and of equal shape")
+    B, n_new = k_new.shape[0], k_new.shape[1]
+    if slot_out is not None:
+        _want(slot_out, torch.int64, "slot_out")
+    bt = block_tables.contiguous()
+    rc = load().pa_append_kv_fp8(_ptr(k_new), _ptr(v_new), _ptr(k8_cache), _ptr(v8_cache), stride,
+                                 _ptr(bt), bt.shape[1], _ptr(positions.contiguous()), B, n_new,
+                                 Hkv, d, bs, N, _ptr(slot_out), _ptr(err_flag), _stream(stream))
+    _check("pa_append_kv_fp8", rc)
+
+
+def pa_decode_fp8(out, q, k8_cache, v8_cache, block_tables, ctx_lens, scale, err_flag,
+                  workspace=None, num_splits=0, stream=None):
+    """Paged decode attention over e4m3 pools, widened exactly in registers."""
+    _decode_checks(out, q, block_tables, ctx_lens, err_flag)
+    _want(k8_cache, torch.uint8, "k8_cache")
+    _want(v8_cache, torch.uint8, "v8_cache")
+    N, bs, Hkv, d, stride = _pool_geometry(k8_cache, "k8_cache")
+    _same_pool(k8_cache, v8_cache)
+    B, Hq, dq = q.shape
+    if dq != d:
+        raise ValueError("q head_dim differs from the pool's")
+    bt = block_tables.contiguous()
+    ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel() *
+                                                        workspace.element_size())
+    rc = load().pa_decode_fp8(_ptr(out), _ptr(q), _ptr(k8_cache), _ptr(v8_cache), stride,
+                              _ptr(bt), bt.shape[1], _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d,
+                              bs, N, float(scale), int(num_splits), ws_ptr, ws_n, _ptr(err_flag),
+                              _stream(stream))
+    _check("pa_decode_fp8", rc)

@@ -50,6 +50,7 @@ class Config:
     append: bool = True             # one new token appended per sequence per layer
     score: bool = False             # step includes the PagedEviction score + argmin
     int8: bool = False
+    fp8: bool = False               # e4m3 pools (history cast by the FP8 append)
     outlier_frac: float = 0.0
     spare: float = 0.10
     nano_layout: bool = False       # K/V in one [2, L, N, bs, Hkv, d] tensor
@@ -169,8 +170,8 @@ def generate(cfg: Config, device="cpu", layers: Optional[int] = None,
             outliers.append([(int(c) // d, int(c) % d) for c in ch])
         else:
             outliers.append([])
-    if cfg.int8:
-        # history drawn in bf16, quantised later by the INT8 append
+    if cfg.int8 or cfg.fp8:
+        # history drawn in bf16, quantised later by the INT8 / FP8 append
         k_hist = randn(L, B, int(old.max()), Hkv, d)
         v_hist = randn(L, B, int(old.max()), Hkv, d)
     else:

@@ -73,7 +73,10 @@ class Device:
         self.v_new = None if wl.v_new is None else wl.v_new.to(dev)
         L, B = self.q.shape[0], cfg.batch
         N, bs, Hkv, d = wl.num_blocks, cfg.block_size, cfg.hkv, cfg.head_dim
-        if cfg.int8:
+        if cfg.fp8:
+            self.k8 = torch.zeros(L, N, bs, Hkv, d, dtype=torch.uint8, device=dev)
+            self.v8 = torch.zeros_like(self.k8)
+        elif cfg.int8:
             self.kq = torch.zeros(L, N, bs, Hkv, d, dtype=torch.int8, device=dev)
             self.vq = torch.zeros_like(self.kq)
             self.ks = torch.zeros(L, N, bs, Hkv, dtype=torch.float32, device=dev)
@@ -90,28 +93,41 @@ class Device:
         self.ws = pk.alloc_workspace(B, cfg.hq, Hkv, d, bs, wl.max_blocks, num_splits, dev)
         self.slots = torch.full((B, 1), -7, dtype=torch.int64, device=dev)
 
+    def _append_hist(self, layer, k, v, bt, pos):
+        if self.wl.cfg.fp8:
+            pk.pa_append_kv_fp8(k, v, self.k8[layer], self.v8[layer], bt, pos, self.err)
+        else:
+            pk.pa_append_kv_int8(k, v, self.kq[layer], self.vq[layer], self.ks[layer],
+                                 self.vs[layer], bt, pos, self.err)
+
     def fill_int8_history(self, layer):
+        """Quantise the bf16 history into the INT8 (or FP8) pools with the append."""
         wl = self.wl
         zeros = torch.zeros(wl.cfg.batch, dtype=torch.int32, device=self.dev)
         kh, vh = wl.k_hist[layer].to(self.dev), wl.v_hist[layer].to(self.dev)
         if (wl.old_lens == wl.old_lens[0]).all():
-            pk.pa_append_kv_int8(kh[:, :int(wl.old_lens[0])].contiguous(),
-                                 vh[:, :int(wl.old_lens[0])].contiguous(), self.kq[layer],
-                                 self.vq[layer], self.ks[layer], self.vs[layer], self.bt, zeros,
-                                 self.err)
+            n = int(wl.old_lens[0])
+            self._append_hist(layer, kh[:, :n].contiguous(), vh[:, :n].contiguous(), self.bt,
+                              zeros)
         else:
             for b in range(wl.cfg.batch):
                 n = int(wl.old_lens[b])
                 if n == 0:
                     continue
-                pk.pa_append_kv_int8(kh[b:b + 1, :n].contiguous(), vh[b:b + 1, :n].contiguous(),
-                                     self.kq[layer], self.vq[layer], self.ks[layer],
-                                     self.vs[layer], self.bt[b:b + 1], zeros[b:b + 1], self.err)
+                self._append_hist(layer, kh[b:b + 1, :n].contiguous(),
+                                  vh[b:b + 1, :n].contiguous(), self.bt[b:b + 1], zeros[b:b + 1])
 
     def step(self, layer, score=False):
         """append (when the workload appends) then decode; optional score+select."""
         cfg = self.wl.cfg
-        if cfg.int8:
+        if cfg.fp8:
+            if self.k_new is not None:
+                pk.pa_append_kv_fp8(self.k_new[layer], self.v_new[layer], self.k8[layer],
+                                    self.v8[layer], self.bt, self.pos, self.err,
+                                    slot_out=self.slots)
+            pk.pa_decode_fp8(self.out[layer], self.q[layer], self.k8[layer], self.v8[layer],
+                             self.bt, self.ctx, self.wl.scale, self.err, self.ws, self.num_splits)
+        elif cfg.int8:
             if self.k_new is not None:
                 pk.pa_append_kv_int8(self.k_new[layer], self.v_new[layer], self.kq[layer],
                                      self.vq[layer], self.ks[layer], self.vs[layer], self.bt,
@@ -149,7 +165,22 @@ def oracle_step(wl: W.Workload, layer: int, seqs, score=False):
     stride = bs * Hkv * d
     n = s["num_blocks"]
     res = {"ctx_lens": s["ctx_lens"]}
-    if cfg.int8:
+    if cfg.fp8:
+        k8 = np.zeros(n * stride, np.uint8)
+        v8 = np.zeros_like(k8)
+        zeros = np.zeros(len(s["ctx_lens"]), np.int32)
+        for r in range(len(s["ctx_lens"])):
+            m = int(s["old_lens"][r])
+            if m:
+                oracle.append_kv_fp8(s["k_hist"][r:r + 1, :m], s["v_hist"][r:r + 1, :m], k8, v8,
+                                     stride, s["block_tables"][r:r + 1], zeros[r:r + 1], bs)
+        if "k_new" in s:
+            res["slots"] = oracle.append_kv_fp8(s["k_new"], s["v_new"], k8, v8, stride,
+                                                s["block_tables"], s["positions"], bs)
+        res["out"] = oracle.paged_decode_fp8(s["q"], k8, v8, stride, s["block_tables"],
+                                             s["ctx_lens"], Hkv, bs, wl.scale)
+        res.update(k8=k8, v8=v8)
+    elif cfg.int8:
         kq = np.zeros(n * stride, np.int8)
         vq = np.zeros_like(kq)
         ks = np.zeros(n * bs * Hkv, np.float32)

@@ -36,6 +36,14 @@ MEDIUM = {
     "i8g16": W.scaled(C["c5"], key="i8g16", batch=3, hq=64, hkv=4, old_lens=(100, 37, 300)),
     # INT8 with d = 64: the general-shape kernel
     "i8d64": W.scaled(C["c5"], key="i8d64", batch=3, head_dim=64, old_lens=(70, 5, 200)),
+    # FP8 (e4m3) pools: staged kernel (d = 128), G = 16 with two sub-tiles per stage, and the
+    # general kernel (d = 64)
+    "f8": W.scaled(C["c5"], key="f8", int8=False, fp8=True, batch=5,
+                   old_lens=(300, 1, 16, 255, 512)),
+    "f8g16": W.scaled(C["c5"], key="f8g16", int8=False, fp8=True, batch=3, hq=64, hkv=4,
+                      old_lens=(100, 37, 300)),
+    "f8d64": W.scaled(C["c5"], key="f8d64", int8=False, fp8=True, batch=3, head_dim=64,
+                      old_lens=(70, 5, 200)),
 }
 
 
@@ -94,10 +102,12 @@ def test_medium_workloads(key):
 
 
 @pytest.mark.parametrize("num_splits", [1, 2, 3, 8, 0])
-@pytest.mark.parametrize("kv", ["bf16", "int8"])
+@pytest.mark.parametrize("kv", ["bf16", "int8", "fp8"])
 def test_split_count_invariance(num_splits, kv):
     base = C["c3"] if kv == "bf16" else C["c5"]
     cfg = W.scaled(base, key="split", layers=1, batch=3, old_lens=(2000, 700, 45))
+    if kv == "fp8":
+        cfg = W.scaled(cfg, int8=False, fp8=True)
     wl = W.generate(cfg, "cpu")
     _parity(wl, [0], num_splits=num_splits)
 
@@ -235,3 +245,15 @@ def test_select_evict_bit_exact_on_given_scores():
     assert np.array_equal(np.isnan(gmn), np.isnan(means))
     ok = ~np.isnan(means)
     assert np.array_equal(gmn[ok], means[ok].astype(np.float32))
+
+
+def test_fp8_codes_bit_exact():
+    wl = W.generate(MEDIUM["f8"], "cpu")
+    ref = oracle_step(wl, 0, range(wl.cfg.batch))
+    dev = Device(wl)
+    dev.fill_int8_history(0)
+    dev.step(0)
+    torch.cuda.synchronize()
+    ids = torch.as_tensor(wl.block_tables[wl.block_tables >= 0], device="cuda")
+    assert np.array_equal(dev.k8[0][ids].cpu().numpy().ravel(), ref["k8"])
+    assert np.array_equal(dev.v8[0][ids].cpu().numpy().ravel(), ref["v8"])
