@@ -56,6 +56,14 @@ def _lib():
         lib.or_quantize_int8.argtypes = [p, i64, i32, p, p]
         lib.or_quantize_e4m3.restype = None
         lib.or_quantize_e4m3.argtypes = [p, i64, p]
+        lib.or_prefill_scores.restype = None
+        lib.or_prefill_scores.argtypes = [p, p, p, i64, i32, i32]
+        lib.or_prefill_select.restype = None
+        lib.or_prefill_select.argtypes = [p, p, p, p, i32, i32]
+        lib.or_prefill_pack.restype = None
+        lib.or_prefill_pack.argtypes = [p, p, p, p, p, i32, p, p, i64, p, i32, i32, i32, i32, i32]
+        lib.or_evict_compact.restype = None
+        lib.or_evict_compact.argtypes = [p, p, p, p, i32, i32, i32]
         lib.or_e4m3_to_f64.restype = dbl
         lib.or_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         lib.or_append_kv_fp8.restype = None
@@ -270,3 +278,59 @@ def paged_decode_fp8(q, k_cache, v_cache, block_stride, bt, ctx_lens, Hkv, bs, s
     _lib().or_paged_decode_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), block_stride,
                                _ptr(bt), bt.shape[1], _ptr(ctx_lens), B, Hq, Hkv, d, bs, scale)
     return out
+
+
+# --------------------------------------------------------------------------- prefill stage
+def prefill_scores(k, v):
+    """Token importance at prefill ([KVL] PagedEviction two-stage strategy): the
+    mean over kv heads of ||V||/||K||.  k, v [T, Hkv, d] bf16 bits -> [T] float64."""
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    T, Hkv, d = k.shape
+    scores = np.empty(T, np.float64)
+    _lib().or_prefill_scores(_ptr(scores), _ptr(k), _ptr(v), T, Hkv, d)
+    return scores
+
+
+def prefill_select(scores, cu, budget):
+    """Keep set per prompt: the `budget` highest-ranking tokens in prompt order
+    (ties evict the earlier token; NaN ranks as -inf).  scores [T] (any float
+    dtype, widened to fp64), cu [B+1].  Returns (keep_idx [B, budget] int32,
+    -1 after the last kept token; kept_len [B] int32)."""
+    scores = np.ascontiguousarray(scores, dtype=np.float64)
+    cu = _c(cu, np.int32)
+    B = cu.size - 1
+    keep = np.empty((B, budget), np.int32)
+    kept = np.empty(B, np.int32)
+    _lib().or_prefill_select(_ptr(keep), _ptr(kept), _ptr(scores), _ptr(cu), B, budget)
+    return keep, kept
+
+
+def prefill_pack(k, v, cu, keep_idx, kept_len, k_cache, v_cache, block_stride, bt, bs):
+    """Write the kept prompt rows at positions 0.. of each sequence through the
+    block table (pools flat uint16, modified in place)."""
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    cu = _c(cu, np.int32)
+    keep_idx = _c(keep_idx, np.int32)
+    kept_len = _c(kept_len, np.int32)
+    bt = _c(bt, np.int32)
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    assert k_cache.dtype == np.uint16 and v_cache.dtype == np.uint16
+    T, Hkv, d = k.shape
+    B, MB = bt.shape
+    _lib().or_prefill_pack(_ptr(k), _ptr(v), _ptr(cu), _ptr(keep_idx), _ptr(kept_len),
+                           keep_idx.shape[1], _ptr(k_cache), _ptr(v_cache), block_stride,
+                           _ptr(bt), MB, B, Hkv, d, bs)
+
+
+def evict_compact(bt, ctx_lens, evict, bs):
+    """Remove the evicted logical block from each table.  Returns new copies
+    (bt [B, MB] int32, ctx_lens [B] int32, freed [B] int32)."""
+    bt = np.array(bt, dtype=np.int32, order="C", copy=True)
+    ctx = np.array(ctx_lens, dtype=np.int32, copy=True)
+    evict = _c(evict, np.int32)
+    B, MB = bt.shape
+    freed = np.empty(B, np.int32)
+    _lib().or_evict_compact(_ptr(bt), _ptr(ctx), _ptr(freed), _ptr(evict), B, MB, bs)
+    return bt, ctx, freed

@@ -457,3 +457,124 @@ void or_paged_decode_fp8(double *out, const uint16_t *q, const uint8_t *k_cache,
     decode_common(out, q, k_cache, v_cache, NULL, NULL, load_fp8, block_stride, 0, bt, MB,
                   ctx_lens, B, Hq, Hkv, d, bs, scale);
 }
+
+/* ------------------------------------------------------------------------ */
+/* PagedEviction prefill stage and block-table compaction                    */
+/* ------------------------------------------------------------------------ */
+
+/* Prefill token importance ([KVL] "PagedEviction 块级驱逐机制", the two-stage
+ * strategy: at prefill every token is scored and the lowest-scoring tokens are
+ * evicted down to the cache budget).  Reading: one slot holds a token for all
+ * kv heads, so a token is kept or evicted as a whole and its importance is the
+ * mean over the Hkv heads of the per-head ratio ||V||/||K|| (zero rule as in
+ * norm_ratio); this is the same per-entry average the decode-phase block mean
+ * takes.  k, v [T][Hkv][d] bf16 bits (the prompt rows, token-major); scores [T]. */
+void or_prefill_scores(double *scores, const uint16_t *k, const uint16_t *v, int64_t T, int Hkv,
+                       int d) {
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double sum = 0.0;
+        for (int h = 0; h < Hkv; ++h) {
+            const int64_t base = (t * Hkv + h) * (int64_t)d;
+            double kk = 0.0, vv = 0.0;
+            for (int e = 0; e < d; ++e) {
+                const double x = bf16_to_f64(k[base + e]), y = bf16_to_f64(v[base + e]);
+                kk += x * x;
+                vv += y * y;
+            }
+            sum += norm_ratio(kk, vv);
+        }
+        scores[t] = sum / (double)Hkv;
+    }
+}
+
+/* Value order used by the keep decision: numeric, NaN counted as -inf, -0 equal
+ * to +0; equal values are ordered by token index, the later token ranking higher. */
+static double rank_value(double x) { return x != x ? -INFINITY : x; }
+
+typedef struct {
+    double s;
+    int32_t i;
+} scored_token;
+
+/* qsort comparator: best first (higher value, then higher index). */
+static int best_first(const void *pa, const void *pb) {
+    const scored_token *a = (const scored_token *)pa, *b = (const scored_token *)pb;
+    if (a->s != b->s) return a->s > b->s ? -1 : 1;
+    return a->i > b->i ? -1 : (a->i < b->i ? 1 : 0);
+}
+
+static int by_index(const void *pa, const void *pb) {
+    const int32_t a = *(const int32_t *)pa, b = *(const int32_t *)pb;
+    return (a > b) - (a < b);
+}
+
+/* Prefill keep set ([KVL] two-stage strategy, prefill side).  Readings: the
+ * `budget` tokens that rank highest stay, all others are evicted; on equal
+ * importance the earlier token goes first (the decode-side argmin also takes the
+ * lowest index on ties); a prompt of n <= budget tokens keeps every token; kept
+ * tokens keep their prompt order.
+ * scores: one value per prompt token, prompts concatenated; cu [B+1] offsets;
+ * keep_idx [B][budget]: prompt-local index of the p-th kept token, -1 after the
+ * last; kept_len [B] = min(n_b, budget). */
+void or_prefill_select(int32_t *keep_idx, int32_t *kept_len, const double *scores,
+                       const int32_t *cu, int B, int budget) {
+    for (int b = 0; b < B; ++b) {
+        const int n = cu[b + 1] - cu[b];
+        const int kept = n < budget ? n : budget;
+        scored_token *tok = (scored_token *)malloc(sizeof(scored_token) * (size_t)(n > 0 ? n : 1));
+        for (int i = 0; i < n; ++i) {
+            tok[i].s = rank_value(scores[cu[b] + i]);
+            tok[i].i = i;
+        }
+        qsort(tok, (size_t)n, sizeof(scored_token), best_first);
+        int32_t *row = keep_idx + (int64_t)b * budget;
+        for (int p = 0; p < budget; ++p) row[p] = p < kept ? tok[p].i : -1;
+        qsort(row, (size_t)kept, sizeof(int32_t), by_index);
+        kept_len[b] = kept;
+        free(tok);
+    }
+}
+
+/* Packing the kept prompt tokens into the paged pool: the p-th kept token of
+ * sequence b is written at position p through the block table ([VKV] §2.1,
+ * slot = bt[b][p/bs]*bs + p%bs), so the compressed prompt fills its blocks
+ * densely and only the last one may be partial.  k, v [T][Hkv][d] bf16 bits
+ * (prompts concatenated, offsets cu); pools [N][bs][Hkv][d]. */
+void or_prefill_pack(const uint16_t *k, const uint16_t *v, const int32_t *cu,
+                     const int32_t *keep_idx, const int32_t *kept_len, int budget,
+                     uint16_t *k_cache, uint16_t *v_cache, int64_t block_stride,
+                     const int32_t *bt, int MB, int B, int Hkv, int d, int bs) {
+    const int64_t row = (int64_t)Hkv * d;
+    for (int b = 0; b < B; ++b) {
+        for (int p = 0; p < kept_len[b]; ++p) {
+            const int64_t src = ((int64_t)cu[b] + keep_idx[(int64_t)b * budget + p]) * row;
+            const int64_t slot = or_slot(bt + (int64_t)b * MB, p, bs);
+            const int64_t dst = (slot / bs) * block_stride + (slot % bs) * row;
+            memcpy(k_cache + dst, k + src, (size_t)row * sizeof(uint16_t));
+            memcpy(v_cache + dst, v + src, (size_t)row * sizeof(uint16_t));
+        }
+    }
+}
+
+/* Block-table compaction after a decode-phase eviction ([KVL]: eviction drops a
+ * whole block, so no partially filled block is left behind).  Reading: logical
+ * block j = evict[b] leaves sequence b's table, the entries after it move down
+ * by one, the last used entry becomes -1, the context length drops by bs and the
+ * freed physical id is returned in freed[b].  evict[b] < 0, or an index that is
+ * not a full block, leaves the sequence unchanged (freed[b] = -1).  Physical blocks do not move, so the cached rows
+ * and any per-slot data stay where they are. */
+void or_evict_compact(int32_t *bt, int32_t *ctx_lens, int32_t *freed, const int32_t *evict,
+                      int B, int MB, int bs) {
+    for (int b = 0; b < B; ++b) {
+        int32_t *row = bt + (int64_t)b * MB;
+        const int j = evict[b];
+        freed[b] = -1;
+        if (j < 0 || j >= ctx_lens[b] / bs) continue;   /* only full blocks are candidates */
+        const int nblk = (int)or_num_blocks(ctx_lens[b], bs);
+        freed[b] = row[j];
+        for (int x = j; x < nblk - 1; ++x) row[x] = row[x + 1];
+        row[nblk - 1] = -1;
+        ctx_lens[b] -= bs;
+    }
+}

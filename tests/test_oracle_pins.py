@@ -538,3 +538,176 @@ def test_fp8_decode_equals_sdpa_on_decoded_values():
         o = torch.nn.functional.scaled_dot_product_attention(
             torch.from_numpy(q[b]).unsqueeze(1), Kt, Vt, scale=1 / math.sqrt(d))[:, 0].numpy()
         np.testing.assert_allclose(out[b], o, rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- prefill stage
+def test_prefill_score_closed_forms():
+    """V = c_h K in head h gives a token score of mean_h |c_h|; K = 0 with V != 0
+    gives +inf; K = V = 0 gives 0."""
+    rng = np.random.default_rng(11)
+    T, Hkv, d = 5, 4, 32
+    k = rng.standard_normal((T, Hkv, d))
+    c = np.array([0.5, -2.0, 0.25, 4.0])          # powers of two: c*K stays exact in bf16
+    kb = bf16_bits(k)
+    v = bf16_vals(kb).reshape(T, Hkv, d) * c[None, :, None]
+    s = oracle.prefill_scores(kb.reshape(T, Hkv, d), bf16_bits(v).reshape(T, Hkv, d))
+    assert np.allclose(s, np.abs(c).mean(), rtol=1e-15, atol=0)
+    z = np.zeros((1, Hkv, d))
+    one = np.ones((1, Hkv, d))
+    assert oracle.prefill_scores(bf16_bits(z).reshape(1, Hkv, d),
+                                 bf16_bits(one).reshape(1, Hkv, d))[0] == math.inf
+    assert oracle.prefill_scores(bf16_bits(z).reshape(1, Hkv, d),
+                                 bf16_bits(z).reshape(1, Hkv, d))[0] == 0.0
+
+
+def test_prefill_score_is_head_mean_of_paged_score():
+    """Written into a pool by the (pinned) append, the per-(token, head) paged
+    scores averaged over heads equal the prefill scores."""
+    rng = np.random.default_rng(12)
+    T, Hkv, d, bs = 37, 2, 16, 8
+    k = bf16_bits(rng.standard_normal((1, T, Hkv, d)))
+    v = bf16_bits(rng.standard_normal((1, T, Hkv, d)) * 3)
+    nb = -(-T // bs)
+    bt = rng.permutation(nb).astype(np.int32)[None, :]
+    stride = bs * Hkv * d
+    kc = np.zeros(nb * stride, np.uint16)
+    vc = np.zeros_like(kc)
+    oracle.append_kv(k, v, kc, vc, stride, bt, np.zeros(1, np.int32), bs)
+    paged = oracle.score_tokens(kc, vc, stride, bt, np.array([T], np.int32), Hkv, d, bs)
+    s = oracle.prefill_scores(k[0], v[0])
+    assert np.allclose(s, paged[0, :T].mean(axis=1), rtol=1e-14, atol=0)
+
+
+def _keep_by_subsets(scores, budget):
+    """Brute force: the unique kept set K of size budget such that every kept
+    token outranks every evicted one, ranking by (value, index)."""
+    import itertools
+    n = len(scores)
+    if n <= budget:
+        return list(range(n))
+    key = [((-math.inf if s != s else s), i) for i, s in enumerate(scores)]
+    found = [c for c in itertools.combinations(range(n), budget)
+             if min(key[i] for i in c) > max(key[i] for i in range(n) if i not in c)]
+    assert len(found) == 1
+    return list(found[0])
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_prefill_select_brute_force_over_subsets(seed):
+    rng = np.random.default_rng(100 + seed)
+    lens = [9, 3, 0, 7, 8]
+    budget = 4
+    # few distinct values: many ties
+    vals = np.array([0.5, 1.0, 2.0, math.inf, math.nan, 0.0])
+    scores = rng.choice(vals, size=sum(lens))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    keep, kept = oracle.prefill_select(scores, cu, budget)
+    for b, n in enumerate(lens):
+        want = _keep_by_subsets(list(scores[cu[b]:cu[b + 1]]), budget)
+        assert kept[b] == len(want)
+        assert keep[b, :kept[b]].tolist() == want
+        assert (keep[b, kept[b]:] == -1).all()
+
+
+def test_prefill_select_closed_forms():
+    cu = np.array([0, 10], np.int32)
+    inc = np.arange(10, dtype=np.float64)
+    assert oracle.prefill_select(inc, cu, 4)[0][0].tolist() == [6, 7, 8, 9]
+    assert oracle.prefill_select(inc[::-1].copy(), cu, 4)[0][0].tolist() == [0, 1, 2, 3]
+    # all equal: the latest tokens stay
+    assert oracle.prefill_select(np.ones(10), cu, 3)[0][0].tolist() == [7, 8, 9]
+    # planted low-importance tokens are the ones that go
+    s = np.full(10, 2.0)
+    s[[1, 4, 8]] = 0.1
+    assert oracle.prefill_select(s, cu, 7)[0][0].tolist() == [0, 2, 3, 5, 6, 7, 9]
+    # budget >= n keeps every token in order
+    keep, kept = oracle.prefill_select(np.random.default_rng(0).random(10), cu, 16)
+    assert kept[0] == 10 and keep[0, :10].tolist() == list(range(10))
+    # -0 and +0 tie (index decides), NaN ranks below -inf... as -inf (index decides)
+    s = np.array([0.0, -0.0, math.nan, -math.inf, 1.0])
+    assert oracle.prefill_select(s, np.array([0, 5], np.int32), 3)[0][0].tolist() == [0, 1, 4]
+    assert oracle.prefill_select(s, np.array([0, 5], np.int32), 4)[0][0].tolist() == [0, 1, 3, 4]
+
+
+def test_prefill_pack_keep_all_equals_append():
+    """With budget >= n the pack is the plain append of every prompt row."""
+    rng = np.random.default_rng(13)
+    lens = [5, 17, 16]
+    Hkv, d, bs = 2, 8, 4
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    k = bf16_bits(rng.standard_normal((T, Hkv, d))).reshape(T, Hkv, d)
+    v = bf16_bits(rng.standard_normal((T, Hkv, d))).reshape(T, Hkv, d)
+    MB = max(-(-n // bs) for n in lens)
+    N = 20
+    perm = rng.permutation(N).astype(np.int32)
+    bt = np.full((3, MB), -1, np.int32)
+    c = 0
+    for b, n in enumerate(lens):
+        for j in range(-(-n // bs)):
+            bt[b, j] = perm[c]
+            c += 1
+    stride = bs * Hkv * d
+    kc1 = np.zeros(N * stride, np.uint16); vc1 = np.zeros_like(kc1)
+    kc2 = np.zeros_like(kc1); vc2 = np.zeros_like(kc1)
+    keep, kept = oracle.prefill_select(oracle.prefill_scores(k, v), cu, 64)
+    oracle.prefill_pack(k, v, cu, keep, kept, kc1, vc1, stride, bt, bs)
+    for b, n in enumerate(lens):
+        oracle.append_kv(k[None, cu[b]:cu[b + 1]], v[None, cu[b]:cu[b + 1]], kc2, vc2, stride,
+                         bt[b:b + 1], np.zeros(1, np.int32), bs)
+    assert np.array_equal(kc1, kc2) and np.array_equal(vc1, vc2)
+
+
+def test_prefill_pack_places_kept_rows_densely():
+    """Logical gather of the packed pool returns exactly the kept rows in order."""
+    rng = np.random.default_rng(14)
+    lens = [23]
+    Hkv, d, bs, budget = 1, 4, 4, 10
+    cu = np.array([0, 23], np.int32)
+    k = bf16_bits(rng.standard_normal((23, Hkv, d))).reshape(23, Hkv, d)
+    v = bf16_bits(rng.standard_normal((23, Hkv, d))).reshape(23, Hkv, d)
+    keep, kept = oracle.prefill_select(oracle.prefill_scores(k, v), cu, budget)
+    bt = np.array([[5, 1, 3]], np.int32)
+    stride = bs * Hkv * d
+    kc = np.zeros(6 * stride, np.uint16); vc = np.zeros_like(kc)
+    oracle.prefill_pack(k, v, cu, keep, kept, kc, vc, stride, bt, bs)
+    for p in range(budget):
+        blk, off = bt[0, p // bs], p % bs
+        row = kc[blk * stride + off * Hkv * d: blk * stride + (off + 1) * Hkv * d]
+        assert np.array_equal(row, k[keep[0, p]].ravel())
+    # the two unused slots of the last block stay untouched
+    assert not kc[3 * stride + 2 * d:3 * stride + 4 * d].any()
+
+
+def test_evict_compact_preserves_token_to_slot_map():
+    """Every token outside the evicted block keeps its physical slot, at a
+    logical position bs lower when it came after the block; the freed id is the
+    evicted block's; the table entries plus freed ids are a permutation of the old."""
+    rng = np.random.default_rng(15)
+    bs, MB = 4, 6
+    lens = np.array([24, 17, 4, 3, 9], np.int32)
+    evict = np.array([2, 0, 0, 0, 3], np.int32)      # seq 3 has no full block; 3 >= 9 // 4
+    N = 40
+    perm = rng.permutation(N).astype(np.int32)
+    bt = np.full((5, MB), -1, np.int32)
+    c = 0
+    for b, n in enumerate(lens):
+        for j in range(-(-int(n) // bs)):
+            bt[b, j] = perm[c]
+            c += 1
+    nbt, nlen, freed = oracle.evict_compact(bt, lens, evict, bs)
+    for b in range(5):
+        j = int(evict[b])
+        if not 0 <= j < lens[b] // bs:
+            assert freed[b] == -1 and nlen[b] == lens[b] and (nbt[b] == bt[b]).all()
+            continue
+        assert freed[b] == bt[b, j] and nlen[b] == lens[b] - bs
+        for p in range(lens[b]):
+            if j * bs <= p < (j + 1) * bs:
+                continue
+            q = p - bs if p >= (j + 1) * bs else p
+            assert oracle.slot(nbt[b], q, bs) == oracle.slot(bt[b], p, bs)
+        old = sorted(x for x in bt[b] if x >= 0)
+        new = sorted([x for x in nbt[b] if x >= 0] + [int(freed[b])])
+        assert old == new
+        assert (nbt[b, -(-int(nlen[b]) // bs):] == -1).all()
