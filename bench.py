@@ -41,7 +41,7 @@ from paged_kv_cache_396_b200 import workloads as W  # noqa: E402
 
 METRIC = "paged decode-attention HBM GB/s (% of B200 peak) and decode tokens/s at 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
-DECODE_SOURCES = ["decode_simple.cu", "decode_tc.cu", "kernels.h", "common.cuh"]
+DECODE_SOURCES = ["decode_simple.cu", "decode_tc.cu", "kernels.h", "common.cuh", "ptx.cuh"]
 
 
 def parse():
@@ -49,8 +49,11 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="c3", choices=["c2", "c3", "c4", "c5"])
+    ap.add_argument("--workload", default="c3", choices=["c2", "c3", "c4", "c5", "p1"],
+                    help="c2..c5: decode steps; p1: PagedEviction prefill compression")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--kv", default=None, choices=["bf16", "int8", "fp8"],
+                    help="KV storage type (default: the workload's own)")
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--evict", default="full", choices=["full", "incremental"],
                     help="workloads with a score pass: rescore the whole context per layer "
@@ -169,7 +172,7 @@ def decode_algorithmic_bytes(cfg, ctx_lens, partial_slots, n_units=0):
     token (plus INT8 scales), q and out, the table entries and lengths read, the
     partition partials written and read back by the merge (partial_slots slots
     of Hq rows of d + 2 floats), and the partition list of the staged kernel."""
-    elt = 1 if cfg.int8 else 2
+    elt = 1 if (cfg.int8 or cfg.fp8) else 2
     tok = int(np.sum(ctx_lens))
     kv = tok * cfg.hkv * cfg.head_dim * 2 * elt
     if cfg.int8:
@@ -204,6 +207,17 @@ class Runner:
                                                                   num_splits)
         # the staged kernel launches plan + decode (+ merge); the general one decode (+ merge)
         self.staged = self.dec_launches - (1 if self.S > 1 else 0) >= 2
+        if cfg.fp8:
+            N = wl.num_blocks
+            self.k8 = torch.zeros(self.L, N, bs, Hkv, d, dtype=torch.uint8, device=device)
+            self.v8 = torch.zeros_like(self.k8)
+            zeros = torch.zeros(B, dtype=torch.int32, device=device)
+            for l in range(self.L):
+                for b in range(B):  # one prompt-style append per sequence
+                    n = int(wl.old_lens[b])
+                    pk.pa_append_kv_fp8(wl.k_hist[l, b:b + 1, :n].contiguous(),
+                                        wl.v_hist[l, b:b + 1, :n].contiguous(), self.k8[l],
+                                        self.v8[l], self.bt[b:b + 1], zeros[b:b + 1], self.err)
         if cfg.int8:
             N = wl.num_blocks
             self.kq = torch.zeros(self.L, N, bs, Hkv, d, dtype=torch.int8, device=device)
@@ -274,7 +288,14 @@ class Runner:
     def step(self, ev=None):
         pk, cfg = self.pk, self.cfg
         for l in range(self.L):
-            if cfg.int8:
+            if cfg.fp8:
+                pk.pa_append_kv_fp8(self.k_new[l], self.v_new[l], self.k8[l], self.v8[l], self.bt,
+                                    self.pos, self.err)
+                if ev is not None:
+                    ev[l][0].record()
+                pk.pa_decode_fp8(self.out[l], self.q[l], self.k8[l], self.v8[l], self.bt, self.ctx,
+                                 self.wl.scale, self.err, self.ws, self.num_splits)
+            elif cfg.int8:
                 pk.pa_append_kv_int8(self.k_new[l], self.v_new[l], self.kq[l], self.vq[l],
                                      self.ks[l], self.vs[l], self.bt, self.pos, self.err)
                 if ev is not None:
@@ -324,7 +345,17 @@ def oracle_throughput(wl, budget_s, max_layers=None):
         seqs = list(range(s0, min(cfg.batch, s0 + per_call)))
         c = W.compact(wl, l, seqs)
         t0 = time.perf_counter()
-        if cfg.int8:
+        if cfg.fp8:
+            n = c["num_blocks"]
+            k8 = np.zeros(n * stride, np.uint8); v8 = np.zeros_like(k8)
+            oracle.append_kv_fp8(c["k_hist"], c["v_hist"], k8, v8, stride, c["block_tables"],
+                                 np.zeros(len(seqs), np.int32), bs)
+            t0 = time.perf_counter()   # the history fill is set-up, not the step
+            oracle.append_kv_fp8(c["k_new"], c["v_new"], k8, v8, stride, c["block_tables"],
+                                 c["positions"], bs)
+            oracle.paged_decode_fp8(c["q"], k8, v8, stride, c["block_tables"], c["ctx_lens"], Hkv,
+                                    bs, wl.scale)
+        elif cfg.int8:
             n = c["num_blocks"]
             kq = np.zeros(n * stride, np.int8); vq = np.zeros_like(kq)
             ks = np.zeros(n * bs * Hkv, np.float32); vs = np.zeros_like(ks)
@@ -363,7 +394,9 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    cfg = W.CONFIGS[args.workload]
+    if args.workload in W.PREFILL:
+        return run_reference_prefill(args)
+    cfg = workload_cfg(args)
     wl = W.generate(cfg, "cpu", layers=1)
     per = max(1.0, args.cpu_seconds / max(1, args.steps))
     for _ in range(args.warmup):
@@ -390,6 +423,54 @@ def run_reference(args):
     return 0
 
 
+def kv_name(cfg):
+    return "fp8_e4m3" if cfg.fp8 else "int8" if cfg.int8 else "bf16"
+
+
+def workload_cfg(args):
+    """The named workload, with its KV storage type replaced when --kv asks."""
+    cfg = W.CONFIGS[args.workload]
+    if args.kv is not None:
+        cfg = W.scaled(cfg, int8=args.kv == "int8", fp8=args.kv == "fp8")
+    return cfg
+
+
+def traffic_key(args, cfg):
+    return args.workload + ("" if args.kv is None else "-" + kv_name(cfg))
+
+
+def run_reference_prefill(args):
+    """The oracle's prefill stage timed on bounded samples of the prefill workload."""
+    import dataclasses
+    cfg = W.PREFILL[args.workload]
+    # one prompt's worth of rows per sample keeps the host footprint small
+    small = dataclasses.replace(cfg, batch=4, prompt_lens=cfg.prompt_lens[:4])
+    wl = W.generate_prefill(small, "cpu")
+    per = max(1.0, args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        prefill_oracle_throughput(wl, per / 4)
+    vals, desc, cores = [], "", 0
+    for _ in range(args.steps):
+        v, cores, desc = prefill_oracle_throughput(wl, per)
+        vals.append(v)
+    value = statistics.median(vals)
+    T = sum(cfg.prompt_lens)
+    line = {
+        "impl": "reference", "metric": "PagedEviction prefill compression: prompt tokens/s",
+        "value": value, "unit": "prompt tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * T / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{cfg.key} {cfg.name}", "prompts": cfg.batch,
+                   "prompt_tokens": cfg.prompt_lens[0], "budget": cfg.budget},
+        "cpu_baseline": {"value": value, "unit": "prompt tokens/s", "cores": cores,
+                         "kind": "oracle", "sample": "per step: " + desc},
+        "e2e": {"value": value, "unit": "prompt tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def workload_config(cfg):
     lens = (f"{cfg.old_lens[0]}" if cfg.old_lens and len(set(cfg.old_lens)) == 1
             else f"uniform[{cfg.old_len_range[0]},{cfg.old_len_range[1]}]"
@@ -398,9 +479,170 @@ def workload_config(cfg):
         "workload": f"{cfg.key} {cfg.name}", "layers": cfg.layers, "global_batch": cfg.batch,
         "q_heads": cfg.hq, "kv_heads": cfg.hkv, "head_dim": cfg.head_dim,
         "block_size": cfg.block_size, "cached_tokens": lens,
-        "append": cfg.append, "score_pass": cfg.score, "kv_dtype": "int8" if cfg.int8 else "bf16",
+        "append": cfg.append, "score_pass": cfg.score, "kv_dtype": kv_name(cfg),
         "l2": "working set larger than L2 every step (no flush needed)",
     }
+
+
+# ----------------------------------------------------------------------------- prefill
+def prefill_oracle_throughput(wl, budget_s):
+    """The oracle's score + select + pack over whole prompts of the prefill
+    workload for about budget_s seconds; returns (prompt tokens/s, cores, desc)."""
+    import oracle
+    cfg = wl.cfg
+    cu = wl.cu_seqlens
+    Hkv, d, bs = cfg.hkv, cfg.head_dim, cfg.block_size
+    stride = bs * Hkv * d
+    cores = oracle.threads()
+    t_total, tok, n = 0.0, 0, 0
+    for i in range(100000):
+        b = i % cfg.batch
+        kb = W.bits(wl.k[int(cu[b]):int(cu[b + 1])])
+        vb = W.bits(wl.v[int(cu[b]):int(cu[b + 1])])
+        bt = wl.block_tables[b:b + 1]
+        nb = int((bt >= 0).sum())
+        bt_c = np.where(bt >= 0, np.arange(bt.shape[1], dtype=np.int32), -1).astype(np.int32)
+        kc = np.zeros(nb * stride, np.uint16)
+        vc = np.zeros_like(kc)
+        lcu = np.array([0, kb.shape[0]], np.int32)
+        t0 = time.perf_counter()
+        sc = oracle.prefill_scores(kb, vb)
+        keep, kept = oracle.prefill_select(sc, lcu, cfg.budget)
+        oracle.prefill_pack(kb, vb, lcu, keep, kept, kc, vc, stride, bt_c, bs)
+        t_total += time.perf_counter() - t0
+        tok += kb.shape[0]
+        n += 1
+        if t_total >= budget_s:
+            break
+    desc = (f"{n} whole prompts ({tok} tokens) through the oracle's score, select and pack "
+            f"({cores} threads), "
+            f"{t_total:.1f} s")
+    return tok / t_total, cores, desc
+
+
+def run_prefill(args, device, world, rank):
+    """One step = the prefill stage of one layer for every prompt of the
+    workload: token scores, keep sets, packing of the kept rows into the pool."""
+    import paged_kv_cache_396_b200.pagedkv as pk
+    cfg = W.PREFILL[args.workload]
+    wl = W.generate_prefill(cfg, device)
+    B, Hkv, d, bs, budget = cfg.batch, cfg.hkv, cfg.head_dim, cfg.block_size, cfg.budget
+    T = int(wl.cu_seqlens[-1])
+    N = wl.num_blocks
+    kc = torch.zeros(N, bs, Hkv, d, dtype=torch.bfloat16, device=device)
+    vc = torch.zeros_like(kc)
+    bt = torch.as_tensor(wl.block_tables, device=device)
+    cu = torch.as_tensor(wl.cu_seqlens, device=device)
+    scores = torch.empty(T, dtype=torch.float32, device=device)
+    keep = torch.empty(B, budget, dtype=torch.int32, device=device)
+    kept = torch.empty(B, dtype=torch.int32, device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        pk.pe_prefill_scores(scores, wl.k, wl.v)
+        if ev:
+            ev[1].record(stream)
+        pk.pe_prefill_select(keep, kept, scores, cu, err)
+        if ev:
+            ev[2].record(stream)
+        pk.pe_prefill_pack(kc, vc, bt, wl.k, wl.v, cu, keep, kept, err)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    if err.item() != 0:
+        raise SystemExit(f"device error flag {err.item()} during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    clocks = Clocks(device)
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    ms = reduce_max(t0.elapsed_time(t1), world) / args.steps
+    per = [[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in evs]
+    score_s = statistics.mean(p[0] for p in per) / 1000.0
+    select_s = statistics.mean(p[1] for p in per) / 1000.0
+    pack_s = statistics.mean(p[2] for p in per) / 1000.0
+    # algorithmic bytes: every prompt row of K and V read once plus one fp32 score
+    # written per token (score kernel); kept rows read and written (pack)
+    score_bytes = T * Hkv * d * 2 * 2 + T * 4
+    n_kept = int(kept.sum().item())
+    pack_bytes = n_kept * Hkv * d * 2 * 2 * 2 + B * budget * 4
+    peak, peak_kind = peaks()
+    achieved = score_bytes / score_s / 1e9
+
+    # end to end: prompt rows from pinned host memory, keep sets back to the host
+    hk = torch.empty(wl.k.shape, dtype=torch.bfloat16, pin_memory=True)
+    hv = torch.empty_like(hk, pin_memory=True)
+    hk.copy_(wl.k)
+    hv.copy_(wl.v)
+    hkeep = torch.empty(keep.shape, dtype=torch.int32, pin_memory=True)
+    hkept = torch.empty(kept.shape, dtype=torch.int32, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, 10))
+    torch.cuda.synchronize(device)
+    a = torch.cuda.Event(enable_timing=True)
+    z = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        wl.k.copy_(hk, non_blocking=True)
+        wl.v.copy_(hv, non_blocking=True)
+        pk.pe_prefill_compress(kc, vc, bt, wl.k, wl.v, cu, scores, keep, kept, err)
+        hkeep.copy_(keep, non_blocking=True)
+        hkept.copy_(kept, non_blocking=True)
+    z.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = reduce_max(a.elapsed_time(z) / e2e_steps, world)
+    if err.item() != 0:
+        raise SystemExit(f"device error flag {err.item()} during timing")
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_, cores, desc = prefill_oracle_throughput(
+            W.PrefillWorkload(cfg, wl.k.cpu(), wl.v.cpu(), wl.cu_seqlens, wl.block_tables, N),
+            args.cpu_seconds)
+        cpu = {"value": v_, "unit": "prompt tokens/s", "cores": cores, "kind": "oracle",
+               "sample": desc}
+    if rank == 0:
+        line = {
+            "metric": "PagedEviction prefill compression: prompt tokens/s and score-kernel "
+                      "HBM GB/s", "value": world * T / (ms / 1000.0), "unit": "prompt tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"{cfg.key} {cfg.name}", "prompts": B,
+                       "prompt_tokens": cfg.prompt_lens[0], "kv_heads": Hkv, "head_dim": d,
+                       "block_size": bs, "budget": budget, "parallelism": f"replicas{world}",
+                       "l2": "prompt rows (1 GiB) larger than L2 every step (no flush needed)"},
+            "roofline": {"bound": "hbm", "kernel": "pe_prefill_scores", "achieved": achieved,
+                         "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "algorithmic_bytes_per_launch": score_bytes,
+                         "avg_launch_us": score_s * 1e6},
+            "kernels_us": {"pe_prefill_scores": score_s * 1e6,
+                           "pe_prefill_select": select_s * 1e6,
+                           "pe_prefill_pack": pack_s * 1e6},
+            "pack_gbs": pack_bytes / pack_s / 1e9,
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * T / (e2e_ms / 1000.0), "unit": "prompt tokens/s",
+                    "h2d_bytes_per_step": 2 * T * Hkv * d * 2,
+                    "d2h_bytes_per_step": (B * budget + B) * 4, "ms_per_step": e2e_ms},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
 
 
 # ----------------------------------------------------------------------------- main
@@ -420,7 +662,13 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
-    cfg = W.CONFIGS[args.workload]
+    if args.workload in W.PREFILL:
+        rc = run_prefill(args, device, world, rank)
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return rc
+    cfg = workload_cfg(args)
     if args.layers:
         cfg = W.scaled(cfg, layers=args.layers)
     r = Runner(cfg, device, args.num_splits, evict=args.evict)
@@ -545,19 +793,20 @@ def main():
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
 
     if rank == 0:
-        traffic = recorded_traffic(args.workload)
+        traffic = recorded_traffic(traffic_key(args, cfg))
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int8" if cfg.int8 else "bf16", "data": "synthetic",
+            "dtype": {"fp8_e4m3": "e4m3"}.get(kv_name(cfg), kv_name(cfg)), "data": "synthetic",
             "config": dict(workload_config(cfg), parallelism=f"replicas{world}",
                            decode_kernel="staged-tc" if r.staged else "general",
                            evict_scoring=("incremental score pool" if r.incremental else
                                           "full pass per layer") if cfg.score else None,
                            partitions=r.partitions, chunk_tokens=r.chunk_used,
                            cuda_graph=use_graph),
-            "roofline": {"bound": "hbm", "kernel": "pa_decode" + ("_int8" if cfg.int8 else ""),
+            "roofline": {"bound": "hbm", "kernel": {"bf16": "pa_decode", "int8": "pa_decode_int8",
+                                                   "fp8_e4m3": "pa_decode_fp8"}[kv_name(cfg)],
                          "achieved": achieved, "peak": peak, "peak_source": peak_kind,
                          "unit": "GB/s", "frac": achieved / peak,
                          "frac_of_nominal_8tbs": achieved / 8000.0,

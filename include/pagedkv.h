@@ -62,6 +62,7 @@ extern "C" {
 #define PA_DEV_BAD_BLOCK  1  /* a needed block-table entry was outside [0, N)       */
 #define PA_DEV_BAD_LEN    2  /* a context length / position outside [0, MB*bs]     */
 #define PA_DEV_TIMEOUT    4  /* a bounded pipeline wait gave up (kernel returned)   */
+#define PA_DEV_BAD_EVICT  8  /* an eviction index that is not a full block          */
 
 /* Human-readable text of a PA_* status code (static storage). */
 const char *pa_status_string(int code);
@@ -290,6 +291,77 @@ int pa_decode_static_scratch(uint16_t *out, const uint16_t *q,
                              int max_blocks_per_seq, const int32_t *ctx_lens, int B, int Hq,
                              int Hkv, int d, int bs, int64_t num_blocks, float scale,
                              int num_splits, int32_t *err_flag, void *stream);
+
+/* ============================================================================
+ * PagedEviction prefill stage  ([KVL] "PagedEviction 块级驱逐机制", two-stage
+ * strategy: at prefill each token gets an importance and the lowest-scoring
+ * tokens are evicted down to the cache budget; the survivors fill whole blocks).
+ *
+ * Prompts arrive contiguous and token-major: k, v [T][Hkv][d] bf16 (all B
+ * prompts concatenated; cu_seqlens [B+1] int32 device array of offsets, prompt b
+ * = tokens cu_seqlens[b] .. cu_seqlens[b+1]-1).  d in {64, 128, 256}; k, v and
+ * the pools 16-byte aligned.
+ *
+ * pe_prefill_scores: scores[t] (fp32, [T]) = mean over the Hkv heads of
+ *   ||V[t,h]||_2 / ||K[t,h]||_2 (fp32 sums of squares; ||K|| = 0 gives +inf when
+ *   ||V|| > 0, else 0).  Reading: a token is kept or evicted for all heads at
+ *   once (one slot holds them all), so its importance is the head mean.
+ *
+ * pe_prefill_select: per prompt, the source indices of the tokens that stay.
+ *   The budget tokens that rank highest stay; ranking is by score (numeric
+ *   order, NaN counted as -inf, -0 equal to +0), and on equal scores the
+ *   earlier token is evicted first.  Kept tokens keep their prompt order.
+ *   keep_idx [B][budget] int32: prompt-local index of the p-th kept token, -1
+ *   after the last; kept_len [B] = min(prompt length, budget).  budget >= 1.
+ *   A negative prompt length sets PA_DEV_BAD_LEN and keeps nothing.
+ *
+ * pe_prefill_pack: writes the p-th kept token of prompt b (p < kept_len[b]) at
+ *   position p of sequence b, slot = block_tables[b][p/bs]*bs + p%bs (every kv
+ *   head), so the compressed prompt fills ceil(kept/bs) blocks densely.  The
+ *   caller's allocator has placed those blocks in the table.  An index outside
+ *   the prompt or p/bs >= MB sets PA_DEV_BAD_LEN; a block id outside [0, N)
+ *   sets PA_DEV_BAD_BLOCK; the token is skipped.
+ *
+ * pe_prefill_compress: pe_prefill_scores, pe_prefill_select and
+ *   pe_prefill_pack in one call (three launches on `stream`); scores,
+ *   keep_idx and kept_len are outputs the caller may read afterwards.
+ * ==========================================================================*/
+int pe_prefill_scores(float *scores, const uint16_t *k, const uint16_t *v, int64_t T, int Hkv,
+                      int d, void *stream);
+
+int pe_prefill_select(int32_t *keep_idx, int32_t *kept_len, const float *scores,
+                      const int32_t *cu_seqlens, int B, int budget, int32_t *err_flag,
+                      void *stream);
+
+int pe_prefill_pack(uint16_t *k_cache, uint16_t *v_cache, int64_t block_stride,
+                    const int32_t *block_tables, int max_blocks_per_seq, const uint16_t *k,
+                    const uint16_t *v, const int32_t *cu_seqlens, const int32_t *keep_idx,
+                    const int32_t *kept_len, int B, int budget, int Hkv, int d, int bs,
+                    int64_t num_blocks, int32_t *err_flag, void *stream);
+
+int pe_prefill_compress(uint16_t *k_cache, uint16_t *v_cache, int64_t block_stride,
+                        const int32_t *block_tables, int max_blocks_per_seq, const uint16_t *k,
+                        const uint16_t *v, const int32_t *cu_seqlens, int64_t T, int B,
+                        int budget, int Hkv, int d, int bs, int64_t num_blocks, float *scores,
+                        int32_t *keep_idx, int32_t *kept_len, int32_t *err_flag, void *stream);
+
+/* ============================================================================
+ * Block-table compaction after a decode-phase eviction  ([KVL] "PagedEviction
+ * 块级驱逐机制": eviction removes whole blocks, never part of one).
+ *
+ * For every sequence b with evict[b] = j >= 0 (the logical index that
+ * pe_select_evict_block returned): entries j+1 .. ceil(len_b/bs)-1 of
+ * block_tables[b] move down by one, the last used entry becomes -1,
+ * ctx_lens[b] drops by bs, and freed[b] (nullable [B]) receives the physical id
+ * that left the table (the caller's allocator takes it back).  evict[b] < 0
+ * leaves sequence b alone (freed[b] = -1).  Physical blocks do not move, so the
+ * cached rows and a score pool stay valid.  j not a full block (j >= len/bs)
+ * sets PA_DEV_BAD_EVICT, a length outside [0, MB*bs] PA_DEV_BAD_LEN; the
+ * sequence is left unchanged.  block_tables and ctx_lens are updated in place.
+ * ==========================================================================*/
+int pe_evict_compact(int32_t *block_tables, int max_blocks_per_seq, int32_t *ctx_lens,
+                     int32_t *freed, const int32_t *evict, int B, int bs, int32_t *err_flag,
+                     void *stream);
 
 #ifdef __cplusplus
 }

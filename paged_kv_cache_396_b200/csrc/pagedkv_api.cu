@@ -8,6 +8,7 @@
 #include <atomic>
 
 #include "kernels.h"
+#include "prefill.h"
 #include "pagedkv.h"
 
 namespace {
@@ -416,3 +417,108 @@ int pa_decode_static_scratch(uint16_t *out, const uint16_t *q, const uint16_t *k
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// PagedEviction prefill stage and table compaction
+// ---------------------------------------------------------------------------
+namespace {
+int check_prefill_rows(const uint16_t *k, const uint16_t *v, int64_t T, int Hkv, int d) {
+    if (!k || !v) return PA_ERR_NULL;
+    if (T < 0 || Hkv < 1 || Hkv > 65535) return PA_ERR_SHAPE;
+    if (d != 64 && d != 128 && d != 256) return PA_ERR_SHAPE;
+    if (!al16(k) || !al16(v)) return PA_ERR_ALIGN;
+    return PA_OK;
+}
+}  // namespace
+
+int pe_prefill_scores(float *scores, const uint16_t *k, const uint16_t *v, int64_t T, int Hkv,
+                      int d, void *stream) {
+    if (T == 0) return PA_OK;
+    if (!scores) return PA_ERR_NULL;
+    int rc = check_prefill_rows(k, v, T, Hkv, d);
+    if (rc) return rc;
+    if ((T + 7) / 8 > INT32_MAX) return PA_ERR_SHAPE;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    return finish(pkv::launch_prefill_scores(scores, k, v, T, Hkv, d,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+int pe_prefill_select(int32_t *keep_idx, int32_t *kept_len, const float *scores,
+                      const int32_t *cu_seqlens, int B, int budget, int32_t *err_flag,
+                      void *stream) {
+    if (B == 0) return PA_OK;
+    if (!keep_idx || !kept_len || !scores || !cu_seqlens || !err_flag) return PA_ERR_NULL;
+    if (B < 0 || B > INT32_MAX / 2 || budget < 1) return PA_ERR_SHAPE;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    return finish(pkv::launch_prefill_select(keep_idx, kept_len, scores, cu_seqlens, B, budget,
+                                             err_flag, static_cast<cudaStream_t>(stream)));
+}
+
+int pe_prefill_pack(uint16_t *k_cache, uint16_t *v_cache, int64_t block_stride,
+                    const int32_t *block_tables, int max_blocks_per_seq, const uint16_t *k,
+                    const uint16_t *v, const int32_t *cu_seqlens, const int32_t *keep_idx,
+                    const int32_t *kept_len, int B, int budget, int Hkv, int d, int bs,
+                    int64_t num_blocks, int32_t *err_flag, void *stream) {
+    if (B == 0) return PA_OK;
+    if (!k_cache || !v_cache || !block_tables || !cu_seqlens || !keep_idx || !kept_len ||
+        !err_flag)
+        return PA_ERR_NULL;
+    int rc = check_prefill_rows(k, v, 1, Hkv, d);
+    if (rc) return rc;
+    if (B < 0 || budget < 1 || bs < 1 || max_blocks_per_seq < 1 || num_blocks < 1)
+        return PA_ERR_SHAPE;
+    if (block_stride < (int64_t)bs * Hkv * d) return PA_ERR_SHAPE;
+    if ((int64_t)B * budget > (int64_t)INT32_MAX * 8) return PA_ERR_SHAPE;
+    if (!al16(k_cache) || !al16(v_cache) || (block_stride * 2) % 16 != 0) return PA_ERR_ALIGN;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    return finish(pkv::launch_prefill_pack(k_cache, v_cache, block_stride, block_tables,
+                                           max_blocks_per_seq, k, v, cu_seqlens, keep_idx,
+                                           kept_len, B, budget, Hkv, d, bs, num_blocks, err_flag,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int pe_prefill_compress(uint16_t *k_cache, uint16_t *v_cache, int64_t block_stride,
+                        const int32_t *block_tables, int max_blocks_per_seq, const uint16_t *k,
+                        const uint16_t *v, const int32_t *cu_seqlens, int64_t T, int B,
+                        int budget, int Hkv, int d, int bs, int64_t num_blocks, float *scores,
+                        int32_t *keep_idx, int32_t *kept_len, int32_t *err_flag, void *stream) {
+    if (B == 0) return PA_OK;
+    // validate everything before the first launch
+    if (!scores && T > 0) return PA_ERR_NULL;
+    if (!k_cache || !v_cache || !block_tables || !cu_seqlens || !keep_idx || !kept_len ||
+        !err_flag)
+        return PA_ERR_NULL;
+    int rc = check_prefill_rows(k, v, T, Hkv, d);
+    if (rc) return rc;
+    if (B < 0 || budget < 1 || bs < 1 || max_blocks_per_seq < 1 || num_blocks < 1)
+        return PA_ERR_SHAPE;
+    if (block_stride < (int64_t)bs * Hkv * d) return PA_ERR_SHAPE;
+    if (!al16(k_cache) || !al16(v_cache) || (block_stride * 2) % 16 != 0) return PA_ERR_ALIGN;
+    if (T > 0 && (rc = pe_prefill_scores(scores, k, v, T, Hkv, d, stream))) return rc;
+    // T = 0 (every prompt empty): the select kernel keeps nothing and never reads
+    // scores; a prompt longer than the budget would contradict T and is flagged
+    if ((rc = finish(pkv::launch_prefill_select(keep_idx, kept_len, T > 0 ? scores : nullptr,
+                                                cu_seqlens, B, budget, err_flag,
+                                                static_cast<cudaStream_t>(stream)))))
+        return rc;
+    return pe_prefill_pack(k_cache, v_cache, block_stride, block_tables, max_blocks_per_seq, k, v,
+                           cu_seqlens, keep_idx, kept_len, B, budget, Hkv, d, bs, num_blocks,
+                           err_flag, stream);
+}
+
+int pe_evict_compact(int32_t *block_tables, int max_blocks_per_seq, int32_t *ctx_lens,
+                     int32_t *freed, const int32_t *evict, int B, int bs, int32_t *err_flag,
+                     void *stream) {
+    if (B == 0) return PA_OK;
+    if (!block_tables || !ctx_lens || !evict || !err_flag) return PA_ERR_NULL;
+    if (B < 0 || max_blocks_per_seq < 1 || bs < 1) return PA_ERR_SHAPE;
+    if ((int64_t)max_blocks_per_seq * bs > INT32_MAX) return PA_ERR_SHAPE;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    return finish(pkv::launch_evict_compact(block_tables, max_blocks_per_seq, ctx_lens, freed,
+                                            evict, B, bs, err_flag,
+                                            static_cast<cudaStream_t>(stream)));
+}

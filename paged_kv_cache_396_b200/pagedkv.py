@@ -28,6 +28,7 @@ PA_OK = 0
 PA_DEV_BAD_BLOCK = 1
 PA_DEV_BAD_LEN = 2
 PA_DEV_TIMEOUT = 4
+PA_DEV_BAD_EVICT = 8
 
 EXPORTED = (
     "pa_status_string", "pa_version", "pa_append_kv", "pa_decode_workspace_bytes", "pa_decode_plan",
@@ -35,6 +36,8 @@ EXPORTED = (
     "pe_score_tokens", "pe_select_evict_block", "pa_append_kv_int8", "pa_decode_int8",
     "pa_decode_static_scratch", "pa_append_kv_scored", "pa_append_kv_int8_scored",
     "pe_select_evict_block_pooled", "pa_append_kv_fp8", "pa_decode_fp8",
+    "pe_prefill_scores", "pe_prefill_select", "pe_prefill_pack", "pe_prefill_compress",
+    "pe_evict_compact",
 )
 
 
@@ -94,6 +97,18 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode_fp8.restype = i32
     lib.pa_decode_fp8.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, i64, f32,
                                   i32, p, sz, p, p]
+    lib.pe_prefill_scores.restype = i32
+    lib.pe_prefill_scores.argtypes = [p, p, p, i64, i32, i32, p]
+    lib.pe_prefill_select.restype = i32
+    lib.pe_prefill_select.argtypes = [p, p, p, p, i32, i32, p, p]
+    lib.pe_prefill_pack.restype = i32
+    lib.pe_prefill_pack.argtypes = [p, p, i64, p, i32, p, p, p, p, p, i32, i32, i32, i32, i32,
+                                    i64, p, p]
+    lib.pe_prefill_compress.restype = i32
+    lib.pe_prefill_compress.argtypes = [p, p, i64, p, i32, p, p, p, i64, i32, i32, i32, i32, i32,
+                                        i64, p, p, p, p, p]
+    lib.pe_evict_compact.restype = i32
+    lib.pe_evict_compact.argtypes = [p, i32, p, p, p, i32, i32, p, p]
     lib.pe_score_tokens.restype = i32
     lib.pe_score_tokens.argtypes = [p, p, p, i64, p, i32, p, i32, i32, i32, i32, i64, p, p]
     lib.pe_select_evict_block.restype = i32
@@ -492,3 +507,104 @@ def pa_decode_fp8(out, q, k8_cache, v8_cache, block_tables, ctx_lens, scale, err
                               bs, N, float(scale), int(num_splits), ws_ptr, ws_n, _ptr(err_flag),
                               _stream(stream))
     _check("pa_decode_fp8", rc)
+
+
+# ----------------------------------------------------------------------------- prefill stage
+def _prompt_rows(k, v):
+    _want(k, torch.bfloat16, "k")
+    _want(v, torch.bfloat16, "v")
+    if k.dim() != 3 or k.shape != v.shape or not (k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("k, v: expected contiguous [T, Hkv, d] of equal shape")
+    return k.shape
+
+
+def pe_prefill_scores(scores, k, v, stream=None):
+    """Per-token importance of concatenated prompts: head mean of ||V||/||K||.
+    k, v [T, Hkv, d] bf16 contiguous; scores [T] float32."""
+    T, Hkv, d = _prompt_rows(k, v)
+    _want(scores, torch.float32, "scores")
+    if scores.numel() < T or not scores.is_contiguous():
+        raise ValueError("scores: expected a contiguous float32 tensor of T elements")
+    _check("pe_prefill_scores", load().pe_prefill_scores(_ptr(scores), _ptr(k), _ptr(v), T, Hkv,
+                                                         d, _stream(stream)))
+
+
+def pe_prefill_select(keep_idx, kept_len, scores, cu_seqlens, err_flag, stream=None):
+    """Indices (prompt-local, in order) of the budget highest-ranking tokens of
+    each prompt.  keep_idx [B, budget] int32, kept_len [B] int32, scores [T]
+    float32, cu_seqlens [B+1] int32."""
+    _want(keep_idx, torch.int32, "keep_idx")
+    _want(kept_len, torch.int32, "kept_len")
+    _want(scores, torch.float32, "scores")
+    _want(cu_seqlens, torch.int32, "cu_seqlens")
+    _want(err_flag, torch.int32, "err_flag")
+    B, budget = keep_idx.shape
+    if not keep_idx.is_contiguous() or cu_seqlens.numel() != B + 1:
+        raise ValueError("keep_idx must be contiguous [B, budget] and cu_seqlens [B+1]")
+    _check("pe_prefill_select", load().pe_prefill_select(
+        _ptr(keep_idx), _ptr(kept_len), _ptr(scores), _ptr(cu_seqlens.contiguous()), B, budget,
+        _ptr(err_flag), _stream(stream)))
+
+
+def pe_prefill_pack(k_cache, v_cache, block_tables, k, v, cu_seqlens, keep_idx, kept_len,
+                    err_flag, stream=None):
+    """Write the kept prompt rows at positions 0.. of each sequence."""
+    T, Hkv, d = _prompt_rows(k, v)
+    _want(k_cache, torch.bfloat16, "k_cache")
+    _want(v_cache, torch.bfloat16, "v_cache")
+    N, bs, Hkv_c, d_c, stride = _pool_geometry(k_cache, "k_cache")
+    _same_pool(k_cache, v_cache)
+    if (Hkv_c, d_c) != (Hkv, d):
+        raise ValueError("prompt rows and pool differ in Hkv or d")
+    _want(block_tables, torch.int32, "block_tables")
+    B, budget = keep_idx.shape
+    bt = block_tables.contiguous()
+    _check("pe_prefill_pack", load().pe_prefill_pack(
+        _ptr(k_cache), _ptr(v_cache), stride, _ptr(bt), bt.shape[1], _ptr(k), _ptr(v),
+        _ptr(cu_seqlens.contiguous()), _ptr(keep_idx.contiguous()), _ptr(kept_len), B, budget,
+        Hkv, d, bs, N, _ptr(err_flag), _stream(stream)))
+
+
+def pe_prefill_compress(k_cache, v_cache, block_tables, k, v, cu_seqlens, scores, keep_idx,
+                        kept_len, err_flag, stream=None):
+    """Score, select and pack in one call (budget = keep_idx.shape[1])."""
+    T, Hkv, d = _prompt_rows(k, v)
+    _want(k_cache, torch.bfloat16, "k_cache")
+    _want(v_cache, torch.bfloat16, "v_cache")
+    N, bs, Hkv_c, d_c, stride = _pool_geometry(k_cache, "k_cache")
+    _same_pool(k_cache, v_cache)
+    if (Hkv_c, d_c) != (Hkv, d):
+        raise ValueError("prompt rows and pool differ in Hkv or d")
+    _want(block_tables, torch.int32, "block_tables")
+    _want(scores, torch.float32, "scores")
+    _want(keep_idx, torch.int32, "keep_idx")
+    _want(kept_len, torch.int32, "kept_len")
+    _want(cu_seqlens, torch.int32, "cu_seqlens")
+    _want(err_flag, torch.int32, "err_flag")
+    B, budget = keep_idx.shape
+    if scores.numel() < T or not keep_idx.is_contiguous() or cu_seqlens.numel() != B + 1:
+        raise ValueError("scores [T], keep_idx contiguous [B, budget], cu_seqlens [B+1]")
+    bt = block_tables.contiguous()
+    _check("pe_prefill_compress", load().pe_prefill_compress(
+        _ptr(k_cache), _ptr(v_cache), stride, _ptr(bt), bt.shape[1], _ptr(k), _ptr(v),
+        _ptr(cu_seqlens.contiguous()), T, B, budget, Hkv, d, bs, N, _ptr(scores),
+        _ptr(keep_idx), _ptr(kept_len), _ptr(err_flag), _stream(stream)))
+
+
+def pe_evict_compact(block_tables, ctx_lens, evict, block_size, err_flag, freed=None,
+                     stream=None):
+    """Remove each sequence's evicted logical block from its table in place
+    (block_tables [B, MB] int32 contiguous, ctx_lens [B] int32 lowered by
+    block_size); freed [B] int32 (optional) receives the released physical ids."""
+    _want(block_tables, torch.int32, "block_tables")
+    _want(ctx_lens, torch.int32, "ctx_lens")
+    _want(evict, torch.int32, "evict")
+    _want(err_flag, torch.int32, "err_flag")
+    if not (block_tables.is_contiguous() and ctx_lens.is_contiguous()):
+        raise ValueError("block_tables and ctx_lens are updated in place: pass contiguous tensors")
+    if freed is not None:
+        _want(freed, torch.int32, "freed")
+    B, MB = block_tables.shape
+    _check("pe_evict_compact", load().pe_evict_compact(
+        _ptr(block_tables), MB, _ptr(ctx_lens), _ptr(freed), _ptr(evict.contiguous()), B,
+        int(block_size), _ptr(err_flag), _stream(stream)))

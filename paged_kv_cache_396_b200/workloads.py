@@ -18,7 +18,11 @@ describe; all values bf16 ~ N(0, 1) unless stated):
                 bs=256, one tensor [2, L, N, 256, Hkv, d] (nano-vLLM layout), shuffled.
   c5  INT8 pool: 1 layer, Hq=64, Hkv=8, d=128, B=128, old len 4096 (+1), bs=16;
                 K/V history drawn bf16 and quantised by the INT8 append.
-Seeds are 396 + the workload's index (0..4).
+  p1  prefill compression: 32 prompts of 8192 tokens, Hkv=8, d=128, bs=16,
+                budget 1024 tokens per prompt (the PagedEviction budget); prompt
+                K/V rows [T, Hkv, d] bf16 N(0, 1) with 1% of the (head, channel)
+                pairs scaled x8.
+Seeds are 396 + the workload's index (0..5).
 
 The allocator is the on-demand block pool of the vLLM notes (ybb.press "LLM 推理
 KV Cache 内存管理深度工程实践" §2.1): a shuffled free list, each sequence taking
@@ -233,3 +237,60 @@ def compact(wl: Workload, layer: int, seqs) -> dict:
         out["k_hist"] = bits(wl.k_hist[layer, seqs])
         out["v_hist"] = bits(wl.v_hist[layer, seqs])
     return out
+
+
+# ----------------------------------------------------------------------------- prefill stage
+@dataclass(frozen=True)
+class PrefillConfig:
+    key: str
+    name: str
+    batch: int
+    prompt_lens: tuple
+    hkv: int
+    head_dim: int
+    block_size: int
+    budget: int
+    outlier_frac: float = 0.01
+    spare: float = 0.10
+    seed: int = 401
+
+
+PREFILL = {
+    "p1": PrefillConfig("p1", "PagedEviction prefill compression", 32, (8192,) * 32, 8, 128, 16,
+                        1024),
+}
+
+
+@dataclass
+class PrefillWorkload:
+    cfg: PrefillConfig
+    k: torch.Tensor                 # [T, Hkv, d] bf16, prompts concatenated
+    v: torch.Tensor
+    cu_seqlens: np.ndarray          # [B+1] int32
+    block_tables: np.ndarray        # [B, MB] int32: ceil(min(len, budget)/bs) blocks each
+    num_blocks: int
+
+
+def generate_prefill(cfg: PrefillConfig, device="cpu") -> PrefillWorkload:
+    """Seeded prompt rows and the block tables for the compressed prompts."""
+    rng = np.random.default_rng(cfg.seed)
+    lens = np.asarray(cfg.prompt_lens, np.int64)
+    kept = np.minimum(lens, cfg.budget)
+    bt, N = _allocate(np.maximum(kept, 1), cfg.block_size, cfg.spare, None, rng)
+    g = torch.Generator(device=device)
+    g.manual_seed(cfg.seed)
+    T, Hkv, d = int(lens.sum()), cfg.hkv, cfg.head_dim
+    k = torch.empty(T, Hkv, d, dtype=torch.bfloat16, device=device)
+    v = torch.empty_like(k)
+    step = 1 << 16                  # draw in slices: bounded fp32 staging
+    for t0 in range(0, T, step):
+        n = min(step, T - t0)
+        k[t0:t0 + n].copy_(torch.randn(n, Hkv, d, generator=g, device=device))
+        v[t0:t0 + n].copy_(torch.randn(n, Hkv, d, generator=g, device=device))
+    n_out = int(round(cfg.outlier_frac * Hkv * d))
+    for c in rng.choice(Hkv * d, size=n_out, replace=False):
+        h, e = int(c) // d, int(c) % d
+        k[:, h, e] *= 8
+        v[:, h, e] *= 8
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return PrefillWorkload(cfg=cfg, k=k, v=v, cu_seqlens=cu, block_tables=bt, num_blocks=N)

@@ -9,6 +9,8 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
+
 from helpers import (Device, assert_attention_close, assert_evict_consistent,
                      assert_scores_close, oracle_step)
 from paged_kv_cache_396_b200 import pagedkv as pk
@@ -53,7 +55,7 @@ def _parity(wl, layers, num_splits=0, score=None):
     seqs = range(cfg.batch)
     refs = [oracle_step(wl, l, seqs, score=score) for l in layers]
     dev = Device(wl, num_splits)
-    if cfg.int8:
+    if cfg.int8 or cfg.fp8:
         for l in layers:
             dev.fill_int8_history(l)
     for l, ref in zip(layers, refs):
@@ -257,3 +259,36 @@ def test_fp8_codes_bit_exact():
     ids = torch.as_tensor(wl.block_tables[wl.block_tables >= 0], device="cuda")
     assert np.array_equal(dev.k8[0][ids].cpu().numpy().ravel(), ref["k8"])
     assert np.array_equal(dev.v8[0][ids].cpu().numpy().ravel(), ref["v8"])
+
+
+def test_fp8_append_special_values_bit_exact():
+    """Saturation beyond 448 (and of infinities), NaN, signed zero, subnormal
+    steps and ties to even on both sides of the subnormal/normal boundary."""
+    Hkv, d, bs, N = 2, 128, 16, 4
+    special = [0.0, -0.0, 448.0, -448.0, 449.0, 464.0, 480.0, 1e4, -1e4, float("inf"),
+               float("-inf"), float("nan"), 2.0 ** -9, 3 * 2.0 ** -10, 2.0 ** -10,
+               5 * 2.0 ** -10, 2.0 ** -6, 15 * 2.0 ** -10, 17 * 2.0 ** -10, 1.0625, 1.1875,
+               -1.0625, 240.0, 248.0, 232.0, 0.001, -0.0029296875]
+    g = torch.Generator().manual_seed(17)
+    k = torch.randn(1, 3, Hkv, d, generator=g) * 40
+    flat = k.view(-1)
+    flat[:len(special)] = torch.tensor(special)
+    neg = [-x for x in special if x == x]   # NaN once only: its sign is not a defined result
+    flat[-len(neg):] = torch.tensor(neg)
+    k = k.to(torch.bfloat16)
+    v = (torch.randn(1, 3, Hkv, d, generator=g) * 0.01).to(torch.bfloat16)
+    k8 = torch.zeros(N, bs, Hkv, d, dtype=torch.uint8, device="cuda")
+    v8 = torch.zeros_like(k8)
+    bt = torch.tensor([[2, 0]], dtype=torch.int32, device="cuda")
+    pos = torch.tensor([14], dtype=torch.int32, device="cuda")   # rows 14, 15 of block 2, row 0 of block 0
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pk.pa_append_kv_fp8(k.cuda(), v.cuda(), k8, v8, bt, pos, err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    got = torch.stack([k8[2, 14], k8[2, 15], k8[0, 0]]).cpu().numpy().ravel()
+    expect = oracle.quantize_e4m3(W.bits(k)).ravel()
+    assert np.array_equal(got, expect)
+    gotv = torch.stack([v8[2, 14], v8[2, 15], v8[0, 0]]).cpu().numpy().ravel()
+    assert np.array_equal(gotv, oracle.quantize_e4m3(W.bits(v)).ravel())
+    # nothing else in the pools was touched
+    assert int(k8.count_nonzero()) == int(np.count_nonzero(got))
