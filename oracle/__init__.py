@@ -64,6 +64,11 @@ def _lib():
         lib.or_prefill_pack.argtypes = [p, p, p, p, p, i32, p, p, i64, p, i32, i32, i32, i32, i32]
         lib.or_evict_compact.restype = None
         lib.or_evict_compact.argtypes = [p, p, p, p, i32, i32, i32]
+        lib.or_select_evict_threshold.restype = None
+        lib.or_select_evict_threshold.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i64, i64,
+                                                  dbl, dbl]
+        lib.or_evict_compact_mask.restype = None
+        lib.or_evict_compact_mask.argtypes = [p, p, p, p, i32, i32, i32]
         lib.or_e4m3_to_f64.restype = dbl
         lib.or_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         lib.or_append_kv_fp8.restype = None
@@ -333,4 +338,36 @@ def evict_compact(bt, ctx_lens, evict, bs):
     B, MB = bt.shape
     freed = np.empty(B, np.int32)
     _lib().or_evict_compact(_ptr(bt), _ptr(ctx), _ptr(freed), _ptr(evict), B, MB, bs)
+    return bt, ctx, freed
+
+
+def select_evict_threshold(scores, ctx_lens, bs, used_blocks, total_blocks, eviction_ratio,
+                           importance_threshold):
+    """Threshold policy: once used_blocks > (1 - eviction_ratio) * total_blocks,
+    every full block with mean importance below importance_threshold is marked,
+    else the lowest-mean full block.  Returns (mask [B, MB] uint8, count [B] int32,
+    means [B, MB] float64)."""
+    scores = np.ascontiguousarray(scores, dtype=np.float64)
+    ctx_lens = _c(ctx_lens, np.int32)
+    B, T, Hkv = scores.shape
+    MB = T // bs
+    mask = np.empty((B, MB), np.uint8)
+    count = np.empty(B, np.int32)
+    means = np.empty((B, MB), np.float64)
+    _lib().or_select_evict_threshold(_ptr(mask), _ptr(count), _ptr(means), _ptr(scores),
+                                     _ptr(ctx_lens), B, MB, Hkv, bs, int(used_blocks),
+                                     int(total_blocks), float(eviction_ratio),
+                                     float(importance_threshold))
+    return mask, count, means
+
+
+def evict_compact_mask(bt, ctx_lens, mask, bs):
+    """Remove every marked full block.  Returns new copies (bt, ctx_lens, freed
+    [B, MB] int32 listing freed ids in logical order, -1 after the last)."""
+    bt = np.array(bt, dtype=np.int32, order="C", copy=True)
+    ctx = np.array(ctx_lens, dtype=np.int32, copy=True)
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    B, MB = bt.shape
+    freed = np.empty((B, MB), np.int32)
+    _lib().or_evict_compact_mask(_ptr(bt), _ptr(ctx), _ptr(freed), _ptr(mask), B, MB, bs)
     return bt, ctx, freed

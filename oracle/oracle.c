@@ -578,3 +578,64 @@ void or_evict_compact(int32_t *bt, int32_t *ctx_lens, int32_t *freed, const int3
         ctx_lens[b] -= bs;
     }
 }
+
+/* Threshold eviction policy (blog.hotdry.top nano-vLLM KV cache page, section
+ * "工程落地：参数配置与监控要点": eviction_ratio = 0.2 starts eviction once cache
+ * usage passes 80 %, and blocks whose importance is below importance_threshold
+ * are evicted first).  Readings: the trigger is used_blocks > (1 - eviction_ratio)
+ * * total_blocks, evaluated in fp64 (below it nothing is evicted); once triggered,
+ * every full block of a sequence whose mean importance (the decode-phase block
+ * mean) is below importance_threshold is evicted, and a sequence with no such
+ * block evicts its single lowest-mean full block (the decode-phase rule, ties to
+ * the lowest index); a sequence with no full block evicts nothing.
+ * scores [B][MB*bs][Hkv] fp64; mask [B][MB] (1 = evict); count [B]; means
+ * (nullable) [B][MB] as in or_select_evict_block. */
+void or_select_evict_threshold(uint8_t *mask, int32_t *count, double *means,
+                               const double *scores, const int32_t *ctx_lens, int B, int MB,
+                               int Hkv, int bs, int64_t used_blocks, int64_t total_blocks,
+                               double eviction_ratio, double importance_threshold) {
+    const int triggered = (double)used_blocks > (1.0 - eviction_ratio) * (double)total_blocks;
+    double *m = (double *)malloc(sizeof(double) * (size_t)B * (size_t)MB);
+    int32_t *argmin = (int32_t *)malloc(sizeof(int32_t) * (size_t)(B > 0 ? B : 1));
+    or_select_evict_block(argmin, m, NULL, scores, ctx_lens, B, MB, Hkv, bs);
+    for (int b = 0; b < B; ++b) {
+        int n = 0;
+        for (int j = 0; j < MB; ++j) {
+            const double mj = m[(int64_t)b * MB + j];
+            const int below = triggered && mj == mj && mj < importance_threshold;
+            mask[(int64_t)b * MB + j] = (uint8_t)below;
+            n += below;
+        }
+        if (triggered && n == 0 && argmin[b] >= 0) {
+            mask[(int64_t)b * MB + argmin[b]] = 1;
+            n = 1;
+        }
+        count[b] = n;
+    }
+    if (means) memcpy(means, m, sizeof(double) * (size_t)B * (size_t)MB);
+    free(m);
+    free(argmin);
+}
+
+/* Table compaction for several evicted blocks per sequence: the full blocks
+ * marked in mask[b] leave the table, the remaining entries keep their order and
+ * close up, the context length drops by bs per evicted block, and the freed
+ * physical ids are listed in freed[b][0..] in logical order (-1 after the last).
+ * A mark on a block that is not full is ignored. */
+void or_evict_compact_mask(int32_t *bt, int32_t *ctx_lens, int32_t *freed, const uint8_t *mask,
+                           int B, int MB, int bs) {
+    for (int b = 0; b < B; ++b) {
+        int32_t *row = bt + (int64_t)b * MB;
+        int32_t *fr = freed + (int64_t)b * MB;
+        const int len = ctx_lens[b];
+        const int nfull = len / bs, nblk = (int)or_num_blocks(len, bs);
+        int w = 0, nf = 0;
+        for (int j = 0; j < nblk; ++j) {
+            if (j < nfull && mask[(int64_t)b * MB + j]) fr[nf++] = row[j];
+            else row[w++] = row[j];
+        }
+        for (int j = w; j < nblk; ++j) row[j] = -1;
+        for (int j = nf; j < MB; ++j) fr[j] = -1;
+        ctx_lens[b] = len - nf * bs;
+    }
+}

@@ -711,3 +711,105 @@ def test_evict_compact_preserves_token_to_slot_map():
         new = sorted([x for x in nbt[b] if x >= 0] + [int(freed[b])])
         assert old == new
         assert (nbt[b, -(-int(nlen[b]) // bs):] == -1).all()
+
+
+# ----------------------------------------------------------------------------- threshold policy
+def _block_scores(consts, bs, Hkv, tail=0, tail_value=0.0):
+    """One sequence whose full block j holds the constant score consts[j] in
+    every (token, head) entry (so its mean is exactly consts[j]), plus a
+    partial block of `tail` tokens."""
+    MB = len(consts) + (1 if tail else 0)
+    s = np.full((1, MB * bs, Hkv), np.nan)
+    for j, c in enumerate(consts):
+        s[0, j * bs:(j + 1) * bs] = c
+    if tail:
+        s[0, len(consts) * bs:len(consts) * bs + tail] = tail_value
+    return s, np.array([len(consts) * bs + tail], np.int32)
+
+
+def test_threshold_policy_trigger_boundary():
+    s, lens = _block_scores([0.5, 0.01, 2.0], 4, 2)
+    # usage 80 of 100 with eviction_ratio 0.2 is not above 80 %: nothing happens
+    mask, count, _ = oracle.select_evict_threshold(s, lens, 4, 80, 100, 0.2, 0.1)
+    assert count[0] == 0 and not mask.any()
+    mask, count, _ = oracle.select_evict_threshold(s, lens, 4, 81, 100, 0.2, 0.1)
+    assert count[0] == 1 and mask[0].tolist() == [0, 1, 0]
+
+
+def test_threshold_policy_marks_every_block_below_threshold():
+    # dyadic constants: every block sum and mean is exact in fp64
+    consts = [0.5, 0.0625, 2.0, 0.09375, 0.125, 3.0, 0.1171875]
+    s, lens = _block_scores(consts, 16, 8, tail=5, tail_value=0.001)
+    mask, count, means = oracle.select_evict_threshold(s, lens, 16, 95, 100, 0.2, 0.125)
+    # strictly below 0.125; the partial last block never counts however low it is
+    assert mask[0].tolist() == [0, 1, 0, 1, 0, 0, 1, 0]
+    assert count[0] == 3
+    assert means[0, :7].tolist() == consts
+
+
+def test_threshold_policy_without_low_blocks_is_the_decode_argmin():
+    rng = np.random.default_rng(21)
+    B, MB, bs, Hkv = 5, 9, 8, 2
+    lens = np.array([72, 71, 8, 7, 40], np.int32)
+    s = np.abs(rng.standard_normal((B, MB * bs, Hkv))) + 0.5
+    mask, count, _ = oracle.select_evict_threshold(s, lens, bs, 99, 100, 0.2, 0.1)
+    ev, _, _ = oracle.select_evict_block(s, lens, bs)
+    for b in range(B):
+        want = np.zeros(MB, np.uint8)
+        if ev[b] >= 0:
+            want[ev[b]] = 1
+        assert mask[b].tolist() == want.tolist() and count[b] == int(ev[b] >= 0)
+
+
+def test_compact_mask_single_block_equals_single_eviction():
+    rng = np.random.default_rng(22)
+    bs, MB = 4, 7
+    lens = np.array([28, 27, 9, 3], np.int32)
+    bt = np.full((4, MB), -1, np.int32)
+    perm = rng.permutation(40).astype(np.int32)
+    c = 0
+    for b, n in enumerate(lens):
+        m = -(-int(n) // bs)
+        bt[b, :m] = perm[c:c + m]
+        c += m
+    evict = np.array([6, 3, 1, -1], np.int32)
+    mask = np.zeros((4, MB), np.uint8)
+    for b, j in enumerate(evict):
+        if j >= 0:
+            mask[b, j] = 1
+    a_bt, a_len, a_fr = oracle.evict_compact(bt, lens, evict, bs)
+    m_bt, m_len, m_fr = oracle.evict_compact_mask(bt, lens, mask, bs)
+    assert np.array_equal(a_bt, m_bt) and np.array_equal(a_len, m_len)
+    assert np.array_equal(m_fr[:, 0], a_fr) and (m_fr[:, 1:] == -1).all()
+
+
+def test_compact_mask_preserves_token_to_slot_map():
+    rng = np.random.default_rng(23)
+    bs, MB = 4, 12
+    lens = np.array([46, 48, 13], np.int32)
+    bt = np.full((3, MB), -1, np.int32)
+    perm = rng.permutation(60).astype(np.int32)
+    c = 0
+    for b, n in enumerate(lens):
+        m = -(-int(n) // bs)
+        bt[b, :m] = perm[c:c + m]
+        c += m
+    mask = np.zeros((3, MB), np.uint8)
+    mask[0, [0, 3, 4, 10]] = 1
+    mask[0, 11] = 1           # the partial block: ignored
+    mask[1, [11, 5]] = 1      # includes the newest full block
+    mask[2, 3] = 1            # partial: ignored
+    nbt, nlen, fr = oracle.evict_compact_mask(bt, lens, mask, bs)
+    for b in range(3):
+        full = lens[b] // bs
+        gone = [j for j in range(full) if mask[b, j]]
+        assert nlen[b] == lens[b] - bs * len(gone)
+        assert fr[b, :len(gone)].tolist() == [int(bt[b, j]) for j in gone]
+        assert (fr[b, len(gone):] == -1).all()
+        for p in range(lens[b]):
+            j = p // bs
+            if j in gone:
+                continue
+            q = p - bs * sum(1 for g in gone if g < j)
+            assert oracle.slot(nbt[b], q, bs) == oracle.slot(bt[b], p, bs)
+        assert (nbt[b, -(-int(nlen[b]) // bs):] == -1).all()
