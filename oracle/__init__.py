@@ -69,6 +69,9 @@ def _lib():
                                                   dbl, dbl]
         lib.or_evict_compact_mask.restype = None
         lib.or_evict_compact_mask.argtypes = [p, p, p, p, i32, i32, i32]
+        lib.or_paged_prefill.restype = None
+        lib.or_paged_prefill.argtypes = [p, p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32,
+                                         dbl]
         lib.or_e4m3_to_f64.restype = dbl
         lib.or_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         lib.or_append_kv_fp8.restype = None
@@ -371,3 +374,22 @@ def evict_compact_mask(bt, ctx_lens, mask, bs):
     freed = np.empty((B, MB), np.int32)
     _lib().or_evict_compact_mask(_ptr(bt), _ptr(ctx), _ptr(freed), _ptr(mask), B, MB, bs)
     return bt, ctx, freed
+
+
+# --------------------------------------------------------------------------- chunked prefill
+def paged_prefill(q, cu_q, k_cache, v_cache, block_stride, bt, ctx_lens, Hkv, bs, scale):
+    """fp64 multi-query paged attention: the q_len_b query tokens of sequence b
+    are its last q_len_b cached tokens and attend causally.  q [Tq, Hq, d] bf16
+    bits, cu_q [B+1] int32.  Returns out [Tq, Hq, d] float64."""
+    q = _c(q, np.uint16)
+    cu_q = _c(cu_q, np.int32)
+    k_cache = _c(k_cache, np.uint16)
+    v_cache = _c(v_cache, np.uint16)
+    bt = _c(bt, np.int32)
+    ctx_lens = _c(ctx_lens, np.int32)
+    Tq, Hq, d = q.shape
+    B, MB = bt.shape
+    out = np.empty((Tq, Hq, d), np.float64)
+    _lib().or_paged_prefill(_ptr(out), _ptr(q), _ptr(cu_q), _ptr(k_cache), _ptr(v_cache),
+                            block_stride, _ptr(bt), MB, _ptr(ctx_lens), B, Hq, Hkv, d, bs, scale)
+    return out

@@ -639,3 +639,48 @@ void or_evict_compact_mask(int32_t *bt, int32_t *ctx_lens, int32_t *freed, const
         ctx_lens[b] = len - nf * bs;
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Multi-query paged attention (chunked prefill)                             */
+/* ------------------------------------------------------------------------ */
+
+/* Paged attention with several query tokens per sequence, as a chunked prefill
+ * runs it (t6page "KV cache" page, "Chunked prefill：让 prefill 不阻塞 decode": a
+ * long prompt is prefilled 512 tokens at a time, each chunk batched with the
+ * running decodes; the operator is the paged attention of "PagedAttention 的算子"
+ * and [VKV] §2.2 with more than one query row).  Readings: the chunk's own K/V
+ * rows were appended before the call, so sequence b holds ctx_lens[b] tokens and
+ * its q_len_b = cu_q[b+1] - cu_q[b] query tokens are the last q_len_b of them;
+ * query token i of b sits at position p = ctx_lens[b] - q_len_b + i and attends
+ * exactly the tokens t <= p (causal), softmax over all of them; q_len_b = 1 is
+ * a decode step.  A sequence with q_len_b > ctx_lens[b] or a length outside
+ * [0, MB*bs] is invalid and its output rows are zero.
+ * q [Tq][Hq][d] bf16 (Tq = cu_q[B]); out [Tq][Hq][d] fp64. */
+void or_paged_prefill(double *out, const uint16_t *q, const int32_t *cu_q,
+                      const uint16_t *k_cache, const uint16_t *v_cache, int64_t block_stride,
+                      const int32_t *bt, int MB, const int32_t *ctx_lens, int B, int Hq, int Hkv,
+                      int d, int bs, double scale) {
+    const int G = Hq / Hkv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b) {
+        const int ql = cu_q[b + 1] - cu_q[b];
+        int len = ctx_lens[b];
+        const int bad = len < 0 || (int64_t)len > (int64_t)MB * bs || ql > len;
+        if (bad) len = 0;
+        double *Kc = (double *)malloc(sizeof(double) * ((size_t)len * Hkv * d + 1));
+        double *Vc = (double *)malloc(sizeof(double) * ((size_t)len * Hkv * d + 1));
+        double *s = (double *)malloc(sizeof(double) * ((size_t)len + 1));
+        double *qv = (double *)malloc(sizeof(double) * (size_t)d);
+        gather_seq(Kc, Vc, k_cache, v_cache, NULL, NULL, load_bf16, block_stride, 0,
+                   bt + (int64_t)b * MB, len, Hkv, d, bs);
+        for (int r = 0; r < ql; ++r) {
+            const int64_t row = (int64_t)cu_q[b] + r;
+            const int upto = bad ? 0 : len - ql + r + 1;   /* tokens 0 .. p */
+            for (int i = 0; i < Hq; ++i) {
+                for (int e = 0; e < d; ++e) qv[e] = bf16_to_f64(q[(row * Hq + i) * d + e]);
+                attend_one(out + (row * Hq + i) * d, qv, Kc, Vc, upto, Hkv, i / G, d, scale, s);
+            }
+        }
+        free(Kc); free(Vc); free(s); free(qv);
+    }
+}

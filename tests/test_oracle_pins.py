@@ -813,3 +813,59 @@ def test_compact_mask_preserves_token_to_slot_map():
             q = p - bs * sum(1 for g in gone if g < j)
             assert oracle.slot(nbt[b], q, bs) == oracle.slot(bt[b], p, bs)
         assert (nbt[b, -(-int(nlen[b]) // bs):] == -1).all()
+
+
+# ----------------------------------------------------------------------------- chunked prefill
+def _prefill_case(seed, qlens, lens, Hq=8, Hkv=2, d=16, bs=4, N=60):
+    c = rand_case(seed, B=len(lens), Hq=Hq, Hkv=Hkv, d=d, bs=bs, N=N, lens=tuple(lens))
+    rng = np.random.default_rng(seed + 1000)
+    cu = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    c["qp"] = bf16_bits(rng.standard_normal((int(cu[-1]), Hq, d))).reshape(-1, Hq, d)
+    c["cu"] = cu
+    return c
+
+
+def run_prefill(c):
+    return oracle.paged_prefill(c["qp"], c["cu"], c["kc"].ravel(), c["vc"].ravel(),
+                                c["bs"] * c["Hkv"] * c["d"], c["bt"], c["lens"], c["Hkv"],
+                                c["bs"], 1.0 / math.sqrt(c["d"]))
+
+
+@pytest.mark.parametrize("seed,Hq,Hkv,d,bs", [(1, 8, 2, 16, 4), (2, 4, 4, 8, 3), (3, 8, 1, 32, 5)])
+def test_prefill_attention_equals_causal_sdpa(seed, Hq, Hkv, d, bs):
+    """Against torch's fp64 scaled_dot_product_attention on the logically
+    gathered K/V with the offset causal mask (query i of a q_len chunk at the
+    end of n tokens sees tokens 0 .. n - q_len + i)."""
+    qlens, lens = [5, 1, 13, 0], [23, 9, 13, 4]
+    c = _prefill_case(seed, qlens, lens, Hq=Hq, Hkv=Hkv, d=d, bs=bs)
+    got = run_prefill(c)
+    for b, (ql, n) in enumerate(zip(qlens, lens)):
+        if ql == 0:
+            continue
+        K, V = gather_logical(c, b)
+        Kt = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)
+        Vt = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)
+        qt = torch.from_numpy(bf16_vals(c["qp"][c["cu"][b]:c["cu"][b + 1]])).permute(1, 0, 2)
+        allowed = torch.arange(n)[None, :] <= (n - ql + torch.arange(ql))[:, None]
+        o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, attn_mask=allowed,
+                                                             scale=1 / math.sqrt(d))
+        assert np.allclose(got[c["cu"][b]:c["cu"][b + 1]], o.permute(1, 0, 2).numpy(),
+                           rtol=1e-12, atol=1e-13)
+
+
+def test_prefill_attention_single_query_is_decode():
+    lens = [23, 9, 13, 1]
+    c = _prefill_case(5, [1, 1, 1, 1], lens)
+    c["q"] = c["qp"].reshape(len(lens), c["Hq"], c["d"])
+    assert np.array_equal(run_prefill(c), run_decode(c))
+
+
+def test_prefill_attention_is_causal_and_invalid_rows_are_zero():
+    c = _prefill_case(6, [6, 3], [20, 2])   # sequence 1 asks 3 queries of 2 tokens: invalid
+    base = run_prefill(c)
+    assert not base[6:].any()
+    # change the last token of sequence 0: only its last query row moves
+    b0_last = c["bt"][0, (20 - 1) // c["bs"]]
+    c["kc"][b0_last, (20 - 1) % c["bs"]] = bf16_bits(np.full((c["Hkv"], c["d"]), 3.0))
+    moved = run_prefill(c)
+    assert np.array_equal(moved[:5], base[:5]) and not np.array_equal(moved[5], base[5])
