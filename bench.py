@@ -49,8 +49,9 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="c3", choices=["c2", "c3", "c4", "c5", "p1"],
-                    help="c2..c5: decode steps; p1: PagedEviction prefill compression")
+    ap.add_argument("--workload", default="c3", choices=["c2", "c3", "c4", "c5", "p1", "p2"],
+                    help="c2..c5: decode steps; p1: PagedEviction prefill compression; "
+                         "p2: chunked prefill attention")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--kv", default=None, choices=["bf16", "int8", "fp8"],
                     help="KV storage type (default: the workload's own)")
@@ -396,6 +397,8 @@ def run_reference(args):
         return 0
     if args.workload in W.PREFILL:
         return run_reference_prefill(args)
+    if args.workload in W.CHUNKED:
+        return run_reference_chunked(args)
     cfg = workload_cfg(args)
     wl = W.generate(cfg, "cpu", layers=1)
     per = max(1.0, args.cpu_seconds / max(1, args.steps))
@@ -465,6 +468,35 @@ def run_reference_prefill(args):
         "cpu_baseline": {"value": value, "unit": "prompt tokens/s", "cores": cores,
                          "kind": "oracle", "sample": "per step: " + desc},
         "e2e": {"value": value, "unit": "prompt tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference_chunked(args):
+    """The oracle's chunked prefill attention timed on row samples of the workload."""
+    cfg = W.CHUNKED[args.workload]
+    wl = W.generate_chunked(cfg, "cpu")
+    per = max(1.0, args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        chunk_oracle_throughput(wl, per / 4)
+    vals, desc, cores = [], "", 0
+    for _ in range(args.steps):
+        v, cores, desc = chunk_oracle_throughput(wl, per)
+        vals.append(v)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": "chunked prefill attention: chunk tokens/s",
+        "value": value, "unit": "chunk tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.batch * cfg.chunk / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{cfg.key} {cfg.name}", "sequences": cfg.batch,
+                   "chunk": cfg.chunk, "context": cfg.ctx_len},
+        "cpu_baseline": {"value": value, "unit": "chunk tokens/s", "cores": cores,
+                         "kind": "oracle", "sample": "per step: " + desc},
+        "e2e": {"value": value, "unit": "chunk tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -645,6 +677,161 @@ def run_prefill(args, device, world, rank):
     return 0
 
 
+# ----------------------------------------------------------------------------- chunked prefill
+def chunk_flops(cfg):
+    """QK^T and PV flops of one chunk step: query token i of a chunk ending at
+    context n sees n - chunk + i + 1 tokens; 4*d flops per (row, token, head)."""
+    seen = sum(cfg.ctx_len - cfg.chunk + i + 1 for i in range(cfg.chunk))
+    return 4.0 * cfg.head_dim * cfg.hq * seen * cfg.batch
+
+
+def chunk_oracle_throughput(wl, budget_s):
+    """The oracle's append + multi-query attention on query-row samples: one
+    sequence's chunk, a slice of its query rows at a time (rows cost in
+    proportion to the tokens they see, so the sample is scaled by that)."""
+    import oracle
+    cfg = wl.cfg
+    Hkv, d, bs = cfg.hkv, cfg.head_dim, cfg.block_size
+    stride = bs * Hkv * d
+    kc = W.bits(wl.k_pool).ravel().copy()
+    vc = W.bits(wl.v_pool).ravel().copy()
+    bt = wl.block_tables[:1]
+    oracle.append_kv(W.bits(wl.k_new[:1]), W.bits(wl.v_new[:1]), kc, vc, stride, bt,
+                     wl.positions[:1], bs)
+    t_total, seen, rows = 0.0, 0, 0
+    step = 16
+    for r0 in range(0, cfg.chunk, step):
+        # rows r0 .. r0+step-1 of the chunk as their own causal chunk ending at their position
+        n = cfg.ctx_len - cfg.chunk + r0 + step
+        q = W.bits(wl.q[r0:r0 + step])
+        t0 = time.perf_counter()
+        oracle.paged_prefill(q, np.array([0, step], np.int32), kc, vc, stride, bt,
+                             np.array([n], np.int32), Hkv, bs, wl.scale)
+        t_total += time.perf_counter() - t0
+        seen += sum(n - step + i + 1 for i in range(step))
+        rows += step
+        if t_total >= budget_s:
+            break
+    full_seen = cfg.batch * sum(cfg.ctx_len - cfg.chunk + i + 1 for i in range(cfg.chunk))
+    step_s = t_total / seen * full_seen
+    desc = (f"{rows} query rows of one chunk ({seen} row-token pairs, all heads), "
+            f"{t_total:.1f} s, scaled by the {full_seen} row-token pairs of a step")
+    return cfg.batch * cfg.chunk / step_s, oracle.threads(), desc
+
+
+def run_chunked(args, device, world, rank):
+    """One step = append the chunk's K/V rows and run the multi-query attention
+    for every sequence of the workload."""
+    import paged_kv_cache_396_b200.pagedkv as pk
+    cfg = W.CHUNKED[args.workload]
+    wl = W.generate_chunked(cfg, device)
+    B = cfg.batch
+    Tq = B * cfg.chunk
+    bt = torch.as_tensor(wl.block_tables, device=device)
+    ctx = torch.as_tensor(wl.ctx_lens, device=device)
+    pos = torch.as_tensor(wl.positions, device=device)
+    cu = torch.as_tensor(wl.cu_q, device=device)
+    out = torch.empty(Tq, cfg.hq, cfg.head_dim, dtype=torch.bfloat16, device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        pk.pa_append_kv(wl.k_new, wl.v_new, wl.k_pool, wl.v_pool, bt, pos, err)
+        if ev:
+            ev[0].record(stream)
+        pk.pa_prefill_attention(out, wl.q, cu, cfg.chunk, wl.k_pool, wl.v_pool, bt, ctx,
+                                wl.scale, err)
+        if ev:
+            ev[1].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    if err.item() != 0:
+        raise SystemExit(f"device error flag {err.item()} during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    clocks = Clocks(device)
+    time.sleep(0.3)
+    total = 0.0
+    for k in range(args.steps):
+        flush.zero_()                 # L2 flushed between timed steps (K/V is ~140 MB)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        step(evs[k])
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+        total += t0.elapsed_time(t1)
+    clk = clocks.stop()
+    ms = reduce_max(total / args.steps, world)
+    attn_s = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) / 1000.0
+    flops = chunk_flops(cfg)
+    peak_t = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"] \
+        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 1590.0
+    achieved = flops / attn_s / 1e12
+
+    # end to end: queries and chunk rows from pinned host memory, output back
+    h_in = []
+    for t in (wl.q, wl.k_new, wl.v_new):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        h_in.append((h, t))
+    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    torch.cuda.synchronize(device)
+    a = torch.cuda.Event(enable_timing=True)
+    z = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 20))
+    a.record(stream)
+    for _ in range(e2e_steps):
+        for h, t in h_in:
+            t.copy_(h, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+    z.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = reduce_max(a.elapsed_time(z) / e2e_steps, world)
+    if err.item() != 0:
+        raise SystemExit(f"device error flag {err.item()} during timing")
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_, cores, desc = chunk_oracle_throughput(
+            W.ChunkWorkload(cfg, wl.k_pool.cpu(), wl.v_pool.cpu(), wl.k_new.cpu(),
+                            wl.v_new.cpu(), wl.q.cpu(), wl.cu_q, wl.ctx_lens, wl.positions,
+                            wl.block_tables, wl.num_blocks), args.cpu_seconds)
+        cpu = {"value": v_, "unit": "chunk tokens/s", "cores": cores, "kind": "oracle",
+               "sample": desc}
+    if rank == 0:
+        line = {
+            "metric": "chunked prefill attention: chunk tokens/s and tensor TFLOP/s",
+            "value": world * Tq / (ms / 1000.0), "unit": "chunk tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"{cfg.key} {cfg.name}", "sequences": B,
+                       "chunk": cfg.chunk, "context": cfg.ctx_len, "q_heads": cfg.hq,
+                       "kv_heads": cfg.hkv, "head_dim": cfg.head_dim,
+                       "block_size": cfg.block_size, "parallelism": f"replicas{world}",
+                       "l2": "flushed (256 MB write) before every timed step"},
+            "roofline": {"bound": "tensor", "kernel": "pa_prefill_attention",
+                         "achieved": achieved, "peak": peak_t, "peak_source": "measured burst",
+                         "unit": "TFLOP/s", "frac": achieved / peak_t, "traffic": None,
+                         "algorithmic_flops_per_launch": flops, "avg_launch_us": attn_s * 1e6},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * Tq / (e2e_ms / 1000.0), "unit": "chunk tokens/s",
+                    "h2d_bytes_per_step": sum(t.numel() * t.element_size() for _, t in h_in),
+                    "d2h_bytes_per_step": out.numel() * out.element_size(),
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- main
 def main():
     args = parse()
@@ -662,8 +849,9 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
-    if args.workload in W.PREFILL:
-        rc = run_prefill(args, device, world, rank)
+    if args.workload in W.PREFILL or args.workload in W.CHUNKED:
+        fn = run_prefill if args.workload in W.PREFILL else run_chunked
+        rc = fn(args, device, world, rank)
         if world > 1:
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()

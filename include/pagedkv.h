@@ -363,6 +363,67 @@ int pe_evict_compact(int32_t *block_tables, int max_blocks_per_seq, int32_t *ctx
                      int32_t *freed, const int32_t *evict, int B, int bs, int32_t *err_flag,
                      void *stream);
 
+/* ============================================================================
+ * Threshold eviction policy  (blog.hotdry.top nano-vLLM KV cache page, section
+ * "工程落地：参数配置与监控要点": eviction_ratio = 0.2 starts eviction once the
+ * cache is more than 80 % used; blocks below importance_threshold go first).
+ *
+ * pe_select_evict_threshold: the trigger is evaluated on the host, in fp64, as
+ *   used_blocks > (1 - eviction_ratio) * total_blocks (the caller's allocator
+ *   counts).  Triggered: for each sequence every full block whose mean
+ *   importance (as in pe_select_evict_block) is below importance_threshold is
+ *   marked; a sequence with no such block marks its single lowest-mean full
+ *   block (ties to the lowest index); no full block marks nothing.  Not
+ *   triggered: nothing is marked.  Reading: the page gives the two parameters
+ *   and their intent, not how many blocks go; this is the plainest rule that
+ *   honours both and reduces to the decode-phase rule when nothing is below
+ *   the threshold.
+ *   mask [B][MB] uint8 (1 = evict), count [B] int32 (marked blocks),
+ *   block_means (nullable) [B][MB] float, NaN for non-candidates.
+ *   eviction_ratio in [0, 1]; importance_threshold not NaN.
+ *
+ * pe_evict_compact_mask: pe_evict_compact for any number of marked full blocks
+ *   per sequence: marked full blocks leave the table, the other entries keep
+ *   their order and close up, ctx_lens[b] drops by bs per removed block, and
+ *   freed (nullable [B][MB]) lists the removed physical ids in logical order,
+ *   -1 after the last.  A mark on the partial last block sets
+ *   PA_DEV_BAD_EVICT and is ignored; marks at j >= ceil(len/bs) are not read.
+ * ==========================================================================*/
+int pe_select_evict_threshold(uint8_t *mask, int32_t *count, float *block_means,
+                              const float *scores, const int32_t *ctx_lens, int B,
+                              int max_blocks_per_seq, int Hkv, int bs, int64_t used_blocks,
+                              int64_t total_blocks, double eviction_ratio,
+                              double importance_threshold, void *stream);
+
+int pe_evict_compact_mask(int32_t *block_tables, int max_blocks_per_seq, int32_t *ctx_lens,
+                          int32_t *freed, const uint8_t *mask, int B, int bs, int32_t *err_flag,
+                          void *stream);
+
+/* ============================================================================
+ * Multi-query paged attention for a chunked prefill  (t6page.pages.dev "KV
+ * cache", "Chunked prefill：让 prefill 不阻塞 decode": a long prompt is prefilled
+ * in chunks, 512 tokens each, batched with the running decodes; the operator is
+ * the paged attention of "PagedAttention 的算子" / [VKV] §2.2 with several query
+ * tokens per sequence).
+ *
+ * Sequence b has q_len_b = cu_q[b+1] - cu_q[b] query tokens, rows cu_q[b] ..
+ * cu_q[b+1]-1 of q and out ([Tq][Hq][d] bf16, Tq = cu_q[B]).  Its chunk's K/V
+ * rows were appended before the call (pa_append_kv with n_new = q_len_b), so
+ * the queries are the last q_len_b of its ctx_lens[b] cached tokens: query i
+ * sits at position p = ctx_lens[b] - q_len_b + i and attends exactly the tokens
+ * t <= p (causal), softmax over all of them, GQA groups as in pa_decode.
+ * q_len_b = 1 is a decode step (pa_decode is the faster call for those).
+ * max_q_len >= every q_len_b (sizes the grid).  d in {64, 128}; G = Hq/Hkv in
+ * {1, 2, 4, 8, 16}.  A sequence with q_len_b > ctx_lens[b] or a length outside
+ * [0, MB*bs] gets zero output rows and sets PA_DEV_BAD_LEN; a block id outside
+ * [0, N) sets PA_DEV_BAD_BLOCK and reads as zeros.  No workspace.
+ * ==========================================================================*/
+int pa_prefill_attention(uint16_t *out, const uint16_t *q, const int32_t *cu_q, int max_q_len,
+                         const uint16_t *k_cache, const uint16_t *v_cache, int64_t block_stride,
+                         const int32_t *block_tables, int max_blocks_per_seq,
+                         const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
+                         int64_t num_blocks, float scale, int32_t *err_flag, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -661,7 +661,6 @@ void or_paged_prefill(double *out, const uint16_t *q, const int32_t *cu_q,
                       const int32_t *bt, int MB, const int32_t *ctx_lens, int B, int Hq, int Hkv,
                       int d, int bs, double scale) {
     const int G = Hq / Hkv;
-#pragma omp parallel for schedule(dynamic, 1)
     for (int b = 0; b < B; ++b) {
         const int ql = cu_q[b + 1] - cu_q[b];
         int len = ctx_lens[b];
@@ -669,18 +668,22 @@ void or_paged_prefill(double *out, const uint16_t *q, const int32_t *cu_q,
         if (bad) len = 0;
         double *Kc = (double *)malloc(sizeof(double) * ((size_t)len * Hkv * d + 1));
         double *Vc = (double *)malloc(sizeof(double) * ((size_t)len * Hkv * d + 1));
-        double *s = (double *)malloc(sizeof(double) * ((size_t)len + 1));
-        double *qv = (double *)malloc(sizeof(double) * (size_t)d);
         gather_seq(Kc, Vc, k_cache, v_cache, NULL, NULL, load_bf16, block_stride, 0,
                    bt + (int64_t)b * MB, len, Hkv, d, bs);
-        for (int r = 0; r < ql; ++r) {
+        /* every (query token, head) row is independent: rows in parallel */
+#pragma omp parallel for schedule(dynamic, 1)
+        for (int64_t ri = 0; ri < (int64_t)ql * Hq; ++ri) {
+            const int r = (int)(ri / Hq), i = (int)(ri % Hq);
             const int64_t row = (int64_t)cu_q[b] + r;
             const int upto = bad ? 0 : len - ql + r + 1;   /* tokens 0 .. p */
-            for (int i = 0; i < Hq; ++i) {
-                for (int e = 0; e < d; ++e) qv[e] = bf16_to_f64(q[(row * Hq + i) * d + e]);
-                attend_one(out + (row * Hq + i) * d, qv, Kc, Vc, upto, Hkv, i / G, d, scale, s);
-            }
+            double *s = (double *)malloc(sizeof(double) * ((size_t)len + 1));
+            double *qv = (double *)malloc(sizeof(double) * (size_t)d);
+            for (int e = 0; e < d; ++e) qv[e] = bf16_to_f64(q[(row * Hq + i) * d + e]);
+            attend_one(out + (row * Hq + i) * d, qv, Kc, Vc, upto, Hkv, i / G, d, scale, s);
+            free(s);
+            free(qv);
         }
-        free(Kc); free(Vc); free(s); free(qv);
+        free(Kc);
+        free(Vc);
     }
 }

@@ -1,0 +1,50 @@
+// blockmean.cuh -- the decode-phase block mean of PagedEviction (blog.hotdry.top
+// "KV缓存内存布局优化", "PagedEviction 块级驱逐机制": the mean importance of
+// every complete block), computed by one warp per block.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <limits.h>
+#include <stdint.h>
+
+namespace pkv {
+
+// Mean of the `per` fp32 scores at p (bs*Hkv entries of one block): coalesced
+// loads, fp64 partial sums per lane, butterfly reduction.  Every lane returns
+// the same value.
+__device__ __forceinline__ double warp_block_mean(const float *__restrict__ p, int per,
+                                                  int lane) {
+    double s = 0.0;
+    for (int k = lane; k < per; k += 32) s += (double)__ldg(p + k);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    return s / (double)per;
+}
+
+// (mean, j) argmin with ties to the lowest j; j = INT_MAX marks "none".
+__device__ __forceinline__ void argmin_take(double &best, int &bj, double m, int j) {
+    if (j != INT_MAX && (bj == INT_MAX || m < best || (m == best && j < bj))) {
+        best = m;
+        bj = j;
+    }
+}
+
+// CTA-wide argmin of per-warp candidates (every lane of a warp holds its
+// warp's candidate).  Returns the winner in every thread.
+__device__ __forceinline__ int cta_argmin(double best, int bj) {
+    __shared__ double sb[32];
+    __shared__ int sj[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) {
+        sb[warp] = best;
+        sj[warp] = bj;
+    }
+    __syncthreads();
+    double b = INFINITY;
+    int j = INT_MAX;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) argmin_take(b, j, sb[w], sj[w]);
+    __syncthreads();
+    return j;
+}
+
+}  // namespace pkv

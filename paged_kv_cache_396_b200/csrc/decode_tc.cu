@@ -28,8 +28,9 @@
 //   its query fragments
 //   straight from global memory (L2).  S = Q K^T with the G query heads of the group as
 //   the 16 rows of an m16n8k16 MMA (rows >= G are zero), online softmax on the
-//   fp32 accumulators (exp2 domain), P rounded to bf16, O += P V with V read by
-//   ldmatrix.trans.  The stage is released to the producer through an mbarrier.
+//   fp32 accumulators (exp2 domain), P split into two bf16 parts (hi + lo; for
+//   G <= 8 the lo part fills the empty rows g + 8 of the same MMA), O += P V with
+//   V read by ldmatrix.trans.  The stage is released to the producer through an mbarrier.
 //   At a unit's last stage the warp writes either the normalised bf16 output
 //   (single-partition sequence) or its (O, m, l) partial for the merge kernel.
 // Masking: tokens at or past the unit's end get -inf logits, and their V rows
@@ -317,6 +318,12 @@ __device__ __forceinline__ void load_q_bf16(const Args &a, int b, int h, int g, 
     }
 }
 
+// Low bf16 part of the pair (x, y) whose high parts are packed in `hi`:
+// bf16(x - hi.x), bf16(y - hi.y); the differences are exact in fp32.
+__device__ __forceinline__ uint32_t bf16_lo_part(float x, float y, uint32_t hi) {
+    return ptx::pack_bf16(x - bf16_lo(hi), y - bf16_hi(hi));
+}
+
 template <int D, bool G16>
 __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMeta *meta,
                                          uint64_t *full, uint64_t *empty) {
@@ -412,10 +419,17 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
             const float p2 = exp2f(x2 - mu), p3 = exp2f(x3 - mu);
             l = l * alpha + ((p0 + p1) + (p2 + p3));
             m = mn;
+            // P = hi + lo, both bf16: p - hi is exact in fp32 and lo carries the 8 bits
+            // that one bf16 would drop (a single bf16 P can be off by 2^-9 of the weight,
+            // too coarse when a few tokens hold most of the weight).  For G <= 8 the lo
+            // parts ride in the otherwise empty rows g + 8 of the same MMA.
             const uint32_t pa0 = ptx::pack_bf16(p0, p1), pa2 = ptx::pack_bf16(p2, p3);
-            uint32_t pa1 = 0u, pa3 = 0u;
+            uint32_t pa1 = bf16_lo_part(p0, p1, pa0), pa3 = bf16_lo_part(p2, p3, pa2);
+            uint32_t la0 = 0u, la1 = 0u, la2 = 0u, la3 = 0u;
             float alphab = 1.f;
             if constexpr (G16) {
+                la0 = pa1;
+                la2 = pa3;
                 float y0 = va0 ? s0[2] * sl : -INFINITY, y1 = va1 ? s0[3] * sl : -INFINITY;
                 float y2 = vb0 ? s1[2] * sl : -INFINITY, y3 = vb1 ? s1[3] * sl : -INFINITY;
                 float my = fmaxf(fmaxf(y0, y1), fmaxf(y2, y3));
@@ -430,6 +444,8 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
                 mb = mnb;
                 pa1 = ptx::pack_bf16(q0, q1);
                 pa3 = ptx::pack_bf16(q2, q3);
+                la1 = bf16_lo_part(q0, q1, pa1);
+                la3 = bf16_lo_part(q2, q3, pa3);
             }
             // rescale only when some row maximum moved (alpha == 1 exactly otherwise)
             if (__any_sync(kFull, alpha != 1.f || alphab != 1.f)) {
@@ -468,10 +484,19 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
                 }
                 ptx::mma_bf16(d0, pa0, pa1, pa2, pa3, r[0], r[1]);
                 ptx::mma_bf16(d1, pa0, pa1, pa2, pa3, r[2], r[3]);
-                o[2 * pj][0] = d0[0];
-                o[2 * pj][1] = d0[1];
-                o[2 * pj + 1][0] = d1[0];
-                o[2 * pj + 1][1] = d1[1];
+                if constexpr (G16) {  // the lo parts of all 16 rows: a second product
+                    ptx::mma_bf16(d0, la0, la1, la2, la3, r[0], r[1]);
+                    ptx::mma_bf16(d1, la0, la1, la2, la3, r[2], r[3]);
+                    o[2 * pj][0] = d0[0];
+                    o[2 * pj][1] = d0[1];
+                    o[2 * pj + 1][0] = d1[0];
+                    o[2 * pj + 1][1] = d1[1];
+                } else {              // rows g + 8 hold P_lo V: fold them into rows g
+                    o[2 * pj][0] = d0[0] + d0[2];
+                    o[2 * pj][1] = d0[1] + d0[3];
+                    o[2 * pj + 1][0] = d1[0] + d1[2];
+                    o[2 * pj + 1][1] = d1[1] + d1[3];
+                }
                 if constexpr (G16) {
                     ob[2 * pj][0] = d0[2];
                     ob[2 * pj][1] = d0[3];

@@ -5,8 +5,10 @@
 #include <limits.h>
 #include <math.h>
 
+#include "blockmean.cuh"
 #include "common.cuh"
 #include "kernels.h"
+#include "prefill.h"
 
 namespace pkv {
 
@@ -86,65 +88,74 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
     }
 }
 
-// One CTA per sequence.  Thread k owns the blocks j = k, k + blockDim, ...;
-// each block mean is an fp64 sum over the bs*Hkv fp32 scores in memory order
-// (token-major, then head) divided by bs*Hkv; then a (mean, j) argmin with
-// ties to the lowest j.
+// One CTA per sequence, one warp per full block (blocks j = warp, warp + 8, ...):
+// each block mean is an fp64 sum of its bs*Hkv fp32 scores divided by bs*Hkv;
+// then a (mean, j) argmin with ties to the lowest j.
 __global__ void __launch_bounds__(256) select_evict_kernel(int32_t *evict, float *means,
                                                            const float *scores,
                                                            const int32_t *ctx_lens, int MB,
                                                            int Hkv, int bs) {
     const int b = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     int len = ctx_lens[b];
     if (len < 0 || (int64_t)len > (int64_t)MB * bs) len = 0;
     const int nfull = len / bs;
     const int per = bs * Hkv;
     double best = INFINITY;
     int bj = INT_MAX;
-    for (int j = threadIdx.x; j < MB; j += blockDim.x) {
+    for (int j = warp; j < MB; j += nw) {
         if (j < nfull) {
-            const float *p = scores + ((int64_t)b * MB + j) * per;
-            double s = 0.0;
-            for (int k = 0; k < per; ++k) s += (double)p[k];
-            const double mean = s / (double)per;
-            if (means) means[(int64_t)b * MB + j] = (float)mean;
-            if (bj == INT_MAX || mean < best) {
-                best = mean;
-                bj = j;
-            }
-        } else if (means) {
+            const double mean = warp_block_mean(scores + ((int64_t)b * MB + j) * per, per, lane);
+            if (means && lane == 0) means[(int64_t)b * MB + j] = (float)mean;
+            argmin_take(best, bj, mean, j);
+        } else if (means && lane == 0) {
             means[(int64_t)b * MB + j] = __int_as_float(0x7fc00000);  // NaN: not a candidate
         }
     }
-    // (best, bj) argmin across the block, lowest j on equal means
-    __shared__ double sb[32];
-    __shared__ int sj[32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const double ob = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-        if (oj != INT_MAX && (bj == INT_MAX || ob < best || (ob == best && oj < bj))) {
-            best = ob;
-            bj = oj;
-        }
-    }
-    if (lane == 0) {
-        sb[warp] = best;
-        sj[warp] = bj;
-    }
+    const int win = cta_argmin(best, bj);
+    if (threadIdx.x == 0) evict[b] = (nfull > 0 && win != INT_MAX) ? win : -1;
+}
+
+// Threshold policy: with the trigger on, every full block whose mean is below
+// `thr` is marked, else the lowest-mean full block; with it off nothing is
+// marked.  Means are written either way.
+__global__ void __launch_bounds__(256) select_threshold_kernel(
+    uint8_t *mask, int32_t *count, float *means, const float *scores, const int32_t *ctx_lens,
+    int MB, int Hkv, int bs, double thr, int triggered) {
+    __shared__ int s_count;
+    const int b = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    if (threadIdx.x == 0) s_count = 0;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        const int nw = blockDim.x >> 5;
-        best = sb[0];
-        bj = sj[0];
-        for (int w = 1; w < nw; ++w) {
-            if (sj[w] != INT_MAX && (bj == INT_MAX || sb[w] < best || (sb[w] == best && sj[w] < bj))) {
-                best = sb[w];
-                bj = sj[w];
-            }
+    int len = ctx_lens[b];
+    if (len < 0 || (int64_t)len > (int64_t)MB * bs) len = 0;
+    const int nfull = len / bs;
+    const int per = bs * Hkv;
+    double best = INFINITY;
+    int bj = INT_MAX;
+    for (int j = warp; j < MB; j += nw) {
+        uint8_t below = 0;
+        if (j < nfull) {
+            const double mean = warp_block_mean(scores + ((int64_t)b * MB + j) * per, per, lane);
+            if (means && lane == 0) means[(int64_t)b * MB + j] = (float)mean;
+            argmin_take(best, bj, mean, j);
+            below = triggered && mean < thr;
+        } else if (means && lane == 0) {
+            means[(int64_t)b * MB + j] = __int_as_float(0x7fc00000);
         }
-        evict[b] = (nfull > 0 && bj != INT_MAX) ? bj : -1;
+        if (lane == 0) {
+            mask[(int64_t)b * MB + j] = below;
+            if (below) atomicAdd(&s_count, 1);
+        }
+    }
+    const int win = cta_argmin(best, bj);  // its barriers also order the s_count adds
+    if (threadIdx.x == 0) {
+        int n = s_count;
+        if (triggered && n == 0 && nfull > 0 && win != INT_MAX) {
+            mask[(int64_t)b * MB + win] = 1;
+            n = 1;
+        }
+        count[b] = n;
     }
 }
 
@@ -159,6 +170,14 @@ cudaError_t launch_select_evict(int32_t *evict, float *means, const float *score
                                 const int32_t *ctx_lens, int B, int MB, int Hkv, int bs,
                                 cudaStream_t st) {
     select_evict_kernel<<<B, 256, 0, st>>>(evict, means, scores, ctx_lens, MB, Hkv, bs);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select_threshold(uint8_t *mask, int32_t *count, float *means,
+                                    const float *scores, const int32_t *ctx_lens, int B, int MB,
+                                    int Hkv, int bs, double thr, int triggered, cudaStream_t st) {
+    select_threshold_kernel<<<B, 256, 0, st>>>(mask, count, means, scores, ctx_lens, MB, Hkv, bs,
+                                               thr, triggered);
     return cudaGetLastError();
 }
 

@@ -9,6 +9,7 @@
 
 #include "kernels.h"
 #include "prefill.h"
+#include "prefill_attn.h"
 #include "pagedkv.h"
 
 namespace {
@@ -521,4 +522,84 @@ int pe_evict_compact(int32_t *block_tables, int max_blocks_per_seq, int32_t *ctx
     return finish(pkv::launch_evict_compact(block_tables, max_blocks_per_seq, ctx_lens, freed,
                                             evict, B, bs, err_flag,
                                             static_cast<cudaStream_t>(stream)));
+}
+
+int pe_select_evict_threshold(uint8_t *mask, int32_t *count, float *block_means,
+                              const float *scores, const int32_t *ctx_lens, int B,
+                              int max_blocks_per_seq, int Hkv, int bs, int64_t used_blocks,
+                              int64_t total_blocks, double eviction_ratio,
+                              double importance_threshold, void *stream) {
+    if (B == 0) return PA_OK;
+    if (!mask || !count || !scores || !ctx_lens) return PA_ERR_NULL;
+    if (B < 0 || B > INT32_MAX / 2 || max_blocks_per_seq < 1 || Hkv < 1 || bs < 1)
+        return PA_ERR_SHAPE;
+    if (!(eviction_ratio >= 0.0 && eviction_ratio <= 1.0) ||
+        importance_threshold != importance_threshold || used_blocks < 0 || total_blocks < 0)
+        return PA_ERR_SHAPE;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    const int triggered = (double)used_blocks > (1.0 - eviction_ratio) * (double)total_blocks;
+    return finish(pkv::launch_select_threshold(mask, count, block_means, scores, ctx_lens, B,
+                                               max_blocks_per_seq, Hkv, bs, importance_threshold,
+                                               triggered, static_cast<cudaStream_t>(stream)));
+}
+
+int pe_evict_compact_mask(int32_t *block_tables, int max_blocks_per_seq, int32_t *ctx_lens,
+                          int32_t *freed, const uint8_t *mask, int B, int bs, int32_t *err_flag,
+                          void *stream) {
+    if (B == 0) return PA_OK;
+    if (!block_tables || !ctx_lens || !mask || !err_flag) return PA_ERR_NULL;
+    if (B < 0 || max_blocks_per_seq < 1 || bs < 1) return PA_ERR_SHAPE;
+    if ((int64_t)max_blocks_per_seq * bs > INT32_MAX) return PA_ERR_SHAPE;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    return finish(pkv::launch_evict_compact_mask(block_tables, max_blocks_per_seq, ctx_lens, freed,
+                                                 mask, B, bs, err_flag,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+int pa_prefill_attention(uint16_t *out, const uint16_t *q, const int32_t *cu_q, int max_q_len,
+                         const uint16_t *k_cache, const uint16_t *v_cache, int64_t block_stride,
+                         const int32_t *block_tables, int max_blocks_per_seq,
+                         const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
+                         int64_t num_blocks, float scale, int32_t *err_flag, void *stream) {
+    if (B == 0 || max_q_len == 0) return PA_OK;
+    if (!out || !q || !cu_q || !k_cache || !v_cache || !block_tables || !ctx_lens || !err_flag)
+        return PA_ERR_NULL;
+    int rc = check_common(B, Hkv, d, bs, max_blocks_per_seq, num_blocks, block_stride);
+    if (rc) return rc;
+    if (max_q_len < 0 || Hq < Hkv || Hq % Hkv != 0) return PA_ERR_SHAPE;
+    const int G = Hq / Hkv;
+    if (G > 16 || (G & (G - 1)) != 0) return PA_ERR_SHAPE;
+    if (!(scale == scale)) return PA_ERR_SHAPE;
+    if ((int64_t)max_q_len * G / 64 + 1 > INT32_MAX) return PA_ERR_SHAPE;
+    if (!al16(out) || !al16(q) || !al16(k_cache) || !al16(v_cache) || (block_stride * 2) % 16)
+        return PA_ERR_ALIGN;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    pkv::PrefillAttnArgs a;
+    memset(&a, 0, sizeof a);
+    a.out = out;
+    a.q = q;
+    a.cu_q = cu_q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_stride = block_stride;
+    a.block_tables = block_tables;
+    a.ctx_lens = ctx_lens;
+    a.err = err_flag;
+    a.N = num_blocks;
+    a.B = B;
+    a.MB = max_blocks_per_seq;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.G = G;
+    a.d = d;
+    a.bs = bs;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // tcgen05 / TMEM kernel for d = 128 and 16-token-aligned blocks (TMA pages);
+    // the mma.sync kernel covers every other supported shape
+    return finish(pkv::prefill_attn_tc_supported(a) ? pkv::launch_prefill_attn_tc(a, max_q_len, st)
+                                                    : pkv::launch_prefill_attn(a, max_q_len, st));
 }

@@ -288,7 +288,65 @@ __global__ void __launch_bounds__(128) evict_compact_kernel(int32_t *__restrict_
     }
 }
 
+// Several evicted blocks per sequence: the marked full blocks leave the table,
+// the others close up in order.  One warp per sequence walks the table 32
+// entries at a time; a ballot gives each survivor its new index and each
+// evicted entry its place in the freed list.  Writes land at or below the
+// entry being read and every round reads before it writes, so the compaction
+// is in place.
+__global__ void __launch_bounds__(128) evict_compact_mask_kernel(int32_t *__restrict__ bt,
+                                                                 int MB,
+                                                                 int32_t *__restrict__ ctx_lens,
+                                                                 int32_t *__restrict__ freed,
+                                                                 const uint8_t *__restrict__ mask,
+                                                                 int B, int bs, int32_t *err) {
+    const int lane = threadIdx.x & 31;
+    const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (b >= B) return;
+    const int len = ctx_lens[b];
+    int32_t *row = bt + (int64_t)b * MB;
+    int32_t *fr = freed ? freed + (int64_t)b * MB : nullptr;
+    const uint8_t *mk = mask + (int64_t)b * MB;
+    if (len < 0 || (int64_t)len > (int64_t)MB * bs) {
+        if (lane == 0) raise_flag(err, PA_DEV_BAD_LEN);
+        if (fr)
+            for (int x = lane; x < MB; x += 32) fr[x] = -1;
+        return;
+    }
+    const int nfull = len / bs, nblk = (len + bs - 1) / bs;
+    const unsigned below = (1u << lane) - 1u;
+    int w = 0, nf = 0;
+    for (int x0 = 0; x0 < nblk; x0 += 32) {
+        const int x = x0 + lane;
+        const bool in = x < nblk;
+        const int32_t val = in ? row[x] : 0;
+        const bool marked = in && mk[x] != 0;
+        const bool gone = marked && x < nfull;
+        if (marked && !gone) raise_flag(err, PA_DEV_BAD_EVICT);  // a partial block: ignored
+        const unsigned keep_m = __ballot_sync(kFull, in && !gone);
+        const unsigned gone_m = __ballot_sync(kFull, gone);
+        __syncwarp();
+        if (in && !gone) row[w + __popc(keep_m & below)] = val;
+        if (gone && fr) fr[nf + __popc(gone_m & below)] = val;
+        w += __popc(keep_m);
+        nf += __popc(gone_m);
+        __syncwarp();
+    }
+    for (int x = w + lane; x < nblk; x += 32) row[x] = -1;
+    if (fr)
+        for (int x = nf + lane; x < MB; x += 32) fr[x] = -1;
+    if (lane == 0) ctx_lens[b] = len - nf * bs;
+}
+
 }  // namespace
+
+cudaError_t launch_evict_compact_mask(int32_t *bt, int MB, int32_t *ctx_lens, int32_t *freed,
+                                      const uint8_t *mask, int B, int bs, int32_t *err,
+                                      cudaStream_t st) {
+    evict_compact_mask_kernel<<<(B + 3) / 4, 128, 0, st>>>(bt, MB, ctx_lens, freed, mask, B, bs,
+                                                           err);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_prefill_scores(float *scores, const uint16_t *k, const uint16_t *v, int64_t T,
                                   int Hkv, int d, cudaStream_t st) {

@@ -1,6 +1,7 @@
 // prefill.h -- launchers of the PagedEviction prefill stage and of the
-// block-table compaction (prefill.cu).  Argument checking happens in the C ABI
-// entry points; these only launch.
+// block-table compactions (prefill.cu), and of the threshold eviction policy
+// (evict.cu).  Argument checking happens in the C ABI entry points; these only
+// launch.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -21,5 +22,13 @@ cudaError_t launch_prefill_pack(uint16_t *k_cache, uint16_t *v_cache, int64_t bl
 cudaError_t launch_evict_compact(int32_t *bt, int MB, int32_t *ctx_lens, int32_t *freed,
                                  const int32_t *evict, int B, int bs, int32_t *err,
                                  cudaStream_t stream);
+
+cudaError_t launch_evict_compact_mask(int32_t *bt, int MB, int32_t *ctx_lens, int32_t *freed,
+                                      const uint8_t *mask, int B, int bs, int32_t *err,
+                                      cudaStream_t stream);
+cudaError_t launch_select_threshold(uint8_t *mask, int32_t *count, float *means,
+                                    const float *scores, const int32_t *ctx_lens, int B, int MB,
+                                    int Hkv, int bs, double thr, int triggered,
+                                    cudaStream_t stream);
 
 }  // namespace pkv

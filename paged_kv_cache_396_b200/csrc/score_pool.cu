@@ -11,6 +11,7 @@
 #include <limits.h>
 #include <math.h>
 
+#include "blockmean.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -96,11 +97,11 @@ __global__ void __launch_bounds__(256) append_scored_kernel(const uint16_t *__re
     }
 }
 
-// Block selection from the score pool.  One CTA per sequence; thread k owns the
-// full logical blocks j = k, k + blockDim, ...; block j's bs*Hkv scores are the
-// contiguous scores of physical block bt[b][j] (token-major, then head), summed
-// in that order in fp64 -- the same order and precision as the selection over a
-// [B][MB*bs][Hkv] score array, so both agree exactly on equal scores.
+// Block selection from the score pool.  One CTA per sequence, one warp per full
+// logical block (j = warp, warp + 8, ...); block j's bs*Hkv scores are the
+// contiguous scores of physical block bt[b][j] (token-major, then head), reduced
+// by the same warp routine as the selection over a [B][MB*bs][Hkv] score array,
+// so both agree exactly on equal scores.
 __global__ void __launch_bounds__(256) select_pooled_kernel(int32_t *evict, float *means,
                                                             const float *score_pool,
                                                             const int32_t *block_tables,
@@ -108,6 +109,7 @@ __global__ void __launch_bounds__(256) select_pooled_kernel(int32_t *evict, floa
                                                             int32_t *err, int MB, int Hkv, int bs,
                                                             int64_t N) {
     const int b = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     int len = ctx_lens[b];
     if (len < 0 || (int64_t)len > (int64_t)MB * bs) {
         if (threadIdx.x == 0) raise_flag(err, PA_DEV_BAD_LEN);
@@ -117,56 +119,24 @@ __global__ void __launch_bounds__(256) select_pooled_kernel(int32_t *evict, floa
     const int per = bs * Hkv;
     double best = INFINITY;
     int bj = INT_MAX;
-    for (int j = threadIdx.x; j < MB; j += blockDim.x) {
+    for (int j = warp; j < MB; j += nw) {
         bool cand = j < nfull;
         double mean = 0.0;
         if (cand) {
             const int32_t phys = block_tables[(int64_t)b * MB + j];
             if (phys < 0 || (int64_t)phys >= N) {
-                raise_flag(err, PA_DEV_BAD_BLOCK);
+                if (lane == 0) raise_flag(err, PA_DEV_BAD_BLOCK);
                 cand = false;
             } else {
-                const float *p = score_pool + (int64_t)phys * per;
-                double s = 0.0;
-                for (int k = 0; k < per; ++k) s += (double)p[k];
-                mean = s / (double)per;
+                mean = warp_block_mean(score_pool + (int64_t)phys * per, per, lane);
+                argmin_take(best, bj, mean, j);
             }
         }
-        if (means) means[(int64_t)b * MB + j] = cand ? (float)mean : __int_as_float(0x7fc00000);
-        if (cand && (bj == INT_MAX || mean < best)) {
-            best = mean;
-            bj = j;
-        }
+        if (means && lane == 0)
+            means[(int64_t)b * MB + j] = cand ? (float)mean : __int_as_float(0x7fc00000);
     }
-    __shared__ double sb[32];
-    __shared__ int sj[32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const double ob = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-        if (oj != INT_MAX && (bj == INT_MAX || ob < best || (ob == best && oj < bj))) {
-            best = ob;
-            bj = oj;
-        }
-    }
-    if (lane == 0) {
-        sb[warp] = best;
-        sj[warp] = bj;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        best = sb[0];
-        bj = sj[0];
-        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
-            if (sj[w] != INT_MAX &&
-                (bj == INT_MAX || sb[w] < best || (sb[w] == best && sj[w] < bj))) {
-                best = sb[w];
-                bj = sj[w];
-            }
-        }
-        evict[b] = (nfull > 0 && bj != INT_MAX) ? bj : -1;
-    }
+    const int win = cta_argmin(best, bj);
+    if (threadIdx.x == 0) evict[b] = (nfull > 0 && win != INT_MAX) ? win : -1;
 }
 
 cudaError_t launch_append_scored(const uint16_t *k_new, const uint16_t *v_new, uint16_t *k_cache,

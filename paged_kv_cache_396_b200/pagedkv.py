@@ -37,7 +37,8 @@ EXPORTED = (
     "pa_decode_static_scratch", "pa_append_kv_scored", "pa_append_kv_int8_scored",
     "pe_select_evict_block_pooled", "pa_append_kv_fp8", "pa_decode_fp8",
     "pe_prefill_scores", "pe_prefill_select", "pe_prefill_pack", "pe_prefill_compress",
-    "pe_evict_compact",
+    "pe_evict_compact", "pe_select_evict_threshold", "pe_evict_compact_mask",
+    "pa_prefill_attention",
 )
 
 
@@ -109,6 +110,14 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                         i64, p, p, p, p, p]
     lib.pe_evict_compact.restype = i32
     lib.pe_evict_compact.argtypes = [p, i32, p, p, p, i32, i32, p, p]
+    lib.pe_select_evict_threshold.restype = i32
+    lib.pe_select_evict_threshold.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i64, i64,
+                                              ctypes.c_double, ctypes.c_double, p]
+    lib.pe_evict_compact_mask.restype = i32
+    lib.pe_evict_compact_mask.argtypes = [p, i32, p, p, p, i32, i32, p, p]
+    lib.pa_prefill_attention.restype = i32
+    lib.pa_prefill_attention.argtypes = [p, p, p, i32, p, p, i64, p, i32, p, i32, i32, i32, i32,
+                                         i32, i64, f32, p, p]
     lib.pe_score_tokens.restype = i32
     lib.pe_score_tokens.argtypes = [p, p, p, i64, p, i32, p, i32, i32, i32, i32, i64, p, p]
     lib.pe_select_evict_block.restype = i32
@@ -608,3 +617,77 @@ def pe_evict_compact(block_tables, ctx_lens, evict, block_size, err_flag, freed=
     _check("pe_evict_compact", load().pe_evict_compact(
         _ptr(block_tables), MB, _ptr(ctx_lens), _ptr(freed), _ptr(evict.contiguous()), B,
         int(block_size), _ptr(err_flag), _stream(stream)))
+
+
+def pe_select_evict_threshold(mask, count, scores, ctx_lens, block_size, used_blocks,
+                              total_blocks, eviction_ratio=0.2, importance_threshold=0.1,
+                              block_means=None, stream=None):
+    """Threshold policy over token scores [B, MB*bs, Hkv]: mask [B, MB] uint8,
+    count [B] int32 (block_means [B, MB] float32 optional)."""
+    _want(mask, torch.uint8, "mask")
+    _want(count, torch.int32, "count")
+    _want(scores, torch.float32, "scores")
+    _want(ctx_lens, torch.int32, "ctx_lens")
+    B, T, Hkv = scores.shape
+    MB = T // block_size
+    if T != MB * block_size or tuple(mask.shape) != (B, MB) or not mask.is_contiguous():
+        raise ValueError("scores must be [B, MB*bs, Hkv] and mask contiguous [B, MB]")
+    if block_means is not None:
+        _want(block_means, torch.float32, "block_means")
+    _check("pe_select_evict_threshold", load().pe_select_evict_threshold(
+        _ptr(mask), _ptr(count), _ptr(block_means), _ptr(scores.contiguous()),
+        _ptr(ctx_lens.contiguous()), B, MB, Hkv, int(block_size), int(used_blocks),
+        int(total_blocks), float(eviction_ratio), float(importance_threshold), _stream(stream)))
+
+
+def pe_evict_compact_mask(block_tables, ctx_lens, mask, block_size, err_flag, freed=None,
+                          stream=None):
+    """Remove every marked full block from each table in place; freed [B, MB]
+    int32 (optional) lists the released physical ids, -1 padded."""
+    _want(block_tables, torch.int32, "block_tables")
+    _want(ctx_lens, torch.int32, "ctx_lens")
+    _want(mask, torch.uint8, "mask")
+    _want(err_flag, torch.int32, "err_flag")
+    if not (block_tables.is_contiguous() and ctx_lens.is_contiguous()):
+        raise ValueError("block_tables and ctx_lens are updated in place: pass contiguous tensors")
+    B, MB = block_tables.shape
+    if tuple(mask.shape) != (B, MB):
+        raise ValueError("mask must be [B, MB]")
+    if freed is not None:
+        _want(freed, torch.int32, "freed")
+        if tuple(freed.shape) != (B, MB) or not freed.is_contiguous():
+            raise ValueError("freed must be contiguous [B, MB]")
+    _check("pe_evict_compact_mask", load().pe_evict_compact_mask(
+        _ptr(block_tables), MB, _ptr(ctx_lens), _ptr(freed), _ptr(mask.contiguous()), B,
+        int(block_size), _ptr(err_flag), _stream(stream)))
+
+
+# ----------------------------------------------------------------------------- chunked prefill
+def pa_prefill_attention(out, q, cu_q, max_q_len, k_cache, v_cache, block_tables, ctx_lens,
+                         scale, err_flag, stream=None):
+    """Multi-query paged attention: the q_len_b = cu_q[b+1]-cu_q[b] query rows of
+    sequence b are its last q_len_b cached tokens and attend causally.
+    q, out [Tq, Hq, d] bf16 contiguous; cu_q [B+1] int32; ctx_lens [B] int32."""
+    _want(out, torch.bfloat16, "out")
+    _want(q, torch.bfloat16, "q")
+    _want(cu_q, torch.int32, "cu_q")
+    _want(block_tables, torch.int32, "block_tables")
+    _want(ctx_lens, torch.int32, "ctx_lens")
+    _want(err_flag, torch.int32, "err_flag")
+    _want(k_cache, torch.bfloat16, "k_cache")
+    _want(v_cache, torch.bfloat16, "v_cache")
+    N, bs, Hkv, d, stride = _pool_geometry(k_cache, "k_cache")
+    _same_pool(k_cache, v_cache)
+    if q.dim() != 3 or q.shape != out.shape or not (q.is_contiguous() and out.is_contiguous()):
+        raise ValueError("q and out must be contiguous [Tq, Hq, d] of equal shape")
+    Tq, Hq, dq = q.shape
+    if dq != d:
+        raise ValueError("q head_dim differs from the pool's")
+    B = block_tables.shape[0]
+    if cu_q.numel() != B + 1:
+        raise ValueError("cu_q must hold B + 1 offsets")
+    bt = block_tables.contiguous()
+    _check("pa_prefill_attention", load().pa_prefill_attention(
+        _ptr(out), _ptr(q), _ptr(cu_q.contiguous()), int(max_q_len), _ptr(k_cache),
+        _ptr(v_cache), stride, _ptr(bt), bt.shape[1], _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d,
+        bs, N, float(scale), _ptr(err_flag), _stream(stream)))

@@ -22,7 +22,10 @@ describe; all values bf16 ~ N(0, 1) unless stated):
                 budget 1024 tokens per prompt (the PagedEviction budget); prompt
                 K/V rows [T, Hkv, d] bf16 N(0, 1) with 1% of the (head, channel)
                 pairs scaled x8.
-Seeds are 396 + the workload's index (0..5).
+  p2  chunked prefill: 4 sequences, each appending and attending the last
+                512-token chunk of an 8192-token prompt (Sarathi's chunk size),
+                Hq=32, Hkv=8, d=128, bs=16, shuffled pool; values N(0, 1).
+Seeds are 396 + the workload's index (0..6).
 
 The allocator is the on-demand block pool of the vLLM notes (ybb.press "LLM 推理
 KV Cache 内存管理深度工程实践" §2.1): a shuffled free list, each sequence taking
@@ -294,3 +297,65 @@ def generate_prefill(cfg: PrefillConfig, device="cpu") -> PrefillWorkload:
         v[:, h, e] *= 8
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     return PrefillWorkload(cfg=cfg, k=k, v=v, cu_seqlens=cu, block_tables=bt, num_blocks=N)
+
+
+# ----------------------------------------------------------------------------- chunked prefill
+@dataclass(frozen=True)
+class ChunkConfig:
+    key: str
+    name: str
+    batch: int
+    ctx_len: int                    # tokens cached after the chunk's append
+    chunk: int                      # query tokens per sequence
+    hq: int
+    hkv: int
+    head_dim: int
+    block_size: int
+    spare: float = 0.10
+    seed: int = 402
+
+
+CHUNKED = {
+    "p2": ChunkConfig("p2", "chunked prefill attention", 4, 8192, 512, 32, 8, 128, 16),
+}
+
+
+@dataclass
+class ChunkWorkload:
+    cfg: ChunkConfig
+    k_pool: torch.Tensor            # [N, bs, Hkv, d] bf16 (history; the chunk is appended)
+    v_pool: torch.Tensor
+    k_new: torch.Tensor             # [B, chunk, Hkv, d] bf16
+    v_new: torch.Tensor
+    q: torch.Tensor                 # [B*chunk, Hq, d] bf16
+    cu_q: np.ndarray                # [B+1] int32
+    ctx_lens: np.ndarray            # [B] int32 (after the append)
+    positions: np.ndarray           # [B] int32, first position of the chunk
+    block_tables: np.ndarray
+    num_blocks: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.cfg.head_dim)
+
+
+def generate_chunked(cfg: ChunkConfig, device="cpu") -> ChunkWorkload:
+    rng = np.random.default_rng(cfg.seed)
+    B, bs, Hkv, d = cfg.batch, cfg.block_size, cfg.hkv, cfg.head_dim
+    ctx = np.full(B, cfg.ctx_len, np.int32)
+    bt, N = _allocate(ctx, bs, cfg.spare, None, rng)
+    g = torch.Generator(device=device)
+    g.manual_seed(cfg.seed)
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, device=device).to(torch.bfloat16)
+
+    k_pool = randn(N, bs, Hkv, d)
+    v_pool = randn(N, bs, Hkv, d)
+    k_new = randn(B, cfg.chunk, Hkv, d)
+    v_new = randn(B, cfg.chunk, Hkv, d)
+    q = randn(B * cfg.chunk, cfg.hq, d)
+    cu = (np.arange(B + 1) * cfg.chunk).astype(np.int32)
+    return ChunkWorkload(cfg=cfg, k_pool=k_pool, v_pool=v_pool, k_new=k_new, v_new=v_new, q=q,
+                         cu_q=cu, ctx_lens=ctx, positions=(ctx - cfg.chunk).astype(np.int32),
+                         block_tables=bt, num_blocks=N)

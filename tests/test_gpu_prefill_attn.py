@@ -1,0 +1,151 @@
+"""GPU parity of the multi-query (chunked prefill) paged attention through the
+C ABI against the fp64 oracle: |err| <= 2e-3 + 1e-2 |ref| on every output of
+medium cases (several 64-row query tiles, 64-token K/V tiles, ragged tails,
+GQA group sizes 1..16, d 64 and 128, block sizes 12, 16 and 256), the
+append-then-attend sequence, mixed chunk + decode batches, invalid lengths,
+and sampled rows of a full-size 512-token chunk at 8K context."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_attention_close
+from paged_kv_cache_396_b200 import pagedkv as pk
+from paged_kv_cache_396_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(lens, qlens, Hq, Hkv, d, bs, seed, spare=4):
+    g = torch.Generator().manual_seed(seed)
+    rng = np.random.default_rng(seed)
+    nb = [max(1, -(-int(n) // bs)) for n in lens]
+    N = sum(nb) + spare
+    perm = rng.permutation(N).astype(np.int32)
+    MB = max(nb)
+    bt = np.full((len(lens), MB), -1, np.int32)
+    c = 0
+    for b, m in enumerate(nb):
+        bt[b, :m] = perm[c:c + m]
+        c += m
+    k = torch.randn(N, bs, Hkv, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(N, bs, Hkv, d, generator=g).to(torch.bfloat16)
+    cu = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = torch.randn(int(cu[-1]), Hq, d, generator=g).to(torch.bfloat16)
+    return dict(k=k, v=v, q=q, bt=bt, cu=cu, lens=np.asarray(lens, np.int32), Hq=Hq, Hkv=Hkv,
+                d=d, bs=bs, N=N, qlens=list(qlens))
+
+
+def _run(c, err_expected=0):
+    dev = "cuda"
+    out = torch.full(c["q"].shape, float("nan"), dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    pk.pa_prefill_attention(out, c["q"].to(dev), torch.as_tensor(c["cu"]).to(dev),
+                            max(c["qlens"] + [0]), c["k"].to(dev), c["v"].to(dev),
+                            torch.as_tensor(c["bt"]).to(dev), torch.as_tensor(c["lens"]).to(dev),
+                            c["d"] ** -0.5, err)
+    torch.cuda.synchronize()
+    assert err.item() == err_expected
+    return out
+
+
+def _oracle(c):
+    stride = c["bs"] * c["Hkv"] * c["d"]
+    return oracle.paged_prefill(W.bits(c["q"]), c["cu"], W.bits(c["k"]).ravel(),
+                                W.bits(c["v"]).ravel(), stride, c["bt"], c["lens"], c["Hkv"],
+                                c["bs"], c["d"] ** -0.5)
+
+
+CASES = {
+    # Llama-3-8B shape: a 512-token chunk, a whole prompt in one chunk, decodes, an empty row
+    "g4d128": ([2048, 700, 37, 5, 1100], [512, 1, 37, 0, 100], 32, 8, 128, 16),
+    "g1d128": ([300, 129], [130, 64], 8, 8, 128, 16),
+    "g16d128": ([900, 64], [70, 3], 64, 4, 128, 16),
+    "g2d64": ([513, 1000, 65], [257, 1, 65], 16, 8, 64, 16),
+    "g8d64bs12": ([250, 97], [99, 97], 32, 4, 64, 12),
+    "g4bs256": ([1500, 2000], [300, 513], 32, 8, 128, 256),
+}
+
+
+@pytest.mark.parametrize("key", list(CASES))
+def test_prefill_attention_medium(key):
+    lens, qlens, Hq, Hkv, d, bs = CASES[key]
+    c = _case(lens, qlens, Hq, Hkv, d, bs, seed=100 + list(CASES).index(key))
+    out = _run(c)
+    assert_attention_close(out, _oracle(c), key)
+
+
+def test_append_chunk_then_attend():
+    """The chunk's rows written by pa_append_kv (n_new = chunk) and then
+    attended: the same as the oracle's append + prefill attention."""
+    Hq, Hkv, d, bs = 32, 8, 128, 16
+    old, chunk = np.array([1000, 300], np.int32), [512, 200]
+    lens = old + np.array(chunk, np.int32)
+    c = _case(lens, chunk, Hq, Hkv, d, bs, seed=9)
+    g = torch.Generator().manual_seed(10)
+    kn = torch.randn(2, 512, Hkv, d, generator=g).to(torch.bfloat16)
+    vn = torch.randn(2, 512, Hkv, d, generator=g).to(torch.bfloat16)
+    stride = bs * Hkv * d
+    kc, vc = W.bits(c["k"]).ravel().copy(), W.bits(c["v"]).ravel().copy()
+    dev = "cuda"
+    kd, vd = c["k"].to(dev), c["v"].to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    bt = torch.as_tensor(c["bt"]).to(dev)
+    for b in range(2):
+        n = chunk[b]
+        pk.pa_append_kv(kn[b:b + 1, :n].contiguous().to(dev), vn[b:b + 1, :n].contiguous().to(dev),
+                        kd, vd, bt[b:b + 1], torch.as_tensor(old[b:b + 1]).to(dev), err)
+        oracle.append_kv(W.bits(kn[b:b + 1, :n]), W.bits(vn[b:b + 1, :n]), kc, vc, stride,
+                         c["bt"][b:b + 1], old[b:b + 1], bs)
+    out = torch.empty(c["q"].shape, dtype=torch.bfloat16, device=dev)
+    pk.pa_prefill_attention(out, c["q"].to(dev), torch.as_tensor(c["cu"]).to(dev), 512, kd, vd,
+                            bt, torch.as_tensor(lens).to(dev), d ** -0.5, err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ref = oracle.paged_prefill(W.bits(c["q"]), c["cu"], kc, vc, stride, c["bt"], lens, Hkv, bs,
+                               d ** -0.5)
+    assert_attention_close(out, ref, "append + prefill attention")
+
+
+def test_single_query_rows_match_decode_kernel_results():
+    """q_len = 1 everywhere: both the prefill kernel and the decode kernel
+    within tolerance of the same oracle."""
+    lens = [1, 17, 300, 1025]
+    c = _case(lens, [1] * 4, 32, 8, 128, 16, seed=11)
+    out = _run(c)
+    ref = _oracle(c)
+    assert_attention_close(out, ref, "prefill kernel, q_len 1")
+    stride = 16 * 8 * 128
+    ref_dec = oracle.paged_decode(W.bits(c["q"]), W.bits(c["k"]).ravel(), W.bits(c["v"]).ravel(),
+                                  stride, c["bt"], c["lens"], 8, 16, 128 ** -0.5)
+    assert np.array_equal(ref, ref_dec)
+
+
+def test_invalid_query_length_gives_zero_rows_and_flag():
+    c = _case([50, 10], [20, 11], 8, 2, 64, 16, seed=12)
+    out = _run(c, err_expected=pk.PA_DEV_BAD_LEN)
+    ref = _oracle(c)
+    assert not ref[20:].any()
+    assert (out[20:].float() == 0).all()
+    assert_attention_close(out[:20], ref[:20], "valid sequence next to an invalid one")
+
+
+def test_full_size_chunk_sampled_rows():
+    """The last 512-token chunk of an 8192-token prompt, Llama-3-8B shape, 4
+    sequences: sampled query rows against the decode oracle at the row's own
+    position (causality makes query i of the chunk a decode over p + 1 tokens)."""
+    Hq, Hkv, d, bs = 32, 8, 128, 16
+    lens = [8192] * 4
+    c = _case(lens, [512] * 4, Hq, Hkv, d, bs, seed=13)
+    out = _run(c).cpu()
+    rng = np.random.default_rng(14)
+    stride = bs * Hkv * d
+    kb, vb = W.bits(c["k"]).ravel(), W.bits(c["v"]).ravel()
+    for b in range(4):
+        rows = np.concatenate([[0, 511], rng.integers(1, 511, 6)])
+        for i in rows:
+            p = 8192 - 512 + int(i)
+            qrow = c["q"][c["cu"][b] + int(i)].unsqueeze(0)
+            ref = oracle.paged_decode(W.bits(qrow), kb, vb, stride, c["bt"][b:b + 1],
+                                      np.array([p + 1], np.int32), Hkv, bs, d ** -0.5)
+            assert_attention_close(out[c["cu"][b] + int(i)].unsqueeze(0), ref, f"seq {b} row {i}")
