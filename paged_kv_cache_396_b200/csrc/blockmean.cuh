@@ -10,12 +10,18 @@
 namespace pkv {
 
 // Mean of the `per` fp32 scores at p (bs*Hkv entries of one block): coalesced
-// loads, fp64 partial sums per lane, butterfly reduction.  Every lane returns
-// the same value.
+// loads issued four at a time (independent, so their latencies overlap), fp64
+// partial sums per lane, butterfly reduction.  Every lane returns the same value.
 __device__ __forceinline__ double warp_block_mean(const float *__restrict__ p, int per,
                                                   int lane) {
     double s = 0.0;
-    for (int k = lane; k < per; k += 32) s += (double)__ldg(p + k);
+    int k = lane;
+    for (; k + 96 < per; k += 128) {
+        const float a0 = __ldg(p + k), a1 = __ldg(p + k + 32);
+        const float a2 = __ldg(p + k + 64), a3 = __ldg(p + k + 96);
+        s += ((double)a0 + (double)a1) + ((double)a2 + (double)a3);
+    }
+    for (; k < per; k += 32) s += (double)__ldg(p + k);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     return s / (double)per;

@@ -88,10 +88,10 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreArgs a) {
     }
 }
 
-// One CTA per sequence, one warp per full block (blocks j = warp, warp + 8, ...):
+// One CTA per sequence, one warp per full block (blocks j = warp, warp + 32, ...):
 // each block mean is an fp64 sum of its bs*Hkv fp32 scores divided by bs*Hkv;
 // then a (mean, j) argmin with ties to the lowest j.
-__global__ void __launch_bounds__(256) select_evict_kernel(int32_t *evict, float *means,
+__global__ void __launch_bounds__(1024) select_evict_kernel(int32_t *evict, float *means,
                                                            const float *scores,
                                                            const int32_t *ctx_lens, int MB,
                                                            int Hkv, int bs) {
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(256) select_evict_kernel(int32_t *evict, float
 // Threshold policy: with the trigger on, every full block whose mean is below
 // `thr` is marked, else the lowest-mean full block; with it off nothing is
 // marked.  Means are written either way.
-__global__ void __launch_bounds__(256) select_threshold_kernel(
+__global__ void __launch_bounds__(1024) select_threshold_kernel(
     uint8_t *mask, int32_t *count, float *means, const float *scores, const int32_t *ctx_lens,
     int MB, int Hkv, int bs, double thr, int triggered) {
     __shared__ int s_count;
@@ -169,14 +169,14 @@ cudaError_t launch_score(const ScoreArgs &a, cudaStream_t st) {
 cudaError_t launch_select_evict(int32_t *evict, float *means, const float *scores,
                                 const int32_t *ctx_lens, int B, int MB, int Hkv, int bs,
                                 cudaStream_t st) {
-    select_evict_kernel<<<B, 256, 0, st>>>(evict, means, scores, ctx_lens, MB, Hkv, bs);
+    select_evict_kernel<<<B, 1024, 0, st>>>(evict, means, scores, ctx_lens, MB, Hkv, bs);
     return cudaGetLastError();
 }
 
 cudaError_t launch_select_threshold(uint8_t *mask, int32_t *count, float *means,
                                     const float *scores, const int32_t *ctx_lens, int B, int MB,
                                     int Hkv, int bs, double thr, int triggered, cudaStream_t st) {
-    select_threshold_kernel<<<B, 256, 0, st>>>(mask, count, means, scores, ctx_lens, MB, Hkv, bs,
+    select_threshold_kernel<<<B, 1024, 0, st>>>(mask, count, means, scores, ctx_lens, MB, Hkv, bs,
                                                thr, triggered);
     return cudaGetLastError();
 }

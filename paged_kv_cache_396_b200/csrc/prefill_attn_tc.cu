@@ -19,9 +19,9 @@
 //              MN-major) into the O columns; completion through tcgen05.commit.
 //              Its lanes also zero the V rows past the context end in a tile
 //              that holds them (stale or NaN slots must not meet a zero weight).
-//   warp 5     TMA producer (one lane): for every 16-token page of a tile, four
-//              boxes (K and V, two 64-element slices each) at the page's physical
-//              block; two stages.
+//   warp 5     TMA producer: lane p < 8 owns 16-token page p of every tile, looks
+//              up its physical block one tile ahead and issues four boxes (K and V,
+//              two 64-element slices each); three stages.
 // TMEM: S/P buffers at columns [0,128) and [128,256), O at [256,384).
 // Every mbarrier wait is bounded (2 s of globaltimer); a timeout sets
 // PA_DEV_TIMEOUT and the CTA winds down, freeing its TMEM.
@@ -44,13 +44,14 @@ constexpr int kN = 128;          // tokens per K/V tile
 constexpr int kThreads = 192;
 constexpr int kSlice = kN * 128;         // one 64-element slice of a 128-row tile (bytes)
 constexpr int kTileB = 2 * kSlice;       // a K or V tile (d = 128)
-constexpr int kSmem = kTileB /*Q*/ + 2 * 2 * kTileB /*K,V x 2 stages*/ + 1024 /*align*/;
+constexpr int kStages = 3;       // K/V stages in flight
+constexpr int kSmem = kTileB /*Q*/ + kStages * 2 * kTileB /*K,V per stage*/ + 1024 /*align*/;
 constexpr uint32_t kColO = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 // instruction descriptor: D f32, A/B bf16, M = 128, N = 128; B MN-major when mn
-constexpr uint32_t idesc(bool b_mn) {
+__host__ __device__ constexpr uint32_t idesc(bool b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn ? 1u : 0u) << 16) | ((kN / 8u) << 17) |
            ((kM / 16u) << 24);
 }
@@ -120,6 +121,14 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 2^x with the MUFU instruction (ftz; relative error ~2^-22, far inside what the
+// bf16 weights keep); ex2(-inf) = 0
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // bounded wait; false (and the abort flag set) on timeout
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int *abort_flag) {
     const uint64_t t0 = ptx::globaltimer();
@@ -141,8 +150,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int *a
 
 struct Bars {
     uint64_t q_full;          // 128 softmax threads: Q rows in shared memory
-    uint64_t kv_full[2];      // TMA bytes of a K/V stage
-    uint64_t kv_empty[2];     // commit after the P V that read the stage
+    uint64_t kv_full[kStages];   // TMA bytes of a K/V stage
+    uint64_t kv_empty[kStages];  // commit after the P V that read the stage
     uint64_t s_full[2];       // commit after S = Q K^T into buffer b
     uint64_t p_full[2];       // 128 softmax threads: P written over buffer b
     uint64_t pv_done[2];      // commit after O += P V from buffer b
@@ -190,14 +199,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // K/V stages start as zeros: a page that is not loaded (bad block id) then
     // holds finite data only
-    for (int x = tid; x < 2 * 2 * kTileB / 16; x += kThreads)
+    for (int x = tid; x < kStages * 2 * kTileB / 16; x += kThreads)
         *reinterpret_cast<uint4 *>(gbase + kTileB + 16 * x) = make_uint4(0, 0, 0, 0);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (tid == 0) {
         ptx::mbar_init(&bars.q_full, 128);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kStages; ++i) {
             ptx::mbar_init(&bars.kv_full[i], 1);
             ptx::mbar_init(&bars.kv_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&bars.s_full[i], 1);
             ptx::mbar_init(&bars.p_full[i], 128);
             ptx::mbar_init(&bars.pv_done[i], 1);
@@ -244,21 +255,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int bb = j & 1;
             if (!(ok = warp_wait(&bars.s_full[bb], (j >> 1) & 1, abort_flag))) break;
             fence_after();
-            float s[kN];
-#pragma unroll
+            const uint32_t sbuf = lane_base + bb * 128;
+            // tokens t0 + e with e <= lim are visible to this row (lim >= 127: all)
+            const int lim = valid ? pos - j * kN : -1;
+            // ---- pass 1: row maximum of the scaled, masked logits (4 chunks of 32
+            // columns, 8 independent max chains)
+            float mx = -INFINITY;
+#pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t v[32];
-                tmem_ld32(lane_base + bb * 128 + 32 * c, v);
+                tmem_ld32(sbuf + 32 * c, v);
                 tmem_wait_ld();
+                float mk[8];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(v[e]);
-            }
-            const int t0 = j * kN;
-            float mx = -INFINITY;
+                for (int q = 0; q < 8; ++q) mk[q] = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < kN; ++e) {
-                s[e] = (valid && t0 + e <= pos) ? s[e] * sl : -INFINITY;
-                mx = fmaxf(mx, s[e]);
+                for (int e = 0; e < 32; ++e) {
+                    const float x = (32 * c + e <= lim) ? __uint_as_float(v[e]) * sl : -INFINITY;
+                    mk[e & 7] = fmaxf(mk[e & 7], x);
+                }
+#pragma unroll
+                for (int q = 0; q < 8; ++q) mx = fmaxf(mx, mk[q]);
             }
             const float mn = fmaxf(m, mx);
             // lazy rescale: a row moves its reference max only when the tile's max
@@ -270,8 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!(ok = warp_wait(&bars.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)))
                     break;
                 fence_after();
-                const float alpha = rescale ? exp2f(m - mn) : 1.f;
-#pragma unroll
+                const float alpha = rescale ? ex2(m - mn) : 1.f;
+#pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t v[32];
                     tmem_ld32(lane_base + kColO + 32 * c, v);
@@ -285,25 +302,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (move) m = mn;
             const float u = m == -INFINITY ? 0.f : m;
-            // P = hi + lo over the S columns: k-step kk (16 tokens) at columns 16kk
-            // (hi, 8 columns of bf16 pairs) and 16kk + 8 (lo)
-#pragma unroll
+            // ---- pass 2: P = exp2(s - u) as hi + lo bf16 over the S columns: k-step kk
+            // (16 tokens) at columns 16kk (hi, 8 columns of bf16 pairs) and 16kk + 8 (lo)
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
             for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tmem_ld32(sbuf + 32 * c, v);
+                tmem_wait_ld();
                 uint32_t w[32];
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const int e = 32 * c + 16 * half + 2 * q;
-                        const float p0 = exp2f(s[e] - u), p1 = exp2f(s[e + 1] - u);
-                        l += p0 + p1;
+                        const int e = 16 * half + 2 * q;
+                        const float x0 = (32 * c + e <= lim) ? __uint_as_float(v[e]) * sl - u : -INFINITY;
+                        const float x1 =
+                            (32 * c + e + 1 <= lim) ? __uint_as_float(v[e + 1]) * sl - u : -INFINITY;
+                        const float p0 = ex2(x0), p1 = ex2(x1);
+                        ls[q & 3] += p0 + p1;
                         const uint32_t hi = ptx::pack_bf16(p0, p1);
                         w[16 * half + q] = hi;
                         w[16 * half + 8 + q] = ptx::pack_bf16(p0 - bf16_lo(hi), p1 - bf16_hi(hi));
                     }
                 }
-                tmem_st32(lane_base + bb * 128 + 32 * c, w);
+                tmem_st32(sbuf + 32 * c, w);
             }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             tmem_wait_st();
             fence_before();
             ptx::mbar_arrive(&bars.p_full[bb]);
@@ -333,8 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t id_qk = idesc(false), id_pv = idesc(true);
         for (int j = 0; j <= n_kt && ok; ++j) {
             if (j < n_kt) {
-                const int st = j & 1, bb = j & 1;
-                if (!(ok = warp_wait(&bars.kv_full[st], (j >> 1) & 1, abort_flag))) break;
+                const int st = j % kStages, bb = j & 1;
+                if (!(ok = warp_wait(&bars.kv_full[st], (j / kStages) & 1, abort_flag))) break;
                 const int t0 = j * kN;
                 if (t0 + kN > len) {
                     // V rows at or past the context end: zero them (the weights there
@@ -364,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
             }
             if (j >= 1) {
-                const int jj = j - 1, bb = jj & 1, st = jj & 1;
+                const int jj = j - 1, bb = jj & 1, st = jj % kStages;
                 if (!(ok = warp_wait(&bars.p_full[bb], (jj >> 1) & 1, abort_flag))) break;
                 fence_after();
                 if (lane == 0) {
@@ -383,35 +408,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
             }
         }
-    } else if (warp == 5 && lane == 0) {
+    } else if (warp == 5) {
         // ======================= TMA producer =======================
+        // lane pg < 8 owns 16-token page pg of every tile: it looks up the page's
+        // physical block (one tile ahead, so the table read is off the critical
+        // path) and issues the page's four boxes
         const int32_t *btr = a.block_tables + (int64_t)b * a.MB;
+        auto lookup = [&](int j) -> int32_t {
+            const int t = j * kN + 16 * lane;
+            return (lane < kN / 16 && t < len) ? btr[t / a.bs] : -1;
+        };
+        int32_t next = lookup(0);
         bool ok = true;
         for (int j = 0; j < n_kt && ok; ++j) {
-            const int st = j & 1;
-            if (j >= 2 && !(ok = wait_bar(&bars.kv_empty[st], ((j >> 1) - 1) & 1, abort_flag)))
+            const int st = j % kStages;
+            const int32_t blk = next;
+            if (j + 1 < n_kt) next = lookup(j + 1);
+            if (j >= kStages &&
+                !(ok = warp_wait(&bars.kv_empty[st], ((j / kStages) - 1) & 1, abort_flag)))
                 break;
-            const int t0 = j * kN;
-            // pages of this tile inside the context with a valid block id; the others
-            // are not loaded (their rows are masked, and V rows past the end zeroed)
-            uint32_t load_mask = 0;
-            for (int pg = 0; pg < kN / 16; ++pg) {
-                const int t = t0 + 16 * pg;
-                if (t >= len) break;
-                const int32_t blk = btr[t / a.bs];
-                if (blk < 0 || (int64_t)blk >= a.N) raise_flag(a.err, PA_DEV_BAD_BLOCK);
-                else load_mask |= 1u << pg;
-            }
-            ptx::mbar_arrive_expect_tx(&bars.kv_full[st], (uint32_t)__popc(load_mask) * 4u * 2048u);
-            for (int pg = 0; pg < kN / 16; ++pg) {
-                if (!((load_mask >> pg) & 1u)) continue;
-                const int t = t0 + 16 * pg;
-                const int32_t blk = btr[t / a.bs];
+            const int t = j * kN + 16 * lane;
+            const bool in = lane < kN / 16 && t < len;
+            // pages inside the context with a valid block id are loaded; the others
+            // are not (their rows are masked, and V rows past the end zeroed)
+            const bool load = in && blk >= 0 && (int64_t)blk < a.N;
+            if (in && !load) raise_flag(a.err, PA_DEV_BAD_BLOCK);
+            const unsigned lm = __ballot_sync(0xffffffffu, load);
+            if (lane == 0) ptx::mbar_arrive_expect_tx(&bars.kv_full[st], (uint32_t)__popc(lm) * 4u * 2048u);
+            __syncwarp();
+            if (load) {
                 const int off = t % a.bs;
 #pragma unroll
                 for (int sl = 0; sl < 2; ++sl) {
-                    const uint32_t dk = sK(st) + (uint32_t)(sl * kSlice + pg * 16 * 128);
-                    const uint32_t dv = sV(st) + (uint32_t)(sl * kSlice + pg * 16 * 128);
+                    const uint32_t dk = sK(st) + (uint32_t)(sl * kSlice + lane * 16 * 128);
+                    const uint32_t dv = sV(st) + (uint32_t)(sl * kSlice + lane * 16 * 128);
                     ptx::tma_load_5d(gbase + (dk - base), &km, &bars.kv_full[st], 0, off, h, sl,
                                      blk);
                     ptx::tma_load_5d(gbase + (dv - base), &vm, &bars.kv_full[st], 0, off, h, sl,

@@ -98,11 +98,11 @@ __global__ void __launch_bounds__(256) append_scored_kernel(const uint16_t *__re
 }
 
 // Block selection from the score pool.  One CTA per sequence, one warp per full
-// logical block (j = warp, warp + 8, ...); block j's bs*Hkv scores are the
+// logical block (j = warp, warp + 32, ...); block j's bs*Hkv scores are the
 // contiguous scores of physical block bt[b][j] (token-major, then head), reduced
 // by the same warp routine as the selection over a [B][MB*bs][Hkv] score array,
 // so both agree exactly on equal scores.
-__global__ void __launch_bounds__(256) select_pooled_kernel(int32_t *evict, float *means,
+__global__ void __launch_bounds__(1024) select_pooled_kernel(int32_t *evict, float *means,
                                                             const float *score_pool,
                                                             const int32_t *block_tables,
                                                             const int32_t *ctx_lens,
@@ -159,7 +159,7 @@ cudaError_t launch_select_pooled(int32_t *evict, float *means, const float *scor
                                  const int32_t *block_tables, const int32_t *ctx_lens,
                                  int32_t *err, int B, int MB, int Hkv, int bs, int64_t N,
                                  cudaStream_t st) {
-    select_pooled_kernel<<<B, 256, 0, st>>>(evict, means, score_pool, block_tables, ctx_lens,
+    select_pooled_kernel<<<B, 1024, 0, st>>>(evict, means, score_pool, block_tables, ctx_lens,
                                             err, MB, Hkv, bs, N);
     return cudaGetLastError();
 }
