@@ -6,23 +6,28 @@
 // tokens of a sequence are its last q_len cached tokens and attend causally.
 // Used for d = 128 and block sizes that are multiples of 16.
 //
-// One CTA = one (sequence, kv head, tile of 128 query rows); rows are (query
-// token, head of the GQA group) pairs, so each K/V tile serves all G heads.
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns row r = TMEM lane r.  Loads its Q row into
-//              shared memory once; per 128-token tile reads its S row from TMEM,
-//              masks (causal), keeps the running max (lazy: O is rescaled only
-//              when the max grows by more than 2^8), writes P = hi + lo (two bf16
-//              parts) back over the S columns, and at the end normalises O.
-//   warp 4     MMA issue (one lane): S = Q K^T (SS, both K-major) into one of two
-//              S/P column buffers, then O += P_hi V + P_lo V (A from TMEM, V
-//              MN-major) into the O columns; completion through tcgen05.commit.
-//              Its lanes also zero the V rows past the context end in a tile
-//              that holds them (stale or NaN slots must not meet a zero weight).
-//   warp 5     TMA producer: lane p < 8 owns 16-token page p of every tile, looks
+// One CTA = one (sequence, kv head, 256 query rows) as two tiles of 128 rows
+// (the MMA M); rows are (query token, head of the GQA group) pairs, so each K/V
+// tile serves all G heads of both Q tiles.  Warp roles (320 threads):
+//   warps 0-3, 4-7  softmax, one warpgroup per Q tile: thread r owns row r of its
+//              tile = TMEM lane r.  Loads its Q row into shared memory once; per
+//              128-token K/V tile reads its S row from TMEM, masks (causal),
+//              keeps the running max (lazy: O is rescaled only when the max grows
+//              by more than 2^8), writes P = hi + lo (two bf16 parts) back over the
+//              S columns, and at the end normalises O.  The two warpgroups work
+//              half a step apart, so one computes softmax while the tensor core
+//              runs the other tile's products.
+//   warp 8     MMA issue (one lane), in the order PV_A(j), S_A(j+1), PV_B(j),
+//              S_B(j+1): S = Q K^T (SS, both K-major) into the tile's S/P
+//              columns, O += P_hi V + P_lo V (A from TMEM, V MN-major) into its O
+//              columns; completion through tcgen05.commit.  Its lanes also zero
+//              the V rows past the context end in a tile that holds them (stale or
+//              NaN slots must not meet a zero weight).
+//   warp 9     TMA producer: lane p < 8 owns 16-token page p of every tile, looks
 //              up its physical block one tile ahead and issues four boxes (K and V,
-//              two 64-element slices each); three stages.
-// TMEM: S/P buffers at columns [0,128) and [128,256), O at [256,384).
+//              two 64-element slices each); two stages.
+// TMEM: S/P of tile A at columns [0,128), of tile B at [128,256); O of tile A at
+// [256,384), of tile B at [384,512).
 // Every mbarrier wait is bounded (2 s of globaltimer); a timeout sets
 // PA_DEV_TIMEOUT and the CTA winds down, freeing its TMEM.
 #include <cuda.h>
@@ -39,13 +44,14 @@ namespace pkv {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kM = 128;          // query rows per CTA
+constexpr int kM = 128;          // query rows per MMA tile (TMEM lanes)
+constexpr int kRows = 2 * kM;    // query rows per CTA: two tiles
 constexpr int kN = 128;          // tokens per K/V tile
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;    // 8 softmax warps, 1 MMA warp, 1 TMA warp
 constexpr int kSlice = kN * 128;         // one 64-element slice of a 128-row tile (bytes)
-constexpr int kTileB = 2 * kSlice;       // a K or V tile (d = 128)
-constexpr int kStages = 3;       // K/V stages in flight
-constexpr int kSmem = kTileB /*Q*/ + kStages * 2 * kTileB /*K,V per stage*/ + 1024 /*align*/;
+constexpr int kTileB = 2 * kSlice;       // a Q, K or V tile (d = 128)
+constexpr int kStages = 2;       // K/V stages in flight
+constexpr int kSmem = 2 * kTileB /*Q x 2*/ + kStages * 2 * kTileB /*K,V per stage*/ + 1024;
 constexpr uint32_t kColO = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;
@@ -149,13 +155,13 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int *a
 }
 
 struct Bars {
-    uint64_t q_full;          // 128 softmax threads: Q rows in shared memory
-    uint64_t kv_full[kStages];   // TMA bytes of a K/V stage
-    uint64_t kv_empty[kStages];  // commit after the P V that read the stage
-    uint64_t s_full[2];       // commit after S = Q K^T into buffer b
-    uint64_t p_full[2];       // 128 softmax threads: P written over buffer b
-    uint64_t pv_done[2];      // commit after O += P V from buffer b
-    uint64_t o_final;         // commit after the last P V
+    uint64_t q_full;              // 256 softmax threads: Q rows in shared memory
+    uint64_t kv_full[kStages];    // TMA bytes of a K/V stage
+    uint64_t kv_empty[kStages];   // commit after the last P V that read the stage
+    uint64_t s_full[2];           // per Q tile: commit after S = Q K^T
+    uint64_t p_full[2];           // per Q tile: 128 softmax threads wrote P
+    uint64_t pv_done[2];          // per Q tile: commit after O += P V
+    uint64_t o_final;             // commit after the last P V of both tiles
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -166,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     __shared__ Bars bars;
     const int b = blockIdx.z, h = blockIdx.y;
-    const int G = a.G, QT = kM / G;
+    const int G = a.G, QT = kRows / G;   // query tokens per CTA (two tiles of 128 rows)
     const int q0 = a.cu_q[b], ql = a.cu_q[b + 1] - q0;
     const int n_qt = (ql + QT - 1) / QT;
     const int qt = n_qt - 1 - (int)blockIdx.x;   // longest context first
@@ -176,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tok_base = qt * QT;
     if (len < 0 || (int64_t)len > (int64_t)a.MB * a.bs || ql > len) {
         if (blockIdx.x == 0 && h == 0 && tid == 0) raise_flag(a.err, PA_DEV_BAD_LEN);
-        for (int r = warp; r < kM; r += kThreads / 32) {
+        for (int r = warp; r < kRows; r += kThreads / 32) {
             const int i = tok_base + r / G;
             if (i >= ql) continue;
             uint16_t *o = a.out + ((int64_t)(q0 + i) * a.Hq + h * G + r % G) * kD;
@@ -193,17 +199,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = ptx::smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
-    const uint32_t sQ = base;
-    auto sK = [&](int st) { return base + (uint32_t)(kTileB + st * 2 * kTileB); };
-    auto sV = [&](int st) { return base + (uint32_t)(2 * kTileB + st * 2 * kTileB); };
+    auto sQ = [&](int w) { return base + (uint32_t)(w * kTileB); };
+    auto sK = [&](int st) { return base + (uint32_t)(2 * kTileB + st * 2 * kTileB); };
+    auto sV = [&](int st) { return base + (uint32_t)(3 * kTileB + st * 2 * kTileB); };
 
     // K/V stages start as zeros: a page that is not loaded (bad block id) then
     // holds finite data only
     for (int x = tid; x < kStages * 2 * kTileB / 16; x += kThreads)
-        *reinterpret_cast<uint4 *>(gbase + kTileB + 16 * x) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(gbase + 2 * kTileB + 16 * x) = make_uint4(0, 0, 0, 0);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (tid == 0) {
-        ptx::mbar_init(&bars.q_full, 128);
+        ptx::mbar_init(&bars.q_full, 256);
         for (int i = 0; i < kStages; ++i) {
             ptx::mbar_init(&bars.kv_full[i], 1);
             ptx::mbar_init(&bars.kv_empty[i], 1);
@@ -229,35 +235,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tm = bars.tmem_base;
     int *abort_flag = &bars.abort_flag;
 
-    if (warp < 4) {
-        // ======================= softmax warpgroup =======================
-        const int r = tid;                       // row = TMEM lane
-        const int i = tok_base + r / G;          // query token in the sequence's chunk
+    if (warp < 8) {
+        // ======================= softmax: warpgroup w owns Q tile w =======================
+        const int w = warp >> 2;
+        const int r = tid & 127;                 // row of the tile = TMEM lane
+        const int R = w * 128 + r;               // row of the CTA
+        const int i = tok_base + R / G;          // query token in the sequence's chunk
         const bool valid = i < ql;
         const int pos = pos0 + min(i, ql - 1);   // causal limit (inclusive)
         {   // Q row -> shared memory, K-major 128-byte swizzle
             const uint4 *src = reinterpret_cast<const uint4 *>(
-                a.q + ((int64_t)(q0 + min(i, ql - 1)) * a.Hq + h * G + r % G) * kD);
+                a.q + ((int64_t)(q0 + min(i, ql - 1)) * a.Hq + h * G + R % G) * kD);
+            uint8_t *q = gbase + w * kTileB;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const uint4 v = src[c];
-                const uint32_t off = (uint32_t)((c >> 3) * kSlice + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-                *reinterpret_cast<uint4 *>(gbase + off) = v;
+                const uint32_t off =
+                    (uint32_t)((c >> 3) * kSlice + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+                *reinterpret_cast<uint4 *>(q + off) = v;
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             ptx::mbar_arrive(&bars.q_full);
         }
-        const uint32_t lane_base = tm + ((uint32_t)(warp * 32) << 16);
+        const uint32_t lane_base = tm + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t sbuf = lane_base + w * 128;          // S, then P over it
+        const uint32_t obuf = lane_base + kColO + w * 128;  // O
         const float sl = a.scale_log2;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_kt && ok; ++j) {
-            const int bb = j & 1;
-            if (!(ok = warp_wait(&bars.s_full[bb], (j >> 1) & 1, abort_flag))) break;
+            if (!(ok = warp_wait(&bars.s_full[w], j & 1, abort_flag))) break;
             fence_after();
-            const uint32_t sbuf = lane_base + bb * 128;
             // tokens t0 + e with e <= lim are visible to this row (lim >= 127: all)
             const int lim = valid ? pos - j * kN : -1;
+            // tiles every row of the warp sees in full (all but the diagonal ones) skip
+            // the causal select; with scale > 0 the max is taken on the raw logits
+            const bool full = __all_sync(0xffffffffu, lim >= kN - 1) && sl > 0.f;
             // ---- pass 1: row maximum of the scaled, masked logits (4 chunks of 32
             // columns, 8 independent max chains)
             float mx = -INFINITY;
@@ -269,14 +282,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float mk[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) mk[q] = -INFINITY;
+                if (full) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float x = (32 * c + e <= lim) ? __uint_as_float(v[e]) * sl : -INFINITY;
-                    mk[e & 7] = fmaxf(mk[e & 7], x);
+                    for (int e = 0; e < 32; ++e) mk[e & 7] = fmaxf(mk[e & 7], __uint_as_float(v[e]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float x =
+                            (32 * c + e <= lim) ? __uint_as_float(v[e]) * sl : -INFINITY;
+                        mk[e & 7] = fmaxf(mk[e & 7], x);
+                    }
                 }
 #pragma unroll
                 for (int q = 0; q < 8; ++q) mx = fmaxf(mx, mk[q]);
             }
+            if (full) mx *= sl;
             const float mn = fmaxf(m, mx);
             // lazy rescale: a row moves its reference max only when the tile's max
             // exceeds it by more than 8 (weights stay below 2^8 otherwise); the first
@@ -284,19 +304,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool move = mn > m + 8.f;
             const bool rescale = move && j > 0 && m != -INFINITY;  // O holds tiles < j
             if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access
-                if (!(ok = warp_wait(&bars.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)))
-                    break;
+                if (!(ok = warp_wait(&bars.pv_done[w], (j - 1) & 1, abort_flag))) break;
                 fence_after();
                 const float alpha = rescale ? ex2(m - mn) : 1.f;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t v[32];
-                    tmem_ld32(lane_base + kColO + 32 * c, v);
+                    tmem_ld32(obuf + 32 * c, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
                         v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                    tmem_st32(lane_base + kColO + 32 * c, v);
+                    tmem_st32(obuf + 32 * c, v);
                 }
                 l *= alpha;
             }
@@ -310,38 +329,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t v[32];
                 tmem_ld32(sbuf + 32 * c, v);
                 tmem_wait_ld();
-                uint32_t w[32];
+                float x[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] = fmaf(__uint_as_float(v[e]), sl, -u);
+                if (!full) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (32 * c + e > lim) x[e] = -INFINITY;  // weight 0
+                }
+                uint32_t wv[32];
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const int e = 16 * half + 2 * q;
-                        const float x0 = (32 * c + e <= lim) ? __uint_as_float(v[e]) * sl - u : -INFINITY;
-                        const float x1 =
-                            (32 * c + e + 1 <= lim) ? __uint_as_float(v[e + 1]) * sl - u : -INFINITY;
-                        const float p0 = ex2(x0), p1 = ex2(x1);
+                        const float p0 = ex2(x[e]), p1 = ex2(x[e + 1]);
                         ls[q & 3] += p0 + p1;
                         const uint32_t hi = ptx::pack_bf16(p0, p1);
-                        w[16 * half + q] = hi;
-                        w[16 * half + 8 + q] = ptx::pack_bf16(p0 - bf16_lo(hi), p1 - bf16_hi(hi));
+                        wv[16 * half + q] = hi;
+                        wv[16 * half + 8 + q] = ptx::pack_bf16(p0 - bf16_lo(hi), p1 - bf16_hi(hi));
                     }
                 }
-                tmem_st32(sbuf + 32 * c, w);
+                tmem_st32(sbuf + 32 * c, wv);
             }
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             tmem_wait_st();
             fence_before();
-            ptx::mbar_arrive(&bars.p_full[bb]);
+            ptx::mbar_arrive(&bars.p_full[w]);
         }
         if (ok && warp_wait(&bars.o_final, 0, abort_flag)) {
             fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             uint32_t *orow = reinterpret_cast<uint32_t *>(
-                a.out + ((int64_t)(q0 + min(i, ql - 1)) * a.Hq + h * G + r % G) * kD);
-#pragma unroll
+                a.out + ((int64_t)(q0 + min(i, ql - 1)) * a.Hq + h * G + R % G) * kD);
+#pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t v[32];
-                tmem_ld32(lane_base + kColO + 32 * c, v);
+                tmem_ld32(obuf + 32 * c, v);
                 tmem_wait_ld();
                 if (valid) {
 #pragma unroll
@@ -352,64 +376,91 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else if (warp == 4) {
+    } else if (warp == 8) {
         // ======================= MMA issue =======================
-        bool ok = warp_wait(&bars.q_full, 0, abort_flag);
+        // tensor-core order per K/V tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so
+        // each softmax warpgroup works while the other tile's products run
         const uint32_t id_qk = idesc(false), id_pv = idesc(true);
-        for (int j = 0; j <= n_kt && ok; ++j) {
-            if (j < n_kt) {
-                const int st = j % kStages, bb = j & 1;
-                if (!(ok = warp_wait(&bars.kv_full[st], (j / kStages) & 1, abort_flag))) break;
-                const int t0 = j * kN;
-                if (t0 + kN > len) {
-                    // V rows at or past the context end: zero them (the weights there
-                    // are 0, and 0 x NaN would still poison the sum)
-                    const int r0 = max(0, len - t0);
-                    for (int x = r0 * 16 + lane; x < kN * 16; x += 32) {
-                        const int row = x >> 4, c = x & 15;
-                        const uint32_t off = (uint32_t)((c >> 3) * kSlice + row * 128 + (c & 7) * 16);
-                        *reinterpret_cast<uint4 *>(gbase + (sV(st) - base) + off) =
-                            make_uint4(0, 0, 0, 0);
-                    }
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    __syncwarp();
-                }
-                if (j >= 2 && !(ok = warp_wait(&bars.pv_done[bb], ((j >> 1) - 1) & 1, abort_flag)))
-                    break;
-                fence_after();
-                if (lane == 0) {
-#pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
-                        const uint32_t koff = (uint32_t)((ks >> 2) * kSlice + (ks & 3) * 32);
-                        mma_ss(tm + bb * 128, sdesc(sQ + koff, 16, 1024),
-                               sdesc(sK(st) + koff, 16, 1024), id_qk, ks > 0);
-                    }
-                    commit(&bars.s_full[bb]);
-                }
-                __syncwarp();
+        auto zero_tail = [&](int j, int st) {
+            // V rows at or past the context end: zero them (the weights there are 0,
+            // and 0 x NaN would still poison the sum)
+            const int t0 = j * kN;
+            if (t0 + kN <= len) return;
+            const int r0 = max(0, len - t0);
+            for (int x = r0 * 16 + lane; x < kN * 16; x += 32) {
+                const int row = x >> 4, c = x & 15;
+                const uint32_t off = (uint32_t)((c >> 3) * kSlice + row * 128 + (c & 7) * 16);
+                *reinterpret_cast<uint4 *>(gbase + (sV(st) - base) + off) = make_uint4(0, 0, 0, 0);
             }
-            if (j >= 1) {
-                const int jj = j - 1, bb = jj & 1, st = jj % kStages;
-                if (!(ok = warp_wait(&bars.p_full[bb], (jj >> 1) & 1, abort_flag))) break;
-                fence_after();
-                if (lane == 0) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+        };
+        auto issue_s = [&](int w, int st) {
+            if (lane == 0) {
 #pragma unroll
-                    for (int kk = 0; kk < kN / 16; ++kk) {
-                        // V: 16 token rows per k-step; N = 128 dims across the two slices
-                        const uint64_t vd = sdesc(sV(st) + (uint32_t)(kk * 16 * 128), kSlice, 1024);
-                        mma_ts(tm + kColO, tm + bb * 128 + 16 * kk, vd, id_pv,
-                               (jj > 0 || kk > 0) ? 1u : 0u);
-                        mma_ts(tm + kColO, tm + bb * 128 + 16 * kk + 8, vd, id_pv, 1u);
-                    }
-                    commit(&bars.pv_done[bb]);
-                    commit(&bars.kv_empty[st]);
-                    if (jj == n_kt - 1) commit(&bars.o_final);
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const uint32_t koff = (uint32_t)((ks >> 2) * kSlice + (ks & 3) * 32);
+                    mma_ss(tm + w * 128, sdesc(sQ(w) + koff, 16, 1024),
+                           sdesc(sK(st) + koff, 16, 1024), id_qk, ks > 0);
                 }
-                __syncwarp();
+                commit(&bars.s_full[w]);
+            }
+            __syncwarp();
+        };
+        auto issue_pv = [&](int w, int j, int st) {
+            if (lane == 0) {
+#pragma unroll
+                for (int kk = 0; kk < kN / 16; ++kk) {
+                    // V: 16 token rows per k-step; N = 128 dims across the two slices
+                    const uint64_t vd = sdesc(sV(st) + (uint32_t)(kk * 16 * 128), kSlice, 1024);
+                    mma_ts(tm + kColO + w * 128, tm + w * 128 + 16 * kk, vd, id_pv,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tm + kColO + w * 128, tm + w * 128 + 16 * kk + 8, vd, id_pv, 1u);
+                }
+                commit(&bars.pv_done[w]);
+            }
+            __syncwarp();
+        };
+        bool ok = warp_wait(&bars.q_full, 0, abort_flag) &&
+                  warp_wait(&bars.kv_full[0], 0, abort_flag);
+        if (ok) {
+            zero_tail(0, 0);
+            fence_after();
+            issue_s(0, 0);
+            issue_s(1, 0);
+        }
+        for (int j = 0; j < n_kt && ok; ++j) {
+            const int st = j % kStages, st1 = (j + 1) % kStages;
+            const bool more = j + 1 < n_kt;
+            // ---- tile A
+            if (!(ok = warp_wait(&bars.p_full[0], j & 1, abort_flag))) break;
+            fence_after();
+            issue_pv(0, j, st);
+            if (more) {
+                if (!(ok = warp_wait(&bars.kv_full[st1], ((j + 1) / kStages) & 1, abort_flag))) break;
+                zero_tail(j + 1, st1);
+                // S_A(j+1) overwrites the columns PV_A(j) reads its P from
+                if (!(ok = warp_wait(&bars.pv_done[0], j & 1, abort_flag))) break;
+                fence_after();
+                issue_s(0, st1);
+            }
+            // ---- tile B
+            if (!(ok = warp_wait(&bars.p_full[1], j & 1, abort_flag))) break;
+            fence_after();
+            issue_pv(1, j, st);
+            if (lane == 0) {
+                commit(&bars.kv_empty[st]);
+                if (!more) commit(&bars.o_final);
+            }
+            __syncwarp();
+            if (more) {
+                if (!(ok = warp_wait(&bars.pv_done[1], j & 1, abort_flag))) break;
+                fence_after();
+                issue_s(1, st1);
             }
         }
-    } else if (warp == 5) {
-        // ======================= TMA producer =======================
+    } else {
+        // ======================= TMA producer (warp 9) =======================
         // lane pg < 8 owns 16-token page pg of every tile: it looks up the page's
         // physical block (one tile ahead, so the table read is off the critical
         // path) and issues the page's four boxes
@@ -434,7 +485,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool load = in && blk >= 0 && (int64_t)blk < a.N;
             if (in && !load) raise_flag(a.err, PA_DEV_BAD_BLOCK);
             const unsigned lm = __ballot_sync(0xffffffffu, load);
-            if (lane == 0) ptx::mbar_arrive_expect_tx(&bars.kv_full[st], (uint32_t)__popc(lm) * 4u * 2048u);
+            if (lane == 0)
+                ptx::mbar_arrive_expect_tx(&bars.kv_full[st], (uint32_t)__popc(lm) * 4u * 2048u);
             __syncwarp();
             if (load) {
                 const int off = t % a.bs;
@@ -509,7 +561,7 @@ cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs &a, int max_q_len, cuda
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_set[dev] = true;
     }
-    const int QT = kM / a.G;
+    const int QT = kRows / a.G;
     dim3 grid((unsigned)((max_q_len + QT - 1) / QT), (unsigned)a.Hkv, (unsigned)a.B);
     prefill_attn_tc_kernel<<<grid, kThreads, kSmem, st>>>(km, vm, a);
     return cudaGetLastError();
