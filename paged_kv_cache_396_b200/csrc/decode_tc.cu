@@ -796,16 +796,26 @@ __device__ __forceinline__ void consumer_i8(const Args &a, uint8_t *stages, Stag
                         ptx::mma_s8(sl8[nt], ql[kk][0], qlb[kk][0], ql[kk][1], qlb[kk][1], wl[kk],
                                     wh[kk]);
                     } else {
-                        ptx::mma_s8(sh[nt], qh[kk][0], 0u, qh[kk][1], 0u, wl[kk], wh[kk]);
-                        ptx::mma_s8(sl8[nt], ql[kk][0], 0u, ql[kk][1], 0u, wl[kk], wh[kk]);
+                        // G <= 8: the lo parts ride in the empty rows g + 8 of the same MMA
+                        ptx::mma_s8(sh[nt], qh[kk][0], ql[kk][0], qh[kk][1], ql[kk][1], wl[kk],
+                                    wh[kk]);
                     }
                 }
             }
             float s0[4], s1[4];
+            if constexpr (G16) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                s0[i] = (float)(sh[0][i] * 128 + sl8[0][i]) * (i < 2 ? qs : qsb);
-                s1[i] = (float)(sh[1][i] * 128 + sl8[1][i]) * (i < 2 ? qs : qsb);
+                for (int i = 0; i < 4; ++i) {
+                    s0[i] = (float)(sh[0][i] * 128 + sl8[0][i]) * (i < 2 ? qs : qsb);
+                    s1[i] = (float)(sh[1][i] * 128 + sl8[1][i]) * (i < 2 ? qs : qsb);
+                }
+            } else {  // rows g: hi . K in entries 0, 1; lo . K in entries 2, 3
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    s0[i] = (float)(sh[0][i] * 128 + sh[0][i + 2]) * qs;
+                    s1[i] = (float)(sh[1][i] * 128 + sh[1][i + 2]) * qs;
+                }
+                s0[2] = s0[3] = s1[2] = s1[3] = 0.f;
             }
             // ---- online softmax; K scale folded into the logit
             const int t_a = 2 * tig, t_b = 8 + 2 * tig;
