@@ -329,6 +329,31 @@ class Runner:
 
 
 # ----------------------------------------------------------------------------- oracle
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def with_single_core(cpu, fn, budget_s):
+    """Add the same oracle timing on one thread (a quarter of the budget) and the
+    host CPU model to a cpu_baseline dict."""
+    import oracle
+    n = oracle.threads()
+    oracle.set_threads(1)
+    try:
+        v1, _, d1 = fn(budget_s / 4)
+    finally:
+        oracle.set_threads(n)
+    cpu["single_core"] = {"value": v1, "unit": cpu["unit"], "sample": d1}
+    cpu["cpu_model"] = cpu_model()
+    return cpu
+
+
 def oracle_throughput(wl, budget_s, max_layers=None):
     """Time the fp64 oracle (append + decode, plus score + select for c2) on
     (layer, sequence-batch) samples of the workload for about budget_s seconds;
@@ -641,11 +666,12 @@ def run_prefill(args, device, world, rank):
         raise SystemExit(f"device error flag {err.item()} during timing")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v_, cores, desc = prefill_oracle_throughput(
-            W.PrefillWorkload(cfg, wl.k.cpu(), wl.v.cpu(), wl.cu_seqlens, wl.block_tables, N),
-            args.cpu_seconds)
+        host_wl = W.PrefillWorkload(cfg, wl.k.cpu(), wl.v.cpu(), wl.cu_seqlens, wl.block_tables, N)
+        v_, cores, desc = prefill_oracle_throughput(host_wl, args.cpu_seconds)
         cpu = {"value": v_, "unit": "prompt tokens/s", "cores": cores, "kind": "oracle",
                "sample": desc}
+        cpu = with_single_core(cpu, lambda t: prefill_oracle_throughput(host_wl, t),
+                               args.cpu_seconds)
     if rank == 0:
         line = {
             "metric": "PagedEviction prefill compression: prompt tokens/s and score-kernel "
@@ -798,12 +824,14 @@ def run_chunked(args, device, world, rank):
         raise SystemExit(f"device error flag {err.item()} during timing")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v_, cores, desc = chunk_oracle_throughput(
-            W.ChunkWorkload(cfg, wl.k_pool.cpu(), wl.v_pool.cpu(), wl.k_new.cpu(),
-                            wl.v_new.cpu(), wl.q.cpu(), wl.cu_q, wl.ctx_lens, wl.positions,
-                            wl.block_tables, wl.num_blocks), args.cpu_seconds)
+        host_wl = W.ChunkWorkload(cfg, wl.k_pool.cpu(), wl.v_pool.cpu(), wl.k_new.cpu(),
+                                  wl.v_new.cpu(), wl.q.cpu(), wl.cu_q, wl.ctx_lens, wl.positions,
+                                  wl.block_tables, wl.num_blocks)
+        v_, cores, desc = chunk_oracle_throughput(host_wl, args.cpu_seconds)
         cpu = {"value": v_, "unit": "chunk tokens/s", "cores": cores, "kind": "oracle",
                "sample": desc}
+        cpu = with_single_core(cpu, lambda t: chunk_oracle_throughput(host_wl, t),
+                               args.cpu_seconds)
     if rank == 0:
         line = {
             "metric": "chunked prefill attention: chunk tokens/s and tensor TFLOP/s",
@@ -979,6 +1007,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, desc = oracle_throughput(r.wl, args.cpu_seconds)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+        cpu = with_single_core(cpu, lambda t: oracle_throughput(r.wl, t), args.cpu_seconds)
 
     if rank == 0:
         traffic = recorded_traffic(traffic_key(args, cfg))

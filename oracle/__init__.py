@@ -72,6 +72,8 @@ def _lib():
         lib.or_paged_prefill.restype = None
         lib.or_paged_prefill.argtypes = [p, p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32,
                                          dbl]
+        lib.or_set_threads.restype = None
+        lib.or_set_threads.argtypes = [i32]
         lib.or_e4m3_to_f64.restype = dbl
         lib.or_e4m3_to_f64.argtypes = [ctypes.c_uint8]
         lib.or_append_kv_fp8.restype = None
@@ -94,10 +96,23 @@ def _c(a, dtype):
     return a
 
 
+_THREADS = None
+
+
 def threads() -> int:
-    """OpenMP threads the oracle's parallel loops use (OMP_NUM_THREADS or all cores)."""
+    """OpenMP threads the oracle's parallel loops use (set_threads, else
+    OMP_NUM_THREADS, else all cores)."""
+    if _THREADS is not None:
+        return _THREADS
     env = os.environ.get("OMP_NUM_THREADS")
     return int(env) if env else (os.cpu_count() or 1)
+
+
+def set_threads(n: int) -> None:
+    """Use n OpenMP threads from now on (timing only: results do not depend on it)."""
+    global _THREADS
+    _lib().or_set_threads(int(n))
+    _THREADS = int(n)
 
 
 # --------------------------------------------------------------------------- sizes

@@ -38,6 +38,19 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Thread count of the parallel loops below (timing only; results do not depend
+ * on it: every parallel loop writes disjoint outputs). */
+void or_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
 
 /* bf16 is the upper half of an IEEE binary32: widen by a 16-bit shift. */
 static float bf16_to_f32(uint16_t x) {
