@@ -271,31 +271,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             // tiles every row of the warp sees in full (all but the diagonal ones) skip
             // the causal select; with scale > 0 the max is taken on the raw logits
             const bool full = __all_sync(0xffffffffu, lim >= kN - 1) && sl > 0.f;
-            // ---- pass 1: row maximum of the scaled, masked logits (4 chunks of 32
-            // columns, 8 independent max chains)
-            float mx = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tmem_ld32(sbuf + 32 * c, v);
-                tmem_wait_ld();
-                float mk[8];
+            // ---- the row's 128 logits of this tile: four 32-column TMEM reads in
+            // flight, one wait; then the row maximum of the scaled, masked logits (8
+            // independent max chains)
+            uint32_t v[4][32];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) mk[q] = -INFINITY;
-                if (full) {
+            for (int c = 0; c < 4; ++c) tmem_ld32(sbuf + 32 * c, v[c]);
+            tmem_wait_ld();
+            float mk[8];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) mk[e & 7] = fmaxf(mk[e & 7], __uint_as_float(v[e]));
-                } else {
+            for (int q = 0; q < 8; ++q) mk[q] = -INFINITY;
+            if (full) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        mk[e & 7] = fmaxf(mk[e & 7], __uint_as_float(v[c][e]));
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const float x =
-                            (32 * c + e <= lim) ? __uint_as_float(v[e]) * sl : -INFINITY;
+                            (32 * c + e <= lim) ? __uint_as_float(v[c][e]) * sl : -INFINITY;
                         mk[e & 7] = fmaxf(mk[e & 7], x);
                     }
-                }
-#pragma unroll
-                for (int q = 0; q < 8; ++q) mx = fmaxf(mx, mk[q]);
             }
+            float mx = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])),
+                             fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7])));
             if (full) mx *= sl;
             const float mn = fmaxf(m, mx);
             // lazy rescale: a row moves its reference max only when the tile's max
@@ -303,35 +306,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             // finite max always moves it (-inf + 8 = -inf)
             const bool move = mn > m + 8.f;
             const bool rescale = move && j > 0 && m != -INFINITY;  // O holds tiles < j
-            if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access
-                if (!(ok = warp_wait(&bars.pv_done[w], (j - 1) & 1, abort_flag))) break;
-                fence_after();
-                const float alpha = rescale ? ex2(m - mn) : 1.f;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(obuf + 32 * c, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                    tmem_st32(obuf + 32 * c, v);
-                }
-                l *= alpha;
-            }
+            const float alpha = rescale ? ex2(m - mn) : 1.f;
             if (move) m = mn;
             const float u = m == -INFINITY ? 0.f : m;
             // ---- pass 2: P = exp2(s - u) as hi + lo bf16 over the S columns: k-step kk
             // (16 tokens) at columns 16kk (hi, 8 columns of bf16 pairs) and 16kk + 8 (lo)
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
+#pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tmem_ld32(sbuf + 32 * c, v);
-                tmem_wait_ld();
                 float x[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = fmaf(__uint_as_float(v[e]), sl, -u);
+                for (int e = 0; e < 32; ++e) x[e] = fmaf(__uint_as_float(v[c][e]), sl, -u);
                 if (!full) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
@@ -352,7 +337,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tmem_st32(sbuf + 32 * c, wv);
             }
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            // O is rescaled after P is written, when the logits' registers are free; the
+            // P V of this tile is issued only after the arrive below
+            if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access
+                if (!(ok = warp_wait(&bars.pv_done[w], (j - 1) & 1, abort_flag))) break;
+                fence_after();
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(obuf + 32 * c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(obuf + 32 * c, o);
+                }
+            }
+            l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
             tmem_wait_st();
             fence_before();
             ptx::mbar_arrive(&bars.p_full[w]);
