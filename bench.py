@@ -204,10 +204,8 @@ class Runner:
         self.out = torch.empty(self.L, B, Hq, d, dtype=torch.bfloat16, device=device)
         self.ws = pk.alloc_workspace(B, Hq, Hkv, d, bs, MB, num_splits, device)
         self.num_splits = num_splits
-        self.S, self.chunk, self.dec_launches = pk.pa_decode_plan(B, Hq, Hkv, d, bs, MB,
-                                                                  num_splits)
-        # the staged kernel launches plan + decode (+ merge); the general one decode (+ merge)
-        self.staged = self.dec_launches - (1 if self.S > 1 else 0) >= 2
+        self.S, self.chunk, self.dec_launches, self.staged = pk.pa_decode_plan(
+            B, Hq, Hkv, d, bs, MB, num_splits)
         if cfg.fp8:
             N = wl.num_blocks
             self.k8 = torch.zeros(self.L, N, bs, Hkv, d, dtype=torch.uint8, device=device)

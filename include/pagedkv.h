@@ -121,10 +121,14 @@ size_t pa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int bs,
  * receives the maximum number of partitions of one sequence, *chunk_tokens_out
  * the tokens per partition (for the staged kernel: the minimum; it sizes the
  * partitions from the actual lengths on the device), *launches_out (nullable)
- * the kernels one pa_decode call launches.  Returns PA_OK or a PA_ERR_* code. */
+ * the kernels one pa_decode call launches, *staged_out (nullable) 1 when the
+ * staged tensor-core kernel runs (a plan kernel, the decode kernel, then a
+ * merge kernel when a sequence has several partial results), 0 for the
+ * general-shape kernel (decode, then a merge kernel when partitions > 1).
+ * Returns PA_OK or a PA_ERR_* code. */
 int pa_decode_plan(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq,
                    int num_splits, int *num_splits_out, int *chunk_tokens_out,
-                   int *launches_out);
+                   int *launches_out, int *staged_out);
 
 int pa_decode(uint16_t *out, const uint16_t *q,
               const uint16_t *k_cache, const uint16_t *v_cache, int64_t block_stride,

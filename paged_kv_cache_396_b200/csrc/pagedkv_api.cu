@@ -272,7 +272,8 @@ size_t pa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int bs, int max_
 }
 
 int pa_decode_plan(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq, int num_splits,
-                   int *num_splits_out, int *chunk_tokens_out, int *launches_out) {
+                   int *num_splits_out, int *chunk_tokens_out, int *launches_out,
+                   int *staged_out) {
     if (!num_splits_out || !chunk_tokens_out) return PA_ERR_NULL;
     if (B < 0 || Hq < 1 || Hkv < 1 || bs < 1 || max_blocks_per_seq < 1) return PA_ERR_SHAPE;
     if (d != 64 && d != 128) return PA_ERR_SHAPE;
@@ -285,6 +286,7 @@ int pa_decode_plan(int B, int Hq, int Hkv, int d, int bs, int max_blocks_per_seq
     *chunk_tokens_out = p.chunk;
     if (launches_out)
         *launches_out = p.kernel == 1 ? 2 + ((p.S > 1 || p.wph > 1) ? 1 : 0) : 1 + (p.S > 1 ? 1 : 0);
+    if (staged_out) *staged_out = p.kernel == 1 ? 1 : 0;
     return PA_OK;
 }
 

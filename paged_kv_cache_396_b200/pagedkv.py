@@ -74,7 +74,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode_workspace_bytes.restype = sz
     lib.pa_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32]
     lib.pa_decode_plan.restype = i32
-    lib.pa_decode_plan.argtypes = [i32, i32, i32, i32, i32, i32, i32, p, p, p]
+    lib.pa_decode_plan.argtypes = [i32, i32, i32, i32, i32, i32, i32, p, p, p, p]
     lib.pa_decode.restype = i32
     lib.pa_decode.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, i64, f32, i32,
                               p, sz, p, p]
@@ -232,12 +232,12 @@ def pa_decode_workspace_bytes(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits=
 
 def pa_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits=0):
     """(partitions per sequence at most, tokens per partition, kernel launches per
-    call) that pa_decode will use for these sizes."""
-    s, c, n = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    call, staged tensor-core kernel or not) that pa_decode will use for these sizes."""
+    s, c, n, k = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
     _check("pa_decode_plan", load().pa_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq,
                                                    num_splits, ctypes.byref(s), ctypes.byref(c),
-                                                   ctypes.byref(n)))
-    return s.value, c.value, n.value
+                                                   ctypes.byref(n), ctypes.byref(k)))
+    return s.value, c.value, n.value, bool(k.value)
 
 
 def workspace_plan(workspace, B):

@@ -168,6 +168,30 @@ def test_deterministic_bitwise():
     assert torch.equal(a, dev.out[0])
 
 
+@pytest.mark.parametrize("kv", ["bf16", "int8"])
+def test_workspace_reuse_across_calls_with_other_partitions(kv):
+    """The staged kernel's plan, unit list and partials live in the caller's workspace
+    and are rewritten every call.  One workspace (filled with 0xff first) serves calls
+    whose lengths give different partition counts; every call matches the oracle."""
+    base = C["c3"] if kv == "bf16" else C["c5"]
+    c1 = W.scaled(base, key="reuse1", layers=1, batch=4, old_lens=(2500, 40, 900, 1))
+    c2 = W.scaled(base, key="reuse2", layers=1, batch=4, old_lens=(7, 2500, 64, 1300))
+    w1, w2 = W.generate(c1, "cpu"), W.generate(c2, "cpu")
+    r1, r2 = oracle_step(w1, 0, range(4)), oracle_step(w2, 0, range(4))
+    d1, d2 = Device(w1), Device(w2)
+    n = max(d1.ws.numel(), d2.ws.numel())
+    ws = torch.full((n,), 0xFF, dtype=torch.uint8, device="cuda")
+    d1.ws = d2.ws = ws
+    if kv == "int8":
+        d1.fill_int8_history(0)
+        d2.fill_int8_history(0)
+    for dev, ref, tag in ((d1, r1, "first"), (d2, r2, "second"), (d1, r1, "third")):
+        dev.step(0)
+        torch.cuda.synchronize()
+        assert dev.err.item() == 0
+        assert_attention_close(dev.out[0], ref["out"], f"{kv} {tag} call")
+
+
 def test_int8_codes_and_scales_bit_exact():
     wl = W.generate(MEDIUM["c5m"], "cpu")
     ref = oracle_step(wl, 0, range(wl.cfg.batch))
