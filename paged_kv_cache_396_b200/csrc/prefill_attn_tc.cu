@@ -68,23 +68,27 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
            ((uint64_t)((sbo >> 4) & 0x3fff) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The MMA and commit helpers are called by a whole warp with warp-uniform operands;
+// elect.sync picks the one lane that issues (the operands stay warp-uniform, which
+// keeps the issue cost per MMA low).
 __device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t id,
                                        uint32_t acc) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
         "l"(a), "l"(b), "r"(id), "r"(acc));
 }
 __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t id,
                                        uint32_t acc) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
         "r"(a_tmem), "l"(b), "r"(id), "r"(acc));
 }
 __device__ __forceinline__ void commit(uint64_t *bar) {
     asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
             ptx::smem_u32(bar))
         : "memory");
 }
@@ -397,30 +401,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
         };
         auto issue_s = [&](int w, int st) {
-            if (lane == 0) {
 #pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const uint32_t koff = (uint32_t)((ks >> 2) * kSlice + (ks & 3) * 32);
-                    mma_ss(tm + w * 128, sdesc(sQ(w) + koff, 16, 1024),
-                           sdesc(sK(st) + koff, 16, 1024), id_qk, ks > 0);
-                }
-                commit(&bars.s_full[w]);
+            for (int ks = 0; ks < kD / 16; ++ks) {
+                const uint32_t koff = (uint32_t)((ks >> 2) * kSlice + (ks & 3) * 32);
+                mma_ss(tm + w * 128, sdesc(sQ(w) + koff, 16, 1024),
+                       sdesc(sK(st) + koff, 16, 1024), id_qk, ks > 0);
             }
-            __syncwarp();
+            commit(&bars.s_full[w]);
         };
         auto issue_pv = [&](int w, int j, int st) {
-            if (lane == 0) {
 #pragma unroll
-                for (int kk = 0; kk < kN / 16; ++kk) {
-                    // V: 16 token rows per k-step; N = 128 dims across the two slices
-                    const uint64_t vd = sdesc(sV(st) + (uint32_t)(kk * 16 * 128), kSlice, 1024);
-                    mma_ts(tm + kColO + w * 128, tm + w * 128 + 16 * kk, vd, id_pv,
-                           (j > 0 || kk > 0) ? 1u : 0u);
-                    mma_ts(tm + kColO + w * 128, tm + w * 128 + 16 * kk + 8, vd, id_pv, 1u);
-                }
-                commit(&bars.pv_done[w]);
+            for (int kk = 0; kk < kN / 16; ++kk) {
+                // V: 16 token rows per k-step; N = 128 dims across the two slices
+                const uint64_t vd = sdesc(sV(st) + (uint32_t)(kk * 16 * 128), kSlice, 1024);
+                mma_ts(tm + kColO + w * 128, tm + w * 128 + 16 * kk, vd, id_pv,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+                mma_ts(tm + kColO + w * 128, tm + w * 128 + 16 * kk + 8, vd, id_pv, 1u);
             }
-            __syncwarp();
+            commit(&bars.pv_done[w]);
         };
         bool ok = warp_wait(&bars.q_full, 0, abort_flag) &&
                   warp_wait(&bars.kv_full[0], 0, abort_flag);
@@ -449,11 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!(ok = warp_wait(&bars.p_full[1], j & 1, abort_flag))) break;
             fence_after();
             issue_pv(1, j, st);
-            if (lane == 0) {
-                commit(&bars.kv_empty[st]);
-                if (!more) commit(&bars.o_final);
-            }
-            __syncwarp();
+            commit(&bars.kv_empty[st]);
+            if (!more) commit(&bars.o_final);
             if (more) {
                 if (!(ok = warp_wait(&bars.pv_done[1], j & 1, abort_flag))) break;
                 fence_after();
