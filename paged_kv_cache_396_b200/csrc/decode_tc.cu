@@ -93,9 +93,11 @@ struct Args {
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *ctx_lens, int32_t *err,
                                                    TcHeader *hdr, int32_t *ns, int4 *units, int B,
                                                    int max_ctx, int min_chunk, int target_units) {
+    constexpr int kSerialParts = 32, kMaxLong = 256;
     __shared__ long long s_red[32];
     __shared__ int hist[1024];
-    __shared__ int s_chunk;
+    __shared__ int s_chunk, s_nlong;
+    __shared__ int s_long[kMaxLong];
     const int tid = threadIdx.x;
     // launched programmatically after the previous kernel (e.g. the KV append):
     // let the decode kernel's CTAs get resident, then wait for the predecessor
@@ -122,6 +124,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *ctx_lens, int
         if (ch < min_chunk) ch = min_chunk;
         if (ch > max_ctx) ch = (max_ctx + kTile - 1) / kTile * kTile;
         s_chunk = (int)ch;
+        s_nlong = 0;
         hdr->chunk = (int)ch;
     }
     __syncthreads();
@@ -132,16 +135,34 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *ctx_lens, int
         step = len > 0 ? ((len + n - 1) / n + kTile - 1) / kTile * kTile : kTile;
         n = len > 0 ? (len + step - 1) / step : 1;
     };
+    // a thread per sequence (all lengths loaded at once); a sequence with more than
+    // kSerialParts partitions is left to a warp whose lanes take its partitions, so a
+    // few very long sequences do not serialise on a few threads
+    const int warp = tid >> 5, lane = tid & 31, nwarps = (int)(blockDim.x >> 5);
     for (int b = tid; b < B; b += blockDim.x) {
         int len = ctx_lens[b];
         if (len < 0 || len > max_ctx) len = 0;
         int n, step;
         part(len, n, step);
         ns[b] = n;
-        for (int c = 0; c < n; ++c) {
-            const int sz = min(step, len - c * step);
-            atomicAdd(&hist[min(1023, sz / kTile)], 1);
+        const int k = n > kSerialParts ? atomicAdd(&s_nlong, 1) : kMaxLong;
+        if (k < kMaxLong) {
+            s_long[k] = b;
+        } else {
+            for (int c = 0; c < n; ++c)
+                atomicAdd(&hist[min(1023, min(step, len - c * step) / kTile)], 1);
         }
+    }
+    __syncthreads();
+    const int nlong = min(s_nlong, kMaxLong);
+    for (int k = warp; k < nlong; k += nwarps) {
+        const int b = s_long[k];
+        int len = ctx_lens[b];
+        if (len < 0 || len > max_ctx) len = 0;
+        int n, step;
+        part(len, n, step);
+        for (int c = lane; c < n; c += 32)
+            atomicAdd(&hist[min(1023, min(step, len - c * step) / kTile)], 1);
     }
     __syncthreads();
     {   // exclusive prefix over the buckets, largest first (thread t owns bucket 1023 - t)
@@ -179,7 +200,24 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *ctx_lens, int
         if (len < 0 || len > max_ctx) len = 0;
         int n, step;
         part(len, n, step);
+        if (n > kSerialParts && nlong > 0) {   // listed (unless the list overflowed)?
+            bool listed = false;
+            for (int k = 0; k < nlong && !listed; ++k) listed = s_long[k] == b;
+            if (listed) continue;
+        }
         for (int c = 0; c < n; ++c) {
+            const int t0 = c * step, t1 = min(len, t0 + step);
+            const int pos = atomicAdd(&hist[min(1023, (t1 - t0) / kTile)], 1);
+            units[pos] = make_int4(b, c, t0, t1);
+        }
+    }
+    for (int k = warp; k < nlong; k += nwarps) {
+        const int b = s_long[k];
+        int len = ctx_lens[b];
+        if (len < 0 || len > max_ctx) len = 0;
+        int n, step;
+        part(len, n, step);
+        for (int c = lane; c < n; c += 32) {
             const int t0 = c * step, t1 = min(len, t0 + step);
             const int pos = atomicAdd(&hist[min(1023, (t1 - t0) / kTile)], 1);
             units[pos] = make_int4(b, c, t0, t1);
@@ -1204,7 +1242,66 @@ __global__ void __launch_bounds__(kThreads, 1)
         consumer<D, G16>(a, stages, meta, full, empty);
 }
 
-// Merge of the partials of one (sequence, query head) in slot order.
+// Merge of the partials of one (sequence, query head) in slot order:
+// M = max_s m_s, out = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
+// One thread per dim walks the partials; for sequences cut into many partitions
+// (long contexts) the D/32 warps of the CTA split the partials instead (lane:
+// D/32 dims, float4 / float2 loads) and add their sums in warp order, so the
+// loads of many partials are in flight at once.
+constexpr int kWideMerge = 32;   // partials per row from which the warps split them
+
+template <int D>
+__device__ __forceinline__ void merge_wide(const Args &a, int64_t bh, int i, int cnt,
+                                           int64_t base) {
+    constexpr int W = D / 32, E = D / 32;
+    __shared__ float s_max[W], s_l[W];
+    __shared__ float s_acc[W][D];
+    const int e = threadIdx.x, warp = e >> 5, lane = e & 31;
+    float M = -INFINITY;
+    for (int s = e; s < cnt; s += D) M = fmaxf(M, a.ws_ml[((base + s) * a.Hq + i) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+    if (lane == 0) s_max[warp] = M;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < W; ++w) M = fmaxf(M, s_max[w]);
+    float L = 0.f, A[E];
+#pragma unroll
+    for (int k = 0; k < E; ++k) A[k] = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll 8
+        for (int s = warp; s < cnt; s += W) {
+            const int64_t r = (base + s) * a.Hq + i;
+            const float2 ml = *reinterpret_cast<const float2 *>(a.ws_ml + r * 2);
+            const float f = exp2f(ml.x - M);
+            L = fmaf(ml.y, f, L);
+            const float *src = a.ws_acc + r * D + lane * E;
+            if constexpr (E == 4) {
+                const float4 v = *reinterpret_cast<const float4 *>(src);
+                A[0] = fmaf(v.x, f, A[0]);
+                A[1] = fmaf(v.y, f, A[1]);
+                A[2] = fmaf(v.z, f, A[2]);
+                A[3] = fmaf(v.w, f, A[3]);
+            } else {
+                const float2 v = *reinterpret_cast<const float2 *>(src);
+                A[0] = fmaf(v.x, f, A[0]);
+                A[1] = fmaf(v.y, f, A[1]);
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < E; ++k) s_acc[warp][lane * E + k] = A[k];
+    if (lane == 0) s_l[warp] = L;
+    __syncthreads();
+    float As = 0.f, Ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+        As += s_acc[w][e];
+        Ls += s_l[w];
+    }
+    a.out[bh * D + e] = f32_to_bf16_rn(Ls > 0.f ? As / Ls : 0.f);
+}
+
 template <int D>
 __global__ void __launch_bounds__(D) merge_tc_kernel(const Args a) {
     ptx::grid_dependency_wait();  // the decode kernel's partials are complete
@@ -1215,6 +1312,10 @@ __global__ void __launch_bounds__(D) merge_tc_kernel(const Args a) {
     if (nsb == 1 && a.wph == 1) return;  // written directly by the decode kernel
     const int cnt = nsb * a.wph;
     const int64_t base = (int64_t)b * a.S * a.wph;
+    if (cnt > kWideMerge) {   // uniform over the CTA
+        merge_wide<D>(a, bh, i, cnt, base);
+        return;
+    }
     float M = -INFINITY;
     for (int s = 0; s < cnt; ++s) M = fmaxf(M, a.ws_ml[((base + s) * a.Hq + i) * 2]);
     float L = 0.f, A = 0.f;
