@@ -365,19 +365,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && warp_wait(&bars.o_final, 0, abort_flag)) {
             fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            uint32_t *orow = reinterpret_cast<uint32_t *>(
+            uint4 *orow = reinterpret_cast<uint4 *>(
                 a.out + ((int64_t)(q0 + min(i, ql - 1)) * a.Hq + h * G + R % G) * kD);
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t v[32];
                 tmem_ld32(obuf + 32 * c, v);
                 tmem_wait_ld();
-                if (valid) {
+                if (valid) {   // 32 dims = 64 bytes of the row, as four 16-byte stores
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        orow[16 * c + e] =
-                            (uint32_t)f32_to_bf16_rn(__uint_as_float(v[2 * e]) * inv) |
-                            ((uint32_t)f32_to_bf16_rn(__uint_as_float(v[2 * e + 1]) * inv) << 16);
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int e = 4 * e4 + k;
+                            w4[k] = (uint32_t)f32_to_bf16_rn(__uint_as_float(v[2 * e]) * inv) |
+                                    ((uint32_t)f32_to_bf16_rn(__uint_as_float(v[2 * e + 1]) * inv)
+                                     << 16);
+                        }
+                        orow[4 * c + e4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
                 }
             }
         }
