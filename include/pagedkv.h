@@ -420,13 +420,30 @@ int pe_evict_compact_mask(int32_t *block_tables, int max_blocks_per_seq, int32_t
  * max_q_len >= every q_len_b (sizes the grid).  d in {64, 128}; G = Hq/Hkv in
  * {1, 2, 4, 8, 16}.  A sequence with q_len_b > ctx_lens[b] or a length outside
  * [0, MB*bs] gets zero output rows and sets PA_DEV_BAD_LEN; a block id outside
- * [0, N) sets PA_DEV_BAD_BLOCK and reads as zeros.  No workspace.
+ * [0, N) sets PA_DEV_BAD_BLOCK and reads as zeros.
+ *   workspace (nullable) : device scratch of at least
+ *     pa_prefill_attention_workspace_bytes(...) bytes for the same sizes.  With it
+ *     (d = 128, block size a multiple of 16) the work is balanced over the SMs: with
+ *     n query tiles of 256 rows and P SMs, floor(n / P) P tiles run whole, one CTA
+ *     each; the K/V ranges of the others are laid end to end and cut into one equal
+ *     range per SM, and a range cut inside a tile leaves fp32 partial results (O,
+ *     max, sum) in the workspace, merged with the log-sum-exp rule by the part that
+ *     finishes last.  It pays off when the tiles are fewer than the SMs (a chunk of
+ *     one or a few sequences).  Without it (NULL, or too small) one CTA serves each
+ *     query tile whole.  The contents are scratch; calls sharing one workspace must
+ *     be ordered on one stream.  The result is the same either way up to fp32
+ *     rounding.
+ * pa_prefill_attention_workspace_bytes returns 0 when the balanced mode does not
+ * apply to these sizes (the call then needs no workspace).
  * ==========================================================================*/
+size_t pa_prefill_attention_workspace_bytes(int B, int Hq, int Hkv, int d, int bs, int max_q_len);
+
 int pa_prefill_attention(uint16_t *out, const uint16_t *q, const int32_t *cu_q, int max_q_len,
                          const uint16_t *k_cache, const uint16_t *v_cache, int64_t block_stride,
                          const int32_t *block_tables, int max_blocks_per_seq,
                          const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
-                         int64_t num_blocks, float scale, int32_t *err_flag, void *stream);
+                         int64_t num_blocks, float scale, int32_t *err_flag, void *workspace,
+                         size_t workspace_bytes, void *stream);
 
 #ifdef __cplusplus
 }

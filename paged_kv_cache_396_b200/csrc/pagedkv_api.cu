@@ -560,11 +560,30 @@ int pe_evict_compact_mask(int32_t *block_tables, int max_blocks_per_seq, int32_t
                                                  static_cast<cudaStream_t>(stream)));
 }
 
+size_t pa_prefill_attention_workspace_bytes(int B, int Hq, int Hkv, int d, int bs,
+                                            int max_q_len) {
+    if (B <= 0 || max_q_len <= 0 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || bs < 1) return 0;
+    const int G = Hq / Hkv;
+    if (G > 16 || (G & (G - 1)) != 0) return 0;
+    const int sms = device_sms();
+    if (sms < 0) return 0;
+    pkv::PrefillAttnArgs a;
+    memset(&a, 0, sizeof a);
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.G = G;
+    a.d = d;
+    a.bs = bs;
+    return pkv::prefill_attn_tc_workspace_bytes(a, max_q_len, sms);
+}
+
 int pa_prefill_attention(uint16_t *out, const uint16_t *q, const int32_t *cu_q, int max_q_len,
                          const uint16_t *k_cache, const uint16_t *v_cache, int64_t block_stride,
                          const int32_t *block_tables, int max_blocks_per_seq,
                          const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
-                         int64_t num_blocks, float scale, int32_t *err_flag, void *stream) {
+                         int64_t num_blocks, float scale, int32_t *err_flag, void *workspace,
+                         size_t workspace_bytes, void *stream) {
     if (B == 0 || max_q_len == 0) return PA_OK;
     if (!out || !q || !cu_q || !k_cache || !v_cache || !block_tables || !ctx_lens || !err_flag)
         return PA_ERR_NULL;
@@ -602,6 +621,8 @@ int pa_prefill_attention(uint16_t *out, const uint16_t *q, const int32_t *cu_q, 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // tcgen05 / TMEM kernel for d = 128 and 16-token-aligned blocks (TMA pages);
     // the mma.sync kernel covers every other supported shape
-    return finish(pkv::prefill_attn_tc_supported(a) ? pkv::launch_prefill_attn_tc(a, max_q_len, st)
-                                                    : pkv::launch_prefill_attn(a, max_q_len, st));
+    if (workspace && !al16(workspace)) return PA_ERR_ALIGN;
+    return finish(pkv::prefill_attn_tc_supported(a)
+                      ? pkv::launch_prefill_attn_tc(a, max_q_len, workspace, workspace_bytes, sms, st)
+                      : pkv::launch_prefill_attn(a, max_q_len, st));
 }

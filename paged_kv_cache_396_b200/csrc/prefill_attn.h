@@ -23,8 +23,13 @@ struct PrefillAttnArgs {
 
 cudaError_t launch_prefill_attn(const PrefillAttnArgs &a, int max_q_len, cudaStream_t stream);
 
-// tcgen05 / TMEM version (prefill_attn_tc.cu): d = 128, bs a multiple of 16.
+// tcgen05 / TMEM version (prefill_attn_tc.cu): d = 128, bs a multiple of 16.  With a
+// workspace of prefill_attn_tc_workspace_bytes (0: no balanced mode for these sizes)
+// the work is balanced over the SMs (one persistent CTA per SM, items cut at range
+// boundaries, partial results merged); without it, one CTA per item.
 bool prefill_attn_tc_supported(const PrefillAttnArgs &a);
-cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs &a, int max_q_len, cudaStream_t stream);
+size_t prefill_attn_tc_workspace_bytes(const PrefillAttnArgs &a, int max_q_len, int sms);
+cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs &a, int max_q_len, void *ws,
+                                   size_t ws_bytes, int sms, cudaStream_t stream);
 
 }  // namespace pkv

@@ -28,6 +28,12 @@
 //              two 64-element slices each); two stages.
 // TMEM: S/P of tile A at columns [0,128), of tile B at [128,256); O of tile A at
 // [256,384), of tile B at [384,512).
+// Work: an item is (sequence, kv head, 256 query rows); a segment is a run of one
+// item's K/V tiles.  Without a workspace each CTA runs one whole item.  With one
+// (balanced mode) a plan kernel ranks the items: full waves of whole items, then
+// one equal range of the left-over items' tiles per SM; a segment cut from an item
+// leaves fp32 partials that the part finishing last merges (every role walks its
+// CTA's segments in a loop, with barrier phases carried across segments).
 // Every mbarrier wait is bounded (2 s of globaltimer); a timeout sets
 // PA_DEV_TIMEOUT and the CTA winds down, freeing its TMEM.
 #include <cuda.h>
@@ -159,45 +165,157 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int *a
 }
 
 struct Bars {
-    uint64_t q_full;              // 256 softmax threads: Q rows in shared memory
+    uint64_t q_full;              // 256 softmax threads: the segment's Q rows in shared memory
     uint64_t kv_full[kStages];    // TMA bytes of a K/V stage
     uint64_t kv_empty[kStages];   // commit after the last P V that read the stage
     uint64_t s_full[2];           // per Q tile: commit after S = Q K^T
     uint64_t p_full[2];           // per Q tile: 128 softmax threads wrote P
     uint64_t pv_done[2];          // per Q tile: commit after O += P V
-    uint64_t o_final;             // commit after the last P V of both tiles
+    uint64_t o_final;             // commit after the last P V of a segment (both tiles)
+    uint64_t o_free;              // 256 softmax threads: the segment's O read out of TMEM
     uint32_t tmem_base;
     int abort_flag;
 };
 
+// Work items: (sequence b, kv head h, 256-row query tile), dense index
+// d = (b * Hkv + h) * X + x, X = ceil(max_q_len / QT), q tile qt = n_qt(b) - 1 - x
+// (longest context first); x >= n_qt(b) is no item (no tiles).  A segment is a run
+// [jb, je) of one item's K/V tiles.
+struct Item {
+    int b, h, qt, q0, ql, len, pos0, tok_base, n_kt;   // n_kt = 0: no item or bad length
+};
+
+__device__ __forceinline__ Item item_of(const PrefillAttnArgs &a, int d, int X, int QT) {
+    Item it;
+    const int x = d % X, bh = d / X;
+    it.h = bh % a.Hkv;
+    it.b = bh / a.Hkv;
+    it.q0 = a.cu_q[it.b];
+    it.ql = a.cu_q[it.b + 1] - it.q0;
+    it.qt = (it.ql + QT - 1) / QT - 1 - x;
+    it.len = a.ctx_lens[it.b];
+    it.tok_base = it.qt * QT;
+    it.pos0 = it.len - it.ql;
+    it.n_kt = 0;
+    if (it.qt >= 0 && it.len >= 0 && (int64_t)it.len <= (int64_t)a.MB * a.bs && it.ql <= it.len)
+        it.n_kt = (it.pos0 + min(it.ql - 1, it.tok_base + QT - 1)) / kN + 1;
+    return it;
+}
+
+struct Seg {
+    int d;        // dense item index; -1: no more segments
+    int jb, je;   // K/V tiles of the segment
+    int slot;     // partial-result slot; -1: the segment is the whole item
+};
+
+// Balanced mode (a plan kernel writes the lists below every call).  With n items
+// that have rows and P SMs, the first whole = floor(n / P) P items, in item order,
+// run one per CTA (full waves; the CTAs of one (sequence, kv head) sweep its K/V
+// together, from L2).  The r = n - whole items left over are laid end to end (R
+// tiles) and CTA whole + k takes tiles [k L, (k + 1) L), L = ceil(R / P): one or
+// a few segments, the last wave then ends about evenly on every SM.  A segment
+// cut from an item writes its partial result to slot 2k (the item began in an
+// earlier range) or 2k + 1; for each 32 rows (a softmax warp) the part that
+// finishes last merges the item's parts in range order.  CTAs after those zero
+// the rows of items whose length cannot be served.
+struct StreamWs {
+    const int *hdr;     // whole, r, R, L, n_bad
+    const int *items;   // [n + n_bad] item index by rank, then the bad items
+    const int *pre;     // [r + 1] tile offsets of the items left over
+    const int *lrank;   // [n_items] rank among the items left over, -1: not left over
+    int *cnt;           // [n_items][8] parts done per (item, softmax warp)
+    float *part;        // [2P][256][d] O of a part (not normalised)
+    float *ml;          // [2P][256][2] (m, l) of a part; m in the log2 domain
+    int n_items, X, P;
+};
+
+__device__ __forceinline__ Seg left_seg(const StreamWs &w, int lr, int k, int R, int L,
+                                        int whole) {
+    const int a = w.pre[lr], e = w.pre[lr + 1];
+    const int r0 = k * L, r1 = min(R, r0 + L);
+    Seg s;
+    s.d = w.items[whole + lr];
+    s.jb = max(a, r0) - a;
+    s.je = min(e, r1) - a;
+    s.slot = (s.jb == 0 && s.je == e - a) ? -1 : (a < r0 ? 2 * k : 2 * k + 1);
+    return s;
+}
+
+// kStream = false: one CTA per item (grid x, y, z = q tile, kv head, sequence).
+// kStream = true: CTA c runs segment c of the balanced mode's list.  (Every role
+// walks a CTA's segments in a loop, so a CTA could serve several.)
+template <bool kStream>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap km,
-                           const __grid_constant__ CUtensorMap vm, const PrefillAttnArgs a) {
+                           const __grid_constant__ CUtensorMap vm, const PrefillAttnArgs a,
+                           const StreamWs sw) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ Bars bars;
-    const int b = blockIdx.z, h = blockIdx.y;
-    const int G = a.G, QT = kRows / G;   // query tokens per CTA (two tiles of 128 rows)
-    const int q0 = a.cu_q[b], ql = a.cu_q[b + 1] - q0;
-    const int n_qt = (ql + QT - 1) / QT;
-    const int qt = n_qt - 1 - (int)blockIdx.x;   // longest context first
-    if (qt < 0) return;
+    const int G = a.G, QT = kRows / G;   // query tokens per item (two tiles of 128 rows)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int len = a.ctx_lens[b];
-    const int tok_base = qt * QT;
-    if (len < 0 || (int64_t)len > (int64_t)a.MB * a.bs || ql > len) {
-        if (blockIdx.x == 0 && h == 0 && tid == 0) raise_flag(a.err, PA_DEV_BAD_LEN);
+    const int k = blockIdx.x;
+    const int X = kStream ? sw.X : (int)gridDim.x;
+    auto first_seg = [&]() -> Seg {
+        if constexpr (kStream) {
+            const int whole = sw.hdr[0], R = sw.hdr[2], L = sw.hdr[3], n_bad = sw.hdr[4];
+            if (k < whole) {
+                const int d = sw.items[k];
+                return Seg{d, 0, item_of(a, d, X, QT).n_kt, -1};
+            }
+            const int kk = k - whole;
+            if (kk >= sw.P) {   // zero-row CTAs for bad lengths, then nothing
+                if (kk - sw.P < n_bad)
+                    return Seg{sw.items[whole + sw.hdr[1] + kk - sw.P], 0, 0, -2};
+                return Seg{-1, 0, 0, -1};
+            }
+            if (kk * L >= R) return Seg{-1, 0, 0, -1};
+            int lo = 0, hi = sw.hdr[1];   // the left-over item holding tile kk L
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (sw.pre[mid] <= kk * L) lo = mid;
+                else hi = mid;
+            }
+            return left_seg(sw, lo, kk, R, L, whole);
+        } else {
+            const int d = ((int)blockIdx.z * a.Hkv + (int)blockIdx.y) * X + (int)blockIdx.x;
+            const Item it = item_of(a, d, X, QT);
+            return Seg{it.n_kt > 0 ? d : -1, 0, it.n_kt, -1};
+        }
+    };
+    auto next_seg = [&](const Seg &cur) -> Seg {
+        if constexpr (kStream) {
+            const int whole = sw.hdr[0], R = sw.hdr[2], L = sw.hdr[3];
+            const int kk = k - whole;
+            if (kk < 0 || kk >= sw.P) return Seg{-1, 0, 0, -1};
+            const int lr = sw.lrank[cur.d] + 1;
+            if (lr >= sw.hdr[1] || sw.pre[lr] >= min(R, (kk + 1) * L)) return Seg{-1, 0, 0, -1};
+            return left_seg(sw, lr, kk, R, L, whole);
+        } else {
+            return Seg{-1, 0, 0, -1};
+        }
+    };
+    const Seg seg0 = first_seg();
+    // an item whose length cannot be served: zero rows and PA_DEV_BAD_LEN (grid mode:
+    // no segment; balanced mode: a listed zero segment, slot -2)
+    int bad_d = -1;
+    if constexpr (!kStream) {
+        if (seg0.d < 0) bad_d = ((int)blockIdx.z * a.Hkv + (int)blockIdx.y) * X + (int)blockIdx.x;
+    } else {
+        if (seg0.d < 0) return;   // no work for this CTA
+        if (seg0.slot == -2) bad_d = seg0.d;
+    }
+    if (bad_d >= 0) {
+        const Item it = item_of(a, bad_d, X, QT);
+        if (it.qt < 0) return;   // no rows
+        if (bad_d % X == 0 && it.h == 0 && tid == 0) raise_flag(a.err, PA_DEV_BAD_LEN);
         for (int r = warp; r < kRows; r += kThreads / 32) {
-            const int i = tok_base + r / G;
-            if (i >= ql) continue;
-            uint16_t *o = a.out + ((int64_t)(q0 + i) * a.Hq + h * G + r % G) * kD;
+            const int i = it.tok_base + r / G;
+            if (i >= it.ql) continue;
+            uint16_t *o = a.out + ((int64_t)(it.q0 + i) * a.Hq + it.h * G + r % G) * kD;
             for (int e = lane; e < kD; e += 32) o[e] = 0;
         }
         return;
     }
-    const int pos0 = len - ql;
-    const int last_tok = min(ql - 1, tok_base + QT - 1);
-    const int p_max = pos0 + last_tok;
-    const int n_kt = p_max / kN + 1;
 
     // 1024-byte aligned tiles (the 128-byte swizzle pattern repeats every 1024 bytes)
     const uint32_t raw = ptx::smem_u32(smem_raw);
@@ -224,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&bars.pv_done[i], 1);
         }
         ptx::mbar_init(&bars.o_final, 1);
+        ptx::mbar_init(&bars.o_free, 256);
         bars.abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -243,13 +362,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ======================= softmax: warpgroup w owns Q tile w =======================
         const int w = warp >> 2;
         const int r = tid & 127;                 // row of the tile = TMEM lane
-        const int R = w * 128 + r;               // row of the CTA
-        const int i = tok_base + R / G;          // query token in the sequence's chunk
-        const bool valid = i < ql;
-        const int pos = pos0 + min(i, ql - 1);   // causal limit (inclusive)
-        {   // Q row -> shared memory, K-major 128-byte swizzle
+        const int R = w * 128 + r;               // row of the item
+        // Q row of an item -> shared memory, K-major 128-byte swizzle
+        auto load_q = [&](const Item &it) {
+            const int i = it.tok_base + R / G;
             const uint4 *src = reinterpret_cast<const uint4 *>(
-                a.q + ((int64_t)(q0 + min(i, ql - 1)) * a.Hq + h * G + R % G) * kD);
+                a.q + ((int64_t)(it.q0 + min(i, it.ql - 1)) * a.Hq + it.h * G + R % G) * kD);
             uint8_t *q = gbase + w * kTileB;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
@@ -260,140 +378,274 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             ptx::mbar_arrive(&bars.q_full);
-        }
+        };
         const uint32_t lane_base = tm + ((uint32_t)((warp & 3) * 32) << 16);
         const uint32_t sbuf = lane_base + w * 128;          // S, then P over it
         const uint32_t obuf = lane_base + kColO + w * 128;  // O
         const float sl = a.scale_log2;
-        float m = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < n_kt && ok; ++j) {
-            if (!(ok = warp_wait(&bars.s_full[w], j & 1, abort_flag))) break;
-            fence_after();
-            // tokens t0 + e with e <= lim are visible to this row (lim >= 127: all)
-            const int lim = valid ? pos - j * kN : -1;
-            // tiles every row of the warp sees in full (all but the diagonal ones) skip
-            // the causal select; with scale > 0 the max is taken on the raw logits
-            const bool full = __all_sync(0xffffffffu, lim >= kN - 1) && sl > 0.f;
-            // ---- the row's 128 logits of this tile: four 32-column TMEM reads in
-            // flight, one wait; then the row maximum of the scaled, masked logits (8
-            // independent max chains)
-            uint32_t v[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(sbuf + 32 * c, v[c]);
-            tmem_wait_ld();
-            float mk[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) mk[q] = -INFINITY;
-            if (full) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        mk[e & 7] = fmaxf(mk[e & 7], __uint_as_float(v[c][e]));
-            } else {
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float x =
-                            (32 * c + e <= lim) ? __uint_as_float(v[c][e]) * sl : -INFINITY;
-                        mk[e & 7] = fmaxf(mk[e & 7], x);
-                    }
-            }
-            float mx = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])),
-                             fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7])));
-            if (full) mx *= sl;
-            const float mn = fmaxf(m, mx);
-            // lazy rescale: a row moves its reference max only when the tile's max
-            // exceeds it by more than 8 (weights stay below 2^8 otherwise); the first
-            // finite max always moves it (-inf + 8 = -inf)
-            const bool move = mn > m + 8.f;
-            const bool rescale = move && j > 0 && m != -INFINITY;  // O holds tiles < j
-            const float alpha = rescale ? ex2(m - mn) : 1.f;
-            if (move) m = mn;
-            const float u = m == -INFINITY ? 0.f : m;
-            // ---- pass 2: P = exp2(s - u) as hi + lo bf16 over the S columns: k-step kk
-            // (16 tokens) at columns 16kk (hi, 8 columns of bf16 pairs) and 16kk + 8 (lo)
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float x[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = fmaf(__uint_as_float(v[c][e]), sl, -u);
-                if (!full) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (32 * c + e > lim) x[e] = -INFINITY;  // weight 0
-                }
-                uint32_t wv[32];
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int e = 16 * half + 2 * q;
-                        const float p0 = ex2(x[e]), p1 = ex2(x[e + 1]);
-                        ls[q & 3] += p0 + p1;
-                        const uint32_t hi = ptx::pack_bf16(p0, p1);
-                        wv[16 * half + q] = hi;
-                        wv[16 * half + 8 + q] = ptx::pack_bf16(p0 - bf16_lo(hi), p1 - bf16_hi(hi));
-                    }
-                }
-                tmem_st32(sbuf + 32 * c, wv);
-            }
-            // O is rescaled after P is written, when the logits' registers are free; the
-            // P V of this tile is issued only after the arrive below
-            if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access
-                if (!(ok = warp_wait(&bars.pv_done[w], (j - 1) & 1, abort_flag))) break;
+        int jt = 0, sn = 0;   // tiles and segments this CTA has done (barrier phases)
+        Seg sg = seg0;
+        Item it = item_of(a, sg.d, X, QT);
+        load_q(it);
+        while (ok) {
+            const int i = it.tok_base + R / G;       // query token in the sequence's chunk
+            const bool valid = i < it.ql;
+            const int pos = it.pos0 + min(i, it.ql - 1);   // causal limit (inclusive)
+            float m = -INFINITY, l = 0.f;
+            for (int j = sg.jb; j < sg.je && ok; ++j, ++jt) {
+                if (!(ok = warp_wait(&bars.s_full[w], jt & 1, abort_flag))) break;
                 fence_after();
+                // tokens t0 + e with e <= lim are visible to this row (lim >= 127: all)
+                const int lim = valid ? pos - j * kN : -1;
+                // tiles every row of the warp sees in full (all but the diagonal ones)
+                // skip the causal select; with scale > 0 the max is taken on the raw logits
+                const bool full = __all_sync(0xffffffffu, lim >= kN - 1) && sl > 0.f;
+                // ---- the row's 128 logits of this tile: four 32-column TMEM reads in
+                // flight, one wait; then the row maximum of the scaled, masked logits
+                // (8 independent max chains)
+                uint32_t v[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(sbuf + 32 * c, v[c]);
+                tmem_wait_ld();
+                float mk[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) mk[q] = -INFINITY;
+                if (full) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            mk[e & 7] = fmaxf(mk[e & 7], __uint_as_float(v[c][e]));
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const float x =
+                                (32 * c + e <= lim) ? __uint_as_float(v[c][e]) * sl : -INFINITY;
+                            mk[e & 7] = fmaxf(mk[e & 7], x);
+                        }
+                }
+                float mx = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])),
+                                 fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7])));
+                if (full) mx *= sl;
+                const float mn = fmaxf(m, mx);
+                // lazy rescale: a row moves its reference max only when the tile's max
+                // exceeds it by more than 8 (weights stay below 2^8 otherwise); the
+                // first finite max always moves it (-inf + 8 = -inf)
+                const bool move = mn > m + 8.f;
+                const bool rescale = move && j > sg.jb && m != -INFINITY;  // O holds tiles
+                const float alpha = rescale ? ex2(m - mn) : 1.f;
+                if (move) m = mn;
+                const float u = m == -INFINITY ? 0.f : m;
+                // ---- P = exp2(s - u) as hi + lo bf16 over the S columns: k-step kk
+                // (16 tokens) at columns 16kk (hi, 8 columns of bf16 pairs) and 16kk + 8 (lo)
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float x[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] = fmaf(__uint_as_float(v[c][e]), sl, -u);
+                    if (!full) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (32 * c + e > lim) x[e] = -INFINITY;  // weight 0
+                    }
+                    uint32_t wv[32];
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const int e = 16 * half + 2 * q;
+                            const float p0 = ex2(x[e]), p1 = ex2(x[e + 1]);
+                            ls[q & 3] += p0 + p1;
+                            const uint32_t hi = ptx::pack_bf16(p0, p1);
+                            wv[16 * half + q] = hi;
+                            wv[16 * half + 8 + q] =
+                                ptx::pack_bf16(p0 - bf16_lo(hi), p1 - bf16_hi(hi));
+                        }
+                    }
+                    tmem_st32(sbuf + 32 * c, wv);
+                }
+                // O is rescaled after P is written, when the logits' registers are free;
+                // the P V of this tile is issued only after the arrive below
+                if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access
+                    if (!(ok = warp_wait(&bars.pv_done[w], (jt - 1) & 1, abort_flag))) break;
+                    fence_after();
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(obuf + 32 * c, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(obuf + 32 * c, o);
+                    }
+                }
+                l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+                tmem_wait_st();
+                fence_before();
+                ptx::mbar_arrive(&bars.p_full[w]);
+            }
+            if (!ok) break;
+            // every S of this segment is done: the next segment's Q rows can go to
+            // shared memory now, so its first S overlaps this epilogue
+            const Seg nx = next_seg(sg);
+            Item itn;
+            if (nx.d >= 0) {
+                itn = item_of(a, nx.d, X, QT);
+                load_q(itn);
+            }
+            if (!(ok = warp_wait(&bars.o_final, sn & 1, abort_flag))) break;
+            fence_after();
+            if (sg.slot < 0) {   // the whole item: the normalised bf16 output row
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+                uint4 *orow = reinterpret_cast<uint4 *>(
+                    a.out + ((int64_t)(it.q0 + min(i, it.ql - 1)) * a.Hq + it.h * G + R % G) * kD);
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(obuf + 32 * c, o);
+                    uint32_t v[32];
+                    tmem_ld32(obuf + 32 * c, v);
                     tmem_wait_ld();
+                    if (valid) {   // 32 dims = 64 bytes of the row, as four 16-byte stores
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st32(obuf + 32 * c, o);
-                }
-            }
-            l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-            tmem_wait_st();
-            fence_before();
-            ptx::mbar_arrive(&bars.p_full[w]);
-        }
-        if (ok && warp_wait(&bars.o_final, 0, abort_flag)) {
-            fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            uint4 *orow = reinterpret_cast<uint4 *>(
-                a.out + ((int64_t)(q0 + min(i, ql - 1)) * a.Hq + h * G + R % G) * kD);
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
-                tmem_ld32(obuf + 32 * c, v);
-                tmem_wait_ld();
-                if (valid) {   // 32 dims = 64 bytes of the row, as four 16-byte stores
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            uint32_t w4[4];
 #pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        uint32_t w4[4];
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const int e = 4 * e4 + k;
-                            w4[k] = (uint32_t)f32_to_bf16_rn(__uint_as_float(v[2 * e]) * inv) |
-                                    ((uint32_t)f32_to_bf16_rn(__uint_as_float(v[2 * e + 1]) * inv)
-                                     << 16);
+                            for (int q = 0; q < 4; ++q) {
+                                const int e = 4 * e4 + q;
+                                w4[q] = (uint32_t)f32_to_bf16_rn(__uint_as_float(v[2 * e]) * inv) |
+                                        ((uint32_t)f32_to_bf16_rn(__uint_as_float(v[2 * e + 1]) *
+                                                                  inv)
+                                         << 16);
+                            }
+                            orow[4 * c + e4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                         }
-                        orow[4 * c + e4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                }
+            } else {   // a part of the item: its partial result, then the merge
+                // the item's parts: ranges k0 .. k1 of the left-over tiles
+                const int L = sw.hdr[3];
+                const int a0 = sw.pre[sw.lrank[sg.d]];
+                const int k0 = a0 / L, k1 = (a0 + it.n_kt - 1) / L;
+                auto slot_of = [&](int kk) { return a0 < kk * L ? 2 * kk : 2 * kk + 1; };
+                float4 *prow = reinterpret_cast<float4 *>(
+                    sw.part + ((int64_t)sg.slot * kRows + R) * kD);
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(obuf + 32 * c, v);
+                    tmem_wait_ld();
+                    if (valid) {
+#pragma unroll
+                        for (int e4 = 0; e4 < 8; ++e4)
+                            prow[8 * c + e4] = make_float4(
+                                __uint_as_float(v[4 * e4]), __uint_as_float(v[4 * e4 + 1]),
+                                __uint_as_float(v[4 * e4 + 2]), __uint_as_float(v[4 * e4 + 3]));
+                    }
+                }
+                if (valid)
+                    *reinterpret_cast<float2 *>(sw.ml + ((int64_t)sg.slot * kRows + R) * 2) =
+                        make_float2(m, l);
+                // the warp whose part completes its 32 rows' set merges them: a
+                // counter per (item, softmax warp), zeroed by the plan kernel
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0)
+                    last = atomicAdd(sw.cnt + (int64_t)sg.d * 8 + warp, 1) == k1 - k0;
+                if (__shfl_sync(0xffffffffu, last, 0)) {
+                    __threadfence();
+                    // M = max m_c, out = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c over
+                    // the item's parts in range order; the part rows' loads are issued
+                    // 16 at a time (two parts x 32 dims)
+                    auto mlrow = [&](int kk) {
+                        return __ldcg(reinterpret_cast<const float2 *>(
+                            sw.ml + ((int64_t)slot_of(kk) * kRows + R) * 2));
+                    };
+                    float M = -INFINITY;
+#pragma unroll 4
+                    for (int kk = k0; kk <= k1; ++kk) M = fmaxf(M, mlrow(kk).x);
+                    float Ls = 0.f;
+                    if (M != -INFINITY) {
+#pragma unroll 4
+                        for (int kk = k0; kk <= k1; ++kk) {
+                            const float2 ml = mlrow(kk);
+                            Ls = fmaf(ml.y, exp2f(ml.x - M), Ls);
+                        }
+                    }
+                    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+                    uint4 *orow = reinterpret_cast<uint4 *>(
+                        a.out + ((int64_t)(it.q0 + min(i, it.ql - 1)) * a.Hq + it.h * G + R % G) *
+                                    kD);
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {   // 32 dims a chunk
+                        float acc[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+                        auto add = [&](const float4 (&x)[8], float f) {
+#pragma unroll
+                            for (int e4 = 0; e4 < 8; ++e4) {
+                                acc[4 * e4] = fmaf(x[e4].x, f, acc[4 * e4]);
+                                acc[4 * e4 + 1] = fmaf(x[e4].y, f, acc[4 * e4 + 1]);
+                                acc[4 * e4 + 2] = fmaf(x[e4].z, f, acc[4 * e4 + 2]);
+                                acc[4 * e4 + 3] = fmaf(x[e4].w, f, acc[4 * e4 + 3]);
+                            }
+                        };
+                        auto load = [&](int kk, float4 (&x)[8]) {
+                            const float4 *src = reinterpret_cast<const float4 *>(
+                                                    sw.part + ((int64_t)slot_of(kk) * kRows + R) *
+                                                                  kD) +
+                                                8 * c;
+#pragma unroll
+                            for (int e4 = 0; e4 < 8; ++e4) x[e4] = __ldcg(src + e4);
+                        };
+                        if (M != -INFINITY) {
+                            int kk = k0;
+                            for (; kk + 1 <= k1; kk += 2) {
+                                float4 x0[8], x1[8];
+                                load(kk, x0);
+                                load(kk + 1, x1);
+                                add(x0, exp2f(mlrow(kk).x - M));
+                                add(x1, exp2f(mlrow(kk + 1).x - M));
+                            }
+                            if (kk <= k1) {
+                                float4 x0[8];
+                                load(kk, x0);
+                                add(x0, exp2f(mlrow(kk).x - M));
+                            }
+                        }
+                        if (valid) {
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4)
+                                orow[4 * c + q4] = make_uint4(
+                                    (uint32_t)f32_to_bf16_rn(acc[8 * q4] * inv) |
+                                        ((uint32_t)f32_to_bf16_rn(acc[8 * q4 + 1] * inv) << 16),
+                                    (uint32_t)f32_to_bf16_rn(acc[8 * q4 + 2] * inv) |
+                                        ((uint32_t)f32_to_bf16_rn(acc[8 * q4 + 3] * inv) << 16),
+                                    (uint32_t)f32_to_bf16_rn(acc[8 * q4 + 4] * inv) |
+                                        ((uint32_t)f32_to_bf16_rn(acc[8 * q4 + 5] * inv) << 16),
+                                    (uint32_t)f32_to_bf16_rn(acc[8 * q4 + 6] * inv) |
+                                        ((uint32_t)f32_to_bf16_rn(acc[8 * q4 + 7] * inv) << 16));
+                        }
                     }
                 }
             }
+            fence_before();
+            ptx::mbar_arrive(&bars.o_free);
+            ++sn;
+            if (nx.d < 0) break;
+            sg = nx;
+            it = itn;
         }
     } else if (warp == 8) {
         // ======================= MMA issue =======================
         // tensor-core order per K/V tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so
         // each softmax warpgroup works while the other tile's products run
         const uint32_t id_qk = idesc(false), id_pv = idesc(true);
-        auto zero_tail = [&](int j, int st) {
+        auto zero_tail = [&](int j, int st, int len) {
             // V rows at or past the context end: zero them (the weights there are 0,
             // and 0 x NaN would still poison the sum)
             const int t0 = j * kN;
@@ -416,50 +668,64 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             commit(&bars.s_full[w]);
         };
-        auto issue_pv = [&](int w, int j, int st) {
+        // jj: tile index within the segment (0: O starts afresh)
+        auto issue_pv = [&](int w, int jj, int st) {
 #pragma unroll
             for (int kk = 0; kk < kN / 16; ++kk) {
                 // V: 16 token rows per k-step; N = 128 dims across the two slices
                 const uint64_t vd = sdesc(sV(st) + (uint32_t)(kk * 16 * 128), kSlice, 1024);
                 mma_ts(tm + kColO + w * 128, tm + w * 128 + 16 * kk, vd, id_pv,
-                       (j > 0 || kk > 0) ? 1u : 0u);
+                       (jj > 0 || kk > 0) ? 1u : 0u);
                 mma_ts(tm + kColO + w * 128, tm + w * 128 + 16 * kk + 8, vd, id_pv, 1u);
             }
             commit(&bars.pv_done[w]);
         };
-        bool ok = warp_wait(&bars.q_full, 0, abort_flag) &&
-                  warp_wait(&bars.kv_full[0], 0, abort_flag);
-        if (ok) {
-            zero_tail(0, 0);
+        bool ok = true;
+        int jt = 0, sn = 0;
+        for (Seg sg = seg0; sg.d >= 0 && ok; sg = next_seg(sg), ++sn) {
+            const int len = a.ctx_lens[item_of(a, sg.d, X, QT).b];
+            const int nt = sg.je - sg.jb;
+            if (!(ok = warp_wait(&bars.q_full, sn & 1, abort_flag) &&
+                       warp_wait(&bars.kv_full[jt % kStages], (jt / kStages) & 1, abort_flag)))
+                break;
+            // the new S overwrites the columns the previous segment's last P V read P
+            // from: that segment's products are complete first
+            if (sn > 0 && !(ok = warp_wait(&bars.o_final, (sn - 1) & 1, abort_flag))) break;
+            zero_tail(sg.jb, jt % kStages, len);
             fence_after();
-            issue_s(0, 0);
-            issue_s(1, 0);
-        }
-        for (int j = 0; j < n_kt && ok; ++j) {
-            const int st = j % kStages, st1 = (j + 1) % kStages;
-            const bool more = j + 1 < n_kt;
-            // ---- tile A
-            if (!(ok = warp_wait(&bars.p_full[0], j & 1, abort_flag))) break;
-            fence_after();
-            issue_pv(0, j, st);
-            if (more) {
-                if (!(ok = warp_wait(&bars.kv_full[st1], ((j + 1) / kStages) & 1, abort_flag))) break;
-                zero_tail(j + 1, st1);
-                // S_A(j+1) overwrites the columns PV_A(j) reads its P from
-                if (!(ok = warp_wait(&bars.pv_done[0], j & 1, abort_flag))) break;
+            issue_s(0, jt % kStages);
+            issue_s(1, jt % kStages);
+            for (int jj = 0; jj < nt && ok; ++jj, ++jt) {
+                const int st = jt % kStages, st1 = (jt + 1) % kStages;
+                const bool more = jj + 1 < nt;
+                // ---- tile A
+                if (!(ok = warp_wait(&bars.p_full[0], jt & 1, abort_flag))) break;
+                if (jj == 0 && sn > 0 &&   // O of the previous segment is read out
+                    !(ok = warp_wait(&bars.o_free, (sn - 1) & 1, abort_flag)))
+                    break;
                 fence_after();
-                issue_s(0, st1);
-            }
-            // ---- tile B
-            if (!(ok = warp_wait(&bars.p_full[1], j & 1, abort_flag))) break;
-            fence_after();
-            issue_pv(1, j, st);
-            commit(&bars.kv_empty[st]);
-            if (!more) commit(&bars.o_final);
-            if (more) {
-                if (!(ok = warp_wait(&bars.pv_done[1], j & 1, abort_flag))) break;
+                issue_pv(0, jj, st);
+                if (more) {
+                    if (!(ok = warp_wait(&bars.kv_full[st1], ((jt + 1) / kStages) & 1,
+                                         abort_flag)))
+                        break;
+                    zero_tail(sg.jb + jj + 1, st1, len);
+                    // S_A(j+1) overwrites the columns PV_A(j) reads its P from
+                    if (!(ok = warp_wait(&bars.pv_done[0], jt & 1, abort_flag))) break;
+                    fence_after();
+                    issue_s(0, st1);
+                }
+                // ---- tile B
+                if (!(ok = warp_wait(&bars.p_full[1], jt & 1, abort_flag))) break;
                 fence_after();
-                issue_s(1, st1);
+                issue_pv(1, jj, st);
+                commit(&bars.kv_empty[st]);
+                if (!more) commit(&bars.o_final);
+                if (more) {
+                    if (!(ok = warp_wait(&bars.pv_done[1], jt & 1, abort_flag))) break;
+                    fence_after();
+                    issue_s(1, st1);
+                }
             }
         }
     } else {
@@ -467,40 +733,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         // lane pg < 8 owns 16-token page pg of every tile: it looks up the page's
         // physical block (one tile ahead, so the table read is off the critical
         // path) and issues the page's four boxes
-        const int32_t *btr = a.block_tables + (int64_t)b * a.MB;
-        auto lookup = [&](int j) -> int32_t {
-            const int t = j * kN + 16 * lane;
-            return (lane < kN / 16 && t < len) ? btr[t / a.bs] : -1;
-        };
-        int32_t next = lookup(0);
         bool ok = true;
-        for (int j = 0; j < n_kt && ok; ++j) {
-            const int st = j % kStages;
-            const int32_t blk = next;
-            if (j + 1 < n_kt) next = lookup(j + 1);
-            if (j >= kStages &&
-                !(ok = warp_wait(&bars.kv_empty[st], ((j / kStages) - 1) & 1, abort_flag)))
-                break;
-            const int t = j * kN + 16 * lane;
-            const bool in = lane < kN / 16 && t < len;
-            // pages inside the context with a valid block id are loaded; the others
-            // are not (their rows are masked, and V rows past the end zeroed)
-            const bool load = in && blk >= 0 && (int64_t)blk < a.N;
-            if (in && !load) raise_flag(a.err, PA_DEV_BAD_BLOCK);
-            const unsigned lm = __ballot_sync(0xffffffffu, load);
-            if (lane == 0)
-                ptx::mbar_arrive_expect_tx(&bars.kv_full[st], (uint32_t)__popc(lm) * 4u * 2048u);
-            __syncwarp();
-            if (load) {
-                const int off = t % a.bs;
+        int jt = 0;
+        for (Seg sg = seg0; sg.d >= 0 && ok; sg = next_seg(sg)) {
+            const Item it = item_of(a, sg.d, X, QT);
+            const int32_t *btr = a.block_tables + (int64_t)it.b * a.MB;
+            auto lookup = [&](int j) -> int32_t {
+                const int t = j * kN + 16 * lane;
+                return (lane < kN / 16 && t < it.len) ? btr[t / a.bs] : -1;
+            };
+            int32_t next = lookup(sg.jb);
+            for (int j = sg.jb; j < sg.je && ok; ++j, ++jt) {
+                const int st = jt % kStages;
+                const int32_t blk = next;
+                if (j + 1 < sg.je) next = lookup(j + 1);
+                if (jt >= kStages &&
+                    !(ok = warp_wait(&bars.kv_empty[st], ((jt / kStages) - 1) & 1, abort_flag)))
+                    break;
+                const int t = j * kN + 16 * lane;
+                const bool in = lane < kN / 16 && t < it.len;
+                // pages inside the context with a valid block id are loaded; the others
+                // are not (their rows are masked, and V rows past the end zeroed)
+                const bool load = in && blk >= 0 && (int64_t)blk < a.N;
+                if (in && !load) raise_flag(a.err, PA_DEV_BAD_BLOCK);
+                const unsigned lm = __ballot_sync(0xffffffffu, load);
+                if (lane == 0)
+                    ptx::mbar_arrive_expect_tx(&bars.kv_full[st],
+                                               (uint32_t)__popc(lm) * 4u * 2048u);
+                __syncwarp();
+                if (load) {
+                    const int off = t % a.bs;
 #pragma unroll
-                for (int sl = 0; sl < 2; ++sl) {
-                    const uint32_t dk = sK(st) + (uint32_t)(sl * kSlice + lane * 16 * 128);
-                    const uint32_t dv = sV(st) + (uint32_t)(sl * kSlice + lane * 16 * 128);
-                    ptx::tma_load_5d(gbase + (dk - base), &km, &bars.kv_full[st], 0, off, h, sl,
-                                     blk);
-                    ptx::tma_load_5d(gbase + (dv - base), &vm, &bars.kv_full[st], 0, off, h, sl,
-                                     blk);
+                    for (int sl = 0; sl < 2; ++sl) {
+                        const uint32_t dk = sK(st) + (uint32_t)(sl * kSlice + lane * 16 * 128);
+                        const uint32_t dv = sV(st) + (uint32_t)(sl * kSlice + lane * 16 * 128);
+                        ptx::tma_load_5d(gbase + (dk - base), &km, &bars.kv_full[st], 0, off,
+                                         it.h, sl, blk);
+                        ptx::tma_load_5d(gbase + (dv - base), &vm, &bars.kv_full[st], 0, off,
+                                         it.h, sl, blk);
+                    }
                 }
             }
         }
@@ -511,6 +782,93 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tm),
                      "r"(kTmemCols));
+}
+
+// Exclusive prefix sum over the 1024 threads of a CTA; *total receives the sum.
+__device__ __forceinline__ int cta_scan(int v, int *total) {
+    __shared__ int s_w[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) s_w[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int x = s_w[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        s_w[lane] = x;   // inclusive totals of warps 0..lane
+    }
+    __syncthreads();
+    const int before = warp ? s_w[warp - 1] : 0;
+    *total = s_w[31];
+    __syncthreads();
+    return before + inc - v;
+}
+
+// Balanced mode, before the attention kernel (one CTA of 1024 threads): the item
+// ranks, the tile offsets of the items left over, L, zeroed merge counters.
+__global__ void __launch_bounds__(1024) prefill_plan_kernel(const PrefillAttnArgs a,
+                                                            const StreamWs sw) {
+    constexpr int kCache = 4096;   // items whose tile counts are kept in shared memory
+    __shared__ int s_nk[kCache];
+    const int tid = threadIdx.x;
+    const int QT = kRows / a.G, X = sw.X, n_items = sw.n_items, P = sw.P;
+    int *hdr = const_cast<int *>(sw.hdr);
+    int *items = const_cast<int *>(sw.items);
+    int *pre = const_cast<int *>(sw.pre);
+    int *lrank = const_cast<int *>(sw.lrank);
+    for (int x = tid; x < n_items * 8; x += 1024) sw.cnt[x] = 0;
+    // tile count of item d, or -1 when the item has rows but a bad length
+    auto tiles = [&](int d) -> int {
+        if (d < kCache) return s_nk[d];
+        const Item it = item_of(a, d, X, QT);
+        return it.n_kt > 0 ? it.n_kt : (it.qt >= 0 ? -1 : 0);
+    };
+    for (int d = tid; d < min(n_items, kCache); d += 1024) {
+        const Item it = item_of(a, d, X, QT);
+        s_nk[d] = it.n_kt > 0 ? it.n_kt : (it.qt >= 0 ? -1 : 0);
+    }
+    __syncthreads();
+    int n = 0;
+    for (int b0 = 0; b0 < n_items; b0 += 1024) {
+        const int d = b0 + tid;
+        int t;
+        cta_scan(d < n_items && tiles(d) > 0, &t);
+        n += t;
+    }
+    const int whole = n / P * P;
+    int rank0 = 0, bad0 = 0, R = 0;
+    for (int b0 = 0; b0 < n_items; b0 += 1024) {
+        const int d = b0 + tid;
+        const int nk = d < n_items ? tiles(d) : 0;
+        int t;
+        const int rank = rank0 + cta_scan(nk > 0, &t);
+        rank0 += t;
+        const int bad = bad0 + cta_scan(nk < 0, &t);
+        bad0 += t;
+        const bool left = nk > 0 && rank >= whole;
+        const int off = R + cta_scan(left ? nk : 0, &t);
+        R += t;
+        if (nk > 0) items[rank] = d;
+        if (nk < 0) items[n + bad] = d;
+        if (left) pre[rank - whole] = off;
+        if (d < n_items) lrank[d] = left ? rank - whole : -1;
+    }
+    if (tid == 0) {
+        pre[n - whole] = R;
+        hdr[0] = whole;
+        hdr[1] = n - whole;
+        hdr[2] = R;
+        hdr[3] = R > 0 ? (R + P - 1) / P : 1;
+        hdr[4] = bad0;
+    }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tc_encode_fn() {
@@ -550,23 +908,82 @@ bool prefill_attn_tc_supported(const PrefillAttnArgs &a) {
     return a.d == kD && a.bs % 16 == 0;
 }
 
-cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs &a, int max_q_len, cudaStream_t st) {
+namespace {
+inline size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+struct StreamLayout {
+    int64_t n_items;
+    int X;
+    size_t off_items, off_pre, off_lrank, off_cnt, off_part, off_ml, total;
+};
+// header | item ranks | left-over tile offsets | left-over ranks | merge counters |
+// partial results of at most 2P parts
+StreamLayout stream_layout(int B, int Hkv, int G, int max_q_len, int sms) {
+    StreamLayout L;
+    const int QT = kRows / G;
+    L.X = (max_q_len + QT - 1) / QT;
+    L.n_items = (int64_t)B * Hkv * L.X;
+    L.off_items = 256;
+    L.off_pre = L.off_items + up256((size_t)L.n_items * 4);
+    L.off_lrank = L.off_pre + up256((size_t)(L.n_items + 1) * 4);
+    L.off_cnt = L.off_lrank + up256((size_t)L.n_items * 4);
+    L.off_part = L.off_cnt + up256((size_t)L.n_items * 8 * 4);
+    L.off_ml = L.off_part + up256((size_t)2 * sms * kRows * kD * 4);
+    L.total = L.off_ml + up256((size_t)2 * sms * kRows * 2 * 4);
+    return L;
+}
+}  // namespace
+
+size_t prefill_attn_tc_workspace_bytes(const PrefillAttnArgs &a, int max_q_len, int sms) {
+    if (!prefill_attn_tc_supported(a) || max_q_len <= 0 || a.B <= 0) return 0;
+    const StreamLayout L = stream_layout(a.B, a.Hkv, a.G, max_q_len, sms);
+    if (L.n_items + 1 > INT32_MAX) return 0;
+    return L.total;
+}
+
+cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs &a, int max_q_len, void *ws,
+                                   size_t ws_bytes, int sms, cudaStream_t st) {
     CUtensorMap km, vm;
     if (!encode_head_map(&km, a.k_cache, a.N, a.bs, a.Hkv, a.block_stride) ||
         !encode_head_map(&vm, a.v_cache, a.N, a.bs, a.Hkv, a.block_stride))
         return cudaErrorInvalidValue;
-    static bool attr_set[64] = {};
+    const size_t need = prefill_attn_tc_workspace_bytes(a, max_q_len, sms);
+    const bool stream = ws != nullptr && need > 0 && ws_bytes >= need;
+    auto kfn = stream ? prefill_attn_tc_kernel<true> : prefill_attn_tc_kernel<false>;
+    static bool attr_set[2][64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-    if (dev >= 64 || !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_attn_tc_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (dev >= 64 || !attr_set[stream][dev]) {
+        cudaError_t e =
+            cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess) return e;
-        if (dev < 64) attr_set[dev] = true;
+        if (dev < 64) attr_set[stream][dev] = true;
     }
-    const int QT = kRows / a.G;
-    dim3 grid((unsigned)((max_q_len + QT - 1) / QT), (unsigned)a.Hkv, (unsigned)a.B);
-    prefill_attn_tc_kernel<<<grid, kThreads, kSmem, st>>>(km, vm, a);
+    StreamWs sw = {};
+    if (!stream) {
+        const int QT = kRows / a.G;
+        dim3 grid((unsigned)((max_q_len + QT - 1) / QT), (unsigned)a.Hkv, (unsigned)a.B);
+        kfn<<<grid, kThreads, kSmem, st>>>(km, vm, a, sw);
+        return cudaGetLastError();
+    }
+    // balanced: plan, then whole items, one range of the left-over tiles per SM and
+    // the zero-row CTAs (cut items are merged by their last part)
+    const StreamLayout L = stream_layout(a.B, a.Hkv, a.G, max_q_len, sms);
+    char *w = static_cast<char *>(ws);
+    sw.hdr = reinterpret_cast<int *>(w);
+    sw.items = reinterpret_cast<int *>(w + L.off_items);
+    sw.pre = reinterpret_cast<int *>(w + L.off_pre);
+    sw.lrank = reinterpret_cast<int *>(w + L.off_lrank);
+    sw.cnt = reinterpret_cast<int *>(w + L.off_cnt);
+    sw.part = reinterpret_cast<float *>(w + L.off_part);
+    sw.ml = reinterpret_cast<float *>(w + L.off_ml);
+    sw.n_items = (int)L.n_items;
+    sw.X = L.X;
+    sw.P = sms;
+    prefill_plan_kernel<<<1, 1024, 0, st>>>(a, sw);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // whole + P + n_bad <= n_items + P CTAs do work; the rest return at once
+    kfn<<<(unsigned)(L.n_items + sms), kThreads, kSmem, st>>>(km, vm, a, sw);
     return cudaGetLastError();
 }
 

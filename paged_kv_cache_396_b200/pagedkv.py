@@ -38,7 +38,7 @@ EXPORTED = (
     "pe_select_evict_block_pooled", "pa_append_kv_fp8", "pa_decode_fp8",
     "pe_prefill_scores", "pe_prefill_select", "pe_prefill_pack", "pe_prefill_compress",
     "pe_evict_compact", "pe_select_evict_threshold", "pe_evict_compact_mask",
-    "pa_prefill_attention",
+    "pa_prefill_attention", "pa_prefill_attention_workspace_bytes",
 )
 
 
@@ -117,7 +117,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pe_evict_compact_mask.argtypes = [p, i32, p, p, p, i32, i32, p, p]
     lib.pa_prefill_attention.restype = i32
     lib.pa_prefill_attention.argtypes = [p, p, p, i32, p, p, i64, p, i32, p, i32, i32, i32, i32,
-                                         i32, i64, f32, p, p]
+                                         i32, i64, f32, p, p, sz, p]
+    lib.pa_prefill_attention_workspace_bytes.restype = sz
+    lib.pa_prefill_attention_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
     lib.pe_score_tokens.restype = i32
     lib.pe_score_tokens.argtypes = [p, p, p, i64, p, i32, p, i32, i32, i32, i32, i64, p, p]
     lib.pe_select_evict_block.restype = i32
@@ -663,11 +665,24 @@ def pe_evict_compact_mask(block_tables, ctx_lens, mask, block_size, err_flag, fr
 
 
 # ----------------------------------------------------------------------------- chunked prefill
+def pa_prefill_attention_workspace_bytes(B, Hq, Hkv, d, bs, max_q_len) -> int:
+    return int(load().pa_prefill_attention_workspace_bytes(B, Hq, Hkv, d, bs, max_q_len))
+
+
+def alloc_prefill_workspace(B, Hq, Hkv, d, bs, max_q_len, device=None):
+    """Convenience: a device byte tensor for pa_prefill_attention's balanced mode
+    (None when that mode does not apply to these sizes)."""
+    n = pa_prefill_attention_workspace_bytes(B, Hq, Hkv, d, bs, max_q_len)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
 def pa_prefill_attention(out, q, cu_q, max_q_len, k_cache, v_cache, block_tables, ctx_lens,
-                         scale, err_flag, stream=None):
+                         scale, err_flag, workspace=None, stream=None):
     """Multi-query paged attention: the q_len_b = cu_q[b+1]-cu_q[b] query rows of
     sequence b are its last q_len_b cached tokens and attend causally.
-    q, out [Tq, Hq, d] bf16 contiguous; cu_q [B+1] int32; ctx_lens [B] int32."""
+    q, out [Tq, Hq, d] bf16 contiguous; cu_q [B+1] int32; ctx_lens [B] int32.
+    workspace (optional, uint8 device tensor, alloc_prefill_workspace): balances the
+    work over the SMs."""
     _want(out, torch.bfloat16, "out")
     _want(q, torch.bfloat16, "q")
     _want(cu_q, torch.int32, "cu_q")
@@ -676,6 +691,8 @@ def pa_prefill_attention(out, q, cu_q, max_q_len, k_cache, v_cache, block_tables
     _want(err_flag, torch.int32, "err_flag")
     _want(k_cache, torch.bfloat16, "k_cache")
     _want(v_cache, torch.bfloat16, "v_cache")
+    if workspace is not None:
+        _want(workspace, torch.uint8, "workspace")
     N, bs, Hkv, d, stride = _pool_geometry(k_cache, "k_cache")
     _same_pool(k_cache, v_cache)
     if q.dim() != 3 or q.shape != out.shape or not (q.is_contiguous() and out.is_contiguous()):
@@ -690,4 +707,5 @@ def pa_prefill_attention(out, q, cu_q, max_q_len, k_cache, v_cache, block_tables
     _check("pa_prefill_attention", load().pa_prefill_attention(
         _ptr(out), _ptr(q), _ptr(cu_q.contiguous()), int(max_q_len), _ptr(k_cache),
         _ptr(v_cache), stride, _ptr(bt), bt.shape[1], _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d,
-        bs, N, float(scale), _ptr(err_flag), _stream(stream)))
+        bs, N, float(scale), _ptr(err_flag), _ptr(workspace) if workspace is not None else None,
+        workspace.numel() if workspace is not None else 0, _stream(stream)))

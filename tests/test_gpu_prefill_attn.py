@@ -3,7 +3,9 @@ C ABI against the fp64 oracle: |err| <= 2e-3 + 1e-2 |ref| on every output of
 medium cases (several 64-row query tiles, 64-token K/V tiles, ragged tails,
 GQA group sizes 1..16, d 64 and 128, block sizes 12, 16 and 256), the
 append-then-attend sequence, mixed chunk + decode batches, invalid lengths,
-and sampled rows of a full-size 512-token chunk at 8K context."""
+and sampled rows of a full-size 512-token chunk at 8K context; each in the
+one-CTA-per-query-tile mode and in the balanced mode (workspace given: tile ranges
+cut across SMs, partial results merged), which bench.py times."""
 import numpy as np
 import pytest
 import torch
@@ -36,14 +38,25 @@ def _case(lens, qlens, Hq, Hkv, d, bs, seed, spare=4):
                 d=d, bs=bs, N=N, qlens=list(qlens))
 
 
-def _run(c, err_expected=0):
+def _workspace(c, balanced):
+    """The balanced mode's workspace, filled with 0xff (stale scratch), or None."""
+    if not balanced:
+        return None
+    ws = pk.alloc_prefill_workspace(len(c["lens"]), c["Hq"], c["Hkv"], c["d"], c["bs"],
+                                    max(c["qlens"] + [0]), "cuda")
+    if ws is not None:
+        ws.fill_(0xFF)
+    return ws
+
+
+def _run(c, err_expected=0, balanced=False):
     dev = "cuda"
     out = torch.full(c["q"].shape, float("nan"), dtype=torch.bfloat16, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     pk.pa_prefill_attention(out, c["q"].to(dev), torch.as_tensor(c["cu"]).to(dev),
                             max(c["qlens"] + [0]), c["k"].to(dev), c["v"].to(dev),
                             torch.as_tensor(c["bt"]).to(dev), torch.as_tensor(c["lens"]).to(dev),
-                            c["d"] ** -0.5, err)
+                            c["d"] ** -0.5, err, workspace=_workspace(c, balanced))
     torch.cuda.synchronize()
     assert err.item() == err_expected
     return out
@@ -67,12 +80,30 @@ CASES = {
 }
 
 
+@pytest.mark.parametrize("balanced", [False, True])
 @pytest.mark.parametrize("key", list(CASES))
-def test_prefill_attention_medium(key):
+def test_prefill_attention_medium(key, balanced):
     lens, qlens, Hq, Hkv, d, bs = CASES[key]
     c = _case(lens, qlens, Hq, Hkv, d, bs, seed=100 + list(CASES).index(key))
-    out = _run(c)
+    out = _run(c, balanced=balanced)
     assert_attention_close(out, _oracle(c), key)
+
+
+@pytest.mark.parametrize("qlens", [[64], [256, 1], [512, 0, 512]])
+def test_balanced_mode_with_few_long_items(qlens):
+    """Few query tiles over long contexts: every tile range is cut across many SMs
+    (one item in many parts), so the merge combines many partial results."""
+    lens = [6000 + 37 * b for b in range(len(qlens))]
+    c = _case(lens, qlens, 32, 8, 128, 16, seed=21 + len(qlens))
+    out = _run(c, balanced=True)
+    assert_attention_close(out, _oracle(c), f"balanced, q lens {qlens}")
+
+
+def test_balanced_mode_is_deterministic():
+    c = _case([3000, 800], [512, 300], 32, 8, 128, 16, seed=31)
+    a = _run(c, balanced=True)
+    b = _run(c, balanced=True)
+    assert torch.equal(a, b)
 
 
 def test_append_chunk_then_attend():
@@ -121,23 +152,26 @@ def test_single_query_rows_match_decode_kernel_results():
     assert np.array_equal(ref, ref_dec)
 
 
-def test_invalid_query_length_gives_zero_rows_and_flag():
-    c = _case([50, 10], [20, 11], 8, 2, 64, 16, seed=12)
-    out = _run(c, err_expected=pk.PA_DEV_BAD_LEN)
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("balanced", [False, True])
+def test_invalid_query_length_gives_zero_rows_and_flag(d, balanced):
+    c = _case([50, 10], [20, 11], 8, 2, d, 16, seed=12)
+    out = _run(c, err_expected=pk.PA_DEV_BAD_LEN, balanced=balanced)
     ref = _oracle(c)
     assert not ref[20:].any()
     assert (out[20:].float() == 0).all()
     assert_attention_close(out[:20], ref[:20], "valid sequence next to an invalid one")
 
 
-def test_full_size_chunk_sampled_rows():
+@pytest.mark.parametrize("balanced", [False, True])
+def test_full_size_chunk_sampled_rows(balanced):
     """The last 512-token chunk of an 8192-token prompt, Llama-3-8B shape, 4
     sequences: sampled query rows against the decode oracle at the row's own
     position (causality makes query i of the chunk a decode over p + 1 tokens)."""
     Hq, Hkv, d, bs = 32, 8, 128, 16
     lens = [8192] * 4
     c = _case(lens, [512] * 4, Hq, Hkv, d, bs, seed=13)
-    out = _run(c).cpu()
+    out = _run(c, balanced=balanced).cpu()
     rng = np.random.default_rng(14)
     stride = bs * Hkv * d
     kb, vb = W.bits(c["k"]).ravel(), W.bits(c["v"]).ravel()
