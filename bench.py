@@ -42,6 +42,10 @@ from paged_kv_cache_396_b200 import workloads as W  # noqa: E402
 METRIC = "paged decode-attention HBM GB/s (% of B200 peak) and decode tokens/s at 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ["decode_simple.cu", "decode_tc.cu", "kernels.h", "common.cuh", "ptx.cuh"]
+# sources of the other workloads' dominant kernels (their recorded traffic is keyed by them)
+PREFILL_SOURCES = {"p1": ["prefill.cu", "prefill.h", "kernels.h", "common.cuh"],
+                   "p2": ["prefill_attn_tc.cu", "prefill_attn.h", "kernels.h", "common.cuh",
+                          "ptx.cuh"]}
 
 
 def parse():
@@ -96,22 +100,26 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def decode_source_hash() -> str:
+def source_hash(files) -> str:
     h = hashlib.sha256()
-    for f in DECODE_SOURCES:
+    for f in files:
         p = os.path.join(ROOT, "paged_kv_cache_396_b200", "csrc", f)
         if os.path.exists(p):
             h.update(open(p, "rb").read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """dram bytes per decode launch from the committed ncu summary, if it was
-    taken on the current decode sources (else None)."""
-    p = os.path.join(ROOT, "profiles", "decode_traffic.txt")
+def decode_source_hash() -> str:
+    return source_hash(DECODE_SOURCES)
+
+
+def recorded_traffic(workload: str, record="decode_traffic.txt", sources=None):
+    """dram bytes per launch of the dominant kernel from a committed ncu summary
+    (profiles/<record>), if it was taken on the current sources (else None)."""
+    p = os.path.join(ROOT, "profiles", record)
     if not os.path.exists(p):
         return None
-    want = decode_source_hash()
+    want = source_hash(sources if sources is not None else DECODE_SOURCES)
     for line in open(p):
         kv = dict(x.split("=", 1) for x in line.split() if "=" in x)
         if kv.get("workload") == workload and kv.get("sources") == want:
@@ -683,7 +691,9 @@ def run_prefill(args, device, world, rank):
                        "l2": "prompt rows (1 GiB) larger than L2 every step (no flush needed)"},
             "roofline": {"bound": "hbm", "kernel": "pe_prefill_scores", "achieved": achieved,
                          "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak,
+                         "traffic": recorded_traffic("p1", "prefill_traffic.txt",
+                                                     PREFILL_SOURCES["p1"]),
                          "algorithmic_bytes_per_launch": score_bytes,
                          "avg_launch_us": score_s * 1e6},
             "kernels_us": {"pe_prefill_scores": score_s * 1e6,
@@ -848,7 +858,9 @@ def run_chunked(args, device, world, rank):
                        "l2": "flushed (256 MB write) before every timed step"},
             "roofline": {"bound": "tensor", "kernel": "pa_prefill_attention",
                          "achieved": achieved, "peak": peak_t, "peak_source": "measured burst",
-                         "unit": "TFLOP/s", "frac": achieved / peak_t, "traffic": None,
+                         "unit": "TFLOP/s", "frac": achieved / peak_t,
+                         "traffic": recorded_traffic("p2", "prefill_traffic.txt",
+                                                     PREFILL_SOURCES["p2"]),
                          "algorithmic_flops_per_launch": flops, "avg_launch_us": attn_s * 1e6},
             "cpu_baseline": cpu,
             "e2e": {"value": world * Tq / (e2e_ms / 1000.0), "unit": "chunk tokens/s",
