@@ -100,12 +100,31 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """The source without // comments and blank lines (whitespace collapsed), so a
+    comment edit does not invalidate a recorded capture; a // inside a string
+    literal is kept."""
+    out = []
+    for line in text.splitlines():
+        q, cut = False, len(line)
+        for i, ch in enumerate(line):
+            if ch == '"' and (i == 0 or line[i - 1] != "\\"):
+                q = not q
+            elif not q and line.startswith("//", i):
+                cut = i
+                break
+        code = " ".join(line[:cut].split())
+        if code:
+            out.append(code)
+    return "\n".join(out)
+
+
 def source_hash(files) -> str:
     h = hashlib.sha256()
     for f in files:
         p = os.path.join(ROOT, "paged_kv_cache_396_b200", "csrc", f)
         if os.path.exists(p):
-            h.update(open(p, "rb").read())
+            h.update(_code_only(open(p, encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

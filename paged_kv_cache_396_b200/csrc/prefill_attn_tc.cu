@@ -6,23 +6,26 @@
 // tokens of a sequence are its last q_len cached tokens and attend causally.
 // Used for d = 128 and block sizes that are multiples of 16.
 //
-// One CTA = one (sequence, kv head, 256 query rows) as two tiles of 128 rows
+// An item = one (sequence, kv head, 256 query rows) as two tiles of 128 rows
 // (the MMA M); rows are (query token, head of the GQA group) pairs, so each K/V
 // tile serves all G heads of both Q tiles.  Warp roles (320 threads):
 //   warps 0-3, 4-7  softmax, one warpgroup per Q tile: thread r owns row r of its
-//              tile = TMEM lane r.  Loads its Q row into shared memory once; per
-//              128-token K/V tile reads its S row from TMEM, masks (causal),
-//              keeps the running max (lazy: O is rescaled only when the max grows
-//              by more than 2^8), writes P = hi + lo (two bf16 parts) back over the
-//              S columns, and at the end normalises O.  The two warpgroups work
-//              half a step apart, so one computes softmax while the tensor core
-//              runs the other tile's products.
-//   warp 8     MMA issue (one lane), in the order PV_A(j), S_A(j+1), PV_B(j),
-//              S_B(j+1): S = Q K^T (SS, both K-major) into the tile's S/P
-//              columns, O += P_hi V + P_lo V (A from TMEM, V MN-major) into its O
-//              columns; completion through tcgen05.commit.  Its lanes also zero
-//              the V rows past the context end in a tile that holds them (stale or
-//              NaN slots must not meet a zero weight).
+//              tile = TMEM lane r.  Loads its Q row into shared memory per item;
+//              per 128-token K/V tile reads its 128 logits from TMEM (four loads,
+//              one wait), masks (causal, diagonal tiles only), keeps the running
+//              max (lazy: O is rescaled only when the max grows by more than 2^8),
+//              writes P = hi + lo (two bf16 parts) back over the S columns, and at
+//              the end normalises O (or, for a cut item, writes its partial and the
+//              last part merges).  The two warpgroups work half a step apart, so
+//              one computes softmax while the tensor core runs the other tile's
+//              products.
+//   warp 8     MMA issue (warp-uniform operands, elect.sync picks the issuing
+//              lane), in the order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): S = Q K^T
+//              (SS, both K-major) into the tile's S/P columns, O += P_hi V + P_lo V
+//              (A from TMEM, V MN-major) into its O columns; completion through
+//              tcgen05.commit.  Its lanes also zero the V rows past the context end
+//              in a tile that holds them (stale or NaN slots must not meet a zero
+//              weight).
 //   warp 9     TMA producer: lane p < 8 owns 16-token page p of every tile, looks
 //              up its physical block one tile ahead and issues four boxes (K and V,
 //              two 64-element slices each); two stages.
