@@ -445,6 +445,18 @@ int pa_prefill_attention(uint16_t *out, const uint16_t *q, const int32_t *cu_q, 
                          int64_t num_blocks, float scale, int32_t *err_flag, void *workspace,
                          size_t workspace_bytes, void *stream);
 
+/* ============================================================================
+ * Self-test of the device failure path (no counterpart in the pages).
+ * Every pipeline wait in these kernels is bounded: after ~2 s of device time it
+ * gives up, the kernel sets PA_DEV_TIMEOUT in err_flag and returns, and the CUDA
+ * context stays usable.  This call launches one CTA whose wait (the same bounded
+ * mbarrier wait the decode pipeline uses) is on a phase nothing completes, so it
+ * takes that path: *err_flag (device int32, caller-zeroed) gets PA_DEV_TIMEOUT
+ * after ~2 s.  No fault, trap or hang is involved.  Returns PA_OK or a PA_ERR_*
+ * code (PA_ERR_NULL for a NULL flag).
+ * ==========================================================================*/
+int pa_selftest_wait_timeout(int32_t *err_flag, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -10,6 +10,7 @@
 #include "kernels.h"
 #include "prefill.h"
 #include "prefill_attn.h"
+#include "selftest.h"
 #include "pagedkv.h"
 
 namespace {
@@ -625,4 +626,11 @@ int pa_prefill_attention(uint16_t *out, const uint16_t *q, const int32_t *cu_q, 
     return finish(pkv::prefill_attn_tc_supported(a)
                       ? pkv::launch_prefill_attn_tc(a, max_q_len, workspace, workspace_bytes, sms, st)
                       : pkv::launch_prefill_attn(a, max_q_len, st));
+}
+
+int pa_selftest_wait_timeout(int32_t *err_flag, void *stream) {
+    if (!err_flag) return PA_ERR_NULL;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    return finish(pkv::launch_selftest_wait_timeout(err_flag, static_cast<cudaStream_t>(stream)));
 }

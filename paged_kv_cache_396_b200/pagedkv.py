@@ -38,7 +38,7 @@ EXPORTED = (
     "pe_select_evict_block_pooled", "pa_append_kv_fp8", "pa_decode_fp8",
     "pe_prefill_scores", "pe_prefill_select", "pe_prefill_pack", "pe_prefill_compress",
     "pe_evict_compact", "pe_select_evict_threshold", "pe_evict_compact_mask",
-    "pa_prefill_attention", "pa_prefill_attention_workspace_bytes",
+    "pa_prefill_attention", "pa_prefill_attention_workspace_bytes", "pa_selftest_wait_timeout",
 )
 
 
@@ -119,6 +119,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_prefill_attention.argtypes = [p, p, p, i32, p, p, i64, p, i32, p, i32, i32, i32, i32,
                                          i32, i64, f32, p, p, sz, p]
     lib.pa_prefill_attention_workspace_bytes.restype = sz
+    lib.pa_selftest_wait_timeout.restype = i32
+    lib.pa_selftest_wait_timeout.argtypes = [p, p]
     lib.pa_prefill_attention_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
     lib.pe_score_tokens.restype = i32
     lib.pe_score_tokens.argtypes = [p, p, p, i64, p, i32, p, i32, i32, i32, i32, i64, p, p]
@@ -709,3 +711,13 @@ def pa_prefill_attention(out, q, cu_q, max_q_len, k_cache, v_cache, block_tables
         _ptr(v_cache), stride, _ptr(bt), bt.shape[1], _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d,
         bs, N, float(scale), _ptr(err_flag), _ptr(workspace) if workspace is not None else None,
         workspace.numel() if workspace is not None else 0, _stream(stream)))
+
+
+# ----------------------------------------------------------------------------- self-test
+def pa_selftest_wait_timeout(err_flag, stream=None):
+    """Runs the kernels' bounded wait on a phase nothing completes: after ~2 s the
+    device sets PA_DEV_TIMEOUT in err_flag ([1] int32, caller-zeroed) and the kernel
+    returns; the context stays usable."""
+    _want(err_flag, torch.int32, "err_flag")
+    _check("pa_selftest_wait_timeout",
+           load().pa_selftest_wait_timeout(_ptr(err_flag), _stream(stream)))
