@@ -358,9 +358,8 @@ __device__ __forceinline__ void load_q_bf16(const Args &a, int b, int h, int g, 
 
 // Low bf16 part of the pair (x, y) whose high parts are packed in `hi`:
 // bf16(x - hi.x), bf16(y - hi.y); the differences are exact in fp32.
-// 2^x on the MUFU pipe (ex2.approx.ftz: relative error ~2^-22, far inside the fp16
-// weights it feeds; 2^-inf = 0).  The INT8 and FP8 consumers, bound by their
-// instruction stream, use it for the softmax weights.
+// 2^x on the MUFU pipe (ex2.approx.ftz: relative error ~2^-22, far inside the bf16 /
+// fp16 weights it feeds; 2^-inf = 0), for the consumers' softmax weights.
 __device__ __forceinline__ float ex2_fast(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -461,9 +460,9 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
             mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
             const float mn = fmaxf(m, mx);
             const float mu = mn == -INFINITY ? 0.f : mn;
-            const float alpha = exp2f(m - mu);
-            const float p0 = exp2f(x0 - mu), p1 = exp2f(x1 - mu);
-            const float p2 = exp2f(x2 - mu), p3 = exp2f(x3 - mu);
+            const float alpha = ex2_fast(m - mu);
+            const float p0 = ex2_fast(x0 - mu), p1 = ex2_fast(x1 - mu);
+            const float p2 = ex2_fast(x2 - mu), p3 = ex2_fast(x3 - mu);
             l = l * alpha + ((p0 + p1) + (p2 + p3));
             m = mn;
             // P = hi + lo, both bf16: p - hi is exact in fp32 and lo carries the 8 bits
@@ -484,9 +483,9 @@ __device__ __forceinline__ void consumer(const Args &a, uint8_t *stages, StageMe
                 my = fmaxf(my, __shfl_xor_sync(kFull, my, 2));
                 const float mnb = fmaxf(mb, my);
                 const float mub = mnb == -INFINITY ? 0.f : mnb;
-                alphab = exp2f(mb - mub);
-                const float q0 = exp2f(y0 - mub), q1 = exp2f(y1 - mub);
-                const float q2 = exp2f(y2 - mub), q3 = exp2f(y3 - mub);
+                alphab = ex2_fast(mb - mub);
+                const float q0 = ex2_fast(y0 - mub), q1 = ex2_fast(y1 - mub);
+                const float q2 = ex2_fast(y2 - mub), q3 = ex2_fast(y3 - mub);
                 lb = lb * alphab + ((q0 + q1) + (q2 + q3));
                 mb = mnb;
                 pa1 = ptx::pack_bf16(q0, q1);
