@@ -19,7 +19,8 @@
  * Conventions shared by every entry point
  *   - All data pointers are DEVICE pointers owned by the caller; the library
  *     allocates nothing and keeps no state between calls except what the
- *     caller passes in (the decode workspace).
+ *     caller passes in (the decode workspace, the chunked-prefill workspace)
+ *     and the one file-scope scratch array of pa_decode_static_scratch.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *     legacy default stream) and returns after enqueueing.
  *   - Return value: PA_OK (0) when the work was enqueued; a negative PA_ERR_*
