@@ -104,12 +104,15 @@ def test_medium_workloads(key):
 
 
 @pytest.mark.parametrize("num_splits", [1, 2, 3, 8, 0, 96])
-@pytest.mark.parametrize("kv", ["bf16", "bf16-d64", "int8", "fp8"])
+@pytest.mark.parametrize("kv", ["bf16", "bf16-d64", "bf16-g16", "int8", "fp8"])
 def test_split_count_invariance(num_splits, kv):
     """num_splits = 96 cuts the 2000-token sequence into more than 32 partitions, the
-    range where the merge splits the partials across the CTA's warps."""
-    base = {"bf16": C["c3"], "bf16-d64": C["c2"]}.get(kv, C["c5"])
+    range where the merge splits the partials across the CTA's warps; with Hkv = 4
+    (bf16-g16) each partition also leaves two partials per kv head."""
+    base = {"bf16": C["c3"], "bf16-d64": C["c2"], "bf16-g16": C["c3"]}.get(kv, C["c5"])
     cfg = W.scaled(base, key="split", layers=1, batch=3, old_lens=(2000, 700, 45), score=False)
+    if kv == "bf16-g16":
+        cfg = W.scaled(cfg, hq=64, hkv=4)
     if kv == "fp8":
         cfg = W.scaled(cfg, int8=False, fp8=True)
     wl = W.generate(cfg, "cpu")
