@@ -1,0 +1,45 @@
+"""The roofline numerators bench.py reports, pinned by counting: the chunked-prefill
+FLOPs against the closed form of the causal count, and the decode's algorithmic
+bytes against the marginal cost of one more cached token."""
+import dataclasses
+
+import numpy as np
+
+import bench
+from paged_kv_cache_396_b200 import workloads as W
+
+
+def test_chunk_flops_is_the_causal_count():
+    cfg = W.CHUNKED["p2"]
+    # query i of the chunk sees ctx - chunk + i + 1 tokens; QK^T and PV are 2 d flops
+    # each per (row, token, head)
+    n, c = cfg.ctx_len, cfg.chunk
+    seen = c * (n - c + 1) + c * (c - 1) // 2
+    assert bench.chunk_flops(cfg) == 4 * cfg.head_dim * cfg.hq * cfg.batch * seen
+    # brute force on a small chunk
+    small = dataclasses.replace(cfg, ctx_len=40, chunk=7, batch=2)
+    brute = sum(4 * small.head_dim * small.hq * (40 - 7 + i + 1) for i in range(7)) * 2
+    assert bench.chunk_flops(small) == brute
+
+
+def test_decode_bytes_count_each_cached_token_once():
+    for key, elt, scales in (("c3", 2, 0), ("c5", 1, 8)):
+        cfg = W.CONFIGS[key]
+        lens = np.array([100, 17, 16], np.int64)
+        base = bench.decode_algorithmic_bytes(dataclasses.replace(cfg, batch=3), lens, 0)
+        for b in range(3):
+            more = lens.copy()
+            more[b] += 1
+            grown = bench.decode_algorithmic_bytes(dataclasses.replace(cfg, batch=3), more, 0)
+            new_block = 4 if lens[b] % cfg.block_size == 0 else 0
+            per_token = cfg.hkv * cfg.head_dim * 2 * elt + cfg.hkv * scales
+            assert grown - base == per_token + new_block, (key, b)
+
+
+def test_decode_bytes_include_partials_both_ways():
+    cfg = dataclasses.replace(W.CONFIGS["c3"], batch=2)
+    lens = np.array([500, 300], np.int64)
+    a = bench.decode_algorithmic_bytes(cfg, lens, 0)
+    b = bench.decode_algorithmic_bytes(cfg, lens, 3)
+    # three partition slots of Hq rows: (d + 2) fp32 written and read back
+    assert b - a == 2 * 3 * cfg.hq * (cfg.head_dim + 2) * 4
