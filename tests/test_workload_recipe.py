@@ -18,7 +18,10 @@ def test_config_shapes_and_seeds():
     assert C["c3"].old_len_range == (512, 8192) and C["c3"].outlier_frac == 0.01
     assert C["c4"].block_size == 256 and C["c4"].old_lens == (131072,) * 4 and not C["c4"].append
     assert C["c5"].int8 and C["c5"].hq == 64 and C["c5"].old_lens == (4096,) * 128
-    p2 = W.CHUNKED["p2"]
+    p1, p2 = W.PREFILL["p1"], W.CHUNKED["p2"]
+    assert (p1.seed, p2.seed) == (401, 402)
+    assert p1.batch == 32 and set(p1.prompt_lens) == {8192} and p1.budget == 1024
+    assert (p1.hkv, p1.head_dim, p1.block_size) == (8, 128, 16)
     assert (p2.batch, p2.ctx_len, p2.chunk, p2.hq, p2.hkv, p2.head_dim) == (4, 8192, 512, 32, 8, 128)
 
 
