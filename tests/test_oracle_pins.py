@@ -484,6 +484,42 @@ def test_int8_append_matches_quantiser_and_slots():
             assert np.array_equal(ks2[slots[b, i]], cs[b, i])
 
 
+
+def test_int8_score_equals_bf16_score_when_quantisation_is_exact():
+    """Rows of integers in [-127, 127] whose amax is 127, times a power of two per row,
+    quantise exactly (scale = that power of two, codes = the integers).  The score over
+    the dequantised INT8 pools must then equal the bf16 score of the same values, and
+    the numpy norm ratio; K and V rows carry different scales so that a scale taken from
+    the wrong (token, head) row or from the other pool changes the result."""
+    rng = np.random.default_rng(19)
+    c = rand_case(19, lens=(5, 11, 16), d=16)
+    N, bs, Hkv, d = c["N"], c["bs"], c["Hkv"], c["d"]
+
+    def exact_rows():
+        ints = rng.integers(-127, 128, (N, bs, Hkv, d)).astype(np.float64)
+        ints[..., 0] = np.where(rng.random((N, bs, Hkv)) < 0.5, 127.0, -127.0)
+        return ints * 2.0 ** rng.integers(-6, 3, (N, bs, Hkv, 1))
+
+    kx, vx = exact_rows(), exact_rows()
+    kb, vb = bf16_bits(kx), bf16_bits(vx)
+    assert np.array_equal(bf16_vals(kb), kx) and np.array_equal(bf16_vals(vb), vx)
+    kq, ks = oracle.quantize_int8(kb)
+    vq, vs = oracle.quantize_int8(vb)
+    assert np.array_equal(ks[..., None].astype(np.float64) * kq, kx)
+    stride = bs * Hkv * d
+    s8 = oracle.score_tokens_int8(kq.ravel(), vq.ravel(), ks.ravel(), vs.ravel(), stride, c["bt"],
+                                  c["lens"], Hkv, d, bs)
+    s16 = oracle.score_tokens(kb.ravel(), vb.ravel(), stride, c["bt"], c["lens"], Hkv, d, bs)
+    for b in range(c["B"]):
+        n = int(c["lens"][b])
+        np.testing.assert_array_equal(s8[b, :n], s16[b, :n])
+        assert np.isnan(s8[b, n:]).all()
+        ids = c["bt"][b, : -(-n // bs)]
+        K, V = kx[ids].reshape(-1, Hkv, d)[:n], vx[ids].reshape(-1, Hkv, d)[:n]
+        ref = np.linalg.norm(V, axis=-1) / np.linalg.norm(K, axis=-1)
+        np.testing.assert_allclose(s8[b, :n], ref, rtol=1e-13)
+
+
 # ------------------------------------------------------------------ fp8 (e4m3)
 def test_e4m3_golden_codes():
     rows = []
@@ -538,6 +574,34 @@ def test_fp8_decode_equals_sdpa_on_decoded_values():
         o = torch.nn.functional.scaled_dot_product_attention(
             torch.from_numpy(q[b]).unsqueeze(1), Kt, Vt, scale=1 / math.sqrt(d))[:, 0].numpy()
         np.testing.assert_allclose(out[b], o, rtol=1e-12, atol=1e-12)
+
+
+
+def test_fp8_append_matches_torch_cast_and_slots():
+    """The FP8 append stores torch's e4m3 cast of each new row at the slot the block
+    table gives, and touches no other byte of either pool."""
+    rng = np.random.default_rng(34)
+    B, Hkv, d, bs, N = 2, 2, 16, 4, 10
+    bt = np.array([[3, 7, -1], [1, 0, 9]], np.int32)
+    kc = np.zeros(N * bs * Hkv * d, np.uint8)
+    vc = np.zeros_like(kc)
+    kn = bf16_bits(rng.standard_normal((B, 3, Hkv, d)) * 20)
+    vn = bf16_bits(rng.standard_normal((B, 3, Hkv, d)) * 0.05)
+    pos = np.array([2, 7], np.int32)
+    slots = oracle.append_kv_fp8(kn, vn, kc, vc, bs * Hkv * d, bt, pos, bs)
+    assert slots.tolist() == [[14, 15, 28], [3, 36, 37]]
+
+    def cast(bits):
+        return torch.as_tensor(bf16_vals(bits).astype(np.float32)).to(torch.float8_e4m3fn) \
+            .view(torch.uint8).numpy()
+
+    for pool, new in ((kc, kn), (vc, vn)):
+        rows = pool.reshape(N * bs, Hkv, d)
+        want = np.zeros_like(rows)
+        for b in range(B):
+            for i in range(3):
+                want[slots[b, i]] = cast(new[b, i])
+        assert np.array_equal(rows, want)
 
 
 # ----------------------------------------------------------------------------- prefill stage
