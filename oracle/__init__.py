@@ -26,7 +26,9 @@ _LIB = None
 def _lib():
     global _LIB
     if _LIB is None:
-        path = _build.build()
+        # ORACLE_LIB names another build of oracle.c; tests/oracle_mutants.py uses it
+        # to load copies with one planted mistake each
+        path = os.environ.get("ORACLE_LIB") or _build.build()
         lib = ctypes.CDLL(path)
         i64, i32, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
         p = ctypes.c_void_p

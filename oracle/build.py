@@ -12,16 +12,21 @@ SRC = os.path.join(HERE, "oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
 
-def build(force: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
-        return LIB
+def compile_c(src: str, out: str) -> None:
+    """gcc one oracle source into a shared library at `out` (written atomically)."""
     cmd = [
         "gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
         "-fPIC", "-shared", "-Wall", "-Wextra", "-Wno-unused-parameter",
-        SRC, "-o", LIB + ".tmp", "-lm",
+        src, "-o", out + ".tmp", "-lm",
     ]
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(out + ".tmp", out)
+
+
+def build(force: bool = False) -> str:
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+        return LIB
+    compile_c(SRC, LIB)
     return LIB
 
 

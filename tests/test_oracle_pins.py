@@ -342,6 +342,120 @@ def test_global_softmax_differs_from_per_block_normalisation():
     assert np.abs(per_block - out[b, i]).max() > 1e-3
 
 
+
+def _pad_blocks(pool, pad, fill):
+    """Copy [N, bs, Hkv, d] into [N, bs + pad, Hkv, d] with `fill` in the pad rows and
+    return the flat buffer and its block stride."""
+    N, bs, Hkv, d = pool.shape
+    big = np.full((N, bs + pad, Hkv, d), fill, pool.dtype)
+    big[:, :bs] = pool
+    return big.ravel(), (bs + pad) * Hkv * d
+
+
+def test_block_stride_larger_than_a_block_reads_only_the_block():
+    """A pool whose blocks sit block_stride > bs*Hkv*d elements apart (the rest of each
+    block's span holds NaN, or code 127 / e4m3 NaN for the one-byte pools) gives the
+    same decode, chunked-prefill, score and INT8/FP8 results, bit for bit, as the dense
+    pool; so the stride is honoured and the padding is never read."""
+    c = rand_case(41, Hq=8, Hkv=2, d=16, bs=4, N=20, lens=(5, 13, 8))
+    bs, Hkv, d = c["bs"], c["Hkv"], c["d"]
+    dense = bs * Hkv * d
+    sc = 1 / math.sqrt(d)
+    nan16 = np.uint16(0x7fc0)
+    kp, stride = _pad_blocks(c["kc"], 3, nan16)
+    vp, _ = _pad_blocks(c["vc"], 3, nan16)
+    assert stride > dense
+    args = (c["bt"], c["lens"], Hkv, bs, sc)
+    assert np.array_equal(oracle.paged_decode(c["q"], kp, vp, stride, *args), run_decode(c))
+    s_pad = oracle.score_tokens(kp, vp, stride, c["bt"], c["lens"], Hkv, d, bs)
+    s_den = oracle.score_tokens(c["kc"].ravel(), c["vc"].ravel(), dense, c["bt"], c["lens"], Hkv,
+                                d, bs)
+    assert np.array_equal(s_pad, s_den, equal_nan=True)
+    cu = np.array([0, 2, 3, 7], np.int32)
+    qp = bf16_bits(np.random.default_rng(42).standard_normal((7, c["Hq"], d)))
+    assert np.array_equal(oracle.paged_prefill(qp, cu, kp, vp, stride, *args),
+                          oracle.paged_prefill(qp, cu, c["kc"].ravel(), c["vc"].ravel(), dense,
+                                               *args))
+    kq, ks = oracle.quantize_int8(c["kc"])
+    vq, vs = oracle.quantize_int8(c["vc"])
+    kqp, _ = _pad_blocks(kq, 3, np.int8(127))
+    vqp, _ = _pad_blocks(vq, 3, np.int8(127))
+    assert np.array_equal(
+        oracle.paged_decode_int8(c["q"], kqp, vqp, ks.ravel(), vs.ravel(), stride, *args),
+        oracle.paged_decode_int8(c["q"], kq.ravel(), vq.ravel(), ks.ravel(), vs.ravel(), dense,
+                                 *args))
+    assert np.array_equal(
+        oracle.score_tokens_int8(kqp, vqp, ks.ravel(), vs.ravel(), stride, c["bt"], c["lens"],
+                                 Hkv, d, bs),
+        oracle.score_tokens_int8(kq.ravel(), vq.ravel(), ks.ravel(), vs.ravel(), dense, c["bt"],
+                                 c["lens"], Hkv, d, bs), equal_nan=True)
+    k8, v8 = oracle.quantize_e4m3(c["kc"]), oracle.quantize_e4m3(c["vc"])
+    k8p, _ = _pad_blocks(k8, 3, np.uint8(0x7f))
+    v8p, _ = _pad_blocks(v8, 3, np.uint8(0x7f))
+    assert np.array_equal(oracle.paged_decode_fp8(c["q"], k8p, v8p, stride, *args),
+                          oracle.paged_decode_fp8(c["q"], k8.ravel(), v8.ravel(), dense, *args))
+
+
+def test_append_with_padded_block_stride_leaves_the_padding():
+    """Appending through a padded block stride writes the same block contents as the
+    dense append (bf16 and FP8) and leaves every pad element as it was."""
+    rng = np.random.default_rng(43)
+    B, Hkv, d, bs, N, pad = 2, 2, 8, 4, 10, 2
+    bt = np.array([[3, 7, -1], [1, 0, 9]], np.int32)
+    kn = bf16_bits(rng.standard_normal((B, 3, Hkv, d)))
+    vn = bf16_bits(rng.standard_normal((B, 3, Hkv, d)))
+    pos = np.array([2, 7], np.int32)
+    for fn, dt, fill in ((oracle.append_kv, np.uint16, 0x7fc0),
+                         (oracle.append_kv_fp8, np.uint8, 0x7f)):
+        kd = np.full((N, bs, Hkv, d), fill, dt)
+        vd = np.full_like(kd, fill)
+        fn(kn, vn, kd.reshape(-1), vd.reshape(-1), bs * Hkv * d, bt, pos, bs)
+        kp = np.full((N, bs + pad, Hkv, d), fill, dt)
+        vp = np.full_like(kp, fill)
+        fn(kn, vn, kp.reshape(-1), vp.reshape(-1), (bs + pad) * Hkv * d, bt, pos, bs)
+        assert (kp[:, bs:] == fill).all() and (vp[:, bs:] == fill).all()
+        assert np.array_equal(kp[:, :bs], kd) and np.array_equal(vp[:, :bs], vd)
+        assert (kd != fill).any()
+    # INT8: the code pools are padded, the scale pools keep their [N][bs][Hkv] layout
+    pools = {}
+    for p_ in (0, pad):
+        kq = np.full((N, bs + p_, Hkv, d), 127, np.int8)
+        vq = np.full_like(kq, 127)
+        ks = np.full((N, bs, Hkv), -1, np.float32)
+        vs = np.full_like(ks, -1)
+        oracle.append_kv_int8(kn, vn, kq.reshape(-1), vq.reshape(-1), ks.reshape(-1),
+                              vs.reshape(-1), (bs + p_) * Hkv * d, bt, pos, bs)
+        pools[p_] = (kq, vq, ks, vs)
+    kq, vq, ks, vs = pools[pad]
+    assert (kq[:, bs:] == 127).all() and (vq[:, bs:] == 127).all()
+    assert np.array_equal(kq[:, :bs], pools[0][0]) and np.array_equal(vq[:, :bs], pools[0][1])
+    assert np.array_equal(ks, pools[0][2]) and np.array_equal(vs, pools[0][3])
+    assert (pools[0][0] != 127).any()
+
+
+def test_prefill_pack_with_padded_block_stride_leaves_the_padding():
+    """Packing kept prompt rows through a padded block stride writes the same block
+    contents as the dense pack and leaves every pad element as it was."""
+    rng = np.random.default_rng(44)
+    Hkv, d, bs, N, pad = 2, 8, 4, 12, 3
+    cu = np.array([0, 9, 20], np.int32)
+    k = bf16_bits(rng.standard_normal((20, Hkv, d)))
+    v = bf16_bits(rng.standard_normal((20, Hkv, d)))
+    keep, kept = oracle.prefill_select(rng.standard_normal(20), cu, 6)
+    bt = np.array([[5, 2], [0, 11]], np.int32)
+    out = {}
+    for p_ in (0, pad):
+        kc = np.full((N, bs + p_, Hkv, d), 0x7fc0, np.uint16)
+        vc = np.full_like(kc, 0x7fc0)
+        oracle.prefill_pack(k, v, cu, keep, kept, kc.reshape(-1), vc.reshape(-1),
+                            (bs + p_) * Hkv * d, bt, bs)
+        out[p_] = (kc, vc)
+    kc, vc = out[pad]
+    assert (kc[:, bs:] == 0x7fc0).all() and (vc[:, bs:] == 0x7fc0).all()
+    assert np.array_equal(kc[:, :bs], out[0][0]) and np.array_equal(vc[:, :bs], out[0][1])
+    assert (out[0][0] != 0x7fc0).sum() == 12 * Hkv * d
+
+
 # ------------------------------------------------------------------ scores / eviction
 def test_score_is_norm_ratio_closed_forms():
     B, Hkv, d, bs, N = 1, 2, 4, 2, 3
@@ -399,6 +513,12 @@ def test_evict_planted_low_block_and_rules():
     # brute force of the block means for seq 0
     for j in range(5):
         assert abs(means[0, j] - scores[0, j * bs:(j + 1) * bs].mean()) < 1e-15
+    # gap: second-lowest minus lowest candidate mean, +inf with fewer than two
+    for b in range(B):
+        m = np.sort(means[b][~np.isnan(means[b])])
+        assert gap[b] == (m[1] - m[0] if m.size >= 2 else np.inf)
+        assert gap[b] >= 0
+    assert gap[0] == np.sort(means[0])[1] - 0.5 > 0.4
 
 
 def test_evict_scaled_value_block_is_chosen():
