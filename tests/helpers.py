@@ -61,10 +61,25 @@ def assert_evict_consistent(got: np.ndarray, ref_idx, ref_means, ref_gap, what="
 class Device:
     """Device copies of one workload plus outputs and scratch for the C ABI."""
 
-    def __init__(self, wl: W.Workload, num_splits=0):
+    def __init__(self, wl: W.Workload, num_splits=0, pad=0):
+        """pad > 0: every pool is a [:, :, :bs] view of a buffer with bs + pad slots per
+        block, so its block stride is (bs + pad)·Hkv·d; the pad slots hold NaN (bf16),
+        127 (INT8) or the e4m3 NaN code, and pads_untouched() checks they still do."""
         cfg = wl.cfg
         dev = torch.device("cuda")
         self.wl, self.dev, self.num_splits = wl, dev, num_splits
+        self._pads = []
+
+        def pool(shape, dtype, fill, src=None):
+            L_, N_, bs_ = shape[:3]
+            big = torch.full((L_, N_, bs_ + pad) + tuple(shape[3:]), fill, dtype=dtype,
+                             device=dev)
+            view = big[:, :, :bs_]
+            if src is not None:
+                view.copy_(src)
+            if pad:
+                self._pads.append((big[:, :, bs_:], fill))
+            return view
         self.bt = torch.as_tensor(wl.block_tables, device=dev)
         self.ctx = torch.as_tensor(wl.ctx_lens, device=dev)
         self.pos = torch.as_tensor(wl.positions, device=dev)
@@ -74,13 +89,18 @@ class Device:
         L, B = self.q.shape[0], cfg.batch
         N, bs, Hkv, d = wl.num_blocks, cfg.block_size, cfg.hkv, cfg.head_dim
         if cfg.fp8:
-            self.k8 = torch.zeros(L, N, bs, Hkv, d, dtype=torch.uint8, device=dev)
-            self.v8 = torch.zeros_like(self.k8)
+            self.k8 = pool((L, N, bs, Hkv, d), torch.uint8, 0x7f if pad else 0)
+            self.v8 = pool((L, N, bs, Hkv, d), torch.uint8, 0x7f if pad else 0)
         elif cfg.int8:
-            self.kq = torch.zeros(L, N, bs, Hkv, d, dtype=torch.int8, device=dev)
-            self.vq = torch.zeros_like(self.kq)
+            self.kq = pool((L, N, bs, Hkv, d), torch.int8, 127 if pad else 0)
+            self.vq = pool((L, N, bs, Hkv, d), torch.int8, 127 if pad else 0)
             self.ks = torch.zeros(L, N, bs, Hkv, dtype=torch.float32, device=dev)
             self.vs = torch.zeros_like(self.ks)
+        elif pad:
+            k_src = wl.kv[0] if wl.kv is not None else wl.k_pool
+            v_src = wl.kv[1] if wl.kv is not None else wl.v_pool
+            self.k_pool = pool(tuple(k_src.shape), torch.bfloat16, float("nan"), k_src.to(dev))
+            self.v_pool = pool(tuple(v_src.shape), torch.bfloat16, float("nan"), v_src.to(dev))
         else:
             if wl.kv is not None:
                 self.kv = wl.kv.to(dev)
@@ -92,6 +112,15 @@ class Device:
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self.ws = pk.alloc_workspace(B, cfg.hq, Hkv, d, bs, wl.max_blocks, num_splits, dev)
         self.slots = torch.full((B, 1), -7, dtype=torch.int64, device=dev)
+
+    def pads_untouched(self) -> bool:
+        for gap, fill in self._pads:
+            if gap.dtype == torch.bfloat16:
+                if not torch.isnan(gap).all():
+                    return False
+            elif not (gap == fill).all():
+                return False
+        return True
 
     def _append_hist(self, layer, k, v, bt, pos):
         if self.wl.cfg.fp8:

@@ -49,12 +49,12 @@ MEDIUM = {
 }
 
 
-def _parity(wl, layers, num_splits=0, score=None):
+def _parity(wl, layers, num_splits=0, score=None, pad=0):
     cfg = wl.cfg
     score = cfg.score if score is None else score
     seqs = range(cfg.batch)
     refs = [oracle_step(wl, l, seqs, score=score) for l in layers]
-    dev = Device(wl, num_splits)
+    dev = Device(wl, num_splits, pad=pad)
     if cfg.int8 or cfg.fp8:
         for l in layers:
             dev.fill_int8_history(l)
@@ -117,6 +117,25 @@ def test_split_count_invariance(num_splits, kv):
         cfg = W.scaled(cfg, int8=False, fp8=True)
     wl = W.generate(cfg, "cpu")
     _parity(wl, [0], num_splits=num_splits)
+
+
+@pytest.mark.parametrize("kv", ["bf16", "int8", "fp8"])
+def test_padded_block_stride(kv):
+    """Pools whose blocks sit (bs + 3)·Hkv·d elements apart (views of a larger buffer
+    whose gaps hold NaN, code 127 or the e4m3 NaN code): the history and new-token
+    appends, the decode and the score match the oracle on dense pools, and no gap
+    element is read or written."""
+    base = C["c3"] if kv == "bf16" else C["c5"]
+    cfg = W.scaled(base, key="pad", layers=1, batch=4, old_lens=(700, 45, 16, 1),
+                   score=(kv == "bf16"))
+    if kv == "fp8":
+        cfg = W.scaled(cfg, int8=False, fp8=True)
+    wl = W.generate(cfg, "cpu")
+    dev, refs = _parity(wl, [0], pad=3)
+    assert dev.pads_untouched()
+    pool = {"bf16": "k_pool", "int8": "kq", "fp8": "k8"}[kv]
+    N, bs, Hkv, d = getattr(dev, pool)[0].shape
+    assert getattr(dev, pool)[0].stride(0) == (bs + 3) * Hkv * d
 
 
 def test_physical_block_permutation_gives_identical_output():

@@ -49,16 +49,31 @@ def _workspace(c, balanced):
     return ws
 
 
-def _run(c, err_expected=0, balanced=False):
+def _padded(pool, pad):
+    """A [N, bs, Hkv, d] view of a device buffer with bs + pad slots per block whose
+    extra slots hold NaN (block stride (bs + pad)·Hkv·d), and those extra slots."""
+    N, bs, Hkv, d = pool.shape
+    big = torch.full((N, bs + pad, Hkv, d), float("nan"), dtype=pool.dtype, device="cuda")
+    big[:, :bs].copy_(pool)
+    return big[:, :bs], big[:, bs:]
+
+
+def _run(c, err_expected=0, balanced=False, pad=0):
     dev = "cuda"
     out = torch.full(c["q"].shape, float("nan"), dtype=torch.bfloat16, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
+    if pad:
+        (kd, kgap), (vd, vgap) = _padded(c["k"], pad), _padded(c["v"], pad)
+    else:
+        kd, vd = c["k"].to(dev), c["v"].to(dev)
     pk.pa_prefill_attention(out, c["q"].to(dev), torch.as_tensor(c["cu"]).to(dev),
-                            max(c["qlens"] + [0]), c["k"].to(dev), c["v"].to(dev),
+                            max(c["qlens"] + [0]), kd, vd,
                             torch.as_tensor(c["bt"]).to(dev), torch.as_tensor(c["lens"]).to(dev),
                             c["d"] ** -0.5, err, workspace=_workspace(c, balanced))
     torch.cuda.synchronize()
     assert err.item() == err_expected
+    if pad:
+        assert torch.isnan(kgap).all() and torch.isnan(vgap).all()
     return out
 
 
@@ -87,6 +102,17 @@ def test_prefill_attention_medium(key, balanced):
     c = _case(lens, qlens, Hq, Hkv, d, bs, seed=100 + list(CASES).index(key))
     out = _run(c, balanced=balanced)
     assert_attention_close(out, _oracle(c), key)
+
+
+@pytest.mark.parametrize("balanced", [False, True])
+@pytest.mark.parametrize("key", ["g4d128", "g2d64"])
+def test_prefill_attention_padded_block_stride(key, balanced):
+    """Pools whose blocks sit (bs + 3)·Hkv·d elements apart, the extra slots holding
+    NaN: the kernels follow the block stride and read nothing between blocks."""
+    lens, qlens, Hq, Hkv, d, bs = CASES[key]
+    c = _case(lens, qlens, Hq, Hkv, d, bs, seed=141 + list(CASES).index(key))
+    out = _run(c, balanced=balanced, pad=3)
+    assert_attention_close(out, _oracle(c), f"{key}, padded block stride")
 
 
 @pytest.mark.parametrize("qlens", [[64], [256, 1], [512, 0, 512]])
