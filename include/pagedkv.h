@@ -192,6 +192,7 @@ int pa_append_kv_int8(const uint16_t *k_new, const uint16_t *v_new,
  * pa_decode with K[t, h, e] = k_scale[t, h] * kq[t, h, e] and likewise V,
  * dequantised in registers (the K scale multiplies the dot product, the V
  * scale multiplies the softmax weight).  Same workspace rule as pa_decode.
+ * k_scale, v_scale: fp32 [N][bs][Hkv], 16-byte aligned (PA_ERR_ALIGN otherwise).
  * ==========================================================================*/
 int pa_decode_int8(uint16_t *out, const uint16_t *q,
                    const int8_t *kq_cache, const int8_t *vq_cache,

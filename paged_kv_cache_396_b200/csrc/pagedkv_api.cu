@@ -69,7 +69,8 @@ int decode_entry(uint16_t *out, const uint16_t *q, const void *kc, const void *v
     const int elt = kv == pkv::kKvBf16 ? 2 : 1;
     if (!al16(out) || !al16(q) || !al16(kc) || !al16(vc) || (block_stride * elt) % 16 != 0)
         return PA_ERR_ALIGN;
-    if (B == 0) return PA_OK;
+    // the staged kernel bulk-copies each tile's scales (cp.async.bulk: 16-byte source)
+    if (kv == pkv::kKvInt8 && (!al16(ks) || !al16(vs))) return PA_ERR_ALIGN;
     const int sms = device_sms();
     if (sms < 0) return sms;
     const pkv::DecodePlan plan = pkv::make_decode_plan(B, Hq, Hkv, d, bs, MB, num_splits, kv, sms);
@@ -161,7 +162,6 @@ int pa_append_kv(const uint16_t *k_new, const uint16_t *v_new, uint16_t *k_cache
     if (!al16(k_new) || !al16(v_new) || !al16(k_cache) || !al16(v_cache) ||
         (block_stride * 2) % 16 != 0)
         return PA_ERR_ALIGN;
-    if (B == 0 || n_new == 0) return PA_OK;
     const int sms = device_sms();
     if (sms < 0) return sms;
     pkv::AppendArgs a{block_tables, positions, slot_out, err_flag, block_stride, num_blocks,
@@ -185,7 +185,6 @@ int pa_append_kv_int8(const uint16_t *k_new, const uint16_t *v_new, int8_t *kq_c
     if (!al16(k_new) || !al16(v_new) || !al16(kq_cache) || !al16(vq_cache) || !al16(k_scale) ||
         !al16(v_scale) || block_stride % 16 != 0)
         return PA_ERR_ALIGN;
-    if (B == 0 || n_new == 0) return PA_OK;
     const int sms = device_sms();
     if (sms < 0) return sms;
     pkv::AppendArgs a{block_tables, positions, slot_out, err_flag, block_stride, num_blocks,
@@ -354,7 +353,6 @@ int pe_score_tokens(float *scores, const uint16_t *k_cache, const uint16_t *v_ca
     int rc = check_common(B, Hkv, d, bs, max_blocks_per_seq, num_blocks, block_stride);
     if (rc) return rc;
     if (!al16(k_cache) || !al16(v_cache) || (block_stride * 2) % 16 != 0) return PA_ERR_ALIGN;
-    if (B == 0) return PA_OK;
     const int sms = device_sms();
     if (sms < 0) return sms;
     pkv::ScoreArgs a{scores, k_cache, v_cache, block_tables, ctx_lens, err_flag, block_stride,
@@ -368,7 +366,6 @@ int pe_select_evict_block(int32_t *evict, float *block_means, const float *score
     if (B == 0) return PA_OK;
     if (!evict || !scores || !ctx_lens) return PA_ERR_NULL;
     if (B < 0 || max_blocks_per_seq < 1 || Hkv < 1 || bs < 1) return PA_ERR_SHAPE;
-    if (B == 0) return PA_OK;
     const int sms = device_sms();
     if (sms < 0) return sms;
     return finish(pkv::launch_select_evict(evict, block_means, scores, ctx_lens, B,
@@ -383,10 +380,15 @@ int pa_decode_static_scratch(uint16_t *out, const uint16_t *q, const uint16_t *k
                              int64_t num_blocks, float scale, int num_splits, int32_t *err_flag,
                              void *stream) {
     if (B == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !ctx_lens || !err_flag)
+        return PA_ERR_NULL;
     if (num_splits < 0) return PA_ERR_SHAPE;
     int rc = check_common(B, Hkv, d, bs, max_blocks_per_seq, num_blocks, block_stride);
     if (rc) return rc;
     if (Hq < Hkv || Hq % Hkv != 0 || Hq / Hkv > 16) return PA_ERR_SHAPE;
+    if (!(scale == scale)) return PA_ERR_SHAPE;
+    if (!al16(out) || !al16(q) || !al16(k_cache) || !al16(v_cache) || (block_stride * 2) % 16 != 0)
+        return PA_ERR_ALIGN;
     const int sms = device_sms();
     if (sms < 0) return sms;
     const size_t cap = PA_STATIC_SCRATCH_BYTES;
@@ -597,6 +599,7 @@ int pa_prefill_attention(uint16_t *out, const uint16_t *q, const int32_t *cu_q, 
     if ((int64_t)max_q_len * G / 64 + 1 > INT32_MAX) return PA_ERR_SHAPE;
     if (!al16(out) || !al16(q) || !al16(k_cache) || !al16(v_cache) || (block_stride * 2) % 16)
         return PA_ERR_ALIGN;
+    if (workspace && !al16(workspace)) return PA_ERR_ALIGN;
     const int sms = device_sms();
     if (sms < 0) return sms;
     pkv::PrefillAttnArgs a;
@@ -622,7 +625,6 @@ int pa_prefill_attention(uint16_t *out, const uint16_t *q, const int32_t *cu_q, 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // tcgen05 / TMEM kernel for d = 128 and 16-token-aligned blocks (TMA pages);
     // the mma.sync kernel covers every other supported shape
-    if (workspace && !al16(workspace)) return PA_ERR_ALIGN;
     return finish(pkv::prefill_attn_tc_supported(a)
                       ? pkv::launch_prefill_attn_tc(a, max_q_len, workspace, workspace_bytes, sms, st)
                       : pkv::launch_prefill_attn(a, max_q_len, st));
