@@ -276,6 +276,50 @@ def test_plan_and_selftest_reject_bad_arguments_on_host(lib):
     assert lib.pa_selftest_wait_timeout(None, None) == -1
 
 
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "pagedkv.h"
+int main(void) {
+    /* host-side paths only: no device memory is touched */
+    char *fake = (char *)(uintptr_t)(1u << 20);  /* aligned, never dereferenced */
+    int rc_null = pa_decode(NULL, NULL, NULL, NULL, 2048, NULL, 4, NULL, 2, 32, 8, 128, 16, 10,
+                            0.1f, 0, NULL, 0, NULL, NULL);
+    int rc_shape = pe_select_evict_block((int32_t *)fake, NULL, (const float *)fake,
+                                         (const int32_t *)fake, 2, 0, 8, 16, NULL);
+    int rc_empty = pa_append_kv(NULL, NULL, NULL, NULL, 2048, NULL, 4, NULL, 0, 1, 8, 128, 16, 10,
+                                NULL, NULL, NULL);
+    printf("%s|%d|%d|%d|%s\n", pa_version(), rc_null, rc_shape, rc_empty,
+           pa_status_string(PA_ERR_ALIGN));
+    return strncmp(pa_version(), "pagedkv", 7) != 0;
+}
+"""
+
+
+def test_plain_c_client_links_and_calls_the_library(lib, tmp_path):
+    """The boundary is usable from C alone: a C99 program built against
+    include/pagedkv.h links libpagedkv.so and gets the documented host status codes;
+    the header also compiles as C++."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None or shutil.which("g++") is None:
+        pytest.skip("no host C compiler")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    libdir = os.path.dirname(build_lib.build())
+    exe = tmp_path / "client"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I",
+                    os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir,
+                    "-lpagedkv", "-Wl,-rpath," + libdir], check=True)
+    subprocess.run(["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-x",
+                    "c++", "-I", os.path.join(ROOT, "include"), str(src)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.strip()
+    version, rc_null, rc_shape, rc_empty, align_text = out.split("|")
+    assert version == lib.pa_version().decode()
+    assert (int(rc_null), int(rc_shape), int(rc_empty)) == (-1, -2, 0)
+    assert align_text == lib.pa_status_string(-3).decode()
+
+
 def test_product_path_never_imports_the_oracle():
     pkg = os.path.join(ROOT, "paged_kv_cache_396_b200")
     for dirpath, _, files in os.walk(pkg):
