@@ -1053,3 +1053,37 @@ def test_prefill_attention_is_causal_and_invalid_rows_are_zero():
     c["kc"][b0_last, (20 - 1) % c["bs"]] = bf16_bits(np.full((c["Hkv"], c["d"]), 3.0))
     moved = run_prefill(c)
     assert np.array_equal(moved[:5], base[:5]) and not np.array_equal(moved[5], base[5])
+
+
+# ----------------------------------------------------------------------------- mutation check
+def test_mutation_check_still_applies_to_the_oracle():
+    """Every planted mistake of tests/oracle_mutants.py still finds its text exactly
+    once in oracle.c (so the mutation check keeps testing the current oracle), and one
+    mutant, built and loaded through ORACLE_LIB, is rejected by a pin."""
+    import importlib.util
+    import subprocess
+    import sys
+    import tempfile
+    here = os.path.dirname(os.path.abspath(__file__))
+    spec = importlib.util.spec_from_file_location("oracle_mutants",
+                                                  os.path.join(here, "oracle_mutants.py"))
+    mut = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mut)
+    src = open(mut.oracle_build.SRC).read()
+    names = [m[0] for m in mut.MUTANTS]
+    assert len(names) == len(set(names))
+    for name, _, find, repl in mut.MUTANTS:
+        assert src.count(find) == 1, name
+        assert find != repl, name
+    name, _, find, repl = next(m for m in mut.MUTANTS if m[0] == "gqa_mod")
+    with tempfile.TemporaryDirectory() as tmp:
+        c, so = os.path.join(tmp, "m.c"), os.path.join(tmp, "m.so")
+        with open(c, "w") as f:
+            f.write(src.replace(find, repl))
+        mut.oracle_build.compile_c(c, so)
+        r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                            os.path.join(here, "test_oracle_pins.py"), "-k",
+                            "decode_equals_contiguous_sdpa"],
+                           cwd=os.path.dirname(here), env=dict(os.environ, ORACLE_LIB=so),
+                           capture_output=True, text=True)
+        assert r.returncode != 0, r.stdout[-500:]
