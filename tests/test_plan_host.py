@@ -16,7 +16,7 @@ from paged_kv_cache_396_b200 import build_lib
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PKG = os.path.join(ROOT, "paged_kv_cache_396_b200")
 
-# name, B, Hq, Hkv, d, bs, MB, int8, num_splits, staged?
+# name, B, Hq, Hkv, d, bs, MB, kv (0 bf16, 1 INT8, 2 FP8), num_splits, staged?
 CASES = [
     ("c1", 2, 4, 2, 64, 16, 7, 0, 0, 1),
     ("c2", 32, 32, 8, 64, 16, 65, 0, 0, 1),
@@ -31,6 +31,10 @@ CASES = [
     ("bs12", 4, 64, 4, 128, 12, 60, 0, 0, 0),
     ("i8d64", 3, 64, 8, 64, 16, 13, 1, 0, 0),
     ("hkv16", 2, 32, 16, 64, 16, 10, 0, 0, 0),
+    ("f8", 128, 64, 8, 128, 16, 257, 2, 0, 1),
+    ("f8g16", 3, 64, 4, 128, 16, 19, 2, 0, 1),
+    ("f8split96", 3, 64, 8, 128, 16, 126, 2, 96, 1),
+    ("f8d64", 3, 64, 8, 64, 16, 13, 2, 0, 0),
 ]
 
 PROBE = r"""
@@ -39,8 +43,8 @@ PROBE = r"""
 #include "kernels.h"
 int main(int argc, char **argv) {
     int B = atoi(argv[1]), Hq = atoi(argv[2]), Hkv = atoi(argv[3]), d = atoi(argv[4]);
-    int bs = atoi(argv[5]), MB = atoi(argv[6]), i8 = atoi(argv[7]), ns = atoi(argv[8]);
-    pkv::DecodePlan p = pkv::make_decode_plan(B, Hq, Hkv, d, bs, MB, ns, i8 != 0, 148);
+    int bs = atoi(argv[5]), MB = atoi(argv[6]), kv = atoi(argv[7]), ns = atoi(argv[8]);
+    pkv::DecodePlan p = pkv::make_decode_plan(B, Hq, Hkv, d, bs, MB, ns, kv, 148);
     printf("%d %d %d %d %d %d %d %d %d %d %d %d %zu %zu %zu\n", p.kernel, p.S, p.chunk, p.wph,
            p.tpw, p.n_sub, p.nstage, p.stage_bytes, p.smem_bytes, p.v_off, p.ks_off, p.vs_off,
            p.off_ml, p.off_acc, p.ws_total);
@@ -72,8 +76,9 @@ def probe():
 
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_plan_invariants(probe, case):
-    name, B, Hq, Hkv, d, bs, MB, i8, ns, staged = case
-    p = probe(B, Hq, Hkv, d, bs, MB, i8, ns)
+    name, B, Hq, Hkv, d, bs, MB, kv_kind, ns, staged = case
+    p = probe(B, Hq, Hkv, d, bs, MB, kv_kind, ns)
+    i8 = kv_kind == 1
     assert p["kernel"] == staged
     max_ctx = MB * bs
     assert p["S"] * p["chunk"] >= max_ctx            # partitions cover the longest context
@@ -87,7 +92,7 @@ def test_plan_invariants(probe, case):
     assert p["smem_bytes"] <= 227 * 1024
     assert p["stage_bytes"] % 1024 == 0 and p["stage_bytes"] <= 68 * 1024
     # K and V regions of n_sub sub-tiles of 16 tokens x Hkv x d elements, then scales
-    elt = 1 if i8 else 2
+    elt = 1 if kv_kind else 2
     kv = p["n_sub"] * 16 * Hkv * d * elt
     assert p["v_off"] == kv and p["ks_off"] == 2 * kv
     assert p["vs_off"] - p["ks_off"] == (p["n_sub"] * 16 * Hkv * 4 if i8 else 0)
