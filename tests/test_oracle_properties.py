@@ -162,3 +162,40 @@ def test_compaction_keeps_every_surviving_token_at_its_slot(c, seed):
                 continue
             q = p - bs * sum(1 for g in gone if g < j)
             assert oracle.slot(nbt[b], q, bs) == oracle.slot(c["bt"][b], p, bs)
+
+
+@SETTINGS
+@given(st.integers(1, 6), st.sampled_from([4, 16, 64]), st.floats(-20, 20),
+       st.integers(0, 2 ** 31 - 1))
+def test_int8_quantiser_bounds(rows, d, log2_mag, seed):
+    """Codes in [-127, 127] with the row's amax at +-127, scale = amax / 127 in fp32, and
+    |scale * code - x| <= scale / 2 plus the one fp32 rounding of x / scale; an all-zero
+    row gets scale 0 and codes 0."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, d)) * 2.0 ** log2_mag
+    x[0] = 0.0
+    b = bits(x)
+    codes, scales = oracle.quantize_int8(b)
+    xv = vals(b)
+    amax = np.abs(xv).max(axis=1)
+    assert np.array_equal(scales, (amax.astype(np.float32) / np.float32(127)).astype(np.float32))
+    assert scales[0] == 0 and not codes[0].any()
+    nz = amax > 0
+    assert (np.abs(codes[nz]).max(axis=1) == 127).all() and np.abs(codes).max() <= 127
+    s = scales[:, None].astype(np.float64)
+    assert (np.abs(s * codes - xv) <= s * (0.5 + 127 * 2.0 ** -24)).all()
+
+
+@SETTINGS
+@given(st.floats(-12, 8.7), st.integers(0, 2 ** 31 - 1))
+def test_e4m3_cast_is_torchs_in_range_and_saturates_beyond(log2_mag, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal(256) * 2.0 ** log2_mag
+    b = bits(x)
+    xv = vals(b)
+    codes = oracle.quantize_e4m3(b)
+    ok = np.abs(xv) <= 448.0
+    ref = torch.as_tensor(xv[ok].astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8)
+    assert np.array_equal(codes[ok], ref.numpy())
+    big = ~ok
+    assert np.array_equal(codes[big], np.where(xv[big] > 0, 0x7e, 0xfe).astype(np.uint8))
