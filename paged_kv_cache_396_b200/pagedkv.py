@@ -152,6 +152,25 @@ def _want(t: torch.Tensor, dtype, name: str):
         raise TypeError(f"{name}: expected a CUDA tensor")
 
 
+def _covers(t: torch.Tensor, n: int, name: str):
+    """t holds at least the n elements the kernels read (they index by batch row)."""
+    if t.numel() < n:
+        raise ValueError(f"{name}: needs at least {n} elements, got {t.numel()}")
+
+
+def _table_rows(block_tables: torch.Tensor, B: int):
+    if block_tables.dim() != 2 or block_tables.shape[0] < B or block_tables.shape[1] < 1:
+        raise ValueError(f"block_tables: expected [B >= {B}, MB >= 1], got "
+                         f"{tuple(block_tables.shape)}")
+
+
+def _one_device(ref: torch.Tensor, *ts):
+    """Every tensor the call reads or writes is on the pools' device."""
+    for t in ts:
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"all tensors must be on {ref.device}, got one on {t.device}")
+
+
 def _pool_geometry(pool: torch.Tensor, name: str):
     if pool.dim() != 4:
         raise ValueError(f"{name}: expected [N, bs, Hkv, d], got shape {tuple(pool.shape)}")
@@ -167,6 +186,17 @@ def _same_pool(a: torch.Tensor, b: torch.Tensor):
 
 
 # ----------------------------------------------------------------------------- append
+def _append_sizes(k_new, Hkv, d, block_tables, positions, err_flag, slot_out, B, n_new):
+    if tuple(k_new.shape[2:]) != (Hkv, d):
+        raise ValueError("k_new inner dims must match the pool's [Hkv, d]")
+    _table_rows(block_tables, B)
+    _covers(positions, B, "positions")
+    _covers(err_flag, 1, "err_flag")
+    if slot_out is not None:
+        _want(slot_out, torch.int64, "slot_out")
+        _covers(slot_out, B * n_new, "slot_out")
+
+
 def pa_append_kv(k_new, v_new, k_cache, v_cache, block_tables, positions, err_flag,
                  slot_out=None, stream=None):
     """Write new tokens into the paged pools.  k_new/v_new: [B, n_new, Hkv, d] or
@@ -184,10 +214,8 @@ def pa_append_kv(k_new, v_new, k_cache, v_cache, block_tables, positions, err_fl
     if not (k_new.is_contiguous() and v_new.is_contiguous()) or k_new.shape != v_new.shape:
         raise ValueError("k_new/v_new must be contiguous and of equal shape")
     B, n_new = k_new.shape[0], k_new.shape[1]
-    if k_new.shape[2:] != (Hkv, d):
-        raise ValueError("k_new inner dims must match the pool's [Hkv, d]")
-    if slot_out is not None:
-        _want(slot_out, torch.int64, "slot_out")
+    _append_sizes(k_new, Hkv, d, block_tables, positions, err_flag, slot_out, B, n_new)
+    _one_device(k_cache, k_new, v_new, block_tables, positions, err_flag, slot_out)
     bt = block_tables.contiguous()
     rc = load().pa_append_kv(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), stride,
                              _ptr(bt), bt.shape[1], _ptr(positions.contiguous()), B, n_new, Hkv, d,
@@ -218,8 +246,9 @@ def pa_append_kv_int8(k_new, v_new, kq_cache, vq_cache, k_scale, v_scale, block_
     if not (k_new.is_contiguous() and v_new.is_contiguous()) or k_new.shape != v_new.shape:
         raise ValueError("k_new/v_new must be contiguous and of equal shape")
     B, n_new = k_new.shape[0], k_new.shape[1]
-    if slot_out is not None:
-        _want(slot_out, torch.int64, "slot_out")
+    _append_sizes(k_new, Hkv, d, block_tables, positions, err_flag, slot_out, B, n_new)
+    _one_device(kq_cache, k_new, v_new, k_scale, v_scale, block_tables, positions, err_flag,
+                slot_out)
     bt = block_tables.contiguous()
     rc = load().pa_append_kv_int8(_ptr(k_new), _ptr(v_new), _ptr(kq_cache), _ptr(vq_cache),
                                   _ptr(k_scale), _ptr(v_scale), stride, _ptr(bt), bt.shape[1],
@@ -268,6 +297,10 @@ def _decode_checks(out, q, block_tables, ctx_lens, err_flag):
     _want(err_flag, torch.int32, "err_flag")
     if not (out.is_contiguous() and q.is_contiguous()) or out.shape != q.shape or q.dim() != 3:
         raise ValueError("q and out must be contiguous [B, Hq, d] of equal shape")
+    B = q.shape[0]
+    _table_rows(block_tables, B)
+    _covers(ctx_lens, B, "ctx_lens")
+    _covers(err_flag, 1, "err_flag")
 
 
 def pa_decode(out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
@@ -282,6 +315,7 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
     B, Hq, dq = q.shape
     if dq != d:
         raise ValueError("q head_dim differs from the pool's")
+    _one_device(k_cache, out, q, v_cache, block_tables, ctx_lens, err_flag, workspace)
     bt = block_tables.contiguous()
     ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel() *
                                                         workspace.element_size())
@@ -306,6 +340,7 @@ def pa_decode_static_scratch(out, q, k_cache, v_cache, block_tables, ctx_lens, s
     B, Hq, dq = q.shape
     if dq != d:
         raise ValueError("q head_dim differs from the pool's")
+    _one_device(k_cache, out, q, v_cache, block_tables, ctx_lens, err_flag)
     bt = block_tables.contiguous()
     rc = load().pa_decode_static_scratch(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), stride,
                                          _ptr(bt), bt.shape[1], _ptr(ctx_lens.contiguous()), B, Hq,
@@ -330,6 +365,8 @@ def pa_decode_int8(out, q, kq_cache, vq_cache, k_scale, v_scale, block_tables, c
     B, Hq, dq = q.shape
     if dq != d:
         raise ValueError("q head_dim differs from the pool's")
+    _one_device(kq_cache, out, q, vq_cache, k_scale, v_scale, block_tables, ctx_lens, err_flag,
+                workspace)
     bt = block_tables.contiguous()
     ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel() *
                                                         workspace.element_size())
@@ -355,6 +392,9 @@ def pe_score_tokens(scores, k_cache, v_cache, block_tables, ctx_lens, err_flag, 
     B, MB = bt.shape
     if tuple(scores.shape) != (B, MB * bs, Hkv) or not scores.is_contiguous():
         raise ValueError("scores must be contiguous [B, MB*bs, Hkv]")
+    _covers(ctx_lens, B, "ctx_lens")
+    _covers(err_flag, 1, "err_flag")
+    _one_device(k_cache, scores, v_cache, block_tables, ctx_lens, err_flag)
     rc = load().pe_score_tokens(_ptr(scores), _ptr(k_cache), _ptr(v_cache), stride, _ptr(bt), MB,
                                 _ptr(ctx_lens.contiguous()), B, Hkv, d, bs, N, _ptr(err_flag),
                                 _stream(stream))
@@ -374,6 +414,9 @@ def pe_select_evict_block(evict, scores, ctx_lens, bs, block_means=None, stream=
         _want(block_means, torch.float32, "block_means")
         if tuple(block_means.shape) != (B, MB) or not block_means.is_contiguous():
             raise ValueError("block_means must be contiguous [B, MB]")
+    _covers(evict, B, "evict")
+    _covers(ctx_lens, B, "ctx_lens")
+    _one_device(scores, evict, ctx_lens, block_means)
     rc = load().pe_select_evict_block(_ptr(evict), _ptr(block_means), _ptr(scores.contiguous()),
                                       _ptr(ctx_lens.contiguous()), B, MB, Hkv, bs,
                                       _stream(stream))
@@ -404,8 +447,8 @@ def pa_append_kv_scored(k_new, v_new, k_cache, v_cache, score_pool, block_tables
     if not (k_new.is_contiguous() and v_new.is_contiguous()) or k_new.shape != v_new.shape:
         raise ValueError("k_new/v_new must be contiguous and of equal shape")
     B, n_new = k_new.shape[0], k_new.shape[1]
-    if slot_out is not None:
-        _want(slot_out, torch.int64, "slot_out")
+    _append_sizes(k_new, Hkv, d, block_tables, positions, err_flag, slot_out, B, n_new)
+    _one_device(k_cache, k_new, v_new, score_pool, block_tables, positions, err_flag, slot_out)
     bt = block_tables.contiguous()
     rc = load().pa_append_kv_scored(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
                                     stride, _ptr(score_pool), _ptr(bt), bt.shape[1],
@@ -438,8 +481,9 @@ def pa_append_kv_int8_scored(k_new, v_new, kq_cache, vq_cache, k_scale, v_scale,
     if not (k_new.is_contiguous() and v_new.is_contiguous()) or k_new.shape != v_new.shape:
         raise ValueError("k_new/v_new must be contiguous and of equal shape")
     B, n_new = k_new.shape[0], k_new.shape[1]
-    if slot_out is not None:
-        _want(slot_out, torch.int64, "slot_out")
+    _append_sizes(k_new, Hkv, d, block_tables, positions, err_flag, slot_out, B, n_new)
+    _one_device(kq_cache, k_new, v_new, k_scale, v_scale, score_pool, block_tables, positions,
+                err_flag, slot_out)
     bt = block_tables.contiguous()
     rc = load().pa_append_kv_int8_scored(_ptr(k_new), _ptr(v_new), _ptr(kq_cache),
                                          _ptr(vq_cache), _ptr(k_scale), _ptr(v_scale),
@@ -467,6 +511,10 @@ def pe_select_evict_block_pooled(evict, score_pool, block_tables, ctx_lens, err_
         _want(block_means, torch.float32, "block_means")
         if tuple(block_means.shape) != (B, MB) or not block_means.is_contiguous():
             raise ValueError("block_means must be contiguous [B, MB]")
+    _covers(evict, B, "evict")
+    _covers(ctx_lens, B, "ctx_lens")
+    _covers(err_flag, 1, "err_flag")
+    _one_device(score_pool, evict, block_tables, ctx_lens, err_flag, block_means)
     rc = load().pe_select_evict_block_pooled(_ptr(evict), _ptr(block_means), _ptr(score_pool),
                                              _ptr(bt), MB, _ptr(ctx_lens.contiguous()), B, Hkv,
                                              bs, N, _ptr(err_flag), _stream(stream))
@@ -492,8 +540,8 @@ def pa_append_kv_fp8(k_new, v_new, k8_cache, v8_cache, block_tables, positions, 
     if not (k_new.is_contiguous() and v_new.is_contiguous()) or k_new.shape != v_new.shape:
         raise ValueError("k_new/v_new must be contiguous and of equal shape")
     B, n_new = k_new.shape[0], k_new.shape[1]
-    if slot_out is not None:
-        _want(slot_out, torch.int64, "slot_out")
+    _append_sizes(k_new, Hkv, d, block_tables, positions, err_flag, slot_out, B, n_new)
+    _one_device(k8_cache, k_new, v_new, block_tables, positions, err_flag, slot_out)
     bt = block_tables.contiguous()
     rc = load().pa_append_kv_fp8(_ptr(k_new), _ptr(v_new), _ptr(k8_cache), _ptr(v8_cache), stride,
                                  _ptr(bt), bt.shape[1], _ptr(positions.contiguous()), B, n_new,
@@ -512,6 +560,7 @@ def pa_decode_fp8(out, q, k8_cache, v8_cache, block_tables, ctx_lens, scale, err
     B, Hq, dq = q.shape
     if dq != d:
         raise ValueError("q head_dim differs from the pool's")
+    _one_device(k8_cache, out, q, v8_cache, block_tables, ctx_lens, err_flag, workspace)
     bt = block_tables.contiguous()
     ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel() *
                                                         workspace.element_size())
@@ -554,6 +603,9 @@ def pe_prefill_select(keep_idx, kept_len, scores, cu_seqlens, err_flag, stream=N
     B, budget = keep_idx.shape
     if not keep_idx.is_contiguous() or cu_seqlens.numel() != B + 1:
         raise ValueError("keep_idx must be contiguous [B, budget] and cu_seqlens [B+1]")
+    _covers(kept_len, B, "kept_len")
+    _covers(err_flag, 1, "err_flag")
+    _one_device(scores, keep_idx, kept_len, cu_seqlens, err_flag)
     _check("pe_prefill_select", load().pe_prefill_select(
         _ptr(keep_idx), _ptr(kept_len), _ptr(scores), _ptr(cu_seqlens.contiguous()), B, budget,
         _ptr(err_flag), _stream(stream)))
@@ -570,7 +622,17 @@ def pe_prefill_pack(k_cache, v_cache, block_tables, k, v, cu_seqlens, keep_idx, 
     if (Hkv_c, d_c) != (Hkv, d):
         raise ValueError("prompt rows and pool differ in Hkv or d")
     _want(block_tables, torch.int32, "block_tables")
+    _want(cu_seqlens, torch.int32, "cu_seqlens")
+    _want(keep_idx, torch.int32, "keep_idx")
+    _want(kept_len, torch.int32, "kept_len")
+    _want(err_flag, torch.int32, "err_flag")
     B, budget = keep_idx.shape
+    if cu_seqlens.numel() != B + 1:
+        raise ValueError("cu_seqlens must hold B + 1 offsets")
+    _table_rows(block_tables, B)
+    _covers(kept_len, B, "kept_len")
+    _covers(err_flag, 1, "err_flag")
+    _one_device(k_cache, v_cache, block_tables, k, v, cu_seqlens, keep_idx, kept_len, err_flag)
     bt = block_tables.contiguous()
     _check("pe_prefill_pack", load().pe_prefill_pack(
         _ptr(k_cache), _ptr(v_cache), stride, _ptr(bt), bt.shape[1], _ptr(k), _ptr(v),
@@ -597,6 +659,11 @@ def pe_prefill_compress(k_cache, v_cache, block_tables, k, v, cu_seqlens, scores
     B, budget = keep_idx.shape
     if scores.numel() < T or not keep_idx.is_contiguous() or cu_seqlens.numel() != B + 1:
         raise ValueError("scores [T], keep_idx contiguous [B, budget], cu_seqlens [B+1]")
+    _table_rows(block_tables, B)
+    _covers(kept_len, B, "kept_len")
+    _covers(err_flag, 1, "err_flag")
+    _one_device(k_cache, v_cache, block_tables, k, v, cu_seqlens, scores, keep_idx, kept_len,
+                err_flag)
     bt = block_tables.contiguous()
     _check("pe_prefill_compress", load().pe_prefill_compress(
         _ptr(k_cache), _ptr(v_cache), stride, _ptr(bt), bt.shape[1], _ptr(k), _ptr(v),
@@ -618,6 +685,12 @@ def pe_evict_compact(block_tables, ctx_lens, evict, block_size, err_flag, freed=
     if freed is not None:
         _want(freed, torch.int32, "freed")
     B, MB = block_tables.shape
+    _covers(ctx_lens, B, "ctx_lens")
+    _covers(evict, B, "evict")
+    _covers(err_flag, 1, "err_flag")
+    if freed is not None:
+        _covers(freed, B, "freed")
+    _one_device(block_tables, ctx_lens, evict, err_flag, freed)
     _check("pe_evict_compact", load().pe_evict_compact(
         _ptr(block_tables), MB, _ptr(ctx_lens), _ptr(freed), _ptr(evict.contiguous()), B,
         int(block_size), _ptr(err_flag), _stream(stream)))
@@ -638,6 +711,11 @@ def pe_select_evict_threshold(mask, count, scores, ctx_lens, block_size, used_bl
         raise ValueError("scores must be [B, MB*bs, Hkv] and mask contiguous [B, MB]")
     if block_means is not None:
         _want(block_means, torch.float32, "block_means")
+        if tuple(block_means.shape) != (B, MB) or not block_means.is_contiguous():
+            raise ValueError("block_means must be contiguous [B, MB]")
+    _covers(count, B, "count")
+    _covers(ctx_lens, B, "ctx_lens")
+    _one_device(scores, mask, count, ctx_lens, block_means)
     _check("pe_select_evict_threshold", load().pe_select_evict_threshold(
         _ptr(mask), _ptr(count), _ptr(block_means), _ptr(scores.contiguous()),
         _ptr(ctx_lens.contiguous()), B, MB, Hkv, int(block_size), int(used_blocks),
@@ -661,6 +739,9 @@ def pe_evict_compact_mask(block_tables, ctx_lens, mask, block_size, err_flag, fr
         _want(freed, torch.int32, "freed")
         if tuple(freed.shape) != (B, MB) or not freed.is_contiguous():
             raise ValueError("freed must be contiguous [B, MB]")
+    _covers(ctx_lens, B, "ctx_lens")
+    _covers(err_flag, 1, "err_flag")
+    _one_device(block_tables, ctx_lens, mask, err_flag, freed)
     _check("pe_evict_compact_mask", load().pe_evict_compact_mask(
         _ptr(block_tables), MB, _ptr(ctx_lens), _ptr(freed), _ptr(mask.contiguous()), B,
         int(block_size), _ptr(err_flag), _stream(stream)))
@@ -705,6 +786,10 @@ def pa_prefill_attention(out, q, cu_q, max_q_len, k_cache, v_cache, block_tables
     B = block_tables.shape[0]
     if cu_q.numel() != B + 1:
         raise ValueError("cu_q must hold B + 1 offsets")
+    _table_rows(block_tables, B)
+    _covers(ctx_lens, B, "ctx_lens")
+    _covers(err_flag, 1, "err_flag")
+    _one_device(k_cache, out, q, cu_q, v_cache, block_tables, ctx_lens, err_flag, workspace)
     bt = block_tables.contiguous()
     _check("pa_prefill_attention", load().pa_prefill_attention(
         _ptr(out), _ptr(q), _ptr(cu_q.contiguous()), int(max_q_len), _ptr(k_cache),
