@@ -587,6 +587,7 @@ def pe_prefill_scores(scores, k, v, stream=None):
     _want(scores, torch.float32, "scores")
     if scores.numel() < T or not scores.is_contiguous():
         raise ValueError("scores: expected a contiguous float32 tensor of T elements")
+    _one_device(k, v, scores)
     _check("pe_prefill_scores", load().pe_prefill_scores(_ptr(scores), _ptr(k), _ptr(v), T, Hkv,
                                                          d, _stream(stream)))
 
