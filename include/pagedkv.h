@@ -38,7 +38,9 @@
  *     offending block or sequence.
  *   - Supported sizes: d in {64, 128}; Hq % Hkv == 0 with G = Hq/Hkv <= 16;
  *     bs >= 1 (bs a multiple of 16 selects the staged tensor-core decode);
- *     pool/base pointers 16-byte aligned and block_stride*elt a multiple of 16.
+ *     pool/base pointers 16-byte aligned and block_stride*elt a multiple of 16;
+ *     B <= 65535 and Hkv <= 65535 (grid limits), N <= 2^31 - 1 and
+ *     MB*bs <= 2^31 - 1 (token positions are int32).  Outside these: PA_ERR_SHAPE.
  */
 #ifndef PAGEDKV_H
 #define PAGEDKV_H

@@ -71,6 +71,14 @@ def test_decode_rejects_bad_arguments_on_host(lib):
     assert _decode(lib, k=ODD) == -3
     assert _decode(lib, stride=16 * 8 * 128 + 4) == -3  # stride not a multiple of 16 bytes
     assert _decode(lib, B=0) == 0               # empty batch: nothing to do
+    # the documented maximum sizes
+    assert _decode(lib, B=65536) == -2
+    assert _decode(lib, Hq=65536 * 2, Hkv=65536) == -2
+    assert _decode(lib, N=1 << 31) == -2
+    assert _decode(lib, MB=(1 << 27) + 1, bs=16) == -2   # MB*bs > 2^31 - 1
+    # the largest accepted sizes pass the shape checks and stop at the missing workspace
+    # (-4) on a GPU machine, or at the device query (-5 / -6) without one: never a launch
+    assert _decode(lib, B=65535, MB=(1 << 27) - 1) in (-4, -5, -6)
 
 
 def test_append_and_score_reject_bad_arguments_on_host(lib):
