@@ -25,6 +25,9 @@
  *     legacy default stream) and returns after enqueueing.
  *   - Return value: PA_OK (0) when the work was enqueued; a negative PA_ERR_*
  *     code when an argument is invalid, in which case nothing is launched.
+ *     Every call checks its arguments before any CUDA call (its "Host errors"
+ *     line lists them); after that, PA_ERR_DEVICE when the current device is
+ *     not an sm_100 GPU and PA_ERR_CUDA when a runtime call or launch fails.
  *   - bf16 tensors are passed as uint16_t bit patterns.
  *   - Physical KV pool of one layer: [N blocks][bs slots][Hkv heads][d],
  *     element (blk, slot, h, e) at blk*block_stride + (slot*Hkv + h)*d + e,
@@ -88,6 +91,10 @@ const char *pa_version(void);
  *   slot_out     : optional [B][n_new] int64, receives the slots (NULL = skip).
  * Device errors: p outside [0, MB*bs) -> PA_DEV_BAD_LEN; table entry outside
  * [0, N) -> PA_DEV_BAD_BLOCK; that token is skipped.
+ * Host errors: B = 0 or n_new = 0 -> PA_OK (nothing to do); a NULL k_new, v_new,
+ * pool, table, positions or err_flag -> PA_ERR_NULL; n_new < 0 or sizes outside
+ * the supported ranges -> PA_ERR_SHAPE; k_new, v_new or a pool not 16-byte
+ * aligned, or block_stride*2 not a multiple of 16 -> PA_ERR_ALIGN.
  * ==========================================================================*/
 int pa_append_kv(const uint16_t *k_new, const uint16_t *v_new,
                  uint16_t *k_cache, uint16_t *v_cache, int64_t block_stride,
@@ -115,6 +122,14 @@ int pa_append_kv(const uint16_t *k_new, const uint16_t *v_new,
  *                must be ordered on one stream.
  * Device errors: ctx_lens[b] outside [0, MB*bs] -> PA_DEV_BAD_LEN (row zeroed);
  * a needed table entry outside [0, N) -> PA_DEV_BAD_BLOCK (block skipped).
+ * Host errors: B = 0 -> PA_OK; a NULL out, q, pool, table, ctx_lens or err_flag
+ * -> PA_ERR_NULL; Hq not a positive multiple of Hkv, G > 16, a NaN scale or sizes
+ * outside the supported ranges -> PA_ERR_SHAPE; out, q, a pool or the workspace not
+ * 16-byte aligned, or block_stride*2 not a multiple of 16 -> PA_ERR_ALIGN; the
+ * workspace NULL or smaller than pa_decode_workspace_bytes when that is > 0 ->
+ * PA_ERR_WORKSPACE.  pa_decode_workspace_bytes returns 0 for invalid sizes;
+ * pa_decode_plan returns PA_ERR_NULL for a NULL num_splits_out or
+ * chunk_tokens_out and PA_ERR_SHAPE for invalid sizes.
  * ==========================================================================*/
 size_t pa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int bs,
                                  int max_blocks_per_seq, int num_splits);
@@ -148,6 +163,11 @@ int pa_decode(uint16_t *out, const uint16_t *q,
  * ||K|| == 0 the score is +inf if ||V|| > 0, else 0.  Entries with
  * t >= ctx_lens[b] are not written.
  *   scores : [B][MB*bs][Hkv] fp32.
+ * Device errors: ctx_lens[b] outside [0, MB*bs] -> PA_DEV_BAD_LEN (sequence
+ * skipped); a table entry outside [0, N) -> PA_DEV_BAD_BLOCK (block skipped).
+ * Host errors: B = 0 -> PA_OK; a NULL scores, pool, table, ctx_lens or err_flag ->
+ * PA_ERR_NULL; sizes outside the supported ranges -> PA_ERR_SHAPE; a pool not
+ * 16-byte aligned or block_stride*2 not a multiple of 16 -> PA_ERR_ALIGN.
  * ==========================================================================*/
 int pe_score_tokens(float *scores, const uint16_t *k_cache, const uint16_t *v_cache,
                     int64_t block_stride, const int32_t *block_tables, int max_blocks_per_seq,
@@ -167,6 +187,9 @@ int pe_score_tokens(float *scores, const uint16_t *k_cache, const uint16_t *v_ca
  *   block_means : optional [B][MB] fp32 (fp64 mean rounded to nearest); NaN for
  *                 non-candidate blocks.  NULL = skip.
  *   scores      : [B][MB*bs][Hkv] fp32 as written by pe_score_tokens.
+ * A length outside [0, MB*bs] counts as 0 (no full block: -1); there is no
+ * error flag.  Host errors: B = 0 -> PA_OK; a NULL evict, scores or ctx_lens ->
+ * PA_ERR_NULL; B < 0, MB < 1, Hkv < 1 or bs < 1 -> PA_ERR_SHAPE.
  * ==========================================================================*/
 int pe_select_evict_block(int32_t *evict, float *block_means, const float *scores,
                           const int32_t *ctx_lens, int B, int max_blocks_per_seq, int Hkv,
@@ -181,6 +204,8 @@ int pe_select_evict_block(int32_t *evict, float *block_means, const float *score
  *   s == 0  ->  all codes 0.
  *   kq_cache, vq_cache : int8 pools [N][bs][Hkv][d] (block_stride elements).
  *   k_scale, v_scale   : fp32 scale pools [N][bs][Hkv] (block stride bs*Hkv).
+ * Host errors: as pa_append_kv, plus a NULL scale pool -> PA_ERR_NULL, and scale
+ * pools not 16-byte aligned or block_stride not a multiple of 16 -> PA_ERR_ALIGN.
  * ==========================================================================*/
 int pa_append_kv_int8(const uint16_t *k_new, const uint16_t *v_new,
                       int8_t *kq_cache, int8_t *vq_cache, float *k_scale, float *v_scale,
@@ -195,6 +220,8 @@ int pa_append_kv_int8(const uint16_t *k_new, const uint16_t *v_new,
  * dequantised in registers (the K scale multiplies the dot product, the V
  * scale multiplies the softmax weight).  Same workspace rule as pa_decode.
  * k_scale, v_scale: fp32 [N][bs][Hkv], 16-byte aligned (PA_ERR_ALIGN otherwise).
+ * Host errors: as pa_decode, plus a NULL scale pool -> PA_ERR_NULL and
+ * block_stride not a multiple of 16 -> PA_ERR_ALIGN.
  * ==========================================================================*/
 int pa_decode_int8(uint16_t *out, const uint16_t *q,
                    const int8_t *kq_cache, const int8_t *vq_cache,
@@ -215,6 +242,8 @@ int pa_decode_int8(uint16_t *out, const uint16_t *q,
  *   k8_cache, v8_cache : uint8 pools [N][bs][Hkv][d] (block_stride elements).
  * pa_decode_fp8: pa_decode over e4m3 pools; every code is widened exactly (each
  * e4m3 value is an fp16 value) in registers.  Same workspace rule as pa_decode.
+ * Host errors: as pa_append_kv and pa_decode, with block_stride (one-byte
+ * elements) a multiple of 16 -> else PA_ERR_ALIGN.
  * ==========================================================================*/
 int pa_append_kv_fp8(const uint16_t *k_new, const uint16_t *v_new,
                      uint8_t *k8_cache, uint8_t *v8_cache, int64_t block_stride,
@@ -248,6 +277,10 @@ int pa_decode_fp8(uint16_t *out, const uint16_t *q,
  * and precision, so it returns exactly what pe_select_evict_block returns on
  * the equal [B][MB*bs][Hkv] score array.  A needed table entry outside [0, N)
  * raises PA_DEV_BAD_BLOCK and that block is not a candidate.
+ * Host errors: the appends as pa_append_kv / pa_append_kv_int8, plus a NULL
+ * score_pool -> PA_ERR_NULL.  pe_select_evict_block_pooled: B = 0 -> PA_OK; a NULL
+ * evict, score_pool, table, ctx_lens or err_flag -> PA_ERR_NULL; B outside
+ * [0, 65535], MB < 1, Hkv < 1, bs < 1 or N < 1 -> PA_ERR_SHAPE.
  * ==========================================================================*/
 int pa_append_kv_scored(const uint16_t *k_new, const uint16_t *v_new,
                         uint16_t *k_cache, uint16_t *v_cache, int64_t block_stride,
@@ -290,6 +323,8 @@ int pe_select_evict_block_pooled(int32_t *evict, float *block_means, const float
  *   on the GPU (different streams, or different host threads) race and give
  *   wrong results; order them on one stream.  Nothing in the array needs to
  *   start at zero: every call writes what it later reads.
+ * Host errors: as pa_decode without the workspace ones, plus num_splits < 0 ->
+ * PA_ERR_SHAPE and scratch that does not fit -> PA_ERR_WORKSPACE.
  * ==========================================================================*/
 #define PA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 
@@ -333,6 +368,19 @@ int pa_decode_static_scratch(uint16_t *out, const uint16_t *q,
  * pe_prefill_compress: pe_prefill_scores, pe_prefill_select and
  *   pe_prefill_pack in one call (three launches on `stream`); scores,
  *   keep_idx and kept_len are outputs the caller may read afterwards.
+ *
+ * Host errors: pe_prefill_scores: T = 0 -> PA_OK; a NULL scores, k or v ->
+ *   PA_ERR_NULL; T < 0, Hkv outside [1, 65535] or d not in {64, 128, 256} ->
+ *   PA_ERR_SHAPE; k or v not 16-byte aligned -> PA_ERR_ALIGN.
+ *   pe_prefill_select: B = 0 -> PA_OK; a NULL argument -> PA_ERR_NULL; B < 0 or
+ *   budget < 1 -> PA_ERR_SHAPE.
+ *   pe_prefill_pack: B = 0 -> PA_OK; a NULL pool, table, k, v, cu_seqlens,
+ *   keep_idx, kept_len or err_flag -> PA_ERR_NULL; Hkv or d as for
+ *   pe_prefill_scores, B < 0, budget < 1, bs < 1, MB < 1, N < 1 or
+ *   block_stride < bs*Hkv*d -> PA_ERR_SHAPE; pools, k or v not 16-byte
+ *   aligned, or block_stride*2 not a multiple of 16 -> PA_ERR_ALIGN.
+ *   pe_prefill_compress: the union of the three, checked before the first
+ *   launch (a NULL scores with T > 0 -> PA_ERR_NULL).
  * ==========================================================================*/
 int pe_prefill_scores(float *scores, const uint16_t *k, const uint16_t *v, int64_t T, int Hkv,
                       int d, void *stream);
@@ -366,6 +414,8 @@ int pe_prefill_compress(uint16_t *k_cache, uint16_t *v_cache, int64_t block_stri
  * cached rows and a score pool stay valid.  j not a full block (j >= len/bs)
  * sets PA_DEV_BAD_EVICT, a length outside [0, MB*bs] PA_DEV_BAD_LEN; the
  * sequence is left unchanged.  block_tables and ctx_lens are updated in place.
+ * Host errors: B = 0 -> PA_OK; a NULL block_tables, ctx_lens, evict or err_flag
+ * -> PA_ERR_NULL; B < 0, MB < 1, bs < 1 or MB*bs > 2^31 - 1 -> PA_ERR_SHAPE.
  * ==========================================================================*/
 int pe_evict_compact(int32_t *block_tables, int max_blocks_per_seq, int32_t *ctx_lens,
                      int32_t *freed, const int32_t *evict, int B, int bs, int32_t *err_flag,
@@ -396,6 +446,12 @@ int pe_evict_compact(int32_t *block_tables, int max_blocks_per_seq, int32_t *ctx
  *   freed (nullable [B][MB]) lists the removed physical ids in logical order,
  *   -1 after the last.  A mark on the partial last block sets
  *   PA_DEV_BAD_EVICT and is ignored; marks at j >= ceil(len/bs) are not read.
+ *
+ * Host errors: pe_select_evict_threshold: B = 0 -> PA_OK; a NULL mask, count,
+ *   scores or ctx_lens -> PA_ERR_NULL; B < 0, MB < 1, Hkv < 1, bs < 1, eviction_ratio
+ *   outside [0, 1] (or NaN), a NaN importance_threshold or a negative block
+ *   count -> PA_ERR_SHAPE.  pe_evict_compact_mask: as pe_evict_compact, with mask
+ *   in place of evict.
  * ==========================================================================*/
 int pe_select_evict_threshold(uint8_t *mask, int32_t *count, float *block_means,
                               const float *scores, const int32_t *ctx_lens, int B,
@@ -439,6 +495,11 @@ int pe_evict_compact_mask(int32_t *block_tables, int max_blocks_per_seq, int32_t
  *     rounding.
  * pa_prefill_attention_workspace_bytes returns 0 when the balanced mode does not
  * apply to these sizes (the call then needs no workspace).
+ * Host errors: B = 0 or max_q_len = 0 -> PA_OK; a NULL out, q, cu_q, pool, table,
+ * ctx_lens or err_flag -> PA_ERR_NULL; max_q_len < 0, Hq not a positive multiple
+ * of Hkv, G not a power of two up to 16, a NaN scale or sizes outside the
+ * supported ranges -> PA_ERR_SHAPE; out, q, a pool or the workspace not 16-byte
+ * aligned, or block_stride*2 not a multiple of 16 -> PA_ERR_ALIGN.
  * ==========================================================================*/
 size_t pa_prefill_attention_workspace_bytes(int B, int Hq, int Hkv, int d, int bs, int max_q_len);
 
