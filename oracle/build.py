@@ -12,11 +12,12 @@ SRC = os.path.join(HERE, "oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
 
-def compile_c(src: str, out: str) -> None:
-    """gcc one oracle source into a shared library at `out` (written atomically)."""
+def compile_c(src: str, out: str, extra=()) -> None:
+    """gcc one oracle source into a shared library at `out` (written atomically);
+    `extra` flags come last (e.g. -w for deliberately altered copies)."""
     cmd = [
         "gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-        "-fPIC", "-shared", "-Wall", "-Wextra", "-Wno-unused-parameter",
+        "-fPIC", "-shared", "-Wall", "-Wextra", "-Wno-unused-parameter", *extra,
         src, "-o", out + ".tmp", "-lm",
     ]
     subprocess.run(cmd, check=True)

@@ -188,7 +188,7 @@ def main(only) -> int:
             mlib = os.path.join(tmp, name + ".so")
             with open(msrc, "w") as f:
                 f.write(src.replace(find, repl))
-            oracle_build.compile_c(msrc, mlib)
+            oracle_build.compile_c(msrc, mlib, extra=("-w",))
             env = dict(os.environ, ORACLE_LIB=mlib)
             r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                                 os.path.join(HERE, "test_oracle_pins.py")],
