@@ -199,3 +199,42 @@ def test_e4m3_cast_is_torchs_in_range_and_saturates_beyond(log2_mag, seed):
     assert np.array_equal(codes[ok], ref.numpy())
     big = ~ok
     assert np.array_equal(codes[big], np.where(xv[big] > 0, 0x7e, 0xfe).astype(np.uint8))
+
+
+def _sdpa_rows(q, K, V, G, d):
+    Kt = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(G, 0)
+    Vt = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(G, 0)
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).unsqueeze(1), Kt, Vt, scale=1 / math.sqrt(d))[:, 0].numpy()
+
+
+@SETTINGS
+@given(paged_case(), st.sampled_from(["int8", "fp8"]))
+def test_quantised_decode_is_sdpa_on_the_stored_values(c, kind):
+    """INT8: the values are scale * code per (token, head) row; FP8: each e4m3 code's
+    exact value.  Either way the decode equals fp64 SDPA on those values."""
+    Hq, Hkv, d, bs = c["Hq"], c["Hkv"], c["d"], c["bs"]
+    stride = bs * Hkv * d
+    if kind == "int8":
+        kq, ks = oracle.quantize_int8(c["kc"])
+        vq, vs = oracle.quantize_int8(c["vc"])
+        out = oracle.paged_decode_int8(c["q"], kq.ravel(), vq.ravel(), ks.ravel(), vs.ravel(),
+                                       stride, c["bt"], c["lens"], Hkv, bs, 1 / math.sqrt(d))
+        kd = ks[..., None].astype(np.float64) * kq
+        vd = vs[..., None].astype(np.float64) * vq
+    else:
+        k8, v8 = oracle.quantize_e4m3(c["kc"]), oracle.quantize_e4m3(c["vc"])
+        out = oracle.paged_decode_fp8(c["q"], k8.ravel(), v8.ravel(), stride, c["bt"],
+                                      c["lens"], Hkv, bs, 1 / math.sqrt(d))
+        kd, vd = oracle.e4m3_values(k8), oracle.e4m3_values(v8)
+    q = vals(c["q"])
+    for b in range(c["B"]):
+        n = int(c["lens"][b])
+        if n == 0:
+            assert not out[b].any()
+            continue
+        ids = c["bt"][b, : -(-n // bs)]
+        K = kd[ids].reshape(-1, Hkv, d)[:n]
+        V = vd[ids].reshape(-1, Hkv, d)[:n]
+        np.testing.assert_allclose(out[b], _sdpa_rows(q[b], K, V, Hq // Hkv, d), rtol=1e-11,
+                                   atol=1e-12)
