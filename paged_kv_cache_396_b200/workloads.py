@@ -12,8 +12,8 @@ describe; all values bf16 ~ N(0, 1) unless stated):
                 (+1), bs=16, pool = 1.1 x blocks in use, shuffled.
   c3  Llama-3-8B shape: 32 layers, Hq=32, Hkv=8, d=128, B=64, old lens uniform
                 in [512, 8192] (+1), bs=16, pool = 1.1 x in use, shuffled; per
-                layer 1% of the Hkv*d channels (11 (head, channel) pairs) of K
-                and V scaled x8 as outliers.
+                layer 1% of the Hkv*d channels (10 of the 1024 (head, channel)
+                pairs, rounded) of K and V scaled x8 as outliers.
   c4  128K context: 1 layer, Hq=32, Hkv=8, d=128, B=4, len 131072 (no append),
                 bs=256, one tensor [2, L, N, 256, Hkv, d] (nano-vLLM layout), shuffled.
   c5  INT8 pool: 1 layer, Hq=64, Hkv=8, d=128, B=128, old len 4096 (+1), bs=16;
