@@ -69,6 +69,7 @@ extern "C" {
 #define PA_DEV_BAD_LEN    2  /* a context length / position outside [0, MB*bs]     */
 #define PA_DEV_TIMEOUT    4  /* a bounded pipeline wait gave up (kernel returned)   */
 #define PA_DEV_BAD_EVICT  8  /* an eviction index that is not a full block          */
+#define PA_DEV_BAD_PLAN  16  /* the workspace holds no plan for these sizes         */
 
 /* Human-readable text of a PA_* status code (static storage). */
 const char *pa_status_string(int code);
@@ -220,6 +221,14 @@ int pa_append_kv_int8(const uint16_t *k_new, const uint16_t *v_new,
  * dequantised in registers (the K scale multiplies the dot product, the V
  * scale multiplies the softmax weight).  Same workspace rule as pa_decode.
  * k_scale, v_scale: fp32 [N][bs][Hkv], 16-byte aligned (PA_ERR_ALIGN otherwise).
+ * The query stays bf16 (the page quantises the cache only).  With d = 128 and
+ * bs a multiple of 16 the dot products q.kq run on int8 tensor cores: each
+ * query row is scaled by a power of two, rounded to integers of magnitude at
+ * most 8355711 (23 bits) and split exactly into three int8 parts, so the one
+ * approximation is that rounding, below 2^-23 of the row's largest |q| per
+ * element (rows whose largest |q| is at least 2^-104).  Other shapes compute
+ * in fp32 from the bf16 query.  Any finite bf16 query whose logits are finite
+ * in fp32 is valid.
  * Host errors: as pa_decode, plus a NULL scale pool -> PA_ERR_NULL and
  * block_stride not a multiple of 16 -> PA_ERR_ALIGN.
  * ==========================================================================*/
@@ -242,6 +251,12 @@ int pa_decode_int8(uint16_t *out, const uint16_t *q,
  *   k8_cache, v8_cache : uint8 pools [N][bs][Hkv][d] (block_stride elements).
  * pa_decode_fp8: pa_decode over e4m3 pools; every code is widened exactly (each
  * e4m3 value is an fp16 value) in registers.  Same workspace rule as pa_decode.
+ * With d = 128 and bs a multiple of 16 the products run on fp16 tensor cores:
+ * each bf16 query row is first scaled by a power of two that puts its largest
+ * |q| in [2^14, 2^15), so no query overflows fp16 (|q| > 65504 included) and
+ * every element down to 2^-32 of the row's largest converts exactly; the scale
+ * is taken back on the logit.  Any finite bf16 query whose logits are finite
+ * in fp32 is valid.
  * Host errors: as pa_append_kv and pa_decode, with block_stride (one-byte
  * elements) a multiple of 16 -> else PA_ERR_ALIGN.
  * ==========================================================================*/
@@ -257,6 +272,61 @@ int pa_decode_fp8(uint16_t *out, const uint16_t *q,
                   int B, int Hq, int Hkv, int d, int bs, int64_t num_blocks, float scale,
                   int num_splits, void *workspace, size_t workspace_bytes,
                   int32_t *err_flag, void *stream);
+
+/* ============================================================================
+ * One partition plan for several decode calls (no counterpart in the pages:
+ * the split-KV partition exists only in this implementation).
+ *
+ * The staged decode's plan (every sequence's partitions, listed longest first)
+ * depends only on ctx_lens and the sizes, which are the same for every layer of
+ * a decode step.  pa_decode_prepare writes that plan into a workspace (one plan
+ * launch); pa_decode_planned, pa_decode_int8_planned and pa_decode_fp8_planned
+ * are pa_decode, pa_decode_int8 and pa_decode_fp8 taking the plan from the
+ * workspace instead of making it, so each call launches one kernel fewer.  Their
+ * arguments are those of the plain calls, and their results are bit for bit the
+ * same, provided that
+ *   - pa_decode_prepare ran on this workspace, ordered before the call on the
+ *     same stream, with the same ctx_lens contents and the same B, Hq, Hkv, d,
+ *     bs, max_blocks_per_seq and num_splits, and
+ *   - no plain pa_decode* call and no other pa_decode_prepare used the workspace
+ *     in between (a planned call leaves the plan ready for the next one).
+ * One plan serves bf16, INT8 and FP8 calls of the same sizes.  The plan records
+ * a signature of its sizes: a planned call of other sizes computes nothing,
+ * raises PA_DEV_BAD_PLAN and leaves out untouched.  Changed ctx_lens contents are
+ * not detected (the call then attends the ranges of the old lengths, reading
+ * only table entries below max_blocks_per_seq): prepare again after a change.
+ * Shapes served by the general-shape kernel keep no plan: pa_decode_prepare
+ * launches nothing and the planned calls run as the plain ones.
+ * Host errors: pa_decode_prepare: B = 0 -> PA_OK; a NULL ctx_lens or err_flag ->
+ * PA_ERR_NULL; sizes outside the supported ranges -> PA_ERR_SHAPE; the workspace
+ * NULL or smaller than pa_decode_workspace_bytes -> PA_ERR_WORKSPACE, not 16-byte
+ * aligned -> PA_ERR_ALIGN.  The planned calls: as the plain ones.
+ * ==========================================================================*/
+int pa_decode_prepare(const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
+                      int max_blocks_per_seq, int num_splits, void *workspace,
+                      size_t workspace_bytes, int32_t *err_flag, void *stream);
+
+int pa_decode_planned(uint16_t *out, const uint16_t *q,
+                      const uint16_t *k_cache, const uint16_t *v_cache, int64_t block_stride,
+                      const int32_t *block_tables, int max_blocks_per_seq,
+                      const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
+                      int64_t num_blocks, float scale, int num_splits, void *workspace,
+                      size_t workspace_bytes, int32_t *err_flag, void *stream);
+
+int pa_decode_int8_planned(uint16_t *out, const uint16_t *q,
+                           const int8_t *kq_cache, const int8_t *vq_cache,
+                           const float *k_scale, const float *v_scale, int64_t block_stride,
+                           const int32_t *block_tables, int max_blocks_per_seq,
+                           const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
+                           int64_t num_blocks, float scale, int num_splits, void *workspace,
+                           size_t workspace_bytes, int32_t *err_flag, void *stream);
+
+int pa_decode_fp8_planned(uint16_t *out, const uint16_t *q,
+                          const uint8_t *k8_cache, const uint8_t *v8_cache, int64_t block_stride,
+                          const int32_t *block_tables, int max_blocks_per_seq,
+                          const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
+                          int64_t num_blocks, float scale, int num_splits, void *workspace,
+                          size_t workspace_bytes, int32_t *err_flag, void *stream);
 
 /* ============================================================================
  * Incremental PagedEviction scoring  ([KVL] "PagedEviction 块级驱逐机制": the
@@ -309,16 +379,22 @@ int pe_select_evict_block_pooled(int32_t *evict, float *block_means, const float
  * manager owns every byte of the GPU and forbids raw allocations, a plain-C
  * caller that holds only device pointers handed to it, or a process that has
  * reserved its whole memory budget at start-up.  For them this entry point
- * computes exactly what pa_decode computes, with the same arguments minus the
+ * computes what pa_decode computes, with the same arguments minus the
  * workspace, and takes its scratch from a fixed array that lives inside the
  * library: PA_STATIC_SCRATCH_BYTES (16 MiB) on every GPU that loads the library,
  * held until the process exits.  It allocates nothing.
- *   num_splits : as pa_decode, except that 0 picks the largest partition count
- *                whose scratch fits the array.  When the scratch needed for the
- *                given sizes (and a non-zero num_splits) exceeds the array, the
- *                call returns PA_ERR_WORKSPACE and launches nothing.
- *   The first call on each device looks up the array's device address with the
- *   device current; make that first call before any stream capture.
+ *   num_splits : as pa_decode when the scratch of that plan fits the array (then
+ *                the call launches exactly what pa_decode launches, bit for bit
+ *                the same result).  When num_splits = 0 and the automatic plan's
+ *                scratch does not fit, the call takes the largest partition count
+ *                whose scratch fits (so it may partition, and round, differently
+ *                from pa_decode).  When the scratch needed for the given sizes
+ *                and a non-zero num_splits exceeds the array, the call returns
+ *                PA_ERR_WORKSPACE and launches nothing.
+ *   Every call looks up the array's device address with the calling device
+ *   current (a host-side lookup that allocates nothing and follows a reset
+ *   context).  The first call on a device may load the library's device code:
+ *   make it before any stream capture.
  *   All calls on a device share the one array: two calls whose kernels overlap
  *   on the GPU (different streams, or different host threads) race and give
  *   wrong results; order them on one stream.  Nothing in the array needs to

@@ -27,6 +27,42 @@ __device__ __forceinline__ double warp_block_mean(const float *__restrict__ p, i
     return s / (double)per;
 }
 
+// The means of up to four blocks at once (p[i] == nullptr: block i skipped, its
+// out[i] untouched; at least one p[i] is set), each with exactly the arithmetic of
+// warp_block_mean (the same values, bit for bit); the four blocks' loads are in
+// flight together.
+__device__ __forceinline__ void warp_block_mean4(const float *const (&p)[4], int per, int lane,
+                                                 double (&out)[4]) {
+    // skipped blocks read a set block's scores (their sums are discarded)
+    const float *any = p[0] ? p[0] : p[1] ? p[1] : p[2] ? p[2] : p[3];
+    double s[4] = {0.0, 0.0, 0.0, 0.0};
+    int k = lane;
+    for (; k + 96 < per; k += 128) {
+        float a[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float *q = p[i] ? p[i] : any;
+            a[i][0] = __ldg(q + k);
+            a[i][1] = __ldg(q + k + 32);
+            a[i][2] = __ldg(q + k + 64);
+            a[i][3] = __ldg(q + k + 96);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            s[i] += ((double)a[i][0] + (double)a[i][1]) + ((double)a[i][2] + (double)a[i][3]);
+    }
+    for (; k < per; k += 32) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s[i] += (double)__ldg((p[i] ? p[i] : any) + k);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s[i] += __shfl_xor_sync(0xffffffffu, s[i], o);
+        if (p[i]) out[i] = s[i] / (double)per;
+    }
+}
+
 // (mean, j) argmin with ties to the lowest j; j = INT_MAX marks "none".
 __device__ __forceinline__ void argmin_take(double &best, int &bj, double m, int j) {
     if (j != INT_MAX && (bj == INT_MAX || m < best || (m == best && j < bj))) {

@@ -282,6 +282,9 @@ DecodePlan make_decode_plan(int B, int Hq, int Hkv, int d, int bs, int MB, int n
             tpw *= 2;  // doubling keeps the stage (K + V of n_sub sub-tiles) within 64 KB
         p.tpw = tpw;
         p.n_sub = p.wph * tpw;
+        // the INT8 and FP8 consumers take a warp's sub-tiles of a stage as one pair
+        // (the doubling above gives one-byte pools exactly two)
+        if (onebyte && tpw > 2) tc = false;
         const int kv_bytes = p.n_sub * sub_kv;
         const int sc_bytes = p.n_sub * sub_sc;
         p.v_off = kv_bytes;
@@ -311,6 +314,16 @@ DecodePlan make_decode_plan(int B, int Hq, int Hkv, int d, int bs, int MB, int n
         p.off_ml = p.off_units + up256((size_t)B * p.S * 16);
         p.off_acc = p.off_ml + up256(slots * 2 * 4);
         p.ws_total = p.off_acc + up256(slots * d * 4);
+        // sizes the device plan depends on (a plan kept in a workspace is only used by
+        // calls of the same signature): FNV-1a over them.  The element type is not
+        // among them: bf16, INT8 and FP8 calls of the same sizes share one plan.
+        const long long f[10] = {B, Hq, Hkv, d, bs, MB, p.S, p.chunk, p.grid, p.units_per_cta};
+        unsigned long long h = 1469598103934665603ull;
+        for (long long v : f) {
+            h ^= (unsigned long long)v;
+            h *= 1099511628211ull;
+        }
+        p.sig = h | 1ull;  // never 0 (a zeroed workspace holds no plan)
         return p;
     }
     // general-shape kernel: fixed partitions of `chunk` tokens

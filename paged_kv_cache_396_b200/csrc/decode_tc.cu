@@ -85,6 +85,7 @@ struct Args {
     int n_sub;      // sub-tiles per stage (wph * tpw)
     int tpb_shift;  // log2(bs / 16) when bs / 16 is a power of two, else -1
     float scale_log2;
+    unsigned long long sig;  // signature of the sizes; must match the plan's (header)
 };
 
 // ---------------------------------------------------------------------------
@@ -92,7 +93,8 @@ struct Args {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *ctx_lens, int32_t *err,
                                                    TcHeader *hdr, int32_t *ns, int4 *units, int B,
-                                                   int max_ctx, int min_chunk, int target_units) {
+                                                   int max_ctx, int min_chunk, int target_units,
+                                                   unsigned long long sig) {
     constexpr int kSerialParts = 32, kMaxLong = 256;
     __shared__ long long s_red[32];
     __shared__ int hist[1024];
@@ -192,6 +194,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *ctx_lens, int
         if (tid == 1023) {
             hdr->n_units = before + inc;
             hdr->counter = 0u;
+            hdr->done = 0u;
+            hdr->sig = sig;
         }
     }
     __syncthreads();
@@ -240,11 +244,15 @@ __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensor
     const uint32_t sc_bytes = (uint32_t)kTile * a.Hkv * 4;  // one sub-tile's scale rows
     const uint32_t sub_bytes = 2u * DC * (uint32_t)a.box_bytes + (I8 ? 2u * sc_bytes : 0u);
     const int tpb = a.bs / kTile;                            // 16-token tiles per block
-    const int n_units = a.hdr->n_units;
+    // a plan made for other sizes (a kept plan that does not match this call) is
+    // not used: no unit is taken and the call flags it
+    const bool plan_ok = a.hdr->sig == a.sig;
+    const int n_units = plan_ok ? a.hdr->n_units : 0;
+    if (!plan_ok && lane == 0 && blockIdx.x == 0) raise_flag(a.err, PA_DEV_BAD_PLAN);
     const uint64_t policy = ptx::policy_evict_first();
     int stage = 0;
     uint32_t phase = 0;
-    bool ok = true;
+    bool ok = plan_ok;
     if (lane == 0) {
         ptx::prefetch_tensormap(kmap);
         ptx::prefetch_tensormap(vmap);
@@ -322,7 +330,7 @@ __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensor
             }
         }
     }
-    if (ok) {
+    if (ok || !plan_ok) {
         if (ptx::mbar_wait(&empty[stage], phase ^ 1u)) {
             if (lane == 0) {
                 meta[stage].flags = kEnd;
@@ -330,6 +338,16 @@ __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensor
             }
         } else if (lane == 0) {
             raise_flag(a.err, PA_DEV_TIMEOUT);
+        }
+    }
+    // this CTA takes no more units: the last CTA to get here resets the unit counter
+    // (every CTA's last fetch came before its increment), so the plan can serve the
+    // next decode call without the plan kernel
+    if (lane == 0 && plan_ok) {
+        __threadfence();
+        if (atomicAdd(&a.hdr->done, 1u) == gridDim.x - 1) {
+            atomicExch(&a.hdr->counter, 0u);
+            atomicExch(&a.hdr->done, 0u);
         }
     }
 }
@@ -652,24 +670,33 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
     return v;
 }
 
-// 8 bf16 (one uint4) -> 4 fp16x2
-__device__ __forceinline__ void bf16x8_to_f16x2(const uint4 &v, uint32_t *o) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = ptx::pack_f16(bf16_lo(w[i]), bf16_hi(w[i]));
+// Power of two 2^e (e clamped to [-126, 126], so 2^e and 2^-e are normal fp32
+// values) with x * 2^e in [2^top, 2^(top + 1)) for a normal x > 0, from the
+// exponent bits of x; a zero or subnormal x takes the clamp.
+__device__ __forceinline__ float pow2_scale_for(float x, int top) {
+    const int E = (int)((__float_as_uint(x) >> 23) & 0xffu) - 127;
+    const int e = max(-126, min(126, top - E));
+    return __uint_as_float((uint32_t)(e + 127) << 23);
 }
 
-// Query fragments of the INT8 consumer as exact int8 pairs for the s8 MMA.
-// Row g of the group is scaled by a power of two 2^e so that max|q| * 2^e <=
-// 16256, rounded to an integer q' (|q'| < 2^14) and split exactly into
-// q' = 128 * hi + lo with hi in [-127, 127], lo in [-64, 63]; then
-// q.k = (128 * (hi.k) + lo.k) / 2^e with both dot products exact in int32.
+// Query fragments of the INT8 consumer as int8 parts for the s8 MMA.
+// Row g of the group is scaled by a power of two 2^e so that max|q| * 2^e lies
+// in (L/2, L] with L = 8355711 = 127*65536 + 127*256 + 127, rounded to an
+// integer q' (|q'| <= L) and split exactly into q' = 65536*hi + 256*mid + lo
+// with hi in [-127, 127] and mid, lo in [-128, 127]; then
+//   q'.k = 65536*(hi.k) + 256*(mid.k) + lo.k
+// with the three dot products exact in int32.  The only approximation is the
+// rounding q -> q' / 2^e: at most 1/(2 * 2^e) < max|q| / L (about 2^-23 of the
+// row's largest element) per element, for rows whose largest element is at
+// least 2^-104 (smaller rows take the scale 2^126).
 // k-step kk (32 dims) of thread (g, tig) uses dims 16*tig + 4*kk + 0..3 (a0/a1)
 // and 16*(tig + 4) + 4*kk + 0..3 (a2/a3), matching the K words it loads.
-// Returns 1 / 2^e (0 for an all-zero or absent row).
+// Returns 1 / 2^e.
 __device__ __forceinline__ float load_q_i8(const Args &a, int b, int row, bool live, int tig,
-                                           uint32_t (&qh)[4][2], uint32_t (&ql)[4][2]) {
+                                           uint32_t (&qh)[4][2], uint32_t (&qm)[4][2],
+                                           uint32_t (&ql)[4][2]) {
     constexpr int D = 128;
+    constexpr float kL = 8355711.f;
     float v[2][16];
     if (live) {
         const uint4 *qr = reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * a.Hq + row) * D);
@@ -697,26 +724,31 @@ __device__ __forceinline__ float load_q_i8(const Args &a, int b, int row, bool l
         for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(v[half][i]));
     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));  // the quad holds the whole row
     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-    // largest power of two sc with mx * sc <= 16256
-    const float sc = mx > 0.f ? exp2f(floorf(log2f(16256.f / mx))) : 1.f;
+    // largest power of two sc with mx * sc <= L
+    float sc = pow2_scale_for(mx, 22);
+    if (mx * sc > kL) sc *= 0.5f;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            uint32_t hw = 0u, lw = 0u;
+            uint32_t hw = 0u, mw = 0u, lw = 0u;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int qi = __float2int_rn(v[half][4 * w + e] * sc);
-                const int hi = (qi + 64) >> 7;
-                const int lo = qi - hi * 128;
+                const int r1 = (qi + 128) >> 8;   // qi = 256 * r1 + lo
+                const int lo = qi - r1 * 256;
+                const int hi = (r1 + 128) >> 8;   // r1 = 256 * hi + mid
+                const int md = r1 - hi * 256;
                 hw |= (uint32_t)(hi & 0xff) << (8 * e);
+                mw |= (uint32_t)(md & 0xff) << (8 * e);
                 lw |= (uint32_t)(lo & 0xff) << (8 * e);
             }
             qh[w][half] = hw;
+            qm[w][half] = mw;
             ql[w][half] = lw;
         }
     }
-    return mx > 0.f ? 1.f / sc : 0.f;
+    return 1.f / sc;   // exact: sc is a normal power of two
 }
 
 // Final write of one query row of the INT8 consumer: this thread holds dims
@@ -760,7 +792,9 @@ __device__ __forceinline__ void store_i8_row(const Args &a, const StageMeta &mt,
 //   over d is order-free, so thread (g, tig) takes, for k-step kk, the 32-bit
 //   words kk of its two 16-byte chunks (dims 16*tig + 4*kk and 16*(tig+4) +
 //   4*kk, 4 codes each) of its token row as its b0/b1 operands, and the query's
-//   hi/lo int8 parts (load_q_i8) use the same dims.  Rows of odd g load their
+//   hi/mid/lo int8 parts (load_q_i8) use the same dims.  For G <= 8 one MMA takes
+//   hi in rows g and mid in the otherwise empty rows g + 8, a second takes lo;
+//   for G = 16 each part of rows g and g + 8 is one MMA.  Rows of odd g load their
 //   two chunks in the other order (then swap), which keeps the shared-memory
 //   reads conflict-free.
 //  PV: n-tile nt, column g stands for dim 16*g + nt, so a thread reads 16 dims
@@ -770,6 +804,139 @@ __device__ __forceinline__ void store_i8_row(const Args &a, const StageMeta &mt,
 //   1152 times that sum is subtracted at the end.  Output column 2*tig (+1) of
 //   n-tile nt is dim 32*tig + nt (+16).
 //  The K scale multiplies the logit, the V scale the softmax weight.
+//  A warp's two 16-token sub-tiles of a stage (one-byte pools: a stage carries
+//  two per warp) take one softmax step together: both QK^T products, one max
+//  over their 32 logits, one rescale of O, then both PV products.  That halves
+//  the per-token softmax bookkeeping and gives the tensor and ALU pipes two
+//  independent chains.
+
+// Logits of rows g (and g + 8) of one 16-token sub-tile before the K scale:
+// s0 holds tokens 2*tig, 2*tig + 1 (entries 0, 1: rows g; 2, 3: rows g + 8),
+// s1 tokens 8 + 2*tig, 9 + 2*tig.
+template <bool G16>
+__device__ __forceinline__ void qk_i8(uint32_t kbase, int g, int tig, int odd,
+                                      const uint32_t (&qh)[4][2], const uint32_t (&qm)[4][2],
+                                      const uint32_t (&ql)[4][2],
+                                      const uint32_t (&qhb)[G16 ? 4 : 1][2],
+                                      const uint32_t (&qmb)[G16 ? 4 : 1][2],
+                                      const uint32_t (&qlb)[G16 ? 4 : 1][2], float qs, float qsb,
+                                      float (&s0)[4], float (&s1)[4]) {
+    int sh[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, sl8[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+    int sm8[G16 ? 2 : 1][4] = {};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int t = 8 * nt + g;  // swizzle phase of row t is g
+        const uint32_t rb = kbase + t * kBoxRow;
+        const uint4 x0 = lds128(rb + (((tig + 4 * odd) ^ g) << 4));
+        const uint4 x1 = lds128(rb + (((tig + 4 * (1 - odd)) ^ g) << 4));
+        const uint4 lo = odd ? x1 : x0;  // dims 16*tig ..
+        const uint4 hi = odd ? x0 : x1;  // dims 16*(tig+4) ..
+        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            if constexpr (G16) {
+                ptx::mma_s8(sh[nt], qh[kk][0], qhb[kk][0], qh[kk][1], qhb[kk][1], wl[kk], wh[kk]);
+                ptx::mma_s8(sm8[nt], qm[kk][0], qmb[kk][0], qm[kk][1], qmb[kk][1], wl[kk],
+                            wh[kk]);
+                ptx::mma_s8(sl8[nt], ql[kk][0], qlb[kk][0], ql[kk][1], qlb[kk][1], wl[kk],
+                            wh[kk]);
+            } else {
+                // G <= 8: the mid parts ride in the empty rows g + 8 of the hi MMA
+                ptx::mma_s8(sh[nt], qh[kk][0], qm[kk][0], qh[kk][1], qm[kk][1], wl[kk], wh[kk]);
+                ptx::mma_s8(sl8[nt], ql[kk][0], 0u, ql[kk][1], 0u, wl[kk], wh[kk]);
+            }
+        }
+    }
+    // q'.k = 65536 hi.k + 256 mid.k + lo.k: 256 hi.k + mid.k is exact in int32
+    // (|hi.k| <= 128*127*127), the rest in fp32
+    if constexpr (G16) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            s0[i] = fmaf((float)(sh[0][i] * 256 + sm8[0][i]), 256.f, (float)sl8[0][i]) *
+                    (i < 2 ? qs : qsb);
+            s1[i] = fmaf((float)(sh[1][i] * 256 + sm8[1][i]), 256.f, (float)sl8[1][i]) *
+                    (i < 2 ? qs : qsb);
+        }
+    } else {  // hi . K in entries 0, 1, mid . K in entries 2, 3; lo . K in sl8 0, 1
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            s0[i] = fmaf((float)(sh[0][i] * 256 + sh[0][i + 2]), 256.f, (float)sl8[0][i]) * qs;
+            s1[i] = fmaf((float)(sh[1][i] * 256 + sh[1][i + 2]), 256.f, (float)sl8[1][i]) * qs;
+        }
+        s0[2] = s0[3] = s1[2] = s1[3] = 0.f;
+    }
+}
+
+// O += P (V + 1152) for one 16-token sub-tile; column g of n-tile nt is dim
+// 16*g + nt.  (pa0, pa2): the fp16 weights (times the V scale) of rows g for
+// tokens (2*tig, 2*tig + 1) and (8 + 2*tig, 9 + 2*tig); pa1, pa3 those of rows
+// g + 8 (zero for G <= 8).  ol gathers the weights' sums (all-ones column).
+template <bool G16>
+__device__ __forceinline__ void pv_i8(uint32_t vbase, int g, int tig, uint32_t pa0, uint32_t pa1,
+                                      uint32_t pa2, uint32_t pa3, float (&o)[16][2],
+                                      float (&ob)[G16 ? 16 : 1][2], float (&ol)[4]) {
+    const int t_a = 2 * tig, t_b = 8 + 2 * tig;
+    const uint4 ra = lds128(vbase + t_a * kBoxRow + ((g ^ (t_a & 7)) << 4));
+    const uint4 rb = lds128(vbase + (t_a + 1) * kBoxRow + ((g ^ ((t_a + 1) & 7)) << 4));
+    const uint4 rc = lds128(vbase + t_b * kBoxRow + ((g ^ (t_b & 7)) << 4));
+    const uint4 rd = lds128(vbase + (t_b + 1) * kBoxRow + ((g ^ ((t_b + 1) & 7)) << 4));
+    const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w}, wb[4] = {rb.x, rb.y, rb.z, rb.w};
+    const uint32_t wc[4] = {rc.x, rc.y, rc.z, rc.w}, wd[4] = {rd.x, rd.y, rd.z, rd.w};
+    {
+        float dd[4] = {ol[0], ol[1], ol[2], ol[3]};
+        ptx::mma_f16(dd, pa0, pa1, pa2, pa3, kOnes, kOnes);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ol[i] = dd[i];
+    }
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t fa = wa[w] ^ kFlip, fb = wb[w] ^ kFlip;
+        const uint32_t fc = wc[w] ^ kFlip, fd = wd[w] ^ kFlip;
+        const uint32_t X = prmt(fa, fb, 0x5140u), Y = prmt(fa, fb, 0x7362u);
+        const uint32_t Z = prmt(fc, fd, 0x5140u), U = prmt(fc, fd, 0x7362u);
+        const uint32_t b0[4] = {biased_f16x2(X, 0x4140u), biased_f16x2(X, 0x4342u),
+                                biased_f16x2(Y, 0x4140u), biased_f16x2(Y, 0x4342u)};
+        const uint32_t b1[4] = {biased_f16x2(Z, 0x4140u), biased_f16x2(Z, 0x4342u),
+                                biased_f16x2(U, 0x4140u), biased_f16x2(U, 0x4342u)};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int nt = 4 * w + i;
+            float dd[4] = {o[nt][0], o[nt][1], 0.f, 0.f};
+            if constexpr (G16) {
+                dd[2] = ob[nt][0];
+                dd[3] = ob[nt][1];
+            }
+            ptx::mma_f16(dd, pa0, pa1, pa2, pa3, b0[i], b1[i]);
+            o[nt][0] = dd[0];
+            o[nt][1] = dd[1];
+            if constexpr (G16) {
+                ob[nt][0] = dd[2];
+                ob[nt][1] = dd[3];
+            }
+        }
+    }
+}
+
+// One online-softmax step of one query row over the 8 logits a thread holds for
+// a sub-tile pair (x[0..3]: sub-tile A, x[4..7]: B; -inf where masked) with the
+// quad's other 24: updates (m, l), returns alpha = 2^(m_old - m_new) and the
+// weights p (2^(x - m_new)).
+__device__ __forceinline__ float softmax_pair_step(const float (&x)[8], float &m, float &l,
+                                                   float (&p)[8]) {
+    float mx = fmaxf(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])),
+                     fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7])));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+    const float mn = fmaxf(m, mx);
+    const float mu = mn == -INFINITY ? 0.f : mn;
+    const float alpha = ex2_fast(m - mu);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) p[i] = ex2_fast(x[i] - mu);
+    l = l * alpha + (((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7])));
+    m = mn;
+    return alpha;
+}
+
 template <bool G16>
 __device__ __forceinline__ void consumer_i8(const Args &a, uint8_t *stages, StageMeta *meta,
                                             uint64_t *full, uint64_t *empty) {
@@ -781,9 +948,11 @@ __device__ __forceinline__ void consumer_i8(const Args &a, uint8_t *stages, Stag
     const uint32_t head_off = (uint32_t)(h * kTile * kBoxRow);
     const uint32_t sub_bytes = (uint32_t)a.box_bytes;           // one box per sub-tile (d = 128)
     const uint32_t sc_sub = (uint32_t)(kTile * a.Hkv * 4);      // scale rows of one sub-tile
+    const int hs = a.Hkv * 4;                                   // bytes between token scale rows
+    const int t_a = 2 * tig, t_b = 8 + 2 * tig;                 // this thread's token pairs
 
-    uint32_t qh[4][2], ql[4][2];                          // rows g: hi / lo int8 parts
-    uint32_t qhb[G16 ? 4 : 1][2], qlb[G16 ? 4 : 1][2];    // rows g + 8
+    uint32_t qh[4][2], qm[4][2], ql[4][2];                // rows g: hi / mid / lo parts
+    uint32_t qhb[G16 ? 4 : 1][2], qmb[G16 ? 4 : 1][2], qlb[G16 ? 4 : 1][2];  // rows g + 8
     float qs = 0.f, qsb = 0.f;                            // 1 / 2^e of rows g and g + 8
     float o[16][2];
     float ob[G16 ? 16 : 1][2];
@@ -800,8 +969,9 @@ __device__ __forceinline__ void consumer_i8(const Args &a, uint8_t *stages, Stag
         if (mt.flags & kEnd) break;
         const uint32_t sb = stage0 + (uint32_t)stage * a.stage_bytes;
         if (mt.flags & kFirst) {
-            qs = load_q_i8(a, mt.b, h * a.G + g, g < a.G, tig, qh, ql);
-            if constexpr (G16) qsb = load_q_i8(a, mt.b, h * a.G + g + 8, g + 8 < a.G, tig, qhb, qlb);
+            qs = load_q_i8(a, mt.b, h * a.G + g, g < a.G, tig, qh, qm, ql);
+            if constexpr (G16)
+                qsb = load_q_i8(a, mt.b, h * a.G + g + 8, g + 8 < a.G, tig, qhb, qmb, qlb);
             m = -INFINITY;
             l = 0.f;
             mb = -INFINITY;
@@ -814,96 +984,65 @@ __device__ __forceinline__ void consumer_i8(const Args &a, uint8_t *stages, Stag
                 if constexpr (G16) ob[nt][0] = ob[nt][1] = 0.f;
             }
         }
-        for (int k = 0; k < a.tpw; ++k) {
-        const int jj = jw + a.wph * k;  // this warp's k-th sub-tile of the stage
-        const int tj = mt.ts + kTile * jj;
-        const int nv = max(0, min(kTile, mt.te - tj));
-        if (nv > 0 && !((mt.bad >> jj) & 1)) {
-            const uint32_t kbase = sb + jj * sub_bytes + head_off;
-            const uint32_t vbase = sb + a.v_off + jj * sub_bytes + head_off;
-            const uint32_t ksb = sb + a.ks_off + jj * sc_sub + h * 4;
-            const uint32_t vsb = sb + a.vs_off + jj * sc_sub + h * 4;
+        // this warp's two sub-tiles of the stage (A before B in token order)
+        const int jA = jw, jB = jw + a.wph;
+        const int nvA = max(0, min(kTile, mt.te - (mt.ts + kTile * jA)));
+        const int nvB = max(0, min(kTile, mt.te - (mt.ts + kTile * jB)));
+        const bool liveA = nvA > 0 && !((mt.bad >> jA) & 1);
+        const bool liveB = nvB > 0 && !((mt.bad >> jB) & 1);
+        if (liveA || liveB) {
             // ---- S = Q K^T on int8 tensor cores: K codes straight from shared memory
-            int sh[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, sl8[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int t = 8 * nt + g;  // swizzle phase of row t is g
-                const uint32_t rb = kbase + t * kBoxRow;
-                const uint4 x0 = lds128(rb + (((tig + 4 * odd) ^ g) << 4));
-                const uint4 x1 = lds128(rb + (((tig + 4 * (1 - odd)) ^ g) << 4));
-                const uint4 lo = odd ? x1 : x0;  // dims 16*tig ..
-                const uint4 hi = odd ? x0 : x1;  // dims 16*(tig+4) ..
-                const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    if constexpr (G16) {
-                        ptx::mma_s8(sh[nt], qh[kk][0], qhb[kk][0], qh[kk][1], qhb[kk][1], wl[kk],
-                                    wh[kk]);
-                        ptx::mma_s8(sl8[nt], ql[kk][0], qlb[kk][0], ql[kk][1], qlb[kk][1], wl[kk],
-                                    wh[kk]);
-                    } else {
-                        // G <= 8: the lo parts ride in the empty rows g + 8 of the same MMA
-                        ptx::mma_s8(sh[nt], qh[kk][0], ql[kk][0], qh[kk][1], ql[kk][1], wl[kk],
-                                    wh[kk]);
-                    }
-                }
-            }
-            float s0[4], s1[4];
-            if constexpr (G16) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    s0[i] = (float)(sh[0][i] * 128 + sl8[0][i]) * (i < 2 ? qs : qsb);
-                    s1[i] = (float)(sh[1][i] * 128 + sl8[1][i]) * (i < 2 ? qs : qsb);
-                }
-            } else {  // rows g: hi . K in entries 0, 1; lo . K in entries 2, 3
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    s0[i] = (float)(sh[0][i] * 128 + sh[0][i + 2]) * qs;
-                    s1[i] = (float)(sh[1][i] * 128 + sh[1][i + 2]) * qs;
-                }
-                s0[2] = s0[3] = s1[2] = s1[3] = 0.f;
-            }
-            // ---- online softmax; K scale folded into the logit
-            const int t_a = 2 * tig, t_b = 8 + 2 * tig;
-            const bool va0 = t_a < nv, va1 = t_a + 1 < nv, vb0 = t_b < nv, vb1 = t_b + 1 < nv;
+            float sA0[4] = {0.f, 0.f, 0.f, 0.f}, sA1[4] = {0.f, 0.f, 0.f, 0.f};
+            float sB0[4] = {0.f, 0.f, 0.f, 0.f}, sB1[4] = {0.f, 0.f, 0.f, 0.f};
+            if (liveA)
+                qk_i8<G16>(sb + jA * sub_bytes + head_off, g, tig, odd, qh, qm, ql, qhb, qmb,
+                           qlb, qs, qsb, sA0, sA1);
+            if (liveB)
+                qk_i8<G16>(sb + jB * sub_bytes + head_off, g, tig, odd, qh, qm, ql, qhb, qmb,
+                           qlb, qs, qsb, sB0, sB1);
+            // ---- online softmax over both sub-tiles; K scale folded into the logit
+            const bool va[8] = {liveA && t_a < nvA, liveA && t_a + 1 < nvA,
+                                liveA && t_b < nvA, liveA && t_b + 1 < nvA,
+                                liveB && t_a < nvB, liveB && t_a + 1 < nvB,
+                                liveB && t_b < nvB, liveB && t_b + 1 < nvB};
+            const int tok[4] = {t_a, t_a + 1, t_b, t_b + 1};
+            const uint32_t ksA = sb + a.ks_off + jA * sc_sub + h * 4;
+            const uint32_t ksB = sb + a.ks_off + jB * sc_sub + h * 4;
+            const uint32_t vsA = sb + a.vs_off + jA * sc_sub + h * 4;
+            const uint32_t vsB = sb + a.vs_off + jB * sc_sub + h * 4;
             const float sl = a.scale_log2;
-            const int hs = a.Hkv * 4;
-            const float k0 = lds_f32(ksb + t_a * hs) * sl, k1 = lds_f32(ksb + (t_a + 1) * hs) * sl;
-            const float k2 = lds_f32(ksb + t_b * hs) * sl, k3 = lds_f32(ksb + (t_b + 1) * hs) * sl;
-            const float v0 = lds_f32(vsb + t_a * hs), v1 = lds_f32(vsb + (t_a + 1) * hs);
-            const float v2 = lds_f32(vsb + t_b * hs), v3 = lds_f32(vsb + (t_b + 1) * hs);
-            float x0 = va0 ? s0[0] * k0 : -INFINITY, x1 = va1 ? s0[1] * k1 : -INFINITY;
-            float x2 = vb0 ? s1[0] * k2 : -INFINITY, x3 = vb1 ? s1[1] * k3 : -INFINITY;
-            float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-            const float mn = fmaxf(m, mx);
-            const float mu = mn == -INFINITY ? 0.f : mn;
-            const float alpha = ex2_fast(m - mu);
-            const float p0 = ex2_fast(x0 - mu), p1 = ex2_fast(x1 - mu);
-            const float p2 = ex2_fast(x2 - mu), p3 = ex2_fast(x3 - mu);
-            l = l * alpha + ((p0 + p1) + (p2 + p3));
-            m = mn;
-            const uint32_t pa0 = ptx::pack_f16(va0 ? p0 * v0 : 0.f, va1 ? p1 * v1 : 0.f);
-            const uint32_t pa2 = ptx::pack_f16(vb0 ? p2 * v2 : 0.f, vb1 ? p3 * v3 : 0.f);
-            uint32_t pa1 = 0u, pa3 = 0u;
+            float kf[8], vf[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                kf[i] = va[i] ? lds_f32(ksA + tok[i] * hs) * sl : 0.f;
+                kf[4 + i] = va[4 + i] ? lds_f32(ksB + tok[i] * hs) * sl : 0.f;
+                vf[i] = va[i] ? lds_f32(vsA + tok[i] * hs) : 0.f;
+                vf[4 + i] = va[4 + i] ? lds_f32(vsB + tok[i] * hs) : 0.f;
+            }
+            const float rawg[8] = {sA0[0], sA0[1], sA1[0], sA1[1], sB0[0], sB0[1], sB1[0], sB1[1]};
+            float x[8], p[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = va[i] ? rawg[i] * kf[i] : -INFINITY;
+            const float alpha = softmax_pair_step(x, m, l, p);
+            const uint32_t pA0 = ptx::pack_f16(p[0] * vf[0], p[1] * vf[1]);
+            const uint32_t pA2 = ptx::pack_f16(p[2] * vf[2], p[3] * vf[3]);
+            const uint32_t pB0 = ptx::pack_f16(p[4] * vf[4], p[5] * vf[5]);
+            const uint32_t pB2 = ptx::pack_f16(p[6] * vf[6], p[7] * vf[7]);
+            uint32_t pA1 = 0u, pA3 = 0u, pB1 = 0u, pB3 = 0u;
             float alphab = 1.f;
             if constexpr (G16) {
-                float y0 = va0 ? s0[2] * k0 : -INFINITY, y1 = va1 ? s0[3] * k1 : -INFINITY;
-                float y2 = vb0 ? s1[2] * k2 : -INFINITY, y3 = vb1 ? s1[3] * k3 : -INFINITY;
-                float my = fmaxf(fmaxf(y0, y1), fmaxf(y2, y3));
-                my = fmaxf(my, __shfl_xor_sync(kFull, my, 1));
-                my = fmaxf(my, __shfl_xor_sync(kFull, my, 2));
-                const float mnb = fmaxf(mb, my);
-                const float mub = mnb == -INFINITY ? 0.f : mnb;
-                alphab = ex2_fast(mb - mub);
-                const float q0 = ex2_fast(y0 - mub), q1 = ex2_fast(y1 - mub);
-                const float q2 = ex2_fast(y2 - mub), q3 = ex2_fast(y3 - mub);
-                lb = lb * alphab + ((q0 + q1) + (q2 + q3));
-                mb = mnb;
-                pa1 = ptx::pack_f16(va0 ? q0 * v0 : 0.f, va1 ? q1 * v1 : 0.f);
-                pa3 = ptx::pack_f16(vb0 ? q2 * v2 : 0.f, vb1 ? q3 * v3 : 0.f);
+                const float rawb[8] = {sA0[2], sA0[3], sA1[2], sA1[3],
+                                       sB0[2], sB0[3], sB1[2], sB1[3]};
+                float y[8], q[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = va[i] ? rawb[i] * kf[i] : -INFINITY;
+                alphab = softmax_pair_step(y, mb, lb, q);
+                pA1 = ptx::pack_f16(q[0] * vf[0], q[1] * vf[1]);
+                pA3 = ptx::pack_f16(q[2] * vf[2], q[3] * vf[3]);
+                pB1 = ptx::pack_f16(q[4] * vf[4], q[5] * vf[5]);
+                pB3 = ptx::pack_f16(q[6] * vf[6], q[7] * vf[7]);
             }
+            // rescale only when some row maximum moved (alpha == 1 exactly otherwise)
             if (__any_sync(kFull, alpha != 1.f || alphab != 1.f)) {
                 ol[0] *= alpha;
                 ol[1] *= alpha;
@@ -919,47 +1058,13 @@ __device__ __forceinline__ void consumer_i8(const Args &a, uint8_t *stages, Stag
                     }
                 }
             }
-            // ---- O += P (V + 1152); column g of n-tile nt is dim 16*g + nt
-            const uint4 ra = lds128(vbase + t_a * kBoxRow + ((g ^ (t_a & 7)) << 4));
-            const uint4 rb = lds128(vbase + (t_a + 1) * kBoxRow + ((g ^ ((t_a + 1) & 7)) << 4));
-            const uint4 rc = lds128(vbase + t_b * kBoxRow + ((g ^ (t_b & 7)) << 4));
-            const uint4 rd = lds128(vbase + (t_b + 1) * kBoxRow + ((g ^ ((t_b + 1) & 7)) << 4));
-            const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w}, wb[4] = {rb.x, rb.y, rb.z, rb.w};
-            const uint32_t wc[4] = {rc.x, rc.y, rc.z, rc.w}, wd[4] = {rd.x, rd.y, rd.z, rd.w};
-            {
-                float dd[4] = {ol[0], ol[1], ol[2], ol[3]};
-                ptx::mma_f16(dd, pa0, pa1, pa2, pa3, kOnes, kOnes);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) ol[i] = dd[i];
-            }
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const uint32_t fa = wa[w] ^ kFlip, fb = wb[w] ^ kFlip;
-                const uint32_t fc = wc[w] ^ kFlip, fd = wd[w] ^ kFlip;
-                const uint32_t X = prmt(fa, fb, 0x5140u), Y = prmt(fa, fb, 0x7362u);
-                const uint32_t Z = prmt(fc, fd, 0x5140u), U = prmt(fc, fd, 0x7362u);
-                const uint32_t b0[4] = {biased_f16x2(X, 0x4140u), biased_f16x2(X, 0x4342u),
-                                        biased_f16x2(Y, 0x4140u), biased_f16x2(Y, 0x4342u)};
-                const uint32_t b1[4] = {biased_f16x2(Z, 0x4140u), biased_f16x2(Z, 0x4342u),
-                                        biased_f16x2(U, 0x4140u), biased_f16x2(U, 0x4342u)};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int nt = 4 * w + i;
-                    float dd[4] = {o[nt][0], o[nt][1], 0.f, 0.f};
-                    if constexpr (G16) {
-                        dd[2] = ob[nt][0];
-                        dd[3] = ob[nt][1];
-                    }
-                    ptx::mma_f16(dd, pa0, pa1, pa2, pa3, b0[i], b1[i]);
-                    o[nt][0] = dd[0];
-                    o[nt][1] = dd[1];
-                    if constexpr (G16) {
-                        ob[nt][0] = dd[2];
-                        ob[nt][1] = dd[3];
-                    }
-                }
-            }
-        }
+            // ---- O += P (V + 1152), sub-tile A then B
+            if (liveA)
+                pv_i8<G16>(sb + a.v_off + jA * sub_bytes + head_off, g, tig, pA0, pA1, pA2, pA3,
+                           o, ob, ol);
+            if (liveB)
+                pv_i8<G16>(sb + a.v_off + jB * sub_bytes + head_off, g, tig, pB0, pB1, pB2, pB3,
+                           o, ob, ol);
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&empty[stage]);
@@ -994,28 +1099,54 @@ __device__ __forceinline__ void e4m3_word_to_f16x2(uint32_t w, uint32_t &lo, uin
 
 // Query fragments (fp16) for the FP8 consumer: k-step kk (16 dims) of thread
 // (g, tig) uses dims 16*(tig + 4*(kk/4)) + 4*(kk%4) + 0..3, the dims of the K
-// word it converts (see consumer_fp8).
-__device__ __forceinline__ void load_q_f16perm(const Args &a, int b, int row, bool live, int tig,
-                                               uint32_t (&qa)[8][2]) {
+// word it converts (see consumer_fp8).  The row is first scaled by a power of
+// two 2^e that puts its largest magnitude in [2^14, 2^15): every bf16 query
+// then fits fp16 without overflow (|q| above 65504 included), and every element
+// no smaller than 2^-32 of the row's largest converts exactly (fp16 keeps 11
+// significant bits against bf16's 8); smaller ones round with an error below
+// 2^-39 of the largest.  Returns 1 / 2^e, which the logit takes back.
+__device__ __forceinline__ float load_q_f16perm(const Args &a, int b, int row, bool live, int tig,
+                                                uint32_t (&qa)[8][2]) {
     constexpr int D = 128;
     const uint4 *qr = reinterpret_cast<const uint4 *>(a.q + ((int64_t)b * a.Hq + row) * D);
+    uint4 w[4];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int c = tig + 4 * half;  // 16 dims = two uint4 of bf16
+        w[2 * half] = live ? __ldg(qr + 2 * c) : make_uint4(0u, 0u, 0u, 0u);
+        w[2 * half + 1] = live ? __ldg(qr + 2 * c + 1) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // |bf16| of a pair word is the word with both sign bits cleared; compare the
+    // halves as floats
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            mx = fmaxf(mx, fmaxf(fabsf(bf16_lo(u[j])), fabsf(bf16_hi(u[j]))));
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));  // the quad holds the whole row
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+    const float sc = pow2_scale_for(mx, 14);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         uint32_t f[8];
-        if (live) {
-            const int c = tig + 4 * half;  // 16 dims = two uint4 of bf16
-            bf16x8_to_f16x2(__ldg(qr + 2 * c), f);
-            bf16x8_to_f16x2(__ldg(qr + 2 * c + 1), f + 4);
-        } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = 0u;
+        for (int k = 0; k < 2; ++k) {
+            const uint4 v = w[2 * half + k];
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                f[4 * k + i] = ptx::pack_f16(bf16_lo(u[i]) * sc, bf16_hi(u[i]) * sc);
         }
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            qa[4 * half + w][0] = f[2 * w];
-            qa[4 * half + w][1] = f[2 * w + 1];
+        for (int kw = 0; kw < 4; ++kw) {
+            qa[4 * half + kw][0] = f[2 * kw];
+            qa[4 * half + kw][1] = f[2 * kw + 1];
         }
     }
+    return 1.f / sc;   // exact: sc is a normal power of two
 }
 
 // FP8 (e4m3) consumer (d = 128).  Same pipeline and softmax as the bf16
@@ -1026,6 +1157,93 @@ __device__ __forceinline__ void load_q_f16perm(const Args &a, int b, int row, bo
 //   the query fragments use the same dims (load_q_f16perm).
 //  PV: as in the INT8 consumer -- n-tile nt, column g is dim 16*g + nt; token
 //   pairs are byte-transposed with prmt before the conversion.
+//  As in the INT8 consumer, a warp's two sub-tiles of a stage take one softmax
+//  step together.
+
+// Logits of rows g (and g + 8) of one 16-token sub-tile, before scale and the
+// query's 2^-e (layout as qk_i8).
+template <bool G16>
+__device__ __forceinline__ void qk_fp8(uint32_t kbase, int g, int tig, int odd,
+                                       const uint32_t (&qa)[8][2],
+                                       const uint32_t (&qb)[G16 ? 8 : 1][2], float (&s0)[4],
+                                       float (&s1)[4]) {
+    float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s0[i] = s1[i] = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int t = 8 * nt + g;  // swizzle phase of row t is g
+        const uint32_t rb = kbase + t * kBoxRow;
+        const uint4 x0 = lds128(rb + (((tig + 4 * odd) ^ g) << 4));
+        const uint4 x1 = lds128(rb + (((tig + 4 * (1 - odd)) ^ g) << 4));
+        const uint4 lo = odd ? x1 : x0;  // dims 16*tig ..
+        const uint4 hi = odd ? x0 : x1;  // dims 16*(tig+4) ..
+        const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            uint32_t b0, b1;
+            e4m3_word_to_f16x2(wd[kk], b0, b1);
+            // even and odd k-steps in separate accumulators: two independent chains
+            float(&acc)[4] = nt == 0 ? ((kk & 1) ? e0 : s0) : ((kk & 1) ? e1 : s1);
+            if constexpr (G16)
+                ptx::mma_f16(acc, qa[kk][0], qb[kk][0], qa[kk][1], qb[kk][1], b0, b1);
+            else
+                ptx::mma_f16(acc, qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        s0[i] += e0[i];
+        s1[i] += e1[i];
+    }
+}
+
+// O += P V for one 16-token sub-tile of e4m3 codes (column g of n-tile nt is dim
+// 16*g + nt).  Masked tokens have P = 0; their codes may be NaN (0x7f), so the
+// rows of tokens outside [0, nv) are zeroed.
+template <bool G16>
+__device__ __forceinline__ void pv_fp8(uint32_t vbase, int g, int tig, int nv, uint32_t pa0,
+                                       uint32_t pa1, uint32_t pa2, uint32_t pa3,
+                                       float (&o)[16][2], float (&ob)[G16 ? 16 : 1][2]) {
+    const int t_a = 2 * tig, t_b = 8 + 2 * tig;
+    const uint4 ra = lds128(vbase + t_a * kBoxRow + ((g ^ (t_a & 7)) << 4));
+    const uint4 rb = lds128(vbase + (t_a + 1) * kBoxRow + ((g ^ ((t_a + 1) & 7)) << 4));
+    const uint4 rc = lds128(vbase + t_b * kBoxRow + ((g ^ (t_b & 7)) << 4));
+    const uint4 rd = lds128(vbase + (t_b + 1) * kBoxRow + ((g ^ ((t_b + 1) & 7)) << 4));
+    const uint32_t za = t_a < nv ? ~0u : 0u, zb = t_a + 1 < nv ? ~0u : 0u;
+    const uint32_t zc = t_b < nv ? ~0u : 0u, zd = t_b + 1 < nv ? ~0u : 0u;
+    const uint32_t wa[4] = {ra.x & za, ra.y & za, ra.z & za, ra.w & za};
+    const uint32_t wb[4] = {rb.x & zb, rb.y & zb, rb.z & zb, rb.w & zb};
+    const uint32_t wc[4] = {rc.x & zc, rc.y & zc, rc.z & zc, rc.w & zc};
+    const uint32_t wdv[4] = {rd.x & zd, rd.y & zd, rd.z & zd, rd.w & zd};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t X = prmt(wa[w], wb[w], 0x5140u), Y = prmt(wa[w], wb[w], 0x7362u);
+        const uint32_t Z = prmt(wc[w], wdv[w], 0x5140u), U = prmt(wc[w], wdv[w], 0x7362u);
+        uint32_t b0[4], b1[4];
+        e4m3_word_to_f16x2(X, b0[0], b0[1]);
+        e4m3_word_to_f16x2(Y, b0[2], b0[3]);
+        e4m3_word_to_f16x2(Z, b1[0], b1[1]);
+        e4m3_word_to_f16x2(U, b1[2], b1[3]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int nt = 4 * w + i;
+            float dd[4] = {o[nt][0], o[nt][1], 0.f, 0.f};
+            if constexpr (G16) {
+                dd[2] = ob[nt][0];
+                dd[3] = ob[nt][1];
+            }
+            ptx::mma_f16(dd, pa0, pa1, pa2, pa3, b0[i], b1[i]);
+            o[nt][0] = dd[0];
+            o[nt][1] = dd[1];
+            if constexpr (G16) {
+                ob[nt][0] = dd[2];
+                ob[nt][1] = dd[3];
+            }
+        }
+    }
+}
+
 template <bool G16>
 __device__ __forceinline__ void consumer_fp8(const Args &a, uint8_t *stages, StageMeta *meta,
                                              uint64_t *full, uint64_t *empty) {
@@ -1036,9 +1254,11 @@ __device__ __forceinline__ void consumer_fp8(const Args &a, uint8_t *stages, Sta
     const uint32_t stage0 = ptx::smem_u32(stages);
     const uint32_t head_off = (uint32_t)(h * kTile * kBoxRow);
     const uint32_t sub_bytes = (uint32_t)a.box_bytes;
+    const int t_a = 2 * tig, t_b = 8 + 2 * tig;   // this thread's token pairs
 
     uint32_t qa[8][2];
     uint32_t qb[G16 ? 8 : 1][2];
+    float qs = 1.f, qsb = 1.f;  // 1 / 2^e of rows g and g + 8 (load_q_f16perm)
     float o[16][2];
     float ob[G16 ? 16 : 1][2];
     float m = -INFINITY, l = 0.f, mb = -INFINITY, lb = 0.f;
@@ -1053,10 +1273,10 @@ __device__ __forceinline__ void consumer_fp8(const Args &a, uint8_t *stages, Sta
         if (mt.flags & kEnd) break;
         const uint32_t sb = stage0 + (uint32_t)stage * a.stage_bytes;
         if (mt.flags & kFirst) {
-            load_q_f16perm(a, mt.b, h * a.G + g, g < a.G, tig, qa);
+            qs = load_q_f16perm(a, mt.b, h * a.G + g, g < a.G, tig, qa);
             if constexpr (G16) {
                 uint32_t t[8][2];
-                load_q_f16perm(a, mt.b, h * a.G + g + 8, g + 8 < a.G, tig, t);
+                qsb = load_q_f16perm(a, mt.b, h * a.G + g + 8, g + 8 < a.G, tig, t);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     qb[kk][0] = t[kk][0];
@@ -1073,75 +1293,44 @@ __device__ __forceinline__ void consumer_fp8(const Args &a, uint8_t *stages, Sta
                 if constexpr (G16) ob[nt][0] = ob[nt][1] = 0.f;
             }
         }
-        for (int k = 0; k < a.tpw; ++k) {
-        const int jj = jw + a.wph * k;  // this warp's k-th sub-tile of the stage
-        const int tj = mt.ts + kTile * jj;
-        const int nv = max(0, min(kTile, mt.te - tj));
-        if (nv > 0 && !((mt.bad >> jj) & 1)) {
-            const uint32_t kbase = sb + jj * sub_bytes + head_off;
-            const uint32_t vbase = sb + a.v_off + jj * sub_bytes + head_off;
+        // this warp's two sub-tiles of the stage (A before B in token order)
+        const int jA = jw, jB = jw + a.wph;
+        const int nvA0 = max(0, min(kTile, mt.te - (mt.ts + kTile * jA)));
+        const int nvB0 = max(0, min(kTile, mt.te - (mt.ts + kTile * jB)));
+        const bool liveA = nvA0 > 0 && !((mt.bad >> jA) & 1);
+        const bool liveB = nvB0 > 0 && !((mt.bad >> jB) & 1);
+        if (liveA || liveB) {
+            const int nvA = liveA ? nvA0 : 0, nvB = liveB ? nvB0 : 0;
             // ---- S = Q K^T (exact fp16 values of the codes)
-            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-            float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
+            float sA0[4] = {0.f, 0.f, 0.f, 0.f}, sA1[4] = {0.f, 0.f, 0.f, 0.f};
+            float sB0[4] = {0.f, 0.f, 0.f, 0.f}, sB1[4] = {0.f, 0.f, 0.f, 0.f};
+            if (liveA) qk_fp8<G16>(sb + jA * sub_bytes + head_off, g, tig, odd, qa, qb, sA0, sA1);
+            if (liveB) qk_fp8<G16>(sb + jB * sub_bytes + head_off, g, tig, odd, qa, qb, sB0, sB1);
+            // ---- online softmax over both sub-tiles (the query's 2^-e folded in, exact)
+            const bool va[8] = {t_a < nvA, t_a + 1 < nvA, t_b < nvA, t_b + 1 < nvA,
+                                t_a < nvB, t_a + 1 < nvB, t_b < nvB, t_b + 1 < nvB};
+            const float sl = a.scale_log2 * qs;
+            const float rawg[8] = {sA0[0], sA0[1], sA1[0], sA1[1], sB0[0], sB0[1], sB1[0], sB1[1]};
+            float x[8], p[8];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int t = 8 * nt + g;  // swizzle phase of row t is g
-                const uint32_t rb = kbase + t * kBoxRow;
-                const uint4 x0 = lds128(rb + (((tig + 4 * odd) ^ g) << 4));
-                const uint4 x1 = lds128(rb + (((tig + 4 * (1 - odd)) ^ g) << 4));
-                const uint4 lo = odd ? x1 : x0;  // dims 16*tig ..
-                const uint4 hi = odd ? x0 : x1;  // dims 16*(tig+4) ..
-                const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    uint32_t b0, b1;
-                    e4m3_word_to_f16x2(wd[kk], b0, b1);
-                    float(&acc)[4] = nt == 0 ? ((kk & 1) ? e0 : s0) : ((kk & 1) ? e1 : s1);
-                    if constexpr (G16)
-                        ptx::mma_f16(acc, qa[kk][0], qb[kk][0], qa[kk][1], qb[kk][1], b0, b1);
-                    else
-                        ptx::mma_f16(acc, qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                s0[i] += e0[i];
-                s1[i] += e1[i];
-            }
-            // ---- online softmax
-            const int t_a = 2 * tig, t_b = 8 + 2 * tig;
-            const bool va0 = t_a < nv, va1 = t_a + 1 < nv, vb0 = t_b < nv, vb1 = t_b + 1 < nv;
-            const float sl = a.scale_log2;
-            float x0 = va0 ? s0[0] * sl : -INFINITY, x1 = va1 ? s0[1] * sl : -INFINITY;
-            float x2 = vb0 ? s1[0] * sl : -INFINITY, x3 = vb1 ? s1[1] * sl : -INFINITY;
-            float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-            const float mn = fmaxf(m, mx);
-            const float mu = mn == -INFINITY ? 0.f : mn;
-            const float alpha = ex2_fast(m - mu);
-            const float p0 = ex2_fast(x0 - mu), p1 = ex2_fast(x1 - mu);
-            const float p2 = ex2_fast(x2 - mu), p3 = ex2_fast(x3 - mu);
-            l = l * alpha + ((p0 + p1) + (p2 + p3));
-            m = mn;
-            const uint32_t pa0 = ptx::pack_f16(p0, p1), pa2 = ptx::pack_f16(p2, p3);
-            uint32_t pa1 = 0u, pa3 = 0u;
+            for (int i = 0; i < 8; ++i) x[i] = va[i] ? rawg[i] * sl : -INFINITY;
+            const float alpha = softmax_pair_step(x, m, l, p);
+            const uint32_t pA0 = ptx::pack_f16(p[0], p[1]), pA2 = ptx::pack_f16(p[2], p[3]);
+            const uint32_t pB0 = ptx::pack_f16(p[4], p[5]), pB2 = ptx::pack_f16(p[6], p[7]);
+            uint32_t pA1 = 0u, pA3 = 0u, pB1 = 0u, pB3 = 0u;
             float alphab = 1.f;
             if constexpr (G16) {
-                float y0 = va0 ? s0[2] * sl : -INFINITY, y1 = va1 ? s0[3] * sl : -INFINITY;
-                float y2 = vb0 ? s1[2] * sl : -INFINITY, y3 = vb1 ? s1[3] * sl : -INFINITY;
-                float my = fmaxf(fmaxf(y0, y1), fmaxf(y2, y3));
-                my = fmaxf(my, __shfl_xor_sync(kFull, my, 1));
-                my = fmaxf(my, __shfl_xor_sync(kFull, my, 2));
-                const float mnb = fmaxf(mb, my);
-                const float mub = mnb == -INFINITY ? 0.f : mnb;
-                alphab = ex2_fast(mb - mub);
-                const float q0 = ex2_fast(y0 - mub), q1 = ex2_fast(y1 - mub);
-                const float q2 = ex2_fast(y2 - mub), q3 = ex2_fast(y3 - mub);
-                lb = lb * alphab + ((q0 + q1) + (q2 + q3));
-                mb = mnb;
-                pa1 = ptx::pack_f16(q0, q1);
-                pa3 = ptx::pack_f16(q2, q3);
+                const float slb = a.scale_log2 * qsb;
+                const float rawb[8] = {sA0[2], sA0[3], sA1[2], sA1[3],
+                                       sB0[2], sB0[3], sB1[2], sB1[3]};
+                float y[8], q[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = va[i] ? rawb[i] * slb : -INFINITY;
+                alphab = softmax_pair_step(y, mb, lb, q);
+                pA1 = ptx::pack_f16(q[0], q[1]);
+                pA3 = ptx::pack_f16(q[2], q[3]);
+                pB1 = ptx::pack_f16(q[4], q[5]);
+                pB3 = ptx::pack_f16(q[6], q[7]);
             }
             if (__any_sync(kFull, alpha != 1.f || alphab != 1.f)) {
 #pragma unroll
@@ -1154,45 +1343,13 @@ __device__ __forceinline__ void consumer_fp8(const Args &a, uint8_t *stages, Sta
                     }
                 }
             }
-            // ---- O += P V; column g of n-tile nt is dim 16*g + nt.  Masked tokens
-            // have P = 0; their codes may be NaN (0x7f), so zero those rows' bytes.
-            const uint4 ra = lds128(vbase + t_a * kBoxRow + ((g ^ (t_a & 7)) << 4));
-            const uint4 rb = lds128(vbase + (t_a + 1) * kBoxRow + ((g ^ ((t_a + 1) & 7)) << 4));
-            const uint4 rc = lds128(vbase + t_b * kBoxRow + ((g ^ (t_b & 7)) << 4));
-            const uint4 rd = lds128(vbase + (t_b + 1) * kBoxRow + ((g ^ ((t_b + 1) & 7)) << 4));
-            const uint32_t za = va0 ? ~0u : 0u, zb = va1 ? ~0u : 0u;
-            const uint32_t zc = vb0 ? ~0u : 0u, zd = vb1 ? ~0u : 0u;
-            const uint32_t wa[4] = {ra.x & za, ra.y & za, ra.z & za, ra.w & za};
-            const uint32_t wb[4] = {rb.x & zb, rb.y & zb, rb.z & zb, rb.w & zb};
-            const uint32_t wc[4] = {rc.x & zc, rc.y & zc, rc.z & zc, rc.w & zc};
-            const uint32_t wdv[4] = {rd.x & zd, rd.y & zd, rd.z & zd, rd.w & zd};
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const uint32_t X = prmt(wa[w], wb[w], 0x5140u), Y = prmt(wa[w], wb[w], 0x7362u);
-                const uint32_t Z = prmt(wc[w], wdv[w], 0x5140u), U = prmt(wc[w], wdv[w], 0x7362u);
-                uint32_t b0[4], b1[4];
-                e4m3_word_to_f16x2(X, b0[0], b0[1]);
-                e4m3_word_to_f16x2(Y, b0[2], b0[3]);
-                e4m3_word_to_f16x2(Z, b1[0], b1[1]);
-                e4m3_word_to_f16x2(U, b1[2], b1[3]);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int nt = 4 * w + i;
-                    float dd[4] = {o[nt][0], o[nt][1], 0.f, 0.f};
-                    if constexpr (G16) {
-                        dd[2] = ob[nt][0];
-                        dd[3] = ob[nt][1];
-                    }
-                    ptx::mma_f16(dd, pa0, pa1, pa2, pa3, b0[i], b1[i]);
-                    o[nt][0] = dd[0];
-                    o[nt][1] = dd[1];
-                    if constexpr (G16) {
-                        ob[nt][0] = dd[2];
-                        ob[nt][1] = dd[3];
-                    }
-                }
-            }
-        }
+            // ---- O += P V, sub-tile A then B
+            if (liveA)
+                pv_fp8<G16>(sb + a.v_off + jA * sub_bytes + head_off, g, tig, nvA, pA0, pA1, pA2,
+                            pA3, o, ob);
+            if (liveB)
+                pv_fp8<G16>(sb + a.v_off + jB * sub_bytes + head_off, g, tig, nvB, pB0, pB1, pB2,
+                            pB3, o, ob);
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&empty[stage]);
@@ -1313,6 +1470,7 @@ __device__ __forceinline__ void merge_wide(const Args &a, int64_t bh, int i, int
 template <int D>
 __global__ void __launch_bounds__(D) merge_tc_kernel(const Args a) {
     ptx::grid_dependency_wait();  // the decode kernel's partials are complete
+    if (a.hdr->sig != a.sig) return;  // no plan for these sizes (flagged by the decode)
     const int64_t bh = blockIdx.x;
     const int b = (int)(bh / a.Hq), i = (int)(bh % a.Hq);
     const int e = threadIdx.x;
@@ -1426,6 +1584,23 @@ cudaError_t launch_typed(const CUtensorMap &km, const CUtensorMap &vm, const Arg
 
 }  // namespace tc
 
+namespace tc {
+// The plan kernel of one decode call (writes the unit list into the workspace).
+cudaError_t launch_plan(const DecodeArgs &d, cudaStream_t st) {
+    const DecodePlan &p = d.plan;
+    char *ws = static_cast<char *>(d.ws);
+    return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, d.ctx_lens, d.err,
+                      reinterpret_cast<TcHeader *>(ws + p.off_hdr),
+                      reinterpret_cast<int32_t *>(ws + p.off_ns),
+                      reinterpret_cast<int4 *>(ws + p.off_units), d.B, d.MB * d.bs, p.chunk,
+                      p.grid * p.units_per_cta, p.sig);
+}
+}  // namespace tc
+
+cudaError_t launch_decode_plan_only(const DecodeArgs &d, cudaStream_t st) {
+    return tc::launch_plan(d, st);
+}
+
 cudaError_t launch_decode_tc(const DecodeArgs &d, int kv, cudaStream_t st) {
     using namespace tc;
     const bool int8 = kv != kKvBf16;  // one-byte pools (int8 codes or e4m3)
@@ -1470,11 +1645,12 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, int kv, cudaStream_t st) {
         a.tpb_shift = (tpb & (tpb - 1)) == 0 ? __builtin_ctz((unsigned)tpb) : -1;
     }
     a.scale_log2 = d.scale_log2;
-    const int max_ctx = d.MB * d.bs;
-    cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, d.ctx_lens, d.err, a.hdr,
-                               const_cast<int32_t *>(a.ns), const_cast<int4 *>(a.units), d.B,
-                               max_ctx, p.chunk, p.grid * p.units_per_cta);
-    if (e != cudaSuccess) return e;
+    a.sig = p.sig;
+    cudaError_t e = cudaSuccess;
+    if (!d.reuse_plan) {
+        e = launch_plan(d, st);
+        if (e != cudaSuccess) return e;
+    }
     const bool g16 = d.G > 8;
     if (kv == kKvInt8)  // one-byte pools: d == 128 only (the plan guarantees it)
         e = g16 ? launch_typed<128, true, kKvInt8>(km, vm, a, p.grid, p.smem_bytes, st)

@@ -20,14 +20,19 @@ struct AppendArgs {
     int B, n_new, Hkv, d, bs, MB;
 };
 
-// Header at the start of the staged decode's workspace (written by its plan
-// kernel every call): unit counter, unit count, partition size chosen.
+// Header at the start of the staged decode's workspace, written by its plan
+// kernel: unit counter, unit count, partition size chosen, the count of decode
+// CTAs that finished taking units (the last one resets both counters, so a plan
+// serves several decode calls), and the signature of the sizes it was made for.
 struct TcHeader {
     unsigned counter;
     int n_units;
     int chunk;
-    int pad[61];
+    unsigned done;
+    unsigned long long sig;
+    int pad[58];
 };
+static_assert(sizeof(TcHeader) == 256, "TcHeader is the workspace's 256-byte header");
 
 // Launch plan of one decode call, decided on the host from the sizes alone.
 struct DecodePlan {
@@ -39,6 +44,7 @@ struct DecodePlan {
     int n_sub;          // staged: 16-token sub-tiles per stage (wph * tpw)
     int nstage, stage_bytes, v_off, ks_off, vs_off, smem_bytes, grid, units_per_cta;
     size_t off_hdr, off_ns, off_units, off_ml, off_acc, ws_total;
+    unsigned long long sig;  // staged: signature of the sizes the device plan is made for
 };
 
 // Decode problem.  K/V element type is given by the launcher (bf16 or int8).
@@ -62,6 +68,7 @@ struct DecodeArgs {
     int chunk;                    // tokens per partition (multiple of 16 when S > 1)
     void *ws;                     // workspace base
     DecodePlan plan;
+    int reuse_plan;               // staged: the workspace already holds the plan (no plan launch)
 };
 
 struct ScoreArgs {
@@ -95,6 +102,9 @@ cudaError_t launch_select_pooled(int32_t *evict, float *means, const float *scor
 // Decode dispatch: the staged tensor-core kernel when the shape allows it,
 // else the general-shape kernel; then the partition merge when S > 1.
 cudaError_t launch_decode(const DecodeArgs &a, int kv, cudaStream_t stream);
+// Staged kernel only: the plan kernel alone (writes the partition plan of
+// a.ctx_lens into the workspace for later calls with reuse_plan set).
+cudaError_t launch_decode_plan_only(const DecodeArgs &a, cudaStream_t stream);
 cudaError_t launch_decode_simple(const DecodeArgs &a, int kv, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeArgs &a, int kv, cudaStream_t stream);
 DecodePlan make_decode_plan(int B, int Hq, int Hkv, int d, int bs, int MB, int num_splits,

@@ -58,7 +58,7 @@ int decode_entry(uint16_t *out, const uint16_t *q, const void *kc, const void *v
                  const float *vs, int kv, int64_t block_stride, const int32_t *bt, int MB,
                  const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs, int64_t N,
                  float scale, int num_splits, void *ws, size_t ws_bytes, int32_t *err,
-                 void *stream) {
+                 void *stream, int reuse_plan = 0) {
     if (B == 0) return PA_OK;  // empty batch: nothing to read or write
     if (!out || !q || !kc || !vc || !bt || !ctx_lens || !err) return PA_ERR_NULL;
     if (kv == pkv::kKvInt8 && (!ks || !vs)) return PA_ERR_NULL;
@@ -108,24 +108,27 @@ int decode_entry(uint16_t *out, const uint16_t *q, const void *kc, const void *v
     a.MB = MB;
     a.num_splits = plan.S;
     a.chunk = plan.chunk;
+    a.reuse_plan = reuse_plan;
     return finish(pkv::launch_decode(a, kv, static_cast<cudaStream_t>(stream)));
 }
 
-// Scratch for pa_decode_static_scratch: a fixed array inside the library, one
-// copy per device that loads it.  Host code must not use the symbol itself as a
-// device address; static_scratch_address() looks the address up per device.
-__device__ __align__(256) unsigned char g_static_scratch[PA_STATIC_SCRATCH_BYTES];
-std::atomic<void *> g_scratch_addr[64];
+}  // namespace
 
-// Device address of g_static_scratch on the current device (looked up once per
-// device, with that device current), or nullptr on failure.
+// Scratch for pa_decode_static_scratch: a fixed array inside the library, one
+// copy on every device that loads it, held until the process exits.  In host code
+// the name g_static_scratch is a host-side stand-in, not a device address; the
+// address comes from static_scratch_address().
+static __device__ __align__(256) unsigned char g_static_scratch[PA_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_static_scratch on the current device, or nullptr on failure.
+// Looked up on every call, with the calling device current: a host-side lookup
+// that allocates nothing, and stays right when the context is reset and the
+// library's device code is loaded again at another address.
 void *static_scratch_address() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    void *p = g_scratch_addr[dev].load();
-    if (p) return p;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return nullptr;
-    g_scratch_addr[dev].store(p);
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
     return p;
 }
 
@@ -343,6 +346,68 @@ int pa_decode_fp8(uint16_t *out, const uint16_t *q, const uint8_t *k8_cache,
                         scale, num_splits, workspace, workspace_bytes, err_flag, stream);
 }
 
+int pa_decode_prepare(const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
+                      int max_blocks_per_seq, int num_splits, void *workspace,
+                      size_t workspace_bytes, int32_t *err_flag, void *stream) {
+    if (B == 0) return PA_OK;
+    if (!ctx_lens || !err_flag) return PA_ERR_NULL;
+    if (B < 0 || B > 65535 || Hkv < 1 || Hkv > 65535 || bs < 1 || max_blocks_per_seq < 1)
+        return PA_ERR_SHAPE;
+    if (d != 64 && d != 128) return PA_ERR_SHAPE;
+    if ((int64_t)max_blocks_per_seq * bs > INT32_MAX) return PA_ERR_SHAPE;
+    if (Hq < Hkv || Hq % Hkv != 0 || Hq / Hkv > 16) return PA_ERR_SHAPE;
+    const int sms = device_sms();
+    if (sms < 0) return sms;
+    const pkv::DecodePlan plan =
+        pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, num_splits, pkv::kKvBf16, sms);
+    if (plan.kernel != 1) return PA_OK;  // the general-shape kernel keeps no device plan
+    if (!workspace || workspace_bytes < plan.ws_total) return PA_ERR_WORKSPACE;
+    if (!al16(workspace)) return PA_ERR_ALIGN;
+    pkv::DecodeArgs a;
+    memset(&a, 0, sizeof a);
+    a.ctx_lens = ctx_lens;
+    a.err = err_flag;
+    a.ws = workspace;
+    a.plan = plan;
+    a.B = B;
+    a.MB = max_blocks_per_seq;
+    a.bs = bs;
+    return finish(pkv::launch_decode_plan_only(a, static_cast<cudaStream_t>(stream)));
+}
+
+int pa_decode_planned(uint16_t *out, const uint16_t *q, const uint16_t *k_cache,
+                      const uint16_t *v_cache, int64_t block_stride, const int32_t *block_tables,
+                      int max_blocks_per_seq, const int32_t *ctx_lens, int B, int Hq, int Hkv,
+                      int d, int bs, int64_t num_blocks, float scale, int num_splits,
+                      void *workspace, size_t workspace_bytes, int32_t *err_flag, void *stream) {
+    return decode_entry(out, q, k_cache, v_cache, nullptr, nullptr, pkv::kKvBf16, block_stride,
+                        block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
+                        scale, num_splits, workspace, workspace_bytes, err_flag, stream, 1);
+}
+
+int pa_decode_int8_planned(uint16_t *out, const uint16_t *q, const int8_t *kq_cache,
+                           const int8_t *vq_cache, const float *k_scale, const float *v_scale,
+                           int64_t block_stride, const int32_t *block_tables,
+                           int max_blocks_per_seq, const int32_t *ctx_lens, int B, int Hq,
+                           int Hkv, int d, int bs, int64_t num_blocks, float scale,
+                           int num_splits, void *workspace, size_t workspace_bytes,
+                           int32_t *err_flag, void *stream) {
+    return decode_entry(out, q, kq_cache, vq_cache, k_scale, v_scale, pkv::kKvInt8, block_stride,
+                        block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
+                        scale, num_splits, workspace, workspace_bytes, err_flag, stream, 1);
+}
+
+int pa_decode_fp8_planned(uint16_t *out, const uint16_t *q, const uint8_t *k8_cache,
+                          const uint8_t *v8_cache, int64_t block_stride,
+                          const int32_t *block_tables, int max_blocks_per_seq,
+                          const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
+                          int64_t num_blocks, float scale, int num_splits, void *workspace,
+                          size_t workspace_bytes, int32_t *err_flag, void *stream) {
+    return decode_entry(out, q, k8_cache, v8_cache, nullptr, nullptr, pkv::kKvFp8, block_stride,
+                        block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
+                        scale, num_splits, workspace, workspace_bytes, err_flag, stream, 1);
+}
+
 int pe_score_tokens(float *scores, const uint16_t *k_cache, const uint16_t *v_cache,
                     int64_t block_stride, const int32_t *block_tables, int max_blocks_per_seq,
                     const int32_t *ctx_lens, int B, int Hkv, int d, int bs, int64_t num_blocks,
@@ -392,29 +457,28 @@ int pa_decode_static_scratch(uint16_t *out, const uint16_t *q, const uint16_t *k
     const int sms = device_sms();
     if (sms < 0) return sms;
     const size_t cap = PA_STATIC_SCRATCH_BYTES;
+    auto ws_for = [&](int s) {
+        return pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, s, pkv::kKvBf16, sms)
+            .ws_total;
+    };
     int splits = num_splits;
-    if (splits == 0) {
-        // largest partition count whose scratch fits, starting from the automatic one
-        int auto_s = pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, 0, pkv::kKvBf16, sms).S;
-        int lo = 1, hi = auto_s < 1 ? 1 : auto_s;
-        if (pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, hi, pkv::kKvBf16, sms)
-                .ws_total <= cap) {
-            lo = hi;
-        } else {
-            while (lo < hi) {  // invariant: ws(lo) fits or lo == 1
-                const int mid = (lo + hi + 1) / 2;
-                if (pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, mid, pkv::kKvBf16, sms)
-                        .ws_total <= cap)
-                    lo = mid;
-                else
-                    hi = mid - 1;
-            }
+    if (splits == 0 && ws_for(0) > cap) {
+        // the automatic plan does not fit: the largest partition count whose scratch
+        // fits (an explicit count; when the automatic plan fits, 0 is passed on and the
+        // call partitions exactly as pa_decode does)
+        int lo = 1, hi = pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, 0,
+                                               pkv::kKvBf16, sms).S;
+        if (hi < 1) hi = 1;
+        while (lo < hi) {  // invariant: ws(lo) fits or lo == 1
+            const int mid = (lo + hi + 1) / 2;
+            if (ws_for(mid) <= cap)
+                lo = mid;
+            else
+                hi = mid - 1;
         }
         splits = lo;
     }
-    if (pkv::make_decode_plan(B, Hq, Hkv, d, bs, max_blocks_per_seq, splits, pkv::kKvBf16, sms).ws_total >
-        cap)
-        return PA_ERR_WORKSPACE;
+    if (ws_for(splits) > cap) return PA_ERR_WORKSPACE;
     void *ws = static_scratch_address();
     if (!ws) return PA_ERR_CUDA;
     return decode_entry(out, q, k_cache, v_cache, nullptr, nullptr, pkv::kKvBf16, block_stride,

@@ -29,12 +29,15 @@ PA_DEV_BAD_BLOCK = 1
 PA_DEV_BAD_LEN = 2
 PA_DEV_TIMEOUT = 4
 PA_DEV_BAD_EVICT = 8
+PA_DEV_BAD_PLAN = 16
 
 EXPORTED = (
     "pa_status_string", "pa_version", "pa_append_kv", "pa_decode_workspace_bytes", "pa_decode_plan",
     "pa_decode",
     "pe_score_tokens", "pe_select_evict_block", "pa_append_kv_int8", "pa_decode_int8",
-    "pa_decode_static_scratch", "pa_append_kv_scored", "pa_append_kv_int8_scored",
+    "pa_decode_static_scratch", "pa_decode_prepare", "pa_decode_planned",
+    "pa_decode_int8_planned", "pa_decode_fp8_planned", "pa_append_kv_scored",
+    "pa_append_kv_int8_scored",
     "pe_select_evict_block_pooled", "pa_append_kv_fp8", "pa_decode_fp8",
     "pe_prefill_scores", "pe_prefill_select", "pe_prefill_pack", "pe_prefill_compress",
     "pe_evict_compact", "pe_select_evict_threshold", "pe_evict_compact_mask",
@@ -81,6 +84,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode_int8.restype = i32
     lib.pa_decode_int8.argtypes = [p, p, p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, i64,
                                    f32, i32, p, sz, p, p]
+    lib.pa_decode_prepare.restype = i32
+    lib.pa_decode_prepare.argtypes = [p, i32, i32, i32, i32, i32, i32, i32, p, sz, p, p]
+    lib.pa_decode_planned.restype = i32
+    lib.pa_decode_planned.argtypes = lib.pa_decode.argtypes
+    lib.pa_decode_int8_planned.restype = i32
+    lib.pa_decode_int8_planned.argtypes = lib.pa_decode_int8.argtypes
     lib.pa_decode_static_scratch.restype = i32
     lib.pa_decode_static_scratch.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32,
                                              i64, f32, i32, p, p]
@@ -98,6 +107,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode_fp8.restype = i32
     lib.pa_decode_fp8.argtypes = [p, p, p, p, i64, p, i32, p, i32, i32, i32, i32, i32, i64, f32,
                                   i32, p, sz, p, p]
+    lib.pa_decode_fp8_planned.restype = i32
+    lib.pa_decode_fp8_planned.argtypes = lib.pa_decode_fp8.argtypes
     lib.pe_prefill_scores.restype = i32
     lib.pe_prefill_scores.argtypes = [p, p, p, i64, i32, i32, p]
     lib.pe_prefill_select.restype = i32
@@ -307,6 +318,43 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
               workspace=None, num_splits=0, stream=None):
     """Paged decode attention (bf16 pools): out[b, i] = softmax(scale q.K) V over
     the ctx_lens[b] tokens of sequence b, kv head i // (Hq/Hkv)."""
+    _decode_bf16("pa_decode", out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
+                 workspace, num_splits, stream)
+
+
+def pa_decode_planned(out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
+                      workspace=None, num_splits=0, stream=None):
+    """pa_decode with the partition plan pa_decode_prepare left in the workspace."""
+    _decode_bf16("pa_decode_planned", out, q, k_cache, v_cache, block_tables, ctx_lens, scale,
+                 err_flag, workspace, num_splits, stream)
+
+
+def pa_decode_prepare(q, k_cache, block_tables, ctx_lens, err_flag, workspace, num_splits=0,
+                      stream=None):
+    """Write the partition plan of ctx_lens into the workspace for the planned decode
+    calls of the same sizes (q [B, Hq, d] and the pool [N, bs, Hkv, d], bf16 or one-byte,
+    give the sizes)."""
+    _want(block_tables, torch.int32, "block_tables")
+    _want(ctx_lens, torch.int32, "ctx_lens")
+    _want(err_flag, torch.int32, "err_flag")
+    N, bs, Hkv, d, _ = _pool_geometry(k_cache, "k_cache")
+    if q.dim() != 3 or q.shape[2] != d:
+        raise ValueError("q must be [B, Hq, d] with the pool's d")
+    B, Hq = q.shape[0], q.shape[1]
+    _table_rows(block_tables, B)
+    _covers(ctx_lens, B, "ctx_lens")
+    _covers(err_flag, 1, "err_flag")
+    _one_device(k_cache, block_tables, ctx_lens, err_flag, workspace)
+    ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel() *
+                                                        workspace.element_size())
+    rc = load().pa_decode_prepare(_ptr(ctx_lens.contiguous()), B, Hq, Hkv, d, bs,
+                                  block_tables.shape[1], int(num_splits), ws_ptr, ws_n,
+                                  _ptr(err_flag), _stream(stream))
+    _check("pa_decode_prepare", rc)
+
+
+def _decode_bf16(fn, out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
+                 workspace, num_splits, stream):
     _decode_checks(out, q, block_tables, ctx_lens, err_flag)
     _want(k_cache, torch.bfloat16, "k_cache")
     _want(v_cache, torch.bfloat16, "v_cache")
@@ -319,11 +367,11 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
     bt = block_tables.contiguous()
     ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel() *
                                                         workspace.element_size())
-    rc = load().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), stride, _ptr(bt),
-                          bt.shape[1], _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d, bs, N,
-                          float(scale), int(num_splits), ws_ptr, ws_n, _ptr(err_flag),
-                          _stream(stream))
-    _check("pa_decode", rc)
+    rc = getattr(load(), fn)(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), stride, _ptr(bt),
+                             bt.shape[1], _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d, bs, N,
+                             float(scale), int(num_splits), ws_ptr, ws_n, _ptr(err_flag),
+                             _stream(stream))
+    _check(fn, rc)
 
 
 def pa_decode_static_scratch(out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
@@ -352,6 +400,19 @@ def pa_decode_static_scratch(out, q, k_cache, v_cache, block_tables, ctx_lens, s
 def pa_decode_int8(out, q, kq_cache, vq_cache, k_scale, v_scale, block_tables, ctx_lens, scale,
                    err_flag, workspace=None, num_splits=0, stream=None):
     """Paged decode attention over INT8 pools dequantised in registers."""
+    _decode_int8("pa_decode_int8", out, q, kq_cache, vq_cache, k_scale, v_scale, block_tables,
+                 ctx_lens, scale, err_flag, workspace, num_splits, stream)
+
+
+def pa_decode_int8_planned(out, q, kq_cache, vq_cache, k_scale, v_scale, block_tables, ctx_lens,
+                           scale, err_flag, workspace=None, num_splits=0, stream=None):
+    """pa_decode_int8 with the partition plan pa_decode_prepare left in the workspace."""
+    _decode_int8("pa_decode_int8_planned", out, q, kq_cache, vq_cache, k_scale, v_scale,
+                 block_tables, ctx_lens, scale, err_flag, workspace, num_splits, stream)
+
+
+def _decode_int8(fn, out, q, kq_cache, vq_cache, k_scale, v_scale, block_tables, ctx_lens, scale,
+                 err_flag, workspace, num_splits, stream):
     _decode_checks(out, q, block_tables, ctx_lens, err_flag)
     _want(kq_cache, torch.int8, "kq_cache")
     _want(vq_cache, torch.int8, "vq_cache")
@@ -370,11 +431,11 @@ def pa_decode_int8(out, q, kq_cache, vq_cache, k_scale, v_scale, block_tables, c
     bt = block_tables.contiguous()
     ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel() *
                                                         workspace.element_size())
-    rc = load().pa_decode_int8(_ptr(out), _ptr(q), _ptr(kq_cache), _ptr(vq_cache), _ptr(k_scale),
-                               _ptr(v_scale), stride, _ptr(bt), bt.shape[1],
-                               _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d, bs, N, float(scale),
-                               int(num_splits), ws_ptr, ws_n, _ptr(err_flag), _stream(stream))
-    _check("pa_decode_int8", rc)
+    rc = getattr(load(), fn)(_ptr(out), _ptr(q), _ptr(kq_cache), _ptr(vq_cache),
+                             _ptr(k_scale), _ptr(v_scale), stride, _ptr(bt), bt.shape[1],
+                             _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d, bs, N, float(scale),
+                             int(num_splits), ws_ptr, ws_n, _ptr(err_flag), _stream(stream))
+    _check(fn, rc)
 
 
 # ----------------------------------------------------------------------------- eviction
@@ -552,6 +613,19 @@ def pa_append_kv_fp8(k_new, v_new, k8_cache, v8_cache, block_tables, positions, 
 def pa_decode_fp8(out, q, k8_cache, v8_cache, block_tables, ctx_lens, scale, err_flag,
                   workspace=None, num_splits=0, stream=None):
     """Paged decode attention over e4m3 pools, widened exactly in registers."""
+    _decode_fp8("pa_decode_fp8", out, q, k8_cache, v8_cache, block_tables, ctx_lens, scale,
+                err_flag, workspace, num_splits, stream)
+
+
+def pa_decode_fp8_planned(out, q, k8_cache, v8_cache, block_tables, ctx_lens, scale, err_flag,
+                          workspace=None, num_splits=0, stream=None):
+    """pa_decode_fp8 with the partition plan pa_decode_prepare left in the workspace."""
+    _decode_fp8("pa_decode_fp8_planned", out, q, k8_cache, v8_cache, block_tables, ctx_lens,
+                scale, err_flag, workspace, num_splits, stream)
+
+
+def _decode_fp8(fn, out, q, k8_cache, v8_cache, block_tables, ctx_lens, scale, err_flag,
+                workspace, num_splits, stream):
     _decode_checks(out, q, block_tables, ctx_lens, err_flag)
     _want(k8_cache, torch.uint8, "k8_cache")
     _want(v8_cache, torch.uint8, "v8_cache")
@@ -564,11 +638,11 @@ def pa_decode_fp8(out, q, k8_cache, v8_cache, block_tables, ctx_lens, scale, err
     bt = block_tables.contiguous()
     ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel() *
                                                         workspace.element_size())
-    rc = load().pa_decode_fp8(_ptr(out), _ptr(q), _ptr(k8_cache), _ptr(v8_cache), stride,
-                              _ptr(bt), bt.shape[1], _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d,
-                              bs, N, float(scale), int(num_splits), ws_ptr, ws_n, _ptr(err_flag),
-                              _stream(stream))
-    _check("pa_decode_fp8", rc)
+    rc = getattr(load(), fn)(_ptr(out), _ptr(q), _ptr(k8_cache), _ptr(v8_cache), stride,
+                             _ptr(bt), bt.shape[1], _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d,
+                             bs, N, float(scale), int(num_splits), ws_ptr, ws_n, _ptr(err_flag),
+                             _stream(stream))
+    _check(fn, rc)
 
 
 # ----------------------------------------------------------------------------- prefill stage

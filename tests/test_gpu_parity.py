@@ -85,16 +85,31 @@ def _parity(wl, layers, num_splits=0, score=None, pad=0):
 
 
 def test_tiny_workload_full_step():
+    """[VKV] §2.1 append_slot and [KVL] "PagedEviction 块级驱逐机制" on the tiny workload:
+    both pools after the append equal the oracle's bit for bit, and each sequence
+    evicts exactly the oracle's block (its decision margins are large)."""
     wl = W.generate(C["c1"], "cpu")
     dev, refs = _parity(wl, [0], score=True)
-    # pool after the append equals the oracle's, bit for bit (tiny pool: compare all of it)
+    # pools after the append equal the oracle's, bit for bit (tiny pool: compare all of it)
     ref = refs[0]
-    s = ref["compact"]
-    ids = wl.block_tables[wl.block_tables >= 0]
-    got_k = dev.k_pool[0][torch.as_tensor(ids, device="cuda")].view(torch.int16).cpu().numpy()
-    assert np.array_equal(got_k.view(np.uint16).ravel(), ref["kc"])
-    # the two full blocks per sequence and the decision (38 -> 2 full, 101 -> 6 full)
+    ids = torch.as_tensor(wl.block_tables[wl.block_tables >= 0], device="cuda")
+    for pool, key in ((dev.k_pool, "kc"), (dev.v_pool, "vc")):
+        got = pool[0][ids].view(torch.int16).cpu().numpy()
+        assert np.array_equal(got.view(np.uint16).ravel(), ref[key]), key
+    # 38 -> 2 full blocks, 101 -> 6 full blocks; the rest are not candidates
     assert (ref["means"][0, 2:] != ref["means"][0, 2:]).all()
+    assert (ref["means"][1, 6:] != ref["means"][1, 6:]).all()
+    assert ((ref["evict"] >= 0) & (ref["evict"] < [2, 6])).all()
+    # the choice is unconditional here: the gap to the runner-up is far above what
+    # 1e-5-relative scores can move a block mean by
+    assert (ref["gap"] > 1e-3).all()
+    got_evict = torch.full((2,), -9, dtype=torch.int32, device="cuda")
+    scores = torch.empty(2, wl.max_blocks * 16, C["c1"].hkv, dtype=torch.float32, device="cuda")
+    pk.pe_score_tokens(scores, dev.k_pool[0], dev.v_pool[0], dev.bt, dev.ctx, dev.err)
+    pk.pe_select_evict_block(got_evict, scores, dev.ctx, 16)
+    torch.cuda.synchronize()
+    assert dev.err.item() == 0
+    assert got_evict.cpu().numpy().tolist() == ref["evict"].tolist()
 
 
 @pytest.mark.parametrize("key", list(MEDIUM))
@@ -340,3 +355,52 @@ def test_fp8_append_special_values_bit_exact():
     assert np.array_equal(gotv, oracle.quantize_e4m3(W.bits(v)).ravel())
     # nothing else in the pools was touched
     assert int(k8.count_nonzero()) == int(np.count_nonzero(got))
+
+
+def wide_range_queries(q: torch.Tensor, seed: int) -> torch.Tensor:
+    """Query rows whose magnitudes span the bf16 range, one kind per query head
+    (cycling): a row mixing 3e4, N(0,1) and 1e-4 elements; a row scaled by 1e5
+    (every element beyond fp16's 65504 for most); per-element magnitudes 2^-20 ..
+    2^12; N(0,1) rows scaled by 10, 30, 300 and 1e-30; one element of 7e4 among
+    N(0,1).  The page's INT8 and FP8 caches quantise K and V only ([VKV] §6.1
+    quantize_kv_cache); the query stays bf16, so every bf16 row is a valid input."""
+    g = torch.Generator().manual_seed(seed)
+    L, B, Hq, d = q.shape
+    out = torch.randn(L, B, Hq, d, generator=g, dtype=torch.float64)
+    for i in range(Hq):
+        kind = i % 8
+        r = out[:, :, i]
+        if kind == 0:
+            r[..., 0] = 3e4
+            r[..., d // 3:] *= 1e-4
+            perm = torch.randperm(d, generator=g)
+            out[:, :, i] = r[..., perm]
+        elif kind == 1:
+            r *= 1e5
+        elif kind == 2:
+            e = torch.randint(-20, 13, r.shape, generator=g).double()
+            r.copy_(torch.sign(r) * torch.pow(2.0, e) * (1 + torch.rand(r.shape, generator=g,
+                                                                       dtype=torch.float64)))
+        elif kind == 3:
+            r *= 10
+        elif kind == 4:
+            r *= 30
+        elif kind == 5:
+            r *= 300
+        elif kind == 6:
+            r *= 1e-30
+        else:
+            r[..., 5] = -7e4
+    return out.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("key", ["c5m", "i8g16", "i8d64", "f8", "f8g16", "f8d64", "c3m", "c2m"])
+def test_wide_range_queries(key):
+    """INT8 (three-part int8 query on the staged kernel), FP8 (power-of-two prescaled fp16
+    query), bf16 and the general kernels against the fp64 oracle on queries whose
+    magnitudes span the bf16 range; no device flag is raised."""
+    cfg = W.scaled(MEDIUM[key], score=False)
+    wl = W.generate(cfg, "cpu")
+    wl.q.copy_(wide_range_queries(wl.q, 396 + len(key)))
+    assert wl.q.float().abs().max() > 65504
+    _parity(wl, list(range(wl.q.shape[0])))

@@ -116,11 +116,20 @@ def _dec(fn, lib, *, kv="bf16", **kw):
     if fn == "fp8":
         return lib.pa_decode_fp8(a["out"], a["q"], a["k"], a["v"], *common, None, 0, a["err"],
                                  None)
+    if fn == "planned":
+        return lib.pa_decode_planned(a["out"], a["q"], a["k"], a["v"], *common, None, 0,
+                                     a["err"], None)
+    if fn == "int8_planned":
+        return lib.pa_decode_int8_planned(a["out"], a["q"], a["k"], a["v"], a["ks"], a["vs"],
+                                          *common, None, 0, a["err"], None)
+    if fn == "fp8_planned":
+        return lib.pa_decode_fp8_planned(a["out"], a["q"], a["k"], a["v"], *common, None, 0,
+                                         a["err"], None)
     return lib.pa_decode_static_scratch(a["out"], a["q"], a["k"], a["v"], *common, a["err"], None)
 
 
 def test_decode_variants_reject_bad_arguments_on_host(lib):
-    for fn in ("int8", "fp8", "static"):
+    for fn in ("int8", "fp8", "static", "planned", "int8_planned", "fp8_planned"):
         assert _dec(fn, lib, q=NUL) == -1, fn
         assert _dec(fn, lib, err=NUL) == -1, fn
         assert _dec(fn, lib, Hq=24, Hkv=16) == -2, fn      # Hq % Hkv != 0
@@ -138,6 +147,29 @@ def test_decode_variants_reject_bad_arguments_on_host(lib):
     assert _dec("fp8", lib, stride=S + 8) == -3
     assert _dec("static", lib, S=-1) == -2
     assert _dec("static", lib, stride=S + 4) == -3         # bf16: 8 bytes
+    assert _dec("int8_planned", lib, ks=NUL) == -1
+    assert _dec("planned", lib, stride=S + 4) == -3
+
+
+def test_decode_prepare_rejects_bad_arguments_on_host(lib):
+    def prep(**kw):
+        a = dict(ctx=FAKE, B=2, Hq=32, Hkv=8, d=128, bs=16, MB=4, S=0, ws=None, wsb=0, err=FAKE)
+        a.update(kw)
+        return lib.pa_decode_prepare(a["ctx"], a["B"], a["Hq"], a["Hkv"], a["d"], a["bs"],
+                                     a["MB"], a["S"], a["ws"], a["wsb"], a["err"], None)
+    assert prep(ctx=NUL) == -1
+    assert prep(err=NUL) == -1
+    assert prep(B=-1) == -2
+    assert prep(B=65536) == -2
+    assert prep(Hq=30) == -2
+    assert prep(Hq=8 * 17) == -2
+    assert prep(d=96) == -2
+    assert prep(bs=0) == -2
+    assert prep(MB=(1 << 27) + 1) == -2
+    assert prep(B=0) == 0
+    # valid sizes stop at the missing workspace on a GPU machine, or at the device query
+    # without one: never a launch
+    assert prep() in (-4, -5, -6)
 
 
 def test_appends_reject_bad_arguments_on_host(lib):
