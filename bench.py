@@ -66,8 +66,15 @@ def parse():
                          "and select blocks from it (incremental)")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling aid: keep only this many layers of the workload")
+    ap.add_argument("--plan", default="step", choices=["step", "call"],
+                    help="staged decode: make the partition plan once per step "
+                         "(pa_decode_prepare + planned calls) or inside every decode call")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--secondary", default=None,
+                    help="comma-separated workloads also measured and reported under "
+                         "'secondary' in the same JSON line (c5-fp8 = c5 on e4m3 pools); "
+                         f"default for the c3 line: {'c4,c2,c5,c5-fp8,p1,p2'}, else none")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every call from Python instead of replaying a CUDA graph")
     return ap.parse_args()
@@ -216,7 +223,8 @@ def decode_algorithmic_bytes(cfg, ctx_lens, partial_slots, n_units=0):
 class Runner:
     """Device state and one decode step of a workload through the binding."""
 
-    def __init__(self, cfg, device, num_splits=0, wl=None, evict="full"):
+    def __init__(self, cfg, device, num_splits=0, wl=None, evict="full", plan="step",
+                 overlap_select=True):
         from paged_kv_cache_396_b200 import pagedkv as pk
         self.pk, self.cfg, self.dev = pk, cfg, device
         wl = W.generate(cfg, device) if wl is None else wl
@@ -233,6 +241,10 @@ class Runner:
         self.num_splits = num_splits
         self.S, self.chunk, self.dec_launches, self.staged = pk.pa_decode_plan(
             B, Hq, Hkv, d, bs, MB, num_splits)
+        # the staged kernel's partition plan: once per step (pa_decode_prepare, then the
+        # planned calls) or inside every decode call; the general kernel keeps no plan
+        self.per_step_plan = self.staged and plan == "step" and not (
+            (cfg.int8 or cfg.fp8) and d != 128)
         if cfg.fp8:
             N = wl.num_blocks
             self.k8 = torch.zeros(self.L, N, bs, Hkv, d, dtype=torch.uint8, device=device)
@@ -268,6 +280,12 @@ class Runner:
         if cfg.score:
             self.scores = torch.zeros(B, MB * bs, Hkv, dtype=torch.float32, device=device)
             self.evict = torch.zeros(B, dtype=torch.int32, device=device)
+        # incremental eviction: the block choice of a layer overlaps its decode (a second
+        # stream joined at the end of the step) unless overlap is off
+        self.side = (torch.cuda.Stream(device) if self.incremental and overlap_select
+                     else None)
+        self.ev_app = [torch.cuda.Event() for _ in range(self.L)]
+        self.ev_join = torch.cuda.Event()
         if self.incremental:
             # paged score pools, filled for the cached history once (set-up): score
             # every cached token, then place each score at its token's slot
@@ -306,51 +324,67 @@ class Runner:
         self.partitions = slots
 
     def launches_per_step(self):
-        per_layer = (1 if self.cfg.append else 0) + self.dec_launches
+        dec = self.dec_launches - (1 if self.per_step_plan else 0)
+        per_layer = (1 if self.cfg.append else 0) + dec
         if self.cfg.score:
             per_layer += 1 if self.incremental else 2
-        return per_layer * self.L
+        return per_layer * self.L + (1 if self.per_step_plan else 0)
 
     def step(self, ev=None):
         pk, cfg = self.pk, self.cfg
+        if self.per_step_plan:
+            # every layer of the step has the same context lengths: one partition plan
+            pk.pa_decode_prepare(self.q[0], self.wl.k_pool[0] if self.wl.k_pool is not None
+                                 else self.kq[0] if cfg.int8 else self.k8[0], self.bt, self.ctx,
+                                 self.err, self.ws, self.num_splits)
+        dec = pk.pa_decode_planned if self.per_step_plan else pk.pa_decode
+        dec8 = pk.pa_decode_int8_planned if self.per_step_plan else pk.pa_decode_int8
+        decf8 = pk.pa_decode_fp8_planned if self.per_step_plan else pk.pa_decode_fp8
         for l in range(self.L):
             if cfg.fp8:
                 pk.pa_append_kv_fp8(self.k_new[l], self.v_new[l], self.k8[l], self.v8[l], self.bt,
                                     self.pos, self.err)
                 if ev is not None:
                     ev[l][0].record()
-                pk.pa_decode_fp8(self.out[l], self.q[l], self.k8[l], self.v8[l], self.bt, self.ctx,
-                                 self.wl.scale, self.err, self.ws, self.num_splits)
+                decf8(self.out[l], self.q[l], self.k8[l], self.v8[l], self.bt, self.ctx,
+                      self.wl.scale, self.err, self.ws, self.num_splits)
             elif cfg.int8:
                 pk.pa_append_kv_int8(self.k_new[l], self.v_new[l], self.kq[l], self.vq[l],
                                      self.ks[l], self.vs[l], self.bt, self.pos, self.err)
                 if ev is not None:
                     ev[l][0].record()
-                pk.pa_decode_int8(self.out[l], self.q[l], self.kq[l], self.vq[l], self.ks[l],
-                                  self.vs[l], self.bt, self.ctx, self.wl.scale, self.err, self.ws,
-                                  self.num_splits)
+                dec8(self.out[l], self.q[l], self.kq[l], self.vq[l], self.ks[l], self.vs[l],
+                     self.bt, self.ctx, self.wl.scale, self.err, self.ws, self.num_splits)
             else:
                 kp = self.wl.k_pool[l]
                 vp = self.wl.v_pool[l]
                 if cfg.append and self.incremental:
                     pk.pa_append_kv_scored(self.k_new[l], self.v_new[l], kp, vp,
                                            self.score_pool[l], self.bt, self.pos, self.err)
+                    if self.side is not None:
+                        # the block choice needs only this layer's score pool: it runs on
+                        # a second stream beside the decode
+                        self.ev_app[l].record()
+                        self.side.wait_event(self.ev_app[l])
                 elif cfg.append:
                     pk.pa_append_kv(self.k_new[l], self.v_new[l], kp, vp, self.bt, self.pos,
                                     self.err)
                 if ev is not None:
                     ev[l][0].record()
-                pk.pa_decode(self.out[l], self.q[l], kp, vp, self.bt, self.ctx, self.wl.scale,
-                             self.err, self.ws, self.num_splits)
+                dec(self.out[l], self.q[l], kp, vp, self.bt, self.ctx, self.wl.scale, self.err,
+                    self.ws, self.num_splits)
             if ev is not None:
                 ev[l][1].record()
             if self.incremental:
                 pk.pe_select_evict_block_pooled(self.evict, self.score_pool[l], self.bt, self.ctx,
-                                                self.err)
+                                                self.err, stream=self.side)
             elif cfg.score:
                 pk.pe_score_tokens(self.scores, self.wl.k_pool[l], self.wl.v_pool[l], self.bt,
                                    self.ctx, self.err)
                 pk.pe_select_evict_block(self.evict, self.scores, self.ctx, cfg.block_size)
+        if self.side is not None:   # the step ends when the block choices are made
+            self.ev_join.record(self.side)
+            torch.cuda.current_stream().wait_event(self.ev_join)
 
 
 # ----------------------------------------------------------------------------- oracle
@@ -441,6 +475,43 @@ def oracle_throughput(wl, budget_s, max_layers=None):
     return cfg.batch / step_s, cores, desc
 
 
+def reference_samples(args, sample):
+    """The reference arm's timing loop: W warm-up samples (a quarter of the budget
+    each) and K timed ones.  sample(budget_s) runs the oracle on a bounded part of the
+    workload for about budget_s seconds and returns (throughput, cores, description).
+    Returns the median throughput, the cores, the last description and the host wall
+    time of one timed sample in ms (the reference arm's "step")."""
+    per = max(1.0, args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        sample(per / 4)
+    vals, walls, desc, cores = [], [], "", 0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        v, cores, desc = sample(per)
+        walls.append(1000.0 * (time.perf_counter() - t0))
+        vals.append(v)
+    return statistics.median(vals), cores, desc, statistics.mean(walls)
+
+
+def reference_line(args, metric, unit, value, cores, desc, wall_ms, full_step_ms, config):
+    """One JSON line of the reference arm.  A step here is one bounded sample of the
+    workload's step (ms_per_step is its measured host wall time, so steps x
+    ms_per_step is the time actually spent); value is the oracle's throughput over
+    the samples, and ms_per_full_step_extrapolated the whole step at that rate."""
+    return {
+        "impl": "reference", "metric": metric, "value": value, "unit": unit,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": wall_ms, "ms_per_full_step_extrapolated": full_step_ms,
+        "step": "one bounded sample of the workload's step on the host cores",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config,
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": "per step: " + desc},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -451,27 +522,11 @@ def run_reference(args):
         return run_reference_chunked(args)
     cfg = workload_cfg(args)
     wl = W.generate(cfg, "cpu", layers=1)
-    per = max(1.0, args.cpu_seconds / max(1, args.steps))
-    for _ in range(args.warmup):
-        oracle_throughput(wl, per / 4, max_layers=1)
-    vals = []
-    desc = ""
-    cores = 0
-    for _ in range(args.steps):
-        v, cores, desc = oracle_throughput(wl, per, max_layers=1)
-        vals.append(v)
-    value = statistics.median(vals)
-    line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1000.0 * cfg.batch / value, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(cfg),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": "per step: " + desc},
-        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
-                "d2h_bytes_per_step": 0},
-    }
+    value, cores, desc, wall = reference_samples(
+        args, lambda t: oracle_throughput(wl, t, max_layers=1))
+    line = reference_line(args, METRIC, "tokens/s", value, cores, desc, wall,
+                          1000.0 * cfg.batch / value,
+                          dict(workload_config(cfg), parallelism="replicas1"))
     print(json.dumps(line), flush=True)
     return 0
 
@@ -492,6 +547,25 @@ def traffic_key(args, cfg):
     return args.workload + ("" if args.kv is None else "-" + kv_name(cfg))
 
 
+METRIC_P1 = "PagedEviction prefill compression: prompt tokens/s and score-kernel HBM GB/s"
+METRIC_P2 = "chunked prefill attention: chunk tokens/s and tensor TFLOP/s"
+
+
+def prefill_config(cfg, world):
+    return {"workload": f"{cfg.key} {cfg.name}", "prompts": cfg.batch,
+            "prompt_tokens": cfg.prompt_lens[0], "kv_heads": cfg.hkv, "head_dim": cfg.head_dim,
+            "block_size": cfg.block_size, "budget": cfg.budget, "parallelism": f"replicas{world}",
+            "l2": "prompt rows (1 GiB) larger than L2 every step (no flush needed)"}
+
+
+def chunked_config(cfg, world):
+    return {"workload": f"{cfg.key} {cfg.name}", "sequences": cfg.batch, "chunk": cfg.chunk,
+            "context": cfg.ctx_len, "q_heads": cfg.hq, "kv_heads": cfg.hkv,
+            "head_dim": cfg.head_dim, "block_size": cfg.block_size,
+            "parallelism": f"replicas{world}",
+            "l2": "flushed (256 MB write) before every timed step"}
+
+
 def run_reference_prefill(args):
     """The oracle's prefill stage timed on bounded samples of the prefill workload."""
     import dataclasses
@@ -499,27 +573,11 @@ def run_reference_prefill(args):
     # one prompt's worth of rows per sample keeps the host footprint small
     small = dataclasses.replace(cfg, batch=4, prompt_lens=cfg.prompt_lens[:4])
     wl = W.generate_prefill(small, "cpu")
-    per = max(1.0, args.cpu_seconds / max(1, args.steps))
-    for _ in range(args.warmup):
-        prefill_oracle_throughput(wl, per / 4)
-    vals, desc, cores = [], "", 0
-    for _ in range(args.steps):
-        v, cores, desc = prefill_oracle_throughput(wl, per)
-        vals.append(v)
-    value = statistics.median(vals)
+    value, cores, desc, wall = reference_samples(
+        args, lambda t: prefill_oracle_throughput(wl, t))
     T = sum(cfg.prompt_lens)
-    line = {
-        "impl": "reference", "metric": "PagedEviction prefill compression: prompt tokens/s",
-        "value": value, "unit": "prompt tokens/s", "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1000.0 * T / value, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{cfg.key} {cfg.name}", "prompts": cfg.batch,
-                   "prompt_tokens": cfg.prompt_lens[0], "budget": cfg.budget},
-        "cpu_baseline": {"value": value, "unit": "prompt tokens/s", "cores": cores,
-                         "kind": "oracle", "sample": "per step: " + desc},
-        "e2e": {"value": value, "unit": "prompt tokens/s", "h2d_bytes_per_step": 0,
-                "d2h_bytes_per_step": 0},
-    }
+    line = reference_line(args, METRIC_P1, "prompt tokens/s", value, cores, desc, wall,
+                          1000.0 * T / value, prefill_config(cfg, 1))
     print(json.dumps(line), flush=True)
     return 0
 
@@ -528,27 +586,10 @@ def run_reference_chunked(args):
     """The oracle's chunked prefill attention timed on row samples of the workload."""
     cfg = W.CHUNKED[args.workload]
     wl = W.generate_chunked(cfg, "cpu")
-    per = max(1.0, args.cpu_seconds / max(1, args.steps))
-    for _ in range(args.warmup):
-        chunk_oracle_throughput(wl, per / 4)
-    vals, desc, cores = [], "", 0
-    for _ in range(args.steps):
-        v, cores, desc = chunk_oracle_throughput(wl, per)
-        vals.append(v)
-    value = statistics.median(vals)
-    line = {
-        "impl": "reference", "metric": "chunked prefill attention: chunk tokens/s",
-        "value": value, "unit": "chunk tokens/s", "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.batch * cfg.chunk / value,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic",
-        "config": {"workload": f"{cfg.key} {cfg.name}", "sequences": cfg.batch,
-                   "chunk": cfg.chunk, "context": cfg.ctx_len},
-        "cpu_baseline": {"value": value, "unit": "chunk tokens/s", "cores": cores,
-                         "kind": "oracle", "sample": "per step: " + desc},
-        "e2e": {"value": value, "unit": "chunk tokens/s", "h2d_bytes_per_step": 0,
-                "d2h_bytes_per_step": 0},
-    }
+    value, cores, desc, wall = reference_samples(
+        args, lambda t: chunk_oracle_throughput(wl, t))
+    line = reference_line(args, METRIC_P2, "chunk tokens/s", value, cores, desc, wall,
+                          1000.0 * cfg.batch * cfg.chunk / value, chunked_config(cfg, 1))
     print(json.dumps(line), flush=True)
     return 0
 
@@ -602,7 +643,7 @@ def prefill_oracle_throughput(wl, budget_s):
     return tok / t_total, cores, desc
 
 
-def run_prefill(args, device, world, rank):
+def run_prefill(args, device, world, rank, cpu_baseline=True):
     """One step = the prefill stage of one layer for every prompt of the
     workload: token scores, keep sets, packing of the kept rows into the pool."""
     import paged_kv_cache_396_b200.pagedkv as pk
@@ -655,9 +696,9 @@ def run_prefill(args, device, world, rank):
     clk = clocks.stop()
     ms = reduce_max(t0.elapsed_time(t1), world) / args.steps
     per = [[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in evs]
-    score_s = statistics.mean(p[0] for p in per) / 1000.0
-    select_s = statistics.mean(p[1] for p in per) / 1000.0
-    pack_s = statistics.mean(p[2] for p in per) / 1000.0
+    score_s = statistics.median(p[0] for p in per) / 1000.0
+    select_s = statistics.median(p[1] for p in per) / 1000.0
+    pack_s = statistics.median(p[2] for p in per) / 1000.0
     # algorithmic bytes: every prompt row of K and V read once plus one fp32 score
     # written per token (score kernel); kept rows read and written (pack)
     score_bytes = T * Hkv * d * 2 * 2 + T * 4
@@ -690,44 +731,39 @@ def run_prefill(args, device, world, rank):
     if err.item() != 0:
         raise SystemExit(f"device error flag {err.item()} during timing")
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if cpu_baseline and rank == 0 and world == 1 and not args.no_cpu_baseline:
         host_wl = W.PrefillWorkload(cfg, wl.k.cpu(), wl.v.cpu(), wl.cu_seqlens, wl.block_tables, N)
         v_, cores, desc = prefill_oracle_throughput(host_wl, args.cpu_seconds)
         cpu = {"value": v_, "unit": "prompt tokens/s", "cores": cores, "kind": "oracle",
                "sample": desc}
         cpu = with_single_core(cpu, lambda t: prefill_oracle_throughput(host_wl, t),
                                args.cpu_seconds)
-    if rank == 0:
-        line = {
-            "metric": "PagedEviction prefill compression: prompt tokens/s and score-kernel "
-                      "HBM GB/s", "value": world * T / (ms / 1000.0), "unit": "prompt tokens/s",
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": f"{cfg.key} {cfg.name}", "prompts": B,
-                       "prompt_tokens": cfg.prompt_lens[0], "kv_heads": Hkv, "head_dim": d,
-                       "block_size": bs, "budget": budget, "parallelism": f"replicas{world}",
-                       "l2": "prompt rows (1 GiB) larger than L2 every step (no flush needed)"},
-            "roofline": {"bound": "hbm", "kernel": "pe_prefill_scores", "achieved": achieved,
-                         "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
-                         "frac": achieved / peak,
-                         "traffic": recorded_traffic("p1", "prefill_traffic.txt",
-                                                     PREFILL_SOURCES["p1"]),
-                         "algorithmic_bytes_per_launch": score_bytes,
-                         "avg_launch_us": score_s * 1e6},
-            "kernels_us": {"pe_prefill_scores": score_s * 1e6,
-                           "pe_prefill_select": select_s * 1e6,
-                           "pe_prefill_pack": pack_s * 1e6},
-            "pack_gbs": pack_bytes / pack_s / 1e9,
-            "cpu_baseline": cpu,
-            "e2e": {"value": world * T / (e2e_ms / 1000.0), "unit": "prompt tokens/s",
-                    "h2d_bytes_per_step": 2 * T * Hkv * d * 2,
-                    "d2h_bytes_per_step": (B * budget + B) * 4, "ms_per_step": e2e_ms},
-            "gpu_launches": 3 * args.steps,
-            "clocks": clk,
-        }
-        print(json.dumps(line), flush=True)
-    return 0
+    line = {
+        "metric": METRIC_P1, "value": world * T / (ms / 1000.0), "unit": "prompt tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": prefill_config(cfg, world),
+        "roofline": {"bound": "hbm", "kernel": "pe_prefill_scores", "achieved": achieved,
+                     "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak,
+                     "traffic": recorded_traffic("p1", "prefill_traffic.txt",
+                                                 PREFILL_SOURCES["p1"]),
+                     "algorithmic_bytes_per_launch": score_bytes,
+                     "avg_launch_us": score_s * 1e6,
+                     "launch_time_statistic": f"median of {args.steps} launches"},
+        "kernels_us": {"pe_prefill_scores": score_s * 1e6,
+                       "pe_prefill_select": select_s * 1e6,
+                       "pe_prefill_pack": pack_s * 1e6},
+        "pack_gbs": pack_bytes / pack_s / 1e9,
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * T / (e2e_ms / 1000.0), "unit": "prompt tokens/s",
+                "h2d_bytes_per_step": 2 * T * Hkv * d * 2,
+                "d2h_bytes_per_step": (B * budget + B) * 4, "ms_per_step": e2e_ms},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+    }
+    return line
 
 
 # ----------------------------------------------------------------------------- chunked prefill
@@ -772,7 +808,7 @@ def chunk_oracle_throughput(wl, budget_s):
     return cfg.batch * cfg.chunk / step_s, oracle.threads(), desc
 
 
-def run_chunked(args, device, world, rank):
+def run_chunked(args, device, world, rank, cpu_baseline=True):
     """One step = append the chunk's K/V rows and run the multi-query attention
     for every sequence of the workload."""
     import paged_kv_cache_396_b200.pagedkv as pk
@@ -825,7 +861,7 @@ def run_chunked(args, device, world, rank):
         total += t0.elapsed_time(t1)
     clk = clocks.stop()
     ms = reduce_max(total / args.steps, world)
-    attn_s = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) / 1000.0
+    attn_s = statistics.median(e[0].elapsed_time(e[1]) for e in evs) / 1000.0
     flops = chunk_flops(cfg)
     peak_t = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"] \
         if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 1590.0
@@ -854,7 +890,7 @@ def run_chunked(args, device, world, rank):
     if err.item() != 0:
         raise SystemExit(f"device error flag {err.item()} during timing")
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if cpu_baseline and rank == 0 and world == 1 and not args.no_cpu_baseline:
         host_wl = W.ChunkWorkload(cfg, wl.k_pool.cpu(), wl.v_pool.cpu(), wl.k_new.cpu(),
                                   wl.v_new.cpu(), wl.q.cpu(), wl.cu_q, wl.ctx_lens, wl.positions,
                                   wl.block_tables, wl.num_blocks)
@@ -863,91 +899,92 @@ def run_chunked(args, device, world, rank):
                "sample": desc}
         cpu = with_single_core(cpu, lambda t: chunk_oracle_throughput(host_wl, t),
                                args.cpu_seconds)
-    if rank == 0:
-        line = {
-            "metric": "chunked prefill attention: chunk tokens/s and tensor TFLOP/s",
-            "value": world * Tq / (ms / 1000.0), "unit": "chunk tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": f"{cfg.key} {cfg.name}", "sequences": B,
-                       "chunk": cfg.chunk, "context": cfg.ctx_len, "q_heads": cfg.hq,
-                       "kv_heads": cfg.hkv, "head_dim": cfg.head_dim,
-                       "block_size": cfg.block_size, "parallelism": f"replicas{world}",
-                       "l2": "flushed (256 MB write) before every timed step"},
-            "roofline": {"bound": "tensor", "kernel": "pa_prefill_attention",
-                         "achieved": achieved, "peak": peak_t, "peak_source": "measured burst",
-                         "unit": "TFLOP/s", "frac": achieved / peak_t,
-                         "traffic": recorded_traffic("p2", "prefill_traffic.txt",
-                                                     PREFILL_SOURCES["p2"]),
-                         "algorithmic_flops_per_launch": flops, "avg_launch_us": attn_s * 1e6},
-            "cpu_baseline": cpu,
-            "e2e": {"value": world * Tq / (e2e_ms / 1000.0), "unit": "chunk tokens/s",
-                    "h2d_bytes_per_step": sum(t.numel() * t.element_size() for _, t in h_in),
-                    "d2h_bytes_per_step": out.numel() * out.element_size(),
-                    "ms_per_step": e2e_ms},
-            "gpu_launches": (1 + attn_launches) * args.steps,
-            "clocks": clk,
-        }
-        print(json.dumps(line), flush=True)
-    return 0
+    line = {
+        "metric": METRIC_P2,
+        "value": world * Tq / (ms / 1000.0), "unit": "chunk tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": chunked_config(cfg, world),
+        "roofline": {"bound": "tensor", "kernel": "pa_prefill_attention",
+                     "achieved": achieved, "peak": peak_t, "peak_source": "measured burst",
+                     "unit": "TFLOP/s", "frac": achieved / peak_t,
+                     "traffic": recorded_traffic("p2", "prefill_traffic.txt",
+                                                 PREFILL_SOURCES["p2"]),
+                     "algorithmic_flops_per_launch": flops, "avg_launch_us": attn_s * 1e6,
+                     "launch_time_statistic": f"median of {args.steps} launches"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * Tq / (e2e_ms / 1000.0), "unit": "chunk tokens/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for _, t in h_in),
+                "d2h_bytes_per_step": out.numel() * out.element_size(),
+                "ms_per_step": e2e_ms},
+        "gpu_launches": (1 + attn_launches) * args.steps,
+        "clocks": clk,
+    }
+    return line
 
 
-# ----------------------------------------------------------------------------- main
-def main():
-    args = parse()
-    if args.impl == "reference":
-        return run_reference(args)
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=device)
-    if args.workload in W.PREFILL or args.workload in W.CHUNKED:
-        fn = run_prefill if args.workload in W.PREFILL else run_chunked
-        rc = fn(args, device, world, rank)
-        if world > 1:
-            torch.distributed.barrier()
-            torch.distributed.destroy_process_group()
-        return rc
-    cfg = workload_cfg(args)
-    if args.layers:
-        cfg = W.scaled(cfg, layers=args.layers)
-    r = Runner(cfg, device, args.num_splits, evict=args.evict)
+# ----------------------------------------------------------------------------- decode
+# distinct captured graphs kept for per-call statistics (older ones are replayed again)
+MAX_GRAPHS = 64
+
+
+def call_stats(call_ms, layers, batch, world):
+    """Median duration (ms) of the decode call over every sample, and the decode-only
+    throughput it implies: a step decodes `batch` tokens per rank through `layers`
+    decode calls, so tokens/s = world * batch / (layers * median call time)."""
+    med = statistics.median(call_ms)
+    return med, world * batch / (layers * med / 1000.0)
+
+
+def chunk_plan(steps, per_graph):
+    """Steps per graph replay of the timed region: full graphs of `per_graph` steps,
+    then one shorter graph for the remainder."""
+    full, rest = divmod(steps, per_graph)
+    return [per_graph] * full + ([rest] if rest else [])
+
+
+def run_decode(args, cfg, device, world, rank, cpu_baseline=True):
+    """One decode workload: warm-up, K timed steps (CUDA graphs of the step with an
+    event pair around every decode call), the end-to-end pass and, optionally, the
+    oracle's CPU baseline.  Returns the JSON line as a dict (printed by rank 0)."""
+    r = Runner(cfg, device, args.num_splits, evict=args.evict, plan=args.plan)
     stream = torch.cuda.current_stream(device)
-
     for _ in range(max(3, args.warmup)):
         r.step()
     torch.cuda.synchronize(device)
     if r.err.item() != 0:
         raise SystemExit(f"device error flag {r.err.item()} during warm-up")
-
     r.account_bytes()
     use_graph = not args.no_graph
-    R = max(1, -(-16 // r.L))          # steps per captured graph: >= 16 decode samples
+    # steps per captured graph: at least 20 decode calls per replay
+    R = max(1, -(-20 // r.L))
 
-    def capture(steps, with_events):
-        ev = ([[torch.cuda.Event(enable_timing=True, external=True),
-                torch.cuda.Event(enable_timing=True, external=True)]
-               for _ in range(r.L * steps)] if with_events else None)
+    def capture(steps):
+        ev = [[torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True)] for _ in range(r.L * steps)]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for k in range(steps):
-                r.step(ev[k * r.L:(k + 1) * r.L] if ev else None)
+                r.step(ev[k * r.L:(k + 1) * r.L])
         return g, ev
 
+    plan = chunk_plan(args.steps, R)
     if use_graph:
-        gR, evR = capture(R, True)
-        g1, ev1 = capture(1, True)
-        gR.replay()
-        g1.replay()
+        # full-size graphs: up to MAX_GRAPHS distinct ones (each keeps its own events),
+        # replayed in turn; the remainder graph is its own
+        n_full = sum(1 for n in plan if n == R)
+        full_graphs = [capture(R) for _ in range(min(n_full, MAX_GRAPHS))]
+        rest_graph = capture(plan[-1]) if plan and plan[-1] != R else None
+        order, j = [], 0
+        for n in plan:
+            if n == R:
+                order.append(full_graphs[j % len(full_graphs)])
+                j += 1
+            else:
+                order.append(rest_graph)
+        for g, _ in full_graphs + ([rest_graph] if rest_graph else []):
+            g.replay()
         torch.cuda.synchronize(device)
     else:
         ev_eager = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
@@ -963,31 +1000,29 @@ def main():
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     if use_graph:
-        for _ in range(args.steps // R):
-            gR.replay()
-        for _ in range(args.steps % R):
-            g1.replay()
+        for g, _ in order:
+            g.replay()
     else:
         for k in range(args.steps):
             r.step(ev_eager[k * r.L:(k + 1) * r.L])
     t_end.record(stream)
     torch.cuda.synchronize(device)
     clk = clocks.stop()
-    total_ms = t_start.elapsed_time(t_end)
+    total_ms = reduce_max(t_start.elapsed_time(t_end), world)
     if use_graph:
-        samples = evR if args.steps >= R else ev1
+        used = {id(g): ev for g, ev in order}      # every distinct graph that ran
+        samples = [pair for ev in used.values() for pair in ev]
     else:
         samples = ev_eager
-    decode_ms = [a.elapsed_time(b) for a, b in samples]
-    total_ms = reduce_max(total_ms, world)
+    call_ms = [a.elapsed_time(b) for a, b in samples]
     ms_per_step = total_ms / args.steps
     value = job_tokens_per_s(world, cfg.batch, ms_per_step)
-    dec_avg_s = statistics.mean(decode_ms) / 1000.0
-    achieved = r.decode_bytes / dec_avg_s / 1e9
+    med_ms, decode_only = call_stats(call_ms, r.L, cfg.batch, world)
+    achieved = r.decode_bytes / (med_ms / 1000.0) / 1e9
     peak, peak_kind = peaks()
 
     # --- end to end: host inputs -> C ABI -> host outputs, copies inside the timed region
-    B, Hq, Hkv, d = cfg.batch, cfg.hq, cfg.hkv, cfg.head_dim
+    B = cfg.batch
     h_q = torch.empty(r.q.shape, dtype=torch.bfloat16, pin_memory=True)
     h_q.copy_(r.q)
     h_out = torch.empty(r.out.shape, dtype=torch.bfloat16, pin_memory=True)
@@ -1029,45 +1064,105 @@ def main():
             e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(device)
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    e2e_ms = reduce_max(e2e_ms, world)
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, world)
     e2e = {"value": job_tokens_per_s(world, B, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
     if r.err.item() != 0:
         raise SystemExit(f"device error flag {r.err.item()} during timing")
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if cpu_baseline and rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, desc = oracle_throughput(r.wl, args.cpu_seconds)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
         cpu = with_single_core(cpu, lambda t: oracle_throughput(r.wl, t), args.cpu_seconds)
 
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": {"fp8_e4m3": "e4m3"}.get(kv_name(cfg), kv_name(cfg)), "data": "synthetic",
+        "config": dict(workload_config(cfg), parallelism=f"replicas{world}"),
+        "launch": {"decode_kernel": "staged-tc" if r.staged else "general",
+                   "evict_scoring": ("incremental score pool" if r.incremental else
+                                     "full pass per layer") if cfg.score else None,
+                   "partitions": r.partitions, "chunk_tokens": r.chunk_used,
+                   "partition_plan": "once per step" if r.per_step_plan else "every call",
+                   "cuda_graph": use_graph, "steps_per_graph": R if use_graph else None},
+        "roofline": {"bound": "hbm", "kernel": {"bf16": "pa_decode", "int8": "pa_decode_int8",
+                                               "fp8_e4m3": "pa_decode_fp8"}[kv_name(cfg)],
+                     "achieved": achieved, "peak": peak, "peak_source": peak_kind,
+                     "unit": "GB/s", "frac": achieved / peak,
+                     "frac_of_nominal_8tbs": achieved / 8000.0,
+                     "traffic": recorded_traffic(traffic_key(args, cfg)),
+                     "algorithmic_bytes_per_launch":
+                         r.decode_bytes,
+                     "avg_launch_us": med_ms * 1000.0, "launch_time_statistic":
+                         f"median of {len(call_ms)} decode calls in the timed region"},
+        "decode_only_tokens_per_s": decode_only,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": r.launches_per_step() * args.steps,
+        "clocks": clk,
+    }
+    del r
+    torch.cuda.empty_cache()
+    return line
+
+
+SECONDARY_DEFAULT = "c4,c2,c5,c5-fp8,p1,p2"
+
+
+def secondary_args(args, spec):
+    """The parsed arguments for one secondary workload ("c5-fp8": c5 on e4m3 pools; c2
+    runs with the incremental score pool)."""
+    import copy
+    a = copy.copy(args)
+    name, _, kv = spec.partition("-")
+    a.workload = name
+    a.kv = kv or None
+    a.layers = 0
+    a.evict = "incremental" if name == "c2" else args.evict
+    return a
+
+
+def run_one(args, device, world, rank, cpu_baseline=True):
+    if args.workload in W.PREFILL:
+        return run_prefill(args, device, world, rank, cpu_baseline)
+    if args.workload in W.CHUNKED:
+        return run_chunked(args, device, world, rank, cpu_baseline)
+    cfg = workload_cfg(args)
+    if args.layers:
+        cfg = W.scaled(cfg, layers=args.layers)
+    return run_decode(args, cfg, device, world, rank, cpu_baseline)
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    line = run_one(args, device, world, rank)
+    spec = args.secondary
+    if spec is None:
+        spec = SECONDARY_DEFAULT if (args.workload == "c3" and args.kv is None and
+                                     not args.layers) else ""
+    extra = [w for w in spec.split(",") if w]
+    if extra:
+        line["secondary"] = [run_one(secondary_args(args, w), device, world, rank,
+                                     cpu_baseline=False) for w in extra]
     if rank == 0:
-        traffic = recorded_traffic(traffic_key(args, cfg))
-        line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": {"fp8_e4m3": "e4m3"}.get(kv_name(cfg), kv_name(cfg)), "data": "synthetic",
-            "config": dict(workload_config(cfg), parallelism=f"replicas{world}",
-                           decode_kernel="staged-tc" if r.staged else "general",
-                           evict_scoring=("incremental score pool" if r.incremental else
-                                          "full pass per layer") if cfg.score else None,
-                           partitions=r.partitions, chunk_tokens=r.chunk_used,
-                           cuda_graph=use_graph),
-            "roofline": {"bound": "hbm", "kernel": {"bf16": "pa_decode", "int8": "pa_decode_int8",
-                                                   "fp8_e4m3": "pa_decode_fp8"}[kv_name(cfg)],
-                         "achieved": achieved, "peak": peak, "peak_source": peak_kind,
-                         "unit": "GB/s", "frac": achieved / peak,
-                         "frac_of_nominal_8tbs": achieved / 8000.0,
-                         "traffic": traffic, "algorithmic_bytes_per_launch": r.decode_bytes,
-                         "avg_launch_us": dec_avg_s * 1e6},
-            "decode_only_tokens_per_s": world * B / (sum(decode_ms) / args.steps / 1000.0),
-            "cpu_baseline": cpu,
-            "e2e": e2e,
-            "gpu_launches": r.launches_per_step() * args.steps,
-            "clocks": clk,
-        }
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

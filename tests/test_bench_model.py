@@ -4,6 +4,7 @@ bytes against the marginal cost of one more cached token."""
 import dataclasses
 
 import numpy as np
+import pytest
 
 import bench
 from paged_kv_cache_396_b200 import workloads as W
@@ -43,3 +44,22 @@ def test_decode_bytes_include_partials_both_ways():
     b = bench.decode_algorithmic_bytes(cfg, lens, 3)
     # three partition slots of Hq rows: (d + 2) fp32 written and read back
     assert b - a == 2 * 3 * cfg.hq * (cfg.head_dim + 2) * 4
+
+
+def test_decode_only_throughput_is_batch_over_the_layers_of_one_step():
+    """A step decodes B tokens per rank through L decode calls (one per layer); with the
+    median call time t, the decode-only throughput is world * B / (L * t), whatever the
+    number of steps the samples came from."""
+    calls = [0.2, 0.25, 0.3, 0.21, 0.19] * 8        # ms; 40 samples from several steps
+    med, tok_s = bench.call_stats(calls, layers=32, batch=64, world=1)
+    assert med == 0.21
+    assert tok_s == pytest.approx(64 / (32 * 0.21e-3), rel=1e-12)
+    _, tok_s2 = bench.call_stats(calls, layers=32, batch=64, world=4)
+    assert tok_s2 == pytest.approx(4 * tok_s, rel=1e-12)
+
+
+def test_timed_region_runs_exactly_the_requested_steps():
+    for steps, per in ((20, 1), (20, 20), (20, 16), (7, 16), (200, 3), (1, 1)):
+        plan = bench.chunk_plan(steps, per)
+        assert sum(plan) == steps
+        assert all(n == per for n in plan[:-1]) and 0 < plan[-1] <= per

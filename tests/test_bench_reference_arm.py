@@ -19,9 +19,16 @@ def _bench(workload, rank="0"):
                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
 
 
+def _timed_bench(workload):
+    import time
+    t0 = time.perf_counter()
+    r = _bench(workload)
+    return r, time.perf_counter() - t0
+
+
 @pytest.mark.parametrize("workload", ["c2", "p1"])
 def test_reference_arm_prints_one_contract_line(workload):
-    r = _bench(workload)
+    r, wall_s = _timed_bench(workload)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
     assert len(lines) == 1
@@ -41,6 +48,9 @@ def test_reference_arm_prints_one_contract_line(workload):
     assert cb["cores"] >= 1 and cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    # a step is one bounded sample: the steps claimed fit in the time the run took
+    assert line["steps"] * line["ms_per_step"] / 1000.0 < wall_s
+    assert line["ms_per_full_step_extrapolated"] > 0
 
 
 def test_reference_arm_other_ranks_do_nothing():
