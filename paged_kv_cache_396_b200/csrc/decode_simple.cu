@@ -300,24 +300,42 @@ DecodePlan make_decode_plan(int B, int Hq, int Hkv, int d, int bs, int MB, int n
     }
     if (tc) {
         p.kernel = 1;
-        int64_t mc = 128;
-        if (num_splits > 0) mc = ((max_ctx + num_splits - 1) / num_splits + 15) / 16 * 16;
-        if (mc < 16) mc = 16;
-        p.chunk = (int)mc;
-        p.S = (int)((max_ctx + mc - 1) / mc);
         p.grid = sms;
         p.units_per_cta = 4;
+        int64_t mc = 128;
+        size_t n_units;
+        if (num_splits > 0 || sms >= 1024) {
+            // explicit split: at most num_splits near-equal partitions per sequence,
+            // taken by the CTAs from a counter, longest first (also the automatic
+            // split on a GPU with more SMs than the balanced plan's ranges)
+            if (num_splits > 0) mc = ((max_ctx + num_splits - 1) / num_splits + 15) / 16 * 16;
+            if (mc < 16) mc = 16;
+            p.S = (int)((max_ctx + mc - 1) / mc);
+            n_units = (size_t)B * p.S;
+        } else {
+            // automatic split: the concatenated contexts are cut into one equal range
+            // of at least mc tokens per CTA (cuts snapped to 16-token tiles); a
+            // sequence holds at most ceil(len / mc) cuts, so at most that many + 1
+            // pieces, and all pieces number at most B + grid
+            p.balanced = 1;
+            p.S = (int)((max_ctx + mc - 1) / mc) + 1;
+            n_units = (size_t)B + (size_t)p.grid;
+        }
+        p.chunk = (int)mc;
         const size_t slots = (size_t)B * p.S * p.wph * Hq;
         p.off_hdr = 0;
         p.off_ns = 256;
         p.off_units = p.off_ns + up256((size_t)B * 4);
-        p.off_ml = p.off_units + up256((size_t)B * p.S * 16);
+        p.off_cta = p.off_units + up256(n_units * 16);
+        p.off_starts = p.off_cta + up256((size_t)(p.grid + 1) * 4);
+        p.off_ml = p.off_starts + up256(p.balanced ? (size_t)B * 8 : 0);
         p.off_acc = p.off_ml + up256(slots * 2 * 4);
         p.ws_total = p.off_acc + up256(slots * d * 4);
         // sizes the device plan depends on (a plan kept in a workspace is only used by
         // calls of the same signature): FNV-1a over them.  The element type is not
         // among them: bf16, INT8 and FP8 calls of the same sizes share one plan.
-        const long long f[10] = {B, Hq, Hkv, d, bs, MB, p.S, p.chunk, p.grid, p.units_per_cta};
+        const long long f[11] = {B,      Hq,     Hkv,    d,      bs,           MB,
+                                 p.S,    p.chunk, p.grid, p.units_per_cta, p.balanced};
         unsigned long long h = 1469598103934665603ull;
         for (long long v : f) {
             h ^= (unsigned long long)v;

@@ -7,12 +7,16 @@
 // the whole context; GQA (§6.2 of the first page): query head i reads kv head i/G.
 //
 // Work decomposition
-//   A plan kernel (one CTA) reads the device context lengths, cuts every
-//   sequence into near-equal partitions of at most `chunk` tokens (chunk sized
-//   so that there are a few partitions per SM), and writes the partitions as a
-//   unit list sorted longest first.  The decode kernel is persistent (one CTA
-//   per SM); its producer warp takes units from an atomic counter, so long units
-//   start first and short ones fill the tail.
+//   A plan kernel (one CTA) reads the device context lengths and writes the
+//   units (sequence, partition, token range) into the workspace.  The decode
+//   kernel is persistent (one CTA per SM).
+//   Automatic split: the contexts, laid end to end, are cut into one equal
+//   token range per SM (at least 128 tokens); a cut inside a sequence snaps to
+//   that sequence's 16-token tiles.  CTA i takes the pieces of range i, so every
+//   SM reads the same number of K/V bytes whatever the mix of lengths.
+//   Explicit split (num_splits > 0): every sequence is cut into near-equal
+//   partitions of at most max_ctx / num_splits tokens, listed longest first, and
+//   the producers take them from an atomic counter.
 // Per CTA
 //   warp 8 (producer): for each stage of 16*n_sub tokens (n_sub sub-tiles of 16
 //   tokens; a stage carries about 64 KB of K and V), lane j looks the physical
@@ -86,6 +90,8 @@ struct Args {
     int tpb_shift;  // log2(bs / 16) when bs / 16 is a power of two, else -1
     float scale_log2;
     unsigned long long sig;  // signature of the sizes; must match the plan's (header)
+    const int32_t *cta_off;  // balanced plan: CTA i takes units cta_off[i] .. cta_off[i+1]-1
+    int balanced;
 };
 
 // ---------------------------------------------------------------------------
@@ -229,6 +235,166 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t *ctx_lens, int
     }
 }
 
+// Exclusive prefix sum over the 1024 threads of a CTA (64-bit); *total gets the sum.
+__device__ __forceinline__ long long cta_scan64(long long v, long long *total) {
+    __shared__ long long s_w[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    long long inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(kFull, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) s_w[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        long long x = s_w[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_up_sync(kFull, x, o);
+            if (lane >= o) x += y;
+        }
+        s_w[lane] = x;   // inclusive totals of warps 0..lane
+    }
+    __syncthreads();
+    const long long before = warp ? s_w[warp - 1] : 0;
+    *total = s_w[31];
+    __syncthreads();
+    return before + inc - v;
+}
+
+// ---------------------------------------------------------------------------
+// balanced plan (automatic split): one CTA of 1024 threads.
+// The contexts, laid end to end (T tokens), are cut into nr equal ranges of
+// `range` = max(16-token multiple of ceil(T / P), min_chunk) tokens, one per decode
+// CTA (nr <= P).  A cut that falls inside a sequence is snapped to the nearest
+// 16-token tile boundary of that sequence, so every piece starts on a tile.  A
+// range's pieces (its parts of consecutive sequences) go to its CTA; piece c of
+// sequence b is partition c of b (ns[b] pieces; a sequence of length 0 has none
+// and the merge writes its zero row).
+// ---------------------------------------------------------------------------
+constexpr int kMaxRanges = 1024;
+
+__global__ void __launch_bounds__(1024) plan_balanced_kernel(
+    const int32_t *ctx_lens, int32_t *err, TcHeader *hdr, int32_t *ns, int4 *units,
+    int32_t *cta_off, long long *starts, int B, int max_ctx, int min_chunk, int P,
+    unsigned long long sig) {
+    __shared__ long long s_R[kMaxRanges + 1];   // snapped cut positions R_0 .. R_nr
+    __shared__ int s_cnt[kMaxRanges];          // pieces per range, then fill positions
+    __shared__ long long s_range, s_T;
+    __shared__ int s_nr;
+    const int tid = threadIdx.x;
+    ptx::grid_launch_dependents();
+    ptx::grid_dependency_wait();
+    auto clamp_len = [&](int b, bool flag) {
+        int len = ctx_lens[b];
+        if (len < 0 || len > max_ctx) {
+            if (flag) raise_flag(err, PA_DEV_BAD_LEN);
+            len = 0;
+        }
+        return len;
+    };
+    // ---- sequence starts (exclusive prefix sums of the lengths)
+    long long run = 0;
+    for (int b0 = 0; b0 < B; b0 += 1024) {
+        const int b = b0 + tid;
+        const int len = b < B ? clamp_len(b, true) : 0;
+        long long tot;
+        const long long st = run + cta_scan64(len, &tot);
+        if (b < B) starts[b] = st;
+        run += tot;
+    }
+    if (tid == 0) {
+        const long long T = run;
+        long long r = (T + P - 1) / P;
+        r = (r + kTile - 1) / kTile * kTile;
+        if (r < min_chunk) r = min_chunk;
+        s_range = r;
+        s_T = T;
+        s_nr = T > 0 ? (int)((T + r - 1) / r) : 0;
+    }
+    __syncthreads();
+    const long long range = s_range, T = s_T;
+    const int nr = s_nr;
+    for (int i = tid; i <= nr; i += 1024) s_R[i] = i < nr ? (long long)i * range : T;
+    for (int i = tid; i < kMaxRanges; i += 1024) s_cnt[i] = 0;
+    __syncthreads();
+    // ---- cuts inside a sequence snap to its 16-token tiles (a sequence's thread
+    // writes the cuts that fall strictly inside it); partitions per sequence
+    for (int b = tid; b < B; b += 1024) {
+        const int len = clamp_len(b, false);
+        const long long st = starts[b];
+        int n = len > 0 ? 1 : 0;
+        if (len > 0) {
+            for (long long i = st / range + 1; i * range < st + len && i < nr; ++i) {
+                const long long o = i * range - st;          // 0 < o < len
+                long long sn = (o + kTile / 2) / kTile * kTile;
+                if (sn >= len) sn = len;
+                s_R[i] = st + sn;
+                if (sn > 0 && sn < len) ++n;
+            }
+        }
+        ns[b] = n;
+    }
+    __syncthreads();
+    // ---- owner range of every piece (the range its first token falls in): count
+    auto owner_of = [&](long long x) {   // largest i < nr with R_i <= x
+        int lo = 0, hi = nr - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_R[mid] <= x) lo = mid;
+            else hi = mid - 1;
+        }
+        return lo;
+    };
+    for (int b = tid; b < B; b += 1024) {
+        const int len = clamp_len(b, false);
+        if (len == 0) continue;
+        const long long st = starts[b];
+        int i = owner_of(st);
+        atomicAdd(&s_cnt[i], 1);
+        for (++i; i < nr && s_R[i] < st + len; ++i)
+            if (s_R[i] > st) atomicAdd(&s_cnt[i], 1);
+    }
+    __syncthreads();
+    // ---- per-range unit offsets (exclusive scan over the ranges; ranges >= nr empty)
+    {
+        long long tot;
+        const int c = tid < nr ? s_cnt[tid] : 0;
+        const long long off = cta_scan64(c, &tot);
+        if (tid <= P) cta_off[tid] = (int)(tid < nr ? off : tot);
+        if (tid < nr) s_cnt[tid] = (int)off;   // fill position of range tid
+        if (tid == 0) {
+            hdr->n_units = (int)tot;
+            hdr->chunk = (int)min(range, (long long)INT32_MAX);
+            hdr->counter = 0u;
+            hdr->done = 0u;
+            hdr->sig = sig;
+        }
+    }
+    __syncthreads();
+    // ---- the pieces: sequence b's cuts in order give partitions c = 0, 1, ...
+    for (int b = tid; b < B; b += 1024) {
+        const int len = clamp_len(b, false);
+        if (len == 0) continue;
+        const long long st = starts[b];
+        int i = owner_of(st);
+        int c = 0;
+        long long t0 = st;
+        for (;;) {
+            int j = i + 1;   // next cut strictly inside the sequence, if any
+            while (j < nr && s_R[j] <= t0) ++j;
+            const long long t1 = (j < nr && s_R[j] < st + len) ? s_R[j] : st + len;
+            const int pos = atomicAdd(&s_cnt[i], 1);
+            units[pos] = make_int4(b, c, (int)(t0 - st), (int)(t1 - st));
+            if (t1 >= st + len) break;
+            i = j;
+            t0 = t1;
+            ++c;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // decode: persistent, warp-specialised
 // ---------------------------------------------------------------------------
@@ -247,7 +413,11 @@ __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensor
     // a plan made for other sizes (a kept plan that does not match this call) is
     // not used: no unit is taken and the call flags it
     const bool plan_ok = a.hdr->sig == a.sig;
-    const int n_units = plan_ok ? a.hdr->n_units : 0;
+    // balanced plan: this CTA's own list of units; otherwise all units, longest first,
+    // taken from the counter
+    const int u_first = plan_ok && a.balanced ? a.cta_off[blockIdx.x] : 0;
+    const int n_units = !plan_ok ? 0 : a.balanced ? a.cta_off[blockIdx.x + 1] : a.hdr->n_units;
+    int u_next = u_first;
     if (!plan_ok && lane == 0 && blockIdx.x == 0) raise_flag(a.err, PA_DEV_BAD_PLAN);
     const uint64_t policy = ptx::policy_evict_first();
     int stage = 0;
@@ -259,8 +429,12 @@ __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensor
     }
     while (ok) {
         unsigned u = 0;
-        if (lane == 0) u = atomicAdd(&a.hdr->counter, 1u);
-        u = __shfl_sync(kFull, u, 0);
+        if (a.balanced) {
+            u = (unsigned)u_next++;
+        } else {
+            if (lane == 0) u = atomicAdd(&a.hdr->counter, 1u);
+            u = __shfl_sync(kFull, u, 0);
+        }
         if ((int)u >= n_units) break;
         const int4 un = a.units[u];
         const int b = un.x, c = un.y, t0 = un.z, t1 = un.w;
@@ -1589,6 +1763,14 @@ namespace tc {
 cudaError_t launch_plan(const DecodeArgs &d, cudaStream_t st) {
     const DecodePlan &p = d.plan;
     char *ws = static_cast<char *>(d.ws);
+    if (p.balanced)
+        return launch_pdl(plan_balanced_kernel, dim3(1), dim3(1024), 0, st, d.ctx_lens, d.err,
+                          reinterpret_cast<TcHeader *>(ws + p.off_hdr),
+                          reinterpret_cast<int32_t *>(ws + p.off_ns),
+                          reinterpret_cast<int4 *>(ws + p.off_units),
+                          reinterpret_cast<int32_t *>(ws + p.off_cta),
+                          reinterpret_cast<long long *>(ws + p.off_starts), d.B, d.MB * d.bs,
+                          p.chunk, p.grid, p.sig);
     return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, d.ctx_lens, d.err,
                       reinterpret_cast<TcHeader *>(ws + p.off_hdr),
                       reinterpret_cast<int32_t *>(ws + p.off_ns),
@@ -1619,6 +1801,8 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, int kv, cudaStream_t st) {
     a.hdr = reinterpret_cast<TcHeader *>(ws + p.off_hdr);
     a.ns = reinterpret_cast<const int32_t *>(ws + p.off_ns);
     a.units = reinterpret_cast<const int4 *>(ws + p.off_units);
+    a.cta_off = reinterpret_cast<const int32_t *>(ws + p.off_cta);
+    a.balanced = p.balanced;
     a.ws_ml = reinterpret_cast<float *>(ws + p.off_ml);
     a.ws_acc = reinterpret_cast<float *>(ws + p.off_acc);
     a.k_scale = d.k_scale;

@@ -394,13 +394,77 @@ def wide_range_queries(q: torch.Tensor, seed: int) -> torch.Tensor:
     return out.to(torch.bfloat16)
 
 
+def _stored_kv(ref, cfg):
+    """The K and V values the oracle attended, per compacted sequence: float64
+    [len, Hkv, d] arrays gathered through the compacted block table."""
+    s = ref["compact"]
+    bs, Hkv, d = cfg.block_size, cfg.hkv, cfg.head_dim
+    if cfg.fp8:
+        dec = lambda c: torch.from_numpy(c).view(torch.float8_e4m3fn).double().numpy()
+        k, v = dec(ref["k8"]), dec(ref["v8"])
+    elif cfg.int8:
+        k = ref["kq"].astype(np.float64) * np.repeat(ref["ks"].astype(np.float64), d)
+        v = ref["vq"].astype(np.float64) * np.repeat(ref["vs"].astype(np.float64), d)
+    else:
+        tobf = lambda c: torch.from_numpy(c.view(np.int16)).view(torch.bfloat16).double().numpy()
+        k, v = tobf(ref["kc"]), tobf(ref["vc"])
+    k = k.reshape(-1, bs, Hkv, d)
+    v = v.reshape(-1, bs, Hkv, d)
+    out = []
+    for b, n in enumerate(ref["ctx_lens"]):
+        blocks = s["block_tables"][b, :(int(n) + bs - 1) // bs]
+        out.append((k[blocks].reshape(-1, Hkv, d)[:n], v[blocks].reshape(-1, Hkv, d)[:n]))
+    return out
+
+
+def fp32_logit_slack(q, kv, G, scale):
+    """Per (sequence, query head): the output error that the logits' fp32 resolution
+    alone allows.  A logit of magnitude |s| is held to about 2^-24 |s|, and the
+    tensor-core accumulation of a k-step aligns its products to the largest, so a
+    row whose logits are huge (a query element of 7e4, or every element 1e5) carries
+    a few ulps of that magnitude: Delta = 2^-22 max_t |scale s_t|.  Weights move by
+    a factor within e^(+-Delta), so the output moves by at most 2 Delta max_t |v_t|.
+    For N(0,1) rows this is below 1e-5; the fp64 oracle has no such limit."""
+    B, Hq, d = q.shape
+    slack = np.zeros((B, Hq, 1))
+    for b in range(B):
+        k, v = kv[b]
+        if len(k) == 0:
+            continue
+        for i in range(Hq):
+            s = k[:, i // G, :] @ q[b, i].astype(np.float64)
+            slack[b, i, 0] = 2.0 * 2.0 ** -22 * np.abs(s * scale).max() * np.abs(v[:, i // G]).max()
+    return slack
+
+
 @pytest.mark.parametrize("key", ["c5m", "i8g16", "i8d64", "f8", "f8g16", "f8d64", "c3m", "c2m"])
 def test_wide_range_queries(key):
     """INT8 (three-part int8 query on the staged kernel), FP8 (power-of-two prescaled fp16
     query), bf16 and the general kernels against the fp64 oracle on queries whose
-    magnitudes span the bf16 range; no device flag is raised."""
+    magnitudes span the bf16 range; no device flag is raised.  The tolerance adds, per
+    row, what the logits' fp32 resolution allows (fp32_logit_slack; negligible except
+    for rows whose logits run into the tens of thousands)."""
     cfg = W.scaled(MEDIUM[key], score=False)
     wl = W.generate(cfg, "cpu")
     wl.q.copy_(wide_range_queries(wl.q, 396 + len(key)))
     assert wl.q.float().abs().max() > 65504
-    _parity(wl, list(range(wl.q.shape[0])))
+    layers = list(range(wl.q.shape[0]))
+    refs = [oracle_step(wl, l, range(cfg.batch)) for l in layers]
+    dev = Device(wl)
+    if cfg.int8 or cfg.fp8:
+        for l in layers:
+            dev.fill_int8_history(l)
+    for l, ref in zip(layers, refs):
+        dev.step(l)
+        torch.cuda.synchronize()
+        assert dev.err.item() == 0, f"device error flag {dev.err.item()}"
+        got = dev.out[l].float().cpu().numpy().astype(np.float64)
+        assert np.isfinite(got).all()
+        q = wl.q[l].double().numpy()
+        slack = fp32_logit_slack(q, _stored_kv(ref, cfg), cfg.hq // cfg.hkv, wl.scale)
+        err = np.abs(got - ref["out"])
+        bound = 2e-3 + 1e-2 * np.abs(ref["out"]) + slack
+        bad = err > bound
+        assert not bad.any(), (f"{key} layer {l}: {bad.sum()} outside; worst excess "
+                               f"{(err - bound).max():.3g}; slack range {slack.min():.2g}.."
+                               f"{slack.max():.2g}")

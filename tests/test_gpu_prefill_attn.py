@@ -209,3 +209,22 @@ def test_full_size_chunk_sampled_rows(balanced):
             ref = oracle.paged_decode(W.bits(qrow), kb, vb, stride, c["bt"][b:b + 1],
                                       np.array([p + 1], np.int32), Hkv, bs, d ** -0.5)
             assert_attention_close(out[c["cu"][b] + int(i)].unsqueeze(0), ref, f"seq {b} row {i}")
+
+
+
+def test_dominant_tokens_keep_the_tolerance():
+    """Rows whose softmax puts almost all weight on two or three tokens with values of
+    opposite sign (the case where one rounding of the weights shows most): keys equal
+    to a multiple of the query make those tokens dominate."""
+    c = _case([900, 400], [128, 64], 32, 8, 128, 16, seed=52)
+    k = c["k"].float()
+    q = c["q"].float()
+    bt = c["bt"]
+    for b, (toks, base) in enumerate((([3, 500, 777], 0), ([10, 399], 128))):
+        for n, t in enumerate(toks):
+            blk, off = bt[b, t // 16], t % 16
+            # head 0's query rows of this sequence all see these keys strongly
+            k[blk, off, 0] = q[c["cu"][b], 0] * (1.2 + 0.05 * n)
+    c["k"] = k.to(torch.bfloat16)
+    out = _run(c)
+    assert_attention_close(out, _oracle(c), "few dominant tokens")
