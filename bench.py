@@ -74,7 +74,8 @@ def parse():
     ap.add_argument("--secondary", default=None,
                     help="comma-separated workloads also measured and reported under "
                          "'secondary' in the same JSON line (c5-fp8 = c5 on e4m3 pools); "
-                         f"default for the c3 line: {'c4,c2,c5,c5-fp8,p1,p2'}, else none")
+                         f"default for the c3 line: {'c4,c2,c5,c5-fp8,p1,p2'}, else none; "
+                         "'none' for no secondary lines")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every call from Python instead of replaying a CUDA graph")
     return ap.parse_args()
@@ -329,6 +330,30 @@ class Runner:
         if self.cfg.score:
             per_layer += 1 if self.incremental else 2
         return per_layer * self.L + (1 if self.per_step_plan else 0)
+
+    def decode_calls(self):
+        """The step's decode calls alone, back to back: the partition plan (once per
+        step) and one decode call per layer, with no other kernel or event between
+        them (an event recorded between two kernels of a graph stops the second from
+        starting while the first drains)."""
+        pk, cfg = self.pk, self.cfg
+        if self.per_step_plan:
+            pk.pa_decode_prepare(self.q[0], self.wl.k_pool[0] if self.wl.k_pool is not None
+                                 else self.kq[0] if cfg.int8 else self.k8[0], self.bt, self.ctx,
+                                 self.err, self.ws, self.num_splits)
+        for l in range(self.L):
+            if cfg.fp8:
+                (pk.pa_decode_fp8_planned if self.per_step_plan else pk.pa_decode_fp8)(
+                    self.out[l], self.q[l], self.k8[l], self.v8[l], self.bt, self.ctx,
+                    self.wl.scale, self.err, self.ws, self.num_splits)
+            elif cfg.int8:
+                (pk.pa_decode_int8_planned if self.per_step_plan else pk.pa_decode_int8)(
+                    self.out[l], self.q[l], self.kq[l], self.vq[l], self.ks[l], self.vs[l],
+                    self.bt, self.ctx, self.wl.scale, self.err, self.ws, self.num_splits)
+            else:
+                (pk.pa_decode_planned if self.per_step_plan else pk.pa_decode)(
+                    self.out[l], self.q[l], self.wl.k_pool[l], self.wl.v_pool[l], self.bt,
+                    self.ctx, self.wl.scale, self.err, self.ws, self.num_splits)
 
     def step(self, ev=None):
         pk, cfg = self.pk, self.cfg
@@ -925,10 +950,6 @@ def run_chunked(args, device, world, rank, cpu_baseline=True):
 
 
 # ----------------------------------------------------------------------------- decode
-# distinct captured graphs kept for per-call statistics (older ones are replayed again)
-MAX_GRAPHS = 64
-
-
 def call_stats(call_ms, layers, batch, world):
     """Median duration (ms) of the decode call over every sample, and the decode-only
     throughput it implies: a step decodes `batch` tokens per rank through `layers`
@@ -945,9 +966,10 @@ def chunk_plan(steps, per_graph):
 
 
 def run_decode(args, cfg, device, world, rank, cpu_baseline=True):
-    """One decode workload: warm-up, K timed steps (CUDA graphs of the step with an
-    event pair around every decode call), the end-to-end pass and, optionally, the
-    oracle's CPU baseline.  Returns the JSON line as a dict (printed by rank 0)."""
+    """One decode workload: warm-up, K timed steps (CUDA graphs of the step), the
+    decode calls' own time and their time inside the step, the end-to-end pass and,
+    optionally, the oracle's CPU baseline.  Returns the JSON line as a dict (printed
+    by rank 0)."""
     r = Runner(cfg, device, args.num_splits, evict=args.evict, plan=args.plan)
     stream = torch.cuda.current_stream(device)
     for _ in range(max(3, args.warmup)):
@@ -960,35 +982,26 @@ def run_decode(args, cfg, device, world, rank, cpu_baseline=True):
     # steps per captured graph: at least 20 decode calls per replay
     R = max(1, -(-20 // r.L))
 
-    def capture(steps):
-        ev = [[torch.cuda.Event(enable_timing=True, external=True),
-               torch.cuda.Event(enable_timing=True, external=True)] for _ in range(r.L * steps)]
+    def capture(steps, with_events=False):
+        ev = ([[torch.cuda.Event(enable_timing=True, external=True),
+                torch.cuda.Event(enable_timing=True, external=True)]
+               for _ in range(r.L * steps)] if with_events else None)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for k in range(steps):
-                r.step(ev[k * r.L:(k + 1) * r.L])
+                r.step(ev[k * r.L:(k + 1) * r.L] if ev else None)
         return g, ev
 
     plan = chunk_plan(args.steps, R)
     if use_graph:
-        # full-size graphs: up to MAX_GRAPHS distinct ones (each keeps its own events),
-        # replayed in turn; the remainder graph is its own
-        n_full = sum(1 for n in plan if n == R)
-        full_graphs = [capture(R) for _ in range(min(n_full, MAX_GRAPHS))]
-        rest_graph = capture(plan[-1]) if plan and plan[-1] != R else None
-        order, j = [], 0
-        for n in plan:
-            if n == R:
-                order.append(full_graphs[j % len(full_graphs)])
-                j += 1
-            else:
-                order.append(rest_graph)
-        for g, _ in full_graphs + ([rest_graph] if rest_graph else []):
+        # the timed steps carry no events (an event between two kernels of a graph
+        # keeps the second from starting while the first drains)
+        full_graph = capture(R)[0] if any(n == R for n in plan) else None
+        rest_graph = capture(plan[-1])[0] if plan and plan[-1] != R else None
+        order = [full_graph if n == R else rest_graph for n in plan]
+        for g in {id(g): g for g in order}.values():
             g.replay()
         torch.cuda.synchronize(device)
-    else:
-        ev_eager = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-                    for _ in range(r.L * args.steps)]
 
     # --- device-timed region: exactly K steps
     if world > 1:
@@ -1000,24 +1013,55 @@ def run_decode(args, cfg, device, world, rank, cpu_baseline=True):
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     if use_graph:
-        for g, _ in order:
+        for g in order:
             g.replay()
     else:
         for k in range(args.steps):
-            r.step(ev_eager[k * r.L:(k + 1) * r.L])
+            r.step()
     t_end.record(stream)
     torch.cuda.synchronize(device)
     clk = clocks.stop()
     total_ms = reduce_max(t_start.elapsed_time(t_end), world)
-    if use_graph:
-        used = {id(g): ev for g, ev in order}      # every distinct graph that ran
-        samples = [pair for ev in used.values() for pair in ev]
-    else:
-        samples = ev_eager
-    call_ms = [a.elapsed_time(b) for a, b in samples]
     ms_per_step = total_ms / args.steps
     value = job_tokens_per_s(world, cfg.batch, ms_per_step)
-    med_ms, decode_only = call_stats(call_ms, r.L, cfg.batch, world)
+
+    # --- each decode call inside the step: the step with an event pair around every
+    # call, >= 20 calls (after the timed region, so its events do not slow it)
+    n_ev = max(1, -(-max(20, args.steps) // r.L))
+    if use_graph:
+        ge, evs = capture(n_ev, with_events=True)
+        ge.replay()
+    else:
+        evs = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+               for _ in range(r.L * n_ev)]
+        for k in range(n_ev):
+            r.step(evs[k * r.L:(k + 1) * r.L])
+    torch.cuda.synchronize(device)
+    call_ms = [a.elapsed_time(b) for a, b in evs]
+    med_in_step_ms, _ = call_stats(call_ms, r.L, cfg.batch, world)
+
+    # --- the decode calls' own time: the step's decode calls back to back (plan once,
+    # then one call per layer) in a graph, >= 20 replays, an event pair per replay
+    reps = max(20, args.steps)
+    if use_graph:
+        gd = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gd):
+            r.decode_calls()
+        gd.replay()
+    torch.cuda.synchronize(device)
+    evd = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+           for _ in range(reps)]
+    for e0_, e1_ in evd:
+        e0_.record(stream)
+        if use_graph:
+            gd.replay()
+        else:
+            r.decode_calls()
+        e1_.record(stream)
+    torch.cuda.synchronize(device)
+    per_call_ms = [a.elapsed_time(b) / r.L for a, b in evd]
+    med_ms = reduce_max(statistics.median(per_call_ms), world)
+    _, decode_only = call_stats([med_ms], r.L, cfg.batch, world)
     achieved = r.decode_bytes / (med_ms / 1000.0) / 1e9
     peak, peak_kind = peaks()
 
@@ -1097,7 +1141,13 @@ def run_decode(args, cfg, device, world, rank, cpu_baseline=True):
                      "algorithmic_bytes_per_launch":
                          r.decode_bytes,
                      "avg_launch_us": med_ms * 1000.0, "launch_time_statistic":
-                         f"median of {len(call_ms)} decode calls in the timed region"},
+                         f"median over {reps} replays of the step's {r.L} decode calls back "
+                         f"to back (plan included), per call",
+                     "avg_launch_us_in_step": med_in_step_ms * 1000.0,
+                     "in_step_statistic": f"median of {len(call_ms)} decode calls inside "
+                         "steps replayed after the timed region, an event pair around each "
+                         "(the events keep each call from overlapping its neighbours' "
+                         "launch)"},
         "decode_only_tokens_per_s": decode_only,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -1158,7 +1208,7 @@ def main():
     if spec is None:
         spec = SECONDARY_DEFAULT if (args.workload == "c3" and args.kv is None and
                                      not args.layers) else ""
-    extra = [w for w in spec.split(",") if w]
+    extra = [w for w in spec.split(",") if w and w != "none"]
     if extra:
         line["secondary"] = [run_one(secondary_args(args, w), device, world, rank,
                                      cpu_baseline=False) for w in extra]

@@ -327,7 +327,8 @@ DecodePlan make_decode_plan(int B, int Hq, int Hkv, int d, int bs, int MB, int n
         p.off_ns = 256;
         p.off_units = p.off_ns + up256((size_t)B * 4);
         p.off_cta = p.off_units + up256(n_units * 16);
-        p.off_starts = p.off_cta + up256((size_t)(p.grid + 1) * 4);
+        p.off_first = p.off_cta + up256((size_t)(p.grid + 1) * 4);
+        p.off_starts = p.off_first + up256((size_t)p.grid * 16);
         p.off_ml = p.off_starts + up256(p.balanced ? (size_t)B * 8 : 0);
         p.off_acc = p.off_ml + up256(slots * 2 * 4);
         p.ws_total = p.off_acc + up256(slots * d * 4);

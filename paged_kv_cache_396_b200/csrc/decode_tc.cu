@@ -91,6 +91,7 @@ struct Args {
     float scale_log2;
     unsigned long long sig;  // signature of the sizes; must match the plan's (header)
     const int32_t *cta_off;  // balanced plan: CTA i takes units cta_off[i] .. cta_off[i+1]-1
+    const int4 *cta_first;   // balanced plan: a copy of CTA i's first unit
     int balanced;
 };
 
@@ -277,8 +278,8 @@ constexpr int kMaxRanges = 1024;
 
 __global__ void __launch_bounds__(1024) plan_balanced_kernel(
     const int32_t *ctx_lens, int32_t *err, TcHeader *hdr, int32_t *ns, int4 *units,
-    int32_t *cta_off, long long *starts, int B, int max_ctx, int min_chunk, int P,
-    unsigned long long sig) {
+    int32_t *cta_off, int4 *cta_first, long long *starts, int B, int max_ctx, int min_chunk,
+    int P, unsigned long long sig) {
     __shared__ long long s_R[kMaxRanges + 1];   // snapped cut positions R_0 .. R_nr
     __shared__ int s_cnt[kMaxRanges];          // pieces per range, then fill positions
     __shared__ long long s_range, s_T;
@@ -294,16 +295,32 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
         }
         return len;
     };
-    // ---- sequence starts (exclusive prefix sums of the lengths)
-    long long run = 0;
+    // ---- sequence starts (exclusive prefix sums of the lengths); a thread keeps its
+    // first sequence's (b = tid) length and start in registers, later ones are read
+    // back from the workspace
+    long long run = 0, st0 = 0;
+    int len0 = 0;
     for (int b0 = 0; b0 < B; b0 += 1024) {
         const int b = b0 + tid;
         const int len = b < B ? clamp_len(b, true) : 0;
         long long tot;
         const long long st = run + cta_scan64(len, &tot);
         if (b < B) starts[b] = st;
+        if (b0 == 0) {
+            len0 = len;
+            st0 = st;
+        }
         run += tot;
     }
+    auto seq = [&](int b, int &len, long long &st) {
+        if (b == tid) {
+            len = len0;
+            st = st0;
+        } else {
+            len = clamp_len(b, false);
+            st = starts[b];
+        }
+    };
     if (tid == 0) {
         const long long T = run;
         long long r = (T + P - 1) / P;
@@ -322,8 +339,9 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
     // ---- cuts inside a sequence snap to its 16-token tiles (a sequence's thread
     // writes the cuts that fall strictly inside it); partitions per sequence
     for (int b = tid; b < B; b += 1024) {
-        const int len = clamp_len(b, false);
-        const long long st = starts[b];
+        int len;
+        long long st;
+        seq(b, len, st);
         int n = len > 0 ? 1 : 0;
         if (len > 0) {
             for (long long i = st / range + 1; i * range < st + len && i < nr; ++i) {
@@ -348,9 +366,10 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
         return lo;
     };
     for (int b = tid; b < B; b += 1024) {
-        const int len = clamp_len(b, false);
+        int len;
+        long long st;
+        seq(b, len, st);
         if (len == 0) continue;
-        const long long st = starts[b];
         int i = owner_of(st);
         atomicAdd(&s_cnt[i], 1);
         for (++i; i < nr && s_R[i] < st + len; ++i)
@@ -375,9 +394,10 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
     __syncthreads();
     // ---- the pieces: sequence b's cuts in order give partitions c = 0, 1, ...
     for (int b = tid; b < B; b += 1024) {
-        const int len = clamp_len(b, false);
+        int len;
+        long long st;
+        seq(b, len, st);
         if (len == 0) continue;
-        const long long st = starts[b];
         int i = owner_of(st);
         int c = 0;
         long long t0 = st;
@@ -393,6 +413,8 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
             ++c;
         }
     }
+    __syncthreads();   // the unit list is complete (and visible to the whole CTA)
+    if (tid < nr) cta_first[tid] = units[cta_off[tid]];
 }
 
 // ---------------------------------------------------------------------------
@@ -417,6 +439,9 @@ __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensor
     // taken from the counter
     const int u_first = plan_ok && a.balanced ? a.cta_off[blockIdx.x] : 0;
     const int n_units = !plan_ok ? 0 : a.balanced ? a.cta_off[blockIdx.x + 1] : a.hdr->n_units;
+    // the first unit's copy is read in the same round as the offsets (one dependent
+    // load less before the first block-table lookup)
+    const int4 un_first = a.balanced ? a.cta_first[blockIdx.x] : make_int4(0, 0, 0, 0);
     int u_next = u_first;
     if (!plan_ok && lane == 0 && blockIdx.x == 0) raise_flag(a.err, PA_DEV_BAD_PLAN);
     const uint64_t policy = ptx::policy_evict_first();
@@ -436,7 +461,7 @@ __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensor
             u = __shfl_sync(kFull, u, 0);
         }
         if ((int)u >= n_units) break;
-        const int4 un = a.units[u];
+        const int4 un = (a.balanced && (int)u == u_first) ? un_first : a.units[u];
         const int b = un.x, c = un.y, t0 = un.z, t1 = un.w;
         const bool direct = (a.wph == 1) && (a.ns[b] == 1);
         const int nst = t1 > t0 ? (t1 - t0 + T_s - 1) / T_s : 1;
@@ -1670,6 +1695,67 @@ __global__ void __launch_bounds__(D) merge_tc_kernel(const Args a) {
     a.out[bh * D + e] = f32_to_bf16_rn(L > 0.f ? A / L : 0.f);
 }
 
+// Merge with one warp per output row (b, i), 8 rows per CTA: lane j takes the
+// (m, l) of partial c0 + j of each 32-partial chunk, the row maximum and the
+// weights f = 2^(m - M) come from warp shuffles, and each lane accumulates its
+// D/32 dims of sum_s f_s acc_s in slot order (the loads of eight partials in
+// flight at once).  Used when every row has few partials (short contexts), where
+// one small CTA per row spends most of its time starting and waiting.
+constexpr int kRowsPerMergeCta = 8;
+
+template <int D>
+__global__ void __launch_bounds__(32 * kRowsPerMergeCta) merge_rows_kernel(const Args a) {
+    constexpr int E = D / 32;
+    ptx::grid_dependency_wait();  // the decode kernel's partials are complete
+    if (a.hdr->sig != a.sig) return;  // no plan for these sizes (flagged by the decode)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t bh = (int64_t)blockIdx.x * kRowsPerMergeCta + warp;
+    if (bh >= (int64_t)a.B * a.Hq) return;
+    const int b = (int)(bh / a.Hq), i = (int)(bh % a.Hq);
+    const int nsb = a.ns[b];
+    if (nsb == 1 && a.wph == 1) return;  // written directly by the decode kernel
+    const int cnt = nsb * a.wph;
+    const int64_t base = (int64_t)b * a.S * a.wph;
+    float M = -INFINITY;
+    for (int s = lane; s < cnt; s += 32) M = fmaxf(M, a.ws_ml[((base + s) * a.Hq + i) * 2]);
+    M = warp_max(M);
+    float L = 0.f, A[E];
+#pragma unroll
+    for (int k = 0; k < E; ++k) A[k] = 0.f;
+    if (M != -INFINITY) {
+        for (int c0 = 0; c0 < cnt; c0 += 32) {
+            float f = 0.f;
+            if (c0 + lane < cnt) {
+                const float2 ml = *reinterpret_cast<const float2 *>(
+                    a.ws_ml + ((base + c0 + lane) * a.Hq + i) * 2);
+                f = exp2f(ml.x - M);
+                L = fmaf(ml.y, f, L);
+            }
+            const int n = min(32, cnt - c0);
+#pragma unroll 8
+            for (int j = 0; j < n; ++j) {
+                const float fj = __shfl_sync(kFull, f, j);
+                const float *src = a.ws_acc + ((base + c0 + j) * a.Hq + i) * D + lane * E;
+                if constexpr (E == 4) {
+                    const float4 v = *reinterpret_cast<const float4 *>(src);
+                    A[0] = fmaf(v.x, fj, A[0]);
+                    A[1] = fmaf(v.y, fj, A[1]);
+                    A[2] = fmaf(v.z, fj, A[2]);
+                    A[3] = fmaf(v.w, fj, A[3]);
+                } else {
+                    const float2 v = *reinterpret_cast<const float2 *>(src);
+                    A[0] = fmaf(v.x, fj, A[0]);
+                    A[1] = fmaf(v.y, fj, A[1]);
+                }
+            }
+        }
+        L = warp_sum(L);
+    }
+    uint16_t *o = a.out + bh * D + lane * E;
+#pragma unroll
+    for (int k = 0; k < E; ++k) o[k] = f32_to_bf16_rn(L > 0.f ? A[k] / L : 0.f);
+}
+
 // ---------------------------------------------------------------------------
 // host
 // ---------------------------------------------------------------------------
@@ -1769,6 +1855,7 @@ cudaError_t launch_plan(const DecodeArgs &d, cudaStream_t st) {
                           reinterpret_cast<int32_t *>(ws + p.off_ns),
                           reinterpret_cast<int4 *>(ws + p.off_units),
                           reinterpret_cast<int32_t *>(ws + p.off_cta),
+                          reinterpret_cast<int4 *>(ws + p.off_first),
                           reinterpret_cast<long long *>(ws + p.off_starts), d.B, d.MB * d.bs,
                           p.chunk, p.grid, p.sig);
     return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, d.ctx_lens, d.err,
@@ -1802,6 +1889,7 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, int kv, cudaStream_t st) {
     a.ns = reinterpret_cast<const int32_t *>(ws + p.off_ns);
     a.units = reinterpret_cast<const int4 *>(ws + p.off_units);
     a.cta_off = reinterpret_cast<const int32_t *>(ws + p.off_cta);
+    a.cta_first = reinterpret_cast<const int4 *>(ws + p.off_first);
     a.balanced = p.balanced;
     a.ws_ml = reinterpret_cast<float *>(ws + p.off_ml);
     a.ws_acc = reinterpret_cast<float *>(ws + p.off_acc);
@@ -1851,8 +1939,21 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, int kv, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     if (p.S > 1 || p.wph > 1) {
         const unsigned rows = (unsigned)((int64_t)d.B * d.Hq);
-        e = d.d == 128 ? launch_pdl(merge_tc_kernel<128>, dim3(rows), dim3(128), 0, st, a)
-                       : launch_pdl(merge_tc_kernel<64>, dim3(rows), dim3(64), 0, st, a);
+        // few partials per row (at most (B + P) / B on average with the balanced split,
+        // S * wph with an explicit one): a warp per row; many (long contexts of a small
+        // batch): a CTA per row, whose warps split the partials
+        const int64_t few = 8;
+        const bool rows_kernel = p.balanced ? (int64_t)d.B + p.grid <= few * d.B
+                                            : (int64_t)p.S * p.wph <= few;
+        if (rows_kernel) {
+            const unsigned ctas = (rows + kRowsPerMergeCta - 1) / kRowsPerMergeCta;
+            const dim3 blk(32 * kRowsPerMergeCta);
+            e = d.d == 128 ? launch_pdl(merge_rows_kernel<128>, dim3(ctas), blk, 0, st, a)
+                           : launch_pdl(merge_rows_kernel<64>, dim3(ctas), blk, 0, st, a);
+        } else {
+            e = d.d == 128 ? launch_pdl(merge_tc_kernel<128>, dim3(rows), dim3(128), 0, st, a)
+                           : launch_pdl(merge_tc_kernel<64>, dim3(rows), dim3(64), 0, st, a);
+        }
     }
     return e;
 }

@@ -44,7 +44,7 @@ struct DecodePlan {
     int n_sub;          // staged: 16-token sub-tiles per stage (wph * tpw)
     int nstage, stage_bytes, v_off, ks_off, vs_off, smem_bytes, grid, units_per_cta;
     int balanced;       // staged: 1 = every CTA takes an equal token range (automatic split)
-    size_t off_hdr, off_ns, off_units, off_cta, off_starts, off_ml, off_acc, ws_total;
+    size_t off_hdr, off_ns, off_units, off_cta, off_first, off_starts, off_ml, off_acc, ws_total;
     unsigned long long sig;  // staged: signature of the sizes the device plan is made for
 };
 

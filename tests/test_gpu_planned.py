@@ -24,6 +24,10 @@ CASES = {
     "int8": W.scaled(C["c5"], key="pl8", layers=2, batch=5, old_lens=(300, 1, 16, 255, 512)),
     "fp8": W.scaled(C["c5"], key="plf8", layers=2, int8=False, fp8=True, batch=5,
                     old_lens=(300, 1, 16, 255, 512)),
+    # full-batch shapes: c2's 32 sequences of 1024 tokens (5-6 pieces each) and 64 INT8
+    # sequences of 512 (2-3 pieces each)
+    "bf16-c2": W.scaled(C["c2"], key="plfu", layers=2, score=False),
+    "int8-b64": W.scaled(C["c5"], key="plfu8", layers=2, batch=64, old_lens=(512,) * 64),
     # general-shape kernel (INT8 with d = 64): no device plan, the planned call is the plain one
     "int8-d64": W.scaled(C["c5"], key="pl8d64", layers=2, batch=3, head_dim=64,
                          old_lens=(70, 5, 200)),
