@@ -432,16 +432,20 @@ __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensor
     const uint32_t sc_bytes = (uint32_t)kTile * a.Hkv * 4;  // one sub-tile's scale rows
     const uint32_t sub_bytes = 2u * DC * (uint32_t)a.box_bytes + (I8 ? 2u * sc_bytes : 0u);
     const int tpb = a.bs / kTile;                            // 16-token tiles per block
+    // The header, this CTA's unit offsets and its first unit's copy are independent
+    // loads issued together, one round trip before the first block-table lookup (the
+    // offset and copy regions exist in every plan layout; an explicit plan ignores them).
+    const unsigned long long hsig = a.hdr->sig;
+    const int h_units = a.hdr->n_units;
+    const int off0 = a.cta_off[blockIdx.x], off1 = a.cta_off[blockIdx.x + 1];
+    const int4 un_first = a.cta_first[blockIdx.x];
     // a plan made for other sizes (a kept plan that does not match this call) is
     // not used: no unit is taken and the call flags it
-    const bool plan_ok = a.hdr->sig == a.sig;
+    const bool plan_ok = hsig == a.sig;
     // balanced plan: this CTA's own list of units; otherwise all units, longest first,
     // taken from the counter
-    const int u_first = plan_ok && a.balanced ? a.cta_off[blockIdx.x] : 0;
-    const int n_units = !plan_ok ? 0 : a.balanced ? a.cta_off[blockIdx.x + 1] : a.hdr->n_units;
-    // the first unit's copy is read in the same round as the offsets (one dependent
-    // load less before the first block-table lookup)
-    const int4 un_first = a.balanced ? a.cta_first[blockIdx.x] : make_int4(0, 0, 0, 0);
+    const int u_first = plan_ok && a.balanced ? off0 : 0;
+    const int n_units = !plan_ok ? 0 : a.balanced ? off1 : h_units;
     int u_next = u_first;
     if (!plan_ok && lane == 0 && blockIdx.x == 0) raise_flag(a.err, PA_DEV_BAD_PLAN);
     const uint64_t policy = ptx::policy_evict_first();
@@ -1698,26 +1702,49 @@ __global__ void __launch_bounds__(D) merge_tc_kernel(const Args a) {
 // Merge with one warp per output row (b, i), 8 rows per CTA: lane j takes the
 // (m, l) of partial c0 + j of each 32-partial chunk, the row maximum and the
 // weights f = 2^(m - M) come from warp shuffles, and each lane accumulates its
-// D/32 dims of sum_s f_s acc_s in slot order (the loads of eight partials in
-// flight at once).  Used when every row has few partials (short contexts), where
-// one small CTA per row spends most of its time starting and waiting.
+// D/32 dims of sum_s f_s acc_s in slot order.  Used when every row has few
+// partials (short contexts), where one small CTA per row spends most of its time
+// starting and waiting.  The plan's signature, the piece count, the first 32
+// (m, l) pairs and the first kAhead partials' accumulators do not depend on one
+// another: they are loaded in one round (slots past the sequence's count are read
+// but never used; every slot of the sequence's S * wph exists), so a row with at
+// most kAhead partials waits for one round trip instead of four.
 constexpr int kRowsPerMergeCta = 8;
+constexpr int kAhead = 8;
 
 template <int D>
 __global__ void __launch_bounds__(32 * kRowsPerMergeCta) merge_rows_kernel(const Args a) {
     constexpr int E = D / 32;
     ptx::grid_dependency_wait();  // the decode kernel's partials are complete
-    if (a.hdr->sig != a.sig) return;  // no plan for these sizes (flagged by the decode)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t bh = (int64_t)blockIdx.x * kRowsPerMergeCta + warp;
     if (bh >= (int64_t)a.B * a.Hq) return;
     const int b = (int)(bh / a.Hq), i = (int)(bh % a.Hq);
+    const int cap = a.S * a.wph;               // partial slots of one sequence
+    const int64_t base = (int64_t)b * cap;
+    const unsigned long long hsig = a.hdr->sig;
     const int nsb = a.ns[b];
+    float2 ml0 = make_float2(-INFINITY, 0.f);
+    if (lane < cap) ml0 = *reinterpret_cast<const float2 *>(a.ws_ml + ((base + lane) * a.Hq + i) * 2);
+    float va[kAhead][E];
+#pragma unroll
+    for (int j = 0; j < kAhead; ++j) {
+        if (j < cap) {
+            const float *src = a.ws_acc + ((base + j) * a.Hq + i) * D + lane * E;
+            if constexpr (E == 4) {
+                const float4 v = *reinterpret_cast<const float4 *>(src);
+                va[j][0] = v.x, va[j][1] = v.y, va[j][2] = v.z, va[j][3] = v.w;
+            } else {
+                const float2 v = *reinterpret_cast<const float2 *>(src);
+                va[j][0] = v.x, va[j][1] = v.y;
+            }
+        }
+    }
+    if (hsig != a.sig) return;  // no plan for these sizes (flagged by the decode)
     if (nsb == 1 && a.wph == 1) return;  // written directly by the decode kernel
     const int cnt = nsb * a.wph;
-    const int64_t base = (int64_t)b * a.S * a.wph;
-    float M = -INFINITY;
-    for (int s = lane; s < cnt; s += 32) M = fmaxf(M, a.ws_ml[((base + s) * a.Hq + i) * 2]);
+    float M = lane < cnt ? ml0.x : -INFINITY;
+    for (int s = lane + 32; s < cnt; s += 32) M = fmaxf(M, a.ws_ml[((base + s) * a.Hq + i) * 2]);
     M = warp_max(M);
     float L = 0.f, A[E];
 #pragma unroll
@@ -1726,14 +1753,27 @@ __global__ void __launch_bounds__(32 * kRowsPerMergeCta) merge_rows_kernel(const
         for (int c0 = 0; c0 < cnt; c0 += 32) {
             float f = 0.f;
             if (c0 + lane < cnt) {
-                const float2 ml = *reinterpret_cast<const float2 *>(
-                    a.ws_ml + ((base + c0 + lane) * a.Hq + i) * 2);
+                const float2 ml = c0 == 0 ? ml0
+                                          : *reinterpret_cast<const float2 *>(
+                                                a.ws_ml + ((base + c0 + lane) * a.Hq + i) * 2);
                 f = exp2f(ml.x - M);
                 L = fmaf(ml.y, f, L);
             }
             const int n = min(32, cnt - c0);
+            int j = 0;
+            if (c0 == 0) {   // the partials loaded ahead
+#pragma unroll
+                for (int k = 0; k < kAhead; ++k) {
+                    if (k < n) {
+                        const float fj = __shfl_sync(kFull, f, k);
+#pragma unroll
+                        for (int e = 0; e < E; ++e) A[e] = fmaf(va[k][e], fj, A[e]);
+                    }
+                }
+                j = kAhead;
+            }
 #pragma unroll 8
-            for (int j = 0; j < n; ++j) {
+            for (; j < n; ++j) {
                 const float fj = __shfl_sync(kFull, f, j);
                 const float *src = a.ws_acc + ((base + c0 + j) * a.Hq + i) * D + lane * E;
                 if constexpr (E == 4) {
