@@ -452,10 +452,6 @@ __device__ __forceinline__ void producer(const CUtensorMap *kmap, const CUtensor
     int stage = 0;
     uint32_t phase = 0;
     bool ok = plan_ok;
-    if (lane == 0) {
-        ptx::prefetch_tensormap(kmap);
-        ptx::prefetch_tensormap(vmap);
-    }
     while (ok) {
         unsigned u = 0;
         if (a.balanced) {
@@ -1595,6 +1591,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::fence_mbar_init();
     }
+    if (threadIdx.x == kConsumerWarps * 32) {   // the tensor maps are launch parameters
+        ptx::prefetch_tensormap(&kmap);
+        ptx::prefetch_tensormap(&vmap);
+    }
     __syncthreads();
     // launched programmatically after the plan kernel: the set-up above overlaps
     // it; the plan (and, through it, the KV append before it) is complete here
@@ -1672,6 +1672,8 @@ __device__ __forceinline__ void merge_wide(const Args &a, int64_t bh, int i, int
 
 template <int D>
 __global__ void __launch_bounds__(D) merge_tc_kernel(const Args a) {
+    // the next kernel may start its set-up now; its own wait still covers this one
+    ptx::grid_launch_dependents();
     ptx::grid_dependency_wait();  // the decode kernel's partials are complete
     if (a.hdr->sig != a.sig) return;  // no plan for these sizes (flagged by the decode)
     const int64_t bh = blockIdx.x;
@@ -1715,6 +1717,8 @@ constexpr int kAhead = 8;
 template <int D>
 __global__ void __launch_bounds__(32 * kRowsPerMergeCta) merge_rows_kernel(const Args a) {
     constexpr int E = D / 32;
+    // the next kernel may start its set-up now; its own wait still covers this one
+    ptx::grid_launch_dependents();
     ptx::grid_dependency_wait();  // the decode kernel's partials are complete
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t bh = (int64_t)blockIdx.x * kRowsPerMergeCta + warp;
