@@ -69,6 +69,10 @@ def parse():
     ap.add_argument("--plan", default="step", choices=["step", "call"],
                     help="staged decode: make the partition plan once per step "
                          "(pa_decode_prepare + planned calls) or inside every decode call")
+    ap.add_argument("--select", default="call", choices=["call", "stream"],
+                    help="incremental eviction: the block selection inside the decode call "
+                         "(pa_decode*_select_pooled: extra CTAs of its merge launch) or as its "
+                         "own kernel on a second stream beside the decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--secondary", default=None,
@@ -225,7 +229,7 @@ class Runner:
     """Device state and one decode step of a workload through the binding."""
 
     def __init__(self, cfg, device, num_splits=0, wl=None, evict="full", plan="step",
-                 overlap_select=True):
+                 overlap_select=True, select="call"):
         from paged_kv_cache_396_b200 import pagedkv as pk
         self.pk, self.cfg, self.dev = pk, cfg, device
         wl = W.generate(cfg, device) if wl is None else wl
@@ -278,12 +282,16 @@ class Runner:
                                          self.vq[l], self.ks[l], self.vs[l], self.bt[b:b + 1],
                                          zeros[b:b + 1], self.err)
         self.incremental = bool(cfg.score) and evict == "incremental"
+        # incremental eviction on bf16 pools: the block choice inside the decode call
+        self.select_in_call = (self.incremental and select == "call" and not cfg.int8
+                               and not cfg.fp8)
         if cfg.score:
             self.scores = torch.zeros(B, MB * bs, Hkv, dtype=torch.float32, device=device)
             self.evict = torch.zeros(B, dtype=torch.int32, device=device)
         # incremental eviction: the block choice of a layer overlaps its decode (a second
         # stream joined at the end of the step) unless overlap is off
-        self.side = (torch.cuda.Stream(device) if self.incremental and overlap_select
+        self.side = (torch.cuda.Stream(device)
+                     if self.incremental and overlap_select and not self.select_in_call
                      else None)
         self.ev_app = [torch.cuda.Event() for _ in range(self.L)]
         self.ev_join = torch.cuda.Event()
@@ -324,11 +332,24 @@ class Runner:
         self.decode_bytes = decode_algorithmic_bytes(cfg, self.wl.ctx_lens, slots, n_units)
         self.partitions = slots
 
+    def selection_rides_on_merge(self):
+        """Whether the decode call's merge launch carries the block selection: the
+        staged kernel with a warp-per-row merge (the library's rule: with the balanced
+        split B + SMs <= 8 B, with an explicit one S * wph <= 8)."""
+        cfg = self.cfg
+        if not (self.select_in_call and self.staged and self.dec_launches >= 3):
+            return False
+        P = torch.cuda.get_device_properties(self.dev).multi_processor_count
+        wph = max(1, 8 // cfg.hkv)
+        if self.num_splits == 0 and P < 1024:
+            return cfg.batch + P <= 8 * cfg.batch
+        return self.S * wph <= 8
+
     def launches_per_step(self):
         dec = self.dec_launches - (1 if self.per_step_plan else 0)
         per_layer = (1 if self.cfg.append else 0) + dec
         if self.cfg.score:
-            per_layer += 1 if self.incremental else 2
+            per_layer += (0 if self.selection_rides_on_merge() else 1) if self.incremental else 2
         return per_layer * self.L + (1 if self.per_step_plan else 0)
 
     def decode_calls(self):
@@ -396,13 +417,21 @@ class Runner:
                                     self.err)
                 if ev is not None:
                     ev[l][0].record()
-                dec(self.out[l], self.q[l], kp, vp, self.bt, self.ctx, self.wl.scale, self.err,
-                    self.ws, self.num_splits)
+                if self.select_in_call:   # decode and this layer's block choice, one call
+                    (pk.pa_decode_planned_select_pooled if self.per_step_plan
+                     else pk.pa_decode_select_pooled)(
+                        self.out[l], self.q[l], kp, vp, self.bt, self.ctx, self.wl.scale,
+                        self.err, self.evict, self.score_pool[l], None, self.ws,
+                        self.num_splits)
+                else:
+                    dec(self.out[l], self.q[l], kp, vp, self.bt, self.ctx, self.wl.scale,
+                        self.err, self.ws, self.num_splits)
             if ev is not None:
                 ev[l][1].record()
             if self.incremental:
-                pk.pe_select_evict_block_pooled(self.evict, self.score_pool[l], self.bt, self.ctx,
-                                                self.err, stream=self.side)
+                if not self.select_in_call:
+                    pk.pe_select_evict_block_pooled(self.evict, self.score_pool[l], self.bt,
+                                                    self.ctx, self.err, stream=self.side)
             elif cfg.score:
                 pk.pe_score_tokens(self.scores, self.wl.k_pool[l], self.wl.v_pool[l], self.bt,
                                    self.ctx, self.err)
@@ -970,7 +999,8 @@ def run_decode(args, cfg, device, world, rank, cpu_baseline=True):
     decode calls' own time and their time inside the step, the end-to-end pass and,
     optionally, the oracle's CPU baseline.  Returns the JSON line as a dict (printed
     by rank 0)."""
-    r = Runner(cfg, device, args.num_splits, evict=args.evict, plan=args.plan)
+    r = Runner(cfg, device, args.num_splits, evict=args.evict, plan=args.plan,
+               select=args.select)
     stream = torch.cuda.current_stream(device)
     for _ in range(max(3, args.warmup)):
         r.step()
@@ -1131,6 +1161,9 @@ def run_decode(args, cfg, device, world, rank, cpu_baseline=True):
                                      "full pass per layer") if cfg.score else None,
                    "partitions": r.partitions, "chunk_tokens": r.chunk_used,
                    "partition_plan": "once per step" if r.per_step_plan else "every call",
+                   "block_selection": (("inside the decode call" if r.select_in_call else
+                                        "own kernel, second stream" if r.side is not None else
+                                        "own kernel") if r.incremental else None),
                    "cuda_graph": use_graph, "steps_per_graph": R if use_graph else None},
         "roofline": {"bound": "hbm", "kernel": {"bf16": "pa_decode", "int8": "pa_decode_int8",
                                                "fp8_e4m3": "pa_decode_fp8"}[kv_name(cfg)],

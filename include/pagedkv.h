@@ -372,6 +372,44 @@ int pe_select_evict_block_pooled(int32_t *evict, float *block_means, const float
                                  int64_t num_blocks, int32_t *err_flag, void *stream);
 
 /* ============================================================================
+ * Decode and pooled block selection in one call ([KVL] "PagedEviction 块级驱逐
+ * 机制": in the decode phase the block to evict is chosen from the scores of
+ * complete blocks; the choice does not depend on the attention output)
+ *
+ * pa_decode_select_pooled is pa_decode followed by pe_select_evict_block_pooled
+ * on the same block_tables, ctx_lens, B, max_blocks_per_seq, Hkv, bs and
+ * num_blocks; pa_decode_planned_select_pooled is the same with pa_decode_planned
+ * (same plan rules).  out is what the decode call gives and evict / block_means
+ * what the selection call gives, bit for bit.  The selection runs in B extra CTAs
+ * at the front of the decode's merge launch, beside the decode kernel, so a decode
+ * layer with incremental eviction is the scored append plus the decode's launches
+ * (plan, decode, merge; no plan for the planned call).  Where the decode has no
+ * merge launch (a single partition, or the general-shape kernel), or merges with
+ * one CTA per row, the selection kernel is launched after it instead.  The score
+ * pool, tables and lengths are only read; the selection's results do not depend
+ * on the plan (a refused plan still gets them).  Only the bf16 decode has this form.
+ * Host errors: those of either call; a NULL evict or score_pool -> PA_ERR_NULL
+ * (block_means may be NULL).
+ * ==========================================================================*/
+int pa_decode_select_pooled(uint16_t *out, const uint16_t *q,
+                            const uint16_t *k_cache, const uint16_t *v_cache,
+                            int64_t block_stride, const int32_t *block_tables,
+                            int max_blocks_per_seq, const int32_t *ctx_lens, int B, int Hq,
+                            int Hkv, int d, int bs, int64_t num_blocks, float scale,
+                            int num_splits, void *workspace, size_t workspace_bytes,
+                            int32_t *evict, float *block_means, const float *score_pool,
+                            int32_t *err_flag, void *stream);
+
+int pa_decode_planned_select_pooled(uint16_t *out, const uint16_t *q,
+                                    const uint16_t *k_cache, const uint16_t *v_cache,
+                                    int64_t block_stride, const int32_t *block_tables,
+                                    int max_blocks_per_seq, const int32_t *ctx_lens, int B,
+                                    int Hq, int Hkv, int d, int bs, int64_t num_blocks,
+                                    float scale, int num_splits, void *workspace,
+                                    size_t workspace_bytes, int32_t *evict, float *block_means,
+                                    const float *score_pool, int32_t *err_flag, void *stream);
+
+/* ============================================================================
  * pa_decode without a caller-provided workspace (no counterpart in the pages;
  * it exists for callers, not for the method).
  *

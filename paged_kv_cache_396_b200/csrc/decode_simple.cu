@@ -247,8 +247,12 @@ cudaError_t launch_merge(const DecodeArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, int kv, cudaStream_t st) {
-    if (a.plan.kernel == 1) return launch_decode_tc(a, kv, st);
-    return launch_decode_simple(a, kv, st);
+    if (a.plan.kernel == 1) return launch_decode_tc(a, kv, st);   // selection included
+    cudaError_t e = launch_decode_simple(a, kv, st);
+    if (e == cudaSuccess && a.sel_evict)
+        e = launch_select_pooled(a.sel_evict, a.sel_means, a.sel_scores, a.block_tables,
+                                 a.ctx_lens, a.err, a.B, a.MB, a.Hkv, a.bs, a.N, st);
+    return e;
 }
 
 namespace {

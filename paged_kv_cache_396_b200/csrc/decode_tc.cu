@@ -50,6 +50,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
+#include "select_pooled.cuh"
 
 namespace pkv {
 namespace tc {
@@ -93,6 +94,11 @@ struct Args {
     const int32_t *cta_off;  // balanced plan: CTA i takes units cta_off[i] .. cta_off[i+1]-1
     const int4 *cta_first;   // balanced plan: a copy of CTA i's first unit
     int balanced;
+    // the merge launch's first sel_ctas CTAs (0 or B) run the pooled block selection
+    int sel_ctas;
+    int32_t *sel_evict;
+    float *sel_means;
+    const float *sel_scores;
 };
 
 // ---------------------------------------------------------------------------
@@ -1597,9 +1603,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     // launched programmatically after the plan kernel: the set-up above overlaps
-    // it; the plan (and, through it, the KV append before it) is complete here
-    ptx::grid_launch_dependents();
+    // it; the plan (and, through it, the KV append before it) is complete here.
+    // The merge launch is released only after this wait, so the selection CTAs at
+    // its front may read the score pool the append wrote without waiting themselves.
     ptx::grid_dependency_wait();
+    ptx::grid_launch_dependents();
     if ((threadIdx.x >> 5) == kConsumerWarps)
         producer<D, KV>(&kmap, &vmap, a, stages, meta, full, empty);
     else if constexpr (KV == kKvInt8)
@@ -1714,14 +1722,24 @@ __global__ void __launch_bounds__(D) merge_tc_kernel(const Args a) {
 constexpr int kRowsPerMergeCta = 8;
 constexpr int kAhead = 8;
 
+static_assert(32 * kRowsPerMergeCta == kSelThreads, "selection CTAs share the merge's block");
+
 template <int D>
 __global__ void __launch_bounds__(32 * kRowsPerMergeCta) merge_rows_kernel(const Args a) {
     constexpr int E = D / 32;
     // the next kernel may start its set-up now; its own wait still covers this one
     ptx::grid_launch_dependents();
+    if ((int)blockIdx.x < a.sel_ctas) {
+        // the block selection of sequence blockIdx.x: it reads the score pool and the
+        // tables only, written before the decode kernel's dependency wait released
+        // this launch, so it runs beside the decode kernel
+        select_pooled_cta(a.sel_evict, a.sel_means, a.sel_scores, a.bt, a.ctx_lens, a.err, a.MB,
+                          a.Hkv, a.bs, a.N, (int)blockIdx.x);
+        return;
+    }
     ptx::grid_dependency_wait();  // the decode kernel's partials are complete
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t bh = (int64_t)blockIdx.x * kRowsPerMergeCta + warp;
+    const int64_t bh = (int64_t)(blockIdx.x - a.sel_ctas) * kRowsPerMergeCta + warp;
     if (bh >= (int64_t)a.B * a.Hq) return;
     const int b = (int)(bh / a.Hq), i = (int)(bh % a.Hq);
     const int cap = a.S * a.wph;               // partial slots of one sequence
@@ -1962,6 +1980,10 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, int kv, cudaStream_t st) {
     }
     a.scale_log2 = d.scale_log2;
     a.sig = p.sig;
+    a.sel_ctas = 0;   // the merge launch below adds the selection CTAs when asked
+    a.sel_evict = nullptr;
+    a.sel_means = nullptr;
+    a.sel_scores = nullptr;
     cudaError_t e = cudaSuccess;
     if (!d.reuse_plan) {
         e = launch_plan(d, st);
@@ -1981,6 +2003,7 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, int kv, cudaStream_t st) {
         e = g16 ? launch_typed<64, true, kKvBf16>(km, vm, a, p.grid, p.smem_bytes, st)
                 : launch_typed<64, false, kKvBf16>(km, vm, a, p.grid, p.smem_bytes, st);
     if (e != cudaSuccess) return e;
+    bool sel_done = d.sel_evict == nullptr;
     if (p.S > 1 || p.wph > 1) {
         const unsigned rows = (unsigned)((int64_t)d.B * d.Hq);
         // few partials per row (at most (B + P) / B on average with the balanced split,
@@ -1990,15 +2013,28 @@ cudaError_t launch_decode_tc(const DecodeArgs &d, int kv, cudaStream_t st) {
         const bool rows_kernel = p.balanced ? (int64_t)d.B + p.grid <= few * d.B
                                             : (int64_t)p.S * p.wph <= few;
         if (rows_kernel) {
-            const unsigned ctas = (rows + kRowsPerMergeCta - 1) / kRowsPerMergeCta;
+            // the selection, when asked for, takes B CTAs at the front of this launch
+            Args am = a;
+            if (!sel_done) {
+                am.sel_ctas = d.B;
+                am.sel_evict = d.sel_evict;
+                am.sel_means = d.sel_means;
+                am.sel_scores = d.sel_scores;
+                sel_done = true;
+            }
+            const unsigned ctas =
+                (rows + kRowsPerMergeCta - 1) / kRowsPerMergeCta + (unsigned)am.sel_ctas;
             const dim3 blk(32 * kRowsPerMergeCta);
-            e = d.d == 128 ? launch_pdl(merge_rows_kernel<128>, dim3(ctas), blk, 0, st, a)
-                           : launch_pdl(merge_rows_kernel<64>, dim3(ctas), blk, 0, st, a);
+            e = d.d == 128 ? launch_pdl(merge_rows_kernel<128>, dim3(ctas), blk, 0, st, am)
+                           : launch_pdl(merge_rows_kernel<64>, dim3(ctas), blk, 0, st, am);
         } else {
             e = d.d == 128 ? launch_pdl(merge_tc_kernel<128>, dim3(rows), dim3(128), 0, st, a)
                            : launch_pdl(merge_tc_kernel<64>, dim3(rows), dim3(64), 0, st, a);
         }
     }
+    if (e == cudaSuccess && !sel_done)   // no merge launch to carry it: its own kernel
+        e = launch_select_pooled(d.sel_evict, d.sel_means, d.sel_scores, d.block_tables,
+                                 d.ctx_lens, d.err, d.B, d.MB, d.Hkv, d.bs, d.N, st);
     return e;
 }
 

@@ -70,6 +70,10 @@ struct DecodeArgs {
     void *ws;                     // workspace base
     DecodePlan plan;
     int reuse_plan;               // staged: the workspace already holds the plan (no plan launch)
+    // optional, in the same call: the pooled block selection (pe_select_evict_block_pooled)
+    int32_t *sel_evict;           // [B], or nullptr: no selection
+    float *sel_means;             // [B][MB] block means, or nullptr
+    const float *sel_scores;      // score pool [N][bs][Hkv] fp32
 };
 
 struct ScoreArgs {

@@ -58,7 +58,8 @@ int decode_entry(uint16_t *out, const uint16_t *q, const void *kc, const void *v
                  const float *vs, int kv, int64_t block_stride, const int32_t *bt, int MB,
                  const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs, int64_t N,
                  float scale, int num_splits, void *ws, size_t ws_bytes, int32_t *err,
-                 void *stream, int reuse_plan = 0) {
+                 void *stream, int reuse_plan = 0, int32_t *sel_evict = nullptr,
+                 float *sel_means = nullptr, const float *sel_scores = nullptr) {
     if (B == 0) return PA_OK;  // empty batch: nothing to read or write
     if (!out || !q || !kc || !vc || !bt || !ctx_lens || !err) return PA_ERR_NULL;
     if (kv == pkv::kKvInt8 && (!ks || !vs)) return PA_ERR_NULL;
@@ -109,6 +110,9 @@ int decode_entry(uint16_t *out, const uint16_t *q, const void *kc, const void *v
     a.num_splits = plan.S;
     a.chunk = plan.chunk;
     a.reuse_plan = reuse_plan;
+    a.sel_evict = sel_evict;
+    a.sel_means = sel_means;
+    a.sel_scores = sel_scores;
     return finish(pkv::launch_decode(a, kv, static_cast<cudaStream_t>(stream)));
 }
 
@@ -383,6 +387,35 @@ int pa_decode_planned(uint16_t *out, const uint16_t *q, const uint16_t *k_cache,
     return decode_entry(out, q, k_cache, v_cache, nullptr, nullptr, pkv::kKvBf16, block_stride,
                         block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
                         scale, num_splits, workspace, workspace_bytes, err_flag, stream, 1);
+}
+
+int pa_decode_select_pooled(uint16_t *out, const uint16_t *q, const uint16_t *k_cache,
+                            const uint16_t *v_cache, int64_t block_stride,
+                            const int32_t *block_tables, int max_blocks_per_seq,
+                            const int32_t *ctx_lens, int B, int Hq, int Hkv, int d, int bs,
+                            int64_t num_blocks, float scale, int num_splits, void *workspace,
+                            size_t workspace_bytes, int32_t *evict, float *block_means,
+                            const float *score_pool, int32_t *err_flag, void *stream) {
+    if (B > 0 && (!evict || !score_pool)) return PA_ERR_NULL;
+    return decode_entry(out, q, k_cache, v_cache, nullptr, nullptr, pkv::kKvBf16, block_stride,
+                        block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
+                        scale, num_splits, workspace, workspace_bytes, err_flag, stream, 0, evict,
+                        block_means, score_pool);
+}
+
+int pa_decode_planned_select_pooled(uint16_t *out, const uint16_t *q, const uint16_t *k_cache,
+                                    const uint16_t *v_cache, int64_t block_stride,
+                                    const int32_t *block_tables, int max_blocks_per_seq,
+                                    const int32_t *ctx_lens, int B, int Hq, int Hkv, int d,
+                                    int bs, int64_t num_blocks, float scale, int num_splits,
+                                    void *workspace, size_t workspace_bytes, int32_t *evict,
+                                    float *block_means, const float *score_pool,
+                                    int32_t *err_flag, void *stream) {
+    if (B > 0 && (!evict || !score_pool)) return PA_ERR_NULL;
+    return decode_entry(out, q, k_cache, v_cache, nullptr, nullptr, pkv::kKvBf16, block_stride,
+                        block_tables, max_blocks_per_seq, ctx_lens, B, Hq, Hkv, d, bs, num_blocks,
+                        scale, num_splits, workspace, workspace_bytes, err_flag, stream, 1, evict,
+                        block_means, score_pool);
 }
 
 int pa_decode_int8_planned(uint16_t *out, const uint16_t *q, const int8_t *kq_cache,

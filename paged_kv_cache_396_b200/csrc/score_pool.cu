@@ -14,6 +14,7 @@
 #include "blockmean.cuh"
 #include "common.cuh"
 #include "kernels.h"
+#include "select_pooled.cuh"
 
 namespace pkv {
 
@@ -97,59 +98,14 @@ __global__ void __launch_bounds__(256) append_scored_kernel(const uint16_t *__re
     }
 }
 
-// Block selection from the score pool.  One CTA of 256 threads per sequence; each
-// warp takes four consecutive full logical blocks at a time (j = 4 w .. 4 w + 3,
-// then 32 further) with their loads in flight together; block j's bs*Hkv scores are
-// the contiguous scores of physical block bt[b][j] (token-major, then head),
-// reduced with the arithmetic of the selection over a [B][MB*bs][Hkv] score array,
-// so both agree exactly on equal scores.  256 threads keep the CTA small enough to
-// run beside the decode kernel when the caller overlaps the two on two streams.
-constexpr int kSelThreads = 256;
-
+// Block selection from the score pool: one CTA of kSelThreads threads per sequence
+// (select_pooled.cuh).  256 threads keep the CTA small enough to run beside the
+// decode kernel when the caller overlaps the two on two streams.
 __global__ void __launch_bounds__(kSelThreads) select_pooled_kernel(
     int32_t *evict, float *means, const float *score_pool, const int32_t *block_tables,
     const int32_t *ctx_lens, int32_t *err, int MB, int Hkv, int bs, int64_t N) {
-    const int b = blockIdx.x;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    int len = ctx_lens[b];
-    if (len < 0 || (int64_t)len > (int64_t)MB * bs) {
-        if (threadIdx.x == 0) raise_flag(err, PA_DEV_BAD_LEN);
-        len = 0;
-    }
-    const int nfull = len / bs;
-    const int per = bs * Hkv;
-    double best = INFINITY;
-    int bj = INT_MAX;
-    for (int j0 = 4 * warp; j0 < MB; j0 += 4 * nw) {
-        const float *p[4] = {nullptr, nullptr, nullptr, nullptr};
-        bool cand[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int j = j0 + i;
-            cand[i] = j < nfull;
-            if (cand[i]) {
-                const int32_t phys = block_tables[(int64_t)b * MB + j];
-                if (phys < 0 || (int64_t)phys >= N) {
-                    if (lane == 0) raise_flag(err, PA_DEV_BAD_BLOCK);
-                    cand[i] = false;
-                } else {
-                    p[i] = score_pool + (int64_t)phys * per;
-                }
-            }
-        }
-        double mean[4] = {0.0, 0.0, 0.0, 0.0};
-        if (cand[0] || cand[1] || cand[2] || cand[3])   // warp-uniform
-            warp_block_mean4(p, per, lane, mean);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int j = j0 + i;
-            if (cand[i]) argmin_take(best, bj, mean[i], j);
-            if (means && lane == 0 && j < MB)
-                means[(int64_t)b * MB + j] = cand[i] ? (float)mean[i] : __int_as_float(0x7fc00000);
-        }
-    }
-    const int win = cta_argmin(best, bj);
-    if (threadIdx.x == 0) evict[b] = (nfull > 0 && win != INT_MAX) ? win : -1;
+    select_pooled_cta(evict, means, score_pool, block_tables, ctx_lens, err, MB, Hkv, bs, N,
+                      blockIdx.x);
 }
 
 cudaError_t launch_append_scored(const uint16_t *k_new, const uint16_t *v_new, uint16_t *k_cache,

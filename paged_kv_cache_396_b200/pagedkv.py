@@ -36,7 +36,8 @@ EXPORTED = (
     "pa_decode",
     "pe_score_tokens", "pe_select_evict_block", "pa_append_kv_int8", "pa_decode_int8",
     "pa_decode_static_scratch", "pa_decode_prepare", "pa_decode_planned",
-    "pa_decode_int8_planned", "pa_decode_fp8_planned", "pa_append_kv_scored",
+    "pa_decode_int8_planned", "pa_decode_fp8_planned", "pa_decode_select_pooled",
+    "pa_decode_planned_select_pooled", "pa_append_kv_scored",
     "pa_append_kv_int8_scored",
     "pe_select_evict_block_pooled", "pa_append_kv_fp8", "pa_decode_fp8",
     "pe_prefill_scores", "pe_prefill_select", "pe_prefill_pack", "pe_prefill_compress",
@@ -88,6 +89,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pa_decode_prepare.argtypes = [p, i32, i32, i32, i32, i32, i32, i32, p, sz, p, p]
     lib.pa_decode_planned.restype = i32
     lib.pa_decode_planned.argtypes = lib.pa_decode.argtypes
+    # pa_decode's arguments with (evict, block_means, score_pool) before err_flag
+    sel_args = lib.pa_decode.argtypes[:-2] + [p, p, p] + lib.pa_decode.argtypes[-2:]
+    lib.pa_decode_select_pooled.restype = i32
+    lib.pa_decode_select_pooled.argtypes = sel_args
+    lib.pa_decode_planned_select_pooled.restype = i32
+    lib.pa_decode_planned_select_pooled.argtypes = sel_args
     lib.pa_decode_int8_planned.restype = i32
     lib.pa_decode_int8_planned.argtypes = lib.pa_decode_int8.argtypes
     lib.pa_decode_static_scratch.restype = i32
@@ -372,6 +379,63 @@ def _decode_bf16(fn, out, q, k_cache, v_cache, block_tables, ctx_lens, scale, er
                              float(scale), int(num_splits), ws_ptr, ws_n, _ptr(err_flag),
                              _stream(stream))
     _check(fn, rc)
+
+
+def _select_checks(evict, score_pool, block_tables, block_means):
+    _want(evict, torch.int32, "evict")
+    _want(score_pool, torch.float32, "score_pool")
+    if score_pool.dim() != 3 or not score_pool.is_contiguous():
+        raise ValueError("score_pool must be contiguous [N, bs, Hkv]")
+    B, MB = block_tables.shape
+    if block_means is not None:
+        _want(block_means, torch.float32, "block_means")
+        if tuple(block_means.shape) != (B, MB) or not block_means.is_contiguous():
+            raise ValueError("block_means must be contiguous [B, MB]")
+    _covers(evict, B, "evict")
+
+
+def _decode_select(fn, out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
+                   evict, score_pool, block_means, workspace, num_splits, stream):
+    _decode_checks(out, q, block_tables, ctx_lens, err_flag)
+    _want(k_cache, torch.bfloat16, "k_cache")
+    _want(v_cache, torch.bfloat16, "v_cache")
+    N, bs, Hkv, d, stride = _pool_geometry(k_cache, "k_cache")
+    _same_pool(k_cache, v_cache)
+    _select_checks(evict, score_pool, block_tables, block_means)
+    if tuple(score_pool.shape) != (N, bs, Hkv):
+        raise ValueError("score_pool must be [N, bs, Hkv] of the KV pool")
+    B, Hq, dq = q.shape
+    if dq != d:
+        raise ValueError("q head_dim differs from the pool's")
+    _one_device(k_cache, out, q, v_cache, block_tables, ctx_lens, err_flag, workspace, evict,
+                score_pool, block_means)
+    bt = block_tables.contiguous()
+    ws_ptr, ws_n = (None, 0) if workspace is None else (_ptr(workspace), workspace.numel() *
+                                                        workspace.element_size())
+    rc = getattr(load(), fn)(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), stride, _ptr(bt),
+                             bt.shape[1], _ptr(ctx_lens.contiguous()), B, Hq, Hkv, d, bs, N,
+                             float(scale), int(num_splits), ws_ptr, ws_n, _ptr(evict),
+                             _ptr(block_means), _ptr(score_pool), _ptr(err_flag), _stream(stream))
+    _check(fn, rc)
+
+
+def pa_decode_select_pooled(out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,
+                            evict, score_pool, block_means=None, workspace=None, num_splits=0,
+                            stream=None):
+    """pa_decode and pe_select_evict_block_pooled in one call: the selection runs in
+    extra CTAs of the decode's merge launch, beside the decode kernel."""
+    _decode_select("pa_decode_select_pooled", out, q, k_cache, v_cache, block_tables, ctx_lens,
+                   scale, err_flag, evict, score_pool, block_means, workspace, num_splits, stream)
+
+
+def pa_decode_planned_select_pooled(out, q, k_cache, v_cache, block_tables, ctx_lens, scale,
+                                    err_flag, evict, score_pool, block_means=None, workspace=None,
+                                    num_splits=0, stream=None):
+    """pa_decode_select_pooled with the partition plan pa_decode_prepare left in the
+    workspace."""
+    _decode_select("pa_decode_planned_select_pooled", out, q, k_cache, v_cache, block_tables,
+                   ctx_lens, scale, err_flag, evict, score_pool, block_means, workspace,
+                   num_splits, stream)
 
 
 def pa_decode_static_scratch(out, q, k_cache, v_cache, block_tables, ctx_lens, scale, err_flag,

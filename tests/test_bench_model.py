@@ -63,3 +63,51 @@ def test_timed_region_runs_exactly_the_requested_steps():
         plan = bench.chunk_plan(steps, per)
         assert sum(plan) == steps
         assert all(n == per for n in plan[:-1]) and 0 < plan[-1] <= per
+
+
+class _Recorder:
+    """Stand-in for the binding: records the name of every call a step makes."""
+
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        def call(*args, **kw):
+            self.calls.append(name)
+        return call
+
+
+def _runner(key, evict, select, per_step_plan=True):
+    """A bench.Runner with its device state replaced by placeholders (no GPU)."""
+    cfg = dataclasses.replace(W.CONFIGS[key], layers=2)
+    r = object.__new__(bench.Runner)
+    r.pk, r.cfg, r.L = _Recorder(), cfg, cfg.layers
+    r.per_step_plan = per_step_plan
+    r.incremental = bool(cfg.score) and evict == "incremental"
+    r.select_in_call = r.incremental and select == "call"
+    r.side = None
+    r.ev_app = [None] * cfg.layers
+    x = [None] * cfg.layers
+
+    class _Wl:
+        k_pool, v_pool, scale = x, x, 0.125
+    r.wl = _Wl()
+    r.q = r.k_new = r.v_new = r.out = r.score_pool = x
+    r.bt = r.ctx = r.pos = r.err = r.ws = r.evict = r.scores = None
+    r.num_splits = 0
+    return r
+
+
+@pytest.mark.parametrize("evict,select,per_layer", [
+    ("incremental", "call", ["pa_append_kv_scored", "pa_decode_planned_select_pooled"]),
+    ("incremental", "stream", ["pa_append_kv_scored", "pa_decode_planned",
+                               "pe_select_evict_block_pooled"]),
+    ("full", "call", ["pa_append_kv", "pa_decode_planned", "pe_score_tokens",
+                      "pe_select_evict_block"]),
+])
+def test_c2_step_makes_each_layers_calls_once(evict, select, per_layer):
+    """The c2 step: one plan, then per layer exactly the calls of its eviction mode (a
+    selection inside the decode call must not bring back the full score pass)."""
+    r = _runner("c2", evict, select)
+    r.step()
+    assert r.pk.calls == ["pa_decode_prepare"] + per_layer * r.L

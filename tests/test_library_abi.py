@@ -106,7 +106,8 @@ S = 16 * 8 * 128   # dense block stride of a [bs=16][Hkv=8][d=128] block
 def _dec(fn, lib, *, kv="bf16", **kw):
     """pa_decode_int8 / pa_decode_fp8 / pa_decode_static_scratch with one argument changed."""
     a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, ks=FAKE, vs=FAKE, stride=S, bt=FAKE, MB=4,
-             ctx=FAKE, B=2, Hq=32, Hkv=8, d=128, bs=16, N=10, scale=0.1, S=0, err=FAKE)
+             ctx=FAKE, B=2, Hq=32, Hkv=8, d=128, bs=16, N=10, scale=0.1, S=0, err=FAKE,
+             ev=FAKE, sp=FAKE)
     a.update(kw)
     common = (a["stride"], a["bt"], a["MB"], a["ctx"], a["B"], a["Hq"], a["Hkv"], a["d"], a["bs"],
               a["N"], a["scale"], a["S"])
@@ -122,6 +123,10 @@ def _dec(fn, lib, *, kv="bf16", **kw):
     if fn == "int8_planned":
         return lib.pa_decode_int8_planned(a["out"], a["q"], a["k"], a["v"], a["ks"], a["vs"],
                                           *common, None, 0, a["err"], None)
+    if fn in ("select", "planned_select"):
+        f = lib.pa_decode_select_pooled if fn == "select" else lib.pa_decode_planned_select_pooled
+        return f(a["out"], a["q"], a["k"], a["v"], *common, None, 0, a["ev"], None, a["sp"],
+                 a["err"], None)
     if fn == "fp8_planned":
         return lib.pa_decode_fp8_planned(a["out"], a["q"], a["k"], a["v"], *common, None, 0,
                                          a["err"], None)
@@ -129,7 +134,8 @@ def _dec(fn, lib, *, kv="bf16", **kw):
 
 
 def test_decode_variants_reject_bad_arguments_on_host(lib):
-    for fn in ("int8", "fp8", "static", "planned", "int8_planned", "fp8_planned"):
+    for fn in ("int8", "fp8", "static", "planned", "int8_planned", "fp8_planned", "select",
+               "planned_select"):
         assert _dec(fn, lib, q=NUL) == -1, fn
         assert _dec(fn, lib, err=NUL) == -1, fn
         assert _dec(fn, lib, Hq=24, Hkv=16) == -2, fn      # Hq % Hkv != 0
@@ -149,6 +155,10 @@ def test_decode_variants_reject_bad_arguments_on_host(lib):
     assert _dec("static", lib, stride=S + 4) == -3         # bf16: 8 bytes
     assert _dec("int8_planned", lib, ks=NUL) == -1
     assert _dec("planned", lib, stride=S + 4) == -3
+    for fn in ("select", "planned_select"):          # the selection's own outputs and input
+        assert _dec(fn, lib, ev=NUL) == -1, fn
+        assert _dec(fn, lib, sp=NUL) == -1, fn
+        assert _dec(fn, lib, ev=NUL, B=0) == 0, fn
 
 
 def test_decode_prepare_rejects_bad_arguments_on_host(lib):
