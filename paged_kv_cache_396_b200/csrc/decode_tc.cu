@@ -281,6 +281,7 @@ __device__ __forceinline__ long long cta_scan64(long long v, long long *total) {
 // and the merge writes its zero row).
 // ---------------------------------------------------------------------------
 constexpr int kMaxRanges = 1024;
+constexpr int kSeqCache = 1024;   // sequences whose length and start stay in shared memory
 
 __global__ void __launch_bounds__(1024) plan_balanced_kernel(
     const int32_t *ctx_lens, int32_t *err, TcHeader *hdr, int32_t *ns, int4 *units,
@@ -288,9 +289,12 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
     int P, unsigned long long sig) {
     __shared__ long long s_R[kMaxRanges + 1];   // snapped cut positions R_0 .. R_nr
     __shared__ int s_cnt[kMaxRanges];          // pieces per range, then fill positions
+    __shared__ int s_off[kMaxRanges];          // first unit of each range
+    __shared__ int s_len[kSeqCache];           // lengths and starts of sequences < kSeqCache
+    __shared__ long long s_st[kSeqCache];
     __shared__ long long s_range, s_T;
     __shared__ int s_nr;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     ptx::grid_launch_dependents();
     ptx::grid_dependency_wait();
     auto clamp_len = [&](int b, bool flag) {
@@ -301,32 +305,21 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
         }
         return len;
     };
-    // ---- sequence starts (exclusive prefix sums of the lengths); a thread keeps its
-    // first sequence's (b = tid) length and start in registers, later ones are read
-    // back from the workspace
-    long long run = 0, st0 = 0;
-    int len0 = 0;
+    // ---- sequence starts (exclusive prefix sums of the lengths): kept in shared
+    // memory for the first kSeqCache sequences, in the workspace for all
+    long long run = 0;
     for (int b0 = 0; b0 < B; b0 += 1024) {
         const int b = b0 + tid;
         const int len = b < B ? clamp_len(b, true) : 0;
         long long tot;
         const long long st = run + cta_scan64(len, &tot);
         if (b < B) starts[b] = st;
-        if (b0 == 0) {
-            len0 = len;
-            st0 = st;
+        if (b < kSeqCache) {
+            s_len[b] = len;
+            s_st[b] = st;
         }
         run += tot;
     }
-    auto seq = [&](int b, int &len, long long &st) {
-        if (b == tid) {
-            len = len0;
-            st = st0;
-        } else {
-            len = clamp_len(b, false);
-            st = starts[b];
-        }
-    };
     if (tid == 0) {
         const long long T = run;
         long long r = (T + P - 1) / P;
@@ -336,32 +329,55 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
         s_T = T;
         s_nr = T > 0 ? (int)((T + r - 1) / r) : 0;
     }
-    __syncthreads();
+    __syncthreads();   // also publishes s_len / s_st and the workspace starts
     const long long range = s_range, T = s_T;
     const int nr = s_nr;
     for (int i = tid; i <= nr; i += 1024) s_R[i] = i < nr ? (long long)i * range : T;
     for (int i = tid; i < kMaxRanges; i += 1024) s_cnt[i] = 0;
     __syncthreads();
-    // ---- cuts inside a sequence snap to its 16-token tiles (a sequence's thread
-    // writes the cuts that fall strictly inside it); partitions per sequence
-    for (int b = tid; b < B; b += 1024) {
-        int len;
+    // The candidate cuts of a sequence, i0 <= i < i1: the range boundaries i * range
+    // strictly inside it.
+    auto seq = [&](int b, int &len, long long &st) {
+        if (b < kSeqCache) {
+            len = s_len[b];
+            st = s_st[b];
+        } else {
+            len = clamp_len(b, false);
+            st = starts[b];
+        }
+    };
+    auto cand = [&](int len, long long st, int &i0, int &i1) {
+        i0 = (int)(st / range) + 1;
+        const long long e = (st + len - 1) / range + 1;
+        i1 = (int)(e < nr ? e : nr);
+    };
+    // Few sequences (B < 32, where one can hold many cuts): a warp takes a sequence
+    // (b = warp, warp + 32, ...) and its lanes the candidate cuts.  Otherwise a thread
+    // takes a sequence and walks its (few) candidates.
+    const bool lanes = B < 32;
+    const int grp = lanes ? lane : 0, gw = lanes ? 32 : 1;      // lane in the group, width
+    const int g0 = lanes ? warp : tid, gstep = lanes ? 32 : 1024;  // first sequence, stride
+    // ---- cuts snap to the sequence's 16-token tiles; a cut snapped onto the
+    // sequence's end (or start) cuts nothing.  Partitions per sequence.
+    for (int b = g0; b < B; b += gstep) {
+        int len, i0, i1;
         long long st;
         seq(b, len, st);
-        int n = len > 0 ? 1 : 0;
+        int n = 0;
         if (len > 0) {
-            for (long long i = st / range + 1; i * range < st + len && i < nr; ++i) {
-                const long long o = i * range - st;          // 0 < o < len
+            cand(len, st, i0, i1);
+            for (int i = i0 + grp; i < i1; i += gw) {
+                const long long o = (long long)i * range - st;   // 0 < o < len
                 long long sn = (o + kTile / 2) / kTile * kTile;
                 if (sn >= len) sn = len;
                 s_R[i] = st + sn;
                 if (sn > 0 && sn < len) ++n;
             }
+            n = 1 + (lanes ? __reduce_add_sync(kFull, n) : n);
         }
-        ns[b] = n;
+        if (grp == 0) ns[b] = n;
     }
     __syncthreads();
-    // ---- owner range of every piece (the range its first token falls in): count
     auto owner_of = [&](long long x) {   // largest i < nr with R_i <= x
         int lo = 0, hi = nr - 1;
         while (lo < hi) {
@@ -371,15 +387,17 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
         }
         return lo;
     };
-    for (int b = tid; b < B; b += 1024) {
-        int len;
+    // ---- pieces per range: a sequence's first piece belongs to the range holding its
+    // start, every later piece to the range its cut begins
+    for (int b = g0; b < B; b += gstep) {
+        int len, i0, i1;
         long long st;
         seq(b, len, st);
         if (len == 0) continue;
-        int i = owner_of(st);
-        atomicAdd(&s_cnt[i], 1);
-        for (++i; i < nr && s_R[i] < st + len; ++i)
-            if (s_R[i] > st) atomicAdd(&s_cnt[i], 1);
+        if (grp == 0) atomicAdd(&s_cnt[owner_of(st)], 1);
+        cand(len, st, i0, i1);
+        for (int i = i0 + grp; i < i1; i += gw)
+            if (s_R[i] > st && s_R[i] < st + len) atomicAdd(&s_cnt[i], 1);
     }
     __syncthreads();
     // ---- per-range unit offsets (exclusive scan over the ranges; ranges >= nr empty)
@@ -388,7 +406,7 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
         const int c = tid < nr ? s_cnt[tid] : 0;
         const long long off = cta_scan64(c, &tot);
         if (tid <= P) cta_off[tid] = (int)(tid < nr ? off : tot);
-        if (tid < nr) s_cnt[tid] = (int)off;   // fill position of range tid
+        if (tid < nr) s_cnt[tid] = s_off[tid] = (int)off;   // fill position of range tid
         if (tid == 0) {
             hdr->n_units = (int)tot;
             hdr->chunk = (int)min(range, (long long)INT32_MAX);
@@ -398,29 +416,60 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
         }
     }
     __syncthreads();
-    // ---- the pieces: sequence b's cuts in order give partitions c = 0, 1, ...
-    for (int b = tid; b < B; b += 1024) {
-        int len;
+    // ---- the pieces: sequence b's valid cuts in order give partitions c = 1, 2, ...
+    // (a warp per sequence: lane order, a carry counting the valid cuts of earlier
+    // 32-candidate chunks); the unit placed first in a range is also copied to that
+    // CTA's cta_first
+    auto place = [&](int own, int4 u) {
+        const int pos = atomicAdd(&s_cnt[own], 1);
+        units[pos] = u;
+        if (pos == s_off[own]) cta_first[own] = u;
+    };
+    for (int b = g0; b < B && !lanes; b += gstep) {   // a thread per sequence
+        int len, i0, i1;
         long long st;
         seq(b, len, st);
         if (len == 0) continue;
-        int i = owner_of(st);
-        int c = 0;
+        cand(len, st, i0, i1);
+        const long long end = st + len;
+        int own = owner_of(st), c = 0;
         long long t0 = st;
-        for (;;) {
-            int j = i + 1;   // next cut strictly inside the sequence, if any
-            while (j < nr && s_R[j] <= t0) ++j;
-            const long long t1 = (j < nr && s_R[j] < st + len) ? s_R[j] : st + len;
-            const int pos = atomicAdd(&s_cnt[i], 1);
-            units[pos] = make_int4(b, c, (int)(t0 - st), (int)(t1 - st));
-            if (t1 >= st + len) break;
-            i = j;
+        for (int i = i0; i <= i1; ++i) {   // each valid cut ends a piece; the end, the last
+            const bool cut = i < i1 && s_R[i] > st && s_R[i] < end;
+            if (i < i1 && !cut) continue;
+            const long long t1 = cut ? s_R[i] : end;
+            place(own, make_int4(b, c, (int)(t0 - st), (int)(t1 - st)));
+            own = i;
             t0 = t1;
             ++c;
         }
     }
-    __syncthreads();   // the unit list is complete (and visible to the whole CTA)
-    if (tid < nr) cta_first[tid] = units[cta_off[tid]];
+    for (int b = warp; b < B && lanes; b += 32) {   // a warp per sequence
+        int len, i0, i1;
+        long long st;
+        seq(b, len, st);
+        if (len == 0) continue;
+        cand(len, st, i0, i1);
+        const long long end = st + len;
+        auto valid = [&](int i) { return s_R[i] > st && s_R[i] < end; };
+        int carry = 0;
+        long long first_cut = end;   // where piece 0 ends
+        for (int k0 = i0; k0 < i1; k0 += 32) {
+            const int i = k0 + lane;
+            const bool v = i < i1 && valid(i);
+            const unsigned m = __ballot_sync(kFull, v);
+            if (first_cut == end && m) first_cut = s_R[k0 + __ffs(m) - 1];
+            if (v) {
+                int j = i + 1;   // the next valid cut (only a sequence's last candidate
+                while (j < i1 && !valid(j)) ++j;   // can be invalid, so this is short)
+                const long long t1 = j < i1 ? s_R[j] : end;
+                const int c = 1 + carry + __popc(m & ((1u << lane) - 1u));
+                place(i, make_int4(b, c, (int)(s_R[i] - st), (int)(t1 - st)));
+            }
+            carry += __popc(m);
+        }
+        if (lane == 0) place(owner_of(st), make_int4(b, 0, 0, (int)(first_cut - st)));
+    }
 }
 
 // ---------------------------------------------------------------------------
