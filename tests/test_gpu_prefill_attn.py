@@ -3,8 +3,8 @@ C ABI against the fp64 oracle: |err| <= 2e-3 + 1e-2 |ref| on every output of
 medium cases (several 64-row query tiles, 64-token K/V tiles, ragged tails,
 GQA group sizes 1..16, d 64 and 128, block sizes 12, 16 and 256), the
 append-then-attend sequence, mixed chunk + decode batches, invalid lengths,
-and sampled rows of a full-size 512-token chunk at 8K context; each in the
-one-CTA-per-query-tile mode and in the balanced mode (workspace given: tile ranges
+sampled rows of a full-size 512-token chunk at 8K context, and 16 seeded random
+shapes; each in the one-CTA-per-query-tile mode and in the balanced mode (workspace given: tile ranges
 cut across SMs, partial results merged), which bench.py times."""
 import numpy as np
 import pytest
@@ -228,3 +228,34 @@ def test_dominant_tokens_keep_the_tolerance():
     c["k"] = k.to(torch.bfloat16)
     out = _run(c)
     assert_attention_close(out, _oracle(c), "few dominant tokens")
+
+
+def _random_case(i):
+    """Seeded random chunked-prefill shape: 1-6 sequences, chunks from 0 rows to the
+    whole context, lengths around tile and block boundaries, G 1-16, d 64 / 128,
+    block sizes 12, 16, 32 and 256."""
+    rng = np.random.default_rng(5000 + i)
+    Hkv = int(rng.choice([1, 2, 4, 8]))
+    G = int(rng.choice([1, 2, 4, 8, 16]))
+    d = int(rng.choice([64, 128, 128]))
+    bs = int(rng.choice([12, 16, 16, 32, 256]))
+    B = int(rng.integers(1, 7))
+    lens, qlens = [], []
+    for _ in range(B):
+        n = int(rng.choice([1, 63, 64, 65, 127, 128, 129, 255, 256, 257])) \
+            if rng.random() < 0.3 else int(rng.integers(1, 2500))
+        q = int(rng.choice([0, 1, n, min(n, 64), min(n, 129), min(n, 300)])) \
+            if rng.random() < 0.5 else int(rng.integers(0, min(n, 700) + 1))
+        lens.append(n)
+        qlens.append(q)
+    return lens, qlens, G * Hkv, Hkv, d, bs
+
+
+@pytest.mark.parametrize("balanced", [False, True])
+@pytest.mark.parametrize("i", range(16))
+def test_prefill_attention_random_shapes(i, balanced):
+    lens, qlens, Hq, Hkv, d, bs = _random_case(i)
+    c = _case(lens, qlens, Hq, Hkv, d, bs, seed=5000 + i)
+    out = _run(c, balanced=balanced)
+    assert_attention_close(out, _oracle(c), f"random case {i}: {lens} {qlens} G{Hq // Hkv} "
+                                            f"d{d} bs{bs}")
