@@ -4,8 +4,9 @@ medium cases (several 64-row query tiles, 64-token K/V tiles, ragged tails,
 GQA group sizes 1..16, d 64 and 128, block sizes 12, 16 and 256), the
 append-then-attend sequence, mixed chunk + decode batches, invalid lengths,
 sampled rows of a full-size 512-token chunk at 8K context, and 16 seeded random
-shapes; each in the one-CTA-per-query-tile mode and in the balanced mode (workspace given: tile ranges
-cut across SMs, partial results merged), which bench.py times."""
+shapes; each in the one-CTA-per-query-tile mode and in the balanced mode
+(workspace given: tile ranges cut across SMs, partial results merged), which
+bench.py times."""
 import numpy as np
 import pytest
 import torch
