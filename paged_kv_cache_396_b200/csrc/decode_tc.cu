@@ -287,14 +287,12 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
     const int32_t *ctx_lens, int32_t *err, TcHeader *hdr, int32_t *ns, int4 *units,
     int32_t *cta_off, int4 *cta_first, long long *starts, int B, int max_ctx, int min_chunk,
     int P, unsigned long long sig) {
-    __shared__ long long s_R[kMaxRanges + 1];   // snapped cut positions R_0 .. R_nr
     __shared__ int s_cnt[kMaxRanges];          // pieces per range, then fill positions
     __shared__ int s_off[kMaxRanges];          // first unit of each range
     __shared__ int s_len[kSeqCache];           // lengths and starts of sequences < kSeqCache
     __shared__ long long s_st[kSeqCache];
-    __shared__ long long s_range, s_T;
-    __shared__ int s_nr;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int i = tid; i < kMaxRanges; i += 1024) s_cnt[i] = 0;   // (read only after barriers)
     ptx::grid_launch_dependents();
     ptx::grid_dependency_wait();
     auto clamp_len = [&](int b, bool flag) {
@@ -320,23 +318,13 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
         }
         run += tot;
     }
-    if (tid == 0) {
-        const long long T = run;
-        long long r = (T + P - 1) / P;
-        r = (r + kTile - 1) / kTile * kTile;
-        if (r < min_chunk) r = min_chunk;
-        s_range = r;
-        s_T = T;
-        s_nr = T > 0 ? (int)((T + r - 1) / r) : 0;
-    }
-    __syncthreads();   // also publishes s_len / s_st and the workspace starts
-    const long long range = s_range, T = s_T;
-    const int nr = s_nr;
-    for (int i = tid; i <= nr; i += 1024) s_R[i] = i < nr ? (long long)i * range : T;
-    for (int i = tid; i < kMaxRanges; i += 1024) s_cnt[i] = 0;
-    __syncthreads();
-    // The candidate cuts of a sequence, i0 <= i < i1: the range boundaries i * range
-    // strictly inside it.
+    // every thread derives the range and the number of ranges from the total
+    const long long T = run;
+    long long range = (T + P - 1) / P;
+    range = (range + kTile - 1) / kTile * kTile;
+    if (range < min_chunk) range = min_chunk;
+    const int nr = T > 0 ? (int)((T + range - 1) / range) : 0;
+    __syncthreads();   // publishes s_len / s_st and the workspace starts
     auto seq = [&](int b, int &len, long long &st) {
         if (b < kSeqCache) {
             len = s_len[b];
@@ -346,10 +334,22 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
             st = starts[b];
         }
     };
+    // The candidate cuts of a sequence, i0 <= i < i1: the range boundaries i * range
+    // strictly inside it; cut i lands on the sequence's nearest 16-token tile boundary
+    // (at most its end).  A cut strictly inside the sequence starts a piece owned by
+    // range i; the first piece belongs to the range holding the sequence's start:
+    // i0 - 1, or i0 when cut i0 snaps onto the start (every earlier cut lies at or
+    // before it, every later one after it).
     auto cand = [&](int len, long long st, int &i0, int &i1) {
         i0 = (int)(st / range) + 1;
         const long long e = (st + len - 1) / range + 1;
         i1 = (int)(e < nr ? e : nr);
+    };
+    auto cut = [&](int i, int len, long long st) {
+        const long long o = (long long)i * range - st;   // 0 < o < len
+        long long sn = (o + kTile / 2) / kTile * kTile;
+        if (sn >= len) sn = len;
+        return st + sn;
     };
     // Few sequences (B < 32, where one can hold many cuts): a warp takes a sequence
     // (b = warp, warp + 32, ...) and its lanes the candidate cuts.  Otherwise a thread
@@ -357,8 +357,7 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
     const bool lanes = B < 32;
     const int grp = lanes ? lane : 0, gw = lanes ? 32 : 1;      // lane in the group, width
     const int g0 = lanes ? warp : tid, gstep = lanes ? 32 : 1024;  // first sequence, stride
-    // ---- cuts snap to the sequence's 16-token tiles; a cut snapped onto the
-    // sequence's end (or start) cuts nothing.  Partitions per sequence.
+    // ---- partitions per sequence and pieces per range, in one pass
     for (int b = g0; b < B; b += gstep) {
         int len, i0, i1;
         long long st;
@@ -367,37 +366,16 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
         if (len > 0) {
             cand(len, st, i0, i1);
             for (int i = i0 + grp; i < i1; i += gw) {
-                const long long o = (long long)i * range - st;   // 0 < o < len
-                long long sn = (o + kTile / 2) / kTile * kTile;
-                if (sn >= len) sn = len;
-                s_R[i] = st + sn;
-                if (sn > 0 && sn < len) ++n;
+                const long long r = cut(i, len, st);
+                if (r > st && r < st + len) {
+                    ++n;
+                    atomicAdd(&s_cnt[i], 1);
+                }
             }
             n = 1 + (lanes ? __reduce_add_sync(kFull, n) : n);
+            if (grp == 0) atomicAdd(&s_cnt[(i0 < i1 && cut(i0, len, st) == st) ? i0 : i0 - 1], 1);
         }
         if (grp == 0) ns[b] = n;
-    }
-    __syncthreads();
-    auto owner_of = [&](long long x) {   // largest i < nr with R_i <= x
-        int lo = 0, hi = nr - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (s_R[mid] <= x) lo = mid;
-            else hi = mid - 1;
-        }
-        return lo;
-    };
-    // ---- pieces per range: a sequence's first piece belongs to the range holding its
-    // start, every later piece to the range its cut begins
-    for (int b = g0; b < B; b += gstep) {
-        int len, i0, i1;
-        long long st;
-        seq(b, len, st);
-        if (len == 0) continue;
-        if (grp == 0) atomicAdd(&s_cnt[owner_of(st)], 1);
-        cand(len, st, i0, i1);
-        for (int i = i0 + grp; i < i1; i += gw)
-            if (s_R[i] > st && s_R[i] < st + len) atomicAdd(&s_cnt[i], 1);
     }
     __syncthreads();
     // ---- per-range unit offsets (exclusive scan over the ranges; ranges >= nr empty)
@@ -432,12 +410,13 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
         if (len == 0) continue;
         cand(len, st, i0, i1);
         const long long end = st + len;
-        int own = owner_of(st), c = 0;
+        int own = (i0 < i1 && cut(i0, len, st) == st) ? i0 : i0 - 1, c = 0;
         long long t0 = st;
         for (int i = i0; i <= i1; ++i) {   // each valid cut ends a piece; the end, the last
-            const bool cut = i < i1 && s_R[i] > st && s_R[i] < end;
-            if (i < i1 && !cut) continue;
-            const long long t1 = cut ? s_R[i] : end;
+            const long long r = i < i1 ? cut(i, len, st) : end;
+            const bool is_cut = i < i1 && r > st && r < end;
+            if (i < i1 && !is_cut) continue;
+            const long long t1 = is_cut ? r : end;
             place(own, make_int4(b, c, (int)(t0 - st), (int)(t1 - st)));
             own = i;
             t0 = t1;
@@ -451,24 +430,31 @@ __global__ void __launch_bounds__(1024) plan_balanced_kernel(
         if (len == 0) continue;
         cand(len, st, i0, i1);
         const long long end = st + len;
-        auto valid = [&](int i) { return s_R[i] > st && s_R[i] < end; };
+        auto valid = [&](long long r) { return r > st && r < end; };
         int carry = 0;
         long long first_cut = end;   // where piece 0 ends
         for (int k0 = i0; k0 < i1; k0 += 32) {
             const int i = k0 + lane;
-            const bool v = i < i1 && valid(i);
+            const long long r = i < i1 ? cut(i, len, st) : end;
+            const bool v = i < i1 && valid(r);
             const unsigned m = __ballot_sync(kFull, v);
-            if (first_cut == end && m) first_cut = s_R[k0 + __ffs(m) - 1];
+            if (first_cut == end && m) first_cut = __shfl_sync(kFull, r, __ffs(m) - 1);
             if (v) {
                 int j = i + 1;   // the next valid cut (only a sequence's last candidate
-                while (j < i1 && !valid(j)) ++j;   // can be invalid, so this is short)
-                const long long t1 = j < i1 ? s_R[j] : end;
+                long long rj = end;   // can be invalid, so this is short)
+                for (; j < i1; ++j) {
+                    rj = cut(j, len, st);
+                    if (valid(rj)) break;
+                }
+                const long long t1 = j < i1 ? rj : end;
                 const int c = 1 + carry + __popc(m & ((1u << lane) - 1u));
-                place(i, make_int4(b, c, (int)(s_R[i] - st), (int)(t1 - st)));
+                place(i, make_int4(b, c, (int)(r - st), (int)(t1 - st)));
             }
             carry += __popc(m);
         }
-        if (lane == 0) place(owner_of(st), make_int4(b, 0, 0, (int)(first_cut - st)));
+        if (lane == 0)
+            place((i0 < i1 && cut(i0, len, st) == st) ? i0 : i0 - 1,
+                  make_int4(b, 0, 0, (int)(first_cut - st)));
     }
 }
 
