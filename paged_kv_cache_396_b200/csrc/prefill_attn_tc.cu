@@ -28,7 +28,10 @@
 //              weight).
 //   warp 9     TMA producer: lane p < 8 owns 16-token page p of every tile, looks
 //              up its physical block one tile ahead and issues four boxes (K and V,
-//              two 64-element slices each); two stages.
+//              two 64-element slices each).  K and V stages have barriers of their
+//              own: a K stage frees when the tile's last S is done, a V stage after
+//              its last P V, so the next K tile is on its way about one P V pair
+//              earlier than with one barrier per K/V stage.
 // TMEM: S/P of tile A at columns [0,128), of tile B at [128,256); O of tile A at
 // [256,384), of tile B at [384,512).
 // Work: an item is (sequence, kv head, 256 query rows); a segment is a run of one
@@ -59,8 +62,10 @@ constexpr int kN = 128;          // tokens per K/V tile
 constexpr int kThreads = 320;    // 8 softmax warps, 1 MMA warp, 1 TMA warp
 constexpr int kSlice = kN * 128;         // one 64-element slice of a 128-row tile (bytes)
 constexpr int kTileB = 2 * kSlice;       // a Q, K or V tile (d = 128)
-constexpr int kStages = 2;       // K/V stages in flight
-constexpr int kSmem = 2 * kTileB /*Q x 2*/ + kStages * 2 * kTileB /*K,V per stage*/ + 1024;
+constexpr int kKStages = 2;      // K tiles in flight
+constexpr int kVStages = 2;      // V tiles in flight
+constexpr int kSmem = (2 /*Q x 2*/ + kKStages + kVStages) * kTileB + 1024;
+static_assert(kSmem <= 227 * 1024 - 256, "dynamic shared memory above the per-CTA limit");
 constexpr uint32_t kColO = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;
@@ -169,8 +174,10 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int *a
 
 struct Bars {
     uint64_t q_full;              // 256 softmax threads: the segment's Q rows in shared memory
-    uint64_t kv_full[kStages];    // TMA bytes of a K/V stage
-    uint64_t kv_empty[kStages];   // commit after the last P V that read the stage
+    uint64_t k_full[kKStages];    // TMA bytes of a stage's K tile
+    uint64_t v_full[kVStages];    // TMA bytes of a stage's V tile
+    uint64_t k_empty[kKStages];   // commit after the last S = Q K^T that read the K tile
+    uint64_t v_empty[kVStages];   // commit after the last P V that read the V tile
     uint64_t s_full[2];           // per Q tile: commit after S = Q K^T
     uint64_t p_full[2];           // per Q tile: 128 softmax threads wrote P
     uint64_t pv_done[2];          // per Q tile: commit after O += P V
@@ -325,19 +332,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
     auto sQ = [&](int w) { return base + (uint32_t)(w * kTileB); };
-    auto sK = [&](int st) { return base + (uint32_t)(2 * kTileB + st * 2 * kTileB); };
-    auto sV = [&](int st) { return base + (uint32_t)(3 * kTileB + st * 2 * kTileB); };
+    auto sK = [&](int st) { return base + (uint32_t)((2 + st) * kTileB); };
+    auto sV = [&](int st) { return base + (uint32_t)((2 + kKStages + st) * kTileB); };
 
     // K/V stages start as zeros: a page that is not loaded (bad block id) then
     // holds finite data only
-    for (int x = tid; x < kStages * 2 * kTileB / 16; x += kThreads)
+    for (int x = tid; x < (kKStages + kVStages) * kTileB / 16; x += kThreads)
         *reinterpret_cast<uint4 *>(gbase + 2 * kTileB + 16 * x) = make_uint4(0, 0, 0, 0);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (tid == 0) {
         ptx::mbar_init(&bars.q_full, 256);
-        for (int i = 0; i < kStages; ++i) {
-            ptx::mbar_init(&bars.kv_full[i], 1);
-            ptx::mbar_init(&bars.kv_empty[i], 1);
+        for (int i = 0; i < kKStages; ++i) {
+            ptx::mbar_init(&bars.k_full[i], 1);
+            ptx::mbar_init(&bars.k_empty[i], 1);
+        }
+        for (int i = 0; i < kVStages; ++i) {
+            ptx::mbar_init(&bars.v_full[i], 1);
+            ptx::mbar_init(&bars.v_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&bars.s_full[i], 1);
@@ -689,30 +700,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int len = a.ctx_lens[item_of(a, sg.d, X, QT).b];
             const int nt = sg.je - sg.jb;
             if (!(ok = warp_wait(&bars.q_full, sn & 1, abort_flag) &&
-                       warp_wait(&bars.kv_full[jt % kStages], (jt / kStages) & 1, abort_flag)))
+                       warp_wait(&bars.k_full[jt % kKStages], (jt / kKStages) & 1, abort_flag)))
                 break;
             // the new S overwrites the columns the previous segment's last P V read P
             // from: that segment's products are complete first
             if (sn > 0 && !(ok = warp_wait(&bars.o_final, (sn - 1) & 1, abort_flag))) break;
-            zero_tail(sg.jb, jt % kStages, len);
             fence_after();
-            issue_s(0, jt % kStages);
-            issue_s(1, jt % kStages);
+            issue_s(0, jt % kKStages);
+            issue_s(1, jt % kKStages);
+            commit(&bars.k_empty[jt % kKStages]);
             for (int jj = 0; jj < nt && ok; ++jj, ++jt) {
-                const int st = jt % kStages, st1 = (jt + 1) % kStages;
+                const int st = jt % kVStages, st1 = (jt + 1) % kKStages;
                 const bool more = jj + 1 < nt;
                 // ---- tile A
                 if (!(ok = warp_wait(&bars.p_full[0], jt & 1, abort_flag))) break;
                 if (jj == 0 && sn > 0 &&   // O of the previous segment is read out
                     !(ok = warp_wait(&bars.o_free, (sn - 1) & 1, abort_flag)))
                     break;
+                if (!(ok = warp_wait(&bars.v_full[st], (jt / kVStages) & 1, abort_flag))) break;
+                zero_tail(sg.jb + jj, st, len);
                 fence_after();
                 issue_pv(0, jj, st);
                 if (more) {
-                    if (!(ok = warp_wait(&bars.kv_full[st1], ((jt + 1) / kStages) & 1,
+                    if (!(ok = warp_wait(&bars.k_full[st1], ((jt + 1) / kKStages) & 1,
                                          abort_flag)))
                         break;
-                    zero_tail(sg.jb + jj + 1, st1, len);
                     // S_A(j+1) overwrites the columns PV_A(j) reads its P from
                     if (!(ok = warp_wait(&bars.pv_done[0], jt & 1, abort_flag))) break;
                     fence_after();
@@ -722,12 +734,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!(ok = warp_wait(&bars.p_full[1], jt & 1, abort_flag))) break;
                 fence_after();
                 issue_pv(1, jj, st);
-                commit(&bars.kv_empty[st]);
+                commit(&bars.v_empty[st]);
                 if (!more) commit(&bars.o_final);
                 if (more) {
                     if (!(ok = warp_wait(&bars.pv_done[1], jt & 1, abort_flag))) break;
                     fence_after();
                     issue_s(1, st1);
+                    commit(&bars.k_empty[st1]);
                 }
             }
         }
@@ -747,12 +760,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             int32_t next = lookup(sg.jb);
             for (int j = sg.jb; j < sg.je && ok; ++j, ++jt) {
-                const int st = jt % kStages;
                 const int32_t blk = next;
                 if (j + 1 < sg.je) next = lookup(j + 1);
-                if (jt >= kStages &&
-                    !(ok = warp_wait(&bars.kv_empty[st], ((jt / kStages) - 1) & 1, abort_flag)))
-                    break;
                 const int t = j * kN + 16 * lane;
                 const bool in = lane < kN / 16 && t < it.len;
                 // pages inside the context with a valid block id are loaded; the others
@@ -760,20 +769,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool load = in && blk >= 0 && (int64_t)blk < a.N;
                 if (in && !load) raise_flag(a.err, PA_DEV_BAD_BLOCK);
                 const unsigned lm = __ballot_sync(0xffffffffu, load);
-                if (lane == 0)
-                    ptx::mbar_arrive_expect_tx(&bars.kv_full[st],
-                                               (uint32_t)__popc(lm) * 4u * 2048u);
-                __syncwarp();
-                if (load) {
-                    const int off = t % a.bs;
+                const int off = t % a.bs;
+                // K first: its stage frees when the tile's last S is done, well before
+                // the V stage (after the last P V)
 #pragma unroll
-                    for (int sl = 0; sl < 2; ++sl) {
-                        const uint32_t dk = sK(st) + (uint32_t)(sl * kSlice + lane * 16 * 128);
-                        const uint32_t dv = sV(st) + (uint32_t)(sl * kSlice + lane * 16 * 128);
-                        ptx::tma_load_5d(gbase + (dk - base), &km, &bars.kv_full[st], 0, off,
-                                         it.h, sl, blk);
-                        ptx::tma_load_5d(gbase + (dv - base), &vm, &bars.kv_full[st], 0, off,
-                                         it.h, sl, blk);
+                for (int kv = 0; kv < 2; ++kv) {
+                    const int ns = kv ? kVStages : kKStages, st = jt % ns;
+                    uint64_t *full = kv ? &bars.v_full[st] : &bars.k_full[st];
+                    uint64_t *empty = kv ? &bars.v_empty[st] : &bars.k_empty[st];
+                    if (jt >= ns && !(ok = warp_wait(empty, ((jt / ns) - 1) & 1, abort_flag)))
+                        break;
+                    if (lane == 0)
+                        ptx::mbar_arrive_expect_tx(full, (uint32_t)__popc(lm) * 2u * 2048u);
+                    __syncwarp();
+                    if (load) {
+                        const CUtensorMap *map = kv ? &vm : &km;
+                        const uint32_t s0 = kv ? sV(st) : sK(st);
+#pragma unroll
+                        for (int sl = 0; sl < 2; ++sl) {
+                            const uint32_t dst = s0 + (uint32_t)(sl * kSlice + lane * 16 * 128);
+                            ptx::tma_load_5d(gbase + (dst - base), map, full, 0, off, it.h, sl,
+                                             blk);
+                        }
                     }
                 }
             }
