@@ -36,10 +36,12 @@
 // [256,384), of tile B at [384,512).
 // Work: an item is (sequence, kv head, 256 query rows); a segment is a run of one
 // item's K/V tiles.  Without a workspace each CTA runs one whole item.  With one
-// (balanced mode) a plan kernel ranks the items: full waves of whole items, then
-// one equal range of the left-over items' tiles per SM; a segment cut from an item
-// leaves fp32 partials that the part finishing last merges (every role walks its
-// CTA's segments in a loop, with barrier phases carried across segments).
+// (balanced mode) a plan kernel ranks the items, then two launches: full waves of
+// whole items, and one equal range of the left-over items' tiles per SM, which
+// starts as the whole-item CTAs retire (programmatic dependent launch); a segment
+// cut from an item leaves fp32 partials that the part finishing last merges (the
+// roles of a range CTA walk its segments in a loop, with barrier phases carried
+// across segments).
 // Every mbarrier wait is bounded (2 s of globaltimer); a timeout sets
 // PA_DEV_TIMEOUT and the CTA winds down, freeing its TMEM.
 #include <cuda.h>
@@ -221,20 +223,21 @@ struct Seg {
 // Balanced mode (a plan kernel writes the lists below every call).  With n items
 // that have rows and P SMs, the first whole = floor(n / P) P items, in item order,
 // run one per CTA (full waves; the CTAs of one (sequence, kv head) sweep its K/V
-// together, from L2).  The r = n - whole items left over are laid end to end (R
-// tiles) and CTA whole + k takes tiles [k L, (k + 1) L), L = ceil(R / P): one or
-// a few segments, the last wave then ends about evenly on every SM.  A segment
-// cut from an item writes its partial result to slot 2k (the item began in an
-// earlier range) or 2k + 1; for each 32 rows (a softmax warp) the part that
-// finishes last merges the item's parts in range order.  CTAs after those zero
-// the rows of items whose length cannot be served.
+// together, from L2); the CTAs after those zero the rows of items whose length
+// cannot be served.  The r = n - whole items left over are laid end to end (R
+// tiles) and CTA k of the second launch takes tiles [k L, (k + 1) L), L =
+// ceil(R / P): one or a few segments, the last wave then ends about evenly on
+// every SM.  A segment cut from an item writes its partial result to slot 2k (the
+// item began in an earlier range) or 2k + 1; for each 32 rows (a softmax warp) the
+// part that finishes last merges the item's parts in range order.
 struct StreamWs {
     const int *hdr;     // whole, r, R, L, n_bad
     const int *items;   // [n + n_bad] item index by rank, then the bad items
     const int *pre;     // [r + 1] tile offsets of the items left over
     const int *lrank;   // [n_items] rank among the items left over, -1: not left over
     int *cnt;           // [n_items][8] parts done per (item, softmax warp)
-    float *part;        // [2P][256][d] O of a part (not normalised)
+    float *part;        // [2P][8 softmax warps][d / 4][32 lanes] float4: O of a part
+                        // (not normalised), row = 32 warp + lane
     float *ml;          // [2P][256][2] (m, l) of a part; m in the log2 domain
     int n_items, X, P;
 };
@@ -251,10 +254,14 @@ __device__ __forceinline__ Seg left_seg(const StreamWs &w, int lr, int k, int R,
     return s;
 }
 
-// kStream = false: one CTA per item (grid x, y, z = q tile, kv head, sequence).
-// kStream = true: CTA c runs segment c of the balanced mode's list.  (Every role
-// walks a CTA's segments in a loop, so a CTA could serve several.)
-template <bool kStream>
+// Modes.  kGrid: one CTA per item (grid x, y, z = q tile, kv head, sequence).  The
+// balanced mode is two launches: kWhole, CTA k runs whole item k of the plan's ranking
+// (k < whole), CTA whole + i zeroes the rows of bad-length item i; kLeft, CTA k runs
+// the k-th equal range of the left-over items' tiles (one or a few segments, walked in
+// a loop by every role).  The whole items keep the loop-free code of the grid mode;
+// only the range CTAs carry the segment state.
+enum { kGrid = 0, kWhole = 1, kLeft = 2 };
+template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap km,
                            const __grid_constant__ CUtensorMap vm, const PrefillAttnArgs a,
@@ -264,28 +271,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int G = a.G, QT = kRows / G;   // query tokens per item (two tiles of 128 rows)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int k = blockIdx.x;
-    const int X = kStream ? sw.X : (int)gridDim.x;
+    const int X = kMode != kGrid ? sw.X : (int)gridDim.x;
+    // the range launch may start as soon as every whole-item CTA has started (it
+    // shares no data with them; it waits for their completion before it exits)
+    if constexpr (kMode == kWhole) ptx::grid_launch_dependents();
     auto first_seg = [&]() -> Seg {
-        if constexpr (kStream) {
-            const int whole = sw.hdr[0], R = sw.hdr[2], L = sw.hdr[3], n_bad = sw.hdr[4];
+        if constexpr (kMode == kWhole) {
+            const int whole = sw.hdr[0], n_bad = sw.hdr[4];
             if (k < whole) {
                 const int d = sw.items[k];
                 return Seg{d, 0, item_of(a, d, X, QT).n_kt, -1};
             }
-            const int kk = k - whole;
-            if (kk >= sw.P) {   // zero-row CTAs for bad lengths, then nothing
-                if (kk - sw.P < n_bad)
-                    return Seg{sw.items[whole + sw.hdr[1] + kk - sw.P], 0, 0, -2};
-                return Seg{-1, 0, 0, -1};
-            }
-            if (kk * L >= R) return Seg{-1, 0, 0, -1};
-            int lo = 0, hi = sw.hdr[1];   // the left-over item holding tile kk L
+            if (k - whole < n_bad)   // zero-row CTAs for bad lengths
+                return Seg{sw.items[whole + sw.hdr[1] + k - whole], 0, 0, -2};
+            return Seg{-1, 0, 0, -1};
+        } else if constexpr (kMode == kLeft) {
+            const int whole = sw.hdr[0], R = sw.hdr[2], L = sw.hdr[3];
+            if (k >= sw.P || k * L >= R) return Seg{-1, 0, 0, -1};
+            int lo = 0, hi = sw.hdr[1];   // the left-over item holding tile k L
             while (hi - lo > 1) {
                 const int mid = (lo + hi) >> 1;
-                if (sw.pre[mid] <= kk * L) lo = mid;
+                if (sw.pre[mid] <= k * L) lo = mid;
                 else hi = mid;
             }
-            return left_seg(sw, lo, kk, R, L, whole);
+            return left_seg(sw, lo, k, R, L, whole);
         } else {
             const int d = ((int)blockIdx.z * a.Hkv + (int)blockIdx.y) * X + (int)blockIdx.x;
             const Item it = item_of(a, d, X, QT);
@@ -293,13 +302,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     };
     auto next_seg = [&](const Seg &cur) -> Seg {
-        if constexpr (kStream) {
+        if constexpr (kMode == kLeft) {
             const int whole = sw.hdr[0], R = sw.hdr[2], L = sw.hdr[3];
-            const int kk = k - whole;
-            if (kk < 0 || kk >= sw.P) return Seg{-1, 0, 0, -1};
             const int lr = sw.lrank[cur.d] + 1;
-            if (lr >= sw.hdr[1] || sw.pre[lr] >= min(R, (kk + 1) * L)) return Seg{-1, 0, 0, -1};
-            return left_seg(sw, lr, kk, R, L, whole);
+            if (lr >= sw.hdr[1] || sw.pre[lr] >= min(R, (k + 1) * L)) return Seg{-1, 0, 0, -1};
+            return left_seg(sw, lr, k, R, L, whole);
         } else {
             return Seg{-1, 0, 0, -1};
         }
@@ -308,10 +315,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // an item whose length cannot be served: zero rows and PA_DEV_BAD_LEN (grid mode:
     // no segment; balanced mode: a listed zero segment, slot -2)
     int bad_d = -1;
-    if constexpr (!kStream) {
+    if constexpr (kMode == kGrid) {
         if (seg0.d < 0) bad_d = ((int)blockIdx.z * a.Hkv + (int)blockIdx.y) * X + (int)blockIdx.x;
     } else {
-        if (seg0.d < 0) return;   // no work for this CTA
+        if (seg0.d < 0) {   // no work for this CTA
+            if constexpr (kMode == kLeft) ptx::grid_dependency_wait();
+            return;
+        }
         if (seg0.slot == -2) bad_d = seg0.d;
     }
     if (bad_d >= 0) {
@@ -400,12 +410,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         int jt = 0, sn = 0;   // tiles and segments this CTA has done (barrier phases)
         Seg sg = seg0;
-        Item it = item_of(a, sg.d, X, QT);
-        load_q(it);
+        load_q(item_of(a, sg.d, X, QT));
         while (ok) {
-            const int i = it.tok_base + R / G;       // query token in the sequence's chunk
-            const bool valid = i < it.ql;
-            const int pos = it.pos0 + min(i, it.ql - 1);   // causal limit (inclusive)
+            // what the row needs from its item, taken once (the item itself is not
+            // kept live across the tile loop)
+            int i, pos, nkt;
+            int64_t orow_off;
+            {
+                const Item it = item_of(a, sg.d, X, QT);
+                i = it.tok_base + R / G;             // query token in the sequence's chunk
+                pos = it.pos0 + min(i, it.ql - 1);   // causal limit (inclusive)
+                orow_off = ((int64_t)(it.q0 + min(i, it.ql - 1)) * a.Hq + it.h * G + R % G) * kD;
+                nkt = it.n_kt;
+                if (i >= it.ql) i = -1;
+            }
+            const bool valid = i >= 0;
             float m = -INFINITY, l = 0.f;
             for (int j = sg.jb; j < sg.je && ok; ++j, ++jt) {
                 if (!(ok = warp_wait(&bars.s_full[w], jt & 1, abort_flag))) break;
@@ -507,17 +526,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // every S of this segment is done: the next segment's Q rows can go to
             // shared memory now, so its first S overlaps this epilogue
             const Seg nx = next_seg(sg);
-            Item itn;
-            if (nx.d >= 0) {
-                itn = item_of(a, nx.d, X, QT);
-                load_q(itn);
-            }
+            if (nx.d >= 0) load_q(item_of(a, nx.d, X, QT));
             if (!(ok = warp_wait(&bars.o_final, sn & 1, abort_flag))) break;
             fence_after();
             if (sg.slot < 0) {   // the whole item: the normalised bf16 output row
                 const float inv = l > 0.f ? 1.f / l : 0.f;
-                uint4 *orow = reinterpret_cast<uint4 *>(
-                    a.out + ((int64_t)(it.q0 + min(i, it.ql - 1)) * a.Hq + it.h * G + R % G) * kD);
+                uint4 *orow = reinterpret_cast<uint4 *>(a.out + orow_off);
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t v[32];
@@ -543,22 +557,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // the item's parts: ranges k0 .. k1 of the left-over tiles
                 const int L = sw.hdr[3];
                 const int a0 = sw.pre[sw.lrank[sg.d]];
-                const int k0 = a0 / L, k1 = (a0 + it.n_kt - 1) / L;
+                const int k0 = a0 / L, k1 = (a0 + nkt - 1) / L;
                 auto slot_of = [&](int kk) { return a0 < kk * L ? 2 * kk : 2 * kk + 1; };
-                float4 *prow = reinterpret_cast<float4 *>(
-                    sw.part + ((int64_t)sg.slot * kRows + R) * kD);
+                // [slot][softmax warp][d/4][lane] float4: each warp store covers 512
+                // contiguous bytes
+                float4 *pw = reinterpret_cast<float4 *>(sw.part) +
+                             ((int64_t)sg.slot * 8 + warp) * (kD / 4) * 32 + lane;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t v[32];
                     tmem_ld32(obuf + 32 * c, v);
                     tmem_wait_ld();
-                    if (valid) {
 #pragma unroll
-                        for (int e4 = 0; e4 < 8; ++e4)
-                            prow[8 * c + e4] = make_float4(
-                                __uint_as_float(v[4 * e4]), __uint_as_float(v[4 * e4 + 1]),
-                                __uint_as_float(v[4 * e4 + 2]), __uint_as_float(v[4 * e4 + 3]));
-                    }
+                    for (int e4 = 0; e4 < 8; ++e4)
+                        pw[(8 * c + e4) * 32] = make_float4(
+                            __uint_as_float(v[4 * e4]), __uint_as_float(v[4 * e4 + 1]),
+                            __uint_as_float(v[4 * e4 + 2]), __uint_as_float(v[4 * e4 + 3]));
                 }
                 if (valid)
                     *reinterpret_cast<float2 *>(sw.ml + ((int64_t)sg.slot * kRows + R) * 2) =
@@ -579,21 +593,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         return __ldcg(reinterpret_cast<const float2 *>(
                             sw.ml + ((int64_t)slot_of(kk) * kRows + R) * 2));
                     };
-                    float M = -INFINITY;
+                    // M and L in one pass: L rescaled whenever M grows
+                    float M = -INFINITY, Ls = 0.f;
 #pragma unroll 4
-                    for (int kk = k0; kk <= k1; ++kk) M = fmaxf(M, mlrow(kk).x);
-                    float Ls = 0.f;
-                    if (M != -INFINITY) {
-#pragma unroll 4
-                        for (int kk = k0; kk <= k1; ++kk) {
-                            const float2 ml = mlrow(kk);
-                            Ls = fmaf(ml.y, exp2f(ml.x - M), Ls);
+                    for (int kk = k0; kk <= k1; ++kk) {
+                        const float2 ml = mlrow(kk);
+                        if (ml.x == -INFINITY) continue;
+                        if (ml.x > M) {
+                            Ls = Ls * exp2f(M - ml.x);   // exp2(-inf) = 0 for the first
+                            M = ml.x;
                         }
+                        Ls = fmaf(ml.y, exp2f(ml.x - M), Ls);
                     }
                     const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-                    uint4 *orow = reinterpret_cast<uint4 *>(
-                        a.out + ((int64_t)(it.q0 + min(i, it.ql - 1)) * a.Hq + it.h * G + R % G) *
-                                    kD);
+                    uint4 *orow = reinterpret_cast<uint4 *>(a.out + orow_off);
 #pragma unroll 1
                     for (int c = 0; c < 4; ++c) {   // 32 dims a chunk
                         float acc[32];
@@ -609,12 +622,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         };
                         auto load = [&](int kk, float4 (&x)[8]) {
-                            const float4 *src = reinterpret_cast<const float4 *>(
-                                                    sw.part + ((int64_t)slot_of(kk) * kRows + R) *
-                                                                  kD) +
-                                                8 * c;
+                            const float4 *src = reinterpret_cast<const float4 *>(sw.part) +
+                                                ((int64_t)slot_of(kk) * 8 + warp) * (kD / 4) * 32 +
+                                                (8 * c) * 32 + lane;
 #pragma unroll
-                            for (int e4 = 0; e4 < 8; ++e4) x[e4] = __ldcg(src + e4);
+                            for (int e4 = 0; e4 < 8; ++e4) x[e4] = __ldcg(src + 32 * e4);
                         };
                         if (M != -INFINITY) {
                             int kk = k0;
@@ -652,7 +664,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++sn;
             if (nx.d < 0) break;
             sg = nx;
-            it = itn;
         }
     } else if (warp == 8) {
         // ======================= MMA issue =======================
@@ -802,6 +813,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tm),
                      "r"(kTmemCols));
+    // the call is complete only when the whole-item launch is
+    if constexpr (kMode == kLeft) ptx::grid_dependency_wait();
 }
 
 // Exclusive prefix sum over the 1024 threads of a CTA; *total receives the sum.
@@ -968,25 +981,28 @@ cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs &a, int max_q_len, void
         return cudaErrorInvalidValue;
     const size_t need = prefill_attn_tc_workspace_bytes(a, max_q_len, sms);
     const bool stream = ws != nullptr && need > 0 && ws_bytes >= need;
-    auto kfn = stream ? prefill_attn_tc_kernel<true> : prefill_attn_tc_kernel<false>;
-    static bool attr_set[2][64] = {};
+    static bool attr_set[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-    if (dev >= 64 || !attr_set[stream][dev]) {
-        cudaError_t e =
-            cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-        if (e != cudaSuccess) return e;
-        if (dev < 64) attr_set[stream][dev] = true;
+    if (dev >= 64 || !attr_set[dev]) {
+        for (auto kfn : {prefill_attn_tc_kernel<kGrid>, prefill_attn_tc_kernel<kWhole>,
+                         prefill_attn_tc_kernel<kLeft>}) {
+            cudaError_t e =
+                cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+            if (e != cudaSuccess) return e;
+        }
+        if (dev < 64) attr_set[dev] = true;
     }
     StreamWs sw = {};
     if (!stream) {
         const int QT = kRows / a.G;
         dim3 grid((unsigned)((max_q_len + QT - 1) / QT), (unsigned)a.Hkv, (unsigned)a.B);
-        kfn<<<grid, kThreads, kSmem, st>>>(km, vm, a, sw);
+        prefill_attn_tc_kernel<kGrid><<<grid, kThreads, kSmem, st>>>(km, vm, a, sw);
         return cudaGetLastError();
     }
-    // balanced: plan, then whole items, one range of the left-over tiles per SM and
-    // the zero-row CTAs (cut items are merged by their last part)
+    // balanced: plan; the whole items and the zero-row CTAs; one range of the left-over
+    // tiles per SM, launched to start as the whole-item CTAs retire (cut items are
+    // merged by their last part)
     const StreamLayout L = stream_layout(a.B, a.Hkv, a.G, max_q_len, sms);
     char *w = static_cast<char *>(ws);
     sw.hdr = reinterpret_cast<int *>(w);
@@ -1002,9 +1018,21 @@ cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs &a, int max_q_len, void
     prefill_plan_kernel<<<1, 1024, 0, st>>>(a, sw);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    // whole + P + n_bad <= n_items + P CTAs do work; the rest return at once
-    kfn<<<(unsigned)(L.n_items + sms), kThreads, kSmem, st>>>(km, vm, a, sw);
-    return cudaGetLastError();
+    // whole + n_bad <= n_items CTAs do work; the rest return at once
+    prefill_attn_tc_kernel<kWhole><<<(unsigned)L.n_items, kThreads, kSmem, st>>>(km, vm, a, sw);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)sms);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_attn_tc_kernel<kLeft>, km, vm, a, sw);
 }
 
 }  // namespace pkv
