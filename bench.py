@@ -879,7 +879,8 @@ def run_chunked(args, device, world, rank, cpu_baseline=True):
     stream = torch.cuda.current_stream(device)
     # one CTA per 256-row query tile (256 tiles here, more than the SMs): the call
     # without a workspace; the balanced mode pays off when the tiles are fewer than
-    # the SMs, and on this workload it measured the same
+    # the SMs, and on this workload it measured slower (370 against 360 us: its range
+    # CTAs lose the K/V tiles that the CTAs of one kv head share in lockstep)
     attn_launches = 1
 
     def step(ev=None):

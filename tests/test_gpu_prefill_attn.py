@@ -126,6 +126,34 @@ def test_balanced_mode_with_few_long_items(qlens):
     assert_attention_close(out, _oracle(c), f"balanced, q lens {qlens}")
 
 
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+def test_balanced_mode_items_a_multiple_of_the_sms():
+    """As many items as SMs (one kv head, a group of 8, one 32-token query tile per
+    sequence): every item runs whole in the first launch and the range launch has
+    no tiles; its CTAs only wait for the first launch."""
+    P = _sms()
+    rng = np.random.default_rng(51)
+    lens = [int(x) for x in rng.integers(33, 400, P)]
+    qlens = [int(x) for x in rng.integers(1, 33, P)]
+    c = _case(lens, qlens, 8, 1, 128, 16, seed=52)
+    assert_attention_close(_run(c, balanced=True), _oracle(c), "items = SMs")
+
+
+def test_balanced_mode_more_than_two_waves_of_whole_items():
+    """2 P + 13 items: two full waves of whole items (the range launch can start only
+    after every whole-item CTA has started), then 13 long items cut into many
+    one-tile ranges, each merged from several parts."""
+    P = _sms()
+    rng = np.random.default_rng(53)
+    lens = [int(x) for x in rng.integers(33, 300, 2 * P)] + [2500 + 97 * i for i in range(13)]
+    qlens = [int(x) for x in rng.integers(1, 33, 2 * P)] + [32] * 13
+    c = _case(lens, qlens, 8, 1, 128, 16, seed=54)
+    assert_attention_close(_run(c, balanced=True), _oracle(c), "2 P + 13 items")
+
+
 def test_balanced_mode_is_deterministic():
     c = _case([3000, 800], [512, 300], 32, 8, 128, 16, seed=31)
     a = _run(c, balanced=True)
