@@ -155,6 +155,31 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Two fp32 lanes per instruction (sm_100 packed fp32): each lane rounds as the scalar
+// fmaf / addition does.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // bounded wait; false (and the abort flag set) on timeout
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, int *abort_flag) {
     const uint64_t t0 = ptx::globaltimer();
@@ -436,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool full = __all_sync(0xffffffffu, lim >= kN - 1) && sl > 0.f;
                 // ---- the row's 128 logits of this tile: four 32-column TMEM reads in
                 // flight, one wait; then the row maximum of the scaled, masked logits
-                // (8 independent max chains)
+                // (8 independent max chains, two logits per three-input max)
                 uint32_t v[4][32];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(sbuf + 32 * c, v[c]);
@@ -448,8 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            mk[e & 7] = fmaxf(mk[e & 7], __uint_as_float(v[c][e]));
+                        for (int e = 0; e < 32; e += 2)
+                            mk[(e >> 1) & 7] = max3(mk[(e >> 1) & 7], __uint_as_float(v[c][e]),
+                                                    __uint_as_float(v[c][e + 1]));
                 } else {
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
@@ -460,8 +486,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mk[e & 7] = fmaxf(mk[e & 7], x);
                         }
                 }
-                float mx = fmaxf(fmaxf(fmaxf(mk[0], mk[1]), fmaxf(mk[2], mk[3])),
-                                 fmaxf(fmaxf(mk[4], mk[5]), fmaxf(mk[6], mk[7])));
+                float mx = max3(max3(mk[0], mk[1], mk[2]), max3(mk[3], mk[4], mk[5]),
+                                fmaxf(mk[6], mk[7]));
                 if (full) mx *= sl;
                 const float mn = fmaxf(m, mx);
                 // lazy rescale: a row moves its reference max only when the tile's max
@@ -474,12 +500,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float u = m == -INFINITY ? 0.f : m;
                 // ---- P = exp2(s - u) as hi + lo bf16 over the S columns: k-step kk
                 // (16 tokens) at columns 16kk (hi, 8 columns of bf16 pairs) and 16kk + 8 (lo)
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                // (scale-subtract, row sums and the lo remainders two lanes at a time)
+                float2 ls[4] = {};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     float x[32];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = fmaf(__uint_as_float(v[c][e]), sl, -u);
+                    for (int e = 0; e < 32; e += 2) {
+                        const float2 y = fma2(make_float2(__uint_as_float(v[c][e]),
+                                                          __uint_as_float(v[c][e + 1])),
+                                              make_float2(sl, sl), make_float2(-u, -u));
+                        x[e] = y.x;
+                        x[e + 1] = y.y;
+                    }
                     if (!full) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
@@ -491,12 +524,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
                             const int e = 16 * half + 2 * q;
-                            const float p0 = ex2(x[e]), p1 = ex2(x[e + 1]);
-                            ls[q & 3] += p0 + p1;
-                            const uint32_t hi = ptx::pack_bf16(p0, p1);
-                            wv[16 * half + q] = hi;
+                            const float2 pp = make_float2(ex2(x[e]), ex2(x[e + 1]));
+                            ls[q & 3] = add2(ls[q & 3], pp);
+                            // hi = each weight's top 16 bits (truncated), lo = the exact
+                            // remainder truncated the same way: hi + lo is within 2^-15 of
+                            // the weight, and no conversion instruction runs
+                            const uint32_t b0 = __float_as_uint(pp.x), b1 = __float_as_uint(pp.y);
+                            wv[16 * half + q] = __byte_perm(b0, b1, 0x7632);
+                            const float2 rr = add2(
+                                pp, make_float2(__uint_as_float((b0 & 0xffff0000u) ^ 0x80000000u),
+                                                __uint_as_float((b1 & 0xffff0000u) ^ 0x80000000u)));
                             wv[16 * half + 8 + q] =
-                                ptx::pack_bf16(p0 - bf16_lo(hi), p1 - bf16_hi(hi));
+                                __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
                         }
                     }
                     tmem_st32(sbuf + 32 * c, wv);
@@ -517,7 +556,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_st32(obuf + 32 * c, o);
                     }
                 }
-                l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+                const float2 ls2 = add2(add2(ls[0], ls[1]), add2(ls[2], ls[3]));
+                l = l * alpha + (ls2.x + ls2.y);
                 tmem_wait_st();
                 fence_before();
                 ptx::mbar_arrive(&bars.p_full[w]);
