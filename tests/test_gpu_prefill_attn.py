@@ -241,7 +241,8 @@ def test_full_size_chunk_sampled_rows(balanced):
 
 
 
-def test_dominant_tokens_keep_the_tolerance():
+@pytest.mark.parametrize("balanced", [False, True])
+def test_dominant_tokens_keep_the_tolerance(balanced):
     """Rows whose softmax puts almost all weight on two or three tokens with values of
     opposite sign (the case where one rounding of the weights shows most): keys equal
     to a multiple of the query make those tokens dominate."""
@@ -255,7 +256,7 @@ def test_dominant_tokens_keep_the_tolerance():
             # head 0's query rows of this sequence all see these keys strongly
             k[blk, off, 0] = q[c["cu"][b], 0] * (1.2 + 0.05 * n)
     c["k"] = k.to(torch.bfloat16)
-    out = _run(c)
+    out = _run(c, balanced=balanced)
     assert_attention_close(out, _oracle(c), "few dominant tokens")
 
 
