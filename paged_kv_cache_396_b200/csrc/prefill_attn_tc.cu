@@ -14,9 +14,11 @@
 //              per 128-token K/V tile reads its 128 logits from TMEM (four loads,
 //              one wait), masks (causal, diagonal tiles only), keeps the running
 //              max (lazy: O is rescaled only when the max grows by more than 2^8),
-//              writes P = hi + lo (two bf16 parts) back over the S columns, and at
-//              the end normalises O (or, for a cut item, writes its partial and the
-//              last part merges).  The two warpgroups work half a step apart, so
+//              writes P = hi + lo (two bf16 parts: the weight's top 16 bits and the
+//              remainder's) back over the S columns, and at the end normalises O
+//              (or, for a cut item, writes its partial and the last part merges).
+//              The per-weight arithmetic runs on packed fp32 pairs: this warp's
+//              instruction stream is on the critical path of the tile period.  The two warpgroups work half a step apart, so
 //              one computes softmax while the tensor core runs the other tile's
 //              products.
 //   warp 8     MMA issue (warp-uniform operands, elect.sync picks the issuing
