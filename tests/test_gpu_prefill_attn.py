@@ -260,6 +260,27 @@ def test_dominant_tokens_keep_the_tolerance(balanced):
     assert_attention_close(out, _oracle(c), "few dominant tokens")
 
 
+@pytest.mark.parametrize("balanced", [False, True])
+def test_late_dominant_tokens_rescale_the_output(balanced):
+    """Online softmax across K/V tiles ([KVP] "PagedAttention 的算子"): keys that
+    dominate only in later tiles, each stronger than the last, move the rows' running
+    maximum by more than a factor 2^8 after O already holds earlier tiles, so the
+    kernel rescales O mid-row (the lazy rescale that random N(0, 1) logits never
+    reach).  Head 0's rows of each chunk see logits of about 10, 20 and 33 (log2
+    units) at those tokens against about 4 elsewhere."""
+    c = _case([900, 700], [128, 256], 32, 8, 128, 16, seed=53)
+    k = c["k"].float()
+    q = c["q"].float()
+    bt = c["bt"]
+    for b, toks in enumerate(((300, 600, 850), (200, 450, 690))):
+        for t, f in zip(toks, (0.6, 1.2, 2.0)):
+            blk, off = bt[b, t // 16], t % 16
+            k[blk, off, 0] = q[c["cu"][b], 0] * f
+    c["k"] = k.to(torch.bfloat16)
+    out = _run(c, balanced=balanced)
+    assert_attention_close(out, _oracle(c), "late dominant tokens")
+
+
 def _random_case(i):
     """Seeded random chunked-prefill shape: 1-6 sequences, chunks from 0 rows to the
     whole context, lengths around tile and block boundaries, G 1-16, d 64 / 128,
