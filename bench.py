@@ -207,6 +207,26 @@ class Clocks:
 
 
 # ----------------------------------------------------------------------------- model
+def clocks_under_load(clk, device, run_steps, seconds=0.8):
+    """The clock record of a run.  The timed region's own samples stand when there are
+    at least 3 (the sampler polls every 200 ms).  A shorter region (p2's 20 steps take
+    about 7 ms) yields samples of the idle GPU around it.  So the same step then runs
+    back to back, untimed, for `seconds` right after the timed region, and its samples
+    are the record; the timed region's own are kept under 'timed_region'."""
+    if clk is not None and clk.get("samples", 0) >= 3:
+        return dict(clk, window="timed region")
+    soak = Clocks(device)
+    t_end = time.perf_counter() + seconds
+    while time.perf_counter() < t_end:
+        run_steps()
+        torch.cuda.synchronize(device)
+    rec = soak.stop()
+    if rec is None:
+        return clk
+    return dict(rec, window=f"the same step back to back for {seconds} s after the timed "
+                            "region (too short for a 200 ms sampler)", timed_region=clk)
+
+
 def decode_algorithmic_bytes(cfg, ctx_lens, partial_slots, n_units=0):
     """Bytes one decode call (one layer) must move: K/V rows of every cached
     token (plus INT8 scales), q and out, the table entries and lengths read, the
@@ -747,7 +767,7 @@ def run_prefill(args, device, world, rank, cpu_baseline=True):
         step(evs[k])
     t1.record(stream)
     torch.cuda.synchronize(device)
-    clk = clocks.stop()
+    clk = clocks_under_load(clocks.stop(), device, lambda: [step() for _ in range(8)])
     ms = reduce_max(t0.elapsed_time(t1), world) / args.steps
     per = [[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in evs]
     score_s = statistics.median(p[0] for p in per) / 1000.0
@@ -915,7 +935,7 @@ def run_chunked(args, device, world, rank, cpu_baseline=True):
         t1.record(stream)
         torch.cuda.synchronize(device)
         total += t0.elapsed_time(t1)
-    clk = clocks.stop()
+    clk = clocks_under_load(clocks.stop(), device, lambda: [step() for _ in range(8)])
     ms = reduce_max(total / args.steps, world)
     attn_s = statistics.median(e[0].elapsed_time(e[1]) for e in evs) / 1000.0
     flops = chunk_flops(cfg)
@@ -1053,7 +1073,16 @@ def run_decode(args, cfg, device, world, rank, cpu_baseline=True):
             r.step()
     t_end.record(stream)
     torch.cuda.synchronize(device)
-    clk = clocks.stop()
+
+    def soak_steps():
+        if use_graph:
+            for g in order:
+                g.replay()
+        else:
+            for _ in range(args.steps):
+                r.step()
+
+    clk = clocks_under_load(clocks.stop(), device, soak_steps)
     total_ms = reduce_max(t_start.elapsed_time(t_end), world)
     ms_per_step = total_ms / args.steps
     value = job_tokens_per_s(world, cfg.batch, ms_per_step)

@@ -111,3 +111,39 @@ def test_c2_step_makes_each_layers_calls_once(evict, select, per_layer):
     r = _runner("c2", evict, select)
     r.step()
     assert r.pk.calls == ["pa_decode_prepare"] + per_layer * r.L
+
+
+class _FakeClocks:
+    """Stands in for the nvidia-smi sampler: records that it ran, returns a soak record."""
+    started = 0
+
+    def __init__(self, device):
+        _FakeClocks.started += 1
+
+    def stop(self):
+        return {"sm_mhz": 1700.0, "sm_max_mhz": 1965.0, "samples": 4, "reasons": ["sw_power_cap"]}
+
+
+def test_clock_record_keeps_a_timed_region_with_enough_samples(monkeypatch):
+    monkeypatch.setattr(bench, "Clocks", _FakeClocks)
+    _FakeClocks.started = 0
+    timed = {"sm_mhz": 1672.0, "sm_max_mhz": 1965.0, "samples": 7, "reasons": ["sw_power_cap"]}
+    calls = []
+    rec = bench.clocks_under_load(timed, "cpu", lambda: calls.append(1))
+    assert rec["sm_mhz"] == 1672.0 and rec["window"] == "timed region"
+    assert calls == [] and _FakeClocks.started == 0
+
+
+@pytest.mark.parametrize("timed", [None, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0,
+                                          "samples": 2, "reasons": []}])
+def test_clock_record_soaks_after_a_short_timed_region(monkeypatch, timed):
+    """Fewer than 3 samples (a region shorter than the sampler's period): the same step
+    runs back to back for the soak time, and its samples become the record."""
+    monkeypatch.setattr(bench, "Clocks", _FakeClocks)
+    monkeypatch.setattr(bench.torch.cuda, "synchronize", lambda device=None: None)
+    _FakeClocks.started = 0
+    calls = []
+    rec = bench.clocks_under_load(timed, "cpu", lambda: calls.append(1), seconds=0.05)
+    assert len(calls) >= 1 and _FakeClocks.started == 1
+    assert rec["sm_mhz"] == 1700.0 and rec["reasons"] == ["sw_power_cap"]
+    assert rec["timed_region"] == timed and "after the timed region" in rec["window"]
