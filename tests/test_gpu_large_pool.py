@@ -245,3 +245,67 @@ def test_chunked_prefill_attention_beyond_2_31_elements(balanced):
     ref = oracle.paged_prefill(W.bits(q), cu, W.bits(ks).ravel(), W.bits(vs).ravel(),
                                BS * HKV * d, x["bt"], lens, HKV, BS, x["scale"])
     assert_attention_close(outs[1], ref, "chunked prefill over a pool past 2^31 elements")
+
+
+def test_scored_append_beyond_2_31_elements():
+    """The append that also writes each new token's ||V|| / ||K|| into the paged score
+    pool ([KVL] "PagedEviction 块级驱逐机制"): the KV rows and the score entries land
+    in the same blocks as in the small pool, bit for bit."""
+    dev, d = "cuda", 128
+    x = _common(1500, d)
+    base, n_big = _layout(BS * HKV * d, x["n_small"])
+    g = x["g"]
+    ks = torch.randn(x["n_small"], BS, HKV, d, generator=g).to(torch.bfloat16).to(dev)
+    vs = torch.randn(x["n_small"], BS, HKV, d, generator=g).to(torch.bfloat16).to(dev)
+    ss = torch.rand(x["n_small"], BS, HKV, generator=g).to(dev)
+    kb, ids = _place(ks, n_big, base, float("nan"))
+    vb, _ = _place(vs, n_big, base, float("nan"))
+    sb, _ = _place(ss, n_big, base, float("nan"))
+    bt_s = torch.as_tensor(x["bt"], device=dev)
+    bt_b = torch.as_tensor(np.where(x["bt"] >= 0, base + STEP * x["bt"], -1).astype(np.int32),
+                           device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    pk.pa_append_kv_scored(x["k_new"], x["v_new"], ks, vs, ss, bt_s, x["pos"], err)
+    pk.pa_append_kv_scored(x["k_new"], x["v_new"], kb, vb, sb, bt_b, x["pos"], err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    _same_bits(kb[ids], ks, "K blocks")
+    _same_bits(vb[ids], vs, "V blocks")
+    _same_bits(sb[ids], ss, "score pool blocks")
+
+
+def test_prefill_compression_beyond_2_31_elements():
+    """PagedEviction's prefill stage ([KVL]): score, keep the budget's highest-ranking
+    prompt tokens, and pack them at positions 0.. of each sequence through its block
+    table.  Written into a pool past 2^31 elements, the blocks equal the small pool's."""
+    dev, d, budget = "cuda", 128, 256
+    g = torch.Generator().manual_seed(1600)
+    plens = [500, 1500, 40]
+    cu = torch.as_tensor(np.concatenate([[0], np.cumsum(plens)]).astype(np.int32), device=dev)
+    T = int(cu[-1])
+    k = torch.randn(T, HKV, d, generator=g).to(torch.bfloat16).to(dev)
+    v = torch.randn(T, HKV, d, generator=g).to(torch.bfloat16).to(dev)
+    B, nb = len(plens), budget // BS
+    n_small = B * nb + 2
+    perm = np.random.default_rng(1600).permutation(n_small).astype(np.int32)
+    bt = perm[:B * nb].reshape(B, nb)
+    base, n_big = _layout(BS * HKV * d, n_small)
+    ks = torch.zeros(n_small, BS, HKV, d, dtype=torch.bfloat16, device=dev)
+    vs = torch.zeros_like(ks)
+    kb, ids = _place(ks, n_big, base, float("nan"))
+    vb, _ = _place(vs, n_big, base, float("nan"))
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    res = []
+    for kc, vc, table in ((ks, vs, bt), (kb, vb, base + STEP * bt)):
+        scores = torch.empty(T, dtype=torch.float32, device=dev)
+        keep = torch.full((B, budget), -7, dtype=torch.int32, device=dev)
+        kept = torch.full((B,), -7, dtype=torch.int32, device=dev)
+        pk.pe_prefill_compress(kc, vc, torch.as_tensor(table.astype(np.int32), device=dev), k, v,
+                               cu, scores, keep, kept, err)
+        res.append((keep, kept))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+    assert res[0][1].tolist() == [min(n, budget) for n in plens]
+    _same_bits(kb[ids], ks, "K blocks after the pack")
+    _same_bits(vb[ids], vs, "V blocks after the pack")
