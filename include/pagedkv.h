@@ -44,6 +44,12 @@
  *     pool/base pointers 16-byte aligned and block_stride*elt a multiple of 16;
  *     B <= 65535 and Hkv <= 65535 (grid limits), N <= 2^31 - 1 and
  *     MB*bs <= 2^31 - 1 (token positions are int32).  Outside these: PA_ERR_SHAPE.
+ *   - Offsets into a pool are formed in 64 bits: N * block_stride may exceed
+ *     2^31 elements (a pool of tens of GB is one pool).
+ *   - pa_decode, pa_decode_int8, pa_decode_fp8, pa_decode_prepare with the
+ *     planned calls, and pa_prefill_attention only enqueue kernels (no host
+ *     synchronisation, copy or allocation), so a caller can capture them in a
+ *     CUDA graph and replay it with new contents in the same buffers.
  */
 #ifndef PAGEDKV_H
 #define PAGEDKV_H
