@@ -207,13 +207,15 @@ class Clocks:
 
 
 # ----------------------------------------------------------------------------- model
-def clocks_under_load(clk, device, run_steps, seconds=0.8):
-    """The clock record of a run.  The timed region's own samples stand when there are
-    at least 3 (the sampler polls every 200 ms).  A shorter region (p2's 20 steps take
-    about 7 ms) yields samples of the idle GPU around it.  So the same step then runs
-    back to back, untimed, for `seconds` right after the timed region, and its samples
-    are the record; the timed region's own are kept under 'timed_region'."""
-    if clk is not None and clk.get("samples", 0) >= 3:
+def clocks_under_load(clk, device, run_steps, timed_s, seconds=0.8):
+    """The clock record of a run.  The sampler polls every 200 ms and starts 0.3 s
+    before the timed region, so a timed region shorter than a second (c2's 20 steps
+    take about 7 ms) yields mostly samples of the idle GPU around it.  The timed
+    region's own samples stand when it lasted at least 1 s (timed_s) and gave at
+    least 3.  Otherwise the same step runs back to back, untimed, for `seconds` right
+    after the timed region, and its samples are the record; the timed region's own
+    are kept under 'timed_region'."""
+    if clk is not None and clk.get("samples", 0) >= 3 and timed_s >= 1.0:
         return dict(clk, window="timed region")
     soak = Clocks(device)
     t_end = time.perf_counter() + seconds
@@ -224,7 +226,7 @@ def clocks_under_load(clk, device, run_steps, seconds=0.8):
     if rec is None:
         return clk
     return dict(rec, window=f"the same step back to back for {seconds} s after the timed "
-                            "region (too short for a 200 ms sampler)", timed_region=clk)
+                            "region (shorter than 1 s: mostly idle samples)", timed_region=clk)
 
 
 def decode_algorithmic_bytes(cfg, ctx_lens, partial_slots, n_units=0):
@@ -767,7 +769,8 @@ def run_prefill(args, device, world, rank, cpu_baseline=True):
         step(evs[k])
     t1.record(stream)
     torch.cuda.synchronize(device)
-    clk = clocks_under_load(clocks.stop(), device, lambda: [step() for _ in range(8)])
+    clk = clocks_under_load(clocks.stop(), device, lambda: [step() for _ in range(8)],
+                            t0.elapsed_time(t1) / 1000.0)
     ms = reduce_max(t0.elapsed_time(t1), world) / args.steps
     per = [[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in evs]
     score_s = statistics.median(p[0] for p in per) / 1000.0
@@ -935,7 +938,8 @@ def run_chunked(args, device, world, rank, cpu_baseline=True):
         t1.record(stream)
         torch.cuda.synchronize(device)
         total += t0.elapsed_time(t1)
-    clk = clocks_under_load(clocks.stop(), device, lambda: [step() for _ in range(8)])
+    clk = clocks_under_load(clocks.stop(), device, lambda: [step() for _ in range(8)],
+                            total / 1000.0)
     ms = reduce_max(total / args.steps, world)
     attn_s = statistics.median(e[0].elapsed_time(e[1]) for e in evs) / 1000.0
     flops = chunk_flops(cfg)
@@ -1082,7 +1086,8 @@ def run_decode(args, cfg, device, world, rank, cpu_baseline=True):
             for _ in range(args.steps):
                 r.step()
 
-    clk = clocks_under_load(clocks.stop(), device, soak_steps)
+    clk = clocks_under_load(clocks.stop(), device, soak_steps,
+                            t_start.elapsed_time(t_end) / 1000.0)
     total_ms = reduce_max(t_start.elapsed_time(t_end), world)
     ms_per_step = total_ms / args.steps
     value = job_tokens_per_s(world, cfg.batch, ms_per_step)

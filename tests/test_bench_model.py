@@ -129,21 +129,25 @@ def test_clock_record_keeps_a_timed_region_with_enough_samples(monkeypatch):
     _FakeClocks.started = 0
     timed = {"sm_mhz": 1672.0, "sm_max_mhz": 1965.0, "samples": 7, "reasons": ["sw_power_cap"]}
     calls = []
-    rec = bench.clocks_under_load(timed, "cpu", lambda: calls.append(1))
+    rec = bench.clocks_under_load(timed, "cpu", lambda: calls.append(1), timed_s=1.5)
     assert rec["sm_mhz"] == 1672.0 and rec["window"] == "timed region"
     assert calls == [] and _FakeClocks.started == 0
 
 
-@pytest.mark.parametrize("timed", [None, {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0,
-                                          "samples": 2, "reasons": []}])
-def test_clock_record_soaks_after_a_short_timed_region(monkeypatch, timed):
-    """Fewer than 3 samples (a region shorter than the sampler's period): the same step
-    runs back to back for the soak time, and its samples become the record."""
+@pytest.mark.parametrize("timed,timed_s", [
+    (None, 2.0),
+    ({"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "samples": 2, "reasons": []}, 2.0),
+    # enough samples, but a 7 ms region: they are the idle GPU around it
+    ({"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "samples": 3, "reasons": []}, 0.007)])
+def test_clock_record_soaks_after_a_short_timed_region(monkeypatch, timed, timed_s):
+    """Fewer than 3 samples, or a region shorter than 1 s: the same step runs back to
+    back for the soak time, and its samples become the record."""
     monkeypatch.setattr(bench, "Clocks", _FakeClocks)
     monkeypatch.setattr(bench.torch.cuda, "synchronize", lambda device=None: None)
     _FakeClocks.started = 0
     calls = []
-    rec = bench.clocks_under_load(timed, "cpu", lambda: calls.append(1), seconds=0.05)
+    rec = bench.clocks_under_load(timed, "cpu", lambda: calls.append(1), timed_s,
+                                  seconds=0.05)
     assert len(calls) >= 1 and _FakeClocks.started == 1
     assert rec["sm_mhz"] == 1700.0 and rec["reasons"] == ["sw_power_cap"]
     assert rec["timed_region"] == timed and "after the timed region" in rec["window"]
