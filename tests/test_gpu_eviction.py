@@ -99,7 +99,7 @@ def _tables(lens, bs, MB, seed):
     return bt
 
 
-@pytest.mark.parametrize("bs", [16, 256])
+@pytest.mark.parametrize("bs", [16, 256, 1, 5])
 def test_compact_mask_bit_exact(bs):
     rng = np.random.default_rng(40 + bs)
     B, MB = 40, 100

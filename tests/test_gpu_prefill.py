@@ -130,7 +130,7 @@ def test_prefill_select_all_equal_and_monotone():
     assert np.array_equal(got[2], np.arange(100))
 
 
-@pytest.mark.parametrize("bs", [16, 256, 12])
+@pytest.mark.parametrize("bs", [16, 256, 12, 1, 3, 8])
 def test_prefill_pack_bit_exact(bs):
     """Keep sets from the oracle's select; packed pools compared byte for byte."""
     Hkv, d, budget = 8, 128, 300
@@ -182,7 +182,7 @@ def _keep_consistent(keep_gpu, kept_gpu, scores_ref, cu, budget):
     return exact
 
 
-@pytest.mark.parametrize("bs", [16, 256])
+@pytest.mark.parametrize("bs", [16, 256, 5])
 def test_prefill_compress_then_decode(bs):
     """One call scores, selects and packs; then a decode step over the
     compressed cache matches the oracle's decode over the oracle's packed pool."""
@@ -276,7 +276,7 @@ def _random_tables(lens, bs, MB, N, seed):
     return bt
 
 
-@pytest.mark.parametrize("bs", [16, 256])
+@pytest.mark.parametrize("bs", [16, 256, 1, 5])
 def test_evict_compact_bit_exact(bs):
     rng = np.random.default_rng(50 + bs)
     B, MB = 64, 80
