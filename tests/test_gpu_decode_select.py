@@ -31,6 +31,11 @@ CASES = {
     # block size 12: the general-shape kernel
     "general": (W.scaled(C["c3"], key="dsg", layers=1, batch=4, block_size=12,
                          old_lens=(100, 37, 12, 300), outlier_frac=0.0), 0),
+    # one-token and three-token blocks: every cached token a block, or nearly
+    "bs1": (W.scaled(C["c3"], key="ds1", layers=1, batch=3, block_size=1,
+                     old_lens=(50, 1, 7), outlier_frac=0.0), 0),
+    "bs3": (W.scaled(C["c3"], key="ds3", layers=1, batch=4, block_size=3,
+                     old_lens=(100, 2, 3, 301), outlier_frac=0.0), 0),
 }
 
 

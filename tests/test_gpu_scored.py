@@ -29,9 +29,10 @@ def _history(wl, layer):
     return out
 
 
-@pytest.mark.parametrize("key,d", [("c2", 64), ("c3", 128)])
-def test_scored_append_and_pooled_select(key, d):
-    cfg = W.scaled(W.CONFIGS[key], key="sc", layers=1, batch=6, head_dim=d,
+@pytest.mark.parametrize("key,d,bs", [("c2", 64, 16), ("c3", 128, 16), ("c2", 64, 1),
+                                      ("c3", 128, 5)])
+def test_scored_append_and_pooled_select(key, d, bs):
+    cfg = W.scaled(W.CONFIGS[key], key="sc", layers=1, batch=6, head_dim=d, block_size=bs,
                    old_lens=(40, 15, 16, 300, 1, 129), old_len_range=(), outlier_frac=0.0)
     wl = W.generate(cfg, "cpu")
     dev = "cuda"
